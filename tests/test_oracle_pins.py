@@ -1,0 +1,346 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+Sources of truth: hand-worked examples (tests/golden), closed forms that follow from
+Eq. (3)-(4) of the RG-LRU section of "Griffin：将门控线性循环与局部注意力混合以实现
+高效的语言模型", invariants of the linear recurrence (superposition, split and
+step equivalence), brute-force enumeration on tiny inputs, and library routines for
+the special cases that reduce to them (torch conv1d, matmul, GeLU, scipy expit).
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+import oracle
+from gated_linear_rnn_conv1d_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.txt")
+
+
+def _parse_golden(path):
+    examples, cur = {}, None
+    for line in open(path, encoding="utf-8"):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        if line.startswith("[example"):
+            cur = examples.setdefault(line[len("[example"):-1].strip(), {})
+            continue
+        key, val = (s.strip() for s in line.split("=", 1))
+        vals = []
+        for v in val.split(","):
+            v = v.strip()
+            sign = -1.0 if v.startswith("-") else 1.0
+            v = v.lstrip("-")
+            vals.append(sign * (math.log(3.0) if v == "ln3" else float(v)))
+        cur[key] = np.array(vals)
+    return examples
+
+
+def _rng_params(rng, R, lam_lo=4.0, lam_hi=9.0, wscale=None):
+    wscale = 1.0 / math.sqrt(R) if wscale is None else wscale
+    return dict(
+        conv_w=rng.normal(0, 0.5, (4, R)), conv_b=rng.normal(0, 0.5, R),
+        W_a=rng.normal(0, wscale, (R, R)), b_a=rng.normal(0, 0.3, R),
+        W_x=rng.normal(0, wscale, (R, R)), b_x=rng.normal(0, 0.3, R),
+        Lambda=rng.uniform(lam_lo, lam_hi, R),
+    )
+
+
+@pytest.mark.parametrize("name", ["identity_conv", "taps_and_state"])
+def test_hand_worked_examples(name):
+    ex = _parse_golden(GOLDEN)[name]
+    T = ex["x"].size
+    x = ex["x"].reshape(1, T, 1)
+    y, h_T, _ = oracle.rglru_forward(
+        x, ex["conv_w"].reshape(4, 1), ex["conv_b"], np.zeros((1, 1)), ex["b_a"],
+        np.zeros((1, 1)), ex["b_x"], ex["Lambda"], h0=ex["h0"].reshape(1, 1))
+    np.testing.assert_allclose(y.ravel(), ex["y"], rtol=1e-15, atol=1e-15)
+    assert h_T.ravel()[0] == y.ravel()[-1]
+    if "u" in ex:
+        u, _ = oracle.conv1d_causal(x, ex["conv_w"].reshape(4, 1), ex["conv_b"])
+        np.testing.assert_allclose(u.ravel(), ex["u"], rtol=0, atol=1e-15)
+
+
+def test_sigmoid_matches_scipy():
+    z = np.concatenate([np.linspace(-800, 800, 4001), [0.0, -1e-300, 1e-300]])
+    np.testing.assert_allclose(oracle.sigmoid(z), expit(z), rtol=1e-15, atol=1e-300)
+
+
+def test_O1_zero_recurrence_gate_keeps_state_bitwise():
+    """r ≡ 0 ⇒ a_t = a^0 = 1 and √(1 − 1) = 0, so h_t = h_0 for every t (the gate's
+    'keep history, discard input' end, §门行为)."""
+    rng = np.random.default_rng(1)
+    B, T, R = 3, 17, 12
+    p = _rng_params(rng, R)
+    p["W_a"] = np.zeros((R, R))
+    p["b_a"] = np.full(R, -1000.0)          # σ(−1000) underflows to exactly 0
+    x = rng.normal(size=(B, T, R))
+    h0 = rng.normal(size=(B, R))
+    y, h_T, _ = oracle.rglru_forward(x, h0=h0, **p)
+    assert np.array_equal(y, np.broadcast_to(h0[:, None, :], y.shape))
+    assert np.array_equal(h_T, h0)
+
+
+def test_O2_constant_gates_geometric_sum():
+    """W_a = W_x = 0 and zero conv taps ⇒ r, i, u constant; Eq. (4) unrolls to
+    h_T = α^T h0 + m i κ (1 − α^T)/(1 − α), α = σ(Λ)^(8σ(b_a)), m = √(1 − α²)."""
+    rng = np.random.default_rng(2)
+    B, T, R = 2, 300, 5
+    kappa = rng.normal(size=R)
+    Lam = rng.uniform(-2, 9, R)
+    b_a = rng.normal(size=R)
+    b_x = rng.normal(size=R)
+    h0 = rng.normal(size=(B, R))
+    x = rng.normal(size=(B, T, R))
+    y, h_T, _ = oracle.rglru_forward(
+        x, np.zeros((4, R)), kappa, np.zeros((R, R)), b_a, np.zeros((R, R)), b_x, Lam, h0=h0)
+    a = expit(Lam)
+    alpha = a ** (8.0 * expit(b_a))
+    m = np.sqrt(1.0 - alpha ** 2)
+    i = expit(b_x)
+    for t in (1, 7, T):
+        want = alpha ** t * h0 + m * i * kappa * (1 - alpha ** t) / (1 - alpha)
+        np.testing.assert_allclose(y[:, t - 1, :], want, rtol=1e-11, atol=1e-12)
+
+
+def test_O3_unit_variance_fixed_point():
+    """i ≡ 1, constant r, identity conv, x i.i.d. N(0,1), h0 = 0:
+    Var(h_t) = (1 − α²) Σ_{k<t} α^{2k} = 1 − α^{2t} (the √(1 − a_t²) normalisation)."""
+    rng = np.random.default_rng(3)
+    B, T, R = 100, 120, 1000
+    Lam = np.full(R, math.log(0.9 ** (1 / 8)) - math.log1p(-(0.9 ** (1 / 8))))
+    w = np.zeros((4, R))
+    w[3] = 1.0
+    x = rng.normal(size=(B, T, R))
+    y, _, _ = oracle.rglru_forward(x, w, np.zeros(R), np.zeros((R, R)), np.zeros(R),
+                                   np.zeros((R, R)), np.full(R, 1000.0), Lam)
+    alpha = 0.9 ** 0.5                      # a^8 = 0.9 and r = 1/2 ⇒ a_t = a^4
+    n = B * R
+    for t in (1, 10, T):
+        var = float(np.mean(y[:, t - 1, :] ** 2))
+        want = 1.0 - alpha ** (2 * t)
+        se = math.sqrt(2.0 / n) * want
+        assert abs(var - want) < 4 * se, (t, var, want)
+
+
+def test_O4_log_space_equals_direct_power():
+    """log-space evaluation of a^(c r) (the page's numerically stable route) equals
+    the direct power over the init range of Λ and r ∈ [0, 1]."""
+    Lam = np.linspace(4.33, 8.99, 257)[:, None]
+    r = np.linspace(0.0, 1.0, 129)[None, :]
+    d = oracle.decay_direct(r, Lam)
+    l = oracle.decay_log_space(r, Lam)
+    assert np.max(np.abs(d - l) / d) <= 1e-14
+    # and over a wide range of Λ, including a ≪ 1
+    Lam = np.linspace(-30, 30, 601)[:, None]
+    d = oracle.decay_direct(r, Lam)
+    l = oracle.decay_log_space(r, Lam)
+    assert np.max(np.abs(d - l) / np.maximum(d, 1e-300)) <= 1e-12
+
+
+def test_O5_brute_force_unrolled_sum():
+    """h_T = (Π_t a_t) h0 + Σ_k (Π_{t>k} a_t) √(1−a_k²) i_k u_k, enumerated term by term."""
+    rng = np.random.default_rng(5)
+    for T in range(1, 9):
+        B, R = 2, 3
+        p = _rng_params(rng, R, lam_lo=-1.0, lam_hi=6.0, wscale=1.0)
+        x = rng.normal(size=(B, T, R))
+        h0 = rng.normal(size=(B, R))
+        y, h_T, _ = oracle.rglru_forward(x, h0=h0, **p)
+        for b, c in itertools.product(range(B), range(R)):
+            # independent scalar recomputation of the inputs of the sum
+            us, ats, ms, iis = [], [], [], []
+            for t in range(T):
+                u = p["conv_b"][c]
+                for k in range(4):
+                    s = t - 3 + k
+                    if s >= 0:
+                        u += p["conv_w"][k][c] * x[b, s, c]
+                us.append(u)
+            for t in range(T):
+                za = p["b_a"][c] + sum(p["W_a"][c][j] * us_j for j, us_j in
+                                       enumerate([_u_at(x, p, b, t, jj) for jj in range(R)]))
+                zx = p["b_x"][c] + sum(p["W_x"][c][j] * _u_at(x, p, b, t, j) for j in range(R))
+                r = 1.0 / (1.0 + math.exp(-za))
+                a = 1.0 / (1.0 + math.exp(-p["Lambda"][c]))
+                at = math.exp(8.0 * r * math.log(a))
+                ats.append(at)
+                ms.append(math.sqrt(1.0 - at * at))
+                iis.append(1.0 / (1.0 + math.exp(-zx)))
+            want = math.prod(ats) * h0[b, c]
+            for k in range(T):
+                want += math.prod(ats[k + 1:]) * ms[k] * iis[k] * us[k]
+            assert abs(h_T[b, c] - want) <= 1e-13 * max(1.0, abs(want)), (T, b, c)
+
+
+def _u_at(x, p, b, t, c):
+    u = p["conv_b"][c]
+    for k in range(4):
+        s = t - 3 + k
+        if s >= 0:
+            u += p["conv_w"][k][c] * x[b, s, c]
+    return u
+
+
+def test_O6_conv_matches_torch_conv1d():
+    rng = np.random.default_rng(6)
+    B, T, R = 3, 37, 16
+    x = rng.normal(size=(B, T, R))
+    w = rng.normal(size=(4, R))
+    bias = rng.normal(size=R)
+    u, state = oracle.conv1d_causal(x, w, bias)
+    xt = torch.from_numpy(x).permute(0, 2, 1)                  # [B][R][T]
+    wt = torch.from_numpy(w).T.reshape(R, 1, 4)                # weight[c][0][k]
+    ref = torch.nn.functional.conv1d(xt, wt, torch.from_numpy(bias), padding=3, groups=R)
+    ref = ref[..., :T].permute(0, 2, 1).numpy()
+    np.testing.assert_allclose(u, ref, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(state, x[:, T - 3:, :])
+    # with a history: equals the conv of the concatenated sequence
+    hist = rng.normal(size=(B, 3, R))
+    u2, _ = oracle.conv1d_causal(x, w, bias, hist)
+    full, _ = oracle.conv1d_causal(np.concatenate([hist, x], axis=1), w, bias)
+    np.testing.assert_allclose(u2, full[:, 3:, :], rtol=1e-13, atol=1e-13)
+
+
+def test_O7_gate_preactivations_match_torch_matmul():
+    rng = np.random.default_rng(7)
+    B, T, R = 2, 9, 24
+    u = rng.normal(size=(B, T, R))
+    Wa, Wx = rng.normal(size=(R, R)), rng.normal(size=(R, R))
+    ba, bx = rng.normal(size=R), rng.normal(size=R)
+    za, zx = oracle.gate_preactivations(u, Wa, ba, Wx, bx)
+    ut = torch.from_numpy(u)
+    np.testing.assert_allclose(za, (torch.matmul(ut, torch.from_numpy(Wa).T) + torch.from_numpy(ba)).numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(zx, (torch.matmul(ut, torch.from_numpy(Wx).T) + torch.from_numpy(bx)).numpy(), rtol=1e-12, atol=1e-12)
+    ch = np.array([5, 0, 23])
+    za2, zx2 = oracle.gate_preactivations(u, Wa, ba, Wx, bx, channels=ch)
+    np.testing.assert_array_equal(za2, za[..., ch])
+    np.testing.assert_array_equal(zx2, zx[..., ch])
+
+
+def test_O8_superposition_in_h0():
+    """y(h0) − y(0) = (Π_{s≤t} a_s) h0: the recurrence is linear in h."""
+    rng = np.random.default_rng(8)
+    B, T, R = 2, 40, 6
+    p = _rng_params(rng, R)
+    x = rng.normal(size=(B, T, R))
+    h0 = rng.normal(size=(B, R))
+    y1, _, _ = oracle.rglru_forward(x, h0=h0, **p)
+    y0, _, _ = oracle.rglru_forward(x, h0=None, **p)
+    u, _ = oracle.conv1d_causal(x, p["conv_w"], p["conv_b"])
+    za, _ = oracle.gate_preactivations(u, p["W_a"], p["b_a"], p["W_x"], p["b_x"])
+    at = expit(p["Lambda"]) ** (8.0 * expit(za))
+    np.testing.assert_allclose(y1 - y0, np.cumprod(at, axis=1) * h0[:, None, :], rtol=1e-11, atol=1e-14)
+
+
+def test_O9_step_equals_forward_and_split_equals_whole():
+    rng = np.random.default_rng(9)
+    B, T, R = 3, 13, 8
+    p = _rng_params(rng, R)
+    x = rng.normal(size=(B, T, R))
+    h0 = rng.normal(size=(B, R))
+    y, h_T, st_T = oracle.rglru_forward(x, h0=h0, **p)
+    # T decode steps from a zero ring equal the forward pass
+    ring, h = np.zeros((B, 3, R)), h0.copy()
+    for t in range(T):
+        yt, h, ring = oracle.rglru_step(x[:, t, :], ring, t, h, **p)
+        np.testing.assert_allclose(yt, y[:, t, :], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(h, h_T, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(oracle.ring_to_time_order(ring, T), st_T)
+    # forward(0:T1) then forward(T1:T) from the carried (h, conv state) equals forward(0:T)
+    for T1 in (1, 5, 12):
+        ya, ha, sa = oracle.rglru_forward(x[:, :T1], h0=h0, **p)
+        yb, hb, sb = oracle.rglru_forward(x[:, T1:], h0=ha, conv_state0=sa, **p)
+        np.testing.assert_allclose(np.concatenate([ya, yb], 1), y, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(hb, h_T, rtol=1e-13, atol=1e-13)
+        np.testing.assert_array_equal(sb, st_T)
+    # a subset of rows gives the same rows
+    yt_all, _, _ = oracle.rglru_step(x[:, 0, :], np.zeros((B, 3, R)), 0, h0, **p)
+    yt_sub, _, _ = oracle.rglru_step(x[:, 0, :], np.zeros((B, 3, R)), 0, h0, rows=[2, 0], **p)
+    np.testing.assert_array_equal(yt_sub, yt_all[[2, 0]])
+    # a subset of channels gives the same channels
+    ch = [7, 1]
+    ys, hs, _ = oracle.rglru_forward(x, h0=h0, channels=ch, **p)
+    np.testing.assert_allclose(ys, y[..., ch], rtol=1e-14, atol=1e-15)
+
+
+def test_O10_parameter_ranges_of_the_init():
+    """a^8 ~ U[0.9, 0.999] ⇒ a ∈ [0.98692, 0.999875]; r ∈ (0, 1) ⇒ a_t ∈ [0.9, 1]."""
+    w = inputs.make_forward(1, 64, 256, torch.float32, seed=0)
+    a = expit(w.params.Lambda.double().numpy())
+    assert a.min() >= 0.9 ** (1 / 8) - 1e-7 and a.max() <= 0.999 ** (1 / 8) + 1e-7
+    assert 0.98692 <= a.min() and a.max() <= 0.999875
+    y, h_T, _ = oracle.rglru_forward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a,
+                                     w.params.b_a, w.params.W_x, w.params.b_x, w.params.Lambda)
+    assert np.isfinite(y).all()
+    u, _ = oracle.conv1d_causal(w.x, w.params.conv_w, w.params.conv_b)
+    za, _ = oracle.gate_preactivations(u, w.params.W_a, w.params.b_a, w.params.W_x, w.params.b_x)
+    at = oracle.decay_direct(oracle.sigmoid(za), w.params.Lambda)
+    assert at.min() >= 0.9 - 1e-12 and at.max() <= 1.0
+
+
+def test_gelu_exact_matches_torch_and_identity():
+    x = np.linspace(-12, 12, 2401)
+    g = oracle.gelu(x)
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="none").numpy()
+    np.testing.assert_allclose(g, ref, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(g - oracle.gelu(-x), x, rtol=1e-14, atol=1e-14)   # xΦ(x)+xΦ(−x) = x
+
+
+def test_block_zero_gate_branch_and_constant_input_branch():
+    """Recurrent block: W_2 = 0 ⇒ GeLU(0) = 0 ⇒ out ≡ 0; W_1 = 0 with W_a = W_x = 0 ⇒
+    u ≡ conv bias, so h follows the geometric closed form and out = (h ⊙ GeLU(g)) W_oᵀ."""
+    rng = np.random.default_rng(11)
+    B, T, D, R = 2, 20, 6, 4
+    x = rng.normal(size=(B, T, D))
+    W1, W2, Wo = rng.normal(size=(R, D)), rng.normal(size=(R, D)), rng.normal(size=(D, R))
+    p = _rng_params(rng, R)
+    out, _ = oracle.recurrent_block(x, W1, np.zeros((R, D)), Wo, **p)
+    assert np.array_equal(out, np.zeros_like(out))
+    p["W_a"] = np.zeros((R, R))
+    p["W_x"] = np.zeros((R, R))
+    out, h_T = oracle.recurrent_block(x, np.zeros((R, D)), W2, Wo, **p)
+    alpha = expit(p["Lambda"]) ** (8.0 * expit(p["b_a"]))
+    m, i, kappa = np.sqrt(1 - alpha ** 2), expit(p["b_x"]), p["conv_b"]
+    t = np.arange(1, T + 1)[:, None]
+    h = m * i * kappa * (1 - alpha ** t) / (1 - alpha)                  # [T][R]
+    g = torch.from_numpy(x @ W2.T)
+    gel = torch.nn.functional.gelu(g, approximate="none").numpy()
+    want = (h[None] * gel) @ Wo.T
+    np.testing.assert_allclose(out, want, rtol=1e-11, atol=1e-12)
+
+
+def test_max_rel_error_definition():
+    ref = np.array([1.0, -2.0, 0.0, 4.0])
+    rms = math.sqrt((1 + 4 + 0 + 16) / 4)
+    got = ref + np.array([0.0, 0.0, 0.1, 0.0])
+    assert abs(oracle.max_rel_error(got, ref) - 0.1 / rms) < 1e-15
+    got = ref + np.array([0.0, 0.0, 0.0, 0.4])
+    assert abs(oracle.max_rel_error(got, ref) - 0.1) < 1e-15
+
+
+def test_planted_mistakes_are_caught():
+    """Plant plausible mistakes in the oracle's arithmetic (on the CPU) and check that
+    the pins above would reject each one."""
+    ex = _parse_golden(GOLDEN)["taps_and_state"]
+    x = ex["x"].reshape(1, -1, 1)
+
+    def run(conv_w):
+        y, _, _ = oracle.rglru_forward(x, conv_w.reshape(4, 1), ex["conv_b"], np.zeros((1, 1)),
+                                       ex["b_a"], np.zeros((1, 1)), ex["b_x"], ex["Lambda"],
+                                       h0=ex["h0"].reshape(1, 1))
+        return y.ravel()
+
+    assert np.allclose(run(ex["conv_w"]), ex["y"], rtol=1e-15)
+    assert not np.allclose(run(ex["conv_w"][::-1].copy()), ex["y"], rtol=1e-6)   # reversed taps
+    # wrong normalisation (1 − a_t instead of 1 − a_t²) changes the hand-worked values
+    at, i, h0 = 9 / 16, 0.75, 1.0
+    h = h0
+    for u in ex["u"]:
+        h = at * h + math.sqrt(1 - at) * i * u
+    assert abs(h - ex["y"][-1]) > 1e-3
