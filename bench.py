@@ -1,0 +1,413 @@
+"""Benchmark of the RG-LRU temporal core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+
+Own arm. One step = one forward pass of the layer (Conv1D(4) → gate GEMM → fused
+gates/decay/chunked scan) over one batch of the Hawk-scale workload
+B=8, T=2048, D_RNN=2048, bf16 IO with float32 state, inputs resident in HBM, L2 flushed
+(256 MB write) before every timed step. The step calls the three stages of
+rglru_forward one by one through the C ABI (the same launches rglru_forward makes) so
+that each kernel's duration is measured with CUDA events on its own stream.
+Reported: tokens/s (all ranks), per-kernel achieved bandwidth / throughput and their
+fractions of the measured B200 peaks, the roofline of the dominant kernel, the same
+metric end to end through the public API with host buffers (pinned H2D of x, D2H of y
+and h_T inside the timed region), decode steps/s on B=256, D_RNN=4096, the GPU clocks
+sampled during the timed region, and the CPU oracle on the host cores.
+
+Under torchrun (N > 1) every rank runs an independent replica on its own GPU (the
+batches are independent; nothing is exchanged on the data path), timing is the max
+over ranks, and rank 0 prints the JSON line.
+
+Reference arm (--impl reference): the float64 CPU oracle, timed as it stands on the
+host cores, each step a bounded sample of the same workload (one batch row, 512 steps,
+all 2048 channels); rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RG-LRU fwd tokens/s and achieved HBM GB/s vs B200 peak; decode steps/s"
+WORKLOAD = dict(B=8, T=2048, R=2048)
+DECODE = dict(B=256, R=4096)
+FLUSH_BYTES = 256 << 20
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
+# summarised under profiles/, keyed by the SHA-256 of the kernel's source at capture
+# time. A source change invalidates the figure (reported as null).
+NCU_TRAFFIC = {}
+
+
+def _sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+_CLOCK_Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+            "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+            "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, dev_index):
+        self.proc = None
+        self.dev = dev_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={_CLOCK_Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ own arm
+def run_own(args):
+    import torch
+    import torch.distributed as dist
+
+    from gated_linear_rnn_conv1d_b200 import inputs, rglru
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    B, T, R = WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["R"]
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=rank)
+    p = rglru.Params.from_host(w.params, dev)
+    x = w.x.to(dev)
+    y = torch.empty_like(x)
+    h_T = torch.empty(B, R, dtype=torch.float32, device=dev)
+    u = torch.empty_like(x)
+    z = torch.empty(B * T, rglru.gate_pitch(R), dtype=torch.bfloat16, device=dev)
+    ws_scan = torch.empty(rglru.scan_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
+    ws_fwd = torch.empty(rglru.forward_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rglru.conv1d(p, x, u=u)
+        if ev is not None:
+            ev[1].record(stream)
+        rglru.gate_proj(p, u.view(B * T, R), z=z)
+        if ev is not None:
+            ev[2].record(stream)
+        rglru.scan(p, x, z, workspace=ws_scan, y=y, h_T=h_T)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if rglru.workspace_status(ws_scan) != 0 or rglru.workspace_status(None) != 0:
+        raise SystemExit("a kernel reported a timeout during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.zero_()                 # L2 flush between timed steps (outside the events)
+        step(evs[k])
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    conv_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    gemm_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    scan_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+    step_ms = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / K)
+    status = rglru.workspace_status(ws_scan)
+
+    tokens = B * T
+    value = world * tokens / (step_ms / 1e3)
+    pk = _peaks()
+    # algorithmic bytes / flops per launch (bf16 = 2 B; packed z = 2 gates × 2 B per channel)
+    conv_bytes = tokens * R * 2 * 2                     # read x, write u
+    scan_bytes = tokens * R * (2 + 4 + 2)               # read x, read z_a and z_x, write y
+    gemm_flops = 2.0 * tokens * (2 * R) * R
+    kern = {
+        "conv1d": {"ms": conv_ms, "GB/s": conv_bytes / conv_ms / 1e6, "bytes": conv_bytes},
+        "gate_gemm": {"ms": gemm_ms, "TFLOP/s": gemm_flops / gemm_ms / 1e9, "flops": gemm_flops},
+        "scan": {"ms": scan_ms, "GB/s": scan_bytes / scan_ms / 1e6, "bytes": scan_bytes},
+    }
+    kern["conv1d"]["frac_hbm"] = kern["conv1d"]["GB/s"] / pk["hbm_gbs"]
+    kern["scan"]["frac_hbm"] = kern["scan"]["GB/s"] / pk["hbm_gbs"]
+    kern["gate_gemm"]["frac_tensor"] = kern["gate_gemm"]["TFLOP/s"] / pk["bf16_tflops"]
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    traffic = None
+    src = os.path.join(ROOT, "gated_linear_rnn_conv1d_b200", "csrc",
+                       {"gate_gemm": "gemm_tc.cu", "scan": "scan.cu", "conv1d": "conv.cu"}[dom])
+    rec = NCU_TRAFFIC.get(dom)
+    if rec and rec["src_sha256"] == _sha(src):
+        traffic = rec["bytes_per_launch"]
+    if dom == "gate_gemm":
+        roof = {"bound": "tensor", "achieved": kern[dom]["TFLOP/s"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": kern[dom]["GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["kernel"] = dom
+    roof["peak_source"] = pk["source"] + " (MEASURED_PEAKS.json burst figure)" if pk["source"] == "measured" else "fallback"
+
+    # ---- end to end through the public API, host buffers -----------------------------
+    x_host = w.x.pin_memory()
+    y_host = torch.empty(B, T, R, dtype=torch.bfloat16).pin_memory()
+    h_host = torch.empty(B, R, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(3, min(K, 50))
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        rglru.forward(p, x_dev, workspace=ws_fwd, y=y, h_T=h_T, want_conv_state=False)
+        y_host.copy_(y, non_blocking=True)
+        h_host.copy_(h_T, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        rglru.forward(p, x_dev, workspace=ws_fwd, y=y, h_T=h_T, want_conv_state=False)
+        y_host.copy_(y, non_blocking=True)
+        h_host.copy_(h_T, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+           "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2 + h_T.numel() * 4}
+    if rglru.workspace_status(ws_fwd) != 0:
+        status = -7
+
+    # ---- decode steps/s ---------------------------------------------------------------
+    dec = run_decode(torch, rglru, inputs, dev, stream, flush, pk, barrier, max_over_ranks, world)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = cpu_baseline(inputs) if world == 1 else None
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs, LeCun-normal gate weights, a^8~U[0.9,0.999])",
+        "config": {"workload": "RG-LRU forward, Hawk-scale layer: B=8 T=2048 D_RNN=2048, bf16 IO, fp32 state",
+                   "B": B, "T": T, "D_RNN": R, "global_batch": B * world, "seq_len": T,
+                   "parallelism": f"replicas x{world} (independent batches, no collective on the data path)",
+                   "l2": "flushed before every timed step (256 MB write, outside the step events)"},
+        "roofline": roof,
+        "kernels": kern,
+        "hbm_gb_per_s": {"scan": kern["scan"]["GB/s"], "conv1d": kern["conv1d"]["GB/s"],
+                         "peak": pk["hbm_gbs"], "peak_source": pk["source"]},
+        "decode": dec,
+        "e2e": e2e,
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+        "status": "ok" if status == 0 else "timeout reported",
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(out))
+
+
+def run_decode(torch, rglru, inputs, dev, stream, flush, pk, barrier, max_over_ranks, world):
+    B, R = DECODE["B"], DECODE["R"]
+    w = inputs.make_decode(B, R, torch.bfloat16, seed=0)
+    p = rglru.Params.from_host(w.params, dev)
+    n_tok = 48
+    toks = torch.stack([inputs.decode_token(k, B, R) for k in range(n_tok)]).to(dev)
+    ring = torch.zeros(B, 3, R, dtype=torch.bfloat16, device=dev)
+    h = torch.zeros(B, R, device=dev)
+    y = torch.empty(B, R, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(rglru.step_workspace_bytes(B, R), dtype=torch.uint8, device=dev)
+    for k in range(6):
+        rglru.step(p, toks[k], ring, h, k, workspace=ws, y_t=y)
+    torch.cuda.synchronize()
+    # graph of n_tok consecutive steps (weights stay L2-warm across steps, as in serving)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for k in range(n_tok):
+            rglru.step(p, toks[k], ring, h, k, workspace=ws, y_t=y)
+    g.replay()
+    torch.cuda.synchronize()
+    reps = 8
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    warm_ms = max_over_ranks(e0.elapsed_time(e1) / (reps * n_tok))
+    # one step at a time with L2 flushed before each step (weights come from HBM)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(24)]
+    for k, (a, b) in enumerate(evs):
+        flush.zero_()
+        a.record(stream)
+        rglru.step(p, toks[k % n_tok], ring, h, k, workspace=ws, y_t=y)
+        b.record(stream)
+    torch.cuda.synchronize()
+    cold_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs))
+    del g
+    step_bytes = 2 * R * R * 2 + B * R * (4 + 4) + B * 3 * R * 2 + B * R * 2 * 3   # W, h r/w, ring r, x/ring w/y
+    return {"workload": "RG-LRU decode B=256 D_RNN=4096 bf16 x_t/y, fp32 h, bf16 3-slot conv ring",
+            "steps_per_s": world / (warm_ms / 1e3), "ms_per_step": warm_ms,
+            "steps_per_s_l2_flushed": world / (cold_ms / 1e3), "ms_per_step_l2_flushed": cold_ms,
+            "bytes_per_step": step_bytes,
+            "GB/s_l2_flushed": step_bytes / cold_ms / 1e6,
+            "frac_hbm_l2_flushed": step_bytes / cold_ms / 1e6 / pk["hbm_gbs"],
+            "gpu_launches_per_step": 2,
+            "timing": "CUDA graph of 48 steps replayed 8x (L2-warm); and 24 single steps with L2 flushed"}
+
+
+# ------------------------------------------------------------------------------ CPU side
+def _host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def _oracle_sample(inputs, rows=1, steps=512):
+    """The oracle on `rows` batch rows × `steps` steps × all channels of the workload."""
+    import torch
+
+    import oracle
+    B, T, R = WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["R"]
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=0)
+    pr = w.params
+    x = w.x[:rows, :steps]
+    t0 = time.perf_counter()
+    oracle.rglru_forward(x, pr.conv_w, pr.conv_b, pr.W_a, pr.b_a, pr.W_x, pr.b_x, pr.Lambda)
+    dt = time.perf_counter() - t0
+    return rows * steps, dt
+
+
+def cpu_baseline(inputs):
+    _oracle_sample(inputs, rows=1, steps=512)          # untimed: first touch of host memory
+    tok, dt = 0, 0.0
+    for _ in range(2):
+        t, d = _oracle_sample(inputs, rows=1, steps=2048)
+        tok += t
+        dt += d
+    return {"value": tok / dt, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
+            "sample": f"2 x (1 batch row x 2048 steps x 2048 channels) of the workload, {dt:.1f} s; "
+                      "float64 numpy, BLAS matmul on the host cores, recurrence vectorised over channels"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from gated_linear_rnn_conv1d_b200 import inputs
+    for _ in range(args.warmup):
+        _oracle_sample(inputs)
+    tot_tok, tot_dt = 0, 0.0
+    for _ in range(args.steps):
+        tok, dt = _oracle_sample(inputs)
+        tot_tok += tok
+        tot_dt += dt
+    value = tot_tok / tot_dt
+    cores = _host_cores()
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "RG-LRU forward, Hawk-scale layer: B=8 T=2048 D_RNN=2048, bf16 IO, fp32 state",
+                   "B": WORKLOAD["B"], "T": WORKLOAD["T"], "D_RNN": WORKLOAD["R"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step: 1 batch row x 512 steps x 2048 channels of the workload"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["own", "reference"], default="own")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_own(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,419 @@
+// bf16 GEMMs on the sm_100a tensor cores (tcgen05.mma, fp32 accumulators in TMEM,
+// operands staged by TMA into 128-byte-swizzled shared memory; no cluster multicast).
+//
+// Uses: the RG-LRU gate projections z = u [W_a | W_x]ᵀ + b ("Griffin：将门控线性循环与
+// 局部注意力混合以实现高效的语言模型", §实门线性循环单元 (RG-LRU), Eq. (1)–(2)) — the only dense
+// contraction of the layer — for prefill (packed z out) and for decode (the RG-LRU update
+// fused into the epilogue, Eq. (3)–(4)); and the recurrent block's D ↔ D_RNN linears
+// (§循环块).
+//
+// Kernel shape: persistent CTAs (one per SM), 192 threads.
+//   warp 0      one lane issues TMA loads of A [128×64] and B [BN×64] k-blocks into a
+//               ring of smem stages (full/empty mbarriers);
+//   warp 1      allocates TMEM (two BN-column accumulators) and one lane issues
+//               tcgen05.mma M=128, N=BN, K=16 (four per k-block), committing each stage
+//               back to the producer and each finished tile to the epilogue;
+//   warps 2–5   epilogue: tcgen05.ld of their 32 TMEM lanes (= 32 output rows), fused
+//               element-wise work, global stores; the accumulator is handed back so the
+//               next tile's MMAs overlap this tile's epilogue.
+// "Dual" B: the gate GEMMs fetch the first BN/2 rows of a B tile from W_a and the second
+// BN/2 from W_x (two tensor maps), so one tile holds both gates of the same channels.
+#include <algorithm>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <mutex>
+
+#include "gate_math.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace rglru {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
+constexpr int kGemmThreads = 192;
+
+enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2 };
+
+struct EpiArgs {
+  __nv_bfloat16* C;   // STORE / GATES output
+  int64_t ldc;        // elements
+  int N;              // STORE: valid columns
+  const float* b_a;   // GATES / STEP
+  const float* b_x;
+  int R;              // channels (GATES / STEP)
+  const __nv_bfloat16* u;  // STEP: u_t [M][R]
+  float* h;                // STEP: state [M][R], in place
+  __nv_bfloat16* y;        // STEP: y_t [M][R]
+  const float* cla;        // STEP: c·log σ(Λ) [R]
+};
+
+template <int BN> struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 1024;  // + alignment slack
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr uint32_t kIdesc = umma_idesc_bf16_f32(BM, BN);
+};
+
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+
+template <int BN, int EPI, bool DUAL>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, int64_t M, int K, int n_tiles_n, int num_tiles,
+                   EpiArgs ep, unsigned* status) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 4);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (DUAL) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int k_blocks = (K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m_blk = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_s)) { ok = false; break; }
+          uint8_t* sa = smem + stage * Cfg::kStageBytes;
+          uint8_t* sb = sa + Cfg::kABytes;
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::kStageBytes);
+          tma_load_2d(sa, &tmA, &full_bar[stage], kb * BK, m_blk * BM);
+          if (DUAL) {
+            tma_load_2d(sb, &tmB0, &full_bar[stage], kb * BK, n_blk * (BN / 2));
+            tma_load_2d(sb + (BN / 2) * BK * 2, &tmB1, &full_bar[stage], kb * BK, n_blk * (BN / 2));
+          } else {
+            tma_load_2d(sb, &tmB0, &full_bar[stage], kb * BK, n_blk * BN);
+          }
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) { abort_s = 1; atomicOr(status, kStatusTimeout); }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, &abort_s)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_s)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * Cfg::kStageBytes);
+          const uint32_t b_addr = a_addr + Cfg::kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            umma_f16(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), Cfg::kIdesc,
+                     (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull_bar[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      if (!ok) {
+        abort_s = 1;
+        atomicOr(status, kStatusTimeout);
+      }
+      // Drain: wait until every MMA issued by this thread has completed before TMEM is
+      // freed (a barrier of its own, so the epilogue's phases are not disturbed).
+      umma_commit(&drain_bar);
+      {
+        volatile int never = 0;
+        (void)mbar_wait(&drain_bar, 0, &never);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int quarter = warp & 3;  // a warp may only touch TMEM lanes 32*(warp%4) .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int m_blk = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_s)) {
+        abort_s = 1;
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const int64_t row = (int64_t)m_blk * BM + row_in_tile;
+      const bool row_ok = row < M;
+
+      if constexpr (EPI == EPI_STORE || EPI == EPI_GATES) {
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + cc * 32, r);
+          tmem_ld_wait();
+          float v[32];
+          const int col0 = cc * 32;
+          if constexpr (EPI == EPI_GATES) {
+            // packed layout: block n_blk holds channels [n_blk*BN/2, +BN/2), z_a then z_x
+            const int half = col0 / (BN / 2);
+            const int ch0 = n_blk * (BN / 2) + (col0 % (BN / 2));
+            const float* bias = half ? ep.b_x : ep.b_a;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int ch = ch0 + j;
+              v[j] = __uint_as_float(r[j]) + (ch < ep.R ? __ldg(bias + ch) : 0.0f);
+            }
+            if (row_ok) store_row_bf16(ep.C + row * ep.ldc + (int64_t)n_blk * BN + col0, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            const int gcol = n_blk * BN + col0;
+            if (row_ok) {
+              if (gcol + 32 <= ep.N) {
+                store_row_bf16(ep.C + row * ep.ldc + gcol, v);
+              } else {
+                uint4* d = reinterpret_cast<uint4*>(ep.C + row * ep.ldc + gcol);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (gcol + 8 * q < ep.N)
+                    d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+              }
+            }
+          }
+        }
+      } else {
+        // EPI_STEP: columns [0, BN/2) are z_a and [BN/2, BN) are z_x of channels
+        // n_blk*BN/2 + j; row = batch index. h ← a_t h + √(1−a_t²) i u ; y = h.
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 64; ++cc) {
+          uint32_t ra[32], rx[32];
+          tmem_ld_32x32b_x32(t_row + cc * 32, ra);
+          tmem_ld_32x32b_x32(t_row + BN / 2 + cc * 32, rx);
+          tmem_ld_wait();
+          const int ch0 = n_blk * (BN / 2) + cc * 32;
+          if (row_ok) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = ch0 + 8 * q;
+              if (c < ep.R) {
+                const uint4 w = *reinterpret_cast<const uint4*>(ep.u + row * ep.R + c);
+                float4* hp = reinterpret_cast<float4*>(ep.h + row * ep.R + c);
+                const float4 h0 = hp[0], h1 = hp[1];
+                float uu[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                               bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+                float hh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const int ch = c + j;
+                  const float za = __uint_as_float(ra[8 * q + j]) + __ldg(ep.b_a + ch);
+                  const float zx = __uint_as_float(rx[8 * q + j]) + __ldg(ep.b_x + ch);
+                  float at, bt;
+                  gate_fast(za, zx, __ldg(ep.cla + ch), uu[j], at, bt);
+                  hh[j] = fmaf(at, hh[j], bt);
+                }
+                hp[0] = make_float4(hh[0], hh[1], hh[2], hh[3]);
+                hp[1] = make_float4(hh[4], hh[5], hh[6], hh[7]);
+                *reinterpret_cast<uint4*>(ep.y + row * ep.R + c) =
+                    make_uint4(pack_bf16x2(hh[0], hh[1]), pack_bf16x2(hh[2], hh[3]), pack_bf16x2(hh[4], hh[5]),
+                               pack_bf16x2(hh[6], hh[7]));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_tiled();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI, bool DUAL>
+cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, int64_t M, int K,
+                      int n_tiles_n, const EpiArgs& ep, unsigned* status, cudaStream_t s) {
+  using Cfg = GemmCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, EPI, DUAL>;
+  static bool attr_set = false;  // per instantiation; benign race (idempotent)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t m_tiles = (M + BM - 1) / BM;
+  const int64_t tiles = m_tiles * n_tiles_n;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  const int grid = (int)std::min<int64_t>(tiles, num_sms());
+  kern<<<grid, kGemmThreads, Cfg::kSmem, s>>>(a, b0, b1, M, K, n_tiles_n, (int)tiles, ep, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Status word for GEMM launches that come without a workspace.
+__device__ unsigned g_gemm_status;
+
+EncodeTiledFn get_encode_tiled() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+int num_sms() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (n[dev] == 0) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
+  return n[dev];
+}
+
+unsigned* global_status_word() {
+  static unsigned* p[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (p[dev] == nullptr) {
+    unsigned* q = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&q), g_gemm_status) != cudaSuccess) return nullptr;
+    p[dev] = q;
+  }
+  return p[dev];
+}
+
+cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
+                                   void* z, int64_t M, int R, unsigned* status, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap ma, mb0, mb1;
+  if (!make_map_2d(&ma, u, R, M, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb0, Wa, R, R, (uint64_t)R * 2, BK, BN / 2)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb1, Wx, R, R, (uint64_t)R * 2, BK, BN / 2)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.C = static_cast<__nv_bfloat16*>(z);
+  ep.ldc = gate_pitch(R);
+  ep.b_a = ba;
+  ep.b_x = bx;
+  ep.R = R;
+  const int n_tiles_n = (R + BN / 2 - 1) / (BN / 2);
+  return launch_tc<BN, EPI_GATES, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
+}
+
+cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
+                             unsigned* status, cudaStream_t s) {
+  constexpr int BN = 256;
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, A, K, M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, BN)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.C = static_cast<__nv_bfloat16*>(C);
+  ep.ldc = ldc;
+  ep.N = N;
+  const int n_tiles_n = (N + BN - 1) / BN;
+  return launch_tc<BN, EPI_STORE, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+}
+
+cudaError_t launch_gemm_step_bf16(const void* u_t, const void* Wa, const float* ba, const void* Wx,
+                                  const float* bx, const float* cla, float* h, void* y_t, int B, int R,
+                                  unsigned* status, cudaStream_t s) {
+  constexpr int BN = 128;
+  CUtensorMap ma, mb0, mb1;
+  if (!make_map_2d(&ma, u_t, R, B, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb0, Wa, R, R, (uint64_t)R * 2, BK, BN / 2)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb1, Wx, R, R, (uint64_t)R * 2, BK, BN / 2)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.b_a = ba;
+  ep.b_x = bx;
+  ep.R = R;
+  ep.u = static_cast<const __nv_bfloat16*>(u_t);
+  ep.h = h;
+  ep.y = static_cast<__nv_bfloat16*>(y_t);
+  ep.cla = cla;
+  const int n_tiles_n = (R + BN / 2 - 1) / (BN / 2);
+  return launch_tc<BN, EPI_STEP, true>(ma, mb0, mb1, B, R, n_tiles_n, ep, status, s);
+}
+
+
+}  // namespace rglru

@@ -1,0 +1,82 @@
+// Launch interfaces of the RG-LRU kernels (host side), shared by the C-ABI layer.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace rglru {
+
+// ---- packed gate layout: 128-channel blocks, [z_a(128) | z_x(128)] per block -----
+constexpr int kGateBlock = 128;
+inline int64_t gate_pitch(int R) { return (int64_t)((R + kGateBlock - 1) / kGateBlock) * 2 * kGateBlock; }
+
+// ---- scan tiling -------------------------------------------------------------------
+constexpr int kScanThreads = 256;
+constexpr int kScanGroups = 16;                         // channel-group threads per CTA
+constexpr int kScanSub = kScanThreads / kScanGroups;    // time sub-chunks per CTA
+constexpr int kScanL = 4;                               // time steps per thread
+constexpr int kScanTC = kScanSub * kScanL;              // time steps per CTA
+inline int scan_vec(bool bf16) { return bf16 ? 8 : 4; }
+inline int scan_cw(bool bf16) { return kScanGroups * scan_vec(bf16); }
+
+struct ScanLayout {
+  int n_cblk, n_chunks;
+  int64_t n_tiles;
+  size_t off_flags, off_carry, bytes;
+};
+ScanLayout scan_layout(int B, int T, int R, bool bf16);
+
+struct ScanArgs {
+  const void* x;        // [B][T][R]
+  const void* z;        // [B*T][pitch] packed
+  const void* state0;   // [B][3][R] or null
+  const float* h0;      // [B][R] or null
+  const void* g;        // [B][T][R] or null (block gate branch)
+  void* y;              // [B][T][R]
+  float* hT;            // [B][R] or null
+  const float* conv_w;  // [4][R]
+  const float* conv_b;  // [R]
+  const float* Lambda;  // [R]
+  unsigned* status;     // device status word
+  unsigned* ticket;     // tile ticket counter (zeroed before launch)
+  unsigned* flags;      // [n_tiles] look-back flags (zeroed before launch)
+  float* carry;         // [n_tiles][3][CW]
+  int B, T, R, n_cblk, n_chunks;
+  int64_t pitch;
+  int64_t stall_tile;   // testing only: this tile never publishes its carry (-1: none)
+};
+// Testing only: the tile index the next scans leave unpublished (-1 disables).
+void set_scan_stall(int64_t tile);
+int64_t scan_stall();
+cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s);
+
+// ---- conv --------------------------------------------------------------------------
+cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* state0, void* u,
+                          void* stateT, int B, int T, int R, bool bf16, cudaStream_t s);
+// Also zeroes *status (the step's status word) before the step's GEMM may set it.
+cudaError_t launch_decode_conv(const float* conv_w, const float* conv_b, const float* Lambda, const void* x_t,
+                               void* ring, int64_t step, void* u_t, float* cla, unsigned* status, int B, int R,
+                               cudaStream_t s);
+
+// ---- GEMMs -------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+int num_sms();
+
+// `status`: device word the kernel ORs kStatusTimeout into if a bounded wait gives up.
+cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
+                                   void* z, int64_t M, int R, unsigned* status, cudaStream_t s);
+cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
+                             unsigned* status, cudaStream_t s);
+cudaError_t launch_gemm_step_bf16(const void* u_t, const void* Wa, const float* ba, const void* Wx,
+                                  const float* bx, const float* cla, float* h, void* y_t, int B, int R,
+                                  unsigned* status, cudaStream_t s);
+// Library-global device status word of the current device (for entry points that take
+// no workspace); null if the symbol address cannot be obtained.
+unsigned* global_status_word();
+cudaError_t launch_gemm_gates_f32(const float* u, const float* Wa, const float* ba, const float* Wx,
+                                  const float* bx, float* z, int64_t M, int R, cudaStream_t s);
+
+}  // namespace rglru

@@ -1,0 +1,385 @@
+// C ABI of librglru.so (declared in include/rglru.h): argument validation, workspace
+// layout and the launch sequence of each entry point. Every argument check happens
+// before the first CUDA call, so an invalid call returns without touching the device.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/rglru.h"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+using namespace rglru;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+int fail_cuda(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return RGLRU_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+size_t esize(int io) { return io == RGLRU_BF16 ? 2 : 4; }
+
+bool valid_dtype(int io) { return io == RGLRU_F32 || io == RGLRU_BF16; }
+
+// R: channels; limits keep every TMA dimension and every 32-bit grid index in range.
+bool valid_R(int R) { return R >= 8 && R % 8 == 0 && R <= 65536; }
+bool valid_tokens(int64_t B, int64_t T) {
+  return B >= 1 && T >= 1 && B <= 65535 && B * T <= (int64_t)INT32_MAX;
+}
+
+// Checks that the current device is a B200-class part (compute capability 10.0).
+int check_device() {
+  static int cc[kMaxDevices] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return RGLRU_ERR_DEVICE;
+  if (cc[dev] == 0) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return fail_cuda(e);
+    cc[dev] = major * 10 + minor;
+  }
+  return cc[dev] == 100 ? RGLRU_OK : RGLRU_ERR_DEVICE;
+}
+
+int check_params(const rglru_params* p) {
+  if (p == nullptr || p->conv_w == nullptr || p->conv_b == nullptr || p->W_a == nullptr || p->b_a == nullptr ||
+      p->W_x == nullptr || p->b_x == nullptr || p->Lambda == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(p->conv_w) || !aligned16(p->conv_b) || !aligned16(p->W_a) || !aligned16(p->b_a) ||
+      !aligned16(p->W_x) || !aligned16(p->b_x) || !aligned16(p->Lambda))
+    return RGLRU_ERR_ALIGN;
+  return RGLRU_OK;
+}
+
+// ---- workspace layouts -------------------------------------------------------------
+struct FwdLayout {
+  ScanLayout scan;
+  size_t off_u, off_z, bytes;
+};
+FwdLayout fwd_layout(int B, int T, int R, int io) {
+  FwdLayout L;
+  L.scan = scan_layout(B, T, R, io == RGLRU_BF16);
+  const size_t ntok = (size_t)B * T;
+  L.off_u = round256(L.scan.bytes);
+  L.off_z = L.off_u + round256(ntok * R * esize(io));
+  L.bytes = L.off_z + round256(ntok * (size_t)gate_pitch(R) * esize(io));
+  return L;
+}
+
+struct BlockLayout {
+  ScanLayout scan;
+  size_t off_v, off_g, off_u, off_z, off_p, bytes;
+};
+BlockLayout block_layout(int B, int T, int R) {
+  BlockLayout L;
+  L.scan = scan_layout(B, T, R, true);
+  const size_t ntok = (size_t)B * T;
+  const size_t act = round256(ntok * R * 2);
+  L.off_v = round256(L.scan.bytes);
+  L.off_g = L.off_v + act;
+  L.off_u = L.off_g + act;
+  L.off_z = L.off_u + act;
+  L.off_p = L.off_z + round256(ntok * (size_t)gate_pitch(R) * 2);
+  L.bytes = L.off_p + act;
+  return L;
+}
+
+struct StepLayout {
+  size_t off_cla, off_u, bytes;
+};
+StepLayout step_layout(int B, int R) {
+  StepLayout L;
+  L.off_cla = 256;
+  L.off_u = L.off_cla + round256((size_t)R * 4);
+  L.bytes = L.off_u + round256((size_t)B * R * 2);
+  return L;
+}
+
+uint8_t* bytes(void* p) { return static_cast<uint8_t*>(p); }
+
+// Queues the scan; with zero_first, first zeroes the status word, the ticket counter and
+// the look-back flags (which must be zero when the scan starts).
+cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_t pitch, const void* state0,
+                     const float* h0, const void* g, void* y, float* hT, int B, int T, int R, bool bf16,
+                     const ScanLayout& sl, void* ws, bool zero_first, cudaStream_t s) {
+  if (zero_first) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, sl.off_carry, s);
+    if (e != cudaSuccess) return e;
+  }
+  ScanArgs a{};
+  a.x = x;
+  a.z = z;
+  a.state0 = state0;
+  a.h0 = h0;
+  a.g = g;
+  a.y = y;
+  a.hT = hT;
+  a.conv_w = p->conv_w;
+  a.conv_b = p->conv_b;
+  a.Lambda = p->Lambda;
+  a.status = reinterpret_cast<unsigned*>(ws);
+  a.ticket = reinterpret_cast<unsigned*>(bytes(ws) + 4);
+  a.flags = reinterpret_cast<unsigned*>(bytes(ws) + sl.off_flags);
+  a.carry = reinterpret_cast<float*>(bytes(ws) + sl.off_carry);
+  a.B = B;
+  a.T = T;
+  a.R = R;
+  a.n_cblk = sl.n_cblk;
+  a.n_chunks = sl.n_chunks;
+  a.pitch = pitch;
+  return launch_scan(a, bf16, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rglru_strerror(int status) {
+  switch (status) {
+    case RGLRU_OK: return "ok";
+    case RGLRU_ERR_NULL: return "a required pointer is NULL";
+    case RGLRU_ERR_SHAPE: return "invalid shape (B, T >= 1; R, D >= 8 and multiples of 8; sizes in range)";
+    case RGLRU_ERR_ALIGN: return "a pointer is not 16-byte aligned (workspace: 256-byte)";
+    case RGLRU_ERR_DTYPE: return "io_dtype not supported by this entry point";
+    case RGLRU_ERR_WORKSPACE: return "workspace missing or too small";
+    case RGLRU_ERR_CUDA: return "a CUDA call failed (see rglru_last_cuda_error)";
+    case RGLRU_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
+    case RGLRU_ERR_DEVICE: return "the current device is not compute capability 10.0 (B200)";
+    default: return "unknown status";
+  }
+}
+
+int rglru_last_cuda_error(void) { return g_last_cuda_error; }
+
+int rglru_debug_scan_stall(int64_t tile) {
+  set_scan_stall(tile < 0 ? -1 : tile);
+  return RGLRU_OK;
+}
+int rglru_version(void) { return 10000; }
+
+int64_t rglru_gate_pitch(int R) { return valid_R(R) ? gate_pitch(R) : 0; }
+
+size_t rglru_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
+  if (!valid_dtype(io_dtype) || !valid_R(R) || !valid_tokens(B, T)) return 0;
+  return scan_layout(B, T, R, io_dtype == RGLRU_BF16).bytes;
+}
+
+size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype) {
+  if (!valid_dtype(io_dtype) || !valid_R(R) || !valid_tokens(B, T)) return 0;
+  return fwd_layout(B, T, R, io_dtype).bytes;
+}
+
+size_t rglru_step_workspace_bytes(int B, int R, int io_dtype) {
+  if (io_dtype != RGLRU_BF16 || !valid_R(R) || !valid_tokens(B, 1)) return 0;
+  return step_layout(B, R).bytes;
+}
+
+size_t rglru_block_workspace_bytes(int B, int T, int D, int R, int io_dtype) {
+  if (io_dtype != RGLRU_BF16 || !valid_R(R) || !valid_R(D) || !valid_tokens(B, T)) return 0;
+  return block_layout(B, T, R).bytes;
+}
+
+int rglru_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* conv_state0, void* u,
+                 void* conv_state_T, int B, int T, int R, int io_dtype, rglru_stream_t stream) {
+  if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  if (conv_w == nullptr || conv_b == nullptr || x == nullptr || u == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(conv_w) || !aligned16(conv_b) || !aligned16(x) || !aligned16(u) || !aligned16(conv_state0) ||
+      !aligned16(conv_state_T))
+    return RGLRU_ERR_ALIGN;
+  int st = check_device();
+  if (st != RGLRU_OK) return st;
+  cudaError_t e = launch_conv1d(conv_w, conv_b, x, conv_state0, u, conv_state_T, B, T, R, io_dtype == RGLRU_BF16,
+                                (cudaStream_t)stream);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_gate_proj(const void* u, const void* W_a, const float* b_a, const void* W_x, const float* b_x, void* z,
+                    int64_t N_tok, int R, int io_dtype, rglru_stream_t stream) {
+  if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || N_tok < 1 || N_tok > (int64_t)INT32_MAX) return RGLRU_ERR_SHAPE;
+  if (u == nullptr || W_a == nullptr || b_a == nullptr || W_x == nullptr || b_x == nullptr || z == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(u) || !aligned16(W_a) || !aligned16(b_a) || !aligned16(W_x) || !aligned16(b_x) || !aligned16(z))
+    return RGLRU_ERR_ALIGN;
+  int st = check_device();
+  if (st != RGLRU_OK) return st;
+  cudaError_t e;
+  if (io_dtype == RGLRU_BF16) {
+    unsigned* status = global_status_word();
+    if (status == nullptr) return fail_cuda(cudaGetLastError());
+    e = launch_gemm_gates_bf16(u, W_a, b_a, W_x, b_x, z, N_tok, R, status, (cudaStream_t)stream);
+  } else {
+    e = launch_gemm_gates_f32(static_cast<const float*>(u), static_cast<const float*>(W_a), b_a,
+                              static_cast<const float*>(W_x), b_x, static_cast<float*>(z), N_tok, R,
+                              (cudaStream_t)stream);
+  }
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_scan(const rglru_params* params, const void* x, const void* z, const void* conv_state0, const float* h0,
+               const void* gate_g, void* y, float* h_T, int B, int T, int R, int io_dtype, void* workspace,
+               size_t workspace_bytes, rglru_stream_t stream) {
+  if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x == nullptr || z == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(x) || !aligned16(z) || !aligned16(y) || !aligned16(conv_state0) || !aligned16(h0) ||
+      !aligned16(gate_g) || !aligned16(h_T))
+    return RGLRU_ERR_ALIGN;
+  const ScanLayout sl = scan_layout(B, T, R, io_dtype == RGLRU_BF16);
+  if (workspace == nullptr || workspace_bytes < sl.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaError_t e = run_scan(params, x, z, gate_pitch(R), conv_state0, h0, gate_g, y, h_T, B, T, R,
+                           io_dtype == RGLRU_BF16, sl, workspace, true, (cudaStream_t)stream);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
+                  float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype, void* workspace,
+                  size_t workspace_bytes, rglru_stream_t stream) {
+  if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(h0) || !aligned16(conv_state0) || !aligned16(h_T) ||
+      !aligned16(conv_state_T))
+    return RGLRU_ERR_ALIGN;
+  const FwdLayout L = fwd_layout(B, T, R, io_dtype);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  const bool bf16 = io_dtype == RGLRU_BF16;
+  cudaStream_t s = (cudaStream_t)stream;
+  void* u = bytes(workspace) + L.off_u;
+  void* z = bytes(workspace) + L.off_z;
+  unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  // status word, ticket and flags are zeroed before the first kernel, so that a status bit
+  // set by the GEMM survives until the caller reads it.
+  cudaError_t e = cudaMemsetAsync(workspace, 0, L.scan.off_carry, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (bf16)
+    e = launch_gemm_gates_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, z, (int64_t)B * T, R, status, s);
+  else
+    e = launch_gemm_gates_f32(static_cast<const float*>(u), static_cast<const float*>(params->W_a), params->b_a,
+                              static_cast<const float*>(params->W_x), params->b_x, static_cast<float*>(z),
+                              (int64_t)B * T, R, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  e = run_scan(params, x, z, gate_pitch(R), conv_state0, h0, nullptr, y, h_T, B, T, R, bf16, L.scan, workspace,
+               false, s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_step(const rglru_params* params, const void* x_t, void* conv_state, float* h, void* y_t, int B, int R,
+               int64_t step, int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_tokens(B, 1) || step < 0) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x_t == nullptr || conv_state == nullptr || h == nullptr || y_t == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(x_t) || !aligned16(conv_state) || !aligned16(h) || !aligned16(y_t)) return RGLRU_ERR_ALIGN;
+  const StepLayout L = step_layout(B, R);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  float* cla = reinterpret_cast<float*>(bytes(workspace) + L.off_cla);
+  void* u_t = bytes(workspace) + L.off_u;
+  unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  cudaError_t e = launch_decode_conv(params->conv_w, params->conv_b, params->Lambda, x_t, conv_state, step, u_t, cla,
+                                     status, B, R, s);
+  if (e != cudaSuccess) return fail_cuda(e);
+  e = launch_gemm_step_bf16(u_t, params->W_a, params->b_a, params->W_x, params->b_x, cla, h, y_t, B, R, status, s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, rglru_stream_t stream) {
+  if (M < 1 || M > (int64_t)INT32_MAX * 128 || !valid_R(N) || !valid_R(K)) return RGLRU_ERR_SHAPE;
+  if (A == nullptr || Bm == nullptr || C == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(A) || !aligned16(Bm) || !aligned16(C)) return RGLRU_ERR_ALIGN;
+  int st = check_device();
+  if (st != RGLRU_OK) return st;
+  unsigned* status = global_status_word();
+  if (status == nullptr) return fail_cuda(cudaGetLastError());
+  cudaError_t e = launch_gemm_bf16(A, Bm, C, M, N, K, N, status, (cudaStream_t)stream);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_block_forward(const rglru_params* params, const void* W_1, const void* W_2, const void* W_o, const void* x,
+                        const float* h0, void* out, float* h_T, int B, int T, int D, int R, int io_dtype,
+                        void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_R(D) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (W_1 == nullptr || W_2 == nullptr || W_o == nullptr || x == nullptr || out == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(W_1) || !aligned16(W_2) || !aligned16(W_o) || !aligned16(x) || !aligned16(out) ||
+      !aligned16(h0) || !aligned16(h_T))
+    return RGLRU_ERR_ALIGN;
+  const BlockLayout L = block_layout(B, T, R);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t ntok = (int64_t)B * T;
+  void* v = bytes(workspace) + L.off_v;
+  void* g = bytes(workspace) + L.off_g;
+  void* u = bytes(workspace) + L.off_u;
+  void* z = bytes(workspace) + L.off_z;
+  void* pbuf = bytes(workspace) + L.off_p;
+  unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(x, W_1, v, ntok, R, D, R, status, s);        // v = x W_1ᵀ
+  if (e == cudaSuccess) e = launch_gemm_bf16(x, W_2, g, ntok, R, D, R, status, s);        // g = x W_2ᵀ
+  if (e == cudaSuccess) e = launch_conv1d(params->conv_w, params->conv_b, v, nullptr, u, nullptr, B, T, R, true, s);
+  if (e == cudaSuccess)
+    e = launch_gemm_gates_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, z, ntok, R, status, s);
+  if (e == cudaSuccess) {
+    // the scan's memset must not clear a status bit the GEMMs above may have set:
+    // zero only the ticket and flags here.
+    e = cudaMemsetAsync(bytes(workspace) + 4, 0, L.scan.off_carry - 4, s);
+    if (e == cudaSuccess) {
+      ScanArgs a{};
+      a.x = v; a.z = z; a.state0 = nullptr; a.h0 = h0; a.g = g; a.y = pbuf; a.hT = h_T;
+      a.conv_w = params->conv_w; a.conv_b = params->conv_b; a.Lambda = params->Lambda;
+      a.status = status;
+      a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
+      a.flags = reinterpret_cast<unsigned*>(bytes(workspace) + L.scan.off_flags);
+      a.carry = reinterpret_cast<float*>(bytes(workspace) + L.scan.off_carry);
+      a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks; a.pitch = gate_pitch(R);
+      e = launch_scan(a, true, s);
+    }
+  }
+  if (e == cudaSuccess) e = launch_gemm_bf16(pbuf, W_o, out, ntok, D, R, D, status, s);  // out = p W_oᵀ
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_workspace_status(void* workspace, rglru_stream_t stream) {
+  unsigned* word = workspace != nullptr ? reinterpret_cast<unsigned*>(workspace) : global_status_word();
+  if (word == nullptr) return fail_cuda(cudaGetLastError());
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail_cuda(e);
+  unsigned v = 0;
+  e = cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e);
+  e = cudaMemset(word, 0, sizeof(v));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return (v & kStatusTimeout) ? RGLRU_ERR_TIMEOUT : RGLRU_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,208 @@
+"""Python binding of librglru.so: the same entry points as include/rglru.h, taking torch
+tensors. Only argument marshalling happens here — PyTorch provides device memory and
+streams; every step of the layer runs in the library's CUDA kernels. There is no CPU or
+PyTorch fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+from . import _abi
+
+_DT = {torch.float32: _abi.RGLRU_F32, torch.bfloat16: _abi.RGLRU_BF16}
+
+
+def _io(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {t.dtype}: use torch.bfloat16 or torch.float32")
+    return _DT[t.dtype]
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("librglru takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("librglru takes contiguous tensors only")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream: Optional[torch.cuda.Stream]):
+    st = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(st.cuda_stream)
+
+
+@dataclass
+class Params:
+    """Device-resident layer parameters (see rglru_params in include/rglru.h)."""
+    conv_w: torch.Tensor   # [4][R] float32
+    conv_b: torch.Tensor   # [R] float32
+    W_a: torch.Tensor      # [R][R] io dtype
+    b_a: torch.Tensor      # [R] float32
+    W_x: torch.Tensor      # [R][R] io dtype
+    b_x: torch.Tensor      # [R] float32
+    Lambda: torch.Tensor   # [R] float32
+
+    @classmethod
+    def from_host(cls, p, device="cuda") -> "Params":
+        """Copies an object with the same fields (e.g. inputs.RGLRUParams) to `device`."""
+        return cls(*(getattr(p, f).to(device).contiguous() for f in
+                     ("conv_w", "conv_b", "W_a", "b_a", "W_x", "b_x", "Lambda")))
+
+    @property
+    def R(self) -> int:
+        return self.conv_b.numel()
+
+    def struct(self) -> _abi.RGLRUParams:
+        return _abi.RGLRUParams(*(t.data_ptr() for t in (self.conv_w, self.conv_b, self.W_a, self.b_a,
+                                                          self.W_x, self.b_x, self.Lambda)))
+
+
+def _workspace(nbytes: int, device, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return ws
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def forward_workspace_bytes(B: int, T: int, R: int, dtype: torch.dtype) -> int:
+    return _abi.load().rglru_forward_workspace_bytes(B, T, R, _DT[dtype])
+
+
+def forward(params: Params, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
+            conv_state0: Optional[torch.Tensor] = None, *, workspace: Optional[torch.Tensor] = None,
+            y: Optional[torch.Tensor] = None, h_T: Optional[torch.Tensor] = None,
+            conv_state_T: Optional[torch.Tensor] = None, want_conv_state: bool = True,
+            stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """rglru_forward: x [B][T][R] → (y [B][T][R], h_T [B][R] fp32, conv_state_T [B][3][R])."""
+    lib = _abi.load()
+    B, T, R = x.shape
+    io = _io(x)
+    y = torch.empty_like(x) if y is None else y
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
+    if conv_state_T is None and want_conv_state:
+        conv_state_T = torch.empty(B, 3, R, dtype=x.dtype, device=x.device)
+    ws = _workspace(lib.rglru_forward_workspace_bytes(B, T, R, io), x.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_forward", lib.rglru_forward(
+        ctypes.byref(st), _p(x), _p(h0), _p(conv_state0), _p(y), _p(h_T), _p(conv_state_T), B, T, R, io,
+        _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+    return y, h_T, conv_state_T
+
+
+def step_workspace_bytes(B: int, R: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    return _abi.load().rglru_step_workspace_bytes(B, R, _DT[dtype])
+
+
+def step(params: Params, x_t: torch.Tensor, conv_state: torch.Tensor, h: torch.Tensor, step_index: int, *,
+         workspace: Optional[torch.Tensor] = None, y_t: Optional[torch.Tensor] = None,
+         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_step: one decode step; updates conv_state and h in place, returns y_t."""
+    lib = _abi.load()
+    B, R = x_t.shape
+    io = _io(x_t)
+    y_t = torch.empty_like(x_t) if y_t is None else y_t
+    ws = _workspace(lib.rglru_step_workspace_bytes(B, R, io), x_t.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_step", lib.rglru_step(
+        ctypes.byref(st), _p(x_t), _p(conv_state), _p(h), _p(y_t), B, R, int(step_index), io, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return y_t
+
+
+def block_workspace_bytes(B: int, T: int, D: int, R: int) -> int:
+    return _abi.load().rglru_block_workspace_bytes(B, T, D, R, _abi.RGLRU_BF16)
+
+
+def block_forward(params: Params, W_1: torch.Tensor, W_2: torch.Tensor, W_o: torch.Tensor, x: torch.Tensor,
+                  h0: Optional[torch.Tensor] = None, *, workspace: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, h_T: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """rglru_block_forward: x [B][T][D] → (out [B][T][D], h_T [B][R])."""
+    lib = _abi.load()
+    B, T, D = x.shape
+    R = W_1.shape[0]
+    io = _io(x)
+    out = torch.empty_like(x) if out is None else out
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_block_workspace_bytes(B, T, D, R, io), x.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_block_forward", lib.rglru_block_forward(
+        ctypes.byref(st), _p(W_1), _p(W_2), _p(W_o), _p(x), _p(h0), _p(out), _p(h_T), B, T, D, R, io, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return out, h_T
+
+
+def conv1d(params: Params, x: torch.Tensor, conv_state0: Optional[torch.Tensor] = None, *,
+           u: Optional[torch.Tensor] = None, conv_state_T: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    lib = _abi.load()
+    B, T, R = x.shape
+    u = torch.empty_like(x) if u is None else u
+    _abi.check("rglru_conv1d", lib.rglru_conv1d(_p(params.conv_w), _p(params.conv_b), _p(x), _p(conv_state0),
+                                                _p(u), _p(conv_state_T), B, T, R, _io(x), _s(stream)))
+    return u
+
+
+def gate_pitch(R: int) -> int:
+    return int(_abi.load().rglru_gate_pitch(R))
+
+
+def gate_proj(params: Params, u: torch.Tensor, *, z: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_gate_proj: u [N][R] (or [B][T][R]) → packed z [N][gate_pitch(R)]."""
+    lib = _abi.load()
+    R = u.shape[-1]
+    N = u.numel() // R
+    z = torch.empty(N, gate_pitch(R), dtype=u.dtype, device=u.device) if z is None else z
+    _abi.check("rglru_gate_proj", lib.rglru_gate_proj(_p(u), _p(params.W_a), _p(params.b_a), _p(params.W_x),
+                                                      _p(params.b_x), _p(z), N, R, _io(u), _s(stream)))
+    return z
+
+
+def scan_workspace_bytes(B: int, T: int, R: int, dtype: torch.dtype) -> int:
+    return _abi.load().rglru_scan_workspace_bytes(B, T, R, _DT[dtype])
+
+
+def scan(params: Params, x: torch.Tensor, z: torch.Tensor, h0: Optional[torch.Tensor] = None,
+         conv_state0: Optional[torch.Tensor] = None, gate_g: Optional[torch.Tensor] = None, *,
+         workspace: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+         h_T: Optional[torch.Tensor] = None,
+         stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """rglru_scan: (x, packed z) → (y, h_T)."""
+    lib = _abi.load()
+    B, T, R = x.shape
+    io = _io(x)
+    y = torch.empty_like(x) if y is None else y
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_scan_workspace_bytes(B, T, R, io), x.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_scan", lib.rglru_scan(
+        ctypes.byref(st), _p(x), _p(z), _p(conv_state0), _p(h0), _p(gate_g), _p(y), _p(h_T), B, T, R, io, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return y, h_T
+
+
+def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, *, C: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_gemm_bf16: C[M][N] = A[M][K] · B[N][K]ᵀ (bf16 in/out, fp32 accumulate)."""
+    lib = _abi.load()
+    K = A.shape[-1]
+    M = A.numel() // K
+    N = Bm.shape[0]
+    C = torch.empty(*A.shape[:-1], N, dtype=torch.bfloat16, device=A.device) if C is None else C
+    _abi.check("rglru_gemm_bf16", lib.rglru_gemm_bf16(_p(A), _p(Bm), _p(C), M, N, K, _s(stream)))
+    return C
+
+
+def workspace_status(workspace: Optional[torch.Tensor], stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronises the stream and returns (and clears) the status word of `workspace`
+    (None: the library-global word used by calls that take no workspace)."""
+    lib = _abi.load()
+    return lib.rglru_workspace_status(_p(workspace) if workspace is not None else None, _s(stream))

@@ -1,0 +1,196 @@
+/*
+ * rglru.h — C ABI of the B200 (sm_100a) RG-LRU temporal core library (librglru.so).
+ *
+ * The layer computed here is the recurrent branch of the Griffin/Hawk recurrent
+ * block: a width-4 causal depthwise Conv1D followed by the Real-Gated Linear
+ * Recurrent Unit, as defined in "Griffin：将门控线性循环与局部注意力混合以实现高效的
+ * 语言模型", §实门线性循环单元 (RG-LRU), Eq. (1)–(4) and the paragraph after them,
+ * and §循环块 (recurrent block, Fig. 2(c)):
+ *
+ *     u_t = conv_b + Σ_{k=0..3} conv_w[k] ⊙ x_{t-3+k}              (Conv1D, width 4)
+ *     r_t = σ(W_a u_t + b_a)                                       (1)
+ *     i_t = σ(W_x u_t + b_x)                                       (2)
+ *     a_t = a^(c r_t),  a = σ(Λ),  c = 8, evaluated in log space    (3)
+ *     h_t = a_t ⊙ h_{t-1} + √(1 − a_t²) ⊙ (i_t ⊙ u_t),  y_t = h_t   (4)
+ *
+ * Conventions shared by every entry point
+ *   - R is D_RNN, the channel count. R must be a multiple of 8 (16-byte rows).
+ *   - Row-major layouts; "[B][T][R]" means R is contiguous.
+ *   - io_dtype selects the type of x, y, u, W_a, W_x and the conv ring:
+ *     RGLRU_BF16 (bfloat16) or RGLRU_F32 (float32). Recurrent state h, all gate
+ *     arithmetic and accumulation are float32 in both cases. Per-channel parameters
+ *     (conv_w, conv_b, b_a, b_x, Λ) are always float32.
+ *   - W_a and W_x are dense [R][R] matrices in [out][in] order (z = W u).
+ *   - conv_w is [4][R]; tap k multiplies x_{t-3+k} (k = 3 is the current input).
+ *   - Every pointer is a DEVICE pointer on the current CUDA device, 16-byte aligned,
+ *     unless stated otherwise. The caller owns every buffer, including workspace;
+ *     the library never allocates, frees, or synchronises (except
+ *     rglru_workspace_status). All work is queued on `stream` (a cudaStream_t;
+ *     NULL means the legacy default stream).
+ *   - Return value: RGLRU_OK (0) or a negative rglru_status. On an argument error
+ *     nothing is launched. Outputs are undefined after any error.
+ *   - Not thread-safe for concurrent calls that share a workspace.
+ */
+#ifndef RGLRU_H_
+#define RGLRU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RGLRU_API __attribute__((visibility("default")))
+#else
+#define RGLRU_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* rglru_stream_t; /* identical to cudaStream_t */
+
+typedef enum { RGLRU_F32 = 0, RGLRU_BF16 = 1 } rglru_dtype;
+
+typedef enum {
+  RGLRU_OK = 0,
+  RGLRU_ERR_NULL = -1,      /* a required pointer is NULL */
+  RGLRU_ERR_SHAPE = -2,     /* B < 1, T < 1, R < 8, R % 8 != 0, D % 8 != 0, or a size overflows int32 indexing */
+  RGLRU_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned */
+  RGLRU_ERR_DTYPE = -4,     /* io_dtype not supported by this entry point */
+  RGLRU_ERR_WORKSPACE = -5, /* workspace NULL or smaller than the *_workspace_bytes query */
+  RGLRU_ERR_CUDA = -6,      /* a CUDA call failed; see rglru_last_cuda_error() */
+  RGLRU_ERR_TIMEOUT = -7,   /* a bounded wait inside a kernel gave up (reported by rglru_workspace_status) */
+  RGLRU_ERR_DEVICE = -8     /* the current device is not compute capability 10.0 (B200) */
+} rglru_status;
+
+/* Per-layer parameters of the Conv1D and the RG-LRU (device pointers). */
+typedef struct {
+  const float* conv_w; /* [4][R]   Conv1D taps, tap k multiplies x_{t-3+k}           */
+  const float* conv_b; /* [R]      Conv1D bias                                         */
+  const void* W_a;     /* [R][R]   recurrence-gate weight, io_dtype, Eq. (1)          */
+  const float* b_a;    /* [R]      recurrence-gate bias, Eq. (1)                       */
+  const void* W_x;     /* [R][R]   input-gate weight, io_dtype, Eq. (2)               */
+  const float* b_x;    /* [R]      input-gate bias, Eq. (2)                            */
+  const float* Lambda; /* [R]      Λ, with a = σ(Λ), Eq. (3)                           */
+} rglru_params;
+
+/* ---------------------------------------------------------------------------------
+ * Full-sequence forward (prefill / training forward): Conv1D(4) → RG-LRU over T steps.
+ * Eq. (1)–(4) above; the time recurrence is evaluated as a chunked scan (the
+ * recurrence is linear in h because neither gate reads h_{t-1}; "Griffin's
+ * Compromise: Combining Gated Linear Recurrence with Local Attention", §Hawk,
+ * "Parallel scan").
+ *
+ *   x            [B][T][R] io_dtype, input of the Conv1D
+ *   h0           [B][R] float32 initial state, or NULL for zeros
+ *   conv_state0  [B][3][R] io_dtype: (x_{-3}, x_{-2}, x_{-1}) in time order, or NULL
+ *                for zeros (zero left padding)
+ *   y            [B][T][R] io_dtype output, y_t = h_t
+ *   h_T          [B][R] float32 final state (may be NULL)
+ *   conv_state_T [B][3][R] io_dtype: (x_{T-3}, x_{T-2}, x_{T-1}) in time order (may be NULL)
+ *   workspace    device buffer of at least rglru_forward_workspace_bytes(B, T, R, io_dtype)
+ *                bytes, 256-byte aligned. It holds u, the gate pre-activations and the
+ *                scan's chunk carries; its contents need no initialisation.
+ * Kernels: conv (x → u), gate GEMM (u → [z_a | z_x], tcgen05 tensor cores for bf16,
+ * FFMA for f32), fused gates + log-space decay + chunked scan (→ y, h_T).
+ * --------------------------------------------------------------------------------- */
+RGLRU_API size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype);
+RGLRU_API int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0,
+                  void* y, float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype,
+                  void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * One decode step on a carried state ("Griffin's Compromise…", §Hawk: generation reads
+ * and writes only the current token and a fixed-size state), Eq. (1)–(4) at one t.
+ *
+ *   x_t         [B][R] io_dtype current input
+ *   conv_state  [B][3][R] io_dtype ring of the last three inputs, updated IN PLACE:
+ *               slot (step mod 3) holds x_{t-3}, slot (step+1) mod 3 holds x_{t-2},
+ *               slot (step+2) mod 3 holds x_{t-1}; on return slot (step mod 3) holds x_t.
+ *               A state in time order (as rglru_forward writes it) is the ring at any
+ *               step ≡ 0 (mod 3).
+ *   step        ≥ 0, the ring position described above
+ *   h           [B][R] float32 state, updated IN PLACE (h_{t-1} → h_t)
+ *   y_t         [B][R] io_dtype output (= new h)
+ *   workspace   at least rglru_step_workspace_bytes(B, R, io_dtype) bytes (holds u_t)
+ * io_dtype must be RGLRU_BF16 (the tensor-core path) for this entry point.
+ * --------------------------------------------------------------------------------- */
+RGLRU_API size_t rglru_step_workspace_bytes(int B, int R, int io_dtype);
+RGLRU_API int rglru_step(const rglru_params* params, const void* x_t, void* conv_state, float* h, void* y_t, int B,
+               int R, int64_t step, int io_dtype, void* workspace, size_t workspace_bytes,
+               rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Recurrent block ("Griffin：…", §循环块, Fig. 2(c)):
+ *   v = x W_1ᵀ, g = x W_2ᵀ                (two D → D_RNN linears, no bias)
+ *   h = RG-LRU(Conv1D(v))                  (as rglru_forward, zero conv history)
+ *   out = (h ⊙ GeLU(g)) W_oᵀ               (exact erf GeLU; D_RNN → D linear, no bias)
+ *
+ *   x [B][T][D], W_1 and W_2 [R][D], W_o [D][R], out [B][T][D]: all bfloat16.
+ *   h0 [B][R] float32 or NULL; h_T [B][R] float32 or NULL.
+ *   io_dtype must be RGLRU_BF16. D % 8 == 0.
+ * --------------------------------------------------------------------------------- */
+RGLRU_API size_t rglru_block_workspace_bytes(int B, int T, int D, int R, int io_dtype);
+RGLRU_API int rglru_block_forward(const rglru_params* params, const void* W_1, const void* W_2, const void* W_o,
+                        const void* x, const float* h0, void* out, float* h_T, int B, int T, int D, int R,
+                        int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * The three stages of rglru_forward, callable one by one (for per-kernel timing and
+ * for testing each stage against the oracle). rglru_forward runs exactly these.
+ *
+ * rglru_conv1d: u = Conv1D(x) (§循环块). x, u [B][T][R] io_dtype; conv_state0 as in
+ *   rglru_forward (NULL = zeros); conv_state_T may be NULL.
+ *
+ * rglru_gate_proj: z = u [W_a | W_x]ᵀ + [b_a | b_x] for N_tok = B·T rows (Eq. (1)–(2)
+ *   arguments of σ). z is written in the PACKED gate layout: row n has
+ *   rglru_gate_pitch(R) elements; channel c's recurrence-gate pre-activation sits at
+ *   column 256·(c / 128) + (c % 128) and its input-gate pre-activation at
+ *   256·(c / 128) + 128 + (c % 128). Columns of a partial last block are unused.
+ *   z has io_dtype (bf16 rounding of the fp32 accumulator for RGLRU_BF16).
+ *
+ * rglru_scan: Eq. (1)–(4) given x and the packed z: recomputes u from x (fp32),
+ *   applies σ, the log-space decay and the chunked recurrence. If gate_g is non-NULL
+ *   ([B][T][R] io_dtype) the output is y_t = h_t ⊙ GeLU(g_t) (the block's product),
+ *   otherwise y_t = h_t. h_T [B][R] (may be NULL) is the final state in both cases.
+ *   workspace: at least rglru_scan_workspace_bytes(B, T, R, io_dtype) bytes.
+ * --------------------------------------------------------------------------------- */
+RGLRU_API int rglru_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* conv_state0, void* u,
+                 void* conv_state_T, int B, int T, int R, int io_dtype, rglru_stream_t stream);
+RGLRU_API int64_t rglru_gate_pitch(int R);
+RGLRU_API int rglru_gate_proj(const void* u, const void* W_a, const float* b_a, const void* W_x, const float* b_x,
+                    void* z, int64_t N_tok, int R, int io_dtype, rglru_stream_t stream);
+RGLRU_API size_t rglru_scan_workspace_bytes(int B, int T, int R, int io_dtype);
+RGLRU_API int rglru_scan(const rglru_params* params, const void* x, const void* z, const void* conv_state0,
+               const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R, int io_dtype,
+               void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+
+/* Dense bf16 GEMM C[M][N] = A[M][K] · B[N][K]ᵀ on the tcgen05 tensor cores (fp32
+ * accumulate, bf16 store), the kernel behind the block's linears. K % 8 == 0, N % 8 == 0. */
+RGLRU_API int rglru_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Status and diagnostics
+ * --------------------------------------------------------------------------------- */
+/* Synchronises `stream`, reads and clears the device status word that kernels using
+ * `workspace` (forward, scan, block) write; returns RGLRU_OK or RGLRU_ERR_TIMEOUT. */
+RGLRU_API int rglru_workspace_status(void* workspace, rglru_stream_t stream);
+/* Text for a status code (static storage). */
+RGLRU_API const char* rglru_strerror(int status);
+/* The cudaError_t of the last RGLRU_ERR_CUDA on this thread (0 if none). */
+RGLRU_API int rglru_last_cuda_error(void);
+/* TESTING ONLY. Makes every later scan (rglru_scan, rglru_forward, rglru_block_forward)
+ * leave the chunk carry of tile `tile` unpublished, so that the CTAs waiting for it run
+ * into their bounded wait (about one second), give up, and set RGLRU_ERR_TIMEOUT in the
+ * workspace status word; the outputs are then wrong but every kernel ends. Tile index =
+ * ((b · n_channel_blocks + channel_block) · n_time_chunks + time_chunk) with 64-step
+ * time chunks and 128 (bf16) or 64 (f32) channels per block. A negative value turns the
+ * injection off. Always returns RGLRU_OK. */
+RGLRU_API int rglru_debug_scan_stall(int64_t tile);
+/* Library version: major*10000 + minor*100 + patch. */
+RGLRU_API int rglru_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RGLRU_H_ */

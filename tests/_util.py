@@ -1,0 +1,48 @@
+"""Shared test helpers: float64 views of tensors, the packed gate layout, oracle calls."""
+import numpy as np
+import torch
+
+import oracle
+
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+
+def f64(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64)
+    return t.detach().to("cpu").double().numpy()
+
+
+def unpack_gates(z, R):
+    """Packed gate rows [N][pitch] → (z_a [N][R], z_x [N][R]).
+
+    Channel c's recurrence-gate pre-activation sits at column 256·(c//128) + c%128, its
+    input-gate pre-activation 128 columns further."""
+    z = f64(z)
+    c = np.arange(R)
+    col_a = 256 * (c // 128) + (c % 128)
+    return z[:, col_a], z[:, col_a + 128]
+
+
+def pack_gates(z_a, z_x, R, dtype, device):
+    """Inverse of unpack_gates (unused columns zero)."""
+    N = z_a.shape[0]
+    pitch = ((R + 127) // 128) * 256
+    out = np.zeros((N, pitch))
+    c = np.arange(R)
+    col_a = 256 * (c // 128) + (c % 128)
+    out[:, col_a] = z_a
+    out[:, col_a + 128] = z_x
+    return torch.from_numpy(out).to(dtype).to(device)
+
+
+def host_params64(p):
+    """float64 numpy copies of a parameter set (so repeated oracle calls skip conversion)."""
+    return dict(conv_w=f64(p.conv_w), conv_b=f64(p.conv_b), W_a=f64(p.W_a), b_a=f64(p.b_a), W_x=f64(p.W_x),
+                b_x=f64(p.b_x), Lambda=f64(p.Lambda))
+
+
+def rel(got, ref):
+    return oracle.max_rel_error(f64(got), f64(ref))

@@ -1,0 +1,103 @@
+"""Host-side checks of librglru.so that need no GPU: it loads, exports every function
+include/rglru.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_linear_rnn_conv1d_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rglru.h")
+
+
+def _declared():
+    text = open(HEADER, encoding="utf-8").read()
+    return sorted(set(re.findall(r"RGLRU_API\s+[\w\s\*]+?\b(rglru_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _abi.load()
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _abi.SIGNATURES, f"binding lacks {n}"
+
+
+def test_version_and_strerror():
+    lib = _abi.load()
+    assert lib.rglru_version() == 10000
+    for code in range(-8, 1):
+        assert lib.rglru_strerror(code)
+    assert lib.rglru_strerror(-99) == b"unknown status"
+
+
+def _fake(addr=0x100000):
+    return ctypes.c_void_p(addr)
+
+
+def _params(addr=0x100000):
+    return _abi.RGLRUParams(*([addr] * 7))
+
+
+def test_argument_errors_are_returned_before_any_launch():
+    lib = _abi.load()
+    p = _params()
+    ws_bytes = lib.rglru_forward_workspace_bytes(1, 64, 256, 1)
+    ok_ptr = _fake()
+    ws = _fake(0x200000)
+    args = lambda **kw: dict(dict(params=ctypes.byref(p), x=ok_ptr, h0=None, st0=None, y=ok_ptr, hT=None, stT=None,
+                                  B=1, T=64, R=256, io=1, ws=ws, wsb=ws_bytes), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return lib.rglru_forward(a["params"], a["x"], a["h0"], a["st0"], a["y"], a["hT"], a["stT"], a["B"], a["T"],
+                                 a["R"], a["io"], a["ws"], a["wsb"], None)
+
+    assert call(io=7) == -4
+    assert call(R=12) == -2
+    assert call(R=0) == -2
+    assert call(T=0) == -2
+    assert call(B=0) == -2
+    assert call(params=None) == -1
+    assert call(x=None) == -1
+    assert call(x=_fake(0x100004)) == -3
+    assert call(ws=None) == -5
+    assert call(wsb=ws_bytes - 1) == -5
+    assert call(ws=_fake(0x200010)) == -3
+    bad = _abi.RGLRUParams(0x100000, 0x100000, 0, 0x100000, 0x100000, 0x100000, 0x100000)
+    assert call(params=ctypes.byref(bad)) == -1
+    # decode takes bf16 only and a non-negative step
+    sb = lib.rglru_step_workspace_bytes(4, 256, 1)
+    assert sb > 0 and lib.rglru_step_workspace_bytes(4, 256, 0) == 0
+    assert lib.rglru_step(ctypes.byref(p), ok_ptr, ok_ptr, ok_ptr, ok_ptr, 4, 256, 0, 0, ws, sb, None) == -4
+    assert lib.rglru_step(ctypes.byref(p), ok_ptr, ok_ptr, ok_ptr, ok_ptr, 4, 256, -1, 1, ws, sb, None) == -2
+    assert lib.rglru_step(ctypes.byref(p), ok_ptr, None, ok_ptr, ok_ptr, 4, 256, 0, 1, ws, sb, None) == -1
+    # GEMM and block
+    assert lib.rglru_gemm_bf16(ok_ptr, ok_ptr, ok_ptr, 0, 64, 64, None) == -2
+    assert lib.rglru_gemm_bf16(ok_ptr, ok_ptr, ok_ptr, 16, 60, 64, None) == -2
+    assert lib.rglru_gemm_bf16(ok_ptr, None, ok_ptr, 16, 64, 64, None) == -1
+    bb = lib.rglru_block_workspace_bytes(1, 8, 64, 64, 1)
+    assert lib.rglru_block_forward(ctypes.byref(p), ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, ok_ptr, None, 1, 8, 64, 64,
+                                   0, ws, bb, None) == -4
+    assert lib.rglru_block_forward(ctypes.byref(p), ok_ptr, ok_ptr, ok_ptr, ok_ptr, None, ok_ptr, None, 1, 8, 60, 64,
+                                   1, ws, bb, None) == -2
+
+
+def test_workspace_queries():
+    lib = _abi.load()
+    assert lib.rglru_forward_workspace_bytes(1, 1, 8, 1) > 0
+    assert lib.rglru_forward_workspace_bytes(1, 1, 7, 1) == 0
+    a = lib.rglru_forward_workspace_bytes(8, 2048, 2048, 1)
+    b = lib.rglru_forward_workspace_bytes(8, 2048, 2048, 0)
+    # bf16: u (2 B) + packed z (2·2 B per channel) per token, plus chunk carries
+    assert 8 * 2048 * 2048 * 6 <= a < 8 * 2048 * 2048 * 6 * 1.05
+    assert b > a
+    assert lib.rglru_gate_pitch(256) == 512
+    assert lib.rglru_gate_pitch(264) == 768      # partial last 128-channel block
+    assert lib.rglru_gate_pitch(5632) == 11264
+    assert lib.rglru_gate_pitch(12) == 0
+    assert lib.rglru_scan_workspace_bytes(1, 64, 128, 1) > 256
+    assert lib.rglru_block_workspace_bytes(4, 4096, 4096, 5632, 1) > 4 * 4096 * 5632 * 2 * 5

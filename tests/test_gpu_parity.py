@@ -1,0 +1,274 @@
+"""CUDA path vs the float64 oracle, element by element, at sizes that span several tiles
+and end in ragged tails; plus the invariants of the recurrence checked on the GPU.
+
+Tolerances (max_i |g−o| / max(|o_i|, rms(o))): 1e-4 on the float32-IO path and 2e-2 on
+the bf16-IO path with float32 state, per output tensor."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_linear_rnn_conv1d_b200 import _abi, inputs, rglru
+
+from _util import TOL, f64, host_params64, pack_gates, rel, unpack_gates
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _wl(B, T, R, dtype, seed=0):
+    w = inputs.make_forward(B, T, R, dtype, seed=seed)
+    g = torch.Generator("cpu").manual_seed(seed + 77)
+    # non-zero biases, initial state and conv history so that every input is exercised
+    w.params.b_a = torch.randn(R, generator=g) * 0.5
+    w.params.b_x = torch.randn(R, generator=g) * 0.5
+    w.h0 = torch.randn(B, R, generator=g)
+    w.extra["state0"] = torch.randn(B, 3, R, generator=g).to(dtype)
+    return w
+
+
+def _nan_like(t):
+    return torch.full_like(t, float("nan"))
+
+
+# ------------------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,B,T,R", [(torch.float32, 1, 256, 256), (torch.bfloat16, 2, 77, 264),
+                                         (torch.bfloat16, 3, 2, 8), (torch.float32, 2, 100, 72)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_conv1d_matches_oracle(dtype, B, T, R, with_state):
+    w = _wl(B, T, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    st0 = w.extra["state0"].to(DEV) if with_state else None
+    u = _nan_like(x)
+    stT = torch.full((B, 3, R), float("nan"), dtype=dtype, device=DEV)
+    rglru.conv1d(p, x, st0, u=u, conv_state_T=stT)
+    u_ref, st_ref = oracle.conv1d_causal(w.x, w.params.conv_w, w.params.conv_b,
+                                         w.extra["state0"] if with_state else None)
+    tol = 1e-6 if dtype == torch.float32 else 4e-3
+    assert rel(u, u_ref) <= tol
+    # the carried conv state is the last three inputs, copied exactly
+    assert np.array_equal(f64(stT), st_ref)
+
+
+@pytest.mark.parametrize("dtype,N,R", [(torch.float32, 256, 256), (torch.bfloat16, 300, 264),
+                                       (torch.bfloat16, 128, 128), (torch.bfloat16, 1000, 1040),
+                                       (torch.float32, 77, 136)])
+def test_gate_projection_matches_oracle(dtype, N, R):
+    w = _wl(1, N, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    g = torch.Generator("cpu").manual_seed(5)
+    u = torch.randn(N, R, generator=g).to(dtype)
+    z = rglru.gate_proj(p, u.to(DEV))
+    za, zx = unpack_gates(z, R)
+    ra, rx = oracle.gate_preactivations(u, w.params.W_a, w.params.b_a, w.params.W_x, w.params.b_x)
+    tol = 1e-5 if dtype == torch.float32 else 8e-3
+    assert rel(za, ra) <= tol and rel(zx, rx) <= tol
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 136, 200), (1024, 512, 1024), (128, 256, 64), (129, 264, 72),
+                                   (4096, 1024, 4096)])
+def test_gemm_bf16_matches_matmul(M, N, K):
+    g = torch.Generator("cpu").manual_seed(M + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    Bm = (torch.randn(N, K, generator=g) / math.sqrt(K)).to(torch.bfloat16)
+    C = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    rglru.gemm_bf16(A.to(DEV), Bm.to(DEV), C=C)
+    ref = f64(A) @ f64(Bm).T
+    assert rel(C, ref) <= 8e-3
+    assert _abi.load().rglru_workspace_status(None, None) == 0
+
+
+def _scan_reference(w, za, zx, with_state, gate=None):
+    """Oracle scan given (rounded) gate pre-activations: the GPU scan's own inputs."""
+    u, _ = oracle.conv1d_causal(w.x, w.params.conv_w, w.params.conv_b, w.extra["state0"] if with_state else None)
+    B, T, R = w.x.shape
+    r = oracle.sigmoid(za.reshape(B, T, R))
+    i = oracle.sigmoid(zx.reshape(B, T, R))
+    a_t = oracle.decay_direct(r, f64(w.params.Lambda))
+    y, h_T = oracle.rglru_recurrence(a_t, i, u, f64(w.h0))
+    if gate is not None:
+        y = y * oracle.gelu(gate)
+    return y, h_T
+
+
+@pytest.mark.parametrize("dtype,B,T,R", [(torch.bfloat16, 2, 200, 264), (torch.float32, 1, 256, 256),
+                                         (torch.float32, 3, 130, 72), (torch.bfloat16, 1, 1000, 128),
+                                         (torch.bfloat16, 2, 3, 8)])
+@pytest.mark.parametrize("gated", [False, True])
+def test_scan_matches_oracle(dtype, B, T, R, gated):
+    w = _wl(B, T, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    u, _ = oracle.conv1d_causal(w.x, w.params.conv_w, w.params.conv_b, w.extra["state0"])
+    za, zx = oracle.gate_preactivations(u.reshape(B * T, R), w.params.W_a, w.params.b_a, w.params.W_x, w.params.b_x)
+    z = pack_gates(za, zx, R, dtype, DEV)
+    za_r, zx_r = unpack_gates(z, R)                 # what the GPU sees after rounding
+    gate = None
+    if gated:
+        gate = torch.randn(B, T, R, generator=torch.Generator("cpu").manual_seed(3)).to(dtype)
+    y = torch.full((B, T, R), float("nan"), dtype=dtype, device=DEV)
+    h_T = torch.full((B, R), float("nan"), device=DEV)
+    rglru.scan(p, w.x.to(DEV), z, w.h0.to(DEV), w.extra["state0"].to(DEV),
+               gate.to(DEV) if gated else None, y=y, h_T=h_T)
+    y_ref, h_ref = _scan_reference(w, za_r, zx_r, True, gate)
+    assert rel(y, y_ref) <= TOL[dtype]
+    assert rel(h_T, h_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype,B,T,R", [(torch.float32, 1, 256, 256), (torch.bfloat16, 2, 200, 264),
+                                         (torch.bfloat16, 1, 65, 8), (torch.bfloat16, 4, 1, 136),
+                                         (torch.float32, 2, 190, 136)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_forward_matches_oracle(dtype, B, T, R, with_state):
+    w = _wl(B, T, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    h0 = w.h0 if with_state else None
+    st0 = w.extra["state0"] if with_state else None
+    y = torch.full((B, T, R), float("nan"), dtype=dtype, device=DEV)
+    y, h_T, stT = rglru.forward(p, w.x.to(DEV), h0.to(DEV) if with_state else None,
+                                st0.to(DEV) if with_state else None, y=y)
+    ws_status = rglru.workspace_status(None)
+    y_ref, h_ref, st_ref = oracle.rglru_forward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a,
+                                                w.params.b_a, w.params.W_x, w.params.b_x, w.params.Lambda,
+                                                h0=h0, conv_state0=st0)
+    assert ws_status == 0
+    assert rel(y, y_ref) <= TOL[dtype]
+    assert rel(h_T, h_ref) <= TOL[dtype]
+    assert np.array_equal(f64(stT), st_ref)
+
+
+# ------------------------------------------------------------------------------------
+# invariants on the GPU path
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_zero_recurrence_gate_keeps_state_bitwise(dtype):
+    """r ≡ 0 ⇒ a_t = 1 and √(1−a_t²) = 0 exactly, so h_t = h_0 bit for bit."""
+    B, T, R = 2, 150, 136
+    w = _wl(B, T, R, dtype)
+    w.params.W_a = torch.zeros(R, R, dtype=dtype)
+    w.params.b_a = torch.full((R,), -1000.0)
+    p = rglru.Params.from_host(w.params)
+    h0 = w.h0.to(DEV)
+    y, h_T, _ = rglru.forward(p, w.x.to(DEV), h0)
+    assert torch.equal(h_T, h0)
+    assert torch.equal(y.float(), h0.to(dtype).float()[:, None, :].expand(B, T, R))
+
+
+def test_batch_rows_are_independent_bitwise():
+    B, T, R = 3, 300, 264
+    w = _wl(B, T, R, torch.bfloat16)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    y, h_T, _ = rglru.forward(p, x)
+    y1, h1, _ = rglru.forward(p, x[1:2].contiguous())
+    assert torch.equal(y[1:2], y1) and torch.equal(h_T[1:2], h1)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_split_sequence_equals_whole(dtype):
+    """forward(0:T1) → (h, conv state) → forward(T1:T) equals forward(0:T)."""
+    B, T, R = 2, 500, 136
+    w = _wl(B, T, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    y, h_T, st = rglru.forward(p, x)
+    for T1 in (1, 64, 129, 499):
+        ya, ha, sa = rglru.forward(p, x[:, :T1].contiguous())
+        yb, hb, sb = rglru.forward(p, x[:, T1:].contiguous(), ha, sa)
+        tol = 1e-5 if dtype == torch.float32 else 8e-3
+        assert rel(torch.cat([ya, yb], 1), y) <= tol, T1
+        assert rel(hb, h_T) <= tol
+        assert torch.equal(sb, st)
+
+
+def test_decode_steps_equal_forward():
+    """T decode steps from a zero state equal one prefill of length T."""
+    B, T, R = 8, 40, 264
+    w = _wl(B, T, R, torch.bfloat16)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    y, h_T, st = rglru.forward(p, x)
+    ring = torch.zeros(B, 3, R, dtype=torch.bfloat16, device=DEV)
+    h = torch.zeros(B, R, device=DEV)
+    ys = []
+    for t in range(T):
+        ys.append(rglru.step(p, x[:, t].contiguous(), ring, h, t).clone())
+    assert rglru.workspace_status(None) == 0
+    assert rel(torch.stack(ys, 1), y) <= 1e-2
+    assert rel(h, h_T) <= 1e-2
+    # after T = 40 ≡ 1 (mod 3) steps the ring's oldest slot is T mod 3
+    order = [(T + j) % 3 for j in range(3)]
+    assert torch.equal(ring[:, order], st)
+
+
+def test_decode_checkpoint_resume_is_bitwise():
+    """The decode state is (h, conv ring, step): saving it and continuing from copies in
+    fresh buffers gives bit-identical outputs."""
+    B, R, n1, n2 = 16, 264, 5, 7
+    w = inputs.make_decode(B, R, torch.bfloat16, seed=4)
+    p = rglru.Params.from_host(w.params)
+    toks = [inputs.decode_token(k, B, R).to(DEV) for k in range(n1 + n2)]
+    ring = torch.zeros(B, 3, R, dtype=torch.bfloat16, device=DEV)
+    h = torch.zeros(B, R, device=DEV)
+    for k in range(n1):
+        rglru.step(p, toks[k], ring, h, k)
+    saved = (h.cpu().clone(), ring.cpu().clone())
+    ref = [rglru.step(p, toks[k], ring, h, k).clone() for k in range(n1, n1 + n2)]
+    h2, ring2 = saved[0].to(DEV), saved[1].to(DEV)
+    got = [rglru.step(p, toks[k], ring2, h2, k).clone() for k in range(n1, n1 + n2)]
+    assert all(torch.equal(a, b) for a, b in zip(ref, got))
+    assert torch.equal(h, h2) and torch.equal(ring, ring2)
+
+
+def test_decode_small_matches_oracle_every_step():
+    B, R, steps = 130, 200, 9
+    w = inputs.make_decode(B, R, torch.bfloat16, seed=2)
+    p = rglru.Params.from_host(w.params)
+    hp = host_params64(w.params)
+    ring = torch.zeros(B, 3, R, dtype=torch.bfloat16, device=DEV)
+    h = torch.zeros(B, R, device=DEV)
+    ring_o, h_o = np.zeros((B, 3, R)), np.zeros((B, R))
+    for k in range(steps):
+        xt = inputs.decode_token(k, B, R)
+        y = rglru.step(p, xt.to(DEV), ring, h, k)
+        y_o, h_o, ring_o = oracle.rglru_step(xt, ring_o, k, h_o, **hp)
+        assert rel(y, y_o) <= TOL[torch.bfloat16], k
+        assert rel(h, h_o) <= TOL[torch.bfloat16], k
+        assert np.array_equal(f64(ring), ring_o)
+
+
+def test_block_small_matches_oracle():
+    B, T, D, R = 2, 150, 136, 264
+    w = inputs.make_block(B, T, D, R, torch.bfloat16, seed=6)
+    p = rglru.Params.from_host(w.params)
+    out = torch.full((B, T, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    out, h_T = rglru.block_forward(p, w.W_1.to(DEV), w.W_2.to(DEV), w.W_o.to(DEV), w.x.to(DEV), out=out)
+    assert rglru.workspace_status(None) == 0
+    ref, h_ref = oracle.recurrent_block(w.x, w.W_1, w.W_2, w.W_o, **host_params64(w.params))
+    assert rel(out, ref) <= TOL[torch.bfloat16]
+    assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
+
+
+# ------------------------------------------------------------------------------------
+# failure detection without a GPU fault: a chunk that never publishes its carry makes
+# its successor's bounded wait run out; the status word reports it and the context
+# stays usable.
+def test_lookback_timeout_is_reported_and_recovered():
+    lib = _abi.load()
+    B, T, R = 1, 64 * 3, 128
+    w = _wl(B, T, R, torch.bfloat16)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    ws = torch.empty(rglru.forward_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=DEV)
+    try:
+        lib.rglru_debug_scan_stall(1)        # (b=0, block 0, chunk 1) stays silent
+        rglru.forward(p, x, workspace=ws)
+        assert rglru.workspace_status(ws) == _abi.STATUS_CODE["RGLRU_ERR_TIMEOUT"]
+    finally:
+        lib.rglru_debug_scan_stall(-1)
+    y, h_T, _ = rglru.forward(p, x, workspace=ws)
+    assert rglru.workspace_status(ws) == 0
+    y_ref, h_ref, _ = oracle.rglru_forward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a, w.params.b_a,
+                                           w.params.W_x, w.params.b_x, w.params.Lambda)
+    assert rel(y, y_ref) <= TOL[torch.bfloat16]
