@@ -25,7 +25,6 @@ all 2048 channels); rank 0 only.
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import os
@@ -112,33 +111,25 @@ class ClockSampler:
 # ------------------------------------------------------------------------------ own arm
 def run_own(args):
     import torch
-    import torch.distributed as dist
 
-    from gated_linear_rnn_conv1d_b200 import inputs, rglru
+    from gated_linear_rnn_conv1d_b200 import inputs, replicas, rglru
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rk = replicas.from_env()
+    world, rank, local = rk.world, rk.rank, rk.local
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    replicas.init(rk, "nccl", device=dev)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(rk)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(rk, v, device=dev)
 
     B, T, R = WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["R"]
-    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=rank)
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=replicas.seed_for(rk))
     p = rglru.Params.from_host(w.params, dev)
     x = w.x.to(dev)
     y = torch.empty_like(x)
@@ -252,9 +243,7 @@ def run_own(args):
     # ---- decode steps/s ---------------------------------------------------------------
     dec = run_decode(torch, rglru, inputs, dev, stream, flush, pk, barrier, max_over_ranks, world)
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.shutdown(rk)
     if rank != 0:
         return
     cpu = cpu_baseline(inputs) if world == 1 else None

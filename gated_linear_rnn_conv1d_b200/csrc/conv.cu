@@ -8,8 +8,10 @@
 // once (plus a 3-row halo per run) and u written once, both coalesced 16-byte accesses.
 //
 // Decode: one thread per 8 channels of one row; reads x_t and the 3-slot ring, writes u_t
-// and overwrites the oldest ring slot with x_t. It also writes c·log σ(Λ) per channel,
-// which the decode GEMM epilogue reads.
+// twice — rounded to bf16 as the gate GEMM's operand, and in float32 for the RG-LRU
+// update in the GEMM epilogue (the same split as the prefill path, where the scan
+// recomputes u in float32) — and overwrites the oldest ring slot with x_t. It also writes
+// c·log σ(Λ) per channel, which the decode GEMM epilogue reads.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
                                                                   const __nv_bfloat16* __restrict__ x_t,
                                                                   __nv_bfloat16* __restrict__ ring, int s0,
                                                                   __nv_bfloat16* __restrict__ u_t,
+                                                                  float* __restrict__ u_f32,
                                                                   float* __restrict__ cla, unsigned* status, int B,
                                                                   int R) {
   constexpr int V = 8;
@@ -143,6 +146,9 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
     o[v] = acc;
   }
   *reinterpret_cast<uint4*>(u_t + (int64_t)b * R + c0) = CV<__nv_bfloat16>::pack(o);
+  float4* uf = reinterpret_cast<float4*>(u_f32 + (int64_t)b * R + c0);
+  uf[0] = make_float4(o[0], o[1], o[2], o[3]);
+  uf[1] = make_float4(o[4], o[5], o[6], o[7]);
   *reinterpret_cast<uint4*>(rb + (int64_t)s0 * R) = raw_c;
   if (b == 0) {
 #pragma unroll
@@ -170,14 +176,14 @@ cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* 
 }
 
 cudaError_t launch_decode_conv(const float* conv_w, const float* conv_b, const float* Lambda, const void* x_t,
-                               void* ring, int64_t step, void* u_t, float* cla, unsigned* status, int B, int R,
-                               cudaStream_t s) {
+                               void* ring, int64_t step, void* u_t, float* u_f32, float* cla, unsigned* status,
+                               int B, int R, cudaStream_t s) {
   dim3 grid((R / 8 + kConvThreads - 1) / kConvThreads, B);
   const int s0 = (int)(step % 3);
   decode_conv_kernel<<<grid, kConvThreads, 0, s>>>(conv_w, conv_b, Lambda,
                                                    static_cast<const __nv_bfloat16*>(x_t),
                                                    static_cast<__nv_bfloat16*>(ring), s0,
-                                                   static_cast<__nv_bfloat16*>(u_t), cla, status, B, R);
+                                                   static_cast<__nv_bfloat16*>(u_t), u_f32, cla, status, B, R);
   return cudaGetLastError();
 }
 

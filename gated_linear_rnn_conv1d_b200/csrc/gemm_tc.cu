@@ -43,7 +43,7 @@ struct EpiArgs {
   const float* b_a;   // GATES / STEP
   const float* b_x;
   int R;              // channels (GATES / STEP)
-  const __nv_bfloat16* u;  // STEP: u_t [M][R]
+  const float* u;          // STEP: u_t [M][R] float32 (the GEMM read its bf16 rounding)
   float* h;                // STEP: state [M][R], in place
   __nv_bfloat16* y;        // STEP: y_t [M][R]
   const float* cla;        // STEP: c·log σ(Λ) [R]
@@ -251,11 +251,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int q = 0; q < 4; ++q) {
               const int c = ch0 + 8 * q;
               if (c < ep.R) {
-                const uint4 w = *reinterpret_cast<const uint4*>(ep.u + row * ep.R + c);
+                const float4* up = reinterpret_cast<const float4*>(ep.u + row * ep.R + c);
+                const float4 u0 = up[0], u1 = up[1];
                 float4* hp = reinterpret_cast<float4*>(ep.h + row * ep.R + c);
                 const float4 h0 = hp[0], h1 = hp[1];
-                float uu[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                               bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+                float uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
                 float hh[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -395,9 +395,9 @@ cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, 
   return launch_tc<BN, EPI_STORE, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
 }
 
-cudaError_t launch_gemm_step_bf16(const void* u_t, const void* Wa, const float* ba, const void* Wx,
-                                  const float* bx, const float* cla, float* h, void* y_t, int B, int R,
-                                  unsigned* status, cudaStream_t s) {
+cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,
+                                  const void* Wx, const float* bx, const float* cla, float* h, void* y_t, int B,
+                                  int R, unsigned* status, cudaStream_t s) {
   constexpr int BN = 128;
   CUtensorMap ma, mb0, mb1;
   if (!make_map_2d(&ma, u_t, R, B, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
@@ -407,7 +407,7 @@ cudaError_t launch_gemm_step_bf16(const void* u_t, const void* Wa, const float* 
   ep.b_a = ba;
   ep.b_x = bx;
   ep.R = R;
-  ep.u = static_cast<const __nv_bfloat16*>(u_t);
+  ep.u = u_f32;
   ep.h = h;
   ep.y = static_cast<__nv_bfloat16*>(y_t);
   ep.cla = cla;

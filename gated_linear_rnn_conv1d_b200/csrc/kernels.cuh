@@ -55,8 +55,8 @@ cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* 
                           void* stateT, int B, int T, int R, bool bf16, cudaStream_t s);
 // Also zeroes *status (the step's status word) before the step's GEMM may set it.
 cudaError_t launch_decode_conv(const float* conv_w, const float* conv_b, const float* Lambda, const void* x_t,
-                               void* ring, int64_t step, void* u_t, float* cla, unsigned* status, int B, int R,
-                               cudaStream_t s);
+                               void* ring, int64_t step, void* u_t, float* u_f32, float* cla, unsigned* status,
+                               int B, int R, cudaStream_t s);
 
 // ---- GEMMs -------------------------------------------------------------------------
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -70,9 +70,9 @@ cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* b
                                    void* z, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
                              unsigned* status, cudaStream_t s);
-cudaError_t launch_gemm_step_bf16(const void* u_t, const void* Wa, const float* ba, const void* Wx,
-                                  const float* bx, const float* cla, float* h, void* y_t, int B, int R,
-                                  unsigned* status, cudaStream_t s);
+cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,
+                                  const void* Wx, const float* bx, const float* cla, float* h, void* y_t, int B,
+                                  int R, unsigned* status, cudaStream_t s);
 // Library-global device status word of the current device (for entry points that take
 // no workspace); null if the symbol address cannot be obtained.
 unsigned* global_status_word();

@@ -95,13 +95,14 @@ BlockLayout block_layout(int B, int T, int R) {
 }
 
 struct StepLayout {
-  size_t off_cla, off_u, bytes;
+  size_t off_cla, off_u, off_uf, bytes;
 };
 StepLayout step_layout(int B, int R) {
   StepLayout L;
   L.off_cla = 256;
   L.off_u = L.off_cla + round256((size_t)R * 4);
-  L.bytes = L.off_u + round256((size_t)B * R * 2);
+  L.off_uf = L.off_u + round256((size_t)B * R * 2);
+  L.bytes = L.off_uf + round256((size_t)B * R * 4);
   return L;
 }
 
@@ -300,11 +301,13 @@ int rglru_step(const rglru_params* params, const void* x_t, void* conv_state, fl
   cudaStream_t s = (cudaStream_t)stream;
   float* cla = reinterpret_cast<float*>(bytes(workspace) + L.off_cla);
   void* u_t = bytes(workspace) + L.off_u;
+  float* u_f32 = reinterpret_cast<float*>(bytes(workspace) + L.off_uf);
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
-  cudaError_t e = launch_decode_conv(params->conv_w, params->conv_b, params->Lambda, x_t, conv_state, step, u_t, cla,
-                                     status, B, R, s);
+  cudaError_t e = launch_decode_conv(params->conv_w, params->conv_b, params->Lambda, x_t, conv_state, step, u_t,
+                                     u_f32, cla, status, B, R, s);
   if (e != cudaSuccess) return fail_cuda(e);
-  e = launch_gemm_step_bf16(u_t, params->W_a, params->b_a, params->W_x, params->b_x, cla, h, y_t, B, R, status, s);
+  e = launch_gemm_step_bf16(u_t, u_f32, params->W_a, params->b_a, params->W_x, params->b_x, cla, h, y_t, B, R,
+                            status, s);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 

@@ -112,7 +112,8 @@ RGLRU_API int rglru_forward(const rglru_params* params, const void* x, const flo
  *   step        ≥ 0, the ring position described above
  *   h           [B][R] float32 state, updated IN PLACE (h_{t-1} → h_t)
  *   y_t         [B][R] io_dtype output (= new h)
- *   workspace   at least rglru_step_workspace_bytes(B, R, io_dtype) bytes (holds u_t)
+ *   workspace   at least rglru_step_workspace_bytes(B, R, io_dtype) bytes (holds u_t, in
+ *               bf16 for the gate GEMM and in float32 for the state update)
  * io_dtype must be RGLRU_BF16 (the tensor-core path) for this entry point.
  * --------------------------------------------------------------------------------- */
 RGLRU_API size_t rglru_step_workspace_bytes(int B, int R, int io_dtype);

@@ -155,14 +155,25 @@ def test_zero_recurrence_gate_keeps_state_bitwise(dtype):
     assert torch.equal(y.float(), h0.to(dtype).float()[:, None, :].expand(B, T, R))
 
 
-def test_batch_rows_are_independent_bitwise():
+def test_batch_rows_are_independent():
+    """A row's result does not depend on the other rows. The conv and the GEMM are
+    bitwise reproducible per row; the scan's look-back composes whichever chunk summaries
+    are ready, so its float32 carries may differ in the last bits between launches."""
     B, T, R = 3, 300, 264
     w = _wl(B, T, R, torch.bfloat16)
     p = rglru.Params.from_host(w.params)
     x = w.x.to(DEV)
     y, h_T, _ = rglru.forward(p, x)
     y1, h1, _ = rglru.forward(p, x[1:2].contiguous())
-    assert torch.equal(y[1:2], y1) and torch.equal(h_T[1:2], h1)
+    assert rel(h_T[1:2], h1) <= 1e-5
+    # y is bf16: at most one rounding step apart wherever the carries differ
+    assert rel(y[1:2], y1) <= 8e-3
+    u = rglru.conv1d(p, x)
+    u1 = rglru.conv1d(p, x[1:2].contiguous())
+    assert torch.equal(u[1:2], u1)
+    z = rglru.gate_proj(p, u.view(B * T, R))
+    z1 = rglru.gate_proj(p, u1.view(T, R))
+    assert torch.equal(z[T:2 * T], z1)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
