@@ -166,6 +166,30 @@ RGLRU_API int rglru_scan(const rglru_params* params, const void* x, const void* 
                const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R, int io_dtype,
                void* workspace, size_t workspace_bytes, rglru_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * rglru_scan without a workspace, for callers that cannot allocate device memory: a
+ * custom operator whose host framework hands it only its input and output buffers, a
+ * serving process whose memory is fully reserved at start-up, or a latency-critical loop
+ * that must not call cudaMalloc (which can synchronise the device). The paper has no
+ * counterpart to this entry point; it exists for those callers only.
+ *
+ * Same arguments and results as rglru_scan, minus the workspace. The scan's scratch
+ * (tile ticket, look-back flags, chunk carries) is a fixed 8 MiB array in the library's
+ * device memory, which every GPU that loads librglru.so holds until the process exits.
+ * Problems needing more (about B·⌈R/128⌉·⌈T/64⌉ > 5400 for bf16, twice that tile count
+ * of 64 channels for float32) are rejected with RGLRU_ERR_WORKSPACE before anything is
+ * launched. Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * All calls on a device share the one array, and it keeps the last call's contents (each
+ * call clears the parts that must start at zero): calls that overlap on the GPU — on
+ * different streams, or from different threads — race and give wrong results. Timeouts of
+ * its bounded waits are reported by rglru_workspace_status(NULL, stream).
+ * --------------------------------------------------------------------------------- */
+RGLRU_API int rglru_scan_noalloc(const rglru_params* params, const void* x, const void* z, const void* conv_state0,
+                                 const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R,
+                                 int io_dtype, rglru_stream_t stream);
+
 /* Dense bf16 GEMM C[M][N] = A[M][K] · B[N][K]ᵀ on the tcgen05 tensor cores (fp32
  * accumulate, bf16 store), the kernel behind the block's linears. K % 8 == 0, N % 8 == 0. */
 RGLRU_API int rglru_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, rglru_stream_t stream);
