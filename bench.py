@@ -44,7 +44,11 @@ FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
 # summarised under profiles/, keyed by the SHA-256 of the kernel's source at capture
 # time. A source change invalidates the figure (reported as null).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/gemm_tc_gates_fwd_hawk_bf16.md
+    "gate_gemm": {"src_sha256": "dfa49050241d1920e769d43dd0c9da256209d9cc555aee56412a6d06798e716d",
+                  "bytes_per_launch": 83942144 + 85779456},
+}
 
 
 def _sha(path):
@@ -209,6 +213,14 @@ def run_own(args):
     roof["traffic"] = traffic
     roof["kernel"] = dom
     roof["peak_source"] = pk["source"] + " (MEASURED_PEAKS.json burst figure)" if pk["source"] == "measured" else "fallback"
+
+    if args.only == "forward":
+        replicas.shutdown(rk)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+                              "warmup": args.warmup, "ms_per_step": step_ms, "kernels": kern, "roofline": roof,
+                              "gpu_launches": 3 * K, "clocks": clk, "only": "forward"}))
+        return
 
     # ---- end to end through the public API, host buffers -----------------------------
     x_host = w.x.pin_memory()
@@ -389,6 +401,8 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
+    ap.add_argument("--only", choices=["all", "forward"], default="all",
+                    help="forward: time the forward steps only (small command for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -3,15 +3,16 @@
 // RG-LRU). u_t[c] = conv_b[c] + Σ_k conv_w[k][c] · x_{t-3+k}[c], zero history unless a
 // conv state is given.
 //
-// Prefill: each thread owns 16 bytes of channels of one batch row and walks a run of
-// kConvRun time steps with the three previous inputs held in registers, so x is read
-// once (plus a 3-row halo per run) and u written once, both coalesced 16-byte accesses.
+// Prefill: tiles of one batch row × 128 (bf16) or 64 (f32) channels × 64 steps; x arrives
+// in shared memory by one TMA copy including the 3-row halo, and each thread writes 4
+// steps of 16 bytes of channels of u with coalesced stores.
 //
 // Decode: one thread per 8 channels of one row; reads x_t and the 3-slot ring, writes u_t
 // twice — rounded to bf16 as the gate GEMM's operand, and in float32 for the RG-LRU
 // update in the GEMM epilogue (the same split as the prefill path, where the scan
 // recomputes u in float32) — and overwrites the oldest ring slot with x_t. It also writes
 // c·log σ(Λ) per channel, which the decode GEMM epilogue reads.
+#include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -23,7 +24,6 @@ namespace rglru {
 namespace {
 
 constexpr int kConvThreads = 128;
-constexpr int kConvRun = 32;
 
 template <typename T> struct CV;
 template <> struct CV<__nv_bfloat16> {
@@ -47,70 +47,144 @@ template <> struct CV<float> {
   }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kConvThreads) conv1d_fwd_kernel(const float* __restrict__ conv_w,
-                                                                 const float* __restrict__ conv_b,
-                                                                 const T* __restrict__ x, const T* __restrict__ state0,
-                                                                 T* __restrict__ u, T* __restrict__ stateT, int B,
-                                                                 int T_, int R) {
-  constexpr int V = CV<T>::N;
-  const int grp = blockIdx.x * kConvThreads + threadIdx.x;
-  const int c0 = grp * V;
-  if (c0 >= R) return;
-  const int b = blockIdx.z;
-  const int t0 = blockIdx.y * kConvRun;
-  const int t1 = min(t0 + kConvRun, T_);
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  return make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+}
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float4& v) {
+  __stcg(reinterpret_cast<uint2*>(p), make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w)));
+}
+__device__ __forceinline__ void store4(float* p, const float4& v) { __stcg(reinterpret_cast<float4*>(p), v); }
 
+// Prefill: persistent CTAs stream tiles of one batch row × CW channels (16 bytes per
+// thread × 16 threads) × 64 steps through a ring of kConvStages shared-memory stages. One
+// thread keeps kConvStages TMA copies in flight (each brings the tile's 67 x rows, the
+// 3-row halo included; rows before t = 0 and channels past R arrive as zeros); the 256
+// threads each produce 4 steps × V channels of u per tile.
+constexpr int kTileThreads = 256;
+constexpr int kTileSteps = 64;
+constexpr int kTileRows = kTileSteps + 3;
+constexpr int kConvStages = 4;
+
+__device__ __forceinline__ void tma_load_x3(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Each CTA keeps one channel block (cblk = blockIdx.x mod n_cblk) for its whole life, so
+// its taps and bias are loaded once; it walks that block's (batch row, time chunk) tiles.
+template <typename T>
+__global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const __grid_constant__ CUtensorMap mx,
+                                                                  const float* __restrict__ conv_w,
+                                                                  const float* __restrict__ conv_b,
+                                                                  const T* __restrict__ state0, T* __restrict__ u,
+                                                                  T* __restrict__ stateT, int B, int T_, int R,
+                                                                  int n_cblk, int n_chunks, unsigned* status) {
+  constexpr int V = CV<T>::N;
+  constexpr int CW = 16 * V;
+  constexpr int kStage = kTileRows * CW * (int)sizeof(T);
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* sbase = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ __align__(8) uint64_t full[kConvStages];
+
+  const int tid = threadIdx.x;
+  const int g = tid % 16, s = tid / 16;
+  const int cblk = blockIdx.x % n_cblk;
+  const int lane0 = blockIdx.x / n_cblk;         // first (b, chunk) pair of this CTA
+  const int stride = gridDim.x / n_cblk;         // CTAs sharing this channel block
+  const int n_pairs = B * n_chunks;
+  auto issue = [&](int k, int pair) {
+    const int b = pair / n_chunks, chunk = pair % n_chunks;
+    mbar_arrive_expect_tx(&full[k], kStage);
+    tma_load_x3(sbase + k * kStage, &mx, &full[k], cblk * CW, chunk * kTileSteps - 3, b);
+  };
+  if (tid == 0) {
+    for (int k = 0; k < kConvStages; ++k) mbar_init(&full[k], 1);
+    fence_barrier_init();
+    for (int k = 0; k < kConvStages; ++k) {
+      const int pair = lane0 + k * stride;
+      if (pair < n_pairs) issue(k, pair);
+    }
+  }
+  const int c0 = cblk * CW + g * V;
+  const bool cvalid = c0 < R;
   float w[4][V], cb[V];
 #pragma unroll
-  for (int v = 0; v < V; ++v) {
+  for (int v = 0; v < V; v += 4) {
+    const int c = cvalid ? c0 + v : 0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) w[k][v] = __ldg(conv_w + k * R + c0 + v);
-    cb[v] = __ldg(conv_b + c0 + v);
+    for (int kk = 0; kk < 4; ++kk) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(conv_w + kk * R + c));
+      w[kk][v] = f.x; w[kk][v + 1] = f.y; w[kk][v + 2] = f.z; w[kk][v + 3] = f.w;
+    }
+    const float4 f = __ldg(reinterpret_cast<const float4*>(conv_b + c));
+    cb[v] = f.x; cb[v + 1] = f.y; cb[v + 2] = f.z; cb[v + 3] = f.w;
   }
-  float hist[3][V];
+  __syncthreads();
+  volatile int no_abort = 0;
+  int it = 0;
+  for (int pair = lane0; pair < n_pairs; pair += stride, ++it) {
+    const int k = it % kConvStages;
+    const uint32_t parity = (uint32_t)((it / kConvStages) & 1);
+    T* sx = reinterpret_cast<T*>(sbase + k * kStage);
+    const int b = pair / n_chunks, chunk = pair % n_chunks;
+    const int t0 = chunk * kTileSteps;
+    if (!mbar_wait(&full[k], parity, &no_abort) && tid == 0) atomicOr(status, kStatusTimeout);
+    if (chunk == 0 && state0 != nullptr) {
+      __syncthreads();
+      if (tid < 48) {
+        // conv history before t = 0 comes from the given state instead of zeros
+        const int j = tid / 16, gg = tid % 16, cc = cblk * CW + gg * V;
+        if (cc < R)
+          *reinterpret_cast<uint4*>(sx + j * CW + gg * V) =
+              __ldg(reinterpret_cast<const uint4*>(state0 + ((int64_t)b * 3 + j) * R + cc));
+      }
+      __syncthreads();
+    }
+    if (cvalid) {
+      float hist[3][V];
 #pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    const int t = t0 - 3 + j;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (t >= 0) raw = __ldg(reinterpret_cast<const uint4*>(x + ((int64_t)b * T_ + t) * R + c0));
-    else if (state0 != nullptr)
-      raw = __ldg(reinterpret_cast<const uint4*>(state0 + ((int64_t)b * 3 + (t + 3)) * R + c0));
-    CV<T>::unpack(raw, hist[j]);
-  }
-  const T* xp = x + ((int64_t)b * T_) * R + c0;
-  T* up = u + ((int64_t)b * T_) * R + c0;
-  constexpr int U = 8;
-  for (int t = t0; t < t1; t += U) {
-    uint4 raw[U];
+      for (int j = 0; j < 3; ++j) CV<T>::unpack(*reinterpret_cast<const uint4*>(sx + (s * 4 + j) * CW + g * V), hist[j]);
 #pragma unroll
-    for (int k = 0; k < U; ++k)
-      if (t + k < t1) raw[k] = __ldcs(reinterpret_cast<const uint4*>(xp + (int64_t)(t + k) * R));
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      if (t + k < t1) {
+      for (int l = 0; l < 4; ++l) {
+        const int t = t0 + s * 4 + l;
         float xc[V], o[V];
-        CV<T>::unpack(raw[k], xc);
+        CV<T>::unpack(*reinterpret_cast<const uint4*>(sx + (s * 4 + l + 3) * CW + g * V), xc);
+#pragma unroll
+        for (int v = 0; v < V; v += 2) {
+          float2 a2 = __ffma2_rn(make_float2(w[0][v], w[0][v + 1]), make_float2(hist[0][v], hist[0][v + 1]),
+                                 make_float2(cb[v], cb[v + 1]));
+          a2 = __ffma2_rn(make_float2(w[1][v], w[1][v + 1]), make_float2(hist[1][v], hist[1][v + 1]), a2);
+          a2 = __ffma2_rn(make_float2(w[2][v], w[2][v + 1]), make_float2(hist[2][v], hist[2][v + 1]), a2);
+          a2 = __ffma2_rn(make_float2(w[3][v], w[3][v + 1]), make_float2(xc[v], xc[v + 1]), a2);
+          o[v] = a2.x;
+          o[v + 1] = a2.y;
+        }
 #pragma unroll
         for (int v = 0; v < V; ++v) {
-          float acc = cb[v];
-          acc = fmaf(w[0][v], hist[0][v], acc);
-          acc = fmaf(w[1][v], hist[1][v], acc);
-          acc = fmaf(w[2][v], hist[2][v], acc);
-          acc = fmaf(w[3][v], xc[v], acc);
-          o[v] = acc;
           hist[0][v] = hist[1][v];
           hist[1][v] = hist[2][v];
           hist[2][v] = xc[v];
         }
-        *reinterpret_cast<uint4*>(up + (int64_t)(t + k) * R) = CV<T>::pack(o);
+        if (t < T_) __stcg(reinterpret_cast<uint4*>(u + ((int64_t)b * T_ + t) * R + c0), CV<T>::pack(o));
       }
     }
-  }
-  if (stateT != nullptr && t1 == T_) {
-#pragma unroll
-    for (int j = 0; j < 3; ++j)
-      *reinterpret_cast<uint4*>(stateT + ((int64_t)b * 3 + j) * R + c0) = CV<T>::pack(hist[j]);
+    if (stateT != nullptr && chunk == n_chunks - 1 && tid < 48) {
+      // the last three inputs x_{T-3}, x_{T-2}, x_{T-1} sit at tile rows T − t0 … T − t0 + 2
+      const int j = tid / 16, gg = tid % 16, cc = cblk * CW + gg * V;
+      if (cc < R)
+        *reinterpret_cast<uint4*>(stateT + ((int64_t)b * 3 + j) * R + cc) =
+            *reinterpret_cast<const uint4*>(sx + (T_ - t0 + j) * CW + gg * V);
+    }
+    __syncthreads();  // stage k fully read
+    if (tid == 0) {
+      const int np = pair + kConvStages * stride;
+      if (np < n_pairs) issue(k, np);
+    }
   }
 }
 
@@ -159,19 +233,50 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
 }  // namespace
 
 cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* state0, void* u,
-                          void* stateT, int B, int T, int R, bool bf16, cudaStream_t s) {
-  const int V = bf16 ? 8 : 4;
-  const int groups = R / V;
-  dim3 grid((groups + kConvThreads - 1) / kConvThreads, (T + kConvRun - 1) / kConvRun, B);
+                          void* stateT, int B, int T, int R, bool bf16, unsigned* status, cudaStream_t s) {
+  const int es = bf16 ? 2 : 4;
+  const int cw = bf16 ? 128 : 64;
+  const int n_cblk = (R + cw - 1) / cw;
+  const int n_chunks = (T + kTileSteps - 1) / kTileSteps;
+  const int64_t tiles = (int64_t)B * n_cblk * n_chunks;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  EncodeTiledFn fn = get_encode_tiled();
+  if (fn == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap mx;
+  cuuint64_t dims[3] = {(cuuint64_t)R, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)R * es, (cuuint64_t)T * R * es};
+  cuuint32_t box[3] = {(cuuint32_t)cw, (cuuint32_t)kTileRows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (fn(&mx, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(x), dims,
+         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int smem = kConvStages * kTileRows * cw * es + 128;
+  static bool attr[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr[bf16][dev]) {
+    e = bf16 ? cudaFuncSetAttribute(conv1d_tile_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+             : cudaFuncSetAttribute(conv1d_tile_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr[bf16][dev] = true;
+  }
+  // a multiple of n_cblk CTAs, about two per SM; each keeps one channel block
+  const int64_t pairs = (int64_t)B * n_chunks;
+  int64_t per_blk = std::max<int64_t>(1, (int64_t)2 * num_sms() / n_cblk);
+  per_blk = std::min<int64_t>(per_blk, pairs);
+  const int64_t grid = per_blk * n_cblk;
+  if (grid > INT32_MAX) return cudaErrorInvalidValue;
   if (bf16)
-    conv1d_fwd_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, s>>>(
-        conv_w, conv_b, static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(state0),
-        static_cast<__nv_bfloat16*>(u), static_cast<__nv_bfloat16*>(stateT), B, T, R);
+    conv1d_tile_kernel<__nv_bfloat16><<<(unsigned)grid, kTileThreads, smem, s>>>(
+        mx, conv_w, conv_b, static_cast<const __nv_bfloat16*>(state0), static_cast<__nv_bfloat16*>(u),
+        static_cast<__nv_bfloat16*>(stateT), B, T, R, n_cblk, n_chunks, status);
   else
-    conv1d_fwd_kernel<float><<<grid, kConvThreads, 0, s>>>(conv_w, conv_b, static_cast<const float*>(x),
-                                                           static_cast<const float*>(state0),
-                                                           static_cast<float*>(u), static_cast<float*>(stateT), B,
-                                                           T, R);
+    conv1d_tile_kernel<float><<<(unsigned)grid, kTileThreads, smem, s>>>(
+        mx, conv_w, conv_b, static_cast<const float*>(state0), static_cast<float*>(u), static_cast<float*>(stateT), B,
+        T, R, n_cblk, n_chunks, status);
   return cudaGetLastError();
 }
 

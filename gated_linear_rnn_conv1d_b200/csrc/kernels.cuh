@@ -22,9 +22,18 @@ inline int scan_cw(bool bf16) { return kScanGroups * scan_vec(bf16); }
 struct ScanLayout {
   int n_cblk, n_chunks;
   int64_t n_tiles;
-  size_t off_flags, off_carry, bytes;
+  // workspace: [status u32 | ticket u32 | pad to 256 B][aggregates: n_tiles × CW × u64]
+  //            [inclusive states: n_tiles × CW × u32]; all of it must be zero at launch
+  size_t off_agg, off_incl, bytes, zero_bytes;
 };
 ScanLayout scan_layout(int B, int T, int R, bool bf16);
+
+// TMA tensor maps the scan reads its tiles through.
+struct ScanMaps {
+  CUtensorMap x;  // [B][T][R], box {CW, 67, 1}
+  CUtensorMap z;  // [B·T][pitch], box {CW, 64}
+  CUtensorMap g;  // [B][T][R], box {CW, 64, 1} (gate branch; unused otherwise)
+};
 
 struct ScanArgs {
   const void* x;        // [B][T][R]
@@ -38,10 +47,10 @@ struct ScanArgs {
   const float* conv_b;  // [R]
   const float* Lambda;  // [R]
   unsigned* status;     // device status word
-  unsigned* ticket;     // tile ticket counter (zeroed before launch)
-  unsigned* flags;      // [n_tiles] look-back flags (zeroed before launch)
-  float* carry;         // [n_tiles][3][CW]
-  int B, T, R, n_cblk, n_chunks;
+  unsigned* ticket;     // tile ticket counter (zero at launch)
+  uint64_t* carry_agg;  // [n_tiles][CW] published aggregates (zero at launch)
+  uint32_t* carry_incl; // [n_tiles][CW] published inclusive states (zero at launch)
+  int B, T, R, n_cblk, n_chunks, n_tiles;
   int64_t pitch;
   int64_t stall_tile;   // testing only: this tile never publishes its carry (-1: none)
 };
@@ -52,7 +61,7 @@ cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s);
 
 // ---- conv --------------------------------------------------------------------------
 cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* state0, void* u,
-                          void* stateT, int B, int T, int R, bool bf16, cudaStream_t s);
+                          void* stateT, int B, int T, int R, bool bf16, unsigned* status, cudaStream_t s);
 // Also zeroes *status (the step's status word) before the step's GEMM may set it.
 cudaError_t launch_decode_conv(const float* conv_w, const float* conv_b, const float* Lambda, const void* x_t,
                                void* ring, int64_t step, void* u_t, float* u_f32, float* cla, unsigned* status,

@@ -114,7 +114,7 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
                      const float* h0, const void* g, void* y, float* hT, int B, int T, int R, bool bf16,
                      const ScanLayout& sl, void* ws, bool zero_first, cudaStream_t s) {
   if (zero_first) {
-    cudaError_t e = cudaMemsetAsync(ws, 0, sl.off_carry, s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, sl.zero_bytes, s);
     if (e != cudaSuccess) return e;
   }
   ScanArgs a{};
@@ -130,13 +130,14 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
   a.Lambda = p->Lambda;
   a.status = reinterpret_cast<unsigned*>(ws);
   a.ticket = reinterpret_cast<unsigned*>(bytes(ws) + 4);
-  a.flags = reinterpret_cast<unsigned*>(bytes(ws) + sl.off_flags);
-  a.carry = reinterpret_cast<float*>(bytes(ws) + sl.off_carry);
+  a.carry_agg = reinterpret_cast<uint64_t*>(bytes(ws) + sl.off_agg);
+  a.carry_incl = reinterpret_cast<uint32_t*>(bytes(ws) + sl.off_incl);
   a.B = B;
   a.T = T;
   a.R = R;
   a.n_cblk = sl.n_cblk;
   a.n_chunks = sl.n_chunks;
+  a.n_tiles = (int)sl.n_tiles;
   a.pitch = pitch;
   return launch_scan(a, bf16, s);
 }
@@ -200,8 +201,10 @@ int rglru_conv1d(const float* conv_w, const float* conv_b, const void* x, const 
     return RGLRU_ERR_ALIGN;
   int st = check_device();
   if (st != RGLRU_OK) return st;
+  unsigned* status = global_status_word();
+  if (status == nullptr) return fail_cuda(cudaGetLastError());
   cudaError_t e = launch_conv1d(conv_w, conv_b, x, conv_state0, u, conv_state_T, B, T, R, io_dtype == RGLRU_BF16,
-                                (cudaStream_t)stream);
+                                status, (cudaStream_t)stream);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
@@ -270,9 +273,9 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
   // status word, ticket and flags are zeroed before the first kernel, so that a status bit
   // set by the GEMM survives until the caller reads it.
-  cudaError_t e = cudaMemsetAsync(workspace, 0, L.scan.off_carry, s);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, L.scan.zero_bytes, s);
   if (e != cudaSuccess) return fail_cuda(e);
-  e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, s);
+  e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, status, s);
   if (e != cudaSuccess) return fail_cuda(e);
   if (bf16)
     e = launch_gemm_gates_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, z, (int64_t)B * T, R, status, s);
@@ -349,22 +352,24 @@ int rglru_block_forward(const rglru_params* params, const void* W_1, const void*
   cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
   if (e == cudaSuccess) e = launch_gemm_bf16(x, W_1, v, ntok, R, D, R, status, s);        // v = x W_1ᵀ
   if (e == cudaSuccess) e = launch_gemm_bf16(x, W_2, g, ntok, R, D, R, status, s);        // g = x W_2ᵀ
-  if (e == cudaSuccess) e = launch_conv1d(params->conv_w, params->conv_b, v, nullptr, u, nullptr, B, T, R, true, s);
+  if (e == cudaSuccess)
+    e = launch_conv1d(params->conv_w, params->conv_b, v, nullptr, u, nullptr, B, T, R, true, status, s);
   if (e == cudaSuccess)
     e = launch_gemm_gates_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, z, ntok, R, status, s);
   if (e == cudaSuccess) {
     // the scan's memset must not clear a status bit the GEMMs above may have set:
     // zero only the ticket and flags here.
-    e = cudaMemsetAsync(bytes(workspace) + 4, 0, L.scan.off_carry - 4, s);
+    e = cudaMemsetAsync(bytes(workspace) + 4, 0, L.scan.zero_bytes - 4, s);
     if (e == cudaSuccess) {
       ScanArgs a{};
       a.x = v; a.z = z; a.state0 = nullptr; a.h0 = h0; a.g = g; a.y = pbuf; a.hT = h_T;
       a.conv_w = params->conv_w; a.conv_b = params->conv_b; a.Lambda = params->Lambda;
       a.status = status;
       a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
-      a.flags = reinterpret_cast<unsigned*>(bytes(workspace) + L.scan.off_flags);
-      a.carry = reinterpret_cast<float*>(bytes(workspace) + L.scan.off_carry);
-      a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks; a.pitch = gate_pitch(R);
+      a.carry_agg = reinterpret_cast<uint64_t*>(bytes(workspace) + L.scan.off_agg);
+      a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);
+      a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks;
+      a.n_tiles = (int)L.scan.n_tiles; a.pitch = gate_pitch(R);
       e = launch_scan(a, true, s);
     }
   }

@@ -26,8 +26,9 @@ using namespace rglru;
 
 namespace {
 
-// 8 MiB per device: enough for B·⌈R/128⌉·⌈T/64⌉ ≈ 5400 bf16 tiles (e.g. B=8, T=2048,
-// R=2048 needs 4096) or ≈ 10800 float32 tiles of 64 channels.
+// 8 MiB per device: enough for B·⌈R/128⌉·⌈T/64⌉ ≈ 5400 bf16 tiles of 128 channels
+// (12 bytes of carries per channel; e.g. B=8, T=2048, R=2048 needs 4096 tiles) or
+// ≈ 10900 float32 tiles of 64 channels.
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -86,8 +87,8 @@ extern "C" RGLRU_API int rglru_scan_noalloc(const rglru_params* p, const void* x
   if (status == nullptr) return RGLRU_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
   // The array keeps whatever the previous call left in it: the ticket counter and the
-  // look-back flags must start at zero, the carries are always written before being read.
-  e = cudaMemsetAsync(scratch, 0, sl.off_carry, s);
+  // published carries must start at zero, so the used part is cleared first.
+  e = cudaMemsetAsync(scratch, 0, sl.zero_bytes, s);
   if (e != cudaSuccess) return RGLRU_ERR_CUDA;
   ScanArgs a{};
   a.x = x;
@@ -102,13 +103,14 @@ extern "C" RGLRU_API int rglru_scan_noalloc(const rglru_params* p, const void* x
   a.Lambda = p->Lambda;
   a.status = status;
   a.ticket = reinterpret_cast<unsigned*>(static_cast<unsigned char*>(scratch) + 4);
-  a.flags = reinterpret_cast<unsigned*>(static_cast<unsigned char*>(scratch) + sl.off_flags);
-  a.carry = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + sl.off_carry);
+  a.carry_agg = reinterpret_cast<uint64_t*>(static_cast<unsigned char*>(scratch) + sl.off_agg);
+  a.carry_incl = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(scratch) + sl.off_incl);
   a.B = B;
   a.T = T;
   a.R = R;
   a.n_cblk = sl.n_cblk;
   a.n_chunks = sl.n_chunks;
+  a.n_tiles = (int)sl.n_tiles;
   a.pitch = gate_pitch(R);
   e = launch_scan(a, bf16, s);
   if (e != cudaSuccess) return RGLRU_ERR_CUDA;
