@@ -292,6 +292,281 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
+// 2-SM form (cta_group::2): a cluster of two CTAs computes a 256×256 tile. Each CTA stages
+// its own 128 rows of A and its own half of the B tile (128 rows); the leader CTA (rank 0)
+// issues tcgen05.mma.cta_group::2 with M = 256, N = 256, which reads both CTAs' shared
+// memory and leaves rows 0–127 of the tile in the leader's TMEM and rows 128–255 in the
+// peer's. Per SM this halves the B bytes pulled from L2 per FLOP. Loads carry no
+// multicast: both CTAs' TMA copies signal the leader's full barrier; the leader's commits
+// are multicast (tcgen05.commit, not a load) to both CTAs' empty / accumulator barriers.
+constexpr int k2Stages = 6;
+constexpr int k2ABytes = BM * BK * 2;            // 16 KB: this CTA's 128 rows of A
+constexpr int k2BBytes = 128 * BK * 2;           // 16 KB: this CTA's half of the B tile
+constexpr int k2StageBytes = k2ABytes + k2BBytes;
+constexpr int k2Smem = k2Stages * k2StageBytes + 1024;
+constexpr int k2TmemCols = 512;                  // two 256-column accumulators
+constexpr uint32_t k2Idesc = umma_idesc_bf16_f32(256, 256);
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_2sm(void* dst, const CUtensorMap* m, uint32_t leader_bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(leader_bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void umma_f16_2sm(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_2sm_both(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "h"(mask)
+               : "memory");
+}
+
+template <int EPI, bool DUAL>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                 const __grid_constant__ CUtensorMap tmB1, int64_t M, int K, int n_tiles_n, int num_tiles, EpiArgs ep,
+                 unsigned* status) {
+  constexpr int S = k2Stages;
+  constexpr int BN = 256;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x / 2;
+  const int n_clusters = gridDim.x / 2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 8);  // 4 epilogue warps in each of the two CTAs
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (DUAL) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
+                 "r"(k2TmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const int k_blocks = (K + BK - 1) / BK;
+  const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), 0);
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
+        const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+        const int arow = m_pair * 256 + (int)rank * 128;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_s)) { ok = false; break; }
+          uint8_t* sa = smem + stage * k2StageBytes;
+          uint8_t* sb = sa + k2ABytes;
+          const uint32_t lbar = leader_full0 + stage * 8;
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * k2StageBytes);
+          tma_load_2d_2sm(sa, &tmA, lbar, kb * BK, arow);
+          if (DUAL) {
+            tma_load_2d_2sm(sb, rank == 0 ? &tmB0 : &tmB1, lbar, kb * BK, n_blk * 128);
+          } else {
+            tma_load_2d_2sm(sb, &tmB0, lbar, kb * BK, n_blk * 256 + (int)rank * 128);
+          }
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) { abort_s = 1; atomicOr(status, kStatusTimeout); }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader CTA only) ----------------
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, &abort_s)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_s)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * k2StageBytes);
+          const uint32_t b_addr = a_addr + k2ABytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_f16_2sm(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), k2Idesc,
+                         (kb | k) != 0 ? 1u : 0u);
+          umma_commit_2sm_both(&empty_bar[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_2sm_both(&tfull_bar[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      if (!ok) { abort_s = 1; atomicOr(status, kStatusTimeout); }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(&drain_bar))
+                   : "memory");
+      volatile int never = 0;
+      (void)mbar_wait(&drain_bar, 0, &never);
+    }
+  } else {
+    // ---------------- epilogue warps (both CTAs) ----------------
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t leader_tempty0 = mapa_rank(smem_u32(&tempty_bar[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < num_tiles; tile += n_clusters) {
+      const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_s)) {
+        abort_s = 1;
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const int64_t row = (int64_t)m_pair * 256 + rank * 128 + row_in_tile;
+      const bool row_ok = row < M;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + cc * 32, r);
+        tmem_ld_wait();
+        float v[32];
+        const int col0 = cc * 32;
+        if constexpr (EPI == EPI_GATES) {
+          const int half = col0 / 128;
+          const int ch0 = n_blk * 128 + (col0 % 128);
+          const float* bias = half ? ep.b_x : ep.b_a;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int ch = ch0 + j;
+            v[j] = __uint_as_float(r[j]) + (ch < ep.R ? __ldg(bias + ch) : 0.0f);
+          }
+          if (row_ok) store_row_bf16(ep.C + row * ep.ldc + (int64_t)n_blk * BN + col0, v);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          const int gcol = n_blk * BN + col0;
+          if (row_ok) {
+            if (gcol + 32 <= ep.N) {
+              store_row_bf16(ep.C + row * ep.ldc + gcol, v);
+            } else {
+              uint4* d = reinterpret_cast<uint4*>(ep.C + row * ep.ldc + gcol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (gcol + 8 * q < ep.N)
+                  d[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                    pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(leader_tempty0 + acc * 8);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's shared memory stays valid until the leader's MMAs are done
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(k2TmemCols)
+                 : "memory");
+  }
+}
+
+template <int EPI, bool DUAL>
+cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, int64_t M, int K,
+                       int n_tiles_n, const EpiArgs& ep, unsigned* status, cudaStream_t s) {
+  auto kern = gemm2_kernel<EPI, DUAL>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int64_t m_pairs = (M + 255) / 256;
+  const int64_t tiles = m_pairs * n_tiles_n;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  const int clusters = (int)std::min<int64_t>(tiles, num_sms() / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = k2Smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, M, K, n_tiles_n, (int)tiles, ep, status);
+}
+
+// ---------------------------------------------------------------------------------------
 EncodeTiledFn g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -366,33 +641,34 @@ unsigned* global_status_word() {
 
 cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
                                    void* z, int64_t M, int R, unsigned* status, cudaStream_t s) {
-  constexpr int BN = 256;
+  // 2-SM tiles: 256 tokens × 256 packed columns (128 channels × two gates); the leader
+  // CTA stages 128 rows of W_a, its peer the same 128 rows of W_x.
   CUtensorMap ma, mb0, mb1;
   if (!make_map_2d(&ma, u, R, M, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
-  if (!make_map_2d(&mb0, Wa, R, R, (uint64_t)R * 2, BK, BN / 2)) return cudaErrorInvalidValue;
-  if (!make_map_2d(&mb1, Wx, R, R, (uint64_t)R * 2, BK, BN / 2)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb0, Wa, R, R, (uint64_t)R * 2, BK, 128)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb1, Wx, R, R, (uint64_t)R * 2, BK, 128)) return cudaErrorInvalidValue;
   EpiArgs ep{};
   ep.C = static_cast<__nv_bfloat16*>(z);
   ep.ldc = gate_pitch(R);
   ep.b_a = ba;
   ep.b_x = bx;
   ep.R = R;
-  const int n_tiles_n = (R + BN / 2 - 1) / (BN / 2);
-  return launch_tc<BN, EPI_GATES, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
+  const int n_tiles_n = (R + 127) / 128;
+  return launch_tc2<EPI_GATES, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
 }
 
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
                              unsigned* status, cudaStream_t s) {
-  constexpr int BN = 256;
+  // 2-SM tiles 256 × 256: each CTA of the pair stages 128 rows of A and 128 rows of B.
   CUtensorMap ma, mb;
   if (!make_map_2d(&ma, A, K, M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
-  if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, BN)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, 128)) return cudaErrorInvalidValue;
   EpiArgs ep{};
   ep.C = static_cast<__nv_bfloat16*>(C);
   ep.ldc = ldc;
   ep.N = N;
-  const int n_tiles_n = (N + BN - 1) / BN;
-  return launch_tc<BN, EPI_STORE, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+  const int n_tiles_n = (N + 255) / 256;
+  return launch_tc2<EPI_STORE, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
 }
 
 cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,

@@ -277,6 +277,8 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     // ---- phase 1 ---------------------------------------------------------------------
     // Channels are taken four at a time, so that only four channels' parameters and
     // conv history are live at once.
+    // Per-step replay values stay in registers: the shared-memory stage is refilled with the
+    // next tile as soon as phase 1 is done.
     uint32_t rp[kAcc ? 1 : L * V];                    // bf16 path: (1 − a_t, b_t) pairs
     float ra[kAcc ? L * V : 1], rb[kAcc ? L * V : 1];  // f32 path: a_t, b_t
     float Ag[V], Bg[V];
@@ -374,12 +376,17 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     if (tid < CW) {
       const int j = tid;
       const int c = tc.cblk * CW + j;
+      // exclusive prefixes (held in registers) map the tile's incoming state to the state
+      // entering sub-chunk q
+      float pA[S], pB[S];
+#pragma unroll
+      for (int q = 0; q < S; ++q) { pA[q] = sA[q * CW + j]; pB[q] = sB[q * CW + j]; }
       float A = 1.0f, Bv = 0.0f;
 #pragma unroll
       for (int q = 0; q < S; ++q) {
-        const float pa = sA[q * CW + j], pb = sB[q * CW + j];
-        sA[q * CW + j] = A;  // exclusive prefix: maps the tile's incoming state to the
-        sB[q * CW + j] = Bv; // state entering sub-chunk q
+        const float pa = pA[q], pb = pB[q];
+        pA[q] = A;
+        pB[q] = Bv;
         Bv = fmaf(pa, Bv, pb);
         A *= pa;
       }
@@ -423,7 +430,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       if (publish) st_relaxed_u32(incl + tc.tix * CW + j, enc(hout));
       if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < R) a.hT[(int64_t)tc.b * R + c] = hout;
 #pragma unroll
-      for (int q = 0; q < S; ++q) sB[q * CW + j] = fmaf(sA[q * CW + j], hin, sB[q * CW + j]);
+      for (int q = 0; q < S; ++q) sB[q * CW + j] = fmaf(pA[q], hin, pB[q]);
     }
     __syncthreads();
 
