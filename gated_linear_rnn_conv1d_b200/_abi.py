@@ -45,6 +45,8 @@ SIGNATURES = {
     "rglru_scan": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "rglru_scan_noalloc": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "rglru_gemm_bf16": (_I, [_P, _P, _P, _L, _I, _I, _P]),
+    "rglru_gate_scan_workspace_bytes": (_S, [_I, _I, _I, _I]),
+    "rglru_gate_scan": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "rglru_workspace_status": (_I, [_P, _P]),
     "rglru_strerror": (ctypes.c_char_p, [_I]),
     "rglru_last_cuda_error": (_I, []),

@@ -34,7 +34,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int kGemmThreads = 192;
 
-enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2 };
+enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2, EPI_SCAN = 3 };
 
 struct EpiArgs {
   __nv_bfloat16* C;   // STORE / GATES output
@@ -47,6 +47,17 @@ struct EpiArgs {
   float* h;                // STEP: state [M][R], in place
   __nv_bfloat16* y;        // STEP: y_t [M][R]
   const float* cla;        // STEP: c·log σ(Λ) [R]
+  // SCAN (gate GEMM fused with the RG-LRU scan):
+  const __nv_bfloat16* x;       // [B][T][R] Conv1D input (u is recomputed from it in float32)
+  const __nv_bfloat16* state0;  // [B][3][R] conv history or null
+  const float* conv_w;          // [4][R]
+  const float* conv_b;          // [R]
+  const float* Lambda;          // [R]
+  const float* h0;              // [B][R] or null
+  float* hT;                    // [B][R] or null
+  uint64_t* carry_agg;          // [B·n_nb·n_chunks][128] aggregates (zero at launch)
+  uint32_t* carry_incl;         // [B·n_nb·n_chunks][128] inclusive states (zero at launch)
+  int T, n_chunks;              // n_chunks = T / 128
 };
 
 template <int BN> struct GemmCfg {
@@ -303,7 +314,6 @@ constexpr int k2Stages = 6;
 constexpr int k2ABytes = BM * BK * 2;            // 16 KB: this CTA's 128 rows of A
 constexpr int k2BBytes = 128 * BK * 2;           // 16 KB: this CTA's half of the B tile
 constexpr int k2StageBytes = k2ABytes + k2BBytes;
-constexpr int k2Smem = k2Stages * k2StageBytes + 1024;
 constexpr int k2TmemCols = 512;                  // two 256-column accumulators
 constexpr uint32_t k2Idesc = umma_idesc_bf16_f32(256, 256);
 
@@ -347,12 +357,73 @@ __device__ __forceinline__ void umma_commit_2sm_both(uint64_t* bar) {
                : "memory");
 }
 
+// Fused-scan epilogue scratch after the pipeline stages: per epilogue warp a 32×33 float2
+// transpose buffer, then aggregates [4][32][2], incoming states [32], parameters [6][128].
+constexpr int kScanStages = 5;
+constexpr int kTbufBytes = 4 * 32 * 33 * 8;
+constexpr int kScanEpiBytes = kTbufBytes + 4 * 32 * 2 * 4 + 32 * 4 + 6 * 128 * 4;
+template <int EPI> __host__ __device__ constexpr int stages_of() { return EPI == EPI_SCAN ? kScanStages : k2Stages; }
+template <int EPI> __host__ __device__ constexpr int smem_of() {
+  return stages_of<EPI>() * k2StageBytes + (EPI == EPI_SCAN ? kScanEpiBytes : 0) + 1024;
+}
+
+// Gate math for two elements: d = 1 − a_t and b_t = √(1−a_t²)·i·u, with r = σ(z_a),
+// log a_t = r·cla, d = −expm1(log a_t) (Taylor polynomial to degree 6 on [−1/8, 0], 1 − ex2
+// beyond), 1 − a_t² = d(2 − d), √(1−a_t²)·i = q·rsqrt(q (1 + e^{−z_x})² + 1e-30).
+__device__ __forceinline__ void gate_fast2_pair(float2 za, float2 zx, float2 cla, float2 u, float2& d, float2& bt) {
+  const float2 na = __fmul2_rn(za, make_float2(-kLog2e, -kLog2e));
+  const float2 nx = __fmul2_rn(zx, make_float2(-kLog2e, -kLog2e));
+  const float2 ea = __fadd2_rn(make_float2(ex2_approx(na.x), ex2_approx(na.y)), make_float2(1.0f, 1.0f));
+  const float2 r = make_float2(rcp_approx(ea.x), rcp_approx(ea.y));
+  const float2 la = __fmul2_rn(r, cla);
+  if (fminf(la.x, la.y) >= -0.125f) {
+    float2 p = __ffma2_rn(la, make_float2(1.0f / 720.0f, 1.0f / 720.0f), make_float2(1.0f / 120.0f, 1.0f / 120.0f));
+    p = __ffma2_rn(p, la, make_float2(1.0f / 24.0f, 1.0f / 24.0f));
+    p = __ffma2_rn(p, la, make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+    p = __ffma2_rn(p, la, make_float2(0.5f, 0.5f));
+    p = __ffma2_rn(p, la, make_float2(1.0f, 1.0f));
+    d = __fmul2_rn(make_float2(-la.x, -la.y), p);
+  } else {
+    d.x = la.x >= -0.125f ? neg_expm1_small(la.x) : 1.0f - ex2_approx(la.x * kLog2e);
+    d.y = la.y >= -0.125f ? neg_expm1_small(la.y) : 1.0f - ex2_approx(la.y * kLog2e);
+  }
+  const float2 q = __fmul2_rn(d, __fadd2_rn(make_float2(2.0f, 2.0f), make_float2(-d.x, -d.y)));
+  const float2 t1 = __fadd2_rn(make_float2(ex2_approx(nx.x), ex2_approx(nx.y)), make_float2(1.0f, 1.0f));
+  const float2 dd = __ffma2_rn(__fmul2_rn(q, t1), t1, make_float2(1e-30f, 1e-30f));
+  const float2 rs = make_float2(rsqrt_approx(dd.x), rsqrt_approx(dd.y));
+  bt = __fmul2_rn(__fmul2_rn(q, rs), u);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed_u32g(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64g(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u32g(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u64g(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// Published carries are stored as their bit pattern XOR 0x7FFFFFFF: exact and reversible,
+// and zero only for one NaN pattern, so zeroed memory reads as "not published yet".
+__device__ __forceinline__ uint32_t enc_carry(float v) { return __float_as_uint(v) ^ 0x7FFFFFFFu; }
+__device__ __forceinline__ float dec_carry(uint32_t w) { return __uint_as_float(w ^ 0x7FFFFFFFu); }
+
 template <int EPI, bool DUAL>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                  const __grid_constant__ CUtensorMap tmB1, int64_t M, int K, int n_tiles_n, int num_tiles, EpiArgs ep,
                  unsigned* status) {
-  constexpr int S = k2Stages;
+  constexpr int S = stages_of<EPI>();
   constexpr int BN = 256;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[S];
@@ -463,7 +534,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       volatile int never = 0;
       (void)mbar_wait(&drain_bar, 0, &never);
     }
-  } else {
+  } else if constexpr (EPI != EPI_SCAN) {
     // ---------------- epilogue warps (both CTAs) ----------------
     const int quarter = warp & 3;
     const int row_in_tile = quarter * 32 + lane;
@@ -521,6 +592,180 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive_remote(leader_tempty0 + acc * 8);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+  } else {
+    // ---------------- fused RG-LRU scan epilogue (both CTAs) ----------------
+    // "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元 (RG-LRU),
+    // Eq. (1)–(4). The CTA's 128 rows are 128 consecutive steps of one batch row (T is a
+    // multiple of 128); its 256 accumulator columns are z_a and z_x of 128 channels. For
+    // each 32-channel block, a warp moves its 32 rows through a shared-memory transpose so
+    // that lane j owns channel j and walks the 32 steps in order: u recomputed in float32
+    // from x, gates, log-space decay, fold into an affine map; the four warps' maps are
+    // composed, the 128-step chunk's incoming state comes from decoupled look-back over
+    // earlier chunks (carries in global memory, bounded waits), and each lane replays its
+    // steps into y.
+    const int q = warp & 3;                 // TMEM lane quarter = rows 32q … 32q+31
+    const int et = q * 32 + lane;           // 0..127 among the epilogue threads
+    uint8_t* escr = smem + S * k2StageBytes;
+    float2* tbuf = reinterpret_cast<float2*>(escr) + q * (32 * 33);
+    float* sAgg = reinterpret_cast<float*>(escr + kTbufBytes);       // [4 warps][32][2]
+    float* sHin = sAgg + 4 * 32 * 2;                                   // [32]
+    float* sPar = sHin + 32;                                           // [6][128]
+    const uint32_t leader_tempty0 = mapa_rank(smem_u32(&tempty_bar[0]), 0);
+    const int R = ep.R;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < num_tiles; tile += n_clusters) {
+      const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_s)) {
+        abort_s = 1;
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int64_t m0 = (int64_t)m_pair * 256 + rank * 128;
+      if (m0 < M) {
+        const int b = (int)(m0 / ep.T);
+        const int t0 = (int)(m0 - (int64_t)b * ep.T);
+        const int chunk = t0 / 128;
+        {
+          const int ch = n_blk * 128 + et;
+          const bool ok = ch < R;
+          sPar[0 * 128 + et] = ok ? __ldg(ep.conv_w + ch) : 0.0f;
+          sPar[1 * 128 + et] = ok ? __ldg(ep.conv_w + R + ch) : 0.0f;
+          sPar[2 * 128 + et] = ok ? __ldg(ep.conv_w + 2 * R + ch) : 0.0f;
+          sPar[3 * 128 + et] = ok ? __ldg(ep.conv_w + 3 * R + ch) : 0.0f;
+          sPar[4 * 128 + et] = ok ? __ldg(ep.conv_b + ch) : 0.0f;
+          sPar[5 * 128 + et] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
+        }
+        named_bar_sync(1, 128);
+        const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          // row phase: this lane's step, 32 channels of z_a and of z_x
+          {
+            uint32_t ra[32], rx[32];
+            tmem_ld_32x32b_x32(t_row + cc * 32, ra);
+            tmem_ld_32x32b_x32(t_row + 128 + cc * 32, rx);
+            tmem_ld_wait();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              tbuf[lane * 33 + jj] = make_float2(__uint_as_float(ra[jj]), __uint_as_float(rx[jj]));
+          }
+          __syncwarp();
+          // column phase: lane = channel, 32 steps in order
+          const int cl = cc * 32 + lane;
+          const int ch = n_blk * 128 + cl;
+          const bool cvalid = ch < R;
+          const int chs = cvalid ? ch : 0;
+          const float w0 = sPar[cl], w1 = sPar[128 + cl], w2 = sPar[256 + cl], w3 = sPar[384 + cl];
+          const float cb = sPar[512 + cl], cla = sPar[640 + cl];
+          const float ba = __ldg(ep.b_a + chs), bx = __ldg(ep.b_x + chs);
+          const int tq = t0 + q * 32;  // first step of this warp's rows
+          const __nv_bfloat16* xb = ep.x + (int64_t)b * ep.T * R + chs;
+          float xm3, xm2, xm1;
+          {
+            float hv[3];
+#pragma unroll
+            for (int k = 0; k < 3; ++k) {
+              const int t = tq - 3 + k;
+              float v = 0.0f;
+              if (t >= 0) v = __bfloat162float(xb[(int64_t)t * R]);
+              else if (ep.state0 != nullptr) v = __bfloat162float(ep.state0[((int64_t)b * 3 + (t + 3)) * R + chs]);
+              hv[k] = v;
+            }
+            xm3 = hv[0]; xm2 = hv[1]; xm1 = hv[2];
+          }
+          uint32_t rp[32];
+          float A = 1.0f, Bv = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float x0 = __bfloat162float(xb[(int64_t)(tq + i) * R]);
+            const float x1 = __bfloat162float(xb[(int64_t)(tq + i + 1) * R]);
+            float2 u;
+            u.x = fmaf(w3, x0, fmaf(w2, xm1, fmaf(w1, xm2, fmaf(w0, xm3, cb))));
+            u.y = fmaf(w3, x1, fmaf(w2, x0, fmaf(w1, xm1, fmaf(w0, xm2, cb))));
+            xm3 = xm1;
+            xm2 = x0;
+            xm1 = x1;
+            const float2 z0 = tbuf[i * 33 + lane], z1 = tbuf[(i + 1) * 33 + lane];
+            float2 d, bt;
+            gate_fast2_pair(make_float2(z0.x + ba, z1.x + ba), make_float2(z0.y + bx, z1.y + bx),
+                            make_float2(cla, cla), u, d, bt);
+            const float a0 = 1.0f - d.x, a1 = 1.0f - d.y;
+            Bv = fmaf(a0, Bv, bt.x);
+            A *= a0;
+            Bv = fmaf(a1, Bv, bt.y);
+            A *= a1;
+            rp[i] = pack_bf16x2(d.x, bt.x);
+            rp[i + 1] = pack_bf16x2(d.y, bt.y);
+          }
+          __syncwarp();  // tbuf free for the next block
+          sAgg[(q * 32 + lane) * 2 + 0] = A;
+          sAgg[(q * 32 + lane) * 2 + 1] = Bv;
+          named_bar_sync(1, 128);
+          // map from the chunk's incoming state to the state entering this warp's rows
+          float eA = 1.0f, eB = 0.0f;
+          for (int w = 0; w < q; ++w) {
+            const float wa = sAgg[(w * 32 + lane) * 2], wb = sAgg[(w * 32 + lane) * 2 + 1];
+            eB = fmaf(wa, eB, wb);
+            eA *= wa;
+          }
+          if (q == 0) {
+            float At = 1.0f, Bt = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float wa = sAgg[(w * 32 + lane) * 2], wb = sAgg[(w * 32 + lane) * 2 + 1];
+              Bt = fmaf(wa, Bt, wb);
+              At *= wa;
+            }
+            const int64_t slot = (((int64_t)b * n_tiles_n + n_blk) * ep.n_chunks + chunk) * 128 + cl;
+            float hin;
+            if (chunk == 0) {
+              hin = (ep.h0 != nullptr && cvalid) ? ep.h0[(int64_t)b * R + ch] : 0.0f;
+            } else {
+              st_relaxed_u64g(ep.carry_agg + slot, ((uint64_t)__float_as_uint(Bt) << 32) | enc_carry(At));
+              float fA = 1.0f, fB = 0.0f;
+              int64_t p = slot - 128;
+              long long tw = 0;
+              while (true) {
+                const uint32_t hw = ld_relaxed_u32g(ep.carry_incl + p);
+                const uint64_t aw = ld_relaxed_u64g(ep.carry_agg + p);
+                if (hw != 0u) { hin = fmaf(fA, dec_carry(hw), fB); break; }
+                if ((uint32_t)aw != 0u) {
+                  fB = fmaf(fA, __uint_as_float((uint32_t)(aw >> 32)), fB);
+                  fA *= dec_carry((uint32_t)aw);
+                  p -= 128;
+                  continue;
+                }
+                if (tw == 0) {
+                  tw = clock64();
+                } else if (clock64() - tw > kWaitCycles) {
+                  atomicOr(status, kStatusTimeout);
+                  hin = fB;
+                  break;
+                }
+              }
+            }
+            const float hout = fmaf(At, hin, Bt);
+            st_relaxed_u32g(ep.carry_incl + slot, enc_carry(hout));
+            if (chunk == ep.n_chunks - 1 && ep.hT != nullptr && cvalid) ep.hT[(int64_t)b * R + ch] = hout;
+            sHin[lane] = hin;
+          }
+          named_bar_sync(1, 128);
+          float h = fmaf(eA, sHin[lane], eB);
+          __nv_bfloat16* yb = ep.y + ((int64_t)b * ep.T + tq) * R + chs;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            h = fmaf(1.0f - bf16lo(rp[i]), h, bf16hi(rp[i]));
+            if (cvalid) yb[(int64_t)i * R] = __float2bfloat16_rn(h);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(leader_tempty0 + acc * 8);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
   }
 
   tc_fence_before();
@@ -543,7 +788,7 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, k2Smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_of<EPI>());
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -554,7 +799,7 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = k2Smem;
+  cfg.dynamicSmemBytes = smem_of<EPI>();
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -625,6 +870,33 @@ int num_sms() {
   cudaGetDevice(&dev);
   if (n[dev] == 0) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
   return n[dev];
+}
+
+cudaError_t launch_gate_scan_bf16(const ScanFusedArgs& f, cudaStream_t s) {
+  // 2-SM gate GEMM with the RG-LRU scan in its epilogue; needs T % 128 == 0.
+  const int64_t M = (int64_t)f.B * f.T;
+  CUtensorMap ma, mb0, mb1;
+  if (!make_map_2d(&ma, f.u, f.R, M, (uint64_t)f.R * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb0, f.W_a, f.R, f.R, (uint64_t)f.R * 2, BK, 128)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb1, f.W_x, f.R, f.R, (uint64_t)f.R * 2, BK, 128)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.b_a = f.b_a;
+  ep.b_x = f.b_x;
+  ep.R = f.R;
+  ep.y = static_cast<__nv_bfloat16*>(f.y);
+  ep.x = static_cast<const __nv_bfloat16*>(f.x);
+  ep.state0 = static_cast<const __nv_bfloat16*>(f.state0);
+  ep.conv_w = f.conv_w;
+  ep.conv_b = f.conv_b;
+  ep.Lambda = f.Lambda;
+  ep.h0 = f.h0;
+  ep.hT = f.hT;
+  ep.carry_agg = f.carry_agg;
+  ep.carry_incl = f.carry_incl;
+  ep.T = f.T;
+  ep.n_chunks = f.T / 128;
+  const int n_tiles_n = (f.R + 127) / 128;
+  return launch_tc2<EPI_SCAN, true>(ma, mb0, mb1, M, f.R, n_tiles_n, ep, f.status, s);
 }
 
 unsigned* global_status_word() {

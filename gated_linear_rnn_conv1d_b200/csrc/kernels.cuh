@@ -82,6 +82,30 @@ cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, 
 cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,
                                   const void* Wx, const float* bx, const float* cla, float* h, void* y_t, int B,
                                   int R, unsigned* status, cudaStream_t s);
+// Gate GEMM (2-SM tcgen05) with the RG-LRU scan fused into its epilogue (bf16 IO,
+// T % 128 == 0): y and h_T straight from x and u, without writing the gate
+// pre-activations. carry_* need n_chunk_tiles × 128 slots (zero at launch).
+struct ScanFusedArgs {
+  const void* u;        // [B·T][R] bf16 conv output (GEMM operand)
+  const void* x;        // [B][T][R] bf16 conv input (u recomputed in float32)
+  const void* state0;   // [B][3][R] or null
+  const void* W_a;
+  const void* W_x;
+  const float* b_a;
+  const float* b_x;
+  const float* conv_w;
+  const float* conv_b;
+  const float* Lambda;
+  const float* h0;      // or null
+  void* y;              // [B][T][R] bf16
+  float* hT;            // or null
+  uint64_t* carry_agg;  // [B · ceil(R/128) · T/128][128]
+  uint32_t* carry_incl; // [B · ceil(R/128) · T/128][128]
+  unsigned* status;
+  int B, T, R;
+};
+cudaError_t launch_gate_scan_bf16(const ScanFusedArgs& f, cudaStream_t s);
+
 // Library-global device status word of the current device (for entry points that take
 // no workspace); null if the symbol address cannot be obtained.
 unsigned* global_status_word();

@@ -76,6 +76,49 @@ FwdLayout fwd_layout(int B, int T, int R, int io) {
   return L;
 }
 
+// Forward through the fused gate-GEMM + scan kernel (bf16 IO, T % 128 == 0):
+// [status, ticket | chunk aggregates | chunk inclusive states][u]. Carries are zeroed per call.
+struct FusedLayout {
+  int64_t n_chunk_tiles;
+  size_t off_agg, off_incl, zero_bytes, off_u, bytes;
+};
+FusedLayout fused_layout(int B, int T, int R) {
+  FusedLayout L;
+  L.n_chunk_tiles = (int64_t)B * ((R + 127) / 128) * (T / 128);
+  L.off_agg = 256;
+  L.off_incl = L.off_agg + round256((size_t)L.n_chunk_tiles * 128 * 8);
+  L.zero_bytes = L.off_incl + round256((size_t)L.n_chunk_tiles * 128 * 4);
+  L.off_u = L.zero_bytes;
+  L.bytes = L.off_u + round256((size_t)B * T * R * 2);
+  return L;
+}
+bool fused_ok(int io, int T) { return io == RGLRU_BF16 && T % 128 == 0; }
+
+ScanFusedArgs fused_args(const rglru_params* p, const void* x, const void* u, const void* state0, const float* h0,
+                         void* y, float* hT, int B, int T, int R, const FusedLayout& L, void* ws) {
+  ScanFusedArgs f{};
+  f.u = u;
+  f.x = x;
+  f.state0 = state0;
+  f.W_a = p->W_a;
+  f.W_x = p->W_x;
+  f.b_a = p->b_a;
+  f.b_x = p->b_x;
+  f.conv_w = p->conv_w;
+  f.conv_b = p->conv_b;
+  f.Lambda = p->Lambda;
+  f.h0 = h0;
+  f.y = y;
+  f.hT = hT;
+  f.carry_agg = reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + L.off_agg);
+  f.carry_incl = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.off_incl);
+  f.status = reinterpret_cast<unsigned*>(ws);
+  f.B = B;
+  f.T = T;
+  f.R = R;
+  return f;
+}
+
 struct BlockLayout {
   ScanLayout scan;
   size_t off_v, off_g, off_u, off_z, off_p, bytes;
@@ -178,7 +221,34 @@ size_t rglru_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
 
 size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype) {
   if (!valid_dtype(io_dtype) || !valid_R(R) || !valid_tokens(B, T)) return 0;
-  return fwd_layout(B, T, R, io_dtype).bytes;
+  return fused_ok(io_dtype, T) ? fused_layout(B, T, R).bytes : fwd_layout(B, T, R, io_dtype).bytes;
+}
+
+size_t rglru_gate_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
+  if (!valid_R(R) || !valid_tokens(B, T) || !fused_ok(io_dtype, T)) return 0;
+  return fused_layout(B, T, R).zero_bytes;
+}
+
+int rglru_gate_scan(const rglru_params* params, const void* x, const void* u, const void* conv_state0,
+                    const float* h0, void* y, float* h_T, int B, int T, int R, int io_dtype, void* workspace,
+                    size_t workspace_bytes, rglru_stream_t stream) {
+  if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_tokens(B, T) || T % 128 != 0) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x == nullptr || u == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(x) || !aligned16(u) || !aligned16(y) || !aligned16(conv_state0) || !aligned16(h0) ||
+      !aligned16(h_T))
+    return RGLRU_ERR_ALIGN;
+  const FusedLayout L = fused_layout(B, T, R);
+  if (workspace == nullptr || workspace_bytes < L.zero_bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, L.zero_bytes, s);
+  if (e == cudaSuccess)
+    e = launch_gate_scan_bf16(fused_args(params, x, u, conv_state0, h0, y, h_T, B, T, R, L, workspace), s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
 size_t rglru_step_workspace_bytes(int B, int R, int io_dtype) {
@@ -262,6 +332,22 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   if (!aligned16(x) || !aligned16(y) || !aligned16(h0) || !aligned16(conv_state0) || !aligned16(h_T) ||
       !aligned16(conv_state_T))
     return RGLRU_ERR_ALIGN;
+  if (fused_ok(io_dtype, T)) {
+    // conv, then the gate GEMM with the scan fused into its epilogue
+    const FusedLayout L = fused_layout(B, T, R);
+    if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+    if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+    if ((st = check_device()) != RGLRU_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    void* u = bytes(workspace) + L.off_u;
+    unsigned* status = reinterpret_cast<unsigned*>(workspace);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, L.zero_bytes, s);
+    if (e == cudaSuccess)
+      e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, true, status, s);
+    if (e == cudaSuccess)
+      e = launch_gate_scan_bf16(fused_args(params, x, u, conv_state0, h0, y, h_T, B, T, R, L, workspace), s);
+    return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+  }
   const FwdLayout L = fwd_layout(B, T, R, io_dtype);
   if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
   if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;

@@ -189,6 +189,28 @@ def scan(params: Params, x: torch.Tensor, z: torch.Tensor, h0: Optional[torch.Te
     return y, h_T
 
 
+def gate_scan_workspace_bytes(B: int, T: int, R: int) -> int:
+    return _abi.load().rglru_gate_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16)
+
+
+def gate_scan(params: Params, x: torch.Tensor, u: torch.Tensor, h0: Optional[torch.Tensor] = None,
+              conv_state0: Optional[torch.Tensor] = None, *, workspace: Optional[torch.Tensor] = None,
+              y: Optional[torch.Tensor] = None, h_T: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """rglru_gate_scan: gate GEMM with the scan fused in its epilogue (bf16, T % 128 == 0)."""
+    lib = _abi.load()
+    B, T, R = x.shape
+    io = _io(x)
+    y = torch.empty_like(x) if y is None else y
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_gate_scan_workspace_bytes(B, T, R, io), x.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_gate_scan", lib.rglru_gate_scan(
+        ctypes.byref(st), _p(x), _p(u), _p(conv_state0), _p(h0), _p(y), _p(h_T), B, T, R, io, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return y, h_T
+
+
 def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, *, C: Optional[torch.Tensor] = None,
               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """rglru_gemm_bf16: C[M][N] = A[M][K] · B[N][K]ᵀ (bf16 in/out, fp32 accumulate)."""
