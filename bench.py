@@ -4,12 +4,12 @@
 
 Own arm. One step = one forward pass of the layer over one batch of the Hawk-scale
 workload B=8, T=2048, D_RNN=2048, bf16 IO with float32 state, inputs resident in HBM, L2
-flushed (256 MB write) before every timed step. The step calls the two stages of
-rglru_forward for this shape one by one through the C ABI — the Conv1D(4) kernel, then the
-gate GEMM with the gates, log-space decay and chunked scan fused into its epilogue — the
-same launches rglru_forward makes, so that each kernel's duration is measured with CUDA
-events on its own stream. The separate gate GEMM and the standalone fused scan kernel are
-timed in a second loop (not part of the step).
+flushed (256 MB write) before every timed step. The step calls the three stages of
+rglru_forward one by one through the C ABI — Conv1D(4), the gate GEMM, the fused gates +
+log-space decay + chunked scan — the same launches rglru_forward makes, so that each
+kernel's duration is measured with CUDA events on its own stream. The alternative second
+stage (gate GEMM with the scan in its epilogue, rglru_gate_scan) is timed in a second loop
+and is not part of the step.
 Reported: tokens/s (all ranks), per-kernel achieved bandwidth / throughput and their
 fractions of the measured B200 peaks, the roofline of the dominant kernel, the same
 metric end to end through the public API with host buffers (pinned H2D of x, D2H of y
@@ -47,8 +47,8 @@ FLUSH_BYTES = 256 << 20
 # summarised under profiles/, keyed by the SHA-256 of the kernel's source at capture
 # time. A source change invalidates the figure (reported as null).
 NCU_TRAFFIC = {
-    # profiles/gemm_tc_gates_fwd_hawk_bf16.md (the standalone gate GEMM)
-    "gate_gemm_standalone": {"src_sha256": "71b04d951a248c53588e9264d9cda6aa0f633f2d7d220f784dec17aa47354089",
+    # profiles/gemm_tc_gates_fwd_hawk_bf16.md
+    "gate_gemm": {"src_sha256": "71b04d951a248c53588e9264d9cda6aa0f633f2d7d220f784dec17aa47354089",
                   "bytes_per_launch": 83971840 + 89110528},
 }
 
@@ -149,34 +149,34 @@ def run_own(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
-        # exactly the launches rglru_forward makes for this shape: conv, then the gate
-        # GEMM with the scan fused into its epilogue
+        # exactly the launches rglru_forward makes: conv, gate GEMM, fused scan
         if ev is not None:
             ev[0].record(stream)
         rglru.conv1d(p, x, u=u)
         if ev is not None:
             ev[1].record(stream)
-        rglru.gate_scan(p, x, u, workspace=ws_gs, y=y, h_T=h_T)
+        rglru.gate_proj(p, u.view(B * T, R), z=z)
         if ev is not None:
             ev[2].record(stream)
-
-    def unfused(ev):
-        # the same layer through the separate gate GEMM and the standalone fused scan
-        ev[0].record(stream)
-        rglru.gate_proj(p, u.view(B * T, R), z=z)
-        ev[1].record(stream)
         rglru.scan(p, x, z, workspace=ws_scan, y=y, h_T=h_T)
-        ev[2].record(stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def fused(ev):
+        # the alternative second stage: gate GEMM with the scan in its epilogue
+        ev[0].record(stream)
+        rglru.gate_scan(p, x, u, workspace=ws_gs, y=y, h_T=h_T)
+        ev[1].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    if rglru.workspace_status(ws_gs) != 0 or rglru.workspace_status(None) != 0:
+    if rglru.workspace_status(ws_scan) != 0 or rglru.workspace_status(None) != 0:
         raise SystemExit("a kernel reported a timeout during warm-up")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
@@ -188,23 +188,23 @@ def run_own(args):
     barrier()
     clk = clocks.stop()
     conv_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
-    gs_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
-    step_ms = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in evs) / K)
-    status = rglru.workspace_status(ws_gs)
+    gemm_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    scan_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+    step_ms = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / K)
+    status = rglru.workspace_status(ws_scan)
 
-    # standalone gate GEMM + scan (not part of the timed forward step)
+    # the fused gate GEMM + scan stage (not part of the timed forward step)
     for _ in range(3):
         flush.zero_()
-        unfused([torch.cuda.Event(enable_timing=True) for _ in range(3)])
-    Ku = max(3, min(K, 50))
-    uev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Ku)]
+        fused([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    Ku = max(3, min(K, 30))
+    uev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(Ku)]
     for k in range(Ku):
         flush.zero_()
-        unfused(uev[k])
+        fused(uev[k])
     torch.cuda.synchronize()
-    gemm_ms = sum(e[0].elapsed_time(e[1]) for e in uev) / Ku
-    scan_ms = sum(e[1].elapsed_time(e[2]) for e in uev) / Ku
-    if rglru.workspace_status(ws_scan) != 0:
+    gs_ms = sum(e[0].elapsed_time(e[1]) for e in uev) / Ku
+    if rglru.workspace_status(ws_gs) != 0:
         status = -7
 
     tokens = B * T
@@ -216,22 +216,24 @@ def run_own(args):
     gemm_flops = 2.0 * tokens * (2 * R) * R
     kern = {
         "conv1d": {"ms": conv_ms, "GB/s": conv_bytes / conv_ms / 1e6, "bytes": conv_bytes},
-        "gate_scan": {"ms": gs_ms, "TFLOP/s": gemm_flops / gs_ms / 1e9, "flops": gemm_flops,
-                      "note": "gate GEMM with the RG-LRU scan fused into its epilogue (the forward's 2nd kernel)"},
-        "gate_gemm_standalone": {"ms": gemm_ms, "TFLOP/s": gemm_flops / gemm_ms / 1e9, "flops": gemm_flops},
-        "scan_standalone": {"ms": scan_ms, "GB/s": scan_bytes / scan_ms / 1e6, "bytes": scan_bytes},
+        "gate_gemm": {"ms": gemm_ms, "TFLOP/s": gemm_flops / gemm_ms / 1e9, "flops": gemm_flops},
+        "scan": {"ms": scan_ms, "GB/s": scan_bytes / scan_ms / 1e6, "bytes": scan_bytes},
+        "gate_scan_fused_alternative": {"ms": gs_ms, "TFLOP/s": gemm_flops / gs_ms / 1e9, "flops": gemm_flops,
+                                        "note": "rglru_gate_scan, timed apart; not part of the step"},
     }
     kern["conv1d"]["frac_hbm"] = kern["conv1d"]["GB/s"] / pk["hbm_gbs"]
-    kern["scan_standalone"]["frac_hbm"] = kern["scan_standalone"]["GB/s"] / pk["hbm_gbs"]
-    kern["gate_scan"]["frac_tensor"] = kern["gate_scan"]["TFLOP/s"] / pk["bf16_tflops"]
-    kern["gate_gemm_standalone"]["frac_tensor"] = kern["gate_gemm_standalone"]["TFLOP/s"] / pk["bf16_tflops"]
-    dom = "gate_scan" if gs_ms >= conv_ms else "conv1d"
+    kern["scan"]["frac_hbm"] = kern["scan"]["GB/s"] / pk["hbm_gbs"]
+    kern["gate_gemm"]["frac_tensor"] = kern["gate_gemm"]["TFLOP/s"] / pk["bf16_tflops"]
+    kern["gate_scan_fused_alternative"]["frac_tensor"] = (kern["gate_scan_fused_alternative"]["TFLOP/s"]
+                                                          / pk["bf16_tflops"])
+    dom = max(("conv1d", "gate_gemm", "scan"), key=lambda k: kern[k]["ms"])
     traffic = None
-    src = os.path.join(ROOT, "gated_linear_rnn_conv1d_b200", "csrc", {"gate_scan": "gemm_tc.cu", "conv1d": "conv.cu"}[dom])
+    src = os.path.join(ROOT, "gated_linear_rnn_conv1d_b200", "csrc",
+                       {"gate_gemm": "gemm_tc.cu", "scan": "scan.cu", "conv1d": "conv.cu"}[dom])
     rec = NCU_TRAFFIC.get(dom)
     if rec and rec["src_sha256"] == _sha(src):
         traffic = rec["bytes_per_launch"]
-    if dom == "gate_scan":
+    if dom == "gate_gemm":
         roof = {"bound": "tensor", "achieved": kern[dom]["TFLOP/s"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": kern[dom]["GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s"}
@@ -246,7 +248,7 @@ def run_own(args):
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
                               "warmup": args.warmup, "ms_per_step": step_ms, "kernels": kern, "roofline": roof,
-                              "gpu_launches": 2 * K, "clocks": clk, "only": "forward"}))
+                              "gpu_launches": 3 * K, "clocks": clk, "only": "forward"}))
         return
 
     # ---- end to end through the public API, host buffers -----------------------------
@@ -296,11 +298,11 @@ def run_own(args):
                    "l2": "flushed before every timed step (256 MB write, outside the step events)"},
         "roofline": roof,
         "kernels": kern,
-        "hbm_gb_per_s": {"scan_standalone": kern["scan_standalone"]["GB/s"], "conv1d": kern["conv1d"]["GB/s"],
+        "hbm_gb_per_s": {"scan": kern["scan"]["GB/s"], "conv1d": kern["conv1d"]["GB/s"],
                          "peak": pk["hbm_gbs"], "peak_source": pk["source"]},
         "decode": dec,
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": 3 * K,
         "clocks": clk,
         "status": "ok" if status == 0 else "timeout reported",
         "cpu_baseline": cpu,

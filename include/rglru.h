@@ -91,12 +91,8 @@ typedef struct {
  *   workspace    device buffer of at least rglru_forward_workspace_bytes(B, T, R, io_dtype)
  *                bytes, 256-byte aligned. It holds u, the gate pre-activations and the
  *                scan's chunk carries; its contents need no initialisation.
- * Kernels: conv (x → u), then
- *   - bf16 IO with T % 128 == 0: the 2-SM tcgen05 gate GEMM with the RG-LRU scan fused
- *     into its epilogue (rglru_gate_scan below; the gate pre-activations never reach
- *     memory);
- *   - otherwise: the gate GEMM (tcgen05 for bf16, FFMA for f32) writing the packed
- *     pre-activations, then the fused gates + log-space decay + chunked scan kernel.
+ * Kernels: conv (x → u), the gate GEMM (2-SM tcgen05 for bf16, FFMA for f32) writing the
+ * packed pre-activations, then the fused gates + log-space decay + chunked scan kernel.
  * --------------------------------------------------------------------------------- */
 RGLRU_API size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype);
 RGLRU_API int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0,
@@ -199,8 +195,10 @@ RGLRU_API int rglru_scan_noalloc(const rglru_params* params, const void* x, cons
  * bf16 (the tensor-core operand). bf16 only; T must be a multiple of 128 (each 128-step
  * chunk of a batch row is one accumulator tile). conv_state0, h0 and h_T as in
  * rglru_forward. workspace: at least rglru_gate_scan_workspace_bytes(B, T, R, io_dtype)
- * bytes, 256-byte aligned (chunk carries; zeroed by the call). This is the second stage
- * of rglru_forward on that path. */
+ * bytes, 256-byte aligned (chunk carries; zeroed by the call). Compared with the separate
+ * gate GEMM + scan it needs no pre-activation buffer (2 instead of 6 bytes of workspace
+ * per token·channel) but on B200 it takes about twice as long: its scan runs in the four
+ * epilogue warps of each SM. */
 RGLRU_API size_t rglru_gate_scan_workspace_bytes(int B, int T, int R, int io_dtype);
 RGLRU_API int rglru_gate_scan(const rglru_params* params, const void* x, const void* u, const void* conv_state0,
                               const float* h0, void* y, float* h_T, int B, int T, int R, int io_dtype,
