@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   constexpr int S = kScanSub;
   constexpr int L = kScanL;
   constexpr bool kAcc = SV<T>::kAccurate;
+  static_assert(2 * CW <= kScanThreads, "phase 2 needs CW look-back threads and CW staging threads");
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -273,6 +274,9 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     if (!mbar_wait(&bar, phase, &no_abort)) {
       if (tid == 0) atomicOr(a.status, kStatusTimeout);
     }
+    // the ticket after `next` is fetched now; its round trip overlaps phase 1
+    unsigned next2 = 0;
+    if (tid == 0) next2 = atomicAdd(a.ticket, 1u);
 
     // ---- phase 1 ---------------------------------------------------------------------
     // Channels are taken four at a time, so that only four channels' parameters and
@@ -368,11 +372,17 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     __syncthreads();
     // the x/z stage is free: prefetch the next tile
     const int next = s_next;
+    __syncthreads();  // every thread has read s_next
+    if (tid == 0) s_next = (int)next2;
     TileCoord nc{};
     if (next < a.n_tiles) nc = coord_of(next, a);
     if (tid == 0 && next < a.n_tiles) issue_tile_loads<T, kGate>(smem, &bar, maps, a, nc);
 
     // ---- phase 2 ---------------------------------------------------------------------
+    // sP is not read after phase 1: the threads the look-back leaves idle stage the next
+    // tile's parameters meanwhile
+    if (tid >= CW && tid < 2 * CW && next < a.n_tiles && nc.cblk != tc.cblk)
+      stage_params(sP, CW, nc.cblk, tid - CW, a);
     if (tid < CW) {
       const int j = tid;
       const int c = tc.cblk * CW + j;
@@ -402,19 +412,38 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         // aggregates until an inclusive state is found. (eA, eB) maps the state at the
         // end of chunk p to the state entering this tile.
         float eA = 1.0f, eB = 0.0f;
-        int64_t p = tc.tix - 1;
+        int64_t p = tc.tix - 1;                      // nearest not yet composed predecessor
+        const int64_t first = tc.tix - tc.chunk;     // chunk 0 of this (b, channel block)
         long long t0 = 0;
         while (true) {
-          const uint32_t hw = ld_relaxed_u32(incl + p * CW + j);
-          const uint64_t aw = ld_relaxed_u64(agg + p * CW + j);
-          if (hw != 0u) {
-            hin = fmaf(eA, dec(hw), eB);
-            break;
+          // one round trip reads the words of up to four predecessors p, p-1, p-2, p-3
+          constexpr int kH = 4;
+          uint32_t hw[kH];
+          uint64_t aw[kH];
+#pragma unroll
+          for (int k = 0; k < kH; ++k) {
+            const int64_t q = p - k;
+            hw[k] = q >= first ? ld_relaxed_u32(incl + q * CW + j) : 0u;
+            aw[k] = q >= first ? ld_relaxed_u64(agg + q * CW + j) : 0ull;
           }
-          if ((uint32_t)aw != 0u) {  // the low half (A) is encoded; B is stored plainly
-            eB = fmaf(eA, __uint_as_float((uint32_t)(aw >> 32)), eB);
-            eA *= dec((uint32_t)aw);
-            --p;
+          bool done = false;
+          int used = 0;
+#pragma unroll
+          for (int k = 0; k < kH; ++k) {
+            if (done || used != k || p - k < first) continue;
+            if (hw[k] != 0u) {
+              hin = fmaf(eA, dec(hw[k]), eB);
+              done = true;
+            } else if ((uint32_t)aw[k] != 0u) {  // the low half (A) is encoded; B is stored plainly
+              eB = fmaf(eA, __uint_as_float((uint32_t)(aw[k] >> 32)), eB);
+              eA *= dec((uint32_t)aw[k]);
+              ++used;
+            }
+          }
+          if (done) break;
+          if (used > 0) {
+            p -= used;
+            t0 = 0;
             continue;
           }
           if (t0 == 0) {
@@ -473,13 +502,8 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         if (t < a.T) __stcs(reinterpret_cast<uint4*>(y + ((int64_t)tc.b * a.T + t) * R + c0), pack_row<V>(o));
       }
     }
-    // sP is not read after phase 1: stage the next tile's parameters now
-    if (tid < CW && next < a.n_tiles && nc.cblk != tc.cblk) stage_params(sP, CW, nc.cblk, tid, a);
     __syncthreads();  // sB and (gated) sg are free
-    if (tid == 0) {
-      if (kGate && next < a.n_tiles) issue_gate_load<T, kGate>(smem, &bar, maps, nc);
-      s_next = (int)atomicAdd(a.ticket, 1u);
-    }
+    if (tid == 0 && kGate && next < a.n_tiles) issue_gate_load<T, kGate>(smem, &bar, maps, nc);
     tile = next;
     phase ^= 1u;
   }
