@@ -11,20 +11,16 @@ constexpr int kGateBlock = 128;
 inline int64_t gate_pitch(int R) { return (int64_t)((R + kGateBlock - 1) / kGateBlock) * 2 * kGateBlock; }
 
 // ---- scan tiling -------------------------------------------------------------------
-constexpr int kScanThreads = 256;
-constexpr int kScanGroups = 16;                         // channel-group threads per CTA
-constexpr int kScanSub = kScanThreads / kScanGroups;    // time sub-chunks per CTA
-constexpr int kScanL = 4;                               // time steps per thread
-constexpr int kScanTC = kScanSub * kScanL;              // time steps per CTA
-inline int scan_vec(bool bf16) { return bf16 ? 8 : 4; }
-inline int scan_cw(bool bf16) { return kScanGroups * scan_vec(bf16); }
+constexpr int kScanTC = 64;   // time steps per tile (one chunk)
+constexpr int kScanSub = 16;  // sub-chunks per tile
+inline int scan_cw(bool bf16) { return bf16 ? 128 : 64; }  // channels per tile
 
 struct ScanLayout {
   int n_cblk, n_chunks;
   int64_t n_tiles;
-  // workspace: [status u32 | ticket u32 | pad to 256 B][aggregates: n_tiles × CW × u64]
-  //            [inclusive states: n_tiles × CW × u32]; all of it must be zero at launch
-  size_t off_agg, off_incl, bytes, zero_bytes;
+  // workspace: [status u32 | ticket u32 | pad to 256 B][inclusive states: n_tiles × CW × u32];
+  // all of it must be zero at launch
+  size_t off_incl, bytes, zero_bytes;
 };
 ScanLayout scan_layout(int B, int T, int R, bool bf16);
 
@@ -48,7 +44,6 @@ struct ScanArgs {
   const float* Lambda;  // [R]
   unsigned* status;     // device status word
   unsigned* ticket;     // tile ticket counter (zero at launch)
-  uint64_t* carry_agg;  // [n_tiles][CW] published aggregates (zero at launch)
   uint32_t* carry_incl; // [n_tiles][CW] published inclusive states (zero at launch)
   int B, T, R, n_cblk, n_chunks, n_tiles;
   int64_t pitch;

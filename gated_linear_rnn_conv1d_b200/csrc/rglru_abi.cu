@@ -176,7 +176,6 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
   a.Lambda = p->Lambda;
   a.status = reinterpret_cast<unsigned*>(ws);
   a.ticket = reinterpret_cast<unsigned*>(bytes(ws) + 4);
-  a.carry_agg = reinterpret_cast<uint64_t*>(bytes(ws) + sl.off_agg);
   a.carry_incl = reinterpret_cast<uint32_t*>(bytes(ws) + sl.off_incl);
   a.B = B;
   a.T = T;
@@ -456,7 +455,6 @@ int rglru_block_forward(const rglru_params* params, const void* W_1, const void*
       a.conv_w = params->conv_w; a.conv_b = params->conv_b; a.Lambda = params->Lambda;
       a.status = status;
       a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
-      a.carry_agg = reinterpret_cast<uint64_t*>(bytes(workspace) + L.scan.off_agg);
       a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);
       a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks;
       a.n_tiles = (int)L.scan.n_tiles; a.pitch = gate_pitch(R);

@@ -10,29 +10,35 @@
 // Local Attention", §Hawk, "Parallel scan").
 //
 // Tiles. A tile is one batch row b, CW consecutive channels (128 for bf16, 64 for f32)
-// and kScanTC = 64 consecutive steps. Its 256 threads are 16 channel groups (16 bytes of
-// channels) × 16 sub-chunks of kScanL = 4 steps.
+// and kScanTC = 64 consecutive steps: 32 channel groups of V channels (4 bf16 or 2 f32)
+// × 16 sub-chunks of 4 steps.
 //
-// Persistent CTAs (as many as fit on the device) take tiles in order from an atomic
-// ticket — time-chunk-major, so every tile a CTA waits for was taken earlier by a running
-// CTA (forward progress) — and prefetch the next ticket and the next tile's data:
-//   load     one thread issues TMA bulk-tensor copies of the tile's x rows (with the
-//            3-row conv halo; rows before t = 0 arrive as zeros), z_a, z_x (and g) into
-//            shared memory; they land while the CTA finishes the previous tile;
-//   phase 1  each thread recomputes u for its 4 steps × V channels in float32, applies
-//            the gates and the log-space decay, folds the 4 steps into an affine map
-//            (float32) and keeps the per-step (1 − a_t, b_t) for the replay; the x/z
-//            stage is then free and the next tile's copies are issued;
-//   phase 2  one thread per channel scans the 16 sub-chunk maps and gets the tile's
-//            incoming state by decoupled look-back over earlier time chunks of the same
-//            (b, channel block). Carries are self-validating words (an exact XOR
-//            encoding whose zero is never a published value, so zeroed memory reads as
-//            "not yet"), so a look-back hop is one round trip with no fence, flag or
-//            barrier; waits are bounded;
-//   phase 3  each thread replays its 4 steps from its incoming state and writes y.
-// The per-step replay values of the bf16 path are held as bf16 pairs (1 − a_t, b_t): their
-// rounding only touches y inside one 4-step run, while the carries and h_T come from the
-// float32 maps.
+// One persistent CTA per SM takes tiles in order from an atomic ticket — time-chunk-major,
+// so every tile a CTA waits for was taken earlier by a running CTA (forward progress) —
+// and runs them through a software pipeline of three warp roles:
+//   producer warp    takes tickets, and two tiles ahead of the compute warps fills a
+//                    3-stage ring: TMA copies of the tile's x rows (with the 3-row conv halo;
+//                    rows before t = 0 arrive as zeros), z_a and z_x, plus the tile's
+//                    parameters (taps, conv bias, c·log σ(Λ)) written into the stage;
+//   compute warps    (16, one per sub-chunk; lane = channel group), for tile k:
+//     phase 1  recompute u in float32, apply the gates and the log-space decay, fold the
+//              sub-chunk's 4 steps into an affine map (float32), and write the per-step
+//              replay values (1 − a_t, b_t) over the z_a, z_x slots they came from;
+//     phase 3  (of tile k − 1, whose incoming states are ready by now) replay the
+//              sub-chunk from its incoming state and write y, then release the stage;
+//   look-back warps  (2, two channels per thread for bf16) read the state entering tile k
+//                    — the inclusive state its predecessor chunk publishes, or h0 — while
+//                    phase 1 of tile k runs; once the 16 sub-chunk maps are in, they chain
+//                    them from that state, publish the tile's inclusive state and hand every
+//                    sub-chunk its incoming state. A published state is a self-validating
+//                    word (an exact XOR encoding whose zero is never a published value, so
+//                    zeroed memory reads as "not yet"): one relaxed load, no fence or flag.
+// Every wait is bounded. Warps of different roles meet at mbarriers (stage full / empty,
+// states ready) and at one named barrier (maps ready) whose id alternates with the tile's
+// parity; the compute warps never wait for one another.
+// The replay values of the bf16 path are stored as bf16 (1 − a_t, b_t): their rounding
+// only touches y inside one 4-step sub-chunk, while the published states and h_T come from
+// the float32 maps.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
@@ -51,29 +57,51 @@ constexpr int kXRows = kScanTC + kHalo;
 
 template <typename T> struct SV;
 template <> struct SV<__nv_bfloat16> {
-  static constexpr int V = 8;
+  static constexpr int V = 4;
   static constexpr bool kAccurate = false;
 };
 template <> struct SV<float> {
-  static constexpr int V = 4;
+  static constexpr int V = 2;
   static constexpr bool kAccurate = true;
 };
 
+constexpr int kGroups = 32;                           // channel groups: the lanes of a compute warp
+constexpr int kSub = kScanSub;                        // sub-chunks: one compute warp each
+constexpr int kL = kScanTC / kSub;                    // steps per sub-chunk
+constexpr int kComputeWarps = kSub;                   // 16
+constexpr int kComputeThreads = kGroups * kSub;       // 512
+constexpr int kLookThreads = 64;
+constexpr int kThreads = kComputeThreads + kLookThreads + 32;  // + one producer warp
+constexpr int kStages = 3;
+// named barrier (id 0 is __syncthreads, which the roles never use after the prologue):
+// + tile parity; compute warps arrive once phase 1 is done, look-back warps wait
+constexpr int kBarMaps = 1;
+
 template <typename T, bool kGate> struct SmemLayout {
-  static constexpr int CW = kScanGroups * SV<T>::V;
+  static constexpr int CW = kGroups * SV<T>::V;
   static constexpr int kX = kXRows * CW * (int)sizeof(T);
   static constexpr int kZ = kScanTC * CW * (int)sizeof(T);
-  static constexpr int kG = kGate ? kZ : 0;
+  // a stage: x rows, z_a, z_x (TMA), then the tile's parameters [6][CW] f32 (taps 0..3,
+  // conv bias, c·log σ(Λ)) written by the producer warp
   static constexpr int offZA = kX;
-  static constexpr int offZX = offZA + kZ;
-  static constexpr int offG = offZX + kZ;
-  static constexpr int offA = offG + kG;
-  static constexpr int offB = offA + kScanSub * CW * 4;
-  static constexpr int offP = offB + kScanSub * CW * 4;   // [6][CW]: taps 0..3, conv bias, c·log σ(Λ)
-  static constexpr int kBytes = offP + 6 * CW * 4;
-  static constexpr int kAlloc = kBytes + 128;  // slack to align the base to 128 bytes
+  static constexpr int offZX = kX + kZ;
+  static constexpr int offPar = kX + 2 * kZ;
+  static constexpr int kStage = offPar + 6 * CW * 4;
+  static constexpr int offMaps = kStages * kStage;     // [2 buffers][A | B][kSub][CW] f32
+  static constexpr int kMaps = 2 * kSub * CW * 4;
+  static constexpr int kBytes = offMaps + 2 * kMaps;
+  static constexpr int kAlloc = kBytes + 128;          // slack to align the base to 128 bytes
   static constexpr uint32_t kTxXZ = kX + 2 * kZ;
+  static_assert(kX % 128 == 0 && kStage % 128 == 0, "TMA destinations 128-byte aligned");
+  static_assert(kAlloc <= 227 * 1024, "shared memory");
 };
+
+__device__ __forceinline__ void bar_sync_n(int id, int n) {  // id is warp-uniform
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void bar_arrive_n(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1, int c2) {
   asm volatile(
@@ -88,16 +116,8 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
   asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
 __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // Published carries are stored as their bit pattern XOR 0x7FFFFFFF: an exact, reversible
@@ -123,24 +143,67 @@ __device__ __forceinline__ TileCoord coord_of(int ticket, const ScanArgs& a) {
 }
 
 template <typename T, bool kGate>
-__device__ __forceinline__ void issue_tile_loads(uint8_t* smem, uint64_t* bar, const ScanMaps& m, const ScanArgs& a,
+__device__ __forceinline__ void issue_tile_loads(uint8_t* stage, uint64_t* bar, const ScanMaps& m, const ScanArgs& a,
                                                  const TileCoord& c) {
   using Ly = SmemLayout<T, kGate>;
   constexpr int CW = Ly::CW;
-  mbar_arrive_expect_tx(bar, Ly::kTxXZ + Ly::kG);
+  mbar_arrive_expect_tx(bar, Ly::kTxXZ);
   const int c0 = c.cblk * CW;
   const int t0 = c.chunk * kScanTC;
-  tma_load_3d(smem, &m.x, bar, c0, t0 - kHalo, c.b);
+  tma_load_3d(stage, &m.x, bar, c0, t0 - kHalo, c.b);
   const int zcol = (c0 / kGateBlock) * 2 * kGateBlock + (c0 % kGateBlock);
   const int zrow = c.b * a.T + t0;
-  tma_load_2d(smem + Ly::offZA, &m.z, bar, zcol, zrow);
-  tma_load_2d(smem + Ly::offZX, &m.z, bar, zcol + kGateBlock, zrow);
+  tma_load_2d(stage + Ly::offZA, &m.z, bar, zcol, zrow);
+  tma_load_2d(stage + Ly::offZX, &m.z, bar, zcol + kGateBlock, zrow);
 }
 
-template <typename T, bool kGate>
-__device__ __forceinline__ void issue_gate_load(uint8_t* smem, uint64_t* bar, const ScanMaps& m, const TileCoord& c) {
-  using Ly = SmemLayout<T, kGate>;
-  tma_load_3d(smem + Ly::offG, &m.g, bar, c.cblk * Ly::CW, c.chunk * kScanTC, c.b);
+// V consecutive elements as floats, and back (shared or global memory).
+__device__ __forceinline__ void ldv(const __nv_bfloat16* p, float (&f)[4]) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  f[0] = bf16lo(r.x); f[1] = bf16hi(r.x); f[2] = bf16lo(r.y); f[3] = bf16hi(r.y);
+}
+__device__ __forceinline__ void ldv(const float* p, float (&f)[2]) {
+  const float2 r = *reinterpret_cast<const float2*>(p);
+  f[0] = r.x; f[1] = r.y;
+}
+__device__ __forceinline__ void stv(__nv_bfloat16* p, const float (&f)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+}
+__device__ __forceinline__ void stv(float* p, const float (&f)[2]) {
+  *reinterpret_cast<float2*>(p) = make_float2(f[0], f[1]);
+}
+// read-only global loads of an input row segment
+__device__ __forceinline__ void ldv_nc(const __nv_bfloat16* p, float (&f)[4]) {
+  const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+  f[0] = bf16lo(r.x); f[1] = bf16hi(r.x); f[2] = bf16lo(r.y); f[3] = bf16hi(r.y);
+}
+__device__ __forceinline__ void ldv_nc(const float* p, float (&f)[2]) {
+  const float2 r = __ldg(reinterpret_cast<const float2*>(p));
+  f[0] = r.x; f[1] = r.y;
+}
+// streaming store of an output row segment (y is not re-read by this kernel)
+__device__ __forceinline__ void stv_cs(__nv_bfloat16* p, const float (&f)[4]) {
+  __stcs(reinterpret_cast<uint2*>(p), make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3])));
+}
+__device__ __forceinline__ void stv_cs(float* p, const float (&f)[2]) {
+  __stcs(reinterpret_cast<float2*>(p), make_float2(f[0], f[1]));
+}
+// V float32 values from shared memory
+template <int V> __device__ __forceinline__ void ldf(const float* p, float (&f)[V]);
+template <> __device__ __forceinline__ void ldf<4>(const float* p, float (&f)[4]) {
+  const float4 r = *reinterpret_cast<const float4*>(p);
+  f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
+}
+template <> __device__ __forceinline__ void ldf<2>(const float* p, float (&f)[2]) {
+  const float2 r = *reinterpret_cast<const float2*>(p);
+  f[0] = r.x; f[1] = r.y;
+}
+template <int V> __device__ __forceinline__ void stf(float* p, const float (&f)[V]);
+template <> __device__ __forceinline__ void stf<4>(float* p, const float (&f)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+}
+template <> __device__ __forceinline__ void stf<2>(float* p, const float (&f)[2]) {
+  *reinterpret_cast<float2*>(p) = make_float2(f[0], f[1]);
 }
 
 // −expm1(x) for x ∈ [−1/8, 0] on a pair of lanes: the Taylor series of e^x − 1 about 0
@@ -159,13 +222,15 @@ __device__ __forceinline__ float2 neg_expm1_eighth2(float2 x) {
 // r = σ(z_a) (ex2 + rcp); log a_t = r·cla; d = −expm1(log a_t) (polynomial on [−1/8, 0],
 // 1 − ex2 beyond); 1 − a_t² = d (2 − d); √(1−a_t²)·i = q·rsqrt(q (1 + e^{−z_x})² + 1e-30)
 // (the tiny term keeps q = 0 exact: 0·finite). Four MUFU operations per element.
+template <bool kSmall = false>
 __device__ __forceinline__ void gate_fast2(float2 za, float2 zx, float2 cla, float2 u, float2& d, float2& bt) {
   const float2 na = __fmul2_rn(za, make_float2(-kLog2e, -kLog2e));
   const float2 nx = __fmul2_rn(zx, make_float2(-kLog2e, -kLog2e));
   const float2 ea = __fadd2_rn(make_float2(ex2_approx(na.x), ex2_approx(na.y)), make_float2(1.0f, 1.0f));
   const float2 r = make_float2(rcp_approx(ea.x), rcp_approx(ea.y));
   const float2 la = __fmul2_rn(r, cla);
-  if (fminf(la.x, la.y) >= -0.125f) {
+  if (kSmall || fminf(la.x, la.y) >= -0.125f) {
+    // kSmall: the caller knows c·log σ(Λ) ≥ −1/8, hence log a_t = r·c·log σ(Λ) ≥ −1/8
     d = neg_expm1_eighth2(la);
   } else {
     d.x = la.x >= -0.125f ? neg_expm1_small(la.x) : 1.0f - ex2_approx(la.x * kLog2e);
@@ -178,358 +243,464 @@ __device__ __forceinline__ void gate_fast2(float2 za, float2 zx, float2 cla, flo
   bt = __fmul2_rn(__fmul2_rn(q, rs), u);
 }
 
-// Stages the per-channel parameters of channel block `cblk` (one thread per channel).
-__device__ __forceinline__ void stage_params(float* sP, int CW, int cblk, int j, const ScanArgs& a) {
-  const int c = cblk * CW + j;
-  const bool ok = c < a.R;
-  const int R = a.R;
-  sP[0 * CW + j] = ok ? __ldg(a.conv_w + c) : 0.0f;
-  sP[1 * CW + j] = ok ? __ldg(a.conv_w + R + c) : 0.0f;
-  sP[2 * CW + j] = ok ? __ldg(a.conv_w + 2 * R + c) : 0.0f;
-  sP[3 * CW + j] = ok ? __ldg(a.conv_w + 3 * R + c) : 0.0f;
-  sP[4 * CW + j] = ok ? __ldg(a.conv_b + c) : 0.0f;
-  sP[5 * CW + j] = ok ? decay_log_coeff(__ldg(a.Lambda + c)) : 0.0f;
+// A producer lane's share of one tile's parameters: PV = CW / 32 consecutive channels.
+template <int PV> struct ParRegs {
+  float w[4][PV], cb[PV], lam[PV];
+};
+// Issues the loads for channels c .. c+PV-1 (taps 0..3, conv bias, Λ); channels past R
+// read as 0 (c is a multiple of PV and R of 8, so a lane's channels are all in or all out).
+// Nothing here waits for the values.
+template <int PV>
+__device__ __forceinline__ void load_params(ParRegs<PV>& p, int c, const ScanArgs& a) {
+#pragma unroll
+  for (int v = 0; v < PV; ++v) {
+    p.w[0][v] = p.w[1][v] = p.w[2][v] = p.w[3][v] = 0.0f;
+    p.cb[v] = p.lam[v] = 0.0f;
+  }
+  if (c < a.R) {
+    const int R = a.R;
+#pragma unroll
+    for (int v = 0; v < PV; ++v) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p.w[i][v] = __ldg(a.conv_w + i * R + c + v);
+      p.cb[v] = __ldg(a.conv_b + c + v);
+      p.lam[v] = __ldg(a.Lambda + c + v);
+    }
+  }
+}
+// Writes them into a stage's parameter block [6][CW] at channel slot jj, with Λ turned into
+// c·log σ(Λ) (0 for channels past R, which makes their steps identities).
+template <int PV>
+__device__ __forceinline__ void store_params(float* sPar, int CW, int jj, bool in_range, const ParRegs<PV>& p) {
+  float cla[PV];
+#pragma unroll
+  for (int v = 0; v < PV; ++v) cla[v] = in_range ? decay_log_coeff(p.lam[v]) : 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) stf<PV>(sPar + i * CW + jj, p.w[i]);
+  stf<PV>(sPar + 4 * CW + jj, p.cb);
+  stf<PV>(sPar + 5 * CW + jj, cla);
 }
 
-// Four consecutive elements of type T from shared memory, as floats.
-template <typename T> __device__ __forceinline__ float4 lds4(const T* p);
-template <> __device__ __forceinline__ float4 lds4<__nv_bfloat16>(const __nv_bfloat16* p) {
-  const uint2 r = *reinterpret_cast<const uint2*>(p);
-  return make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
-}
-template <> __device__ __forceinline__ float4 lds4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
-
-template <int V> __device__ __forceinline__ void unpack_row(const uint4& r, float (&f)[V]);
-template <> __device__ __forceinline__ void unpack_row<8>(const uint4& r, float (&f)[8]) {
-  f[0] = bf16lo(r.x); f[1] = bf16hi(r.x); f[2] = bf16lo(r.y); f[3] = bf16hi(r.y);
-  f[4] = bf16lo(r.z); f[5] = bf16hi(r.z); f[6] = bf16lo(r.w); f[7] = bf16hi(r.w);
-}
-template <> __device__ __forceinline__ void unpack_row<4>(const uint4& r, float (&f)[4]) {
-  f[0] = __uint_as_float(r.x); f[1] = __uint_as_float(r.y); f[2] = __uint_as_float(r.z); f[3] = __uint_as_float(r.w);
-}
-template <int V> __device__ __forceinline__ uint4 pack_row(const float (&f)[V]);
-template <> __device__ __forceinline__ uint4 pack_row<8>(const float (&f)[8]) {
-  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-}
-template <> __device__ __forceinline__ uint4 pack_row<4>(const float (&f)[4]) {
-  return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
-}
-
-template <typename T, bool kGate>
-__global__ void __launch_bounds__(kScanThreads, 2)
-    rglru_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs a) {
+// Phase 1 of one tile for compute thread (g, s): conv, gates, log-space decay and the fold
+// of the sub-chunk's 4 steps into (A, B); the replay values go over the z_a, z_x slots the
+// thread read them from (no other thread reads those slots).
+// kFast: every step of the sub-chunk is inside [0, T) and every channel of the warp has
+// c·log σ(Λ) ≥ −1/8, so neither the identity-step mask nor the wide decay path is needed.
+template <typename T, bool kGate, bool kFast>
+__device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB, const TileCoord& tc, int g, int s,
+                                            const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
   constexpr int V = SV<T>::V;
   constexpr int CW = Ly::CW;
-  constexpr int S = kScanSub;
-  constexpr int L = kScanL;
   constexpr bool kAcc = SV<T>::kAccurate;
-  static_assert(2 * CW <= kScanThreads, "phase 2 needs CW look-back threads and CW staging threads");
+  const T* sx = reinterpret_cast<const T*>(stage);
+  T* sza = reinterpret_cast<T*>(stage + Ly::offZA);
+  T* szx = reinterpret_cast<T*>(stage + Ly::offZX);
+  const float* sP = reinterpret_cast<const float*>(stage + Ly::offPar);
+  const int cc = g * V;
+  const int c0 = tc.cblk * CW + cc;
+  const int t_start = tc.chunk * kScanTC + s * kL;
+
+  float W0[V], W1[V], W2[V], W3[V], CB[V], CL[V];
+  ldf<V>(sP + 0 * CW + cc, W0);
+  ldf<V>(sP + 1 * CW + cc, W1);
+  ldf<V>(sP + 2 * CW + cc, W2);
+  ldf<V>(sP + 3 * CW + cc, W3);
+  ldf<V>(sP + 4 * CW + cc, CB);
+  ldf<V>(sP + 5 * CW + cc, CL);
+  float xm3[V], xm2[V], xm1[V];
+  if (tc.chunk == 0 && s == 0 && a.state0 != nullptr) {
+    // conv history of the first steps: the caller's state, oldest row first
+#pragma unroll
+    for (int v = 0; v < V; ++v) xm3[v] = xm2[v] = xm1[v] = 0.0f;
+    if (c0 < a.R) {
+      const T* st = static_cast<const T*>(a.state0) + (int64_t)tc.b * 3 * a.R + c0;
+      ldv(st, xm3);
+      ldv(st + a.R, xm2);
+      ldv(st + 2 * a.R, xm1);
+    }
+  } else {
+    ldv(sx + (s * kL + 0) * CW + cc, xm3);
+    ldv(sx + (s * kL + 1) * CW + cc, xm2);
+    ldv(sx + (s * kL + 2) * CW + cc, xm1);
+  }
+  float A[V], B[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) { A[v] = 1.0f; B[v] = 0.0f; }
+#pragma unroll
+  for (int l = 0; l < kL; ++l) {
+    const int row = s * kL + l;
+    float xc[V], za[V], zx[V];
+    ldv(sx + (row + kHalo) * CW + cc, xc);
+    ldv(sza + row * CW + cc, za);
+    ldv(szx + row * CW + cc, zx);
+    const bool tv = kFast || (t_start + l) < a.T;
+    float u[V];
+#pragma unroll
+    for (int v = 0; v < V; v += 2) {
+      float2 uu = __ffma2_rn(make_float2(W0[v], W0[v + 1]), make_float2(xm3[v], xm3[v + 1]), make_float2(CB[v], CB[v + 1]));
+      uu = __ffma2_rn(make_float2(W1[v], W1[v + 1]), make_float2(xm2[v], xm2[v + 1]), uu);
+      uu = __ffma2_rn(make_float2(W2[v], W2[v + 1]), make_float2(xm1[v], xm1[v + 1]), uu);
+      uu = __ffma2_rn(make_float2(W3[v], W3[v + 1]), make_float2(xc[v], xc[v + 1]), uu);
+      u[v] = uu.x;
+      u[v + 1] = uu.y;
+    }
+    float at[V], r0[V], bt[V];  // r0: what goes over z_a (a_t, or 1 − a_t on the bf16 path)
+    if constexpr (kAcc) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) gate_accurate(za[v], zx[v], CL[v], u[v], at[v], bt[v]);
+      if (!tv) {
+        // steps past T are identity steps
+#pragma unroll
+        for (int v = 0; v < V; ++v) { at[v] = 1.0f; bt[v] = 0.0f; }
+      }
+#pragma unroll
+      for (int v = 0; v < V; ++v) r0[v] = at[v];
+    } else {
+      if (!tv) {
+        // steps past T: r = σ(−∞) = 0 makes a_t = 1 and b_t = 0 (identity steps)
+#pragma unroll
+        for (int v = 0; v < V; ++v) za[v] = -INFINITY;
+      }
+#pragma unroll
+      for (int v = 0; v < V; v += 2) {
+        float2 d, b2;
+        gate_fast2<kFast>(make_float2(za[v], za[v + 1]), make_float2(zx[v], zx[v + 1]),
+                          make_float2(CL[v], CL[v + 1]), make_float2(u[v], u[v + 1]), d, b2);
+        r0[v] = d.x;
+        r0[v + 1] = d.y;
+        bt[v] = b2.x;
+        bt[v + 1] = b2.y;
+        at[v] = 1.0f - d.x;
+        at[v + 1] = 1.0f - d.y;
+      }
+    }
+    stv(sza + row * CW + cc, r0);
+    stv(szx + row * CW + cc, bt);
+    // fold: (A, B) ← (a·A, a·B + b)
+#pragma unroll
+    for (int v = 0; v < V; v += 2) {
+      const float2 a2 = make_float2(at[v], at[v + 1]);
+      const float2 nb = __ffma2_rn(a2, make_float2(B[v], B[v + 1]), make_float2(bt[v], bt[v + 1]));
+      const float2 na = __fmul2_rn(a2, make_float2(A[v], A[v + 1]));
+      A[v] = na.x; A[v + 1] = na.y;
+      B[v] = nb.x; B[v + 1] = nb.y;
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      xm3[v] = xm2[v];
+      xm2[v] = xm1[v];
+      xm1[v] = xc[v];
+    }
+  }
+  stf<V>(mA + s * CW + cc, A);
+  stf<V>(mB + s * CW + cc, B);
+}
+
+template <typename T, bool kGate>
+__device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, const TileCoord& tc, int g, int s,
+                                       const ScanArgs& a) {
+  using Ly = SmemLayout<T, kGate>;
+  constexpr int V = SV<T>::V;
+  bool fast = false;
+  if constexpr (!SV<T>::kAccurate) {
+    const float* CL = reinterpret_cast<const float*>(stage + Ly::offPar) + 5 * Ly::CW + g * V;
+    bool small = true;
+#pragma unroll
+    for (int v = 0; v < V; ++v) small = small && CL[v] >= -0.125f;
+    fast = __all_sync(0xffffffffu, small) && tc.chunk * kScanTC + (s + 1) * kL <= a.T;
+  }
+  if (fast)
+    phase1_body<T, kGate, true>(stage, mA, mB, tc, g, s, a);
+  else
+    phase1_body<T, kGate, false>(stage, mA, mB, tc, g, s, a);
+}
+
+// Phase 3 of one tile for compute thread (g, s): replay the sub-chunk from its incoming
+// state (mH) and write y (times GeLU of the gate branch for the gated scan). Every
+// shared-memory read comes first and is followed by the proxy fence that lets the stage be
+// refilled by asynchronous copies; only then are the global stores issued, so the fence
+// never waits for them.
+template <typename T, bool kGate>
+__device__ __forceinline__ void phase3(const uint8_t* stage, const float* mH, const TileCoord& tc, int g, int s,
+                                       const ScanArgs& a) {
+  using Ly = SmemLayout<T, kGate>;
+  constexpr int V = SV<T>::V;
+  constexpr int CW = Ly::CW;
+  constexpr bool kAcc = SV<T>::kAccurate;
+  const T* sza = reinterpret_cast<const T*>(stage + Ly::offZA);
+  const T* szx = reinterpret_cast<const T*>(stage + Ly::offZX);
+  const int cc = g * V;
+  const int c0 = tc.cblk * CW + cc;
+  const int t_start = tc.chunk * kScanTC + s * kL;
+  float h[V];
+  float r0[kL][V], bt[kL][V], gg[kGate ? kL : 1][V];
+  if constexpr (kGate) {
+    // the gate branch comes straight from global memory; its loads are issued first
+    const T* gsrc = static_cast<const T*>(a.g);
+#pragma unroll
+    for (int l = 0; l < kL; ++l) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) gg[l][v] = 0.0f;
+      if (c0 < a.R && t_start + l < a.T) ldv_nc(gsrc + ((int64_t)tc.b * a.T + t_start + l) * a.R + c0, gg[l]);
+    }
+  }
+  ldf<V>(mH + s * CW + cc, h);
+#pragma unroll
+  for (int l = 0; l < kL; ++l) {
+    const int row = s * kL + l;
+    ldv(sza + row * CW + cc, r0[l]);
+    ldv(szx + row * CW + cc, bt[l]);
+  }
+  fence_proxy_async_smem();
+  if (c0 >= a.R) return;
+  T* __restrict__ y = static_cast<T*>(a.y);
+#pragma unroll
+  for (int l = 0; l < kL; ++l) {
+    float o[V];
+#pragma unroll
+    for (int v = 0; v < V; v += 2) {
+      const float2 a2 =
+          kAcc ? make_float2(r0[l][v], r0[l][v + 1]) : make_float2(1.0f - r0[l][v], 1.0f - r0[l][v + 1]);
+      const float2 h2 = __ffma2_rn(a2, make_float2(h[v], h[v + 1]), make_float2(bt[l][v], bt[l][v + 1]));
+      h[v] = o[v] = h2.x;
+      h[v + 1] = o[v + 1] = h2.y;
+    }
+    if constexpr (kGate) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) o[v] *= gelu_exact(gg[l][v]);
+    }
+    const int t = t_start + l;
+    if (t < a.T) stv_cs(y + ((int64_t)tc.b * a.T + t) * a.R + c0, o);
+  }
+}
+
+// Look-back, first half, for thread j's NCH channel slots j, j + CW/NCH, ...: the state
+// entering the tile, read from the inclusive state its predecessor (the previous time chunk
+// of the same batch row and channel block) publishes, or h0 for the first chunk. It needs
+// nothing of this tile, so it runs while phase 1 of the tile is still in progress.
+template <typename T, bool kGate, int NCH>
+__device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const ScanArgs& a, float (&hin)[NCH]) {
+  constexpr int CW = SmemLayout<T, kGate>::CW;
+  constexpr int kStride = CW / NCH;
+  if (tc.chunk == 0) {
+#pragma unroll
+    for (int n = 0; n < NCH; ++n) {
+      const int c = tc.cblk * CW + j + n * kStride;
+      hin[n] = (a.h0 != nullptr && c < a.R) ? a.h0[(int64_t)tc.b * a.R + c] : 0.0f;
+    }
+    return;
+  }
+  const uint32_t* src = a.carry_incl + (tc.tix - 1) * CW + j;
+  uint32_t w[NCH];
+#pragma unroll
+  for (int n = 0; n < NCH; ++n) w[n] = ld_relaxed_u32(src + n * kStride);
+  bool ready = true;
+#pragma unroll
+  for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
+  if (!ready) {
+    const long long t0 = clock64();
+    while (true) {
+#pragma unroll
+      for (int n = 0; n < NCH; ++n)
+        if (w[n] == 0u) w[n] = ld_relaxed_u32(src + n * kStride);
+      ready = true;
+#pragma unroll
+      for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
+      if (ready) break;
+      if (clock64() - t0 > kWaitCycles) {
+        atomicOr(a.status, kStatusTimeout);
+        break;
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NCH; ++n) hin[n] = w[n] != 0u ? dec(w[n]) : 0.0f;
+}
+
+// Look-back, second half, once phase 1 of the tile is done: scans the sub-chunk maps
+// (mA, mB), publishes the tile's inclusive states, writes h_T for the last chunk, and
+// leaves each sub-chunk's incoming state in mB.
+template <typename T, bool kGate, int NCH>
+__device__ __forceinline__ void lookback_finish(const float* mA, float* mB, const TileCoord& tc, int j,
+                                                const ScanArgs& a, const float (&hin)[NCH]) {
+  constexpr int CW = SmemLayout<T, kGate>::CW;
+  constexpr int S = kSub;
+  constexpr int kStride = CW / NCH;
+  const bool publish = tc.tix != a.stall_tile;
+#pragma unroll
+  for (int n = 0; n < NCH; ++n) {
+    const int jj = j + n * kStride;
+    const int c = tc.cblk * CW + jj;
+    // the state entering each sub-chunk, and after the last one the tile's inclusive state
+    float h = hin[n];
+#pragma unroll
+    for (int q = 0; q < S; ++q) {
+      const float pa = mA[q * CW + jj], pb = mB[q * CW + jj];
+      mB[q * CW + jj] = h;
+      h = fmaf(pa, h, pb);
+    }
+    if (publish) st_relaxed_u32(a.carry_incl + tc.tix * CW + jj, enc(h));
+    if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < a.R) a.hT[(int64_t)tc.b * a.R + c] = h;
+  }
+}
+
+template <typename T, bool kGate>
+__global__ void __launch_bounds__(kThreads, 1)
+    rglru_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs a) {
+  using Ly = SmemLayout<T, kGate>;
+  constexpr int CW = Ly::CW;
+  constexpr int PV = CW / 32;  // channels per producer lane
+  constexpr int NCH = CW / kLookThreads;  // channels per look-back thread
+  static_assert(CW % kLookThreads == 0 && CW % 32 == 0, "thread roles");
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_ticket, s_next;
-  float* sA = reinterpret_cast<float*>(smem + Ly::offA);
-  float* sB = reinterpret_cast<float*>(smem + Ly::offB);
-  float* sP = reinterpret_cast<float*>(smem + Ly::offP);
-  const T* sx = reinterpret_cast<const T*>(smem);
-  const T* sza = reinterpret_cast<const T*>(smem + Ly::offZA);
-  const T* szx = reinterpret_cast<const T*>(smem + Ly::offZX);
-  const T* sg = reinterpret_cast<const T*>(smem + Ly::offG);
-
+  __shared__ __align__(8) uint64_t full[kStages];   // TMA bytes + the producer's parameters
+  __shared__ __align__(8) uint64_t empty[kStages];  // one arrival per compute warp after phase 3
+  __shared__ __align__(8) uint64_t state[2];        // + tile parity: incoming states ready
+  __shared__ int s_tile[kStages];                   // ticket of the tile in each stage
+  float* maps_base = reinterpret_cast<float*>(smem + Ly::offMaps);
   const int tid = threadIdx.x;
-  const int g = tid % kScanGroups;
-  const int s = tid / kScanGroups;
-  const int R = a.R;
-  volatile int no_abort = 0;
+  const int lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(&bar, 1);
-    fence_barrier_init();
-    tma_prefetch_desc(&maps.x);
-    tma_prefetch_desc(&maps.z);
-    if (kGate) tma_prefetch_desc(&maps.g);
-    const int t = (int)atomicAdd(a.ticket, 1u);
-    s_ticket = t;
-    if (t < a.n_tiles) {
-      const TileCoord c = coord_of(t, a);
-      issue_tile_loads<T, kGate>(smem, &bar, maps, a, c);
-      if (kGate) issue_gate_load<T, kGate>(smem, &bar, maps, c);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 2);
+      mbar_init(&empty[i], kComputeWarps);
     }
-    s_next = (int)atomicAdd(a.ticket, 1u);
+    mbar_init(&state[0], kLookThreads);
+    mbar_init(&state[1], kLookThreads);
+    fence_barrier_init();
   }
   __syncthreads();
-  int tile = s_ticket;
-  if (tid < CW && tile < a.n_tiles) stage_params(sP, CW, coord_of(tile, a).cblk, tid, a);
-  __syncthreads();
-  uint32_t phase = 0;
 
-  while (tile < a.n_tiles) {
-    const TileCoord tc = coord_of(tile, a);
-    const int c0 = tc.cblk * CW + g * V;
-    const bool cvalid = c0 < R;
-    const int t_start = tc.chunk * kScanTC + s * L;
-
-    if (!mbar_wait(&bar, phase, &no_abort)) {
-      if (tid == 0) atomicOr(a.status, kStatusTimeout);
-    }
-    // the ticket after `next` is fetched now; its round trip overlaps phase 1
-    unsigned next2 = 0;
-    if (tid == 0) next2 = atomicAdd(a.ticket, 1u);
-
-    // ---- phase 1 ---------------------------------------------------------------------
-    // Channels are taken four at a time, so that only four channels' parameters and
-    // conv history are live at once.
-    // Per-step replay values stay in registers: the shared-memory stage is refilled with the
-    // next tile as soon as phase 1 is done.
-    uint32_t rp[kAcc ? 1 : L * V];                    // bf16 path: (1 − a_t, b_t) pairs
-    float ra[kAcc ? L * V : 1], rb[kAcc ? L * V : 1];  // f32 path: a_t, b_t
-    float Ag[V], Bg[V];
-    const bool from_state = (tc.chunk == 0 && s == 0 && a.state0 != nullptr);
-#pragma unroll
-    for (int vb = 0; vb < V; vb += 4) {
-      const int cc = g * V + vb;  // channel offset inside the tile
-      const float4 W0 = *reinterpret_cast<const float4*>(sP + 0 * CW + cc);
-      const float4 W1 = *reinterpret_cast<const float4*>(sP + 1 * CW + cc);
-      const float4 W2 = *reinterpret_cast<const float4*>(sP + 2 * CW + cc);
-      const float4 W3 = *reinterpret_cast<const float4*>(sP + 3 * CW + cc);
-      const float4 CB = *reinterpret_cast<const float4*>(sP + 4 * CW + cc);
-      const float4 CL = *reinterpret_cast<const float4*>(sP + 5 * CW + cc);
-      float4 xm3, xm2, xm1;
-      if (from_state) {
-        const T* st = static_cast<const T*>(a.state0) + (int64_t)tc.b * 3 * R + c0 + vb;
-        xm3 = cvalid ? lds4<T>(st) : make_float4(0.f, 0.f, 0.f, 0.f);
-        xm2 = cvalid ? lds4<T>(st + R) : make_float4(0.f, 0.f, 0.f, 0.f);
-        xm1 = cvalid ? lds4<T>(st + 2 * R) : make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        xm3 = lds4<T>(sx + (s * L + 0) * CW + cc);
-        xm2 = lds4<T>(sx + (s * L + 1) * CW + cc);
-        xm1 = lds4<T>(sx + (s * L + 2) * CW + cc);
+  if (tid < kComputeThreads) {
+    // ---- compute warps: phase 1 of tile k, then phase 3 of tile k − 1 ----------------
+    const int g = lane;
+    const int s = tid / 32;
+    for (int k = 0;; ++k) {
+      const int st = k % kStages;
+      if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
+        if (lane == 0) atomicOr(a.status, kStatusTimeout);
       }
-      float4 A4 = make_float4(1.f, 1.f, 1.f, 1.f), B4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int l = 0; l < L; ++l) {
-        const int row = s * L + l;
-        const float4 xc = lds4<T>(sx + (row + kHalo) * CW + cc);
-        float4 za = lds4<T>(sza + row * CW + cc);
-        const float4 zx = lds4<T>(szx + row * CW + cc);
-        const bool tv = (t_start + l) < a.T;
-        if (!kAcc && !tv) {
-          // steps past T: r = σ(−∞) = 0 makes a_t = 1 and b_t = 0 (identity steps)
-          za = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      const int tile = s_tile[st];
+      const bool valid = tile < a.n_tiles;
+      if (valid) {
+        float* mA = maps_base + (k & 1) * 2 * kSub * CW;
+        phase1<T, kGate>(smem + st * Ly::kStage, mA, mA + kSub * CW, coord_of(tile, a), g, s, a);
+      }
+      // the look-back warps learn of the end of the tile sequence through this barrier too
+      bar_arrive_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
+      if (k >= 1) {
+        const int kp = k - 1;
+        const int stp = kp % kStages;
+        if (!mbar_wait_sleep(&state[kp & 1], (uint32_t)(kp >> 1) & 1u)) {
+          if (lane == 0) atomicOr(a.status, kStatusTimeout);
         }
-        float2 u01 = __ffma2_rn(make_float2(W0.x, W0.y), make_float2(xm3.x, xm3.y), make_float2(CB.x, CB.y));
-        float2 u23 = __ffma2_rn(make_float2(W0.z, W0.w), make_float2(xm3.z, xm3.w), make_float2(CB.z, CB.w));
-        u01 = __ffma2_rn(make_float2(W1.x, W1.y), make_float2(xm2.x, xm2.y), u01);
-        u23 = __ffma2_rn(make_float2(W1.z, W1.w), make_float2(xm2.z, xm2.w), u23);
-        u01 = __ffma2_rn(make_float2(W2.x, W2.y), make_float2(xm1.x, xm1.y), u01);
-        u23 = __ffma2_rn(make_float2(W2.z, W2.w), make_float2(xm1.z, xm1.w), u23);
-        u01 = __ffma2_rn(make_float2(W3.x, W3.y), make_float2(xc.x, xc.y), u01);
-        u23 = __ffma2_rn(make_float2(W3.z, W3.w), make_float2(xc.z, xc.w), u23);
-        const float4 u = make_float4(u01.x, u01.y, u23.x, u23.y);
-        float2 at0, bt0, at1, bt1;
-        if constexpr (kAcc) {
-          gate_accurate(za.x, zx.x, CL.x, u.x, at0.x, bt0.x);
-          gate_accurate(za.y, zx.y, CL.y, u.y, at0.y, bt0.y);
-          gate_accurate(za.z, zx.z, CL.z, u.z, at1.x, bt1.x);
-          gate_accurate(za.w, zx.w, CL.w, u.w, at1.y, bt1.y);
-          if (!tv) { at0 = at1 = make_float2(1.f, 1.f); bt0 = bt1 = make_float2(0.f, 0.f); }
-          ra[l * V + vb + 0] = at0.x; ra[l * V + vb + 1] = at0.y; ra[l * V + vb + 2] = at1.x; ra[l * V + vb + 3] = at1.y;
-          rb[l * V + vb + 0] = bt0.x; rb[l * V + vb + 1] = bt0.y; rb[l * V + vb + 2] = bt1.x; rb[l * V + vb + 3] = bt1.y;
-        } else {
-          float2 d0, d1;
-          gate_fast2(make_float2(za.x, za.y), make_float2(zx.x, zx.y), make_float2(CL.x, CL.y),
-                     make_float2(u.x, u.y), d0, bt0);
-          gate_fast2(make_float2(za.z, za.w), make_float2(zx.z, zx.w), make_float2(CL.z, CL.w),
-                     make_float2(u.z, u.w), d1, bt1);
-          at0 = make_float2(1.f - d0.x, 1.f - d0.y);
-          at1 = make_float2(1.f - d1.x, 1.f - d1.y);
-          rp[l * V + vb + 0] = pack_bf16x2(d0.x, bt0.x);
-          rp[l * V + vb + 1] = pack_bf16x2(d0.y, bt0.y);
-          rp[l * V + vb + 2] = pack_bf16x2(d1.x, bt1.x);
-          rp[l * V + vb + 3] = pack_bf16x2(d1.y, bt1.y);
-        }
-        // fold: (A, B) ← (a·A, a·B + b)
-        const float2 B01 = __ffma2_rn(at0, make_float2(B4.x, B4.y), bt0);
-        const float2 B23 = __ffma2_rn(at1, make_float2(B4.z, B4.w), bt1);
-        const float2 A01 = __fmul2_rn(at0, make_float2(A4.x, A4.y));
-        const float2 A23 = __fmul2_rn(at1, make_float2(A4.z, A4.w));
-        A4 = make_float4(A01.x, A01.y, A23.x, A23.y);
-        B4 = make_float4(B01.x, B01.y, B23.x, B23.y);
-        xm3 = xm2;
-        xm2 = xm1;
-        xm1 = xc;
+        const float* mH = maps_base + (kp & 1) * 2 * kSub * CW + kSub * CW;
+        phase3<T, kGate>(smem + stp * Ly::kStage, mH, coord_of(s_tile[stp], a), g, s, a);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stp]);
       }
-      Ag[vb + 0] = A4.x; Ag[vb + 1] = A4.y; Ag[vb + 2] = A4.z; Ag[vb + 3] = A4.w;
-      Bg[vb + 0] = B4.x; Bg[vb + 1] = B4.y; Bg[vb + 2] = B4.z; Bg[vb + 3] = B4.w;
+      if (!valid) break;
     }
-#pragma unroll
-    for (int v = 0; v < V; v += 4) {
-      *reinterpret_cast<float4*>(sA + s * CW + g * V + v) = make_float4(Ag[v], Ag[v + 1], Ag[v + 2], Ag[v + 3]);
-      *reinterpret_cast<float4*>(sB + s * CW + g * V + v) = make_float4(Bg[v], Bg[v + 1], Bg[v + 2], Bg[v + 3]);
-    }
-    __syncthreads();
-    // the x/z stage is free: prefetch the next tile
-    const int next = s_next;
-    __syncthreads();  // every thread has read s_next
-    if (tid == 0) s_next = (int)next2;
-    TileCoord nc{};
-    if (next < a.n_tiles) nc = coord_of(next, a);
-    if (tid == 0 && next < a.n_tiles) issue_tile_loads<T, kGate>(smem, &bar, maps, a, nc);
-
-    // ---- phase 2 ---------------------------------------------------------------------
-    // sP is not read after phase 1: the threads the look-back leaves idle stage the next
-    // tile's parameters meanwhile
-    if (tid >= CW && tid < 2 * CW && next < a.n_tiles && nc.cblk != tc.cblk)
-      stage_params(sP, CW, nc.cblk, tid - CW, a);
-    if (tid < CW) {
-      const int j = tid;
-      const int c = tc.cblk * CW + j;
-      // exclusive prefixes (held in registers) map the tile's incoming state to the state
-      // entering sub-chunk q
-      float pA[S], pB[S];
-#pragma unroll
-      for (int q = 0; q < S; ++q) { pA[q] = sA[q * CW + j]; pB[q] = sB[q * CW + j]; }
-      float A = 1.0f, Bv = 0.0f;
-#pragma unroll
-      for (int q = 0; q < S; ++q) {
-        const float pa = pA[q], pb = pB[q];
-        pA[q] = A;
-        pB[q] = Bv;
-        Bv = fmaf(pa, Bv, pb);
-        A *= pa;
+  } else if (tid < kComputeThreads + kLookThreads) {
+    // ---- look-back warps: the incoming state of tile k is read while its phase 1 runs;
+    // once phase 1 is done the tile's states are finished and published ----------------
+    const int j = tid - kComputeThreads;
+    for (int k = 0;; ++k) {
+      const int st = k % kStages;
+      if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
+        if (j == 0) atomicOr(a.status, kStatusTimeout);
       }
-      uint64_t* agg = a.carry_agg;
-      uint32_t* incl = a.carry_incl;
-      const bool publish = tc.tix != a.stall_tile;
-      float hin;
-      if (tc.chunk == 0) {
-        hin = (a.h0 != nullptr && c < R) ? a.h0[(int64_t)tc.b * R + c] : 0.0f;
-      } else {
-        if (publish) st_relaxed_u64(agg + tc.tix * CW + j, ((uint64_t)__float_as_uint(Bv) << 32) | enc(A));
-        // Walk back over earlier chunks of the same (b, channel block), composing their
-        // aggregates until an inclusive state is found. (eA, eB) maps the state at the
-        // end of chunk p to the state entering this tile.
-        float eA = 1.0f, eB = 0.0f;
-        int64_t p = tc.tix - 1;                      // nearest not yet composed predecessor
-        const int64_t first = tc.tix - tc.chunk;     // chunk 0 of this (b, channel block)
-        long long t0 = 0;
-        while (true) {
-          // one round trip reads the words of up to four predecessors p, p-1, p-2, p-3
-          constexpr int kH = 4;
-          uint32_t hw[kH];
-          uint64_t aw[kH];
-#pragma unroll
-          for (int k = 0; k < kH; ++k) {
-            const int64_t q = p - k;
-            hw[k] = q >= first ? ld_relaxed_u32(incl + q * CW + j) : 0u;
-            aw[k] = q >= first ? ld_relaxed_u64(agg + q * CW + j) : 0ull;
-          }
-          bool done = false;
-          int used = 0;
-#pragma unroll
-          for (int k = 0; k < kH; ++k) {
-            if (done || used != k || p - k < first) continue;
-            if (hw[k] != 0u) {
-              hin = fmaf(eA, dec(hw[k]), eB);
-              done = true;
-            } else if ((uint32_t)aw[k] != 0u) {  // the low half (A) is encoded; B is stored plainly
-              eB = fmaf(eA, __uint_as_float((uint32_t)(aw[k] >> 32)), eB);
-              eA *= dec((uint32_t)aw[k]);
-              ++used;
-            }
-          }
-          if (done) break;
-          if (used > 0) {
-            p -= used;
-            t0 = 0;
-            continue;
-          }
-          if (t0 == 0) {
-            t0 = clock64();
-          } else if (clock64() - t0 > kWaitCycles) {
-            atomicOr(a.status, kStatusTimeout);
-            hin = eB;
-            break;
-          }
+      const int tile = s_tile[st];
+      float hin[NCH];
+      if (tile < a.n_tiles) lookback_walk<T, kGate, NCH>(coord_of(tile, a), j, a, hin);
+      bar_sync_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
+      if (tile >= a.n_tiles) break;
+      const float* mA = maps_base + (k & 1) * 2 * kSub * CW;
+      lookback_finish<T, kGate, NCH>(mA, maps_base + (k & 1) * 2 * kSub * CW + kSub * CW, coord_of(tile, a), j, a,
+                                     hin);
+      mbar_arrive(&state[k & 1]);
+    }
+  } else {
+    // ---- producer warp: tickets, TMA copies and parameters, two tiles ahead ----------
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.x);
+      tma_prefetch_desc(&maps.z);
+    }
+    // tickets: t_cur for the tile being loaded, t_nxt for the one after (its parameters
+    // are loaded a step early), pend for the one after that (fetched a step early)
+    unsigned t0 = 0, t1 = 0, pend = 0;
+    if (lane == 0) {
+      t0 = atomicAdd(a.ticket, 1u);
+      t1 = atomicAdd(a.ticket, 1u);
+      pend = atomicAdd(a.ticket, 1u);
+    }
+    int t_cur = (int)__shfl_sync(0xffffffffu, t0, 0);
+    int t_nxt = (int)__shfl_sync(0xffffffffu, t1, 0);
+    ParRegs<PV> par;
+    if (t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
+    for (int jt = 0;; ++jt) {
+      const int st = jt % kStages;
+      if (jt >= kStages) {
+        // the stage's previous tile has been replayed by every compute warp
+        if (!mbar_wait_sleep(&empty[st], (uint32_t)(jt / kStages - 1) & 1u)) {
+          if (lane == 0) atomicOr(a.status, kStatusTimeout);
         }
       }
-      const float hout = fmaf(A, hin, Bv);
-      if (publish) st_relaxed_u32(incl + tc.tix * CW + j, enc(hout));
-      if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < R) a.hT[(int64_t)tc.b * R + c] = hout;
-#pragma unroll
-      for (int q = 0; q < S; ++q) sB[q * CW + j] = fmaf(pA[q], hin, pB[q]);
-    }
-    __syncthreads();
-
-    // ---- phase 3: replay from the incoming state, write y ----------------------------
-    if (cvalid) {
-      float h[V];
-#pragma unroll
-      for (int v = 0; v < V; v += 4) {
-        const float4 f = *reinterpret_cast<const float4*>(sB + s * CW + g * V + v);
-        h[v] = f.x; h[v + 1] = f.y; h[v + 2] = f.z; h[v + 3] = f.w;
-      }
-      T* __restrict__ y = static_cast<T*>(a.y);
-#pragma unroll
-      for (int l = 0; l < L; ++l) {
-        const int t = t_start + l;
-        float o[V];
-#pragma unroll
-        for (int v = 0; v < V; v += 2) {
-          float2 at, bt;
-          if constexpr (kAcc) {
-            at = make_float2(ra[l * V + v], ra[l * V + v + 1]);
-            bt = make_float2(rb[l * V + v], rb[l * V + v + 1]);
-          } else {
-            const uint32_t p0 = rp[l * V + v], p1 = rp[l * V + v + 1];
-            at = make_float2(1.0f - bf16lo(p0), 1.0f - bf16lo(p1));
-            bt = make_float2(bf16hi(p0), bf16hi(p1));
-          }
-          const float2 h2 = __ffma2_rn(at, make_float2(h[v], h[v + 1]), bt);
-          h[v] = h2.x;
-          h[v + 1] = h2.y;
-          o[v] = h2.x;
-          o[v + 1] = h2.y;
+      uint8_t* stage = smem + st * Ly::kStage;
+      if (lane == 0) s_tile[st] = t_cur;
+      if (t_cur >= a.n_tiles) {
+        // end of this CTA's tiles: release the stage with no data
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&full[st]);
+          mbar_arrive(&full[st]);
         }
-        if constexpr (kGate) {
-          float gg[V];
-          unpack_row<V>(*reinterpret_cast<const uint4*>(sg + (s * L + l) * CW + g * V), gg);
-#pragma unroll
-          for (int v = 0; v < V; ++v) o[v] *= gelu_exact(gg[v]);
-        }
-        if (t < a.T) __stcs(reinterpret_cast<uint4*>(y + ((int64_t)tc.b * a.T + t) * R + c0), pack_row<V>(o));
+        break;
       }
+      const TileCoord tc = coord_of(t_cur, a);
+      if (lane == 0) issue_tile_loads<T, kGate>(stage, &full[st], maps, a, tc);
+      store_params<PV>(reinterpret_cast<float*>(stage + Ly::offPar), CW, lane * PV, tc.cblk * CW + lane * PV < a.R,
+                       par);
+      // advance the ticket pipeline and start the next tile's parameter loads
+      const int t_new = (int)__shfl_sync(0xffffffffu, pend, 0);
+      if (lane == 0) pend = atomicAdd(a.ticket, 1u);
+      t_cur = t_nxt;
+      t_nxt = t_new;
+      if (t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[st]);
     }
-    __syncthreads();  // sB and (gated) sg are free
-    if (tid == 0 && kGate && next < a.n_tiles) issue_gate_load<T, kGate>(smem, &bar, maps, nc);
-    tile = next;
-    phase ^= 1u;
   }
 }
 
 std::atomic<int64_t> g_stall_tile{-1};
 
+// One CTA per SM: every CTA of the grid is resident at once, which the look-back's
+// forward-progress argument needs.
 template <typename T, bool kGate>
 cudaError_t launch_typed(const ScanArgs& a, const ScanMaps& maps, cudaStream_t s) {
   using Ly = SmemLayout<T, kGate>;
   auto kern = rglru_scan_kernel<T, kGate>;
-  static int occ[64] = {0};
+  static bool ready[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (occ[dev] == 0) {
+  if (!ready[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
     if (e != cudaSuccess) return e;
     int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kScanThreads, Ly::kAlloc);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, Ly::kAlloc);
     if (e != cudaSuccess) return e;
-    occ[dev] = nb > 0 ? nb : 1;
+    if (nb < 1) return cudaErrorInvalidConfiguration;
+    ready[dev] = true;
   }
-  const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)occ[dev] * num_sms());
-  kern<<<(unsigned)grid, kScanThreads, Ly::kAlloc, s>>>(maps, a);
+  const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)num_sms());
+  kern<<<(unsigned)grid, kThreads, Ly::kAlloc, s>>>(maps, a);
   return cudaGetLastError();
 }
 
@@ -551,8 +722,7 @@ ScanLayout scan_layout(int B, int T, int R, bool bf16) {
   L.n_cblk = (R + cw - 1) / cw;
   L.n_chunks = (T + kScanTC - 1) / kScanTC;
   L.n_tiles = (int64_t)B * L.n_cblk * L.n_chunks;
-  L.off_agg = 256;
-  L.off_incl = L.off_agg + (((size_t)L.n_tiles * cw * 8 + 255) / 256) * 256;
+  L.off_incl = 256;
   L.bytes = L.off_incl + (((size_t)L.n_tiles * cw * 4 + 255) / 256) * 256;
   L.zero_bytes = L.bytes;
   return L;

@@ -103,7 +103,6 @@ extern "C" RGLRU_API int rglru_scan_noalloc(const rglru_params* p, const void* x
   a.Lambda = p->Lambda;
   a.status = status;
   a.ticket = reinterpret_cast<unsigned*>(static_cast<unsigned char*>(scratch) + 4);
-  a.carry_agg = reinterpret_cast<uint64_t*>(static_cast<unsigned char*>(scratch) + sl.off_agg);
   a.carry_incl = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(scratch) + sl.off_incl);
   a.B = B;
   a.T = T;
