@@ -47,9 +47,14 @@ FLUSH_BYTES = 256 << 20
 # summarised under profiles/, keyed by the SHA-256 of the kernel's source at capture
 # time. A source change invalidates the figure (reported as null).
 NCU_TRAFFIC = {
-    # profiles/gemm_tc_gates_fwd_hawk_bf16.md
-    "gate_gemm": {"src_sha256": "71b04d951a248c53588e9264d9cda6aa0f633f2d7d220f784dec17aa47354089",
-                  "bytes_per_launch": 83971840 + 89110528},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of each kernel at this
+    # workload (profiles/), valid while the kernel's source is unchanged
+    "gate_gemm": {"src_sha256": "d7dbf16bd529bc883e141b6278dbddd9b1f18c89b0ebda39d786f244548eaba4",
+                  "bytes_per_launch": 84025088 + 89977344},
+    "scan": {"src_sha256": "e36da071126b0bbbdfa1feac4df5ecff81bf162807b9b9fcffaf9b853c78777a",
+             "bytes_per_launch": 202172928 + 44017408},
+    "conv1d": {"src_sha256": "e0aa6f928d1e43413d438851e4d0396b3c3577e6f198861dfe19a40406128ca6",
+               "bytes_per_launch": 67164672 + 18709504},
 }
 
 
