@@ -374,31 +374,44 @@ def _host_cores():
         return os.cpu_count()
 
 
-def _oracle_sample(inputs, rows=1, steps=512):
-    """The oracle on `rows` batch rows × `steps` steps × all channels of the workload."""
-    import torch
+_HOST_WORKLOAD = {}
 
+
+def _host_workload(inputs):
+    """The bench workload's inputs on the host (generated once per process)."""
+    import torch
+    if "w" not in _HOST_WORKLOAD:
+        _HOST_WORKLOAD["w"] = inputs.make_forward(WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["R"], torch.bfloat16, seed=0)
+    return _HOST_WORKLOAD["w"]
+
+
+def _oracle_sample(inputs, row=0, steps=512):
+    """The oracle on batch row `row`, its first `steps` steps, all channels of the workload."""
     import oracle
-    B, T, R = WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["R"]
-    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=0)
+    w = _host_workload(inputs)
     pr = w.params
-    x = w.x[:rows, :steps]
+    x = w.x[row:row + 1, :steps]
     t0 = time.perf_counter()
     oracle.rglru_forward(x, pr.conv_w, pr.conv_b, pr.W_a, pr.b_a, pr.W_x, pr.b_x, pr.Lambda)
     dt = time.perf_counter() - t0
-    return rows * steps, dt
+    return steps, dt
+
+
+CPU_SAMPLE_SECONDS = 10.0
 
 
 def cpu_baseline(inputs):
-    _oracle_sample(inputs, rows=1, steps=512)          # untimed: first touch of host memory
-    tok, dt = 0, 0.0
-    for _ in range(2):
-        t, d = _oracle_sample(inputs, rows=1, steps=2048)
+    _oracle_sample(inputs, row=0, steps=512)          # untimed: first touch of host memory
+    tok, dt, n = 0, 0.0, 0
+    while dt < CPU_SAMPLE_SECONDS:
+        t, d = _oracle_sample(inputs, row=n % WORKLOAD["B"], steps=WORKLOAD["T"])
         tok += t
         dt += d
+        n += 1
     return {"value": tok / dt, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
-            "sample": f"2 x (1 batch row x 2048 steps x 2048 channels) of the workload, {dt:.1f} s; "
-                      "float64 numpy, BLAS matmul on the host cores, recurrence vectorised over channels"}
+            "sample": f"{n} batch rows (cycling over the {WORKLOAD['B']} rows) x {WORKLOAD['T']} steps x "
+                      f"{WORKLOAD['R']} channels of the workload, {dt:.1f} s; float64 numpy, BLAS matmul on the "
+                      "host cores, recurrence vectorised over channels"}
 
 
 def run_reference(args):
@@ -407,11 +420,11 @@ def run_reference(args):
     if rank != 0:
         return
     from gated_linear_rnn_conv1d_b200 import inputs
-    for _ in range(args.warmup):
-        _oracle_sample(inputs)
+    for i in range(args.warmup):
+        _oracle_sample(inputs, row=i % WORKLOAD["B"])
     tot_tok, tot_dt = 0, 0.0
-    for _ in range(args.steps):
-        tok, dt = _oracle_sample(inputs)
+    for i in range(args.steps):
+        tok, dt = _oracle_sample(inputs, row=i % WORKLOAD["B"])
         tot_tok += tok
         tot_dt += dt
     value = tot_tok / tot_dt
