@@ -149,9 +149,15 @@ def run_own(args):
     z = torch.empty(B * T, rglru.gate_pitch(R), dtype=torch.bfloat16, device=dev)
     ws_gs = torch.empty(rglru.gate_scan_workspace_bytes(B, T, R), dtype=torch.uint8, device=dev)
     ws_scan = torch.empty(rglru.scan_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
-    ws_fwd = torch.empty(rglru.forward_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    if args.only == "decode":
+        dec = run_decode(torch, rglru, inputs, dev, stream, flush, _peaks(), barrier, max_over_ranks, world)
+        replicas.shutdown(rk)
+        if rank == 0:
+            print(json.dumps({"only": "decode", "decode": dec}))
+        return
 
     def step(ev=None):
         # exactly the launches rglru_forward makes: conv, gate GEMM, fused scan
@@ -257,33 +263,31 @@ def run_own(args):
         return
 
     # ---- end to end through the public API, host buffers -----------------------------
+    # rglru.forward_host: row groups of the batch pipelined through pinned host copies in
+    # both directions and rglru_forward on three streams (the call a user with host data makes)
     x_host = w.x.pin_memory()
     y_host = torch.empty(B, T, R, dtype=torch.bfloat16).pin_memory()
     h_host = torch.empty(B, R, dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(x)
+    plan = rglru.HostForwardPlan(B, T, R, torch.bfloat16, groups=E2E_GROUPS, slots=3, device=dev)
     e2e_steps = max(3, min(K, 50))
     for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        rglru.forward(p, x_dev, workspace=ws_fwd, y=y, h_T=h_T, want_conv_state=False)
-        y_host.copy_(y, non_blocking=True)
-        h_host.copy_(h_T, non_blocking=True)
+        rglru.forward_host(p, x_host, y_host, h_host, plan, stream=stream)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        rglru.forward(p, x_dev, workspace=ws_fwd, y=y, h_T=h_T, want_conv_state=False)
-        y_host.copy_(y, non_blocking=True)
-        h_host.copy_(h_T, non_blocking=True)
+        rglru.forward_host(p, x_host, y_host, h_host, plan, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
     e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
-           "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2 + h_T.numel() * 4}
-    if rglru.workspace_status(ws_fwd) != 0:
+           "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2 + h_T.numel() * 4,
+           "api": f"rglru.forward_host: {E2E_GROUPS} row groups, host->device copy, rglru_forward and "
+                  "device->host copy of neighbouring groups overlapped on three streams"}
+    if plan.status() != 0:
         status = -7
 
     # ---- decode steps/s ---------------------------------------------------------------
@@ -398,6 +402,7 @@ def _oracle_sample(inputs, row=0, steps=512):
 
 
 CPU_SAMPLE_SECONDS = 10.0
+E2E_GROUPS = 4   # row groups of the batch that forward_host pipelines in the e2e measurement
 
 
 def cpu_baseline(inputs):
@@ -448,8 +453,8 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
-    ap.add_argument("--only", choices=["all", "forward"], default="all",
-                    help="forward: time the forward steps only (small command for profiler captures)")
+    ap.add_argument("--only", choices=["all", "forward", "decode"], default="all",
+                    help="forward / decode: time that part only (small commands for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

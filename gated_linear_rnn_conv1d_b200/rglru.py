@@ -96,6 +96,84 @@ def forward(params: Params, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
     return y, h_T, conv_state_T
 
 
+class HostForwardPlan:
+    """Device buffers and streams for forward_host on inputs of shape [B][T][R].
+
+    The batch is cut into `groups` row groups; `slots` of them are in flight at once, each
+    slot with its own device copy of x, y, h_T and a forward workspace. Made once and reused,
+    so forward_host itself allocates nothing.
+    """
+
+    def __init__(self, B: int, T: int, R: int, dtype: torch.dtype = torch.bfloat16, *, groups: int = 4,
+                 slots: int = 3, device=None):
+        if B % groups:
+            raise ValueError(f"B={B} is not a multiple of groups={groups}")
+        self.B, self.T, self.R, self.dtype, self.groups = B, T, R, dtype, groups
+        self.rows = B // groups
+        self.slots = min(slots, groups)
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        nws = forward_workspace_bytes(self.rows, T, R, dtype)
+        self.x = [torch.empty(self.rows, T, R, dtype=dtype, device=dev) for _ in range(self.slots)]
+        self.y = [torch.empty(self.rows, T, R, dtype=dtype, device=dev) for _ in range(self.slots)]
+        self.h_T = [torch.empty(self.rows, R, dtype=torch.float32, device=dev) for _ in range(self.slots)]
+        self.ws = [torch.empty(max(nws, 256), dtype=torch.uint8, device=dev) for _ in range(self.slots)]
+        self.copy_in = torch.cuda.Stream(dev)
+        self.compute = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.device = dev
+
+    def status(self) -> int:
+        """The first non-zero status word of the slots' workspaces (0: all calls were clean)."""
+        for ws in self.ws:
+            st = workspace_status(ws)
+            if st != 0:
+                return st
+        return 0
+
+
+def forward_host(params: Params, x_host: torch.Tensor, y_host: torch.Tensor, h_T_host: torch.Tensor,
+                 plan: HostForwardPlan, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """rglru_forward on host tensors (pinned for the copies to overlap): x_host [B][T][R] →
+    y_host [B][T][R], h_T_host [B][R] fp32, zero initial state.
+
+    Batch rows are independent, so the plan's row groups are pipelined: the host→device copy
+    of one group, rglru_forward on the next and the device→host copy of a third run on three
+    streams at once. The work is ordered after `stream` (default: the current stream) and
+    `stream` waits for all of it before later work, so events recorded on it time the whole
+    transfer. Results are bit-identical to one rglru_forward over the whole batch.
+    """
+    if x_host.shape != (plan.B, plan.T, plan.R) or x_host.dtype != plan.dtype:
+        raise ValueError("x_host does not match the plan")
+    outer = torch.cuda.current_stream(plan.device) if stream is None else stream
+    start = torch.cuda.Event()
+    start.record(outer)
+    freed = [None] * plan.slots  # event: the slot's last device→host copy has finished
+    for g in range(plan.groups):
+        k = g % plan.slots
+        rows = slice(g * plan.rows, (g + 1) * plan.rows)
+        with torch.cuda.stream(plan.copy_in):
+            plan.copy_in.wait_event(start)
+            if freed[k] is not None:
+                plan.copy_in.wait_event(freed[k])
+            plan.x[k].copy_(x_host[rows], non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(plan.copy_in)
+        plan.compute.wait_event(loaded)
+        forward(params, plan.x[k], workspace=plan.ws[k], y=plan.y[k], h_T=plan.h_T[k], want_conv_state=False,
+                stream=plan.compute)
+        done = torch.cuda.Event()
+        done.record(plan.compute)
+        with torch.cuda.stream(plan.copy_out):
+            plan.copy_out.wait_event(done)
+            y_host[rows].copy_(plan.y[k], non_blocking=True)
+            h_T_host[rows].copy_(plan.h_T[k], non_blocking=True)
+            freed[k] = torch.cuda.Event()
+            freed[k].record(plan.copy_out)
+    for e in freed:
+        if e is not None:
+            outer.wait_event(e)
+
+
 def step_workspace_bytes(B: int, R: int, dtype: torch.dtype = torch.bfloat16) -> int:
     return _abi.load().rglru_step_workspace_bytes(B, R, _DT[dtype])
 
