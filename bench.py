@@ -41,6 +41,7 @@ sys.path.insert(0, ROOT)
 METRIC = "RG-LRU fwd tokens/s and achieved HBM GB/s vs B200 peak; decode steps/s"
 WORKLOAD = dict(B=8, T=2048, R=2048)
 DECODE = dict(B=256, R=4096)
+BLOCK = dict(B=4, T=4096, D=4096, R=5632)
 FLUSH_BYTES = 256 << 20
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
@@ -157,6 +158,12 @@ def run_own(args):
         replicas.shutdown(rk)
         if rank == 0:
             print(json.dumps({"only": "decode", "decode": dec}))
+        return
+    if args.only == "block":
+        blk = run_block(torch, rglru, inputs, dev, stream, flush, _peaks(), max_over_ranks, world, reps=2)
+        replicas.shutdown(rk)
+        if rank == 0:
+            print(json.dumps({"only": "block", "block": blk}))
         return
 
     def step(ev=None):
@@ -293,6 +300,9 @@ def run_own(args):
     # ---- decode steps/s ---------------------------------------------------------------
     dec = run_decode(torch, rglru, inputs, dev, stream, flush, pk, barrier, max_over_ranks, world)
 
+    # ---- recurrent block ------------------------------------------------------------------
+    blk = run_block(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world)
+
     replicas.shutdown(rk)
     if rank != 0:
         return
@@ -310,6 +320,7 @@ def run_own(args):
         "hbm_gb_per_s": {"scan": kern["scan"]["GB/s"], "conv1d": kern["conv1d"]["GB/s"],
                          "peak": pk["hbm_gbs"], "peak_source": pk["source"]},
         "decode": dec,
+        "block": blk,
         "e2e": e2e,
         "gpu_launches": 3 * K,
         "clocks": clk,
@@ -368,6 +379,40 @@ def run_decode(torch, rglru, inputs, dev, stream, flush, pk, barrier, max_over_r
             "frac_hbm_l2_flushed": step_bytes / cold_ms / 1e6 / pk["hbm_gbs"],
             "gpu_launches_per_step": 2,
             "timing": "CUDA graph of 48 steps replayed 8x (L2-warm); and 24 single steps with L2 flushed"}
+
+
+def run_block(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world, reps=5):
+    """The recurrent block (two input linears, conv, gates, scan with the GeLU branch, output
+    linear) as one rglru_block_forward call, L2 flushed before each timed call."""
+    B, T, D, R = BLOCK["B"], BLOCK["T"], BLOCK["D"], BLOCK["R"]
+    w = inputs.make_block(B, T, D, R, torch.bfloat16, seed=0)
+    p = rglru.Params.from_host(w.params, dev)
+    W_1, W_2, W_o = w.W_1.to(dev), w.W_2.to(dev), w.W_o.to(dev)
+    x = w.x.to(dev)
+    out = torch.empty_like(x)
+    h_T = torch.empty(B, R, dtype=torch.float32, device=dev)
+    ws = torch.empty(rglru.block_workspace_bytes(B, T, D, R), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        rglru.block_forward(p, W_1, W_2, W_o, x, workspace=ws, out=out, h_T=h_T)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        rglru.block_forward(p, W_1, W_2, W_o, x, workspace=ws, out=out, h_T=h_T)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / reps)
+    n_tok = B * T
+    flops = 2.0 * n_tok * (2 * D * R + 2 * R * R + R * D)
+    peak = pk["bf16_tflops_sustained"] or pk["bf16_tflops"]
+    status = rglru.workspace_status(ws)
+    del ws, out, x, W_1, W_2, W_o
+    return {"workload": f"recurrent block B={B} T={T} D={D} D_RNN={R} bf16", "ms_per_call": ms,
+            "tokens_per_s": world * n_tok / (ms / 1e3), "flops_per_call": flops, "TFLOP/s": flops / ms / 1e9,
+            "peak_TFLOP/s": peak, "frac_tensor": flops / ms / 1e9 / peak,
+            "peak_source": "measured sustained bf16 (a multi-ms call)", "status": status,
+            "gpu_launches_per_call": 6, "timing": f"{reps} calls, L2 flushed before each"}
 
 
 # ------------------------------------------------------------------------------ CPU side
@@ -453,8 +498,8 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
-    ap.add_argument("--only", choices=["all", "forward", "decode"], default="all",
-                    help="forward / decode: time that part only (small commands for profiler captures)")
+    ap.add_argument("--only", choices=["all", "forward", "decode", "block"], default="all",
+                    help="forward / decode / block: time that part only (small commands for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
