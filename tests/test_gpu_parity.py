@@ -274,8 +274,11 @@ def test_decode_checkpoint_resume_is_bitwise():
     assert torch.equal(h, h2) and torch.equal(ring, ring2)
 
 
-def test_decode_small_matches_oracle_every_step():
-    B, R, steps = 130, 200, 9
+# (130, 200): the 1-SM step kernel (R not a multiple of 128); the others run the transposed
+# split-K kernel, with a ragged batch (5), one batch half (128) and both halves (130, 256)
+@pytest.mark.parametrize("B,R", [(130, 200), (5, 256), (128, 384), (130, 256), (256, 128)])
+def test_decode_small_matches_oracle_every_step(B, R):
+    steps = 9
     w = inputs.make_decode(B, R, torch.bfloat16, seed=2)
     p = rglru.Params.from_host(w.params)
     hp = host_params64(w.params)
