@@ -778,6 +778,259 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Decode step GEMM, transposed and split over K inside a 4-CTA cluster.
+// "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元 (RG-LRU),
+// Eq. (1)–(4), one token: z = u_t · [W_a | W_x]ᵀ + b, then h ← a_t h + √(1−a_t²) i u_t, y = h.
+// The weights are the large operand, so they are the MMA's M side and every weight row is
+// read once per step. A cluster owns 128 channels. It holds two CTA pairs (cluster ranks
+// 0–1 and 2–3), one per half of K; each pair runs 2-SM MMAs (cta_group::2, M = 256,
+// N = 256): each CTA of a pair stages 64 rows of W_a and the same 64 rows of W_x, and 128 of
+// the 256 batch rows. The two K halves then meet in shared memory: each CTA writes the
+// partial sums of the batch half it does not own into its K-partner's shared memory
+// (distributed shared memory, between two cluster barriers), adds the partner's, and
+// applies the state update to its 64 channels × 128 batch rows with all its warps.
+struct StepArgs {
+  const float* b_a;
+  const float* b_x;
+  const float* u;        // u_t [B][R] float32
+  float* h;              // [B][R], in place
+  __nv_bfloat16* y;      // [B][R]
+  const float* cla;      // [R]
+  int B, R;
+};
+constexpr int kStepStages = 6;
+constexpr int kStepABytes = 128 * BK * 2;  // 64 rows of W_a + the same 64 rows of W_x
+constexpr int kStepBBytes = 128 * BK * 2;  // this CTA's 128 batch rows of u_t
+constexpr int kStepStageBytes = kStepABytes + kStepBBytes;
+constexpr int kStepSmem = kStepStages * kStepStageBytes + 1024;
+constexpr int kStepTmemCols = 256;
+constexpr int kStepHalf = 128 * 128;  // floats: 128 accumulator rows × 128 batch columns
+// warps: 0 TMA, 1 MMA, 2–9 TMEM readers (warp w reads lane quarter w % 4, column half
+// (w − 2) / 4), all twelve for the state update
+constexpr int kStepThreads = 384;
+static_assert(2 * kStepHalf * 4 <= kStepStages * kStepStageBytes, "z staging and the partner's half fit the ring");
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "h"(mask)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kStepThreads, 1)
+    step_kernel(const __grid_constant__ CUtensorMap tmWa, const __grid_constant__ CUtensorMap tmWx,
+                const __grid_constant__ CUtensorMap tmU, StepArgs ep, unsigned* status) {
+  constexpr int S = kStepStages;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[S];
+  __shared__ __align__(8) uint64_t empty_bar[S];
+  __shared__ __align__(8) uint64_t tfull_bar;
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t crank = cluster_ctarank();  // 0..3
+  const uint32_t rank = crank & 1u;          // rank inside the CTA pair
+  const uint32_t pair_leader = crank & 2u;   // cluster rank of this pair's leader
+  const bool leader = rank == 0;
+  const int kh = (int)(crank >> 1);          // K half, and the batch half this CTA updates
+  const uint16_t pair_mask = (uint16_t)(0x3u << pair_leader);
+  const int cblk = blockIdx.x / 4;           // 128-channel block
+  const int Kh = ep.R / 2;
+  const int k0 = kh * Kh;
+  const int k_blocks = Kh / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    mbar_init(&tfull_bar, 1);
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmWa);
+    tma_prefetch_desc(&tmWx);
+    tma_prefetch_desc(&tmU);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_s)),
+                 "r"(kStepTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // every CTA's barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_s;
+  const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), pair_leader);
+
+  if (warp == 0) {
+    // ---------------- TMA producer (every CTA) ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const int wrow = cblk * 128 + (int)rank * 64;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_s)) { ok = false; break; }
+        uint8_t* sa = smem + stage * kStepStageBytes;
+        uint8_t* sb = sa + kStepABytes;
+        const uint32_t lbar = leader_full0 + stage * 8;
+        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStepStageBytes);
+        const int kc = k0 + kb * BK;
+        tma_load_2d_2sm(sa, &tmWa, lbar, kc, wrow);
+        tma_load_2d_2sm(sa + 64 * BK * 2, &tmWx, lbar, kc, wrow);
+        tma_load_2d_2sm(sb, &tmU, lbar, kc, (int)rank * 128);
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) { abort_s = 1; atomicOr(status, kStatusTimeout); }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (pair leaders only) ----------------
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, &abort_s)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + stage * kStepStageBytes);
+        const uint32_t b_addr = a_addr + kStepABytes;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_f16_2sm(tmem_base, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), k2Idesc,
+                       (kb | k) != 0 ? 1u : 0u);
+        umma_commit_pair(&empty_bar[stage], pair_mask);
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+      if (ok) umma_commit_pair(&tfull_bar, pair_mask);
+      if (!ok) { abort_s = 1; atomicOr(status, kStatusTimeout); }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(&drain_bar))
+                   : "memory");
+      volatile int never = 0;
+      (void)mbar_wait(&drain_bar, 0, &never);
+    }
+  }
+
+  // ---------------- K-half exchange and state update (every CTA, every warp) ----------------
+  const int q = warp & 3;          // TMEM lanes 32q … 32q+31
+  const int row = q * 32 + lane;   // accumulator row: W_a row (row < 64) or W_x row
+  const bool epi = warp >= 2 && warp < 10;  // TMEM readers
+  const int chalf = (warp - 2) / 4;         // which 64 of a 128-column half this warp moves
+  const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+  constexpr int kRecvPitch = 132;  // floats per received row (keeps 16-byte reads conflict-free)
+  float* zs = reinterpret_cast<float*>(smem);                       // [128 batch cols][128 rows]
+  float* recv = reinterpret_cast<float*>(smem + kStepHalf * 4);     // [128 rows][kRecvPitch]
+  static_assert(kStepHalf * 4 + 128 * kRecvPitch * 4 <= kStepStages * kStepStageBytes, "exchange buffers");
+  if (epi) {
+    if (!mbar_wait(&tfull_bar, 0, &abort_s)) {
+      abort_s = 1;
+      atomicOr(status, kStatusTimeout);
+    }
+    tc_fence_after();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // every MMA of the cluster is done: all rings are free
+  tc_fence_after();
+  if (epi) {
+    // the partial sums of the batch half the K-partner updates, into its shared memory
+    const uint32_t dst = mapa_rank(smem_u32(recv + row * kRecvPitch), crank ^ 2u);
+    const int other = 1 - kh;
+#pragma unroll 1
+    for (int cc = 2 * chalf; cc < 2 * chalf + 2; ++cc) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + other * 128 + cc * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        st_cluster_v4(dst + (uint32_t)((cc * 32 + j) * 4),
+                      make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                  __uint_as_float(r[j + 3])));
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // the partners' sums are in place
+  tc_fence_after();
+  if (epi) {
+    // full sums of this CTA's batch half, staged as zs[batch column][accumulator row]
+    const float* in = recv + row * kRecvPitch;
+#pragma unroll 1
+    for (int cc = 2 * chalf; cc < 2 * chalf + 2; ++cc) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + kh * 128 + cc * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 p = *reinterpret_cast<const float4*>(in + cc * 32 + j);
+        zs[(cc * 32 + j + 0) * 128 + row] = __uint_as_float(r[j + 0]) + p.x;
+        zs[(cc * 32 + j + 1) * 128 + row] = __uint_as_float(r[j + 1]) + p.y;
+        zs[(cc * 32 + j + 2) * 128 + row] = __uint_as_float(r[j + 2]) + p.z;
+        zs[(cc * 32 + j + 3) * 128 + row] = __uint_as_float(r[j + 3]) + p.w;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  {
+    // h ← a_t h + √(1−a_t²) i u_t and y = h for 64 channels × 128 batch rows, by all twelve
+    // warps, in two groups of kG batch rows whose u and h loads are all issued before any of
+    // the group's stores
+    const int t = threadIdx.x;
+    const int j = t % 64;
+    const int ch = cblk * 128 + (int)rank * 64 + j;
+    const float ba = __ldg(ep.b_a + ch), bx = __ldg(ep.b_x + ch), cl = __ldg(ep.cla + ch);
+    constexpr int kPhases = kStepThreads / 64;  // batch columns interleaved over 6 thread groups
+    constexpr int kG = (128 + 2 * kPhases - 1) / (2 * kPhases);  // two groups per thread
+#pragma unroll 1
+    for (int c0 = t / 64; c0 < 128; c0 += kPhases * kG) {
+      float uv[kG], hv[kG];
+#pragma unroll
+      for (int i = 0; i < kG; ++i) {
+        const int c = c0 + kPhases * i;
+        const int b = kh * 128 + c;
+        const int64_t idx = (int64_t)b * ep.R + ch;
+        uv[i] = (c < 128 && b < ep.B) ? __ldg(ep.u + idx) : 0.0f;
+        hv[i] = (c < 128 && b < ep.B) ? ep.h[idx] : 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < kG; ++i) {
+        const int c = c0 + kPhases * i;
+        const int b = kh * 128 + c;
+        if (c < 128 && b < ep.B) {
+          const int64_t idx = (int64_t)b * ep.R + ch;
+          float at, bt;
+          gate_fast(zs[c * 128 + j] + ba, zs[c * 128 + 64 + j] + bx, cl, uv[i], at, bt);
+          const float hn = fmaf(at, hv[i], bt);
+          ep.h[idx] = hn;
+          ep.y[idx] = __float2bfloat16_rn(hn);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kStepTmemCols)
+                 : "memory");
+  }
+}
+
 template <int EPI, bool DUAL>
 cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1, int64_t M, int K,
                        int n_tiles_n, const EpiArgs& ep, unsigned* status, cudaStream_t s) {
@@ -943,9 +1196,68 @@ cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, 
   return launch_tc2<EPI_STORE, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
 }
 
+namespace {
+// Whether the cluster step kernel covers (B, R) on the current device.
+bool step_cluster_usable(int B, int R) {
+  if (B > 256 || R % 128 != 0) return false;
+  static int ok[64] = {0};  // 0 unknown, 1 usable, -1 not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (ok[dev] == 0) {
+    ok[dev] = -1;
+    if (cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem) == cudaSuccess &&
+        cudaFuncSetAttribute(step_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(4);
+      cfg.blockDim = dim3(kStepThreads);
+      cfg.dynamicSmemBytes = kStepSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 4;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, step_kernel, &cfg) == cudaSuccess && n >= 1) ok[dev] = 1;
+    }
+    (void)cudaGetLastError();
+  }
+  return ok[dev] == 1;
+}
+}  // namespace
+
 cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,
                                   const void* Wx, const float* bx, const float* cla, float* h, void* y_t, int B,
                                   int R, unsigned* status, cudaStream_t s) {
+  if (step_cluster_usable(B, R)) {
+    CUtensorMap mwa, mwx, mu;
+    if (!make_map_2d(&mwa, Wa, R, R, (uint64_t)R * 2, BK, 64)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&mwx, Wx, R, R, (uint64_t)R * 2, BK, 64)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&mu, u_t, R, B, (uint64_t)R * 2, BK, 128)) return cudaErrorInvalidValue;
+    StepArgs ep{};
+    ep.b_a = ba;
+    ep.b_x = bx;
+    ep.u = u_f32;
+    ep.h = h;
+    ep.y = static_cast<__nv_bfloat16*>(y_t);
+    ep.cla = cla;
+    ep.B = B;
+    ep.R = R;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(4 * (R / 128));
+    cfg.blockDim = dim3(kStepThreads);
+    cfg.dynamicSmemBytes = kStepSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 4;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, step_kernel, mwa, mwx, mu, ep, status);
+  }
   constexpr int BN = 128;
   CUtensorMap ma, mb0, mb1;
   if (!make_map_2d(&ma, u_t, R, B, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
