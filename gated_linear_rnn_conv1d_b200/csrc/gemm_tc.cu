@@ -803,17 +803,30 @@ constexpr int kStepStages = 6;
 constexpr int kStepABytes = 128 * BK * 2;  // 64 rows of W_a + the same 64 rows of W_x
 constexpr int kStepBBytes = 128 * BK * 2;  // this CTA's 128 batch rows of u_t
 constexpr int kStepStageBytes = kStepABytes + kStepBBytes;
-constexpr int kStepSmem = kStepStages * kStepStageBytes + 1024;
+constexpr int kStepRecvPitch = 132;  // floats per exchanged row (keeps 16-byte reads conflict-free)
+constexpr int kStepXBytes = 128 * kStepRecvPitch * 4;  // one exchanged half: 128 rows
+// after the mainloop: zs [0, 64 KB), the half received [64 KB, +kStepXBytes), the half sent after it
+constexpr int kStepSmem = 65536 + 2 * kStepXBytes + 1024;
 constexpr int kStepTmemCols = 256;
 constexpr int kStepHalf = 128 * 128;  // floats: 128 accumulator rows × 128 batch columns
 // warps: 0 TMA, 1 MMA, 2–9 TMEM readers (warp w reads lane quarter w % 4, column half
 // (w − 2) / 4), all twelve for the state update
 constexpr int kStepThreads = 384;
-static_assert(2 * kStepHalf * 4 <= kStepStages * kStepStageBytes, "z staging and the partner's half fit the ring");
+static_assert(kStepStages * kStepStageBytes + 1024 <= kStepSmem, "the ring fits");
+static_assert(kStepSmem <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float4 v) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z),
                "f"(v.w)
+               : "memory");
+}
+// Bulk copy of `bytes` from this CTA's shared memory to another CTA's (cluster addresses for
+// the destination and its mbarrier), completing on that mbarrier.
+__device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst_cluster, const void* src, uint32_t bytes,
+                                                 uint32_t mbar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(smem_u32(src)), "r"(bytes), "r"(mbar_cluster)
                : "memory");
 }
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
@@ -832,6 +845,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   __shared__ __align__(8) uint64_t empty_bar[S];
   __shared__ __align__(8) uint64_t tfull_bar;
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t xbar;  // the K-partner's half has landed
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
 
@@ -856,8 +870,10 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     }
     mbar_init(&tfull_bar, 1);
     mbar_init(&drain_bar, 1);
+    mbar_init(&xbar, 1);
     abort_s = 0;
     fence_barrier_init();
+    mbar_arrive_expect_tx(&xbar, kStepXBytes);
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmWa);
@@ -875,6 +891,24 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
   const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), pair_leader);
+
+  // The state update's inputs do not depend on the GEMM: every thread loads its u_t and h
+  // values now and holds them in registers through the mainloop. Thread t updates channel
+  // j = t % 64 of this CTA's 64 and the batch columns c = t / 64 + kPhases·i of its half.
+  constexpr int kPhases = kStepThreads / 64;
+  constexpr int kPer = (128 + kPhases - 1) / kPhases;
+  const int uj = threadIdx.x % 64;
+  const int uch = cblk * 128 + (int)rank * 64 + uj;
+  float uv[kPer], hv[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int c = (int)threadIdx.x / 64 + kPhases * i;
+    const int b = kh * 128 + c;
+    const int64_t idx = (int64_t)b * ep.R + uch;
+    const bool ok = c < 128 && b < ep.B;
+    uv[i] = ok ? __ldg(ep.u + idx) : 0.0f;
+    hv[i] = ok ? ep.h[idx] : 0.0f;
+  }
 
   if (warp == 0) {
     // ---------------- TMA producer (every CTA) ----------------
@@ -931,24 +965,19 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const bool epi = warp >= 2 && warp < 10;  // TMEM readers
   const int chalf = (warp - 2) / 4;         // which 64 of a 128-column half this warp moves
   const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
-  constexpr int kRecvPitch = 132;  // floats per received row (keeps 16-byte reads conflict-free)
-  float* zs = reinterpret_cast<float*>(smem);                       // [128 batch cols][128 rows]
-  float* recv = reinterpret_cast<float*>(smem + kStepHalf * 4);     // [128 rows][kRecvPitch]
-  static_assert(kStepHalf * 4 + 128 * kRecvPitch * 4 <= kStepStages * kStepStageBytes, "exchange buffers");
+  constexpr int kRecvPitch = kStepRecvPitch;
+  float* zs = reinterpret_cast<float*>(smem);                                    // [128 batch cols][128 rows]
+  float* recv = reinterpret_cast<float*>(smem + kStepHalf * 4);                  // [128 rows][kRecvPitch]
+  float* sendb = reinterpret_cast<float*>(smem + kStepHalf * 4 + kStepXBytes);   // [128 rows][kRecvPitch]
   if (epi) {
     if (!mbar_wait(&tfull_bar, 0, &abort_s)) {
       abort_s = 1;
       atomicOr(status, kStatusTimeout);
     }
     tc_fence_after();
-  }
-  tc_fence_before();
-  cluster_sync_all();  // every MMA of the cluster is done: all rings are free
-  tc_fence_after();
-  if (epi) {
-    // the partial sums of the batch half the K-partner updates, into its shared memory
-    const uint32_t dst = mapa_rank(smem_u32(recv + row * kRecvPitch), crank ^ 2u);
+    // the partial sums of the batch half the K-partner updates, staged for the copy
     const int other = 1 - kh;
+    float* out = sendb + row * kRecvPitch;
 #pragma unroll 1
     for (int cc = 2 * chalf; cc < 2 * chalf + 2; ++cc) {
       uint32_t r[32];
@@ -956,15 +985,26 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       tmem_ld_wait();
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
-        st_cluster_v4(dst + (uint32_t)((cc * 32 + j) * 4),
-                      make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                  __uint_as_float(r[j + 3])));
+        *reinterpret_cast<float4*>(out + cc * 32 + j) =
+            make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                        __uint_as_float(r[j + 3]));
     }
+    fence_proxy_async_smem();  // the staged half is read by the bulk copy
   }
   tc_fence_before();
-  cluster_sync_all();  // the partners' sums are in place
+  cluster_sync_all();  // every MMA of the cluster is done (the rings are free) and the halves are staged
   tc_fence_after();
+  if (threadIdx.x == 0) {
+    // one bulk copy into the K-partner's receive buffer, completing on its mbarrier
+    const uint32_t partner = crank ^ 2u;
+    bulk_copy_to_cta(mapa_rank(smem_u32(recv), partner), sendb, kStepXBytes, mapa_rank(smem_u32(&xbar), partner));
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  }
   if (epi) {
+    if (!mbar_wait(&xbar, 0, &abort_s)) {
+      abort_s = 1;
+      atomicOr(status, kStatusTimeout);
+    }
     // full sums of this CTA's batch half, staged as zs[batch column][accumulator row]
     const float* in = recv + row * kRecvPitch;
 #pragma unroll 1
@@ -986,41 +1026,24 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   __syncthreads();
   {
     // h ← a_t h + √(1−a_t²) i u_t and y = h for 64 channels × 128 batch rows, by all twelve
-    // warps, in two groups of kG batch rows whose u and h loads are all issued before any of
-    // the group's stores
-    const int t = threadIdx.x;
-    const int j = t % 64;
-    const int ch = cblk * 128 + (int)rank * 64 + j;
-    const float ba = __ldg(ep.b_a + ch), bx = __ldg(ep.b_x + ch), cl = __ldg(ep.cla + ch);
-    constexpr int kPhases = kStepThreads / 64;  // batch columns interleaved over 6 thread groups
-    constexpr int kG = (128 + 2 * kPhases - 1) / (2 * kPhases);  // two groups per thread
-#pragma unroll 1
-    for (int c0 = t / 64; c0 < 128; c0 += kPhases * kG) {
-      float uv[kG], hv[kG];
+    // warps, from the u_t and h values loaded at the start
+    const float ba = __ldg(ep.b_a + uch), bx = __ldg(ep.b_x + uch), cl = __ldg(ep.cla + uch);
 #pragma unroll
-      for (int i = 0; i < kG; ++i) {
-        const int c = c0 + kPhases * i;
-        const int b = kh * 128 + c;
-        const int64_t idx = (int64_t)b * ep.R + ch;
-        uv[i] = (c < 128 && b < ep.B) ? __ldg(ep.u + idx) : 0.0f;
-        hv[i] = (c < 128 && b < ep.B) ? ep.h[idx] : 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < kG; ++i) {
-        const int c = c0 + kPhases * i;
-        const int b = kh * 128 + c;
-        if (c < 128 && b < ep.B) {
-          const int64_t idx = (int64_t)b * ep.R + ch;
-          float at, bt;
-          gate_fast(zs[c * 128 + j] + ba, zs[c * 128 + 64 + j] + bx, cl, uv[i], at, bt);
-          const float hn = fmaf(at, hv[i], bt);
-          ep.h[idx] = hn;
-          ep.y[idx] = __float2bfloat16_rn(hn);
-        }
+    for (int i = 0; i < kPer; ++i) {
+      const int c = (int)threadIdx.x / 64 + kPhases * i;
+      const int b = kh * 128 + c;
+      if (c < 128 && b < ep.B) {
+        const int64_t idx = (int64_t)b * ep.R + uch;
+        float at, bt;
+        gate_fast(zs[c * 128 + uj] + ba, zs[c * 128 + 64 + uj] + bx, cl, uv[i], at, bt);
+        const float hn = fmaf(at, hv[i], bt);
+        ep.h[idx] = hn;
+        ep.y[idx] = __float2bfloat16_rn(hn);
       }
     }
   }
 
+  if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();
