@@ -198,6 +198,8 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
                                                                   float* __restrict__ cla, unsigned* status, int B,
                                                                   int R) {
   constexpr int V = 8;
+  // the step GEMM that follows may start its prologue now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int c0 = (blockIdx.x * kConvThreads + threadIdx.x) * V;
   const int b = blockIdx.y;
   if (blockIdx.x == 0 && b == 0 && threadIdx.x == 0) *status = 0u;

@@ -891,6 +891,9 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
   const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), pair_leader);
+  // launched as a programmatic dependent of the decode conv kernel: everything above
+  // overlapped it; u_t, u_t in float32 and c·log σ(Λ) are its results
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // The state update's inputs do not depend on the GEMM: every thread loads its u_t and h
   // values now and holds them in registers through the mainloop. Thread t updates channel
@@ -1272,13 +1275,15 @@ cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const voi
     cfg.blockDim = dim3(kStepThreads);
     cfg.dynamicSmemBytes = kStepSmem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 4;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the decode conv's tail
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, step_kernel, mwa, mwx, mu, ep, status);
   }
   constexpr int BN = 128;
