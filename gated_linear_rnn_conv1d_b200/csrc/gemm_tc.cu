@@ -415,7 +415,11 @@ __device__ __forceinline__ void st_relaxed_u64g(uint64_t* p, uint64_t v) {
 }
 // Published carries are stored as their bit pattern XOR 0x7FFFFFFF: exact and reversible,
 // and zero only for one NaN pattern, so zeroed memory reads as "not published yet".
-__device__ __forceinline__ uint32_t enc_carry(float v) { return __float_as_uint(v) ^ 0x7FFFFFFFu; }
+// (the NaN pattern 0x7FFFFFFF, whose image would be zero, is stored as another NaN's image)
+__device__ __forceinline__ uint32_t enc_carry(float v) {
+  const uint32_t w = __float_as_uint(v) ^ 0x7FFFFFFFu;
+  return w != 0u ? w : 1u;
+}
 __device__ __forceinline__ float dec_carry(uint32_t w) { return __uint_as_float(w ^ 0x7FFFFFFFu); }
 
 template <int EPI, bool DUAL>

@@ -120,11 +120,15 @@ __device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Published carries are stored as their bit pattern XOR 0x7FFFFFFF: an exact, reversible
-// encoding whose only zero is the image of one NaN pattern, so zeroed memory reads as
-// "not published yet" and every finite value round-trips bit for bit.
+// Published carries are stored as their bit pattern XOR 0x7FFFFFFF: exact and reversible
+// for every value but the NaN pattern 0x7FFFFFFF, whose image would be zero; that one is
+// stored as the image of another NaN, so zeroed memory reads as "not published yet", no
+// published word is zero, and every non-NaN value round-trips bit for bit.
 constexpr uint32_t kCarryKey = 0x7FFFFFFFu;
-__device__ __forceinline__ uint32_t enc(float v) { return __float_as_uint(v) ^ kCarryKey; }
+__device__ __forceinline__ uint32_t enc(float v) {
+  const uint32_t w = __float_as_uint(v) ^ kCarryKey;
+  return w != 0u ? w : 1u;
+}
 __device__ __forceinline__ float dec(uint32_t w) { return __uint_as_float(w ^ kCarryKey); }
 
 struct TileCoord {
@@ -491,10 +495,14 @@ __device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const 
     }
     return;
   }
+  // channels past R (the padding of the last channel block) carry nothing: they neither
+  // wait for nor publish a state, so whatever their padding inputs hold cannot stall a tile
   const uint32_t* src = a.carry_incl + (tc.tix - 1) * CW + j;
+  const uint32_t kNothing = enc(0.0f);
   uint32_t w[NCH];
 #pragma unroll
-  for (int n = 0; n < NCH; ++n) w[n] = ld_relaxed_u32(src + n * kStride);
+  for (int n = 0; n < NCH; ++n)
+    w[n] = tc.cblk * CW + j + n * kStride < a.R ? ld_relaxed_u32(src + n * kStride) : kNothing;
   bool ready = true;
 #pragma unroll
   for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
@@ -503,7 +511,7 @@ __device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const 
     while (true) {
 #pragma unroll
       for (int n = 0; n < NCH; ++n)
-        if (w[n] == 0u) w[n] = ld_relaxed_u32(src + n * kStride);
+        if (w[n] == 0u) w[n] = ld_relaxed_u32(src + n * kStride);  // only channels < R can be 0
       ready = true;
 #pragma unroll
       for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
@@ -540,7 +548,7 @@ __device__ __forceinline__ void lookback_finish(const float* mA, float* mB, cons
       mB[q * CW + jj] = h;
       h = fmaf(pa, h, pb);
     }
-    if (publish) st_relaxed_u32(a.carry_incl + tc.tix * CW + jj, enc(h));
+    if (publish && c < a.R) st_relaxed_u32(a.carry_incl + tc.tix * CW + jj, enc(h));
     if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < a.R) a.hT[(int64_t)tc.b * a.R + c] = h;
   }
 }

@@ -198,6 +198,37 @@ def test_batch_rows_are_independent():
     assert torch.equal(z[T:2 * T], z1)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_nan_in_gate_padding_neither_stalls_nor_leaks(dtype):
+    """The packed pre-activations of channels past R are padding: filled with the canonical
+    NaN (whose carry encoding would otherwise read as "not published"), they must neither
+    stall the chunk chain — a stall costs a full bounded wait and a timeout status — nor
+    change any output."""
+    import time
+    B, T, R = 2, 200, 136
+    w = _wl(B, T, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    u = rglru.conv1d(p, x)
+    z = rglru.gate_proj(p, u.view(B * T, R))
+    y_ref, h_ref = rglru.scan(p, x, z)
+    n_pad = 128 * ((R + 127) // 128)
+    cols = [256 * (c // 128) + (c % 128) + off for c in range(R, n_pad) for off in (0, 128)]
+    nan_bits = torch.tensor([0x7FFFFFFF], dtype=torch.int32).view(torch.float32) if dtype == torch.float32 \
+        else torch.tensor([0x7FFF], dtype=torch.int16).view(torch.bfloat16)
+    zp = z.clone()
+    zp[:, cols] = nan_bits.to(DEV)
+    ws = torch.zeros(rglru.scan_workspace_bytes(B, T, R, dtype), dtype=torch.uint8, device=DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    y, h = rglru.scan(p, x, zp, workspace=ws)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert rglru.workspace_status(ws) == 0
+    assert dt < 0.5
+    assert torch.equal(y, y_ref) and torch.equal(h, h_ref)
+
+
 def test_forward_host_equals_forward():
     """forward_host pipelines row groups through host copies on three streams; the result is
     bit-identical to one rglru_forward over the whole batch, on every call."""
