@@ -47,16 +47,6 @@ template <> struct CV<float> {
   }
 };
 
-__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-  const uint2 r = *reinterpret_cast<const uint2*>(p);
-  return make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
-}
-__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ void store4(__nv_bfloat16* p, const float4& v) {
-  __stcg(reinterpret_cast<uint2*>(p), make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w)));
-}
-__device__ __forceinline__ void store4(float* p, const float4& v) { __stcg(reinterpret_cast<float4*>(p), v); }
-
 // Prefill: persistent CTAs stream tiles of one batch row × CW channels (16 bytes per
 // thread × 16 threads) × 64 steps through a ring of kConvStages shared-memory stages. One
 // thread keeps kConvStages TMA copies in flight (each brings the tile's 67 x rows, the
@@ -188,6 +178,14 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const __grid_
   }
 }
 
+// 8 consecutive floats (16-byte aligned) through the read-only path
+__device__ __forceinline__ void ld8(const float* p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
 __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* __restrict__ conv_w,
                                                                   const float* __restrict__ conv_b,
                                                                   const float* __restrict__ Lambda,
@@ -212,13 +210,21 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
   CV<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(rb + (int64_t)s1 * R), xm2);
   CV<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(rb + (int64_t)s2 * R), xm1);
   CV<__nv_bfloat16>::unpack(raw_c, xc);
+  // taps and bias of the thread's 8 channels as 16-byte loads (parameters are 16-byte
+  // aligned, c0 a multiple of 8 and R of 8)
+  float w0[V], w1[V], w2[V], w3[V], cb[V];
+  ld8(conv_w + c0, w0);
+  ld8(conv_w + R + c0, w1);
+  ld8(conv_w + 2 * R + c0, w2);
+  ld8(conv_w + 3 * R + c0, w3);
+  ld8(conv_b + c0, cb);
 #pragma unroll
   for (int v = 0; v < V; ++v) {
-    float acc = __ldg(conv_b + c0 + v);
-    acc = fmaf(__ldg(conv_w + c0 + v), xo[v], acc);
-    acc = fmaf(__ldg(conv_w + R + c0 + v), xm2[v], acc);
-    acc = fmaf(__ldg(conv_w + 2 * R + c0 + v), xm1[v], acc);
-    acc = fmaf(__ldg(conv_w + 3 * R + c0 + v), xc[v], acc);
+    float acc = cb[v];
+    acc = fmaf(w0[v], xo[v], acc);
+    acc = fmaf(w1[v], xm2[v], acc);
+    acc = fmaf(w2[v], xm1[v], acc);
+    acc = fmaf(w3[v], xc[v], acc);
     o[v] = acc;
   }
   *reinterpret_cast<uint4*>(u_t + (int64_t)b * R + c0) = CV<__nv_bfloat16>::pack(o);
@@ -227,8 +233,13 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
   uf[1] = make_float4(o[4], o[5], o[6], o[7]);
   *reinterpret_cast<uint4*>(rb + (int64_t)s0 * R) = raw_c;
   if (b == 0) {
+    float lam[V];
+    ld8(Lambda + c0, lam);
 #pragma unroll
-    for (int v = 0; v < V; ++v) cla[c0 + v] = decay_log_coeff(__ldg(Lambda + c0 + v));
+    for (int v = 0; v < V; ++v) lam[v] = decay_log_coeff(lam[v]);
+    float4* cp = reinterpret_cast<float4*>(cla + c0);
+    cp[0] = make_float4(lam[0], lam[1], lam[2], lam[3]);
+    cp[1] = make_float4(lam[4], lam[5], lam[6], lam[7]);
   }
 }
 
