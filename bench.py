@@ -449,6 +449,7 @@ E2E_GROUPS = 4   # row groups of the batch that forward_host pipelines in the e2
 
 
 def cpu_baseline(inputs):
+    from threadpoolctl import threadpool_limits
     _oracle_sample(inputs, row=0, steps=512)          # untimed: first touch of host memory
     tok, dt, n = 0, 0.0, 0
     while dt < CPU_SAMPLE_SECONDS:
@@ -456,10 +457,20 @@ def cpu_baseline(inputs):
         tok += t
         dt += d
         n += 1
+    # the same oracle with its BLAS held to one thread (the recurrence is single-threaded numpy)
+    tok1, dt1, n1 = 0, 0.0, 0
+    with threadpool_limits(limits=1):
+        while dt1 < CPU_SAMPLE_SECONDS / 2:
+            t, d = _oracle_sample(inputs, row=n1 % WORKLOAD["B"], steps=WORKLOAD["T"])
+            tok1 += t
+            dt1 += d
+            n1 += 1
     return {"value": tok / dt, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
             "sample": f"{n} batch rows (cycling over the {WORKLOAD['B']} rows) x {WORKLOAD['T']} steps x "
                       f"{WORKLOAD['R']} channels of the workload, {dt:.1f} s; float64 numpy, BLAS matmul on the "
-                      "host cores, recurrence vectorised over channels"}
+                      "host cores, recurrence vectorised over channels",
+            "single_core": {"value": tok1 / dt1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"{n1} batch rows, {dt1:.1f} s, BLAS limited to one thread"}}
 
 
 def run_reference(args):
