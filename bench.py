@@ -145,7 +145,7 @@ def run_own(args):
     y = torch.empty_like(x)
     h_T = torch.empty(B, R, dtype=torch.float32, device=dev)
     u = torch.empty_like(x)
-    z = torch.empty(B * T, rglru.gate_pitch(R), dtype=torch.bfloat16, device=dev)
+    z = torch.empty(B * T, rglru.gate_pitch(R), dtype=torch.float16, device=dev)  # packed coefficients
     ws_gs = torch.empty(rglru.gate_scan_workspace_bytes(B, T, R), dtype=torch.uint8, device=dev)
     ws_scan = torch.empty(rglru.scan_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -165,16 +165,17 @@ def run_own(args):
         return
 
     def step(ev=None):
-        # exactly the launches rglru_forward makes: conv, gate GEMM, fused scan
+        # exactly the launches rglru_forward makes for bf16: conv, gate GEMM forming the
+        # recurrence coefficients, fused scan
         if ev is not None:
             ev[0].record(stream)
         rglru.conv1d(p, x, u=u)
         if ev is not None:
             ev[1].record(stream)
-        rglru.gate_proj(p, u.view(B * T, R), z=z)
+        rglru.gate_coeffs(p, u.view(B * T, R), g=z)
         if ev is not None:
             ev[2].record(stream)
-        rglru.scan(p, x, z, workspace=ws_scan, y=y, h_T=h_T)
+        rglru.scan_coeffs(p, x, z, workspace=ws_scan, y=y, h_T=h_T)
         if ev is not None:
             ev[3].record(stream)
 
@@ -226,9 +227,9 @@ def run_own(args):
     tokens = B * T
     value = world * tokens / (step_ms / 1e3)
     pk = _peaks()
-    # algorithmic bytes / flops per launch (bf16 = 2 B; packed z = 2 gates × 2 B per channel)
+    # algorithmic bytes / flops per launch (bf16 = 2 B; packed coefficients = 2 × 2 B per channel)
     conv_bytes = tokens * R * 2 * 2                     # read x, write u
-    scan_bytes = tokens * R * (2 + 4 + 2)               # read x, read z_a and z_x, write y
+    scan_bytes = tokens * R * (2 + 4 + 2)               # read x, read d and m, write y
     gemm_flops = 2.0 * tokens * (2 * R) * R
     kern = {
         "conv1d": {"ms": conv_ms, "GB/s": conv_bytes / conv_ms / 1e6, "bytes": conv_bytes},

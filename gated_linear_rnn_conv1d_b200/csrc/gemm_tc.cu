@@ -21,6 +21,7 @@
 #include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <mutex>
 
 #include "gate_math.cuh"
@@ -34,7 +35,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int kGemmThreads = 192;
 
-enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2, EPI_SCAN = 3 };
+enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2, EPI_SCAN = 3, EPI_COEF = 4 };
 
 struct EpiArgs {
   __nv_bfloat16* C;   // STORE / GATES output
@@ -363,8 +364,14 @@ constexpr int kScanStages = 5;
 constexpr int kTbufBytes = 4 * 32 * 33 * 8;
 constexpr int kScanEpiBytes = kTbufBytes + 4 * 32 * 2 * 4 + 32 * 4 + 6 * 128 * 4;
 template <int EPI> __host__ __device__ constexpr int stages_of() { return EPI == EPI_SCAN ? kScanStages : k2Stages; }
+constexpr int kCoefEpiBytes = 2 * 3 * 128 * 4;  // per tile parity: b_a, b_x, c·log σ(Λ) of 128 channels
+// warps: 0 TMA, 1 MMA, then epilogue warps — 4 (one per TMEM lane quarter), or 8 for the
+// coefficient epilogue (two per quarter, each taking half of the channels)
+template <int EPI> __host__ __device__ constexpr int epi_warps_of() { return EPI == EPI_COEF ? 8 : 4; }
+template <int EPI> __host__ __device__ constexpr int threads_of() { return 64 + 32 * epi_warps_of<EPI>(); }
 template <int EPI> __host__ __device__ constexpr int smem_of() {
-  return stages_of<EPI>() * k2StageBytes + (EPI == EPI_SCAN ? kScanEpiBytes : 0) + 1024;
+  return stages_of<EPI>() * k2StageBytes + (EPI == EPI_SCAN ? kScanEpiBytes : 0) +
+         (EPI == EPI_COEF ? kCoefEpiBytes : 0) + 1024;
 }
 
 // Gate math for two elements: d = 1 − a_t and b_t = √(1−a_t²)·i·u, with r = σ(z_a),
@@ -423,7 +430,7 @@ __device__ __forceinline__ uint32_t enc_carry(float v) {
 __device__ __forceinline__ float dec_carry(uint32_t w) { return __uint_as_float(w ^ 0x7FFFFFFFu); }
 
 template <int EPI, bool DUAL>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(threads_of<EPI>(), 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                  const __grid_constant__ CUtensorMap tmB1, int64_t M, int K, int n_tiles_n, int num_tiles, EpiArgs ep,
                  unsigned* status) {
@@ -453,7 +460,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 8);  // 4 epilogue warps in each of the two CTAs
+      mbar_init(&tempty_bar[i], 2 * epi_warps_of<EPI>());  // the epilogue warps of both CTAs
     }
     mbar_init(&drain_bar, 1);
     abort_s = 0;
@@ -556,6 +563,53 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       const int64_t row = (int64_t)m_pair * 256 + rank * 128 + row_in_tile;
       const bool row_ok = row < M;
+      if constexpr (EPI == EPI_COEF) {
+        // "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元, Eq. (3)–(4):
+        // columns [0, 128) are z_a and [128, 256) z_x of channels n_blk·128 + j. Each row's
+        // pairs become the recurrence coefficients d = 1 − a_t and m = √(1−a_t²)·i_t (fp16, in
+        // the same packed places), so that the scan only multiplies m by u_t.
+        float* sPar = reinterpret_cast<float*>(smem + S * k2StageBytes) + acc * 3 * 128;
+        const int chalf = (warp - 2) / 4;  // which 64 of the 128 channels this warp forms
+        if (chalf == 0) {
+          const int ch = n_blk * 128 + row_in_tile;
+          const bool ok = ch < ep.R;
+          sPar[row_in_tile] = ok ? __ldg(ep.b_a + ch) : 0.0f;
+          sPar[128 + row_in_tile] = ok ? __ldg(ep.b_x + ch) : 0.0f;
+          sPar[256 + row_in_tile] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
+        }
+        named_bar_sync(1, 32 * epi_warps_of<EPI>());  // this CTA's epilogue warps
+        __half* out = reinterpret_cast<__half*>(ep.C) + row * ep.ldc + (int64_t)n_blk * BN;
+#pragma unroll 1
+        for (int cc = 2 * chalf; cc < 2 * chalf + 2; ++cc) {
+          uint32_t ra[32], rx[32];
+          tmem_ld_32x32b_x32(t_row + cc * 32, ra);
+          tmem_ld_32x32b_x32(t_row + 128 + cc * 32, rx);
+          tmem_ld_wait();
+          uint32_t dh[16], mh[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int c = cc * 32 + j;
+            const float2 za = make_float2(__uint_as_float(ra[j]) + sPar[c], __uint_as_float(ra[j + 1]) + sPar[c + 1]);
+            const float2 zx =
+                make_float2(__uint_as_float(rx[j]) + sPar[128 + c], __uint_as_float(rx[j + 1]) + sPar[128 + c + 1]);
+            float2 d, m;
+            gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), make_float2(1.0f, 1.0f), d, m);
+            const __half2 dd = __floats2half2_rn(d.x, d.y);
+            const __half2 mm = __floats2half2_rn(m.x, m.y);
+            dh[j / 2] = *reinterpret_cast<const uint32_t*>(&dd);
+            mh[j / 2] = *reinterpret_cast<const uint32_t*>(&mm);
+          }
+          if (row_ok) {
+            uint4* pd = reinterpret_cast<uint4*>(out + cc * 32);
+            uint4* pm = reinterpret_cast<uint4*>(out + 128 + cc * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              pd[q] = make_uint4(dh[4 * q], dh[4 * q + 1], dh[4 * q + 2], dh[4 * q + 3]);
+              pm[q] = make_uint4(mh[4 * q], mh[4 * q + 1], mh[4 * q + 2], mh[4 * q + 3]);
+            }
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int cc = 0; cc < BN / 32; ++cc) {
         uint32_t r[32];
@@ -590,6 +644,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
+      }
       }
       tc_fence_before();
       __syncwarp();
@@ -1081,7 +1136,7 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   const int clusters = (int)std::min<int64_t>(tiles, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(threads_of<EPI>());
   cfg.dynamicSmemBytes = smem_of<EPI>();
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1210,6 +1265,24 @@ cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* b
   ep.R = R;
   const int n_tiles_n = (R + 127) / 128;
   return launch_tc2<EPI_GATES, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
+}
+
+cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
+                                    const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s) {
+  // the gate GEMM's tiles, with the recurrence coefficients formed in the epilogue
+  CUtensorMap ma, mb0, mb1;
+  if (!make_map_2d(&ma, u, R, M, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb0, Wa, R, R, (uint64_t)R * 2, BK, 128)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb1, Wx, R, R, (uint64_t)R * 2, BK, 128)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.C = static_cast<__nv_bfloat16*>(g);
+  ep.ldc = gate_pitch(R);
+  ep.b_a = ba;
+  ep.b_x = bx;
+  ep.Lambda = Lambda;
+  ep.R = R;
+  const int n_tiles_n = (R + 127) / 128;
+  return launch_tc2<EPI_COEF, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
 }
 
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,

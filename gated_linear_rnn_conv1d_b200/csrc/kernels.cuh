@@ -52,7 +52,9 @@ struct ScanArgs {
 // Testing only: the tile index the next scans leave unpublished (-1 disables).
 void set_scan_stall(int64_t tile);
 int64_t scan_stall();
-cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s);
+// coef: z holds the recurrence coefficients (fp16 d = 1 − a_t, m = √(1−a_t²)·i_t) that
+// launch_gemm_coeffs_bf16 forms, instead of pre-activations (bf16 IO only).
+cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s, bool coef = false);
 
 // ---- conv --------------------------------------------------------------------------
 cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* state0, void* u,
@@ -70,6 +72,10 @@ EncodeTiledFn get_encode_tiled();
 int num_sms();
 
 // `status`: device word the kernel ORs kStatusTimeout into if a bounded wait gives up.
+// The gate GEMM with the recurrence coefficients formed in its epilogue: g packed like z,
+// fp16 d = 1 − a_t in the z_a places and m = √(1−a_t²)·i_t in the z_x places.
+cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
+                                    const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
                                    void* z, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,

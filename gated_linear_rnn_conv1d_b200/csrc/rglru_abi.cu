@@ -156,9 +156,10 @@ uint8_t* bytes(void* p) { return static_cast<uint8_t*>(p); }
 
 // Queues the scan; with zero_first, first zeroes the status word, the ticket counter and
 // the look-back flags (which must be zero when the scan starts).
+// coef: z holds the recurrence coefficients of launch_gemm_coeffs_bf16, not pre-activations.
 cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_t pitch, const void* state0,
                      const float* h0, const void* g, void* y, float* hT, int B, int T, int R, bool bf16,
-                     const ScanLayout& sl, void* ws, bool zero_first, cudaStream_t s) {
+                     const ScanLayout& sl, void* ws, bool zero_first, cudaStream_t s, bool coef = false) {
   if (zero_first) {
     cudaError_t e = cudaMemsetAsync(ws, 0, sl.zero_bytes, s);
     if (e != cudaSuccess) return e;
@@ -184,7 +185,7 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
   a.n_chunks = sl.n_chunks;
   a.n_tiles = (int)sl.n_tiles;
   a.pitch = pitch;
-  return launch_scan(a, bf16, s);
+  return launch_scan(a, bf16, s, coef);
 }
 
 }  // namespace
@@ -324,6 +325,40 @@ int rglru_scan(const rglru_params* params, const void* x, const void* z, const v
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
+int rglru_gate_coeffs(const rglru_params* params, const void* u, void* g, int64_t N_tok, int R,
+                      rglru_stream_t stream) {
+  if (!valid_R(R) || N_tok < 1 || N_tok > (int64_t)INT32_MAX) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (u == nullptr || g == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(u) || !aligned16(g)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  unsigned* status = global_status_word();
+  if (status == nullptr) return fail_cuda(cudaGetLastError());
+  cudaError_t e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, g,
+                                          N_tok, R, status, (cudaStream_t)stream);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_scan_coeffs(const rglru_params* params, const void* x, const void* g, const void* conv_state0,
+                      const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R, void* workspace,
+                      size_t workspace_bytes, rglru_stream_t stream) {
+  if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x == nullptr || g == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(y) || !aligned16(conv_state0) || !aligned16(h0) ||
+      !aligned16(gate_g) || !aligned16(h_T))
+    return RGLRU_ERR_ALIGN;
+  const ScanLayout sl = scan_layout(B, T, R, true);
+  if (workspace == nullptr || workspace_bytes < sl.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaError_t e = run_scan(params, x, g, gate_pitch(R), conv_state0, h0, gate_g, y, h_T, B, T, R, true, sl, workspace,
+                           true, (cudaStream_t)stream, true);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
 int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
                   float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype, void* workspace,
                   size_t workspace_bytes, rglru_stream_t stream) {
@@ -366,15 +401,17 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   if (e != cudaSuccess) return fail_cuda(e);
   e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, status, s);
   if (e != cudaSuccess) return fail_cuda(e);
+  // bf16: the gate GEMM's epilogue forms the recurrence coefficients (d, m) directly
   if (bf16)
-    e = launch_gemm_gates_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, z, (int64_t)B * T, R, status, s);
+    e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, z,
+                                (int64_t)B * T, R, status, s);
   else
     e = launch_gemm_gates_f32(static_cast<const float*>(u), static_cast<const float*>(params->W_a), params->b_a,
                               static_cast<const float*>(params->W_x), params->b_x, static_cast<float*>(z),
                               (int64_t)B * T, R, s);
   if (e != cudaSuccess) return fail_cuda(e);
   e = run_scan(params, x, z, gate_pitch(R), conv_state0, h0, nullptr, y, h_T, B, T, R, bf16, L.scan, workspace,
-               false, s);
+               false, s, bf16);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
@@ -444,7 +481,8 @@ int rglru_block_forward(const rglru_params* params, const void* W_1, const void*
   if (e == cudaSuccess)
     e = launch_conv1d(params->conv_w, params->conv_b, v, nullptr, u, nullptr, B, T, R, true, status, s);
   if (e == cudaSuccess)
-    e = launch_gemm_gates_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, z, ntok, R, status, s);
+    e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, z, ntok, R,
+                                status, s);
   if (e == cudaSuccess) {
     // the scan's memset must not clear a status bit the GEMMs above may have set:
     // zero only the ticket and flags here.
@@ -458,7 +496,7 @@ int rglru_block_forward(const rglru_params* params, const void* W_1, const void*
       a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);
       a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks;
       a.n_tiles = (int)L.scan.n_tiles; a.pitch = gate_pitch(R);
-      e = launch_scan(a, true, s);
+      e = launch_scan(a, true, s, true);
     }
   }
   if (e == cudaSuccess) e = launch_gemm_bf16(pbuf, W_o, out, ntok, D, R, D, status, s);  // out = p W_oᵀ

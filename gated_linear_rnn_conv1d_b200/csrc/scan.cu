@@ -43,6 +43,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "gate_math.cuh"
 #include "kernels.cuh"
@@ -192,6 +193,19 @@ __device__ __forceinline__ void stv_cs(__nv_bfloat16* p, const float (&f)[4]) {
 __device__ __forceinline__ void stv_cs(float* p, const float (&f)[2]) {
   __stcs(reinterpret_cast<float2*>(p), make_float2(f[0], f[1]));
 }
+// 4 fp16 values as floats, and back (the recurrence coefficients of the coefficient path)
+__device__ __forceinline__ void ldv_h(const __half* p, float (&f)[4]) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+  f[0] = lo.x; f[1] = lo.y; f[2] = hi.x; f[3] = hi.y;
+}
+__device__ __forceinline__ void stv_h(__half* p, const float (&f)[4]) {
+  const __half2 lo = __floats2half2_rn(f[0], f[1]);
+  const __half2 hi = __floats2half2_rn(f[2], f[3]);
+  *reinterpret_cast<uint2*>(p) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
 // V float32 values from shared memory
 template <int V> __device__ __forceinline__ void ldf(const float* p, float (&f)[V]);
 template <> __device__ __forceinline__ void ldf<4>(const float* p, float (&f)[4]) {
@@ -288,9 +302,11 @@ __device__ __forceinline__ void store_params(float* sPar, int CW, int jj, bool i
 // Phase 1 of one tile for compute thread (g, s): conv, gates, log-space decay and the fold
 // of the sub-chunk's 4 steps into (A, B); the replay values go over the z_a, z_x slots the
 // thread read them from (no other thread reads those slots).
-// kFast: every step of the sub-chunk is inside [0, T) and every channel of the warp has
-// c·log σ(Λ) ≥ −1/8, so neither the identity-step mask nor the wide decay path is needed.
-template <typename T, bool kGate, bool kFast>
+// kFast: every step of the sub-chunk is inside [0, T) and (unless kCoef) every channel of
+// the warp has c·log σ(Λ) ≥ −1/8, so neither the identity-step mask nor the wide decay path
+// is needed. kCoef: the z slots hold the recurrence coefficients d = 1 − a_t and
+// m = √(1−a_t²)·i_t (fp16) formed by the gate GEMM, so only b_t = m·u_t is computed here.
+template <typename T, bool kGate, bool kCoef, bool kFast>
 __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB, const TileCoord& tc, int g, int s,
                                             const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
@@ -350,7 +366,24 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
       u[v + 1] = uu.y;
     }
     float at[V], r0[V], bt[V];  // r0: what goes over z_a (a_t, or 1 − a_t on the bf16 path)
-    if constexpr (kAcc) {
+    if constexpr (kCoef) {
+      // za, zx were read as bf16 above; the slots hold fp16 coefficients
+      float dv[V], mv[V];
+      ldv_h(reinterpret_cast<const __half*>(sza) + row * CW + cc, dv);
+      ldv_h(reinterpret_cast<const __half*>(szx) + row * CW + cc, mv);
+#pragma unroll
+      for (int v = 0; v < V; v += 2) {
+        const float2 b2 = __fmul2_rn(make_float2(mv[v], mv[v + 1]), make_float2(u[v], u[v + 1]));
+        r0[v] = tv ? dv[v] : 0.0f;  // steps past T are identity steps
+        r0[v + 1] = tv ? dv[v + 1] : 0.0f;
+        bt[v] = tv ? b2.x : 0.0f;
+        bt[v + 1] = tv ? b2.y : 0.0f;
+        at[v] = 1.0f - r0[v];
+        at[v + 1] = 1.0f - r0[v + 1];
+      }
+      (void)za;
+      (void)zx;
+    } else if constexpr (kAcc) {
 #pragma unroll
       for (int v = 0; v < V; ++v) gate_accurate(za[v], zx[v], CL[v], u[v], at[v], bt[v]);
       if (!tv) {
@@ -379,8 +412,14 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
         at[v + 1] = 1.0f - d.y;
       }
     }
-    stv(sza + row * CW + cc, r0);
-    stv(szx + row * CW + cc, bt);
+    if constexpr (kCoef) {
+      // d stays in place (steps past T need their zero written); b_t replaces m
+      if (!kFast) stv_h(reinterpret_cast<__half*>(sza) + row * CW + cc, r0);
+      stv_h(reinterpret_cast<__half*>(szx) + row * CW + cc, bt);
+    } else {
+      stv(sza + row * CW + cc, r0);
+      stv(szx + row * CW + cc, bt);
+    }
     // fold: (A, B) ← (a·A, a·B + b)
 #pragma unroll
     for (int v = 0; v < V; v += 2) {
@@ -401,13 +440,15 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
   stf<V>(mB + s * CW + cc, B);
 }
 
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kCoef>
 __device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, const TileCoord& tc, int g, int s,
                                        const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
   constexpr int V = SV<T>::V;
   bool fast = false;
-  if constexpr (!SV<T>::kAccurate) {
+  if constexpr (kCoef) {
+    fast = tc.chunk * kScanTC + (s + 1) * kL <= a.T;
+  } else if constexpr (!SV<T>::kAccurate) {
     const float* CL = reinterpret_cast<const float*>(stage + Ly::offPar) + 5 * Ly::CW + g * V;
     bool small = true;
 #pragma unroll
@@ -415,9 +456,9 @@ __device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, con
     fast = __all_sync(0xffffffffu, small) && tc.chunk * kScanTC + (s + 1) * kL <= a.T;
   }
   if (fast)
-    phase1_body<T, kGate, true>(stage, mA, mB, tc, g, s, a);
+    phase1_body<T, kGate, kCoef, true>(stage, mA, mB, tc, g, s, a);
   else
-    phase1_body<T, kGate, false>(stage, mA, mB, tc, g, s, a);
+    phase1_body<T, kGate, kCoef, false>(stage, mA, mB, tc, g, s, a);
 }
 
 // Phase 3 of one tile for compute thread (g, s): replay the sub-chunk from its incoming
@@ -425,7 +466,7 @@ __device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, con
 // shared-memory read comes first and is followed by the proxy fence that lets the stage be
 // refilled by asynchronous copies; only then are the global stores issued, so the fence
 // never waits for them.
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kCoef>
 __device__ __forceinline__ void phase3(const uint8_t* stage, const float* mH, const TileCoord& tc, int g, int s,
                                        const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
@@ -453,8 +494,13 @@ __device__ __forceinline__ void phase3(const uint8_t* stage, const float* mH, co
 #pragma unroll
   for (int l = 0; l < kL; ++l) {
     const int row = s * kL + l;
-    ldv(sza + row * CW + cc, r0[l]);
-    ldv(szx + row * CW + cc, bt[l]);
+    if constexpr (kCoef) {
+      ldv_h(reinterpret_cast<const __half*>(sza) + row * CW + cc, r0[l]);
+      ldv_h(reinterpret_cast<const __half*>(szx) + row * CW + cc, bt[l]);
+    } else {
+      ldv(sza + row * CW + cc, r0[l]);
+      ldv(szx + row * CW + cc, bt[l]);
+    }
   }
   fence_proxy_async_smem();
   if (c0 >= a.R) return;
@@ -553,7 +599,7 @@ __device__ __forceinline__ void lookback_finish(const float* mA, float* mB, cons
   }
 }
 
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kCoef>
 __global__ void __launch_bounds__(kThreads, 1)
     rglru_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs a) {
   using Ly = SmemLayout<T, kGate>;
@@ -596,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = tile < a.n_tiles;
       if (valid) {
         float* mA = maps_base + (k & 1) * 2 * kSub * CW;
-        phase1<T, kGate>(smem + st * Ly::kStage, mA, mA + kSub * CW, coord_of(tile, a), g, s, a);
+        phase1<T, kGate, kCoef>(smem + st * Ly::kStage, mA, mA + kSub * CW, coord_of(tile, a), g, s, a);
       }
       // the look-back warps learn of the end of the tile sequence through this barrier too
       bar_arrive_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
@@ -607,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) atomicOr(a.status, kStatusTimeout);
         }
         const float* mH = maps_base + (kp & 1) * 2 * kSub * CW + kSub * CW;
-        phase3<T, kGate>(smem + stp * Ly::kStage, mH, coord_of(s_tile[stp], a), g, s, a);
+        phase3<T, kGate, kCoef>(smem + stp * Ly::kStage, mH, coord_of(s_tile[stp], a), g, s, a);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stp]);
       }
@@ -689,10 +735,10 @@ std::atomic<int64_t> g_stall_tile{-1};
 
 // One CTA per SM: every CTA of the grid is resident at once, which the look-back's
 // forward-progress argument needs.
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kCoef>
 cudaError_t launch_typed(const ScanArgs& a, const ScanMaps& maps, cudaStream_t s) {
   using Ly = SmemLayout<T, kGate>;
-  auto kern = rglru_scan_kernel<T, kGate>;
+  auto kern = rglru_scan_kernel<T, kGate, kCoef>;
   static bool ready[64] = {false};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -739,7 +785,8 @@ ScanLayout scan_layout(int B, int T, int R, bool bf16) {
 void set_scan_stall(int64_t tile) { g_stall_tile.store(tile); }
 int64_t scan_stall() { return g_stall_tile.load(); }
 
-cudaError_t launch_scan(const ScanArgs& a_in, bool bf16, cudaStream_t s) {
+cudaError_t launch_scan(const ScanArgs& a_in, bool bf16, cudaStream_t s, bool coef) {
+  if (coef && !bf16) return cudaErrorInvalidValue;
   ScanArgs a = a_in;
   a.stall_tile = scan_stall();
   ScanMaps maps;
@@ -762,11 +809,17 @@ cudaError_t launch_scan(const ScanArgs& a_in, bool bf16, cudaStream_t s) {
     cuuint64_t dims[2] = {(cuuint64_t)a.pitch, (cuuint64_t)a.B * a.T};
     cuuint64_t strides[1] = {(cuuint64_t)a.pitch * es};
     cuuint32_t box[2] = {(cuuint32_t)cw, (cuuint32_t)kScanTC};
-    if (!encode(&maps.z, dt, 2, a.z, dims, strides, box)) return cudaErrorInvalidValue;
+    const CUtensorMapDataType zdt = coef ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : dt;
+    if (!encode(&maps.z, zdt, 2, a.z, dims, strides, box)) return cudaErrorInvalidValue;
   }
   const bool gate = a.g != nullptr;
-  if (bf16) return gate ? launch_typed<__nv_bfloat16, true>(a, maps, s) : launch_typed<__nv_bfloat16, false>(a, maps, s);
-  return gate ? launch_typed<float, true>(a, maps, s) : launch_typed<float, false>(a, maps, s);
+  if (coef)
+    return gate ? launch_typed<__nv_bfloat16, true, true>(a, maps, s)
+                : launch_typed<__nv_bfloat16, false, true>(a, maps, s);
+  if (bf16)
+    return gate ? launch_typed<__nv_bfloat16, true, false>(a, maps, s)
+                : launch_typed<__nv_bfloat16, false, false>(a, maps, s);
+  return gate ? launch_typed<float, true, false>(a, maps, s) : launch_typed<float, false, false>(a, maps, s);
 }
 
 }  // namespace rglru

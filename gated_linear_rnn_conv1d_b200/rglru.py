@@ -267,6 +267,36 @@ def scan(params: Params, x: torch.Tensor, z: torch.Tensor, h0: Optional[torch.Te
     return y, h_T
 
 
+def gate_coeffs(params: Params, u: torch.Tensor, *, g: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_gate_coeffs: u [N_tok][R] bf16 → packed fp16 recurrence coefficients
+    (d = 1 − a_t in the recurrence-gate places, m = √(1−a_t²)·i_t in the input-gate places)."""
+    lib = _abi.load()
+    N, R = u.shape
+    g = torch.empty(N, gate_pitch(R), dtype=torch.float16, device=u.device) if g is None else g
+    st = params.struct()
+    _abi.check("rglru_gate_coeffs", lib.rglru_gate_coeffs(ctypes.byref(st), _p(u), _p(g), N, R, _s(stream)))
+    return g
+
+
+def scan_coeffs(params: Params, x: torch.Tensor, g: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                conv_state0: Optional[torch.Tensor] = None, gate_g: Optional[torch.Tensor] = None, *,
+                workspace: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                h_T: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """rglru_scan_coeffs: (x bf16, packed coefficients) → (y, h_T)."""
+    lib = _abi.load()
+    B, T, R = x.shape
+    y = torch.empty_like(x) if y is None else y
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16), x.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_scan_coeffs", lib.rglru_scan_coeffs(
+        ctypes.byref(st), _p(x), _p(g), _p(conv_state0), _p(h0), _p(gate_g), _p(y), _p(h_T), B, T, R, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return y, h_T
+
+
 def gate_scan_workspace_bytes(B: int, T: int, R: int) -> int:
     return _abi.load().rglru_gate_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16)
 

@@ -137,8 +137,10 @@ RGLRU_API int rglru_block_forward(const rglru_params* params, const void* W_1, c
                         int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
- * The three stages of rglru_forward, callable one by one (for per-kernel timing and
- * for testing each stage against the oracle). rglru_forward runs exactly these.
+ * The stages of rglru_forward, callable one by one (for per-kernel timing and for
+ * testing each stage against the oracle). rglru_forward runs exactly rglru_conv1d, then
+ * for RGLRU_BF16 rglru_gate_coeffs and rglru_scan_coeffs, for RGLRU_F32 rglru_gate_proj
+ * and rglru_scan.
  *
  * rglru_conv1d: u = Conv1D(x) (§循环块). x, u [B][T][R] io_dtype; conv_state0 as in
  *   rglru_forward (NULL = zeros); conv_state_T may be NULL.
@@ -165,6 +167,25 @@ RGLRU_API size_t rglru_scan_workspace_bytes(int B, int T, int R, int io_dtype);
 RGLRU_API int rglru_scan(const rglru_params* params, const void* x, const void* z, const void* conv_state0,
                const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R, int io_dtype,
                void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+
+/* rglru_gate_coeffs (bf16 u and weights): the gate GEMM with the gates applied in its
+ *   epilogue ("Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元,
+ *   Eq. (1)–(4)): with z as in rglru_gate_proj, r = σ(z_a), i = σ(z_x),
+ *   log a_t = r·c·log σ(Λ), it writes the recurrence coefficients d = 1 − a_t and
+ *   m = √(1 − a_t²)·i (so that a_t = 1 − d and the input term is m·u_t) as IEEE fp16 in
+ *   the packed layout of z: d in the recurrence-gate places, m in the input-gate places.
+ *   g is [N_tok][rglru_gate_pitch(R)] fp16, 16-byte aligned. fp16 keeps 11 significant
+ *   bits of d, whose relative error multiplies into every carried state.
+ *
+ * rglru_scan_coeffs: rglru_scan for bf16 IO given those coefficients instead of z:
+ *   recomputes u from x (fp32), forms a_t = 1 − d and b_t = m·u_t, and runs the chunked
+ *   recurrence. Arguments and workspace as rglru_scan with io_dtype = RGLRU_BF16.
+ */
+RGLRU_API int rglru_gate_coeffs(const rglru_params* params, const void* u, void* g, int64_t N_tok, int R,
+                                rglru_stream_t stream);
+RGLRU_API int rglru_scan_coeffs(const rglru_params* params, const void* x, const void* g, const void* conv_state0,
+                                const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R,
+                                void* workspace, size_t workspace_bytes, rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * rglru_scan without a workspace, for callers that cannot allocate device memory: a
