@@ -429,6 +429,28 @@ __device__ __forceinline__ uint32_t enc_carry(float v) {
 }
 __device__ __forceinline__ float dec_carry(uint32_t w) { return __uint_as_float(w ^ 0x7FFFFFFFu); }
 
+
+// 16 columns of this warp's TMEM lane quarter; the values are valid only after
+// tmem_ld_wait16 on the same registers (which ties every use to the wait).
+__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait16(uint32_t (&a)[16], uint32_t (&b)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                 "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]),
+                 "+r"(a[15]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]),
+                 "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]),
+                 "+r"(b[14]), "+r"(b[15])
+               :
+               : "memory");
+}
+
 template <int EPI, bool DUAL>
 __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
@@ -579,19 +601,27 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         }
         named_bar_sync(1, 32 * epi_warps_of<EPI>());  // this CTA's epilogue warps
         __half* out = reinterpret_cast<__half*>(ep.C) + row * ep.ldc + (int64_t)n_blk * BN;
-#pragma unroll 1
-        for (int cc = 2 * chalf; cc < 2 * chalf + 2; ++cc) {
-          uint32_t ra[32], rx[32];
-          tmem_ld_32x32b_x32(t_row + cc * 32, ra);
-          tmem_ld_32x32b_x32(t_row + 128 + cc * 32, rx);
-          tmem_ld_wait();
-          uint32_t dh[16], mh[16];
+        // 4 chunks of 16 channels; the next chunk's TMEM load is in flight while one is formed
+        uint32_t ra[2][16], rx[2][16];
+        tmem_ld_x16(t_row + chalf * 64, ra[0]);
+        tmem_ld_x16(t_row + 128 + chalf * 64, rx[0]);
+        tmem_ld_wait16(ra[0], rx[0]);
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int c = cc * 32 + j;
-            const float2 za = make_float2(__uint_as_float(ra[j]) + sPar[c], __uint_as_float(ra[j + 1]) + sPar[c + 1]);
-            const float2 zx =
-                make_float2(__uint_as_float(rx[j]) + sPar[128 + c], __uint_as_float(rx[j + 1]) + sPar[128 + c + 1]);
+        for (int k = 0; k < 4; ++k) {
+          const int cur = k & 1;
+          if (k + 1 < 4) {
+            tmem_ld_x16(t_row + chalf * 64 + (k + 1) * 16, ra[cur ^ 1]);
+            tmem_ld_x16(t_row + 128 + chalf * 64 + (k + 1) * 16, rx[cur ^ 1]);
+          }
+          const int c0 = chalf * 64 + k * 16;
+          uint32_t dh[8], mh[8];
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const int c = c0 + j;
+            const float2 za =
+                make_float2(__uint_as_float(ra[cur][j]) + sPar[c], __uint_as_float(ra[cur][j + 1]) + sPar[c + 1]);
+            const float2 zx = make_float2(__uint_as_float(rx[cur][j]) + sPar[128 + c],
+                                          __uint_as_float(rx[cur][j + 1]) + sPar[128 + c + 1]);
             float2 d, m;
             gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), make_float2(1.0f, 1.0f), d, m);
             const __half2 dd = __floats2half2_rn(d.x, d.y);
@@ -600,14 +630,14 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
             mh[j / 2] = *reinterpret_cast<const uint32_t*>(&mm);
           }
           if (row_ok) {
-            uint4* pd = reinterpret_cast<uint4*>(out + cc * 32);
-            uint4* pm = reinterpret_cast<uint4*>(out + 128 + cc * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              pd[q] = make_uint4(dh[4 * q], dh[4 * q + 1], dh[4 * q + 2], dh[4 * q + 3]);
-              pm[q] = make_uint4(mh[4 * q], mh[4 * q + 1], mh[4 * q + 2], mh[4 * q + 3]);
-            }
+            uint4* pd = reinterpret_cast<uint4*>(out + c0);
+            uint4* pm = reinterpret_cast<uint4*>(out + 128 + c0);
+            pd[0] = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+            pd[1] = make_uint4(dh[4], dh[5], dh[6], dh[7]);
+            pm[0] = make_uint4(mh[0], mh[1], mh[2], mh[3]);
+            pm[1] = make_uint4(mh[4], mh[5], mh[6], mh[7]);
           }
+          if (k + 1 < 4) tmem_ld_wait16(ra[cur ^ 1], rx[cur ^ 1]);
         }
       } else {
 #pragma unroll 1
