@@ -572,9 +572,10 @@ __device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const 
   for (int n = 0; n < NCH; ++n) hin[n] = w[n] != 0u ? dec(w[n]) : 0.0f;
 }
 
-// Look-back, second half, once phase 1 of the tile is done: scans the sub-chunk maps
-// (mA, mB), publishes the tile's inclusive states, writes h_T for the last chunk, and
-// leaves each sub-chunk's incoming state in mB.
+// Look-back, second half, once phase 1 of the tile is done: composes the 16 sub-chunk maps
+// (mA, mB) into the tile's map, publishes the tile's inclusive state A·h_in + B at once (the
+// next chunk waits for it), writes h_T for the last chunk, and then leaves each sub-chunk's
+// incoming state in mB. The channels of a thread are interleaved so their chains overlap.
 template <typename T, bool kGate, int NCH>
 __device__ __forceinline__ void lookback_finish(const float* mA, float* mB, const TileCoord& tc, int j,
                                                 const ScanArgs& a, const float (&hin)[NCH]) {
@@ -582,20 +583,40 @@ __device__ __forceinline__ void lookback_finish(const float* mA, float* mB, cons
   constexpr int S = kSub;
   constexpr int kStride = CW / NCH;
   const bool publish = tc.tix != a.stall_tile;
+  float A[NCH], Bv[NCH];
+#pragma unroll
+  for (int n = 0; n < NCH; ++n) { A[n] = 1.0f; Bv[n] = 0.0f; }
+#pragma unroll
+  for (int q = 0; q < S; ++q) {
+#pragma unroll
+    for (int n = 0; n < NCH; ++n) {
+      const int jj = j + n * kStride;
+      const float pa = mA[q * CW + jj], pb = mB[q * CW + jj];
+      Bv[n] = fmaf(pa, Bv[n], pb);
+      A[n] *= pa;
+    }
+  }
 #pragma unroll
   for (int n = 0; n < NCH; ++n) {
     const int jj = j + n * kStride;
     const int c = tc.cblk * CW + jj;
-    // the state entering each sub-chunk, and after the last one the tile's inclusive state
-    float h = hin[n];
+    const float hout = fmaf(A[n], hin[n], Bv[n]);
+    if (publish && c < a.R) st_relaxed_u32(a.carry_incl + tc.tix * CW + jj, enc(hout));
+    if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < a.R) a.hT[(int64_t)tc.b * a.R + c] = hout;
+  }
+  // the state entering each sub-chunk
+  float h[NCH];
 #pragma unroll
-    for (int q = 0; q < S; ++q) {
+  for (int n = 0; n < NCH; ++n) h[n] = hin[n];
+#pragma unroll
+  for (int q = 0; q < S; ++q) {
+#pragma unroll
+    for (int n = 0; n < NCH; ++n) {
+      const int jj = j + n * kStride;
       const float pa = mA[q * CW + jj], pb = mB[q * CW + jj];
-      mB[q * CW + jj] = h;
-      h = fmaf(pa, h, pb);
+      mB[q * CW + jj] = h[n];
+      h[n] = fmaf(pa, h[n], pb);
     }
-    if (publish && c < a.R) st_relaxed_u32(a.carry_incl + tc.tix * CW + jj, enc(h));
-    if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < a.R) a.hT[(int64_t)tc.b * a.R + c] = h;
   }
 }
 
