@@ -93,9 +93,8 @@ FusedLayout fused_layout(int B, int T, int R) {
   return L;
 }
 bool fused_ok(int io, int T) { return io == RGLRU_BF16 && T % 128 == 0; }
-// rglru_forward keeps the separate gate GEMM + scan: on B200 the fused epilogue (4 warps
-// per SM) is slower than the standalone scan (16 warps per SM) at every shape measured.
-constexpr bool kForwardUsesFusedScan = false;
+// (rglru_forward keeps the separate gate GEMM + scan: on B200 the fused epilogue, with 4
+// warps per SM for the scan, is slower than the standalone scan's 16 warps per SM.)
 
 ScanFusedArgs fused_args(const rglru_params* p, const void* x, const void* u, const void* state0, const float* h0,
                          void* y, float* hT, int B, int T, int R, const FusedLayout& L, void* ws) {
@@ -224,8 +223,7 @@ size_t rglru_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
 
 size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype) {
   if (!valid_dtype(io_dtype) || !valid_R(R) || !valid_tokens(B, T)) return 0;
-  return (kForwardUsesFusedScan && fused_ok(io_dtype, T)) ? fused_layout(B, T, R).bytes
-                                                          : fwd_layout(B, T, R, io_dtype).bytes;
+  return fwd_layout(B, T, R, io_dtype).bytes;
 }
 
 size_t rglru_gate_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
@@ -370,22 +368,6 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   if (!aligned16(x) || !aligned16(y) || !aligned16(h0) || !aligned16(conv_state0) || !aligned16(h_T) ||
       !aligned16(conv_state_T))
     return RGLRU_ERR_ALIGN;
-  if (kForwardUsesFusedScan && fused_ok(io_dtype, T)) {
-    // conv, then the gate GEMM with the scan fused into its epilogue
-    const FusedLayout L = fused_layout(B, T, R);
-    if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
-    if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
-    if ((st = check_device()) != RGLRU_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
-    void* u = bytes(workspace) + L.off_u;
-    unsigned* status = reinterpret_cast<unsigned*>(workspace);
-    cudaError_t e = cudaMemsetAsync(workspace, 0, L.zero_bytes, s);
-    if (e == cudaSuccess)
-      e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, true, status, s);
-    if (e == cudaSuccess)
-      e = launch_gate_scan_bf16(fused_args(params, x, u, conv_state0, h0, y, h_T, B, T, R, L, workspace), s);
-    return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
-  }
   const FwdLayout L = fwd_layout(B, T, R, io_dtype);
   if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
   if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
