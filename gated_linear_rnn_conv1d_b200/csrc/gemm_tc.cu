@@ -904,11 +904,6 @@ constexpr int kStepThreads = 384;
 static_assert(kStepStages * kStepStageBytes + 1024 <= kStepSmem, "the ring fits");
 static_assert(kStepSmem <= 227 * 1024, "shared memory");
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z),
-               "f"(v.w)
-               : "memory");
-}
 // Bulk copy of `bytes` from this CTA's shared memory to another CTA's (cluster addresses for
 // the destination and its mbarrier), completing on that mbarrier.
 __device__ __forceinline__ void bulk_copy_to_cta(uint32_t dst_cluster, const void* src, uint32_t bytes,
