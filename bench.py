@@ -175,7 +175,7 @@ def run_own(args):
         rglru.gate_coeffs(p, u.view(B * T, R), g=z)
         if ev is not None:
             ev[2].record(stream)
-        rglru.scan_coeffs(p, x, z, workspace=ws_scan, y=y, h_T=h_T)
+        rglru.scan_coeffs(z, B, T, R, workspace=ws_scan, y=y, h_T=h_T)
         if ev is not None:
             ev[3].record(stream)
 
@@ -229,7 +229,7 @@ def run_own(args):
     pk = _peaks()
     # algorithmic bytes / flops per launch (bf16 = 2 B; packed coefficients = 2 × 2 B per channel)
     conv_bytes = tokens * R * 2 * 2                     # read x, write u
-    scan_bytes = tokens * R * (2 + 4 + 2)               # read x, read d and m, write y
+    scan_bytes = tokens * R * (4 + 2)                   # read d and b (fp16), write y
     gemm_flops = 2.0 * tokens * (2 * R) * R
     kern = {
         "conv1d": {"ms": conv_ms, "GB/s": conv_bytes / conv_ms / 1e6, "bytes": conv_bytes},

@@ -48,6 +48,7 @@ struct EpiArgs {
   float* h;                // STEP: state [M][R], in place
   __nv_bfloat16* y;        // STEP: y_t [M][R]
   const float* cla;        // STEP: c·log σ(Λ) [R]
+  const __nv_bfloat16* ub; // COEF: u [M][R] bf16, the GEMM's A operand (b_t = m·u_t)
   // SCAN (gate GEMM fused with the RG-LRU scan):
   const __nv_bfloat16* x;       // [B][T][R] Conv1D input (u is recomputed from it in float32)
   const __nv_bfloat16* state0;  // [B][3][R] conv history or null
@@ -576,6 +577,19 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     uint32_t acc_phase = 0;
     for (int tile = cluster; tile < num_tiles; tile += n_clusters) {
       const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+      const int64_t row = (int64_t)m_pair * 256 + rank * 128 + row_in_tile;
+      const bool row_ok = row < M;
+      // COEF: this thread's 64 values of u_t (its row, its half of the tile's channels),
+      // loaded before the accumulator is ready; 8 channels are all valid or all not (R % 8 = 0)
+      [[maybe_unused]] uint4 uq[EPI == EPI_COEF ? 8 : 1];
+      if constexpr (EPI == EPI_COEF) {
+        const int ch0 = n_blk * 128 + ((warp - 2) / 4) * 64;
+        const __nv_bfloat16* urow = ep.ub + row * ep.R + ch0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          uq[q] = (row_ok && ch0 + 8 * q < ep.R) ? __ldg(reinterpret_cast<const uint4*>(urow) + q)
+                                                 : make_uint4(0u, 0u, 0u, 0u);
+      }
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_s)) {
         abort_s = 1;
         atomicOr(status, kStatusTimeout);
@@ -583,13 +597,11 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
       }
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      const int64_t row = (int64_t)m_pair * 256 + rank * 128 + row_in_tile;
-      const bool row_ok = row < M;
       if constexpr (EPI == EPI_COEF) {
         // "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元, Eq. (3)–(4):
         // columns [0, 128) are z_a and [128, 256) z_x of channels n_blk·128 + j. Each row's
-        // pairs become the recurrence coefficients d = 1 − a_t and m = √(1−a_t²)·i_t (fp16, in
-        // the same packed places), so that the scan only multiplies m by u_t.
+        // pairs become the recurrence coefficients d = 1 − a_t and b_t = √(1−a_t²)·i_t·u_t
+        // (fp16, in the same packed places): the recurrence is then h_t = (1 − d)·h_{t−1} + b_t.
         float* sPar = reinterpret_cast<float*>(smem + S * k2StageBytes) + acc * 3 * 128;
         const int chalf = (warp - 2) / 4;  // which 64 of the 128 channels this warp forms
         if (chalf == 0) {
@@ -614,16 +626,19 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
             tmem_ld_x16(t_row + 128 + chalf * 64 + (k + 1) * 16, rx[cur ^ 1]);
           }
           const int c0 = chalf * 64 + k * 16;
+          const uint32_t uw[8] = {uq[2 * k].x, uq[2 * k].y, uq[2 * k].z, uq[2 * k].w,
+                                  uq[2 * k + 1].x, uq[2 * k + 1].y, uq[2 * k + 1].z, uq[2 * k + 1].w};
           uint32_t dh[8], mh[8];
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
             const int c = c0 + j;
+            const float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[j / 2]));
             const float2 za =
                 make_float2(__uint_as_float(ra[cur][j]) + sPar[c], __uint_as_float(ra[cur][j + 1]) + sPar[c + 1]);
             const float2 zx = make_float2(__uint_as_float(rx[cur][j]) + sPar[128 + c],
                                           __uint_as_float(rx[cur][j + 1]) + sPar[128 + c + 1]);
             float2 d, m;
-            gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), make_float2(1.0f, 1.0f), d, m);
+            gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), u2, d, m);
             const __half2 dd = __floats2half2_rn(d.x, d.y);
             const __half2 mm = __floats2half2_rn(m.x, m.y);
             dh[j / 2] = *reinterpret_cast<const uint32_t*>(&dd);
@@ -1306,6 +1321,7 @@ cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* 
   ep.b_x = bx;
   ep.Lambda = Lambda;
   ep.R = R;
+  ep.ub = static_cast<const __nv_bfloat16*>(u);
   const int n_tiles_n = (R + 127) / 128;
   return launch_tc2<EPI_COEF, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
 }

@@ -26,9 +26,8 @@ ScanLayout scan_layout(int B, int T, int R, bool bf16);
 
 // TMA tensor maps the scan reads its tiles through.
 struct ScanMaps {
-  CUtensorMap x;  // [B][T][R], box {CW, 67, 1}
+  CUtensorMap x;  // [B][T][R], box {CW, 67, 1} (not encoded for the coefficient scan)
   CUtensorMap z;  // [B·T][pitch], box {CW, 64}
-  CUtensorMap g;  // [B][T][R], box {CW, 64, 1} (gate branch; unused otherwise)
 };
 
 struct ScanArgs {

@@ -155,7 +155,8 @@ uint8_t* bytes(void* p) { return static_cast<uint8_t*>(p); }
 
 // Queues the scan; with zero_first, first zeroes the status word, the ticket counter and
 // the look-back flags (which must be zero when the scan starts).
-// coef: z holds the recurrence coefficients of launch_gemm_coeffs_bf16, not pre-activations.
+// coef: z holds the recurrence coefficients of launch_gemm_coeffs_bf16, not pre-activations;
+// x, state0 and p are then not read (p may be null).
 cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_t pitch, const void* state0,
                      const float* h0, const void* g, void* y, float* hT, int B, int T, int R, bool bf16,
                      const ScanLayout& sl, void* ws, bool zero_first, cudaStream_t s, bool coef = false) {
@@ -171,9 +172,11 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
   a.g = g;
   a.y = y;
   a.hT = hT;
-  a.conv_w = p->conv_w;
-  a.conv_b = p->conv_b;
-  a.Lambda = p->Lambda;
+  if (p != nullptr) {
+    a.conv_w = p->conv_w;
+    a.conv_b = p->conv_b;
+    a.Lambda = p->Lambda;
+  }
   a.status = reinterpret_cast<unsigned*>(ws);
   a.ticket = reinterpret_cast<unsigned*>(bytes(ws) + 4);
   a.carry_incl = reinterpret_cast<uint32_t*>(bytes(ws) + sl.off_incl);
@@ -338,22 +341,19 @@ int rglru_gate_coeffs(const rglru_params* params, const void* u, void* g, int64_
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
-int rglru_scan_coeffs(const rglru_params* params, const void* x, const void* g, const void* conv_state0,
-                      const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R, void* workspace,
-                      size_t workspace_bytes, rglru_stream_t stream) {
+int rglru_scan_coeffs(const void* g, const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R,
+                      void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
-  int st = check_params(params);
-  if (st != RGLRU_OK) return st;
-  if (x == nullptr || g == nullptr || y == nullptr) return RGLRU_ERR_NULL;
-  if (!aligned16(x) || !aligned16(g) || !aligned16(y) || !aligned16(conv_state0) || !aligned16(h0) ||
-      !aligned16(gate_g) || !aligned16(h_T))
+  if (g == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(g) || !aligned16(y) || !aligned16(h0) || !aligned16(gate_g) || !aligned16(h_T))
     return RGLRU_ERR_ALIGN;
   const ScanLayout sl = scan_layout(B, T, R, true);
   if (workspace == nullptr || workspace_bytes < sl.bytes) return RGLRU_ERR_WORKSPACE;
   if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
-  if ((st = check_device()) != RGLRU_OK) return st;
-  cudaError_t e = run_scan(params, x, g, gate_pitch(R), conv_state0, h0, gate_g, y, h_T, B, T, R, true, sl, workspace,
-                           true, (cudaStream_t)stream, true);
+  int st = check_device();
+  if (st != RGLRU_OK) return st;
+  cudaError_t e = run_scan(nullptr, nullptr, g, gate_pitch(R), nullptr, h0, gate_g, y, h_T, B, T, R, true, sl,
+                           workspace, true, (cudaStream_t)stream, true);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
@@ -383,7 +383,7 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   if (e != cudaSuccess) return fail_cuda(e);
   e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, status, s);
   if (e != cudaSuccess) return fail_cuda(e);
-  // bf16: the gate GEMM's epilogue forms the recurrence coefficients (d, m) directly
+  // bf16: the gate GEMM's epilogue forms the recurrence coefficients (d, b) directly
   if (bf16)
     e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, z,
                                 (int64_t)B * T, R, status, s);
@@ -471,8 +471,7 @@ int rglru_block_forward(const rglru_params* params, const void* W_1, const void*
     e = cudaMemsetAsync(bytes(workspace) + 4, 0, L.scan.zero_bytes - 4, s);
     if (e == cudaSuccess) {
       ScanArgs a{};
-      a.x = v; a.z = z; a.state0 = nullptr; a.h0 = h0; a.g = g; a.y = pbuf; a.hT = h_T;
-      a.conv_w = params->conv_w; a.conv_b = params->conv_b; a.Lambda = params->Lambda;
+      a.z = z; a.h0 = h0; a.g = g; a.y = pbuf; a.hT = h_T;  // coefficients: no x or conv parameters
       a.status = status;
       a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
       a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);

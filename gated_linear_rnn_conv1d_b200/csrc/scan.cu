@@ -1,5 +1,8 @@
-// Fused RG-LRU scan: Conv1D recompute + σ gates + log-space decay + chunked diagonal
-// recurrence; one HBM read of x and of the gate pre-activations, one write of y.
+// RG-LRU chunked scan, in two forms:
+//  * from pre-activations: Conv1D recompute + σ gates + log-space decay + chunked diagonal
+//    recurrence; one HBM read of x and of the packed gate pre-activations z, one write of y;
+//  * from recurrence coefficients (bf16 IO): d = 1 − a_t and b_t = √(1−a_t²)·i_t·u_t, both
+//    fp16, formed by the gate GEMM's epilogue; one HBM read of (d, b), one write of y.
 //
 // Math: "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型",
 // §实门线性循环单元 (RG-LRU), Eq. (1)–(4); §循环块 for the Conv1D and the GeLU branch.
@@ -16,32 +19,38 @@
 // One persistent CTA per SM takes tiles in order from an atomic ticket — time-chunk-major,
 // so every tile a CTA waits for was taken earlier by a running CTA (forward progress) —
 // and runs them through a software pipeline of three warp roles:
-//   producer warp    takes tickets, and two tiles ahead of the compute warps fills a
-//                    3-stage ring: TMA copies of the tile's x rows (with the 3-row conv halo;
-//                    rows before t = 0 arrive as zeros), z_a and z_x, plus the tile's
-//                    parameters (taps, conv bias, c·log σ(Λ)) written into the stage;
+//   producer warp    takes tickets and, ahead of the compute warps, fills a ring of stages
+//                    (3, or 5 for the smaller coefficient stages): TMA copies of the tile's
+//                    x rows (with the 3-row conv halo; rows before t = 0 arrive as zeros),
+//                    z_a and z_x, plus the tile's parameters (taps, conv bias, c·log σ(Λ))
+//                    written into the stage — or only the two coefficient blocks — and the
+//                    tile's decoded coordinates;
 //   compute warps    (16, one per sub-chunk; lane = channel group), for tile k:
-//     phase 1  recompute u in float32, apply the gates and the log-space decay, fold the
-//              sub-chunk's 4 steps into an affine map (float32), and write the per-step
-//              replay values (1 − a_t, b_t) over the z_a, z_x slots they came from;
+//     phase 1  recompute u in float32, apply the gates and the log-space decay (or read
+//              the coefficients), fold the sub-chunk's 4 steps into an affine map
+//              (float32); the pre-activation form writes the per-step replay values
+//              (1 − a_t, b_t) over the z_a, z_x slots they came from;
 //     phase 3  (of tile k − 1, whose incoming states are ready by now) replay the
 //              sub-chunk from its incoming state and write y, then release the stage;
-//   look-back warps  (2, two channels per thread for bf16) read the state entering tile k
-//                    — the inclusive state its predecessor chunk publishes, or h0 — while
-//                    phase 1 of tile k runs; once the 16 sub-chunk maps are in, they chain
-//                    them from that state, publish the tile's inclusive state and hand every
+//   look-back warps  (groups of 2 warps, two channels per thread for bf16; the coefficient
+//                    form has two groups taking alternate tiles) read the state entering
+//                    tile k — the inclusive state its predecessor chunk publishes, or h0 —
+//                    while phase 1 of tile k runs; once the 16 sub-chunk maps are in, they
+//                    compose them, publish the tile's inclusive state and hand every
 //                    sub-chunk its incoming state. A published state is a self-validating
 //                    word (an exact XOR encoding whose zero is never a published value, so
 //                    zeroed memory reads as "not yet"): one relaxed load, no fence or flag.
 // Every wait is bounded. Warps of different roles meet at mbarriers (stage full / empty,
 // states ready) and at one named barrier (maps ready) whose id alternates with the tile's
 // parity; the compute warps never wait for one another.
-// The replay values of the bf16 path are stored as bf16 (1 − a_t, b_t): their rounding
-// only touches y inside one 4-step sub-chunk, while the published states and h_T come from
-// the float32 maps.
+// The replay values of the pre-activation bf16 path are stored as bf16 (1 − a_t, b_t): their
+// rounding only touches y inside one 4-step sub-chunk, while the published states and h_T
+// come from the float32 maps. The coefficients are fp16 (11 significant bits); everything
+// composed from them (maps, states, h_T) is float32.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstring>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -71,23 +80,32 @@ constexpr int kSub = kScanSub;                        // sub-chunks: one compute
 constexpr int kL = kScanTC / kSub;                    // steps per sub-chunk
 constexpr int kComputeWarps = kSub;                   // 16
 constexpr int kComputeThreads = kGroups * kSub;       // 512
-constexpr int kLookThreads = 64;
-constexpr int kThreads = kComputeThreads + kLookThreads + 32;  // + one producer warp
-constexpr int kStages = 3;
+// Look-back groups of two warps: the coefficient scan's tiles are short, so two groups take
+// alternate tiles (tile k goes to group k mod 2) and one tile's look-back overlaps the next
+// one's. (Its 21 warps put 6 on some scheduler partition, which leaves a thread 80
+// registers; 19 warps leave 96.)
+template <bool kCoef> constexpr int look_groups() { return kCoef ? 2 : 1; }
+template <bool kCoef> constexpr int look_threads() { return 64; }  // per group
+template <bool kCoef> constexpr int threads_of() {
+  return kComputeThreads + look_groups<kCoef>() * look_threads<kCoef>() + 32;  // + one producer warp
+}
 // named barrier (id 0 is __syncthreads, which the roles never use after the prologue):
 // + tile parity; compute warps arrive once phase 1 is done, look-back warps wait
 constexpr int kBarMaps = 1;
 
-template <typename T, bool kGate> struct SmemLayout {
+// kCoef: the stage holds only the two coefficient blocks (d = 1 − a_t, b_t; fp16), which
+// need neither x nor parameters, so the ring is deeper.
+template <typename T, bool kGate, bool kCoef = false> struct SmemLayout {
   static constexpr int CW = kGroups * SV<T>::V;
-  static constexpr int kX = kXRows * CW * (int)sizeof(T);
+  static constexpr int kStages = kCoef ? 5 : 3;
+  static constexpr int kX = kCoef ? 0 : kXRows * CW * (int)sizeof(T);
   static constexpr int kZ = kScanTC * CW * (int)sizeof(T);
   // a stage: x rows, z_a, z_x (TMA), then the tile's parameters [6][CW] f32 (taps 0..3,
   // conv bias, c·log σ(Λ)) written by the producer warp
   static constexpr int offZA = kX;
   static constexpr int offZX = kX + kZ;
   static constexpr int offPar = kX + 2 * kZ;
-  static constexpr int kStage = offPar + 6 * CW * 4;
+  static constexpr int kStage = offPar + (kCoef ? 0 : 6 * CW * 4);
   static constexpr int offMaps = kStages * kStage;     // [2 buffers][A | B][kSub][CW] f32
   static constexpr int kMaps = 2 * kSub * CW * 4;
   static constexpr int kBytes = offMaps + 2 * kMaps;
@@ -133,8 +151,8 @@ __device__ __forceinline__ uint32_t enc(float v) {
 __device__ __forceinline__ float dec(uint32_t w) { return __uint_as_float(w ^ kCarryKey); }
 
 struct TileCoord {
-  int chunk, b, cblk;
-  int64_t tix;  // carry slot: ((b · n_cblk + cblk) · n_chunks + chunk)
+  int chunk, b, cblk;  // chunk < 0: no tile (the end of a CTA's sequence)
+  int tix;             // carry slot: ((b · n_cblk + cblk) · n_chunks + chunk) < n_tiles
 };
 __device__ __forceinline__ TileCoord coord_of(int ticket, const ScanArgs& a) {
   TileCoord c;
@@ -143,19 +161,19 @@ __device__ __forceinline__ TileCoord coord_of(int ticket, const ScanArgs& a) {
   const int rem = ticket - c.chunk * per_chunk;
   c.b = rem / a.n_cblk;
   c.cblk = rem - c.b * a.n_cblk;
-  c.tix = ((int64_t)c.b * a.n_cblk + c.cblk) * a.n_chunks + c.chunk;
+  c.tix = (c.b * a.n_cblk + c.cblk) * a.n_chunks + c.chunk;
   return c;
 }
 
-template <typename T, bool kGate>
+template <typename T, bool kGate, bool kCoef>
 __device__ __forceinline__ void issue_tile_loads(uint8_t* stage, uint64_t* bar, const ScanMaps& m, const ScanArgs& a,
                                                  const TileCoord& c) {
-  using Ly = SmemLayout<T, kGate>;
+  using Ly = SmemLayout<T, kGate, kCoef>;
   constexpr int CW = Ly::CW;
   mbar_arrive_expect_tx(bar, Ly::kTxXZ);
   const int c0 = c.cblk * CW;
   const int t0 = c.chunk * kScanTC;
-  tma_load_3d(stage, &m.x, bar, c0, t0 - kHalo, c.b);
+  if constexpr (!kCoef) tma_load_3d(stage, &m.x, bar, c0, t0 - kHalo, c.b);
   const int zcol = (c0 / kGateBlock) * 2 * kGateBlock + (c0 % kGateBlock);
   const int zrow = c.b * a.T + t0;
   tma_load_2d(stage + Ly::offZA, &m.z, bar, zcol, zrow);
@@ -302,11 +320,9 @@ __device__ __forceinline__ void store_params(float* sPar, int CW, int jj, bool i
 // Phase 1 of one tile for compute thread (g, s): conv, gates, log-space decay and the fold
 // of the sub-chunk's 4 steps into (A, B); the replay values go over the z_a, z_x slots the
 // thread read them from (no other thread reads those slots).
-// kFast: every step of the sub-chunk is inside [0, T) and (unless kCoef) every channel of
-// the warp has c·log σ(Λ) ≥ −1/8, so neither the identity-step mask nor the wide decay path
-// is needed. kCoef: the z slots hold the recurrence coefficients d = 1 − a_t and
-// m = √(1−a_t²)·i_t (fp16) formed by the gate GEMM, so only b_t = m·u_t is computed here.
-template <typename T, bool kGate, bool kCoef, bool kFast>
+// kFast: every step of the sub-chunk is inside [0, T) and every channel of the warp has
+// c·log σ(Λ) ≥ −1/8, so neither the identity-step mask nor the wide decay path is needed.
+template <typename T, bool kGate, bool kFast>
 __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB, const TileCoord& tc, int g, int s,
                                             const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
@@ -366,24 +382,7 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
       u[v + 1] = uu.y;
     }
     float at[V], r0[V], bt[V];  // r0: what goes over z_a (a_t, or 1 − a_t on the bf16 path)
-    if constexpr (kCoef) {
-      // za, zx were read as bf16 above; the slots hold fp16 coefficients
-      float dv[V], mv[V];
-      ldv_h(reinterpret_cast<const __half*>(sza) + row * CW + cc, dv);
-      ldv_h(reinterpret_cast<const __half*>(szx) + row * CW + cc, mv);
-#pragma unroll
-      for (int v = 0; v < V; v += 2) {
-        const float2 b2 = __fmul2_rn(make_float2(mv[v], mv[v + 1]), make_float2(u[v], u[v + 1]));
-        r0[v] = tv ? dv[v] : 0.0f;  // steps past T are identity steps
-        r0[v + 1] = tv ? dv[v + 1] : 0.0f;
-        bt[v] = tv ? b2.x : 0.0f;
-        bt[v + 1] = tv ? b2.y : 0.0f;
-        at[v] = 1.0f - r0[v];
-        at[v + 1] = 1.0f - r0[v + 1];
-      }
-      (void)za;
-      (void)zx;
-    } else if constexpr (kAcc) {
+    if constexpr (kAcc) {
 #pragma unroll
       for (int v = 0; v < V; ++v) gate_accurate(za[v], zx[v], CL[v], u[v], at[v], bt[v]);
       if (!tv) {
@@ -412,14 +411,8 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
         at[v + 1] = 1.0f - d.y;
       }
     }
-    if constexpr (kCoef) {
-      // d stays in place (steps past T need their zero written); b_t replaces m
-      if (!kFast) stv_h(reinterpret_cast<__half*>(sza) + row * CW + cc, r0);
-      stv_h(reinterpret_cast<__half*>(szx) + row * CW + cc, bt);
-    } else {
-      stv(sza + row * CW + cc, r0);
-      stv(szx + row * CW + cc, bt);
-    }
+    stv(sza + row * CW + cc, r0);
+    stv(szx + row * CW + cc, bt);
     // fold: (A, B) ← (a·A, a·B + b)
 #pragma unroll
     for (int v = 0; v < V; v += 2) {
@@ -440,15 +433,111 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
   stf<V>(mB + s * CW + cc, B);
 }
 
-template <typename T, bool kGate, bool kCoef>
+// The coefficients of one tile as one compute thread holds them between its two phases:
+// kL steps × 4 channels of d and of b, as packed fp16 pairs (bf16 IO only).
+struct CoefRegs {
+  uint32_t d[kL][2], b[kL][2];
+};
+
+// Reads the thread's coefficients of the tile out of the stage (after which the stage may
+// be refilled).
+template <bool kGate>
+__device__ __forceinline__ void coef_load(const uint8_t* stage, int g, int s, CoefRegs& r) {
+  using Ly = SmemLayout<__nv_bfloat16, kGate, true>;
+  constexpr int CW = Ly::CW;
+  const __half* sd = reinterpret_cast<const __half*>(stage + Ly::offZA);
+  const __half* sb = reinterpret_cast<const __half*>(stage + Ly::offZX);
+  const int cc = g * 4;
+#pragma unroll
+  for (int l = 0; l < kL; ++l) {
+    const int row = s * kL + l;
+    const uint2 vd = *reinterpret_cast<const uint2*>(sd + row * CW + cc);
+    const uint2 vb = *reinterpret_cast<const uint2*>(sb + row * CW + cc);
+    r.d[l][0] = vd.x; r.d[l][1] = vd.y;
+    r.b[l][0] = vb.x; r.b[l][1] = vb.y;
+  }
+}
+__device__ __forceinline__ float2 h2f(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+// Phase 1 of the coefficient scan from registers: fold the sub-chunk's 4 steps,
+// (A, B) ← (a·A, a·B + b) with a = 1 − d, into its map. Steps past T are identity steps.
+template <bool kGate>
+__device__ __forceinline__ void coef_fold(const CoefRegs& r, float* mA, float* mB, const TileCoord& tc, int g, int s,
+                                          const ScanArgs& a) {
+  constexpr int CW = SmemLayout<__nv_bfloat16, kGate, true>::CW;
+  const int cc = g * 4;
+  const int t_start = tc.chunk * kScanTC + s * kL;
+  float2 A[2] = {make_float2(1.0f, 1.0f), make_float2(1.0f, 1.0f)};
+  float2 B[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+  const bool whole = t_start + kL <= a.T;
+#pragma unroll
+  for (int l = 0; l < kL; ++l) {
+    if (whole || t_start + l < a.T) {
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float2 d2 = h2f(r.d[l][p]);
+        const float2 a2 = make_float2(1.0f - d2.x, 1.0f - d2.y);
+        B[p] = __ffma2_rn(a2, B[p], h2f(r.b[l][p]));
+        A[p] = __fmul2_rn(a2, A[p]);
+      }
+    }
+  }
+  *reinterpret_cast<float4*>(mA + s * CW + cc) = make_float4(A[0].x, A[0].y, A[1].x, A[1].y);
+  *reinterpret_cast<float4*>(mB + s * CW + cc) = make_float4(B[0].x, B[0].y, B[1].x, B[1].y);
+}
+
+// Phase 3 of the coefficient scan from registers: replay the sub-chunk from its incoming
+// state (mH) and write y (times GeLU of the gate branch for the gated scan).
+template <bool kGate>
+__device__ __forceinline__ void coef_replay(const CoefRegs& r, const float* mH, const TileCoord& tc, int g, int s,
+                                            const ScanArgs& a) {
+  constexpr int CW = SmemLayout<__nv_bfloat16, kGate, true>::CW;
+  const int cc = g * 4;
+  const int c0 = tc.cblk * CW + cc;
+  const int t_start = tc.chunk * kScanTC + s * kL;
+  float gg[kGate ? kL : 1][4];
+  if constexpr (kGate) {
+    const __nv_bfloat16* gsrc = static_cast<const __nv_bfloat16*>(a.g);
+#pragma unroll
+    for (int l = 0; l < kL; ++l) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) gg[l][v] = 0.0f;
+      if (c0 < a.R && t_start + l < a.T) ldv_nc(gsrc + ((int64_t)tc.b * a.T + t_start + l) * a.R + c0, gg[l]);
+    }
+  }
+  const float4 h4 = *reinterpret_cast<const float4*>(mH + s * CW + cc);
+  if (c0 >= a.R) return;
+  float2 h[2] = {make_float2(h4.x, h4.y), make_float2(h4.z, h4.w)};
+  __nv_bfloat16* __restrict__ y = static_cast<__nv_bfloat16*>(a.y);
+#pragma unroll
+  for (int l = 0; l < kL; ++l) {
+    float o[4];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const float2 d2 = h2f(r.d[l][p]);
+      const float2 a2 = make_float2(1.0f - d2.x, 1.0f - d2.y);
+      h[p] = __ffma2_rn(a2, h[p], h2f(r.b[l][p]));
+      o[2 * p] = h[p].x;
+      o[2 * p + 1] = h[p].y;
+    }
+    if constexpr (kGate) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) o[v] *= gelu_exact(gg[l][v]);
+    }
+    const int t = t_start + l;
+    if (t < a.T) stv_cs(y + ((int64_t)tc.b * a.T + t) * a.R + c0, o);
+  }
+}
+
+template <typename T, bool kGate>
 __device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, const TileCoord& tc, int g, int s,
                                        const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
   constexpr int V = SV<T>::V;
   bool fast = false;
-  if constexpr (kCoef) {
-    fast = tc.chunk * kScanTC + (s + 1) * kL <= a.T;
-  } else if constexpr (!SV<T>::kAccurate) {
+  if constexpr (!SV<T>::kAccurate) {
     const float* CL = reinterpret_cast<const float*>(stage + Ly::offPar) + 5 * Ly::CW + g * V;
     bool small = true;
 #pragma unroll
@@ -456,9 +545,9 @@ __device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, con
     fast = __all_sync(0xffffffffu, small) && tc.chunk * kScanTC + (s + 1) * kL <= a.T;
   }
   if (fast)
-    phase1_body<T, kGate, kCoef, true>(stage, mA, mB, tc, g, s, a);
+    phase1_body<T, kGate, true>(stage, mA, mB, tc, g, s, a);
   else
-    phase1_body<T, kGate, kCoef, false>(stage, mA, mB, tc, g, s, a);
+    phase1_body<T, kGate, false>(stage, mA, mB, tc, g, s, a);
 }
 
 // Phase 3 of one tile for compute thread (g, s): replay the sub-chunk from its incoming
@@ -466,7 +555,7 @@ __device__ __forceinline__ void phase1(uint8_t* stage, float* mA, float* mB, con
 // shared-memory read comes first and is followed by the proxy fence that lets the stage be
 // refilled by asynchronous copies; only then are the global stores issued, so the fence
 // never waits for them.
-template <typename T, bool kGate, bool kCoef>
+template <typename T, bool kGate>
 __device__ __forceinline__ void phase3(const uint8_t* stage, const float* mH, const TileCoord& tc, int g, int s,
                                        const ScanArgs& a) {
   using Ly = SmemLayout<T, kGate>;
@@ -494,13 +583,8 @@ __device__ __forceinline__ void phase3(const uint8_t* stage, const float* mH, co
 #pragma unroll
   for (int l = 0; l < kL; ++l) {
     const int row = s * kL + l;
-    if constexpr (kCoef) {
-      ldv_h(reinterpret_cast<const __half*>(sza) + row * CW + cc, r0[l]);
-      ldv_h(reinterpret_cast<const __half*>(szx) + row * CW + cc, bt[l]);
-    } else {
-      ldv(sza + row * CW + cc, r0[l]);
-      ldv(szx + row * CW + cc, bt[l]);
-    }
+    ldv(sza + row * CW + cc, r0[l]);
+    ldv(szx + row * CW + cc, bt[l]);
   }
   fence_proxy_async_smem();
   if (c0 >= a.R) return;
@@ -526,11 +610,15 @@ __device__ __forceinline__ void phase3(const uint8_t* stage, const float* mH, co
 }
 
 // Look-back, first half, for thread j's NCH channel slots j, j + CW/NCH, ...: the state
-// entering the tile, read from the inclusive state its predecessor (the previous time chunk
-// of the same batch row and channel block) publishes, or h0 for the first chunk. It needs
-// nothing of this tile, so it runs while phase 1 of the tile is still in progress.
+// entering the tile is the inclusive state its predecessor (the previous time chunk of the
+// same batch row and channel block) publishes, or h0 for the first chunk. It needs nothing
+// of this tile, so its first read is issued before phase 1 of the tile is done and is only
+// waited for (lookback_end) once the tile's maps are composed. Channels past R (the padding
+// of the last channel block) neither wait for nor publish a state, so whatever their
+// padding inputs hold cannot stall a tile.
 template <typename T, bool kGate, int NCH>
-__device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const ScanArgs& a, float (&hin)[NCH]) {
+__device__ __forceinline__ void lookback_begin(const TileCoord& tc, int j, const ScanArgs& a, uint32_t (&w)[NCH],
+                                               float (&hin)[NCH]) {
   constexpr int CW = SmemLayout<T, kGate>::CW;
   constexpr int kStride = CW / NCH;
   if (tc.chunk == 0) {
@@ -538,17 +626,27 @@ __device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const 
     for (int n = 0; n < NCH; ++n) {
       const int c = tc.cblk * CW + j + n * kStride;
       hin[n] = (a.h0 != nullptr && c < a.R) ? a.h0[(int64_t)tc.b * a.R + c] : 0.0f;
+      w[n] = 1u;
     }
     return;
   }
-  // channels past R (the padding of the last channel block) carry nothing: they neither
-  // wait for nor publish a state, so whatever their padding inputs hold cannot stall a tile
-  const uint32_t* src = a.carry_incl + (tc.tix - 1) * CW + j;
+  // the read is unconditional (every channel slot of a tile exists), so nothing waits for
+  // its result before lookback_end
+  const uint32_t* src = a.carry_incl + (int64_t)(tc.tix - 1) * CW + j;
+#pragma unroll
+  for (int n = 0; n < NCH; ++n) w[n] = ld_relaxed_u32(src + n * kStride);
+}
+template <typename T, bool kGate, int NCH>
+__device__ __forceinline__ void lookback_end(const TileCoord& tc, int j, const ScanArgs& a, uint32_t (&w)[NCH],
+                                             float (&hin)[NCH]) {
+  constexpr int CW = SmemLayout<T, kGate>::CW;
+  constexpr int kStride = CW / NCH;
+  if (tc.chunk == 0) return;
+  const uint32_t* src = a.carry_incl + (int64_t)(tc.tix - 1) * CW + j;
   const uint32_t kNothing = enc(0.0f);
-  uint32_t w[NCH];
 #pragma unroll
   for (int n = 0; n < NCH; ++n)
-    w[n] = tc.cblk * CW + j + n * kStride < a.R ? ld_relaxed_u32(src + n * kStride) : kNothing;
+    if (tc.cblk * CW + j + n * kStride >= a.R) w[n] = kNothing;
   bool ready = true;
 #pragma unroll
   for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
@@ -573,12 +671,15 @@ __device__ __forceinline__ void lookback_walk(const TileCoord& tc, int j, const 
 }
 
 // Look-back, second half, once phase 1 of the tile is done: composes the 16 sub-chunk maps
-// (mA, mB) into the tile's map, publishes the tile's inclusive state A·h_in + B at once (the
-// next chunk waits for it), writes h_T for the last chunk, and then leaves each sub-chunk's
-// incoming state in mB. The channels of a thread are interleaved so their chains overlap.
+// (mA, mB) into the tile's map, waits for the incoming state, publishes the tile's inclusive
+// state A·h_in + B at once (the next chunk waits for it), writes h_T for the last chunk, and
+// then leaves each sub-chunk's incoming state in mB. mA and mB are separate buffers and each
+// slot is read before it is overwritten, so the reads of the second pass need not wait for
+// its stores.
 template <typename T, bool kGate, int NCH>
-__device__ __forceinline__ void lookback_finish(const float* mA, float* mB, const TileCoord& tc, int j,
-                                                const ScanArgs& a, const float (&hin)[NCH]) {
+__device__ __forceinline__ void lookback_finish(const float* __restrict__ mA, float* __restrict__ mB,
+                                                const TileCoord& tc, int j, const ScanArgs& a, uint32_t (&w)[NCH],
+                                                float (&hin)[NCH]) {
   constexpr int CW = SmemLayout<T, kGate>::CW;
   constexpr int S = kSub;
   constexpr int kStride = CW / NCH;
@@ -586,44 +687,51 @@ __device__ __forceinline__ void lookback_finish(const float* mA, float* mB, cons
   float A[NCH], Bv[NCH];
 #pragma unroll
   for (int n = 0; n < NCH; ++n) { A[n] = 1.0f; Bv[n] = 0.0f; }
-#pragma unroll
+#pragma unroll 8
   for (int q = 0; q < S; ++q) {
 #pragma unroll
     for (int n = 0; n < NCH; ++n) {
-      const int jj = j + n * kStride;
-      const float pa = mA[q * CW + jj], pb = mB[q * CW + jj];
+      const float pa = mA[q * CW + j + n * kStride], pb = mB[q * CW + j + n * kStride];
       Bv[n] = fmaf(pa, Bv[n], pb);
       A[n] *= pa;
     }
   }
+  lookback_end<T, kGate, NCH>(tc, j, a, w, hin);
 #pragma unroll
   for (int n = 0; n < NCH; ++n) {
     const int jj = j + n * kStride;
     const int c = tc.cblk * CW + jj;
     const float hout = fmaf(A[n], hin[n], Bv[n]);
-    if (publish && c < a.R) st_relaxed_u32(a.carry_incl + tc.tix * CW + jj, enc(hout));
+    if (publish && c < a.R) st_relaxed_u32(a.carry_incl + (int64_t)tc.tix * CW + jj, enc(hout));
     if (tc.chunk == a.n_chunks - 1 && a.hT != nullptr && c < a.R) a.hT[(int64_t)tc.b * a.R + c] = hout;
   }
   // the state entering each sub-chunk
   float h[NCH];
 #pragma unroll
   for (int n = 0; n < NCH; ++n) h[n] = hin[n];
-#pragma unroll
+#pragma unroll 8
   for (int q = 0; q < S; ++q) {
 #pragma unroll
     for (int n = 0; n < NCH; ++n) {
-      const int jj = j + n * kStride;
-      const float pa = mA[q * CW + jj], pb = mB[q * CW + jj];
-      mB[q * CW + jj] = h[n];
+      const int o = q * CW + j + n * kStride;
+      const float pa = mA[o], pb = mB[o];
+      mB[o] = h[n];
       h[n] = fmaf(pa, h[n], pb);
     }
   }
 }
 
 template <typename T, bool kGate, bool kCoef>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of<kCoef>(), 1)
     rglru_scan_kernel(const __grid_constant__ ScanMaps maps, const ScanArgs a) {
-  using Ly = SmemLayout<T, kGate>;
+  using Ly = SmemLayout<T, kGate, kCoef>;
+  constexpr int kStages = Ly::kStages;
+  // a stage is free once every compute warp is done with it — and, for the coefficient
+  // scan, whose compute warps let go of a stage right after phase 1, once both look-back
+  // warps have read its tile index
+  constexpr int kGroups = look_groups<kCoef>();
+  constexpr int kLookThreads = look_threads<kCoef>();
+  constexpr int kEmptyArrivals = kComputeWarps;
   constexpr int CW = Ly::CW;
   constexpr int PV = CW / 32;  // channels per producer lane
   constexpr int NCH = CW / kLookThreads;  // channels per look-back thread
@@ -634,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t full[kStages];   // TMA bytes + the producer's parameters
   __shared__ __align__(8) uint64_t empty[kStages];  // one arrival per compute warp after phase 3
   __shared__ __align__(8) uint64_t state[2];        // + tile parity: incoming states ready
-  __shared__ int s_tile[kStages];                   // ticket of the tile in each stage
+  __shared__ TileCoord s_tc[kStages];               // the tile in each stage (decoded once)
   float* maps_base = reinterpret_cast<float*>(smem + Ly::offMaps);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -642,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 2);
-      mbar_init(&empty[i], kComputeWarps);
+      mbar_init(&empty[i], kEmptyArrivals);
     }
     mbar_init(&state[0], kLookThreads);
     mbar_init(&state[1], kLookThreads);
@@ -651,58 +759,76 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   if (tid < kComputeThreads) {
-    // ---- compute warps: phase 1 of tile k, then phase 3 of tile k − 1 ----------------
-    const int g = lane;
-    const int s = tid / 32;
-    for (int k = 0;; ++k) {
-      const int st = k % kStages;
-      if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
-        if (lane == 0) atomicOr(a.status, kStatusTimeout);
-      }
-      const int tile = s_tile[st];
-      const bool valid = tile < a.n_tiles;
-      if (valid) {
-        float* mA = maps_base + (k & 1) * 2 * kSub * CW;
-        phase1<T, kGate, kCoef>(smem + st * Ly::kStage, mA, mA + kSub * CW, coord_of(tile, a), g, s, a);
-      }
-      // the look-back warps learn of the end of the tile sequence through this barrier too
-      bar_arrive_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
-      if (k >= 1) {
-        const int kp = k - 1;
-        const int stp = kp % kStages;
-        if (!mbar_wait_sleep(&state[kp & 1], (uint32_t)(kp >> 1) & 1u)) {
+    {
+      // ---- compute warps: phase 1 of tile k, then phase 3 of tile k − 1 ----------------
+      const int g = lane;
+      const int s = tid / 32;
+      for (int k = 0;; ++k) {
+        const int st = k % kStages;
+        if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
           if (lane == 0) atomicOr(a.status, kStatusTimeout);
         }
-        const float* mH = maps_base + (kp & 1) * 2 * kSub * CW + kSub * CW;
-        phase3<T, kGate, kCoef>(smem + stp * Ly::kStage, mH, coord_of(s_tile[stp], a), g, s, a);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stp]);
+        const TileCoord tc = s_tc[st];
+        const bool valid = tc.chunk >= 0;
+        if (valid) {
+          float* mA = maps_base + (k & 1) * 2 * kSub * CW;
+          if constexpr (kCoef) {
+            CoefRegs r;
+            coef_load<kGate>(smem + st * Ly::kStage, g, s, r);
+            coef_fold<kGate>(r, mA, mA + kSub * CW, tc, g, s, a);
+          } else {
+            phase1<T, kGate>(smem + st * Ly::kStage, mA, mA + kSub * CW, tc, g, s, a);
+          }
+        }
+        if (valid) bar_arrive_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
+        if (k >= 1) {
+          const int kp = k - 1;
+          const int stp = kp % kStages;
+          if (!mbar_wait_sleep(&state[kp & 1], (uint32_t)(kp >> 1) & 1u)) {
+            if (lane == 0) atomicOr(a.status, kStatusTimeout);
+          }
+          const float* mH = maps_base + (kp & 1) * 2 * kSub * CW + kSub * CW;
+          if constexpr (kCoef) {
+            // the coefficients are read again from the stage, which is released only now
+            CoefRegs r;
+            coef_load<kGate>(smem + stp * Ly::kStage, g, s, r);
+            coef_replay<kGate>(r, mH, s_tc[stp], g, s, a);
+          } else {
+            phase3<T, kGate>(smem + stp * Ly::kStage, mH, s_tc[stp], g, s, a);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[stp]);
+        }
+        if (!valid) break;
       }
-      if (!valid) break;
     }
-  } else if (tid < kComputeThreads + kLookThreads) {
+  } else if (tid < kComputeThreads + kGroups * kLookThreads) {
     // ---- look-back warps: the incoming state of tile k is read while its phase 1 runs;
-    // once phase 1 is done the tile's states are finished and published ----------------
-    const int j = tid - kComputeThreads;
-    for (int k = 0;; ++k) {
+    // once phase 1 is done the tile's states are finished and published. Group gr takes
+    // tiles gr, gr + kGroups, ... (the maps barrier, the maps buffer and the state barrier
+    // of tile k all go by k mod 2, so each of two groups has its own) ----------------------
+    const int gr = (tid - kComputeThreads) / kLookThreads;
+    const int j = (tid - kComputeThreads) % kLookThreads;
+    for (int k = gr;; k += kGroups) {
       const int st = k % kStages;
       if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
         if (j == 0) atomicOr(a.status, kStatusTimeout);
       }
-      const int tile = s_tile[st];
+      const TileCoord tc = s_tc[st];
+      const bool valid = tc.chunk >= 0;
+      if (!valid) break;  // the end of this CTA's tiles (the compute warps have left)
       float hin[NCH];
-      if (tile < a.n_tiles) lookback_walk<T, kGate, NCH>(coord_of(tile, a), j, a, hin);
+      uint32_t w[NCH];
+      lookback_begin<T, kGate, NCH>(tc, j, a, w, hin);
       bar_sync_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
-      if (tile >= a.n_tiles) break;
       const float* mA = maps_base + (k & 1) * 2 * kSub * CW;
-      lookback_finish<T, kGate, NCH>(mA, maps_base + (k & 1) * 2 * kSub * CW + kSub * CW, coord_of(tile, a), j, a,
-                                     hin);
+      lookback_finish<T, kGate, NCH>(mA, maps_base + (k & 1) * 2 * kSub * CW + kSub * CW, tc, j, a, w, hin);
       mbar_arrive(&state[k & 1]);
     }
   } else {
     // ---- producer warp: tickets, TMA copies and parameters, two tiles ahead ----------
     if (lane == 0) {
-      tma_prefetch_desc(&maps.x);
+      if constexpr (!kCoef) tma_prefetch_desc(&maps.x);
       tma_prefetch_desc(&maps.z);
     }
     // tickets: t_cur for the tile being loaded, t_nxt for the one after (its parameters
@@ -716,7 +842,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int t_cur = (int)__shfl_sync(0xffffffffu, t0, 0);
     int t_nxt = (int)__shfl_sync(0xffffffffu, t1, 0);
     ParRegs<PV> par;
-    if (t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
+    if (!kCoef && t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
+    int ends = 0;
     for (int jt = 0;; ++jt) {
       const int st = jt % kStages;
       if (jt >= kStages) {
@@ -726,26 +853,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       uint8_t* stage = smem + st * Ly::kStage;
-      if (lane == 0) s_tile[st] = t_cur;
+      if (lane == 0) s_tc[st] = t_cur < a.n_tiles ? coord_of(t_cur, a) : TileCoord{-1, 0, 0, 0};
       if (t_cur >= a.n_tiles) {
-        // end of this CTA's tiles: release the stage with no data
+        // end of this CTA's tiles: release the stage with no data, once for each look-back
+        // group (the compute warps stop at the first)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&full[st]);
           mbar_arrive(&full[st]);
         }
-        break;
+        if (++ends == kGroups) break;
+        continue;
       }
       const TileCoord tc = coord_of(t_cur, a);
-      if (lane == 0) issue_tile_loads<T, kGate>(stage, &full[st], maps, a, tc);
-      store_params<PV>(reinterpret_cast<float*>(stage + Ly::offPar), CW, lane * PV, tc.cblk * CW + lane * PV < a.R,
-                       par);
+      if (lane == 0) issue_tile_loads<T, kGate, kCoef>(stage, &full[st], maps, a, tc);
+      if constexpr (!kCoef)
+        store_params<PV>(reinterpret_cast<float*>(stage + Ly::offPar), CW, lane * PV, tc.cblk * CW + lane * PV < a.R,
+                         par);
       // advance the ticket pipeline and start the next tile's parameter loads
       const int t_new = (int)__shfl_sync(0xffffffffu, pend, 0);
       if (lane == 0) pend = atomicAdd(a.ticket, 1u);
       t_cur = t_nxt;
       t_nxt = t_new;
-      if (t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
+      if (!kCoef && t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);
     }
@@ -758,7 +888,7 @@ std::atomic<int64_t> g_stall_tile{-1};
 // forward-progress argument needs.
 template <typename T, bool kGate, bool kCoef>
 cudaError_t launch_typed(const ScanArgs& a, const ScanMaps& maps, cudaStream_t s) {
-  using Ly = SmemLayout<T, kGate>;
+  using Ly = SmemLayout<T, kGate, kCoef>;
   auto kern = rglru_scan_kernel<T, kGate, kCoef>;
   static bool ready[64] = {false};
   int dev = 0;
@@ -769,13 +899,13 @@ cudaError_t launch_typed(const ScanArgs& a, const ScanMaps& maps, cudaStream_t s
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
     if (e != cudaSuccess) return e;
     int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, Ly::kAlloc);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, threads_of<kCoef>(), Ly::kAlloc);
     if (e != cudaSuccess) return e;
     if (nb < 1) return cudaErrorInvalidConfiguration;
     ready[dev] = true;
   }
   const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)num_sms());
-  kern<<<(unsigned)grid, kThreads, Ly::kAlloc, s>>>(maps, a);
+  kern<<<(unsigned)grid, threads_of<kCoef>(), Ly::kAlloc, s>>>(maps, a);
   return cudaGetLastError();
 }
 
@@ -814,17 +944,14 @@ cudaError_t launch_scan(const ScanArgs& a_in, bool bf16, cudaStream_t s, bool co
   const CUtensorMapDataType dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const int es = bf16 ? 2 : 4;
   const int cw = scan_cw(bf16);
-  {
+  if (!coef) {
+    // the coefficient scan reads no x: the gate GEMM's epilogue already formed b_t from u_t
     cuuint64_t dims[3] = {(cuuint64_t)a.R, (cuuint64_t)a.T, (cuuint64_t)a.B};
     cuuint64_t strides[2] = {(cuuint64_t)a.R * es, (cuuint64_t)a.T * a.R * es};
     cuuint32_t box[3] = {(cuuint32_t)cw, (cuuint32_t)kXRows, 1};
     if (!encode(&maps.x, dt, 3, a.x, dims, strides, box)) return cudaErrorInvalidValue;
-    if (a.g != nullptr) {
-      cuuint32_t gbox[3] = {(cuuint32_t)cw, (cuuint32_t)kScanTC, 1};
-      if (!encode(&maps.g, dt, 3, a.g, dims, strides, gbox)) return cudaErrorInvalidValue;
-    } else {
-      maps.g = maps.x;
-    }
+  } else {
+    memset(&maps.x, 0, sizeof(maps.x));
   }
   {
     cuuint64_t dims[2] = {(cuuint64_t)a.pitch, (cuuint64_t)a.B * a.T};

@@ -270,7 +270,8 @@ def scan(params: Params, x: torch.Tensor, z: torch.Tensor, h0: Optional[torch.Te
 def gate_coeffs(params: Params, u: torch.Tensor, *, g: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """rglru_gate_coeffs: u [N_tok][R] bf16 → packed fp16 recurrence coefficients
-    (d = 1 − a_t in the recurrence-gate places, m = √(1−a_t²)·i_t in the input-gate places)."""
+    (d = 1 − a_t in the recurrence-gate places, b_t = √(1−a_t²)·i_t·u_t in the input-gate
+    places)."""
     lib = _abi.load()
     N, R = u.shape
     g = torch.empty(N, gate_pitch(R), dtype=torch.float16, device=u.device) if g is None else g
@@ -279,21 +280,20 @@ def gate_coeffs(params: Params, u: torch.Tensor, *, g: Optional[torch.Tensor] = 
     return g
 
 
-def scan_coeffs(params: Params, x: torch.Tensor, g: torch.Tensor, h0: Optional[torch.Tensor] = None,
-                conv_state0: Optional[torch.Tensor] = None, gate_g: Optional[torch.Tensor] = None, *,
-                workspace: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-                h_T: Optional[torch.Tensor] = None,
+def scan_coeffs(g: torch.Tensor, B: int, T: int, R: int, h0: Optional[torch.Tensor] = None,
+                gate_g: Optional[torch.Tensor] = None, *, workspace: Optional[torch.Tensor] = None,
+                y: Optional[torch.Tensor] = None, h_T: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """rglru_scan_coeffs: (x bf16, packed coefficients) → (y, h_T)."""
+    """rglru_scan_coeffs: packed coefficients of B·T rows (from gate_coeffs) → (y [B][T][R]
+    bf16, h_T [B][R] float32); needs neither x nor the parameters."""
     lib = _abi.load()
-    B, T, R = x.shape
-    y = torch.empty_like(x) if y is None else y
-    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
-    ws = _workspace(lib.rglru_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16), x.device, workspace)
-    st = params.struct()
+    if g.shape[0] != B * T or g.dtype != torch.float16:
+        raise ValueError("g must be the float16 packed coefficients of B·T rows")
+    y = torch.empty(B, T, R, dtype=torch.bfloat16, device=g.device) if y is None else y
+    h_T = torch.empty(B, R, dtype=torch.float32, device=g.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16), g.device, workspace)
     _abi.check("rglru_scan_coeffs", lib.rglru_scan_coeffs(
-        ctypes.byref(st), _p(x), _p(g), _p(conv_state0), _p(h0), _p(gate_g), _p(y), _p(h_T), B, T, R, _p(ws),
-        ws.numel() * ws.element_size(), _s(stream)))
+        _p(g), _p(h0), _p(gate_g), _p(y), _p(h_T), B, T, R, _p(ws), ws.numel() * ws.element_size(), _s(stream)))
     return y, h_T
 
 

@@ -172,20 +172,23 @@ RGLRU_API int rglru_scan(const rglru_params* params, const void* x, const void* 
  *   epilogue ("Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元,
  *   Eq. (1)–(4)): with z as in rglru_gate_proj, r = σ(z_a), i = σ(z_x),
  *   log a_t = r·c·log σ(Λ), it writes the recurrence coefficients d = 1 − a_t and
- *   m = √(1 − a_t²)·i (so that a_t = 1 − d and the input term is m·u_t) as IEEE fp16 in
- *   the packed layout of z: d in the recurrence-gate places, m in the input-gate places.
+ *   b_t = √(1 − a_t²)·i·u_t (so that h_t = (1 − d)·h_{t−1} + b_t) as IEEE fp16 in the
+ *   packed layout of z: d in the recurrence-gate places, b in the input-gate places. u is
+ *   the bf16 Conv1D output [N_tok][R] (the GEMM's operand; the same u enters b_t).
  *   g is [N_tok][rglru_gate_pitch(R)] fp16, 16-byte aligned. fp16 keeps 11 significant
- *   bits of d, whose relative error multiplies into every carried state.
+ *   bits of d, whose relative error multiplies into every carried state; |b_t| must stay
+ *   below the fp16 maximum 65504 (|u_t| below it is enough, since √(1 − a_t²)·i ≤ 1).
  *
- * rglru_scan_coeffs: rglru_scan for bf16 IO given those coefficients instead of z:
- *   recomputes u from x (fp32), forms a_t = 1 − d and b_t = m·u_t, and runs the chunked
- *   recurrence. Arguments and workspace as rglru_scan with io_dtype = RGLRU_BF16.
+ * rglru_scan_coeffs: the chunked recurrence h_t = (1 − d)·h_{t−1} + b_t over those
+ *   coefficients, for bf16 IO: y_t = h_t, or h_t ⊙ GeLU(gate_g_t) when gate_g is non-NULL,
+ *   and h_T, exactly as rglru_scan. It reads neither x nor the parameters. g [B·T rows] as
+ *   written by rglru_gate_coeffs; h0, gate_g, y, h_T and the workspace as rglru_scan with
+ *   io_dtype = RGLRU_BF16.
  */
 RGLRU_API int rglru_gate_coeffs(const rglru_params* params, const void* u, void* g, int64_t N_tok, int R,
                                 rglru_stream_t stream);
-RGLRU_API int rglru_scan_coeffs(const rglru_params* params, const void* x, const void* g, const void* conv_state0,
-                                const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R,
-                                void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+RGLRU_API int rglru_scan_coeffs(const void* g, const float* h0, const void* gate_g, void* y, float* h_T, int B, int T,
+                                int R, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * rglru_scan without a workspace, for callers that cannot allocate device memory: a

@@ -97,13 +97,14 @@ def test_coefficient_stages_reject_bad_arguments_before_any_launch():
     assert lib.rglru_gate_coeffs(ctypes.byref(p), _fake(0x100004), ok_ptr, 64, 256, None) == -3
     wsb = lib.rglru_scan_workspace_bytes(1, 64, 256, 1)
     ws = _fake(0x200000)
-    call = lambda **kw: lib.rglru_scan_coeffs(kw.get("p", ctypes.byref(p)), kw.get("x", ok_ptr), kw.get("g", ok_ptr),
-                                              None, None, None, kw.get("y", ok_ptr), None, 1, kw.get("T", 64),
-                                              kw.get("R", 256), kw.get("ws", ws), kw.get("wsb", wsb), None)
+    call = lambda **kw: lib.rglru_scan_coeffs(kw.get("g", ok_ptr), kw.get("h0", None), None, kw.get("y", ok_ptr),
+                                              None, 1, kw.get("T", 64), kw.get("R", 256), kw.get("ws", ws),
+                                              kw.get("wsb", wsb), None)
     assert call(R=12) == -2
     assert call(T=0) == -2
     assert call(g=None) == -1
     assert call(y=_fake(0x100008)) == -3
+    assert call(h0=_fake(0x100004)) == -3
     assert call(ws=None) == -5
     assert call(wsb=wsb - 1) == -5
 

@@ -70,19 +70,19 @@ def test_gate_projection_matches_oracle(dtype, N, R):
 
 @pytest.mark.parametrize("N,R", [(300, 136), (1024, 512), (129, 264)])
 def test_gate_coeffs_match_oracle(N, R):
-    """rglru_gate_coeffs: d = 1 − a_t and m = √(1−a_t²)·i_t (fp16) in the packed places."""
+    """rglru_gate_coeffs: d = 1 − a_t and b_t = √(1−a_t²)·i_t·u_t (fp16) in the packed places."""
     w = _wl(1, N, R, torch.bfloat16)
     p = rglru.Params.from_host(w.params)
     g = torch.Generator("cpu").manual_seed(5)
     u = torch.randn(N, R, generator=g).to(torch.bfloat16)
     co = rglru.gate_coeffs(p, u.to(DEV))
     assert co.dtype == torch.float16
-    d, m = unpack_gates(co, R)
+    d, b = unpack_gates(co, R)
     za, zx = oracle.gate_preactivations(u, w.params.W_a, w.params.b_a, w.params.W_x, w.params.b_x)
     a_t = oracle.decay_log_space(oracle.sigmoid(za), w.params.Lambda)
     d_o = 1.0 - a_t
-    m_o = np.sqrt(1.0 - a_t * a_t) * oracle.sigmoid(zx)
-    assert rel(d, d_o) <= 1e-2 and rel(m, m_o) <= 1e-2
+    b_o = np.sqrt(1.0 - a_t * a_t) * oracle.sigmoid(zx) * f64(u)
+    assert rel(d, d_o) <= 1e-2 and rel(b, b_o) <= 1e-2
 
 
 def test_coeff_stages_equal_forward():
@@ -95,7 +95,7 @@ def test_coeff_stages_equal_forward():
     y_f, h_f, _ = rglru.forward(p, x, h0)
     u = rglru.conv1d(p, x)
     co = rglru.gate_coeffs(p, u.view(B * T, R))
-    y_s, h_s = rglru.scan_coeffs(p, x, co, h0)
+    y_s, h_s = rglru.scan_coeffs(co, B, T, R, h0)
     assert torch.equal(y_f, y_s) and torch.equal(h_f, h_s)
 
 
