@@ -25,24 +25,29 @@
 //                    z_a and z_x, plus the tile's parameters (taps, conv bias, c·log σ(Λ))
 //                    written into the stage — or only the two coefficient blocks — and the
 //                    tile's decoded coordinates;
-//   compute warps    (16, one per sub-chunk; lane = channel group), for tile k:
+//   compute warps    (16, one per sub-chunk of 4 steps; lane = channel group; the
+//                    coefficient form splits them into two groups of 8 on alternate tiles,
+//                    one per sub-chunk of 8 steps), for tile k:
 //     phase 1  recompute u in float32, apply the gates and the log-space decay (or read
 //              the coefficients), fold the sub-chunk's 4 steps into an affine map
 //              (float32); the pre-activation form writes the per-step replay values
 //              (1 − a_t, b_t) over the z_a, z_x slots they came from;
-//     phase 3  (of tile k − 1, whose incoming states are ready by now) replay the
-//              sub-chunk from its incoming state and write y, then release the stage;
+//     phase 3  (of the group's previous tile, whose incoming states are ready by now)
+//              replay the sub-chunk from its incoming state and write y, then release
+//              the stage;
 //   look-back warps  (groups of 2 warps, two channels per thread for bf16; the coefficient
 //                    form has two groups taking alternate tiles) read the state entering
 //                    tile k — the inclusive state its predecessor chunk publishes, or h0 —
-//                    while phase 1 of tile k runs; once the 16 sub-chunk maps are in, they
+//                    while phase 1 of tile k runs; once the sub-chunk maps are in, they
 //                    compose them, publish the tile's inclusive state and hand every
 //                    sub-chunk its incoming state. A published state is a self-validating
 //                    word (an exact XOR encoding whose zero is never a published value, so
 //                    zeroed memory reads as "not yet"): one relaxed load, no fence or flag.
 // Every wait is bounded. Warps of different roles meet at mbarriers (stage full / empty,
-// states ready) and at one named barrier (maps ready) whose id alternates with the tile's
-// parity; the compute warps never wait for one another.
+// states ready) and at a named barrier (maps ready); map buffers, maps barriers and states
+// barriers rotate with the tile number (mod 2, or mod 4 for two compute groups) so that
+// none is reused before every role is done with it. The compute warps never wait for one
+// another.
 // The replay values of the pre-activation bf16 path are stored as bf16 (1 − a_t, b_t): their
 // rounding only touches y inside one 4-step sub-chunk, while the published states and h_T
 // come from the float32 maps. The coefficients are fp16 (11 significant bits); everything
@@ -80,6 +85,11 @@ constexpr int kSub = kScanSub;                        // sub-chunks: one compute
 constexpr int kL = kScanTC / kSub;                    // steps per sub-chunk
 constexpr int kComputeWarps = kSub;                   // 16
 constexpr int kComputeThreads = kGroups * kSub;       // 512
+// The coefficient scan splits its compute warps into two groups of 8 that take alternate
+// tiles; a warp then folds and replays 8 steps, so a tile has 8 sub-chunk maps, not 16.
+constexpr int kLC = 8;                                // steps per coefficient sub-chunk
+constexpr int kSubC = kScanTC / kLC;                  // 8 sub-chunks: one warp of the group each
+static_assert(2 * kSubC == kComputeWarps, "two compute groups");
 // Look-back groups of two warps: the coefficient scan's tiles are short, so two groups take
 // alternate tiles (tile k goes to group k mod 2) and one tile's look-back overlaps the next
 // one's. (Its 21 warps put 6 on some scheduler partition, which leaves a thread 80
@@ -89,15 +99,17 @@ template <bool kCoef> constexpr int look_threads() { return 64; }  // per group
 template <bool kCoef> constexpr int threads_of() {
   return kComputeThreads + look_groups<kCoef>() * look_threads<kCoef>() + 32;  // + one producer warp
 }
-// named barrier (id 0 is __syncthreads, which the roles never use after the prologue):
-// + tile parity; compute warps arrive once phase 1 is done, look-back warps wait
+// named barriers (id 0 is __syncthreads, which the roles never use after the prologue):
+// kBarMaps + (tile k mod 2, or mod 4 for two compute groups); compute warps arrive once
+// phase 1 is done, look-back warps wait
 constexpr int kBarMaps = 1;
 
 // kCoef: the stage holds only the two coefficient blocks (d = 1 − a_t, b_t; fp16), which
 // need neither x nor parameters, so the ring is deeper.
 template <typename T, bool kGate, bool kCoef = false> struct SmemLayout {
   static constexpr int CW = kGroups * SV<T>::V;
-  static constexpr int kStages = kCoef ? 5 : 3;
+  static constexpr int kStages = kCoef ? 6 : 3;
+  static constexpr int kSubs = kCoef ? kSubC : kSub;   // sub-chunk maps per tile
   static constexpr int kX = kCoef ? 0 : kXRows * CW * (int)sizeof(T);
   static constexpr int kZ = kScanTC * CW * (int)sizeof(T);
   // a stage: x rows, z_a, z_x (TMA), then the tile's parameters [6][CW] f32 (taps 0..3,
@@ -106,9 +118,15 @@ template <typename T, bool kGate, bool kCoef = false> struct SmemLayout {
   static constexpr int offZX = kX + kZ;
   static constexpr int offPar = kX + 2 * kZ;
   static constexpr int kStage = offPar + (kCoef ? 0 : 6 * CW * 4);
-  static constexpr int offMaps = kStages * kStage;     // [2 buffers][A | B][kSub][CW] f32
-  static constexpr int kMaps = 2 * kSub * CW * 4;
-  static constexpr int kBytes = offMaps + 2 * kMaps;
+  // Tile k uses map buffer, maps barrier and states barrier number k mod kMapBufs. Each is
+  // in use from the tile's phase 1 until its phase 3 has read the handed-out states, and a
+  // role reaches the next tile with the same number only after that: with one compute
+  // group, tile k + 2 starts phase 1 after phase 3 of tile k; with two groups (each on
+  // every other tile) that holds for tile k + 4, so each group needs two of each.
+  static constexpr int kMapBufs = kCoef ? 4 : 2;
+  static constexpr int offMaps = kStages * kStage;     // [kMapBufs][A | B][kSubs][CW] f32
+  static constexpr int kMaps = 2 * kSubs * CW * 4;
+  static constexpr int kBytes = offMaps + kMapBufs * kMaps;
   static constexpr int kAlloc = kBytes + 128;          // slack to align the base to 128 bytes
   static constexpr uint32_t kTxXZ = kX + 2 * kZ;
   static_assert(kX % 128 == 0 && kStage % 128 == 0, "TMA destinations 128-byte aligned");
@@ -433,10 +451,10 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
   stf<V>(mB + s * CW + cc, B);
 }
 
-// The coefficients of one tile as one compute thread holds them between its two phases:
-// kL steps × 4 channels of d and of b, as packed fp16 pairs (bf16 IO only).
+// The coefficients of one sub-chunk as one compute thread holds them: kLC steps × 4
+// channels of d and of b, as packed fp16 pairs (bf16 IO only).
 struct CoefRegs {
-  uint32_t d[kL][2], b[kL][2];
+  uint32_t d[kLC][2], b[kLC][2];
 };
 
 // Reads the thread's coefficients of the tile out of the stage (after which the stage may
@@ -449,8 +467,8 @@ __device__ __forceinline__ void coef_load(const uint8_t* stage, int g, int s, Co
   const __half* sb = reinterpret_cast<const __half*>(stage + Ly::offZX);
   const int cc = g * 4;
 #pragma unroll
-  for (int l = 0; l < kL; ++l) {
-    const int row = s * kL + l;
+  for (int l = 0; l < kLC; ++l) {
+    const int row = s * kLC + l;
     const uint2 vd = *reinterpret_cast<const uint2*>(sd + row * CW + cc);
     const uint2 vb = *reinterpret_cast<const uint2*>(sb + row * CW + cc);
     r.d[l][0] = vd.x; r.d[l][1] = vd.y;
@@ -468,12 +486,12 @@ __device__ __forceinline__ void coef_fold(const CoefRegs& r, float* mA, float* m
                                           const ScanArgs& a) {
   constexpr int CW = SmemLayout<__nv_bfloat16, kGate, true>::CW;
   const int cc = g * 4;
-  const int t_start = tc.chunk * kScanTC + s * kL;
+  const int t_start = tc.chunk * kScanTC + s * kLC;
   float2 A[2] = {make_float2(1.0f, 1.0f), make_float2(1.0f, 1.0f)};
   float2 B[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-  const bool whole = t_start + kL <= a.T;
+  const bool whole = t_start + kLC <= a.T;
 #pragma unroll
-  for (int l = 0; l < kL; ++l) {
+  for (int l = 0; l < kLC; ++l) {
     if (whole || t_start + l < a.T) {
 #pragma unroll
       for (int p = 0; p < 2; ++p) {
@@ -488,46 +506,62 @@ __device__ __forceinline__ void coef_fold(const CoefRegs& r, float* mA, float* m
   *reinterpret_cast<float4*>(mB + s * CW + cc) = make_float4(B[0].x, B[0].y, B[1].x, B[1].y);
 }
 
-// Phase 3 of the coefficient scan from registers: replay the sub-chunk from its incoming
-// state (mH) and write y (times GeLU of the gate branch for the gated scan).
+// Phase 3 of the coefficient scan: replay the sub-chunk from its incoming state (mH) with
+// the coefficients read again from the stage, and write y (times GeLU of the gate branch
+// for the gated scan). The 8 steps go in two halves, each with its coefficient and gate
+// loads issued before its arithmetic, so that at most half of them are held at a time.
 template <bool kGate>
-__device__ __forceinline__ void coef_replay(const CoefRegs& r, const float* mH, const TileCoord& tc, int g, int s,
+__device__ __forceinline__ void coef_replay(const uint8_t* stage, const float* mH, const TileCoord& tc, int g, int s,
                                             const ScanArgs& a) {
-  constexpr int CW = SmemLayout<__nv_bfloat16, kGate, true>::CW;
+  using Ly = SmemLayout<__nv_bfloat16, kGate, true>;
+  constexpr int CW = Ly::CW;
+  constexpr int kHalf = kLC / 2;
+  const __half* sd = reinterpret_cast<const __half*>(stage + Ly::offZA);
+  const __half* sb = reinterpret_cast<const __half*>(stage + Ly::offZX);
   const int cc = g * 4;
   const int c0 = tc.cblk * CW + cc;
-  const int t_start = tc.chunk * kScanTC + s * kL;
-  float gg[kGate ? kL : 1][4];
-  if constexpr (kGate) {
-    const __nv_bfloat16* gsrc = static_cast<const __nv_bfloat16*>(a.g);
-#pragma unroll
-    for (int l = 0; l < kL; ++l) {
-#pragma unroll
-      for (int v = 0; v < 4; ++v) gg[l][v] = 0.0f;
-      if (c0 < a.R && t_start + l < a.T) ldv_nc(gsrc + ((int64_t)tc.b * a.T + t_start + l) * a.R + c0, gg[l]);
-    }
-  }
+  const int t_start = tc.chunk * kScanTC + s * kLC;
   const float4 h4 = *reinterpret_cast<const float4*>(mH + s * CW + cc);
-  if (c0 >= a.R) return;
   float2 h[2] = {make_float2(h4.x, h4.y), make_float2(h4.z, h4.w)};
   __nv_bfloat16* __restrict__ y = static_cast<__nv_bfloat16*>(a.y);
+  const bool in_range = c0 < a.R;
 #pragma unroll
-  for (int l = 0; l < kL; ++l) {
-    float o[4];
+  for (int l0 = 0; l0 < kLC; l0 += kHalf) {
+    uint32_t d[kHalf][2], b[kHalf][2];
+    float gg[kGate ? kHalf : 1][4];
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      const float2 d2 = h2f(r.d[l][p]);
-      const float2 a2 = make_float2(1.0f - d2.x, 1.0f - d2.y);
-      h[p] = __ffma2_rn(a2, h[p], h2f(r.b[l][p]));
-      o[2 * p] = h[p].x;
-      o[2 * p + 1] = h[p].y;
+    for (int l = 0; l < kHalf; ++l) {
+      const int row = s * kLC + l0 + l;
+      const uint2 vd = *reinterpret_cast<const uint2*>(sd + row * CW + cc);
+      const uint2 vb = *reinterpret_cast<const uint2*>(sb + row * CW + cc);
+      d[l][0] = vd.x; d[l][1] = vd.y;
+      b[l][0] = vb.x; b[l][1] = vb.y;
+      if constexpr (kGate) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) gg[l][v] = 0.0f;
+        const int t = t_start + l0 + l;
+        if (in_range && t < a.T)
+          ldv_nc(static_cast<const __nv_bfloat16*>(a.g) + ((int64_t)tc.b * a.T + t) * a.R + c0, gg[l]);
+      }
     }
-    if constexpr (kGate) {
 #pragma unroll
-      for (int v = 0; v < 4; ++v) o[v] *= gelu_exact(gg[l][v]);
+    for (int l = 0; l < kHalf; ++l) {
+      float o[4];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float2 d2 = h2f(d[l][p]);
+        const float2 a2 = make_float2(1.0f - d2.x, 1.0f - d2.y);
+        h[p] = __ffma2_rn(a2, h[p], h2f(b[l][p]));
+        o[2 * p] = h[p].x;
+        o[2 * p + 1] = h[p].y;
+      }
+      if constexpr (kGate) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) o[v] *= gelu_exact(gg[l][v]);
+      }
+      const int t = t_start + l0 + l;
+      if (in_range && t < a.T) stv_cs(y + ((int64_t)tc.b * a.T + t) * a.R + c0, o);
     }
-    const int t = t_start + l;
-    if (t < a.T) stv_cs(y + ((int64_t)tc.b * a.T + t) * a.R + c0, o);
   }
 }
 
@@ -670,18 +704,17 @@ __device__ __forceinline__ void lookback_end(const TileCoord& tc, int j, const S
   for (int n = 0; n < NCH; ++n) hin[n] = w[n] != 0u ? dec(w[n]) : 0.0f;
 }
 
-// Look-back, second half, once phase 1 of the tile is done: composes the 16 sub-chunk maps
+// Look-back, second half, once phase 1 of the tile is done: composes the S sub-chunk maps
 // (mA, mB) into the tile's map, waits for the incoming state, publishes the tile's inclusive
 // state A·h_in + B at once (the next chunk waits for it), writes h_T for the last chunk, and
 // then leaves each sub-chunk's incoming state in mB. mA and mB are separate buffers and each
 // slot is read before it is overwritten, so the reads of the second pass need not wait for
 // its stores.
-template <typename T, bool kGate, int NCH>
+template <typename T, bool kGate, int NCH, int S>
 __device__ __forceinline__ void lookback_finish(const float* __restrict__ mA, float* __restrict__ mB,
                                                 const TileCoord& tc, int j, const ScanArgs& a, uint32_t (&w)[NCH],
                                                 float (&hin)[NCH]) {
   constexpr int CW = SmemLayout<T, kGate>::CW;
-  constexpr int S = kSub;
   constexpr int kStride = CW / NCH;
   const bool publish = tc.tix != a.stall_tile;
   float A[NCH], Bv[NCH];
@@ -731,7 +764,12 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
   // warps have read its tile index
   constexpr int kGroups = look_groups<kCoef>();
   constexpr int kLookThreads = look_threads<kCoef>();
-  constexpr int kEmptyArrivals = kComputeWarps;
+  constexpr int kSubs = Ly::kSubs;  // sub-chunk maps per tile
+  // each tile is folded and replayed by all 16 compute warps, or for the coefficient scan
+  // by one group of 8 (tile k by group k mod 2)
+  constexpr int kTileWarps = kCoef ? kSubC : kComputeWarps;
+  constexpr int kEmptyArrivals = kTileWarps;
+  constexpr int kMapsBar = kTileWarps * 32 + kLookThreads;  // maps barrier participants
   constexpr int CW = Ly::CW;
   constexpr int PV = CW / 32;  // channels per producer lane
   constexpr int NCH = CW / kLookThreads;  // channels per look-back thread
@@ -741,7 +779,7 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   __shared__ __align__(8) uint64_t full[kStages];   // TMA bytes + the producer's parameters
   __shared__ __align__(8) uint64_t empty[kStages];  // one arrival per compute warp after phase 3
-  __shared__ __align__(8) uint64_t state[2];        // + tile parity: incoming states ready
+  __shared__ __align__(8) uint64_t state[Ly::kMapBufs];  // tile k mod kMapBufs: incoming states ready
   __shared__ TileCoord s_tc[kStages];               // the tile in each stage (decoded once)
   float* maps_base = reinterpret_cast<float*>(smem + Ly::offMaps);
   const int tid = threadIdx.x;
@@ -752,55 +790,55 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
       mbar_init(&full[i], 2);
       mbar_init(&empty[i], kEmptyArrivals);
     }
-    mbar_init(&state[0], kLookThreads);
-    mbar_init(&state[1], kLookThreads);
+    for (int i = 0; i < Ly::kMapBufs; ++i) mbar_init(&state[i], kLookThreads);
     fence_barrier_init();
   }
   __syncthreads();
 
   if (tid < kComputeThreads) {
-    {
-      // ---- compute warps: phase 1 of tile k, then phase 3 of tile k − 1 ----------------
-      const int g = lane;
-      const int s = tid / 32;
-      for (int k = 0;; ++k) {
-        const int st = k % kStages;
-        if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
+    // ---- compute warps: phase 1 of tile k, then phase 3 of the group's previous tile ----
+    // (all 16 warps on every tile, sub-chunk = warp; or for the coefficient scan, group
+    // cg = warp / 8 on tiles cg, cg + 2, ..., sub-chunk = warp % 8)
+    const int g = lane;
+    const int warp = tid / 32;
+    const int s = kCoef ? warp % kSubC : warp;
+    const int k0 = kCoef ? warp / kSubC : 0;
+    constexpr int dk = kCoef ? 2 : 1;
+    for (int k = k0;; k += dk) {
+      const int st = k % kStages;
+      if (!mbar_wait_sleep(&full[st], (uint32_t)(k / kStages) & 1u)) {
+        if (lane == 0) atomicOr(a.status, kStatusTimeout);
+      }
+      const TileCoord tc = s_tc[st];
+      const bool valid = tc.chunk >= 0;
+      if (valid) {
+        float* mA = maps_base + (k % Ly::kMapBufs) * 2 * kSubs * CW;
+        if constexpr (kCoef) {
+          CoefRegs r;
+          coef_load<kGate>(smem + st * Ly::kStage, g, s, r);
+          coef_fold<kGate>(r, mA, mA + kSubs * CW, tc, g, s, a);
+        } else {
+          phase1<T, kGate>(smem + st * Ly::kStage, mA, mA + kSubs * CW, tc, g, s, a);
+        }
+        bar_arrive_n(kBarMaps + k % Ly::kMapBufs, kMapsBar);
+      }
+      if (k >= dk) {
+        const int kp = k - dk;
+        const int stp = kp % kStages;
+        if (!mbar_wait_sleep(&state[kp % Ly::kMapBufs], (uint32_t)(kp / Ly::kMapBufs) & 1u)) {
           if (lane == 0) atomicOr(a.status, kStatusTimeout);
         }
-        const TileCoord tc = s_tc[st];
-        const bool valid = tc.chunk >= 0;
-        if (valid) {
-          float* mA = maps_base + (k & 1) * 2 * kSub * CW;
-          if constexpr (kCoef) {
-            CoefRegs r;
-            coef_load<kGate>(smem + st * Ly::kStage, g, s, r);
-            coef_fold<kGate>(r, mA, mA + kSub * CW, tc, g, s, a);
-          } else {
-            phase1<T, kGate>(smem + st * Ly::kStage, mA, mA + kSub * CW, tc, g, s, a);
-          }
+        const float* mH = maps_base + (kp % Ly::kMapBufs) * 2 * kSubs * CW + kSubs * CW;
+        if constexpr (kCoef) {
+          // the coefficients are read again from the stage, which is released only now
+          coef_replay<kGate>(smem + stp * Ly::kStage, mH, s_tc[stp], g, s, a);
+        } else {
+          phase3<T, kGate>(smem + stp * Ly::kStage, mH, s_tc[stp], g, s, a);
         }
-        if (valid) bar_arrive_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
-        if (k >= 1) {
-          const int kp = k - 1;
-          const int stp = kp % kStages;
-          if (!mbar_wait_sleep(&state[kp & 1], (uint32_t)(kp >> 1) & 1u)) {
-            if (lane == 0) atomicOr(a.status, kStatusTimeout);
-          }
-          const float* mH = maps_base + (kp & 1) * 2 * kSub * CW + kSub * CW;
-          if constexpr (kCoef) {
-            // the coefficients are read again from the stage, which is released only now
-            CoefRegs r;
-            coef_load<kGate>(smem + stp * Ly::kStage, g, s, r);
-            coef_replay<kGate>(r, mH, s_tc[stp], g, s, a);
-          } else {
-            phase3<T, kGate>(smem + stp * Ly::kStage, mH, s_tc[stp], g, s, a);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[stp]);
-        }
-        if (!valid) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stp]);
       }
+      if (!valid) break;
     }
   } else if (tid < kComputeThreads + kGroups * kLookThreads) {
     // ---- look-back warps: the incoming state of tile k is read while its phase 1 runs;
@@ -820,10 +858,10 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
       float hin[NCH];
       uint32_t w[NCH];
       lookback_begin<T, kGate, NCH>(tc, j, a, w, hin);
-      bar_sync_n(kBarMaps + (k & 1), kComputeThreads + kLookThreads);
-      const float* mA = maps_base + (k & 1) * 2 * kSub * CW;
-      lookback_finish<T, kGate, NCH>(mA, maps_base + (k & 1) * 2 * kSub * CW + kSub * CW, tc, j, a, w, hin);
-      mbar_arrive(&state[k & 1]);
+      bar_sync_n(kBarMaps + k % Ly::kMapBufs, kMapsBar);
+      float* mA = maps_base + (k % Ly::kMapBufs) * 2 * kSubs * CW;
+      lookback_finish<T, kGate, NCH, kSubs>(mA, mA + kSubs * CW, tc, j, a, w, hin);
+      mbar_arrive(&state[k % Ly::kMapBufs]);
     }
   } else {
     // ---- producer warp: tickets, TMA copies and parameters, two tiles ahead ----------
