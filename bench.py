@@ -4,12 +4,14 @@
 
 Own arm. One step = one forward pass of the layer over one batch of the Hawk-scale
 workload B=8, T=2048, D_RNN=2048, bf16 IO with float32 state, inputs resident in HBM, L2
-flushed (256 MB write) before every timed step. The step calls the three stages of
-rglru_forward one by one through the C ABI — Conv1D(4), the gate GEMM, the fused gates +
-log-space decay + chunked scan — the same launches rglru_forward makes, so that each
-kernel's duration is measured with CUDA events on its own stream. The alternative second
-stage (gate GEMM with the scan in its epilogue, rglru_gate_scan) is timed in a second loop
-and is not part of the step.
+flushed (256 MB write) before every timed step. The step is one rglru_forward call
+through the C ABI: Conv1D(4) (which also zeroes the scan's workspace), the gate GEMM that
+forms the recurrence coefficients, and the coefficient scan, the last two launched as
+programmatic dependents of the kernel before. A second loop launches the same three
+kernels one stage call at a time (the scan's call adds its workspace memset) so that each
+kernel's duration is measured with CUDA events. The alternative second stage (gate GEMM
+with the scan in its epilogue, rglru_gate_scan) is timed in a third loop and is not part
+of the step.
 Reported: tokens/s (all ranks), per-kernel achieved bandwidth / throughput and their
 fractions of the measured B200 peaks, the roofline of the dominant kernel, the same
 metric end to end through the public API with host buffers (pinned H2D of x, D2H of y
@@ -148,6 +150,7 @@ def run_own(args):
     z = torch.empty(B * T, rglru.gate_pitch(R), dtype=torch.float16, device=dev)  # packed coefficients
     ws_gs = torch.empty(rglru.gate_scan_workspace_bytes(B, T, R), dtype=torch.uint8, device=dev)
     ws_scan = torch.empty(rglru.scan_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
+    ws_fwd = torch.empty(rglru.forward_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -164,9 +167,15 @@ def run_own(args):
             print(json.dumps({"only": "block", "block": blk}))
         return
 
+    def forward_step():
+        # the timed step: one rglru_forward call (conv, gate GEMM forming the recurrence
+        # coefficients, coefficient scan; the last two launched as programmatic dependents)
+        rglru.forward(p, x, workspace=ws_fwd, y=y, h_T=h_T, want_conv_state=False)
+
     def step(ev=None):
-        # exactly the launches rglru_forward makes for bf16: conv, gate GEMM forming the
-        # recurrence coefficients, fused scan
+        # the same three kernels through the stage entry points, for the per-kernel times
+        # (the scan's interval also holds its workspace memset, which rglru_forward leaves
+        # to the conv kernel)
         if ev is not None:
             ev[0].record(stream)
         rglru.conv1d(p, x, u=u)
@@ -187,28 +196,40 @@ def run_own(args):
 
     for _ in range(args.warmup):
         flush.zero_()
+        forward_step()
+        flush.zero_()
         step()
     torch.cuda.synchronize()
-    if rglru.workspace_status(ws_scan) != 0 or rglru.workspace_status(None) != 0:
+    if (rglru.workspace_status(ws_scan) != 0 or rglru.workspace_status(ws_fwd) != 0
+            or rglru.workspace_status(None) != 0):
         raise SystemExit("a kernel reported a timeout during warm-up")
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
     for k in range(K):
         flush.zero_()                 # L2 flush between timed steps (outside the events)
-        step(evs[k])
+        fevs[k][0].record(stream)
+        forward_step()
+        fevs[k][1].record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
+    step_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in fevs) / K)
+    status = rglru.workspace_status(ws_fwd)
+    # per-kernel times: the same kernels launched one stage call at a time
+    for k in range(K):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
     conv_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
     gemm_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
     scan_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
-    step_ms = max_over_ranks(sum(e[0].elapsed_time(e[3]) for e in evs) / K)
-    status = rglru.workspace_status(ws_scan)
+    status = status or rglru.workspace_status(ws_scan)
 
     # the fused gate GEMM + scan stage (not part of the timed forward step)
     for _ in range(3):

@@ -73,7 +73,8 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const __grid_
                                                                   const float* __restrict__ conv_b,
                                                                   const T* __restrict__ state0, T* __restrict__ u,
                                                                   T* __restrict__ stateT, int B, int T_, int R,
-                                                                  int n_cblk, int n_chunks, unsigned* status) {
+                                                                  int n_cblk, int n_chunks, unsigned* status,
+                                                                  uint4* __restrict__ zero, int64_t zero_n16) {
   constexpr int V = CV<T>::N;
   constexpr int CW = 16 * V;
   constexpr int kStage = kTileRows * CW * (int)sizeof(T);
@@ -82,6 +83,13 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const __grid_
   __shared__ __align__(8) uint64_t full[kConvStages];
 
   const int tid = threadIdx.x;
+  // the next kernel (launched as a programmatic dependent) may be scheduled from now on
+  pdl_launch_dependents();
+  // zero the scan's workspace header and carries for the kernels after this one (saves a
+  // separate memset launch); its status word is set only after a wait of about a second,
+  // long after every CTA of this grid has passed this point
+  for (int64_t i = (int64_t)blockIdx.x * kTileThreads + tid; i < zero_n16; i += (int64_t)gridDim.x * kTileThreads)
+    zero[i] = make_uint4(0u, 0u, 0u, 0u);
   const int g = tid % 16, s = tid / 16;
   const int cblk = blockIdx.x % n_cblk;
   const int lane0 = blockIdx.x / n_cblk;         // first (b, chunk) pair of this CTA
@@ -197,7 +205,7 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
                                                                   int R) {
   constexpr int V = 8;
   // the step GEMM that follows may start its prologue now; it waits for this grid's results
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_launch_dependents();
   const int c0 = (blockIdx.x * kConvThreads + threadIdx.x) * V;
   const int b = blockIdx.y;
   if (blockIdx.x == 0 && b == 0 && threadIdx.x == 0) *status = 0u;
@@ -246,7 +254,10 @@ __global__ void __launch_bounds__(kConvThreads) decode_conv_kernel(const float* 
 }  // namespace
 
 cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* state0, void* u,
-                          void* stateT, int B, int T, int R, bool bf16, unsigned* status, cudaStream_t s) {
+                          void* stateT, int B, int T, int R, bool bf16, unsigned* status, cudaStream_t s, void* zero,
+                          size_t zero_bytes) {
+  if (zero_bytes % 16 != 0 || (zero_bytes != 0 && (reinterpret_cast<uintptr_t>(zero) & 15) != 0))
+    return cudaErrorInvalidValue;
   const int es = bf16 ? 2 : 4;
   const int cw = bf16 ? 128 : 64;
   const int n_cblk = (R + cw - 1) / cw;
@@ -285,11 +296,12 @@ cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* 
   if (bf16)
     conv1d_tile_kernel<__nv_bfloat16><<<(unsigned)grid, kTileThreads, smem, s>>>(
         mx, conv_w, conv_b, static_cast<const __nv_bfloat16*>(state0), static_cast<__nv_bfloat16*>(u),
-        static_cast<__nv_bfloat16*>(stateT), B, T, R, n_cblk, n_chunks, status);
+        static_cast<__nv_bfloat16*>(stateT), B, T, R, n_cblk, n_chunks, status, static_cast<uint4*>(zero),
+        (int64_t)(zero_bytes / 16));
   else
     conv1d_tile_kernel<float><<<(unsigned)grid, kTileThreads, smem, s>>>(
         mx, conv_w, conv_b, static_cast<const float*>(state0), static_cast<float*>(u), static_cast<float*>(stateT), B,
-        T, R, n_cblk, n_chunks, status);
+        T, R, n_cblk, n_chunks, status, static_cast<uint4*>(zero), (int64_t)(zero_bytes / 16));
   return cudaGetLastError();
 }
 

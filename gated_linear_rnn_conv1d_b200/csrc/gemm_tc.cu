@@ -503,6 +503,10 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
+  // launched as a programmatic dependent: everything above overlapped the previous kernel;
+  // its results (the A operand, or anything else an epilogue reads) are visible from here
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tmem_base = tmem_base_s;
   const int k_blocks = (K + BK - 1) / BK;
   const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), 0);
@@ -992,7 +996,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), pair_leader);
   // launched as a programmatic dependent of the decode conv kernel: everything above
   // overlapped it; u_t, u_t in float32 and c·log σ(Λ) are its results
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
 
   // The state update's inputs do not depend on the GEMM: every thread loads its u_t and h
   // values now and holds them in registers through the mainloop. Thread t updates channel
@@ -1179,13 +1183,15 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   cfg.blockDim = dim3(threads_of<EPI>());
   cfg.dynamicSmemBytes = smem_of<EPI>();
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits (pdl_wait)
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, a, b0, b1, M, K, n_tiles_n, (int)tiles, ep, status);
 }
 

@@ -56,8 +56,11 @@ int64_t scan_stall();
 cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s, bool coef = false);
 
 // ---- conv --------------------------------------------------------------------------
+// zero/zero_bytes (16-byte aligned, a multiple of 16): a region the kernel also zeroes (the
+// scan workspace of the same forward), or none.
 cudaError_t launch_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* state0, void* u,
-                          void* stateT, int B, int T, int R, bool bf16, unsigned* status, cudaStream_t s);
+                          void* stateT, int B, int T, int R, bool bf16, unsigned* status, cudaStream_t s,
+                          void* zero = nullptr, size_t zero_bytes = 0);
 // Also zeroes *status (the step's status word) before the step's GEMM may set it.
 cudaError_t launch_decode_conv(const float* conv_w, const float* conv_b, const float* Lambda, const void* x_t,
                                void* ring, int64_t step, void* u_t, float* u_f32, float* cla, unsigned* status,

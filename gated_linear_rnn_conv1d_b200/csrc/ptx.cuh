@@ -91,6 +91,16 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) 
   }
 }
 
+// ---- programmatic dependent launch ------------------------------------------------
+// A kernel launched with cudaLaunchAttributeProgrammaticStreamSerialization may start
+// before the previous kernel in its stream has finished; it must call pdl_wait() before it
+// touches memory that kernel (or any earlier one) writes. pdl_launch_dependents() lets the
+// next such kernel start as soon as resources allow.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- TMA (cp.async.bulk.tensor), no multicast -------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -377,11 +377,11 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   void* u = bytes(workspace) + L.off_u;
   void* z = bytes(workspace) + L.off_z;
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
-  // status word, ticket and flags are zeroed before the first kernel, so that a status bit
-  // set by the GEMM survives until the caller reads it.
-  cudaError_t e = cudaMemsetAsync(workspace, 0, L.scan.zero_bytes, s);
-  if (e != cudaSuccess) return fail_cuda(e);
-  e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, status, s);
+  // the conv kernel also zeroes the status word, the scan's ticket and its chunk carries,
+  // so that a status bit set by the GEMM or the scan survives until the caller reads it;
+  // the GEMM and the scan are launched as programmatic dependents of the kernel before
+  cudaError_t e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, bf16, status,
+                                s, workspace, L.scan.zero_bytes);
   if (e != cudaSuccess) return fail_cuda(e);
   // bf16: the gate GEMM's epilogue forms the recurrence coefficients (d, b) directly
   if (bf16)

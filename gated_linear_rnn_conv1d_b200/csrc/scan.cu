@@ -794,6 +794,10 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
     fence_barrier_init();
   }
   __syncthreads();
+  // launched as a programmatic dependent: the inputs and the zeroed workspace of the
+  // kernels before are visible from here
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (tid < kComputeThreads) {
     // ---- compute warps: phase 1 of tile k, then phase 3 of the group's previous tile ----
@@ -943,8 +947,17 @@ cudaError_t launch_typed(const ScanArgs& a, const ScanMaps& maps, cudaStream_t s
     ready[dev] = true;
   }
   const int64_t grid = std::min<int64_t>(a.n_tiles, (int64_t)num_sms());
-  kern<<<(unsigned)grid, threads_of<kCoef>(), Ly::kAlloc, s>>>(maps, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(threads_of<kCoef>());
+  cfg.dynamicSmemBytes = Ly::kAlloc;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // the kernel waits (pdl_wait)
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, maps, a);
 }
 
 bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
