@@ -52,10 +52,10 @@ FLUSH_BYTES = 256 << 20
 NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of each kernel at this
     # workload (profiles/), valid while the kernel's source file is unchanged
-    "gate_gemm": {"src_sha256": "fa8dcb65fc6b9484ea8fb988f63e04371ba45dfcd01ce683b4079a91d828cc7e",
-                  "bytes_per_launch": 84259328 + 88713472},
-    "scan": {"src_sha256": "a899a994f0432fa9ae3483ee89bb3224ab943af47721b4daf585ac6671645593",
-             "bytes_per_launch": 136002304 + 32659712},
+    "gate_gemm": {"src_sha256": "2e11617f8e4c5203c2fd035550522193e8197818163d003d53f3fcbe570a8072",
+                  "bytes_per_launch": 84228608 + 90254336},
+    "scan": {"src_sha256": "50268f349d15f02d10e778a4e0eb84186c2d4b09ad248e1618579269a1345bc5",
+             "bytes_per_launch": 135250176 + 30820864},
 }
 
 
