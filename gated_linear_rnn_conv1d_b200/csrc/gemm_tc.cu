@@ -1015,6 +1015,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     uv[i] = ok ? __ldg(ep.u + idx) : 0.0f;
     hv[i] = ok ? ep.h[idx] : 0.0f;
   }
+  const float ba = __ldg(ep.b_a + uch), bx = __ldg(ep.b_x + uch), cl = __ldg(ep.cla + uch);
 
   if (warp == 0) {
     // ---------------- TMA producer (every CTA) ----------------
@@ -1133,18 +1134,28 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   {
     // h ← a_t h + √(1−a_t²) i u_t and y = h for 64 channels × 128 batch rows, by all twelve
     // warps, from the u_t and h values loaded at the start
-    const float ba = __ldg(ep.b_a + uch), bx = __ldg(ep.b_x + uch), cl = __ldg(ep.cla + uch);
+    // two batch columns at a time, in packed f32x2 arithmetic (d = 1 − a_t, b_t)
+    static_assert(kPer % 2 == 0, "columns in pairs");
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int c = (int)threadIdx.x / 64 + kPhases * i;
-      const int b = kh * 128 + c;
-      if (c < 128 && b < ep.B) {
-        const int64_t idx = (int64_t)b * ep.R + uch;
-        float at, bt;
-        gate_fast(zs[c * 128 + uj] + ba, zs[c * 128 + 64 + uj] + bx, cl, uv[i], at, bt);
-        const float hn = fmaf(at, hv[i], bt);
-        ep.h[idx] = hn;
-        ep.y[idx] = __float2bfloat16_rn(hn);
+    for (int i = 0; i < kPer; i += 2) {
+      const int c0 = (int)threadIdx.x / 64 + kPhases * i;
+      const int c1 = c0 + kPhases;
+      const int c1r = c1 < 128 ? c1 : 127;  // (a column past the half is computed, not stored)
+      float2 d, bt;
+      gate_fast2_pair(make_float2(zs[c0 * 128 + uj] + ba, zs[c1r * 128 + uj] + ba),
+                      make_float2(zs[c0 * 128 + 64 + uj] + bx, zs[c1r * 128 + 64 + uj] + bx), make_float2(cl, cl),
+                      make_float2(uv[i], uv[i + 1]), d, bt);
+      const float2 hn = __ffma2_rn(make_float2(1.0f - d.x, 1.0f - d.y), make_float2(hv[i], hv[i + 1]), bt);
+      const int b0 = kh * 128 + c0, b1 = kh * 128 + c1;
+      if (c0 < 128 && b0 < ep.B) {
+        const int64_t idx = (int64_t)b0 * ep.R + uch;
+        ep.h[idx] = hn.x;
+        ep.y[idx] = __float2bfloat16_rn(hn.x);
+      }
+      if (c1 < 128 && b1 < ep.B) {
+        const int64_t idx = (int64_t)b1 * ep.R + uch;
+        ep.h[idx] = hn.y;
+        ep.y[idx] = __float2bfloat16_rn(hn.y);
       }
     }
   }
