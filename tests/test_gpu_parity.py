@@ -170,6 +170,26 @@ def test_forward_matches_oracle(dtype, B, T, R, with_state):
     assert np.array_equal(f64(stT), st_ref)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_forward_on_a_garbage_workspace(dtype):
+    """rglru_forward leaves the zeroing of the scan's status word, ticket and chunk carries
+    to its Conv1D kernel (no memset): a workspace full of arbitrary bytes — words that read as
+    published carries among them — gives the same result as a zeroed one, bit for bit, and
+    a clean status."""
+    B, T, R = 3, 300, 264
+    w = _wl(B, T, R, dtype)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    nbytes = rglru.forward_workspace_bytes(B, T, R, dtype)
+    ws0 = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
+    y0, h0, _ = rglru.forward(p, x, workspace=ws0)
+    g = torch.Generator().manual_seed(7)
+    ws1 = torch.randint(0, 256, (nbytes,), generator=g, dtype=torch.uint8).to(DEV)
+    y1, h1, _ = rglru.forward(p, x, workspace=ws1)
+    assert rglru.workspace_status(ws0) == 0 and rglru.workspace_status(ws1) == 0
+    assert torch.equal(y0, y1) and torch.equal(h0, h1)
+
+
 @pytest.mark.parametrize("B,T,R", [(2, 256, 264), (1, 128, 128), (3, 384, 136), (1, 640, 8)])
 @pytest.mark.parametrize("with_state", [False, True])
 def test_fused_gate_scan_matches_oracle(B, T, R, with_state):
