@@ -280,6 +280,10 @@ def run_own(args):
     roof["kernel"] = dom
     roof["peak_source"] = ("measured: MEASURED_PEAKS.json burst figure" if pk["source"] == "measured"
                            else "fallback")
+    if dom == "gate_gemm" and pk.get("bf16_tflops_sustained"):
+        # the GEMM runs power-capped (sw_power_cap) inside the step loop; its fraction of the
+        # measured sustained figure, for context (frac above stays against the burst peak)
+        roof["frac_of_sustained"] = roof["achieved"] / pk["bf16_tflops_sustained"]
 
     if args.only == "forward":
         replicas.shutdown(rk)
