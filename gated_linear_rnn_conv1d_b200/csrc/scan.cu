@@ -229,19 +229,6 @@ __device__ __forceinline__ void stv_cs(__nv_bfloat16* p, const float (&f)[4]) {
 __device__ __forceinline__ void stv_cs(float* p, const float (&f)[2]) {
   __stcs(reinterpret_cast<float2*>(p), make_float2(f[0], f[1]));
 }
-// 4 fp16 values as floats, and back (the recurrence coefficients of the coefficient path)
-__device__ __forceinline__ void ldv_h(const __half* p, float (&f)[4]) {
-  const uint2 r = *reinterpret_cast<const uint2*>(p);
-  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
-  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
-  f[0] = lo.x; f[1] = lo.y; f[2] = hi.x; f[3] = hi.y;
-}
-__device__ __forceinline__ void stv_h(__half* p, const float (&f)[4]) {
-  const __half2 lo = __floats2half2_rn(f[0], f[1]);
-  const __half2 hi = __floats2half2_rn(f[2], f[3]);
-  *reinterpret_cast<uint2*>(p) =
-      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
-}
 // V float32 values from shared memory
 template <int V> __device__ __forceinline__ void ldf(const float* p, float (&f)[V]);
 template <> __device__ __forceinline__ void ldf<4>(const float* p, float (&f)[4]) {
