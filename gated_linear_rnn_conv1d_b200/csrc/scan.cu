@@ -16,8 +16,9 @@
 // and kScanTC = 64 consecutive steps: 32 channel groups of V channels (4 bf16 or 2 f32)
 // × 16 sub-chunks of 4 steps.
 //
-// One persistent CTA per SM takes tiles in order from an atomic ticket — time-chunk-major,
-// so every tile a CTA waits for was taken earlier by a running CTA (forward progress) —
+// One persistent CTA per SM takes tiles in order of a ticket (its first two fixed, the rest
+// from an atomic counter) — time-chunk-major, so every tile a CTA waits for was taken
+// earlier by a running CTA (forward progress) —
 // and runs them through a software pipeline of three warp roles:
 //   producer warp    takes tickets and, ahead of the compute warps, fills a ring of stages
 //                    (3, or 5 for the smaller coefficient stages): TMA copies of the tile's
@@ -861,15 +862,15 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
       tma_prefetch_desc(&maps.z);
     }
     // tickets: t_cur for the tile being loaded, t_nxt for the one after (its parameters
-    // are loaded a step early), pend for the one after that (fetched a step early)
-    unsigned t0 = 0, t1 = 0, pend = 0;
-    if (lane == 0) {
-      t0 = atomicAdd(a.ticket, 1u);
-      t1 = atomicAdd(a.ticket, 1u);
-      pend = atomicAdd(a.ticket, 1u);
-    }
-    int t_cur = (int)__shfl_sync(0xffffffffu, t0, 0);
-    int t_nxt = (int)__shfl_sync(0xffffffffu, t1, 0);
+    // are loaded a step early), pend for the one after that (fetched a step early). A
+    // CTA's first two tickets are fixed (blockIdx.x and blockIdx.x + gridDim.x, so the
+    // first loads go out without a round trip to the counter); the counter hands out the
+    // rest from 2·gridDim.x on. A CTA still takes its tickets in increasing order.
+    const unsigned t_fixed = 2u * gridDim.x;
+    unsigned pend = 0;
+    if (lane == 0) pend = atomicAdd(a.ticket, 1u) + t_fixed;
+    int t_cur = (int)blockIdx.x;
+    int t_nxt = (int)(blockIdx.x + gridDim.x);
     ParRegs<PV> par;
     if (!kCoef && t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
     int ends = 0;
@@ -901,7 +902,7 @@ __global__ void __launch_bounds__(threads_of<kCoef>(), 1)
                          par);
       // advance the ticket pipeline and start the next tile's parameter loads
       const int t_new = (int)__shfl_sync(0xffffffffu, pend, 0);
-      if (lane == 0) pend = atomicAdd(a.ticket, 1u);
+      if (lane == 0) pend = atomicAdd(a.ticket, 1u) + t_fixed;
       t_cur = t_nxt;
       t_nxt = t_new;
       if (!kCoef && t_cur < a.n_tiles) load_params<PV>(par, coord_of(t_cur, a).cblk * CW + lane * PV, a);
