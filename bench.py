@@ -401,6 +401,11 @@ def run_decode(torch, rglru, inputs, dev, stream, flush, pk, barrier, max_over_r
             "bytes_per_step": step_bytes,
             "GB/s_l2_flushed": step_bytes / cold_ms / 1e6,
             "frac_hbm_l2_flushed": step_bytes / cold_ms / 1e6 / pk["hbm_gbs"],
+            # at B=256 the step is at the compute/bandwidth ridge: with the weights L2-warm it is
+            # bound by the gate GEMM's 2·B·2R·R FLOP
+            "flops_per_step": 2.0 * B * (2 * R) * R,
+            "TFLOP/s_warm": 2.0 * B * (2 * R) * R / warm_ms / 1e9,
+            "frac_tensor_warm": 2.0 * B * (2 * R) * R / warm_ms / 1e9 / pk["bf16_tflops"],
             "gpu_launches_per_step": 2,
             "timing": "CUDA graph of 48 steps replayed 8x (L2-warm); and 24 single steps with L2 flushed"}
 
