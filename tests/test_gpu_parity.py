@@ -190,6 +190,28 @@ def test_forward_on_a_garbage_workspace(dtype):
     assert torch.equal(y0, y1) and torch.equal(h0, h1)
 
 
+def test_back_to_back_forwards_share_a_workspace():
+    """Calls queued back to back on one stream, one workspace, no synchronisation between
+    them: the second call's Conv1D kernel zeroes the workspace the first call's scan used,
+    and the gate GEMM and scan start early as programmatic dependents — each result must
+    equal the same call made alone, bit for bit."""
+    B, T, R = 4, 256, 520
+    w1 = _wl(B, T, R, torch.bfloat16, seed=1)
+    w2 = _wl(B, T, R, torch.bfloat16, seed=2)
+    p = rglru.Params.from_host(w1.params)
+    x1, x2 = w1.x.to(DEV), w2.x.to(DEV)
+    ws = torch.empty(rglru.forward_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=DEV)
+    ya, ha, _ = rglru.forward(p, x1, workspace=ws)
+    torch.cuda.synchronize()
+    yb, hb, _ = rglru.forward(p, x2, workspace=ws)
+    torch.cuda.synchronize()
+    outs = [rglru.forward(p, x, workspace=ws, want_conv_state=False) for x in (x1, x2, x1, x2)]
+    torch.cuda.synchronize()
+    assert rglru.workspace_status(ws) == 0
+    for (y, h, _), (yr, hr) in zip(outs, [(ya, ha), (yb, hb), (ya, ha), (yb, hb)]):
+        assert torch.equal(y, yr) and torch.equal(h, hr)
+
+
 @pytest.mark.parametrize("B,T,R", [(2, 256, 264), (1, 128, 128), (3, 384, 136), (1, 640, 8)])
 @pytest.mark.parametrize("with_state", [False, True])
 def test_fused_gate_scan_matches_oracle(B, T, R, with_state):
