@@ -51,8 +51,9 @@ struct ScanArgs {
 // Testing only: the tile index the next scans leave unpublished (-1 disables).
 void set_scan_stall(int64_t tile);
 int64_t scan_stall();
-// coef: z holds the recurrence coefficients (fp16 d = 1 − a_t, m = √(1−a_t²)·i_t) that
-// launch_gemm_coeffs_bf16 forms, instead of pre-activations (bf16 IO only).
+// coef: z holds the recurrence coefficients (fp16 d = 1 − a_t, b_t = √(1−a_t²)·i_t·u_t)
+// that launch_gemm_coeffs_bf16 forms, instead of pre-activations (bf16 IO only); x, the
+// conv parameters and Λ are then not read.
 cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s, bool coef = false);
 
 // ---- conv --------------------------------------------------------------------------
@@ -75,7 +76,8 @@ int num_sms();
 
 // `status`: device word the kernel ORs kStatusTimeout into if a bounded wait gives up.
 // The gate GEMM with the recurrence coefficients formed in its epilogue: g packed like z,
-// fp16 d = 1 − a_t in the z_a places and m = √(1−a_t²)·i_t in the z_x places.
+// fp16 d = 1 − a_t in the z_a places and b_t = √(1−a_t²)·i_t·u_t in the z_x places (the
+// epilogue reads its rows of u, the GEMM's A operand).
 cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
                                     const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
