@@ -201,6 +201,86 @@ def recurrent_block(x, W_1, W_2, W_o, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda
     return out, h_T
 
 
+def rglru_backward(x, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda, dy, h0=None, conv_state0=None,
+                   dh_T=None, c=C_DECAY):
+    """Gradients of the full-sequence forward (rglru_forward) by reverse-mode
+    differentiation of the same definition, step by step, in float64.
+
+    For a scalar loss ℓ with ∂ℓ/∂y = dy [B][T][R] and ∂ℓ/∂h_T = dh_T [B][R] (zero if
+    None), returns a dict with dx [B][T][R], dconv_w [4][R], dconv_b [R], dW_a, dW_x
+    [R][R], db_a, db_x, dLambda [R], dh0 [B][R] and dconv_state0 [B][3][R].
+
+    The forward, per batch row and channel (Eq. (1)–(4) with log a_t = c r_t log σ(Λ)):
+        r_t = σ(z_a,t), i_t = σ(z_x,t), a_t = exp(c r_t L), L = log σ(Λ),
+        m_t = √(1 − a_t²), h_t = a_t h_{t-1} + m_t i_t u_t, y_t = h_t.
+    Walking t from T−1 down to 0 with g = ∂ℓ/∂h_t (g starts at dh_T and takes dy_t at
+    each step): ∂a_t = g h_{t-1}, ∂m_t = g i_t u_t, ∂i_t = g m_t u_t, ∂u_t += g m_t i_t,
+    then g ← a_t g for h_{t-1}. Through a_t and m_t (∂m/∂log a = −a²/m):
+    ∂log a_t = ∂a_t a_t − ∂m_t a_t²/m_t; ∂r_t = ∂log a_t c L; ∂L += ∂log a_t c r_t;
+    ∂z_a = ∂r r(1 − r), ∂z_x = ∂i i(1 − i). Both uses of ∂log a_t carry a factor r_t, so
+    they are formed from ∂log a_t·r_t = ∂a_t a_t r_t − ∂m_t a_t² (r_t/m_t), where r_t/m_t → 0
+    as r_t → 0 (m_t ≈ √(−2 c r_t L)); at r_t = 0 exactly (a_t = 1, m_t = 0) it is taken as its
+    limit 0. Then the two linears and the Conv1D are differentiated as written
+    (dΛ = ∂L·σ(−Λ), since L = −log(1 + e^{−Λ})).
+    """
+    x = _f64(x)
+    B, T, R = x.shape
+    Wa, Wx = _f64(W_a), _f64(W_x)
+    u, _ = conv1d_causal(x, conv_w, conv_b, conv_state0)
+    z_a, z_x = gate_preactivations(u, W_a, b_a, W_x, b_x)
+    r, i = sigmoid(z_a), sigmoid(z_x)
+    Lam = _f64(Lambda)
+    L = -np.logaddexp(0.0, -Lam)                        # log σ(Λ)
+    a = np.exp(c * r * L)
+    m = np.sqrt(1.0 - a * a)
+    h_prev0 = np.zeros((B, R)) if h0 is None else _f64(h0)
+    y, _ = rglru_recurrence(a, i, u, h_prev0)
+    dy = _f64(dy)
+    g = np.zeros((B, R)) if dh_T is None else _f64(dh_T).copy()
+    dz_a = np.empty((B, T, R))
+    dz_x = np.empty((B, T, R))
+    du = np.empty((B, T, R))
+    dL = np.zeros(R)
+    for t in range(T - 1, -1, -1):
+        g = g + dy[:, t]
+        hp = y[:, t - 1] if t > 0 else h_prev0
+        at, mt, it, ut, rt = a[:, t], m[:, t], i[:, t], u[:, t], r[:, t]
+        d_a = g * hp
+        d_m = g * it * ut
+        d_i = g * mt * ut
+        du[:, t] = g * mt * it
+        r_over_m = np.divide(rt, mt, out=np.zeros_like(rt), where=mt > 0.0)
+        d_loga_r = d_a * at * rt - d_m * at * at * r_over_m      # ∂log a_t · r_t
+        dz_a[:, t] = d_loga_r * c * L * (1.0 - rt)
+        dL += np.sum(d_loga_r * c, axis=0)
+        dz_x[:, t] = d_i * it * (1.0 - it)
+        g = g * at
+    dh0 = g
+    zf_a = dz_a.reshape(B * T, R)
+    zf_x = dz_x.reshape(B * T, R)
+    uf = u.reshape(B * T, R)
+    dW_a = zf_a.T @ uf
+    dW_x = zf_x.T @ uf
+    db_a = zf_a.sum(axis=0)
+    db_x = zf_x.sum(axis=0)
+    du = du + (zf_a @ Wa + zf_x @ Wx).reshape(B, T, R)
+    # Conv1D: u_t = b + Σ_k w_k x_{t-3+k}, history (x_{-3}, x_{-2}, x_{-1}) from conv_state0
+    w = _f64(conv_w)
+    hist = np.zeros((B, CONV_WIDTH - 1, R)) if conv_state0 is None else _f64(conv_state0)
+    xp = np.concatenate([hist, x], axis=1)              # xp[:, s] = x_{s-3}
+    dxp = np.zeros_like(xp)
+    dconv_w = np.empty((CONV_WIDTH, R))
+    for k in range(CONV_WIDTH):
+        dconv_w[k] = np.sum(du * xp[:, k:k + T, :], axis=(0, 1))
+        dxp[:, k:k + T, :] += w[k] * du
+    return {
+        "dx": dxp[:, CONV_WIDTH - 1:, :], "dconv_state0": dxp[:, :CONV_WIDTH - 1, :],
+        "dconv_w": dconv_w, "dconv_b": du.sum(axis=(0, 1)),
+        "dW_a": dW_a, "db_a": db_a, "dW_x": dW_x, "db_x": db_x,
+        "dLambda": dL * sigmoid(-Lam), "dh0": dh0,
+    }
+
+
 def max_rel_error(got, ref):
     """Error measure for parity: max_i |g_i − o_i| / max(|o_i|, rms(o)).
 

@@ -344,3 +344,72 @@ def test_planted_mistakes_are_caught():
     for u in ex["u"]:
         h = at * h + math.sqrt(1 - at) * i * u
     assert abs(h - ex["y"][-1]) > 1e-3
+
+
+def _bwd_problem(seed, lam_lo, lam_hi, B=2, T=6, R=3):
+    rng = np.random.default_rng(seed)
+    P = {
+        "x": rng.normal(size=(B, T, R)),
+        "conv_w": rng.normal(size=(4, R)) * 0.5,
+        "conv_b": rng.normal(size=R) * 0.5,
+        "W_a": rng.normal(size=(R, R)) / math.sqrt(R),
+        "b_a": rng.normal(size=R) * 0.5,
+        "W_x": rng.normal(size=(R, R)) / math.sqrt(R),
+        "b_x": rng.normal(size=R) * 0.5,
+        "Lambda": rng.uniform(lam_lo, lam_hi, size=R),
+        "h0": rng.normal(size=(B, R)),
+        "conv_state0": rng.normal(size=(B, 3, R)),
+    }
+    dy = rng.normal(size=(B, T, R))
+    dh_T = rng.normal(size=(B, R))
+    return P, dy, dh_T
+
+
+def _loss(P, dy, dh_T):
+    y, h_T, _ = oracle.rglru_forward(P["x"], P["conv_w"], P["conv_b"], P["W_a"], P["b_a"], P["W_x"], P["b_x"],
+                                     P["Lambda"], h0=P["h0"], conv_state0=P["conv_state0"])
+    return float(np.sum(dy * y) + np.sum(dh_T * h_T))
+
+
+@pytest.mark.parametrize("seed,lam_lo,lam_hi", [(3, 1.0, 4.0), (4, 4.33, 8.99)])
+def test_backward_matches_central_differences(seed, lam_lo, lam_hi):
+    """The oracle's backward against central differences of the forward oracle — an
+    independent derivative of the definition — for every input: x, the taps and bias, W_a,
+    b_a, W_x, b_x, Λ (also in the configs' range, where a_t is close to 1 and √(1 − a_t²)
+    is small), h0 and the conv history. A dropped term, a wrong sign or a transposed
+    operand in the backward shows up here."""
+    P, dy, dh_T = _bwd_problem(seed, lam_lo, lam_hi)
+    G = oracle.rglru_backward(P["x"], P["conv_w"], P["conv_b"], P["W_a"], P["b_a"], P["W_x"], P["b_x"],
+                              P["Lambda"], dy, h0=P["h0"], conv_state0=P["conv_state0"], dh_T=dh_T)
+    names = {"x": "dx", "conv_w": "dconv_w", "conv_b": "dconv_b", "W_a": "dW_a", "b_a": "db_a", "W_x": "dW_x",
+             "b_x": "db_x", "Lambda": "dLambda", "h0": "dh0", "conv_state0": "dconv_state0"}
+    eps = 1e-6
+    for name, gname in names.items():
+        g = G[gname]
+        assert g.shape == P[name].shape, name
+        fd = np.empty_like(P[name])
+        for idx in np.ndindex(P[name].shape):
+            orig = P[name][idx]
+            P[name][idx] = orig + eps
+            lp = _loss(P, dy, dh_T)
+            P[name][idx] = orig - eps
+            lm = _loss(P, dy, dh_T)
+            P[name][idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        scale = max(float(np.max(np.abs(fd))), 1e-3)
+        assert np.max(np.abs(g - fd)) <= 1e-6 * scale, (name, np.max(np.abs(g - fd)), scale)
+
+
+def test_backward_of_a_frozen_state_is_plain_accumulation():
+    """With r ≡ 0 (W_a = 0, b_a = −1000: a_t = 1 and √(1 − a_t²) = 0 exactly) the state
+    never changes, h_t = h0, so ∂ℓ/∂h0 = Σ_t dy_t + dh_T and no gradient reaches x, the
+    taps or the input gate."""
+    B, T, R = 2, 5, 3
+    P, dy, dh_T = _bwd_problem(5, 1.0, 4.0, B, T, R)
+    P["W_a"][:] = 0.0
+    P["b_a"][:] = -1000.0
+    G = oracle.rglru_backward(P["x"], P["conv_w"], P["conv_b"], P["W_a"], P["b_a"], P["W_x"], P["b_x"],
+                              P["Lambda"], dy, h0=P["h0"], conv_state0=P["conv_state0"], dh_T=dh_T)
+    assert np.allclose(G["dh0"], dy.sum(axis=1) + dh_T, rtol=1e-13, atol=1e-13)
+    for k in ("dx", "dconv_w", "dconv_b", "dW_x", "db_x", "dLambda"):
+        assert np.all(G[k] == 0.0), k
