@@ -31,6 +31,14 @@ class RGLRUParams(ctypes.Structure):
 
 _PP = ctypes.POINTER(RGLRUParams)
 
+
+class RGLRUGrads(ctypes.Structure):
+    _fields_ = [("dx", _P), ("dconv_state0", _P), ("dconv_w", _P), ("dconv_b", _P), ("dW_a", _P), ("db_a", _P),
+                ("dW_x", _P), ("db_x", _P), ("dLambda", _P), ("dh0", _P)]
+
+
+_GP = ctypes.POINTER(RGLRUGrads)
+
 SIGNATURES = {
     "rglru_forward_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "rglru_forward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
@@ -47,6 +55,8 @@ SIGNATURES = {
     "rglru_scan_coeffs": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _S, _P]),
     "rglru_scan_noalloc": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "rglru_gemm_bf16": (_I, [_P, _P, _P, _L, _I, _I, _P]),
+    "rglru_backward_workspace_bytes": (_S, [_I, _I, _I]),
+    "rglru_backward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _GP, _I, _I, _I, _P, _S, _P]),
     "rglru_gate_scan_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "rglru_gate_scan": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "rglru_workspace_status": (_I, [_P, _P]),

@@ -1,0 +1,387 @@
+// Backward of Conv1D(4) + RG-LRU for bf16 IO (float32 arithmetic).
+//
+// Math: reverse-mode differentiation of "Griffin：将门控线性循环与局部注意力混合以实现高效的
+// 语言模型", §实门线性循环单元 (RG-LRU), Eq. (1)–(4) with the log-space decay of the paragraph
+// after them, and of the Conv1D of §循环块. Per batch row and channel, with r = σ(z_a),
+// i = σ(z_x), log a_t = r_t·c·log σ(Λ), m_t = √(1 − a_t²), h_t = a_t h_{t−1} + m_t i_t u_t and
+// g_t = ∂ℓ/∂h_t (which takes ∂ℓ/∂y_t = dy_t at each step and a_{t+1} g_{t+1} from the next):
+//   ∂a_t = g_t h_{t−1}, ∂m_t = g_t i_t u_t, ∂i_t = g_t m_t u_t, ∂u_t ⊃ g_t m_t i_t,
+//   ∂log a_t·r_t = ∂a_t a_t r_t − ∂m_t a_t² (r_t/m_t)      (r/m → 0 as r → 0),
+//   ∂z_a = ∂log a_t·r_t · c log σ(Λ) · (1 − r_t),  ∂z_x = ∂i_t i_t (1 − i_t),
+//   ∂ℓ/∂(log σ(Λ)) = Σ ∂log a_t·r_t · c,  ∂Λ = that · σ(−Λ).
+//
+// The reverse recurrence g_t = dy_t + a_{t+1} g_{t+1} is linear in g, so it runs in 64-step
+// chunks like the forward scan: each chunk folds itself into a map g_{t0} = P g_{t1} + Q
+// (bwd_maps_kernel); a short sequential pass per (row, channel) hands every chunk the g
+// entering it from the right (bwd_carries_kernel); each chunk then replays its steps with
+// the gate gradients fused (bwd_grads_kernel). The linears' gradients are tensor-core GEMMs
+// (gemm_tc.cu) on transposed copies made here; the Conv1D backward is its own kernel.
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "gate_math.cuh"
+#include "kernels.cuh"
+
+namespace rglru {
+
+namespace {
+
+constexpr int kBwdThreads = 128;  // threads per block; each thread takes 2 channels
+
+__device__ __forceinline__ float2 ld_bf2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+// column of channel c's recurrence-gate pre-activation in a packed gate row
+__device__ __forceinline__ int64_t zcol(int c) { return (int64_t)256 * (c / 128) + (c % 128); }
+
+// a_t from z_a (with its bias) and c·log σ(Λ)
+__device__ __forceinline__ float decay_of(float za, float cla) {
+  const float r = 1.0f / (1.0f + expf(-za));
+  return expf(r * cla);
+}
+
+struct BwdDims {
+  int B, T, R, n_chunks;
+  int64_t pitch;  // packed gate row
+};
+
+// Pass 1: the map g_{t0} = P·g_{t1} + Q of each 64-step chunk [t0, t1).
+__global__ void __launch_bounds__(kBwdThreads) bwd_maps_kernel(const __nv_bfloat16* __restrict__ z,
+                                                               const __nv_bfloat16* __restrict__ dy,
+                                                               const float* __restrict__ Lambda, float* __restrict__ P,
+                                                               float* __restrict__ Q, BwdDims d) {
+  const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
+  if (c >= d.R) return;
+  const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
+  const int t0 = chunk * kScanTC, t1 = min(t0 + kScanTC, d.T);
+  const float cl0 = decay_log_coeff(Lambda[c]), cl1 = decay_log_coeff(Lambda[c + 1]);
+  const __nv_bfloat16* zb = z + (int64_t)b * d.T * d.pitch + zcol(c);
+  const __nv_bfloat16* dyb = dy + (int64_t)b * d.T * d.R + c;
+  float2 an = make_float2(1.0f, 1.0f);
+  if (t1 < d.T) {
+    const float2 za = ld_bf2(zb + (int64_t)t1 * d.pitch);
+    an = make_float2(decay_of(za.x, cl0), decay_of(za.y, cl1));
+  }
+  float2 p = make_float2(1.0f, 1.0f), q = make_float2(0.0f, 0.0f);
+  for (int t = t1 - 1; t >= t0; --t) {
+    const float2 g = ld_bf2(dyb + (int64_t)t * d.R);
+    p = make_float2(an.x * p.x, an.y * p.y);
+    q = make_float2(fmaf(an.x, q.x, g.x), fmaf(an.y, q.y, g.y));
+    const float2 za = ld_bf2(zb + (int64_t)t * d.pitch);
+    an = make_float2(decay_of(za.x, cl0), decay_of(za.y, cl1));
+  }
+  const int64_t o = ((int64_t)b * d.n_chunks + chunk) * d.R + c;
+  *reinterpret_cast<float2*>(P + o) = p;
+  *reinterpret_cast<float2*>(Q + o) = q;
+}
+
+// Pass 2: per (row, channel), from the last chunk to the first, the g entering each chunk
+// from the right (g_{t1}; dh_T for the last chunk).
+__global__ void __launch_bounds__(kBwdThreads) bwd_carries_kernel(const float* __restrict__ P,
+                                                                  const float* __restrict__ Q,
+                                                                  const float* __restrict__ dh_T,
+                                                                  float* __restrict__ gin, BwdDims d) {
+  const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
+  if (c >= d.R) return;
+  const int b = blockIdx.y;
+  float2 G = dh_T != nullptr ? *reinterpret_cast<const float2*>(dh_T + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
+  for (int chunk = d.n_chunks - 1; chunk >= 0; --chunk) {
+    const int64_t o = ((int64_t)b * d.n_chunks + chunk) * d.R + c;
+    *reinterpret_cast<float2*>(gin + o) = G;
+    const float2 p = *reinterpret_cast<const float2*>(P + o), q = *reinterpret_cast<const float2*>(Q + o);
+    G = make_float2(fmaf(p.x, G.x, q.x), fmaf(p.y, G.y, q.y));
+  }
+}
+
+struct BwdGradArgs {
+  const __nv_bfloat16* z;   // packed pre-activations (with biases) [B·T][pitch]
+  const __nv_bfloat16* u;   // Conv1D output [B][T][R]
+  const __nv_bfloat16* y;   // forward output = h_t [B][T][R]
+  const __nv_bfloat16* dy;  // [B][T][R]
+  const float* h0;          // [B][R] or null (zeros)
+  const float* Lambda;      // [R]
+  const float* gin;         // [B][n_chunks][R]
+  __nv_bfloat16* dz;        // [B·T][2R]: ∂z_a in columns [0, R), ∂z_x in [R, 2R)
+  float* du;                // [B][T][R] the direct term ∂ℓ/∂u_t ⊃ g m i
+  float* dLsum;             // [R] Σ ∂log a·r·c (atomic)
+  float* db_a;              // [R] (atomic)
+  float* db_x;              // [R] (atomic)
+  float* dh0;               // [B][R] or null
+};
+
+// Pass 3: each chunk replays its steps from the g entering it, with the gate gradients.
+__global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, BwdDims d) {
+  const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
+  if (c >= d.R) return;
+  const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
+  const int t0 = chunk * kScanTC, t1 = min(t0 + kScanTC, d.T);
+  const float cl[2] = {decay_log_coeff(a.Lambda[c]), decay_log_coeff(a.Lambda[c + 1])};
+  const int64_t row0 = (int64_t)b * d.T;
+  const __nv_bfloat16* zb = a.z + row0 * d.pitch + zcol(c);
+  float gn[2], an[2];
+  {
+    const float2 g = *reinterpret_cast<const float2*>(a.gin + ((int64_t)b * d.n_chunks + chunk) * d.R + c);
+    gn[0] = g.x;
+    gn[1] = g.y;
+    an[0] = an[1] = 1.0f;
+    if (t1 < d.T) {
+      const float2 za = ld_bf2(zb + (int64_t)t1 * d.pitch);
+      an[0] = decay_of(za.x, cl[0]);
+      an[1] = decay_of(za.y, cl[1]);
+    }
+  }
+  float sL[2] = {0.f, 0.f}, sa[2] = {0.f, 0.f}, sx[2] = {0.f, 0.f};
+  for (int t = t1 - 1; t >= t0; --t) {
+    const int64_t e = (row0 + t) * d.R + c;
+    const float2 dy2 = ld_bf2(a.dy + e), u2 = ld_bf2(a.u + e);
+    const float2 za2 = ld_bf2(zb + (int64_t)t * d.pitch), zx2 = ld_bf2(zb + (int64_t)t * d.pitch + 128);
+    float2 hp2;
+    if (t > 0) hp2 = ld_bf2(a.y + e - d.R);
+    else hp2 = a.h0 != nullptr ? *reinterpret_cast<const float2*>(a.h0 + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
+    const float dyv[2] = {dy2.x, dy2.y}, uv[2] = {u2.x, u2.y}, zav[2] = {za2.x, za2.y}, zxv[2] = {zx2.x, zx2.y},
+                hpv[2] = {hp2.x, hp2.y};
+    float dza[2], dzx[2], dud[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float g = fmaf(an[j], gn[j], dyv[j]);
+      const float r = 1.0f / (1.0f + expf(-zav[j]));
+      const float i = 1.0f / (1.0f + expf(-zxv[j]));
+      const float la = r * cl[j];
+      const float at = expf(la);
+      const float mt = sqrtf(-expm1f(2.0f * la));
+      const float d_a = g * hpv[j];
+      const float d_m = g * i * uv[j];
+      const float d_i = g * mt * uv[j];
+      dud[j] = g * mt * i;
+      const float r_over_m = mt > 0.0f ? r / mt : 0.0f;
+      const float dlr = d_a * at * r - d_m * at * at * r_over_m;  // ∂log a_t · r_t
+      dza[j] = dlr * cl[j] * (1.0f - r);
+      dzx[j] = d_i * i * (1.0f - i);
+      sL[j] = fmaf(dlr, kDecayC, sL[j]);
+      sa[j] += dza[j];
+      sx[j] += dzx[j];
+      gn[j] = g;
+      an[j] = at;
+    }
+    st_bf2(a.dz + (row0 + t) * 2 * d.R + c, dza[0], dza[1]);
+    st_bf2(a.dz + (row0 + t) * 2 * d.R + d.R + c, dzx[0], dzx[1]);
+    *reinterpret_cast<float2*>(a.du + e) = make_float2(dud[0], dud[1]);
+  }
+  if (chunk == 0 && a.dh0 != nullptr)  // the gradient reaching h_{−1} = h0
+    *reinterpret_cast<float2*>(a.dh0 + (int64_t)b * d.R + c) = make_float2(an[0] * gn[0], an[1] * gn[1]);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    atomicAdd(a.dLsum + c + j, sL[j]);
+    atomicAdd(a.db_a + c + j, sa[j]);
+    atomicAdd(a.db_x + c + j, sx[j]);
+  }
+}
+
+// ∂Λ = ∂ℓ/∂(log σ(Λ)) · σ(−Λ), since log σ(Λ) = −log(1 + e^{−Λ}).
+__global__ void bwd_lambda_kernel(const float* __restrict__ dLsum, const float* __restrict__ Lambda,
+                                  float* __restrict__ dLambda, int R) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c < R) dLambda[c] = dLsum[c] / (1.0f + expf(Lambda[c]));
+}
+
+struct BwdConvArgs {
+  const __nv_bfloat16* x;       // [B][T][R]
+  const __nv_bfloat16* state0;  // [B][3][R] (x_{−3}, x_{−2}, x_{−1}) or null
+  const float* conv_w;          // [4][R]
+  const float* du;              // [B][T][R] direct term
+  const __nv_bfloat16* dug;     // [B][T][R] gate-GEMM term
+  __nv_bfloat16* dx;            // [B][T][R]
+  __nv_bfloat16* dstate0;       // [B][3][R] or null
+  float* dconv_w;               // [4][R] (atomic)
+  float* dconv_b;               // [R] (atomic)
+};
+
+// Conv1D backward, u_t = b + Σ_k w_k x_{t−3+k}: dx_s = Σ_k w_k du_{s+3−k} (t < T),
+// dw_k = Σ du_t x_{t−3+k}, db = Σ du_t; for the first chunk also the conv history's gradient.
+__global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, BwdDims d) {
+  const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
+  if (c >= d.R) return;
+  const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
+  const int t0 = chunk * kScanTC, t1 = min(t0 + kScanTC, d.T);
+  const int64_t base = (int64_t)b * d.T * d.R + c;
+  float w[4][2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 wk = *reinterpret_cast<const float2*>(a.conv_w + k * d.R + c);
+    w[k][0] = wk.x;
+    w[k][1] = wk.y;
+  }
+  auto du_at = [&](int t) -> float2 {  // total ∂ℓ/∂u_t, zero past T
+    if (t >= d.T) return make_float2(0.f, 0.f);
+    const float2 p = *reinterpret_cast<const float2*>(a.du + base + (int64_t)t * d.R);
+    const float2 q = ld_bf2(a.dug + base + (int64_t)t * d.R);
+    return make_float2(p.x + q.x, p.y + q.y);
+  };
+  auto x_at = [&](int t) -> float2 {  // x_t, from the conv history for t < 0
+    if (t >= 0) return ld_bf2(a.x + base + (int64_t)t * d.R);
+    if (a.state0 == nullptr) return make_float2(0.f, 0.f);
+    return ld_bf2(a.state0 + ((int64_t)b * 3 + (t + 3)) * d.R + c);
+  };
+  // sliding windows: du_{t..t+3} and x_{t−3..t}
+  float2 dwin[4], xwin[4];
+  for (int j = 0; j < 4; ++j) dwin[j] = du_at(t0 + j);
+  for (int j = 0; j < 3; ++j) xwin[j] = x_at(t0 - 3 + j);
+  float sw[4][2] = {}, sb[2] = {0.f, 0.f};
+  for (int t = t0; t < t1; ++t) {
+    xwin[3] = x_at(t);
+    float dxv[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float dut = j ? dwin[0].y : dwin[0].x;
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc = fmaf(w[k][j], j ? dwin[3 - k].y : dwin[3 - k].x, acc);
+      dxv[j] = acc;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sw[k][j] = fmaf(dut, j ? xwin[k].y : xwin[k].x, sw[k][j]);
+      sb[j] += dut;
+    }
+    st_bf2(a.dx + base + (int64_t)t * d.R, dxv[0], dxv[1]);
+    for (int j = 0; j < 3; ++j) { dwin[j] = dwin[j + 1]; xwin[j] = xwin[j + 1]; }
+    dwin[3] = du_at(t + 4);
+  }
+  if (chunk == 0 && a.dstate0 != nullptr) {
+    // history slot s = 0, 1, 2 holds x_{s−3}: its gradient is Σ_k w_k du_{s−k}, 0 ≤ s−k < T
+    for (int s = 0; s < 3; ++s) {
+      float acc[2] = {0.f, 0.f};
+      for (int k = 0; k <= s; ++k) {
+        const float2 dv = du_at(s - k);
+        acc[0] = fmaf(w[k][0], dv.x, acc[0]);
+        acc[1] = fmaf(w[k][1], dv.y, acc[1]);
+      }
+      st_bf2(a.dstate0 + ((int64_t)b * 3 + s) * d.R + c, acc[0], acc[1]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) atomicAdd(a.dconv_w + k * d.R + c + j, sw[k][j]);
+    atomicAdd(a.dconv_b + c + j, sb[j]);
+  }
+}
+
+// out[j][i] = in[i][j] for a rows × cols bf16 matrix (leading dimensions ld_in, ld_out);
+// columns cols..cols_pad−1 of out (rows of in past `rows`) are written as zeros.
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in,
+                                                             __nv_bfloat16* __restrict__ out, int64_t rows,
+                                                             int64_t cols, int64_t ld_in, int64_t ld_out,
+                                                             int64_t rows_pad) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;  // 32 × 8
+  for (int k = ty; k < 32; k += 8) {
+    const int64_t r = r0 + k, c = c0 + tx;
+    tile[k][tx] = (r < rows && c < cols) ? in[r * ld_in + c] : __float2bfloat16(0.0f);
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int64_t c = c0 + k, r = r0 + tx;  // out row c, column r
+    if (c < cols && r < rows_pad) out[c * ld_out + r] = tile[tx][k];
+  }
+}
+
+cudaError_t transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols, int64_t ld_in, int64_t ld_out,
+                           int64_t rows_pad, cudaStream_t s) {
+  const dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows_pad + 31) / 32));
+  if (grid.y > 65535u) return cudaErrorInvalidValue;
+  transpose_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out),
+                                              rows, cols, ld_in, ld_out, rows_pad);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+BwdLayout bwd_layout(int B, int T, int R) {
+  BwdLayout L;
+  const int64_t n = (int64_t)B * T;
+  const int64_t np = (n + 63) / 64 * 64;  // token count padded for the transposed operands
+  const int n_chunks = (T + kScanTC - 1) / kScanTC;
+  auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
+  size_t o = 256;  // status word
+  L.off_u = o;      o += r256((size_t)n * R * 2);
+  L.off_z = o;      o += r256((size_t)n * gate_pitch(R) * 2);
+  L.off_P = o;      o += r256((size_t)B * n_chunks * R * 4);
+  L.off_Q = o;      o += r256((size_t)B * n_chunks * R * 4);
+  L.off_gin = o;    o += r256((size_t)B * n_chunks * R * 4);
+  L.off_dz = o;     o += r256((size_t)n * 2 * R * 2);
+  L.off_du = o;     o += r256((size_t)n * R * 4);
+  L.off_dug = o;    o += r256((size_t)n * R * 2);
+  L.off_wt = o;     o += r256((size_t)2 * R * R * 2);
+  L.off_dzt = o;    o += r256((size_t)2 * R * np * 2);
+  L.off_ut = o;     o += r256((size_t)R * np * 2);
+  L.off_dL = o;     o += r256((size_t)R * 4);
+  L.bytes = o;
+  L.n_pad = np;
+  L.n_chunks = n_chunks;
+  return L;
+}
+
+cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cudaStream_t s) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  unsigned* status = reinterpret_cast<unsigned*>(w);
+  const int B = g.B, T = g.T, R = g.R;
+  const int64_t n = (int64_t)B * T;
+  void* u = w + L.off_u;
+  void* z = w + L.off_z;
+  float* P = reinterpret_cast<float*>(w + L.off_P);
+  float* Q = reinterpret_cast<float*>(w + L.off_Q);
+  float* gin = reinterpret_cast<float*>(w + L.off_gin);
+  __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(w + L.off_dz);
+  float* du = reinterpret_cast<float*>(w + L.off_du);
+  __nv_bfloat16* dug = reinterpret_cast<__nv_bfloat16*>(w + L.off_dug);
+  __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(w + L.off_wt);
+  __nv_bfloat16* dzt = reinterpret_cast<__nv_bfloat16*>(w + L.off_dzt);
+  __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(w + L.off_ut);
+  float* dLsum = reinterpret_cast<float*>(w + L.off_dL);
+  cudaError_t e;
+  // the accumulated outputs start at zero
+  if ((e = cudaMemsetAsync(status, 0, 4, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(dLsum, 0, (size_t)R * 4, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(g.db_a, 0, (size_t)R * 4, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(g.db_x, 0, (size_t)R * 4, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(g.dconv_w, 0, (size_t)4 * R * 4, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(g.dconv_b, 0, (size_t)R * 4, s)) != cudaSuccess) return e;
+  // recompute u = Conv1D(x) and the packed pre-activations z (with biases)
+  if ((e = launch_conv1d(g.conv_w, g.conv_b, g.x, g.state0, u, nullptr, B, T, R, true, status, s)) != cudaSuccess)
+    return e;
+  if ((e = launch_gemm_gates_bf16(u, g.W_a, g.b_a, g.W_x, g.b_x, z, n, R, status, s)) != cudaSuccess) return e;
+  BwdDims d{B, T, R, L.n_chunks, gate_pitch(R)};
+  const unsigned gx = (unsigned)((R / 2 + kBwdThreads - 1) / kBwdThreads);
+  const dim3 g_chunks(gx, (unsigned)(B * L.n_chunks)), g_rows(gx, (unsigned)B);
+  bwd_maps_kernel<<<g_chunks, kBwdThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(z),
+                                                   static_cast<const __nv_bfloat16*>(g.dy), g.Lambda, P, Q, d);
+  bwd_carries_kernel<<<g_rows, kBwdThreads, 0, s>>>(P, Q, g.dh_T, gin, d);
+  BwdGradArgs ga{static_cast<const __nv_bfloat16*>(z), static_cast<const __nv_bfloat16*>(u),
+                 static_cast<const __nv_bfloat16*>(g.y), static_cast<const __nv_bfloat16*>(g.dy), g.h0, g.Lambda, gin,
+                 dz, du, dLsum, g.db_a, g.db_x, g.dh0};
+  bwd_grads_kernel<<<g_chunks, kBwdThreads, 0, s>>>(ga, d);
+  bwd_lambda_kernel<<<(R + 255) / 256, 256, 0, s>>>(dLsum, g.Lambda, g.dLambda, R);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // ∂ℓ/∂u ⊃ [∂z_a | ∂z_x]·[W_a; W_x]: B operand [W_a; W_x]ᵀ = [R][2R]
+  if ((e = transpose_bf16(g.W_a, wt, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
+  if ((e = transpose_bf16(g.W_x, wt + R, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
+  if ((e = launch_gemm_bf16(dz, wt, dug, n, R, 2 * R, R, status, s)) != cudaSuccess) return e;
+  // ∂W_a = ∂z_aᵀ u, ∂W_x = ∂z_xᵀ u over the tokens (K = tokens, zero-padded to n_pad)
+  if ((e = transpose_bf16(dz, dzt, n, 2 * R, 2 * R, L.n_pad, L.n_pad, s)) != cudaSuccess) return e;
+  if ((e = transpose_bf16(u, ut, n, R, R, L.n_pad, L.n_pad, s)) != cudaSuccess) return e;
+  if ((e = launch_gemm_f32out(dzt, ut, g.dW_a, R, R, (int)L.n_pad, R, status, s)) != cudaSuccess) return e;
+  if ((e = launch_gemm_f32out(dzt + (int64_t)R * L.n_pad, ut, g.dW_x, R, R, (int)L.n_pad, R, status, s)) !=
+      cudaSuccess)
+    return e;
+  // Conv1D backward
+  BwdConvArgs ca{static_cast<const __nv_bfloat16*>(g.x), static_cast<const __nv_bfloat16*>(g.state0), g.conv_w, du,
+                 dug, static_cast<__nv_bfloat16*>(g.dx), static_cast<__nv_bfloat16*>(g.dstate0), g.dconv_w,
+                 g.dconv_b};
+  bwd_conv_kernel<<<g_chunks, kBwdThreads, 0, s>>>(ca, d);
+  return cudaGetLastError();
+}
+
+}  // namespace rglru

@@ -35,10 +35,11 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
 constexpr int kGemmThreads = 192;
 
-enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2, EPI_SCAN = 3, EPI_COEF = 4 };
+enum EpiKind { EPI_STORE = 0, EPI_GATES = 1, EPI_STEP = 2, EPI_SCAN = 3, EPI_COEF = 4, EPI_STORE_F32 = 5 };
 
 struct EpiArgs {
   __nv_bfloat16* C;   // STORE / GATES output
+  float* Cf;          // STORE_F32 output
   int64_t ldc;        // elements
   int N;              // STORE: valid columns
   const float* b_a;   // GATES / STEP
@@ -676,6 +677,17 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
             v[j] = __uint_as_float(r[j]) + (ch < ep.R ? __ldg(bias + ch) : 0.0f);
           }
           if (row_ok) store_row_bf16(ep.C + row * ep.ldc + (int64_t)n_blk * BN + col0, v);
+        } else if constexpr (EPI == EPI_STORE_F32) {
+          // float32 rows (N a multiple of 4): eight 16-byte stores per 32 columns
+          const int gcol = n_blk * BN + col0;
+          if (row_ok) {
+            float4* d = reinterpret_cast<float4*>(ep.Cf + row * ep.ldc + gcol);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (gcol + 4 * q < ep.N)
+                d[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                   __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -1355,6 +1367,20 @@ cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, 
   ep.N = N;
   const int n_tiles_n = (N + 255) / 256;
   return launch_tc2<EPI_STORE, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+}
+
+cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t M, int N, int K, int64_t ldc,
+                               unsigned* status, cudaStream_t s) {
+  // as launch_gemm_bf16, with float32 output rows
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, A, K, M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, 128)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.Cf = C;
+  ep.ldc = ldc;
+  ep.N = N;
+  const int n_tiles_n = (N + 255) / 256;
+  return launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
 }
 
 namespace {

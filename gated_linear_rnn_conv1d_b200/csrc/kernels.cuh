@@ -84,6 +84,10 @@ cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* b
                                    void* z, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
                              unsigned* status, cudaStream_t s);
+// C = A·Bᵀ as launch_gemm_bf16 (A [M][K], B [N][K] bf16, K-contiguous), C float32 [M][ldc],
+// N a multiple of 4.
+cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t M, int N, int K, int64_t ldc,
+                               unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,
                                   const void* Wx, const float* bx, const float* cla, float* h, void* y_t, int B,
                                   int R, unsigned* status, cudaStream_t s);
@@ -116,5 +120,42 @@ cudaError_t launch_gate_scan_bf16(const ScanFusedArgs& f, cudaStream_t s);
 unsigned* global_status_word();
 cudaError_t launch_gemm_gates_f32(const float* u, const float* Wa, const float* ba, const float* Wx,
                                   const float* bx, float* z, int64_t M, int R, cudaStream_t s);
+
+// ---- backward (bf16 IO) --------------------------------------------------------------
+// Workspace of launch_backward: [status | u | z | chunk maps P, Q | chunk carries | ∂z |
+// direct ∂u (f32) | gate-GEMM ∂u | [W_a; W_x]ᵀ | ∂zᵀ | uᵀ | Σ ∂log a·r·c].
+struct BwdLayout {
+  size_t off_u, off_z, off_P, off_Q, off_gin, off_dz, off_du, off_dug, off_wt, off_dzt, off_ut, off_dL, bytes;
+  int64_t n_pad;  // tokens rounded up to 64 (the transposed operands' row length)
+  int n_chunks;
+};
+BwdLayout bwd_layout(int B, int T, int R);
+struct BwdArgs {
+  const void* x;        // [B][T][R] bf16
+  const void* y;        // forward output [B][T][R] bf16
+  const void* dy;       // [B][T][R] bf16
+  const float* h0;      // [B][R] or null
+  const float* dh_T;    // [B][R] or null
+  const void* state0;   // [B][3][R] bf16 or null
+  const float* conv_w;  // [4][R]
+  const float* conv_b;
+  const void* W_a;      // [R][R] bf16
+  const float* b_a;
+  const void* W_x;
+  const float* b_x;
+  const float* Lambda;
+  void* dx;             // [B][T][R] bf16
+  void* dstate0;        // [B][3][R] bf16 or null
+  float* dconv_w;       // [4][R]
+  float* dconv_b;       // [R]
+  float* dW_a;          // [R][R]
+  float* db_a;
+  float* dW_x;
+  float* db_x;
+  float* dLambda;
+  float* dh0;           // [B][R] or null
+  int B, T, R;
+};
+cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cudaStream_t s);
 
 }  // namespace rglru

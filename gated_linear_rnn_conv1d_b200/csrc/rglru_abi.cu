@@ -434,6 +434,47 @@ int rglru_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, in
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
+size_t rglru_backward_workspace_bytes(int B, int T, int R) {
+  if (!valid_R(R) || !valid_tokens(B, T)) return 0;
+  return bwd_layout(B, T, R).bytes;
+}
+
+int rglru_backward(const rglru_params* params, const void* x, const void* y, const void* dy, const float* h0,
+                   const float* dh_T, const void* conv_state0, const rglru_grads* grads, int B, int T, int R,
+                   void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  // the transposed token axis of the weight-gradient GEMMs (and its 32-row transpose
+  // tiles) must stay within int32 and the grid's y limit
+  if ((int64_t)B * T > (int64_t)65535 * 32 - 64) return RGLRU_ERR_SHAPE;
+  // the chunked kernels index (batch row, 64-step chunk) with the grid's y dimension
+  if ((int64_t)B * ((T + kScanTC - 1) / kScanTC) > 65535) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x == nullptr || y == nullptr || dy == nullptr || grads == nullptr) return RGLRU_ERR_NULL;
+  const rglru_grads& g = *grads;
+  if (g.dx == nullptr || g.dconv_w == nullptr || g.dconv_b == nullptr || g.dW_a == nullptr || g.db_a == nullptr ||
+      g.dW_x == nullptr || g.db_x == nullptr || g.dLambda == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(dy) || !aligned16(h0) || !aligned16(dh_T) ||
+      !aligned16(conv_state0) || !aligned16(g.dx) || !aligned16(g.dconv_state0) || !aligned16(g.dconv_w) ||
+      !aligned16(g.dconv_b) || !aligned16(g.dW_a) || !aligned16(g.db_a) || !aligned16(g.dW_x) ||
+      !aligned16(g.db_x) || !aligned16(g.dLambda) || !aligned16(g.dh0))
+    return RGLRU_ERR_ALIGN;
+  const BwdLayout L = bwd_layout(B, T, R);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  BwdArgs a{};
+  a.x = x; a.y = y; a.dy = dy; a.h0 = h0; a.dh_T = dh_T; a.state0 = conv_state0;
+  a.conv_w = params->conv_w; a.conv_b = params->conv_b; a.W_a = params->W_a; a.b_a = params->b_a;
+  a.W_x = params->W_x; a.b_x = params->b_x; a.Lambda = params->Lambda;
+  a.dx = g.dx; a.dstate0 = g.dconv_state0; a.dconv_w = g.dconv_w; a.dconv_b = g.dconv_b; a.dW_a = g.dW_a;
+  a.db_a = g.db_a; a.dW_x = g.dW_x; a.db_x = g.db_x; a.dLambda = g.dLambda; a.dh0 = g.dh0;
+  a.B = B; a.T = T; a.R = R;
+  cudaError_t e = launch_backward(a, L, workspace, (cudaStream_t)stream);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
 int rglru_block_forward(const rglru_params* params, const void* W_1, const void* W_2, const void* W_o, const void* x,
                         const float* h0, void* out, float* h_T, int B, int T, int D, int R, int io_dtype,
                         void* workspace, size_t workspace_bytes, rglru_stream_t stream) {

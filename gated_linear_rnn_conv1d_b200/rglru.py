@@ -96,6 +96,41 @@ def forward(params: Params, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
     return y, h_T, conv_state_T
 
 
+def backward_workspace_bytes(B: int, T: int, R: int) -> int:
+    return _abi.load().rglru_backward_workspace_bytes(B, T, R)
+
+
+def backward(params: Params, x: torch.Tensor, y: torch.Tensor, dy: torch.Tensor, h0: Optional[torch.Tensor] = None,
+             dh_T: Optional[torch.Tensor] = None, conv_state0: Optional[torch.Tensor] = None, *,
+             want_dh0: bool = True, want_dconv_state0: bool = True, workspace: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """rglru_backward (bf16 IO): gradients of a loss with ∂ℓ/∂y = dy (and ∂ℓ/∂h_T = dh_T)
+    for the forward that mapped x (with h0, conv_state0) to y. Returns a dict with dx
+    [B][T][R] bf16, dconv_state0 [B][3][R] bf16 (or None), dconv_w [4][R], dconv_b, dW_a,
+    db_a, dW_x, db_x, dLambda and dh0 [B][R] (or None), all float32 but dx and dconv_state0."""
+    lib = _abi.load()
+    B, T, R = x.shape
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {
+        "dx": torch.empty_like(x),
+        "dconv_state0": torch.empty(B, 3, R, dtype=x.dtype, device=dev) if want_dconv_state0 else None,
+        "dconv_w": torch.empty(4, R, **f32), "dconv_b": torch.empty(R, **f32),
+        "dW_a": torch.empty(R, R, **f32), "db_a": torch.empty(R, **f32),
+        "dW_x": torch.empty(R, R, **f32), "db_x": torch.empty(R, **f32),
+        "dLambda": torch.empty(R, **f32),
+        "dh0": torch.empty(B, R, **f32) if want_dh0 else None,
+    }
+    g = _abi.RGLRUGrads(*(_p(out[k]) for k in ("dx", "dconv_state0", "dconv_w", "dconv_b", "dW_a", "db_a", "dW_x",
+                                                  "db_x", "dLambda", "dh0")))
+    ws = _workspace(lib.rglru_backward_workspace_bytes(B, T, R), dev, workspace)
+    st = params.struct()
+    _abi.check("rglru_backward", lib.rglru_backward(
+        ctypes.byref(st), _p(x), _p(y), _p(dy), _p(h0), _p(dh_T), _p(conv_state0), ctypes.byref(g), B, T, R, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return out
+
+
 class HostForwardPlan:
     """Device buffers and streams for forward_host on inputs of shape [B][T][R].
 

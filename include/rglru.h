@@ -137,6 +137,50 @@ RGLRU_API int rglru_block_forward(const rglru_params* params, const void* W_1, c
                         int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Backward of rglru_forward for bf16 IO: the gradients of a scalar loss ℓ with respect to
+ * the input, the parameters, the initial state and the conv history, given ∂ℓ/∂y and
+ * ∂ℓ/∂h_T. Reverse-mode differentiation of Eq. (1)–(4) above (with the log-space decay
+ * of the paragraph after them: log a_t = r_t·c·log σ(Λ)) and of the Conv1D of §循环块:
+ * with g_t = ∂ℓ/∂h_t = dy_t + a_{t+1} g_{t+1} (g after the last step = dh_T),
+ *   ∂z_a = (g h_{t-1} a_t r_t − g i_t u_t a_t² r_t/√(1−a_t²))·c·log σ(Λ)·(1 − r_t),
+ *   ∂z_x = g √(1−a_t²) u_t · i_t (1 − i_t),  ∂u_t = g √(1−a_t²) i_t + ∂z_a W_a + ∂z_x W_x,
+ *   ∂W_a = Σ_t ∂z_aᵀ u_t, ∂b_a = Σ_t ∂z_a (same for x), ∂Λ = Σ (∂log a_t) c r_t · σ(−Λ),
+ *   ∂h0 = a_0 g_0, and the Conv1D's transpose for ∂x, the taps, the bias and the history.
+ * u and the gate pre-activations are recomputed from x; h_{t-1} is read from y.
+ *   params        as rglru_forward (W_a, W_x bf16)
+ *   x             [B][T][R] bf16, the forward's input
+ *   y             [B][T][R] bf16, the forward's output for the same x, h0, conv_state0
+ *   dy            [B][T][R] bf16, ∂ℓ/∂y
+ *   h0            [B][R] float32 or NULL (zeros), as in the forward
+ *   dh_T          [B][R] float32 or NULL (zeros), ∂ℓ/∂h_T
+ *   conv_state0   [B][3][R] bf16 or NULL (zeros), as in the forward
+ *   grads         output buffers (all 16-byte aligned; the library writes every one, and
+ *                 zeroes the accumulated ones first): dx [B][T][R] bf16; dconv_state0
+ *                 [B][3][R] bf16 or NULL; dconv_w [4][R], dconv_b, db_a, db_x, dLambda [R],
+ *                 dW_a, dW_x [R][R] (row-major [out][in]) and dh0 [B][R] (or NULL) float32
+ *   workspace     at least rglru_backward_workspace_bytes(B, T, R) bytes, 256-byte aligned
+ * Shapes: as rglru_forward, and B·T ≤ 2,097,056 and B·⌈T/64⌉ ≤ 65535 (RGLRU_ERR_SHAPE).
+ * The accumulated outputs (the taps, biases and Λ) are summed with atomics, so their
+ * last bits may vary between runs; everything else is deterministic.
+ * --------------------------------------------------------------------------------- */
+typedef struct {
+  void* dx;           /* [B][T][R] bf16                          */
+  void* dconv_state0; /* [B][3][R] bf16, or NULL                 */
+  float* dconv_w;     /* [4][R]                                  */
+  float* dconv_b;     /* [R]                                     */
+  float* dW_a;        /* [R][R]                                  */
+  float* db_a;        /* [R]                                     */
+  float* dW_x;        /* [R][R]                                  */
+  float* db_x;        /* [R]                                     */
+  float* dLambda;     /* [R]                                     */
+  float* dh0;         /* [B][R], or NULL                         */
+} rglru_grads;
+RGLRU_API size_t rglru_backward_workspace_bytes(int B, int T, int R);
+RGLRU_API int rglru_backward(const rglru_params* params, const void* x, const void* y, const void* dy,
+                             const float* h0, const float* dh_T, const void* conv_state0, const rglru_grads* grads,
+                             int B, int T, int R, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * The stages of rglru_forward, callable one by one (for per-kernel timing and for
  * testing each stage against the oracle). rglru_forward runs exactly rglru_conv1d, then
  * for RGLRU_BF16 rglru_gate_coeffs and rglru_scan_coeffs, for RGLRU_F32 rglru_gate_proj

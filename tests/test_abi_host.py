@@ -127,3 +127,30 @@ def test_workspace_queries():
     assert lib.rglru_gate_pitch(12) == 0
     assert lib.rglru_scan_workspace_bytes(1, 64, 128, 1) > 256
     assert lib.rglru_block_workspace_bytes(4, 4096, 4096, 5632, 1) > 4 * 4096 * 5632 * 2 * 5
+
+
+def test_backward_rejects_bad_arguments_before_any_launch():
+    lib = _abi.load()
+    p = _params()
+    ok = _fake()
+    assert lib.rglru_backward_workspace_bytes(2, 64, 256) > 0
+    assert lib.rglru_backward_workspace_bytes(2, 64, 12) == 0
+    grads = _abi.RGLRUGrads(*([0x100000] * 10))
+    wsb = lib.rglru_backward_workspace_bytes(1, 64, 256)
+    ws = _fake(0x200000)
+
+    def call(**kw):
+        g = kw.get("g", grads)
+        return lib.rglru_backward(kw.get("p", ctypes.byref(p)), kw.get("x", ok), ok, ok, kw.get("h0", None), None,
+                                  None, ctypes.byref(g) if g is not None else None, 1, kw.get("T", 64),
+                                  kw.get("R", 256), kw.get("ws", ws), kw.get("wsb", wsb), None)
+    assert call(R=12) == -2
+    assert call(T=0) == -2
+    assert call(p=None) == -1
+    assert call(x=None) == -1
+    assert call(g=None) == -1
+    assert call(g=_abi.RGLRUGrads(*([0x100000] * 8 + [None, 0x100000]))) == -1   # dLambda missing
+    assert call(g=_abi.RGLRUGrads(*([0x100000] + [0x100008] + [0x100000] * 8))) == -3  # dconv_state0 misaligned
+    assert call(h0=_fake(0x100004)) == -3
+    assert call(ws=None) == -5
+    assert call(wsb=wsb - 1) == -5
