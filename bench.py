@@ -166,6 +166,12 @@ def run_own(args):
         if rank == 0:
             print(json.dumps({"only": "block", "block": blk}))
         return
+    if args.only == "backward":
+        bwd = run_backward(torch, rglru, inputs, dev, stream, flush, _peaks(), max_over_ranks, world, reps=3)
+        replicas.shutdown(rk)
+        if rank == 0:
+            print(json.dumps({"only": "backward", "backward": bwd}))
+        return
 
     def forward_step():
         # the timed step: one rglru_forward call (conv, gate GEMM forming the recurrence
@@ -326,6 +332,8 @@ def run_own(args):
 
     # ---- recurrent block ------------------------------------------------------------------
     blk = run_block(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world)
+    # ---- backward of the forward step ---------------------------------------------------
+    bwd = run_backward(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world)
 
     replicas.shutdown(rk)
     if rank != 0:
@@ -345,6 +353,7 @@ def run_own(args):
                          "peak": pk["hbm_gbs"], "peak_source": pk["source"]},
         "decode": dec,
         "block": blk,
+        "backward": bwd,
         "e2e": e2e,
         "gpu_launches": 3 * K,
         "clocks": clk,
@@ -444,6 +453,40 @@ def run_block(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, worl
             "gpu_launches_per_call": 6, "timing": f"{reps} calls, L2 flushed before each"}
 
 
+def run_backward(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world, reps=5):
+    """The backward of the forward step (rglru_backward at the forward workload: recompute
+    of u and z, the chunked reverse recurrence with the gate gradients, the ∂u and weight
+    gradient GEMMs on transposed copies, the Conv1D backward), L2 flushed before each call."""
+    B, T, R = WORKLOAD["B"], WORKLOAD["T"], WORKLOAD["R"]
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=0)
+    p = rglru.Params.from_host(w.params, dev)
+    x = w.x.to(dev)
+    y, _, _ = rglru.forward(p, x)
+    g = torch.Generator("cpu").manual_seed(1)
+    dy = torch.randn(B, T, R, generator=g).to(torch.bfloat16).to(dev)
+    ws = torch.empty(rglru.backward_workspace_bytes(B, T, R), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        rglru.backward(p, x, y, dy, workspace=ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        rglru.backward(p, x, y, dy, workspace=ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / reps)
+    n_tok = B * T
+    # tensor-core work: z recomputed (2·N·2R·R), ∂u (2·N·2R·R), ∂W_a and ∂W_x (2·2R·R·N)
+    flops = 3 * 2.0 * n_tok * (2 * R) * R
+    status = rglru.workspace_status(ws)
+    del ws, x, y, dy
+    return {"workload": f"RG-LRU backward B={B} T={T} D_RNN={R} bf16 (dL/dy given)", "ms_per_call": ms,
+            "tokens_per_s": world * n_tok / (ms / 1e3), "gemm_flops_per_call": flops,
+            "gemm_TFLOP/s_over_the_call": flops / ms / 1e9, "status": status, "gpu_launches_per_call": 14,
+            "timing": f"{reps} calls, L2 flushed before each"}
+
+
 # ------------------------------------------------------------------------------ CPU side
 def _host_cores():
     try:
@@ -538,7 +581,7 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
-    ap.add_argument("--only", choices=["all", "forward", "decode", "block"], default="all",
+    ap.add_argument("--only", choices=["all", "forward", "decode", "block", "backward"], default="all",
                     help="forward / decode / block: time that part only (small commands for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -269,28 +269,42 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, Bw
 }
 
 // out[j][i] = in[i][j] for a rows × cols bf16 matrix (leading dimensions ld_in, ld_out);
-// columns cols..cols_pad−1 of out (rows of in past `rows`) are written as zeros.
+// columns rows..rows_pad−1 of out are written as zeros. 64 × 64 tiles through shared
+// memory with 16-byte loads and stores: cols, ld_in, ld_out and rows_pad are multiples of 8
+// and both pointers 16-byte aligned.
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in,
                                                              __nv_bfloat16* __restrict__ out, int64_t rows,
                                                              int64_t cols, int64_t ld_in, int64_t ld_out,
                                                              int64_t rows_pad) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
-  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;  // 32 × 8
-  for (int k = ty; k < 32; k += 8) {
-    const int64_t r = r0 + k, c = c0 + tx;
-    tile[k][tx] = (r < rows && c < cols) ? in[r * ld_in + c] : __float2bfloat16(0.0f);
+  __shared__ __align__(16) __nv_bfloat16 tile[64][72];  // rows padded to 144 bytes
+  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
+  for (int i = threadIdx.x; i < 512; i += 256) {
+    const int rr = i / 8, cv = i % 8;
+    const int64_t r = r0 + rr, c = c0 + cv * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < rows && c < cols) v = *reinterpret_cast<const uint4*>(in + r * ld_in + c);
+    *reinterpret_cast<uint4*>(&tile[rr][cv * 8]) = v;
   }
   __syncthreads();
-  for (int k = ty; k < 32; k += 8) {
-    const int64_t c = c0 + k, r = r0 + tx;  // out row c, column r
-    if (c < cols && r < rows_pad) out[c * ld_out + r] = tile[tx][k];
+  for (int i = threadIdx.x; i < 512; i += 256) {
+    const int cc = i / 8, rv = i % 8;
+    const int64_t c = c0 + cc, r = r0 + rv * 8;
+    if (c < cols && r < rows_pad) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 pr = __halves2bfloat162(tile[rv * 8 + 2 * q][cc], tile[rv * 8 + 2 * q + 1][cc]);
+        w[q] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+      *reinterpret_cast<uint4*>(out + c * ld_out + r) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
 cudaError_t transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols, int64_t ld_in, int64_t ld_out,
                            int64_t rows_pad, cudaStream_t s) {
-  const dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows_pad + 31) / 32));
+  if (cols % 8 || ld_in % 8 || ld_out % 8 || rows_pad % 8) return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows_pad + 63) / 64));
   if (grid.y > 65535u) return cudaErrorInvalidValue;
   transpose_bf16_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out),
                                               rows, cols, ld_in, ld_out, rows_pad);
