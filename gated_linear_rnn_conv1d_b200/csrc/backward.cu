@@ -192,7 +192,7 @@ struct BwdConvArgs {
   const __nv_bfloat16* state0;  // [B][3][R] (x_{−3}, x_{−2}, x_{−1}) or null
   const float* conv_w;          // [4][R]
   const float* du;              // [B][T][R] direct term
-  const __nv_bfloat16* dug;     // [B][T][R] gate-GEMM term
+  const float* dug;             // [B][T][R] gate-GEMM term
   __nv_bfloat16* dx;            // [B][T][R]
   __nv_bfloat16* dstate0;       // [B][3][R] or null
   float* dconv_w;               // [4][R] (atomic)
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, Bw
   auto du_at = [&](int t) -> float2 {  // total ∂ℓ/∂u_t, zero past T
     if (t >= d.T) return make_float2(0.f, 0.f);
     const float2 p = *reinterpret_cast<const float2*>(a.du + base + (int64_t)t * d.R);
-    const float2 q = ld_bf2(a.dug + base + (int64_t)t * d.R);
+    const float2 q = *reinterpret_cast<const float2*>(a.dug + base + (int64_t)t * d.R);
     return make_float2(p.x + q.x, p.y + q.y);
   };
   auto x_at = [&](int t) -> float2 {  // x_t, from the conv history for t < 0
@@ -327,7 +327,7 @@ BwdLayout bwd_layout(int B, int T, int R) {
   L.off_gin = o;    o += r256((size_t)B * n_chunks * R * 4);
   L.off_dz = o;     o += r256((size_t)n * 2 * R * 2);
   L.off_du = o;     o += r256((size_t)n * R * 4);
-  L.off_dug = o;    o += r256((size_t)n * R * 2);
+  L.off_dug = o;    o += r256((size_t)n * R * 4);
   L.off_wt = o;     o += r256((size_t)2 * R * R * 2);
   L.off_dzt = o;    o += r256((size_t)2 * R * np * 2);
   L.off_ut = o;     o += r256((size_t)R * np * 2);
@@ -350,7 +350,7 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   float* gin = reinterpret_cast<float*>(w + L.off_gin);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(w + L.off_dz);
   float* du = reinterpret_cast<float*>(w + L.off_du);
-  __nv_bfloat16* dug = reinterpret_cast<__nv_bfloat16*>(w + L.off_dug);
+  float* dug = reinterpret_cast<float*>(w + L.off_dug);
   __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(w + L.off_wt);
   __nv_bfloat16* dzt = reinterpret_cast<__nv_bfloat16*>(w + L.off_dzt);
   __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(w + L.off_ut);
@@ -382,7 +382,8 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   // ∂ℓ/∂u ⊃ [∂z_a | ∂z_x]·[W_a; W_x]: B operand [W_a; W_x]ᵀ = [R][2R]
   if ((e = transpose_bf16(g.W_a, wt, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
   if ((e = transpose_bf16(g.W_x, wt + R, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
-  if ((e = launch_gemm_bf16(dz, wt, dug, n, R, 2 * R, R, status, s)) != cudaSuccess) return e;
+  // (in float32: this term reaches ∂x through the Conv1D backward without another rounding)
+  if ((e = launch_gemm_f32out(dz, wt, dug, n, R, 2 * R, R, status, s)) != cudaSuccess) return e;
   // ∂W_a = ∂z_aᵀ u, ∂W_x = ∂z_xᵀ u over the tokens (K = tokens, zero-padded to n_pad)
   if ((e = transpose_bf16(dz, dzt, n, 2 * R, 2 * R, L.n_pad, L.n_pad, s)) != cudaSuccess) return e;
   if ((e = transpose_bf16(u, ut, n, R, R, L.n_pad, L.n_pad, s)) != cudaSuccess) return e;

@@ -123,7 +123,7 @@ cudaError_t launch_gemm_gates_f32(const float* u, const float* Wa, const float* 
 
 // ---- backward (bf16 IO) --------------------------------------------------------------
 // Workspace of launch_backward: [status | u | z | chunk maps P, Q | chunk carries | ∂z |
-// direct ∂u (f32) | gate-GEMM ∂u | [W_a; W_x]ᵀ | ∂zᵀ | uᵀ | Σ ∂log a·r·c].
+// direct ∂u (f32) | gate-GEMM ∂u (f32) | [W_a; W_x]ᵀ | ∂zᵀ | uᵀ | Σ ∂log a·r·c].
 struct BwdLayout {
   size_t off_u, off_z, off_P, off_Q, off_gin, off_dz, off_du, off_dug, off_wt, off_dzt, off_ut, off_dL, bytes;
   int64_t n_pad;  // tokens rounded up to 64 (the transposed operands' row length)

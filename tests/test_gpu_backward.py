@@ -44,7 +44,7 @@ def _dev(t):
 
 
 @pytest.mark.parametrize("B,T,R,with_state", [(2, 200, 264, True), (1, 65, 8, False), (3, 130, 136, True),
-                                               (2, 64, 128, False), (1, 1, 16, True)])
+                                               (2, 64, 128, False), (1, 1, 16, True), (2, 1024, 1024, True)])
 def test_backward_matches_oracle(B, T, R, with_state):
     w, h0, st0, dy, dh_T = _problem(B, T, R, with_state, seed=B * 1000 + T + R)
     p = rglru.Params.from_host(w.params)
