@@ -413,3 +413,40 @@ def test_backward_of_a_frozen_state_is_plain_accumulation():
     assert np.allclose(G["dh0"], dy.sum(axis=1) + dh_T, rtol=1e-13, atol=1e-13)
     for k in ("dx", "dconv_w", "dconv_b", "dW_x", "db_x", "dLambda"):
         assert np.all(G[k] == 0.0), k
+
+
+def test_backward_pins_reject_planted_mistakes():
+    """Plausible slips in a backward — the derivative of log σ(Λ) taken as σ(Λ) instead of
+    σ(−Λ), a weight gradient transposed, ∂h0 missing the first step's decay a_0 — are each
+    rejected by the central-difference comparison used above."""
+    P, dy, dh_T = _bwd_problem(9, 1.0, 4.0)
+    G = oracle.rglru_backward(P["x"], P["conv_w"], P["conv_b"], P["W_a"], P["b_a"], P["W_x"], P["b_x"],
+                              P["Lambda"], dy, h0=P["h0"], conv_state0=P["conv_state0"], dh_T=dh_T)
+
+    def fd(name):
+        out = np.empty_like(P[name])
+        for idx in np.ndindex(P[name].shape):
+            orig = P[name][idx]
+            P[name][idx] = orig + 1e-6
+            lp = _loss(P, dy, dh_T)
+            P[name][idx] = orig - 1e-6
+            lm = _loss(P, dy, dh_T)
+            P[name][idx] = orig
+            out[idx] = (lp - lm) / 2e-6
+        return out
+
+    def agrees(g, ref):
+        return np.max(np.abs(g - ref)) <= 1e-6 * max(float(np.max(np.abs(ref))), 1e-3)
+
+    ref_L, ref_Wa = fd("Lambda"), fd("W_a")
+    assert agrees(G["dLambda"], ref_L) and agrees(G["dW_a"], ref_Wa)
+    s_pos = 1.0 / (1.0 + np.exp(-P["Lambda"]))
+    assert not agrees(G["dLambda"] / (1.0 - s_pos) * s_pos, ref_L)          # σ(Λ) for σ(−Λ)
+    assert not agrees(G["dW_a"].T, ref_Wa)                                   # transposed ∂W
+    # ∂h0 taken as g_0 (the gradient at h_0) without the last step's decay a_0
+    u, _ = oracle.conv1d_causal(P["x"], P["conv_w"], P["conv_b"], P["conv_state0"])
+    z_a, _ = oracle.gate_preactivations(u[:, 0], P["W_a"], P["b_a"], P["W_x"], P["b_x"])
+    a0 = oracle.decay_direct(oracle.sigmoid(z_a), P["Lambda"])
+    ref_h0 = fd("h0")
+    assert agrees(G["dh0"], ref_h0)
+    assert not agrees(G["dh0"] / a0, ref_h0)
