@@ -16,6 +16,9 @@ It is the plain definition, written out in float64 with numpy:
   * the same page, §循环块 (recurrent block): two D → D_RNN linears; branch 1 is a
     width-4 Conv1D followed by the RG-LRU, branch 2 is GeLU; the branches are
     multiplied elementwise and a final D_RNN → D linear follows.
+  * the same page, §残块 (residual block, Fig. 2(a)) and §MLP块 (Fig. 2(b)): RMSNorm
+    ahead of the temporal-mixing block and of a gated MLP (two D → M·D linears, GeLU
+    on one, elementwise product, M·D → D linear), each merged with its skip connection.
   * "Griffin's Compromise: Combining Gated Linear Recurrence with Local Attention",
     §Hawk: during generation the layer reads and writes only the current token and
     a fixed-size state (the decode step below).
@@ -23,7 +26,8 @@ It is the plain definition, written out in float64 with numpy:
 Readings where the pages are silent (each one is listed with its reason in the
 design notes): the Conv1D is causal with zero left padding, per channel, with a
 bias, tap k multiplying x_{t-3+k}; W_a and W_x are dense D_RNN × D_RNN; GeLU is the
-exact erf form; the block linears have no bias.
+exact erf form; the block and MLP linears have no bias; RMSNorm has a per-channel
+gain and ε = 1e-6.
 
 a_t is evaluated as the direct power a**(c*r_t) in float64. The log-space form the
 page prescribes for numerical stability is kept as its own function
@@ -198,6 +202,43 @@ def recurrent_block(x, W_1, W_2, W_o, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda
     h, h_T, _ = rglru_forward(v, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda, h0, c=c)
     p = h * gelu(g)
     out = p @ _f64(W_o).T
+    return out, h_T
+
+
+# ε of RMSNorm: the page gives none; 1e-6 is taken (a reading, listed in the design notes).
+RMS_EPS = 1e-6
+
+
+def rms_norm(x, scale, eps=RMS_EPS):
+    """RMSNorm (Zhang & Sennrich, 2019) over the last axis, as the residual block applies
+    it ahead of each of its two sub-blocks (§残块, Fig. 2(a)):
+        n = x / √(mean_j x_j² + ε) ⊙ scale,   scale [D] a per-channel gain, no bias."""
+    x = _f64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * _f64(scale)
+
+
+def gated_mlp(x, W_gate, W_up, W_down):
+    """Gated MLP block (§MLP块, Fig. 2(b)): two D → M·D linears, GeLU on the first
+    (gate) branch, the branches multiplied elementwise, then an M·D → D linear.
+    W_gate, W_up [M·D][D]; W_down [D][M·D]; no biases."""
+    x = _f64(x)
+    return (gelu(x @ _f64(W_gate).T) * (x @ _f64(W_up).T)) @ _f64(W_down).T
+
+
+def hawk_residual_layer(x, norm1_scale, W_1, W_2, W_o, norm2_scale, W_gate, W_up, W_down,
+                        conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda, h0=None, eps=RMS_EPS, c=C_DECAY):
+    """One residual block of Hawk (§残块, Fig. 2(a)) with the recurrent block as its
+    temporal-mixing block. Two components in sequence, each pre-normed and merged with
+    the skip connection from its own RMSNorm input:
+        y   = x + RecurrentBlock(RMSNorm₁(x))
+        out = y + MLP(RMSNorm₂(y))
+    Returns out [B][T][D] and the RG-LRU's h_T."""
+    x = _f64(x)
+    o, h_T = recurrent_block(rms_norm(x, norm1_scale, eps), W_1, W_2, W_o, conv_w, conv_b, W_a, b_a,
+                             W_x, b_x, Lambda, h0, c=c)
+    y = x + o
+    out = y + gated_mlp(rms_norm(y, norm2_scale, eps), W_gate, W_up, W_down)
     return out, h_T
 
 

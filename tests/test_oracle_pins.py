@@ -450,3 +450,94 @@ def test_backward_pins_reject_planted_mistakes():
     ref_h0 = fd("h0")
     assert agrees(G["dh0"], ref_h0)
     assert not agrees(G["dh0"] / a0, ref_h0)
+
+
+# ------------------------------------------------------------------------------------
+# Hawk residual layer: RMSNorm, gated MLP and their wiring around the recurrent block
+# ("Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §残块, Fig. 2(a);
+# §MLP块, Fig. 2(b)).
+def test_rms_norm_worked_example_and_invariants():
+    # x = (3, 4): mean square 12.5; gain (1, 2)
+    n = oracle.rms_norm(np.array([3.0, 4.0]), np.array([1.0, 2.0]), eps=0.0)
+    np.testing.assert_allclose(n, [3 / math.sqrt(12.5), 8 / math.sqrt(12.5)], rtol=1e-15)
+    # ε enters under the root: x = (1, 1, 1, 1), ε = 3 ⇒ 1/√(1 + 3) = 1/2
+    np.testing.assert_allclose(oracle.rms_norm(np.ones(4), np.ones(4), eps=3.0), 0.5 * np.ones(4), rtol=1e-15)
+    # an all-zero row stays zero (ε keeps the root away from zero)
+    assert np.array_equal(oracle.rms_norm(np.zeros((2, 8)), np.ones(8)), np.zeros((2, 8)))
+    rng = np.random.default_rng(11)
+    x = rng.normal(0, 3, (5, 7, 64))
+    ones = np.ones(64)
+    n = oracle.rms_norm(x, ones, eps=0.0)
+    # unit gain, ε = 0: every row has mean square exactly 1 (up to rounding)
+    np.testing.assert_allclose(np.mean(n * n, axis=-1), 1.0, rtol=1e-13)
+    # scale invariance per row, odd symmetry, and the gain multiplies channel by channel
+    c = rng.uniform(0.1, 10, (5, 7, 1))
+    np.testing.assert_allclose(oracle.rms_norm(c * x, ones, eps=0.0), n, rtol=1e-12)
+    np.testing.assert_allclose(oracle.rms_norm(-x, ones, eps=0.0), -n, rtol=1e-15)
+    gam = rng.uniform(0.5, 1.5, 64)
+    np.testing.assert_allclose(oracle.rms_norm(x, gam, eps=0.0), n * gam, rtol=1e-15)
+
+
+def test_gated_mlp_worked_example_and_branch_roles():
+    Phi1, Phi2 = 0.8413447460685429, 0.9772498680518208  # standard normal table: Φ(1), Φ(2)
+    I2 = np.eye(2)
+    # identity gate and down projections, up = 2·I: out_j = GeLU(x_j) · 2 x_j
+    out = oracle.gated_mlp(np.array([1.0, -1.0]), I2, 2 * I2, I2)
+    np.testing.assert_allclose(out, [2 * Phi1, 2 * (1 - Phi1)], rtol=1e-15)
+    # GeLU sits on the gate branch only: swapping the two branches gives GeLU(2)·1 = 2Φ(2)
+    swapped = oracle.gated_mlp(np.array([1.0, -1.0]), 2 * I2, I2, I2)
+    np.testing.assert_allclose(swapped[0], 2 * Phi2, rtol=1e-15)
+    # a zero gate projection zeroes the block (GeLU(0) = 0)
+    rng = np.random.default_rng(12)
+    x = rng.normal(0, 1, (3, 16))
+    Wu, Wd = rng.normal(0, 0.25, (48, 16)), rng.normal(0, 0.15, (16, 48))
+    assert np.array_equal(oracle.gated_mlp(x, np.zeros((48, 16)), Wu, Wd), np.zeros((3, 16)))
+    # library cross-check: torch's exact GeLU and matmuls in float64
+    Wg = rng.normal(0, 0.25, (48, 16))
+    xt = torch.from_numpy(x)
+    ref = (torch.nn.functional.gelu(xt @ torch.from_numpy(Wg).T) * (xt @ torch.from_numpy(Wu).T)) \
+        @ torch.from_numpy(Wd).T
+    np.testing.assert_allclose(oracle.gated_mlp(x, Wg, Wu, Wd), ref.numpy(), rtol=1e-12, atol=1e-14)
+
+
+def test_hawk_layer_worked_example():
+    ex = _parse_golden(GOLDEN)["hawk_layer"]
+    m = lambda k: ex[k].reshape(1, 1)  # noqa: E731
+    out, h_T = oracle.hawk_residual_layer(
+        ex["x"].reshape(1, 1, 1), ex["norm1_scale"], m("W_1"), m("W_2"), m("W_o"), ex["norm2_scale"],
+        m("W_gate"), m("W_up"), m("W_down"), ex["conv_w"].reshape(4, 1), ex["conv_b"], np.zeros((1, 1)),
+        np.zeros(1), np.zeros((1, 1)), np.zeros(1), ex["Lambda"], eps=0.0)
+    np.testing.assert_allclose(h_T.ravel(), ex["h_T"], rtol=1e-14)
+    np.testing.assert_allclose(out.ravel(), ex["out"], rtol=1e-14)
+    # the residual stream between the two components, through the zero-MLP special case
+    y, _ = oracle.hawk_residual_layer(
+        ex["x"].reshape(1, 1, 1), ex["norm1_scale"], m("W_1"), m("W_2"), m("W_o"), ex["norm2_scale"],
+        m("W_gate"), m("W_up"), np.zeros((1, 1)), ex["conv_w"].reshape(4, 1), ex["conv_b"], np.zeros((1, 1)),
+        np.zeros(1), np.zeros((1, 1)), np.zeros(1), ex["Lambda"], eps=0.0)
+    np.testing.assert_allclose(y.ravel(), ex["y"], rtol=1e-14)
+
+
+def test_hawk_layer_zero_branches_and_block_special_case():
+    rng = np.random.default_rng(13)
+    B, T, D, R = 2, 9, 16, 24
+    P = _rng_params(rng, R)
+    x = rng.normal(0, 1, (B, T, D))
+    W_1, W_2 = rng.normal(0, 0.25, (R, D)), rng.normal(0, 0.25, (R, D))
+    W_o = rng.normal(0, 0.2, (D, R))
+    Wg, Wu, Wd = rng.normal(0, 0.25, (3 * D, D)), rng.normal(0, 0.25, (3 * D, D)), rng.normal(0, 0.15, (D, 3 * D))
+    g1, g2 = rng.uniform(0.5, 1.5, D), rng.uniform(0.5, 1.5, D)
+    # both output projections zero: the layer is the identity on its input, bitwise
+    out, _ = oracle.hawk_residual_layer(x, g1, W_1, W_2, np.zeros((D, R)), g2, Wg, Wu, np.zeros((D, 3 * D)), **P)
+    assert np.array_equal(out, x)
+    # zero MLP output projection: x plus the recurrent block of the normalised input
+    out, h_T = oracle.hawk_residual_layer(x, g1, W_1, W_2, W_o, g2, Wg, Wu, np.zeros((D, 3 * D)), **P)
+    n1 = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + oracle.RMS_EPS) * g1
+    blk, h_blk = oracle.recurrent_block(n1, W_1, W_2, W_o, **P)
+    np.testing.assert_allclose(out, x + blk, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(h_T, h_blk)
+    # the layer is causal: changing the last step leaves every earlier output unchanged
+    x2 = x.copy()
+    x2[:, -1, :] += 1.0
+    o1, _ = oracle.hawk_residual_layer(x, g1, W_1, W_2, W_o, g2, Wg, Wu, Wd, **P)
+    o2, _ = oracle.hawk_residual_layer(x2, g1, W_1, W_2, W_o, g2, Wg, Wu, Wd, **P)
+    assert np.array_equal(o1[:, :-1], o2[:, :-1]) and not np.allclose(o1[:, -1], o2[:, -1])
