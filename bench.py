@@ -166,6 +166,12 @@ def run_own(args):
         if rank == 0:
             print(json.dumps({"only": "block", "block": blk}))
         return
+    if args.only == "layer":
+        lay = run_layer(torch, rglru, inputs, dev, stream, flush, _peaks(), max_over_ranks, world)
+        replicas.shutdown(rk)
+        if rank == 0:
+            print(json.dumps({"only": "layer", "layer": lay}))
+        return
     if args.only == "backward":
         bwd = run_backward(torch, rglru, inputs, dev, stream, flush, _peaks(), max_over_ranks, world, reps=3)
         replicas.shutdown(rk)
@@ -453,6 +459,43 @@ def run_block(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, worl
             "gpu_launches_per_call": 6, "timing": f"{reps} calls, L2 flushed before each"}
 
 
+def run_layer(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world, reps=3):
+    """One Hawk residual layer at the recurrent block's sizes with the gated MLP (M = 3):
+    RMSNorm, the recurrent block, residual add fused with the second RMSNorm, the MLP's
+    three linears and GeLU product, residual add — one rglru_layer_forward call, L2
+    flushed before each timed call."""
+    B, T, D, R, M = BLOCK["B"], BLOCK["T"], BLOCK["D"], BLOCK["R"], 3
+    H = M * D
+    w = inputs.make_layer(B, T, D, R, M, torch.bfloat16, seed=0)
+    p = rglru.Params.from_host(w.params, dev)
+    lw = rglru.LayerWeights.from_host(w, dev)
+    x = w.x.to(dev)
+    out = torch.empty_like(x)
+    h_T = torch.empty(B, R, dtype=torch.float32, device=dev)
+    ws = torch.empty(rglru.layer_workspace_bytes(B, T, D, R, H), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        rglru.layer_forward(p, lw, x, workspace=ws, out=out, h_T=h_T)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        rglru.layer_forward(p, lw, x, workspace=ws, out=out, h_T=h_T)
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / reps)
+    n_tok = B * T
+    flops = 2.0 * n_tok * (2 * D * R + 2 * R * R + R * D) + 2.0 * n_tok * 3 * D * H
+    peak = pk["bf16_tflops_sustained"] or pk["bf16_tflops"]
+    status = rglru.workspace_status(ws)
+    del ws, out, x, lw
+    return {"workload": f"Hawk residual layer B={B} T={T} D={D} D_RNN={R} MLP {H} bf16", "ms_per_call": ms,
+            "tokens_per_s": world * n_tok / (ms / 1e3), "flops_per_call": flops, "TFLOP/s": flops / ms / 1e9,
+            "peak_TFLOP/s": peak, "frac_tensor": flops / ms / 1e9 / peak,
+            "peak_source": "measured sustained bf16 (a multi-ms call)", "status": status,
+            "gpu_launches_per_call": 13, "timing": f"{reps} calls, L2 flushed before each"}
+
+
 def run_backward(torch, rglru, inputs, dev, stream, flush, pk, max_over_ranks, world, reps=5):
     """The backward of the forward step (rglru_backward at the forward workload: recompute
     of u and z, the chunked reverse recurrence with the gate gradients, the ∂u and weight
@@ -581,7 +624,7 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
-    ap.add_argument("--only", choices=["all", "forward", "decode", "block", "backward"], default="all",
+    ap.add_argument("--only", choices=["all", "forward", "decode", "block", "backward", "layer"], default="all",
                     help="forward / decode / block: time that part only (small commands for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -39,6 +39,14 @@ class RGLRUGrads(ctypes.Structure):
 
 _GP = ctypes.POINTER(RGLRUGrads)
 
+
+class RGLRULayerWeights(ctypes.Structure):
+    _fields_ = [("norm1_scale", _P), ("W_1", _P), ("W_2", _P), ("W_o", _P), ("norm2_scale", _P), ("W_gate", _P),
+                ("W_up", _P), ("W_down", _P)]
+
+
+_LWP = ctypes.POINTER(RGLRULayerWeights)
+
 SIGNATURES = {
     "rglru_forward_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "rglru_forward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
@@ -46,6 +54,8 @@ SIGNATURES = {
     "rglru_step": (_I, [_PP, _P, _P, _P, _P, _I, _I, _L, _I, _P, _S, _P]),
     "rglru_block_workspace_bytes": (_S, [_I, _I, _I, _I, _I]),
     "rglru_block_forward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P]),
+    "rglru_layer_workspace_bytes": (_S, [_I, _I, _I, _I, _I, _I]),
+    "rglru_layer_forward": (_I, [_PP, _LWP, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _S, _P]),
     "rglru_conv1d": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "rglru_gate_pitch": (_L, [_I]),
     "rglru_gate_proj": (_I, [_P, _P, _P, _P, _P, _P, _L, _I, _I, _P]),

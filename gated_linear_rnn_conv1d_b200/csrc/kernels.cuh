@@ -121,6 +121,14 @@ unsigned* global_status_word();
 cudaError_t launch_gemm_gates_f32(const float* u, const float* Wa, const float* ba, const float* Wx,
                                   const float* bx, float* z, int64_t M, int R, cudaStream_t s);
 
+// ---- Hawk residual layer: elementwise kernels (bf16, 16-byte aligned, D % 8 == 0) ------
+// y = x + o (skipped if o is null; y then unused) and n = RMSNorm(y or x) ⊙ scale (skipped
+// if n is null) over rows of D channels; x, o, y, n distinct.
+cudaError_t launch_add_rmsnorm(const void* x, const void* o, void* y, void* n, const float* scale, int64_t rows,
+                               int D, float eps, cudaStream_t s);
+// p = GeLU(gate) ⊙ up over n elements (n % 8 == 0); p may be gate.
+cudaError_t launch_gelu_mul(const void* gate, const void* up, void* p, int64_t n, cudaStream_t s);
+
 // ---- backward (bf16 IO) --------------------------------------------------------------
 // Workspace of launch_backward: [status | u | z | chunk maps P, Q | chunk carries | ∂z |
 // direct ∂u (f32) | gate-GEMM ∂u (f32) | [W_a; W_x]ᵀ | ∂zᵀ | uᵀ | Σ ∂log a·r·c].

@@ -153,6 +153,66 @@ StepLayout step_layout(int B, int R) {
 
 uint8_t* bytes(void* p) { return static_cast<uint8_t*>(p); }
 
+// Hawk residual layer: [recurrent block workspace (status word at 0) | n: RMSNorm output
+// [B·T][D] (RMSNorm₁, then RMSNorm₂) | o: component output [B·T][D] (the block's, then
+// the MLP's) | y: residual stream [B·T][D] | gate (then p) [B·T][H] | up [B·T][H]], bf16.
+struct LayerLayout {
+  BlockLayout block;
+  size_t off_n, off_o, off_y, off_gate, off_up, bytes;
+};
+LayerLayout layer_layout(int B, int T, int D, int R, int H) {
+  LayerLayout L;
+  L.block = block_layout(B, T, R);
+  const size_t ntok = (size_t)B * T;
+  const size_t actD = round256(ntok * D * 2), actH = round256(ntok * H * 2);
+  L.off_n = round256(L.block.bytes);
+  L.off_o = L.off_n + actD;
+  L.off_y = L.off_o + actD;
+  L.off_gate = L.off_y + actD;
+  L.off_up = L.off_gate + actH;
+  L.bytes = L.off_up + actH;
+  return L;
+}
+
+// The recurrent block (§循环块, Fig. 2(c)) after its status word is zeroed: the two
+// D → D_RNN linears, Conv1D, the coefficient GEMM, the gated scan (p = h ⊙ GeLU(g)) and
+// the D_RNN → D linear, queued on s with the block workspace layout L.
+cudaError_t block_sequence(const rglru_params* params, const void* W_1, const void* W_2, const void* W_o,
+                           const void* x, const float* h0, void* out, float* h_T, int B, int T, int D, int R,
+                           const BlockLayout& L, void* workspace, cudaStream_t s) {
+  const int64_t ntok = (int64_t)B * T;
+  void* v = bytes(workspace) + L.off_v;
+  void* g = bytes(workspace) + L.off_g;
+  void* u = bytes(workspace) + L.off_u;
+  void* z = bytes(workspace) + L.off_z;
+  void* pbuf = bytes(workspace) + L.off_p;
+  unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  cudaError_t e = launch_gemm_bf16(x, W_1, v, ntok, R, D, R, status, s);  // v = x W_1ᵀ
+  if (e == cudaSuccess) e = launch_gemm_bf16(x, W_2, g, ntok, R, D, R, status, s);        // g = x W_2ᵀ
+  if (e == cudaSuccess)
+    e = launch_conv1d(params->conv_w, params->conv_b, v, nullptr, u, nullptr, B, T, R, true, status, s);
+  if (e == cudaSuccess)
+    e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, z, ntok, R,
+                                status, s);
+  if (e == cudaSuccess) {
+    // the scan's memset must not clear a status bit the GEMMs above may have set:
+    // zero only the ticket and flags here.
+    e = cudaMemsetAsync(bytes(workspace) + 4, 0, L.scan.zero_bytes - 4, s);
+    if (e == cudaSuccess) {
+      ScanArgs a{};
+      a.z = z; a.h0 = h0; a.g = g; a.y = pbuf; a.hT = h_T;  // coefficients: no x or conv parameters
+      a.status = status;
+      a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
+      a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);
+      a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks;
+      a.n_tiles = (int)L.scan.n_tiles; a.pitch = gate_pitch(R);
+      e = launch_scan(a, true, s, true);
+    }
+  }
+  if (e == cudaSuccess) e = launch_gemm_bf16(pbuf, W_o, out, ntok, D, R, D, status, s);  // out = p W_oᵀ
+  return e;
+}
+
 // Queues the scan; with zero_first, first zeroes the status word, the ticket counter and
 // the look-back flags (which must be zero when the scan starts).
 // coef: z holds the recurrence coefficients of launch_gemm_coeffs_bf16, not pre-activations;
@@ -491,37 +551,57 @@ int rglru_block_forward(const rglru_params* params, const void* W_1, const void*
   if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
   if ((st = check_device()) != RGLRU_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess) e = block_sequence(params, W_1, W_2, W_o, x, h0, out, h_T, B, T, D, R, L, workspace, s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+size_t rglru_layer_workspace_bytes(int B, int T, int D, int R, int H, int io_dtype) {
+  if (io_dtype != RGLRU_BF16 || !valid_R(R) || !valid_R(D) || !valid_R(H) || !valid_tokens(B, T)) return 0;
+  return layer_layout(B, T, D, R, H).bytes;
+}
+
+int rglru_layer_forward(const rglru_params* params, const rglru_layer_weights* w, const void* x, const float* h0,
+                        void* out, float* h_T, int B, int T, int D, int R, int H, float eps, int io_dtype,
+                        void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_R(D) || !valid_R(H) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  if (!(eps >= 0.0f) || eps > 1.0f) return RGLRU_ERR_SHAPE;  // also rejects NaN
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (w == nullptr || x == nullptr || out == nullptr) return RGLRU_ERR_NULL;
+  if (w->norm1_scale == nullptr || w->W_1 == nullptr || w->W_2 == nullptr || w->W_o == nullptr ||
+      w->norm2_scale == nullptr || w->W_gate == nullptr || w->W_up == nullptr || w->W_down == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(w->norm1_scale) || !aligned16(w->W_1) || !aligned16(w->W_2) || !aligned16(w->W_o) ||
+      !aligned16(w->norm2_scale) || !aligned16(w->W_gate) || !aligned16(w->W_up) || !aligned16(w->W_down) ||
+      !aligned16(x) || !aligned16(out) || !aligned16(h0) || !aligned16(h_T))
+    return RGLRU_ERR_ALIGN;
+  if (out == x) return RGLRU_ERR_SHAPE;  // the residual stream is read after out is written
+  const LayerLayout L = layer_layout(B, T, D, R, H);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
   const int64_t ntok = (int64_t)B * T;
-  void* v = bytes(workspace) + L.off_v;
-  void* g = bytes(workspace) + L.off_g;
-  void* u = bytes(workspace) + L.off_u;
-  void* z = bytes(workspace) + L.off_z;
-  void* pbuf = bytes(workspace) + L.off_p;
+  void* nrm = bytes(workspace) + L.off_n;
+  void* o = bytes(workspace) + L.off_o;
+  void* yres = bytes(workspace) + L.off_y;
+  void* gate = bytes(workspace) + L.off_gate;
+  void* up = bytes(workspace) + L.off_up;
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
   cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
-  if (e == cudaSuccess) e = launch_gemm_bf16(x, W_1, v, ntok, R, D, R, status, s);        // v = x W_1ᵀ
-  if (e == cudaSuccess) e = launch_gemm_bf16(x, W_2, g, ntok, R, D, R, status, s);        // g = x W_2ᵀ
+  // y = x + RecurrentBlock(RMSNorm₁(x))
+  if (e == cudaSuccess) e = launch_add_rmsnorm(x, nullptr, nullptr, nrm, w->norm1_scale, ntok, D, eps, s);
   if (e == cudaSuccess)
-    e = launch_conv1d(params->conv_w, params->conv_b, v, nullptr, u, nullptr, B, T, R, true, status, s);
-  if (e == cudaSuccess)
-    e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, z, ntok, R,
-                                status, s);
-  if (e == cudaSuccess) {
-    // the scan's memset must not clear a status bit the GEMMs above may have set:
-    // zero only the ticket and flags here.
-    e = cudaMemsetAsync(bytes(workspace) + 4, 0, L.scan.zero_bytes - 4, s);
-    if (e == cudaSuccess) {
-      ScanArgs a{};
-      a.z = z; a.h0 = h0; a.g = g; a.y = pbuf; a.hT = h_T;  // coefficients: no x or conv parameters
-      a.status = status;
-      a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
-      a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);
-      a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks;
-      a.n_tiles = (int)L.scan.n_tiles; a.pitch = gate_pitch(R);
-      e = launch_scan(a, true, s, true);
-    }
-  }
-  if (e == cudaSuccess) e = launch_gemm_bf16(pbuf, W_o, out, ntok, D, R, D, status, s);  // out = p W_oᵀ
+    e = block_sequence(params, w->W_1, w->W_2, w->W_o, nrm, h0, o, h_T, B, T, D, R, L.block, workspace, s);
+  if (e == cudaSuccess) e = launch_add_rmsnorm(x, o, yres, nrm, w->norm2_scale, ntok, D, eps, s);
+  // out = y + (GeLU(n W_gateᵀ) ⊙ n W_upᵀ) W_downᵀ
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_gate, gate, ntok, H, D, H, status, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_up, up, ntok, H, D, H, status, s);
+  if (e == cudaSuccess) e = launch_gelu_mul(gate, up, gate, ntok * H, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(gate, w->W_down, o, ntok, D, H, D, status, s);
+  if (e == cudaSuccess) e = launch_add_rmsnorm(yres, o, out, nullptr, nullptr, ntok, D, eps, s);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 

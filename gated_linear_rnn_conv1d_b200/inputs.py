@@ -15,8 +15,8 @@ D → D_RNN linears plus the D_RNN → D output linear (LeCun normal, no biases)
 Conv weights and bias are N(0, 1/4) (std 0.5); gate biases b_a = b_x = 0; x ~ N(0, 1).
 
 Draw order (one torch CPU generator per workload, seeded):
-    x, conv_w, conv_b, W_a, W_x, s(→Λ), [W_1, W_2, W_o]
-Each draw is float32 and is then cast to the IO dtype where the tensor is IO.
+    x, conv_w, conv_b, W_a, W_x, s(→Λ), [W_1, W_2, W_o, [γ₁, γ₂, W_gate, W_up, W_down]]
+(the bracketed draws for the recurrent block and the Hawk residual layer). Each draw is float32 and is then cast to the IO dtype where the tensor is IO.
 Decode inputs x_t for step k come from their own generator seeded 1_000_003 + k.
 """
 from __future__ import annotations
@@ -94,8 +94,8 @@ def make_forward(B: int, T: int, R: int, io_dtype: torch.dtype = torch.bfloat16,
 
 
 def make_block(B: int, T: int, D: int, R: int, io_dtype: torch.dtype = torch.bfloat16,
-               seed: int = 0, name: str = "") -> Workload:
-    g = torch.Generator("cpu").manual_seed(seed)
+               seed: int = 0, name: str = "", g: Optional[torch.Generator] = None) -> Workload:
+    g = torch.Generator("cpu").manual_seed(seed) if g is None else g
     x = _normal(g, (B, T, D), 1.0).to(io_dtype)
     p = make_params(g, R, io_dtype)
     W_1 = _normal(g, (R, D), 1.0 / math.sqrt(D)).to(io_dtype)
@@ -104,6 +104,23 @@ def make_block(B: int, T: int, D: int, R: int, io_dtype: torch.dtype = torch.bfl
     h0 = torch.zeros(B, R, dtype=torch.float32)
     return Workload(name or f"block_B{B}_T{T}_D{D}_R{R}", B, T, R, io_dtype, x, p, h0,
                     D=D, W_1=W_1, W_2=W_2, W_o=W_o)
+
+
+def make_layer(B: int, T: int, D: int, R: int, M: int = 3, io_dtype: torch.dtype = torch.bfloat16,
+               seed: int = 0, name: str = "") -> Workload:
+    """One Hawk residual layer: the block's draws (same order as make_block), then the two
+    RMSNorm gains ~ U[0.5, 1.5] (float32; a gain other than 1 keeps it visible in the
+    output) and the gated MLP's linears, LeCun normal: W_gate, W_up [M·D][D] (std 1/√D),
+    W_down [D][M·D] (std 1/√(M·D)). All of it goes to `extra`."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    w = make_block(B, T, D, R, io_dtype, seed, name or f"layer_B{B}_T{T}_D{D}_R{R}_M{M}", g=g)
+    H = M * D
+    w.extra["norm1_scale"] = 0.5 + torch.rand(D, generator=g, dtype=torch.float32)
+    w.extra["norm2_scale"] = 0.5 + torch.rand(D, generator=g, dtype=torch.float32)
+    w.extra["W_gate"] = _normal(g, (H, D), 1.0 / math.sqrt(D)).to(io_dtype)
+    w.extra["W_up"] = _normal(g, (H, D), 1.0 / math.sqrt(D)).to(io_dtype)
+    w.extra["W_down"] = _normal(g, (D, H), 1.0 / math.sqrt(H)).to(io_dtype)
+    return w
 
 
 def make_decode(B: int, R: int, io_dtype: torch.dtype = torch.bfloat16, seed: int = 0,

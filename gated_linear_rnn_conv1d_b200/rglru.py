@@ -252,6 +252,58 @@ def block_forward(params: Params, W_1: torch.Tensor, W_2: torch.Tensor, W_o: tor
     return out, h_T
 
 
+@dataclass
+class LayerWeights:
+    """Device-resident weights of one Hawk residual layer besides the RG-LRU parameters
+    (see rglru_layer_weights in include/rglru.h). Linears bf16 [out][in]; gains float32."""
+    norm1_scale: torch.Tensor  # [D]
+    W_1: torch.Tensor          # [R][D]
+    W_2: torch.Tensor          # [R][D]
+    W_o: torch.Tensor          # [D][R]
+    norm2_scale: torch.Tensor  # [D]
+    W_gate: torch.Tensor       # [H][D]
+    W_up: torch.Tensor         # [H][D]
+    W_down: torch.Tensor       # [D][H]
+
+    FIELDS = ("norm1_scale", "W_1", "W_2", "W_o", "norm2_scale", "W_gate", "W_up", "W_down")
+
+    @classmethod
+    def from_host(cls, w, device="cuda") -> "LayerWeights":
+        """Copies an object with the same fields (e.g. an inputs.Workload of a layer) to `device`."""
+        src = w.extra if hasattr(w, "extra") and "W_gate" in w.extra else {}
+        return cls(*((src[f] if f in src else getattr(w, f)).to(device).contiguous() for f in cls.FIELDS))
+
+    @property
+    def H(self) -> int:
+        return self.W_gate.shape[0]
+
+    def struct(self) -> _abi.RGLRULayerWeights:
+        return _abi.RGLRULayerWeights(*(getattr(self, f).data_ptr() for f in self.FIELDS))
+
+
+def layer_workspace_bytes(B: int, T: int, D: int, R: int, H: int) -> int:
+    return _abi.load().rglru_layer_workspace_bytes(B, T, D, R, H, _abi.RGLRU_BF16)
+
+
+def layer_forward(params: Params, weights: LayerWeights, x: torch.Tensor, h0: Optional[torch.Tensor] = None, *,
+                  eps: float = 1e-6, workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  h_T: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """rglru_layer_forward: x [B][T][D] → (out [B][T][D], h_T [B][R])."""
+    lib = _abi.load()
+    B, T, D = x.shape
+    R, H = weights.W_1.shape[0], weights.H
+    io = _io(x)
+    out = torch.empty_like(x) if out is None else out
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_layer_workspace_bytes(B, T, D, R, H, io), x.device, workspace)
+    st, wst = params.struct(), weights.struct()
+    _abi.check("rglru_layer_forward", lib.rglru_layer_forward(
+        ctypes.byref(st), ctypes.byref(wst), _p(x), _p(h0), _p(out), _p(h_T), B, T, D, R, H, float(eps), io, _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return out, h_T
+
+
 def conv1d(params: Params, x: torch.Tensor, conv_state0: Optional[torch.Tensor] = None, *,
            u: Optional[torch.Tensor] = None, conv_state_T: Optional[torch.Tensor] = None,
            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:

@@ -137,6 +137,43 @@ RGLRU_API int rglru_block_forward(const rglru_params* params, const void* W_1, c
                         int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Hawk residual layer ("Griffin：…", §残块, Fig. 2(a); §MLP块, Fig. 2(b)): the recurrent
+ * block as the temporal-mixing block, each component pre-normed by RMSNorm (Zhang &
+ * Sennrich) and merged with the skip connection from its own RMSNorm input:
+ *   y   = x + RecurrentBlock(RMSNorm₁(x))          (the recurrent block above)
+ *   out = y + (GeLU(n W_gateᵀ) ⊙ n W_upᵀ) W_downᵀ,  n = RMSNorm₂(y)
+ *   RMSNorm(v) = v / √(mean_j v_j² + eps) ⊙ scale    (per row of D channels)
+ *
+ *   x, out      [B][T][D] bfloat16, distinct buffers
+ *   W_1, W_2    [R][D]; W_o [D][R]; W_gate, W_up [H][D]; W_down [D][H]: bfloat16,
+ *               row-major [out][in], no biases (H = M·D; the pages use M = 3)
+ *   norm1_scale, norm2_scale  [D] float32 gains
+ *   h0, h_T     [B][R] float32 or NULL, as in rglru_block_forward
+ *   eps         RMSNorm ε, 0 ≤ eps ≤ 1 (1e-6 in the tests)
+ *   workspace   at least rglru_layer_workspace_bytes(B, T, D, R, H, io_dtype) bytes,
+ *               256-byte aligned (the block's buffers plus four [B·T][D] and two
+ *               [B·T][H] bf16 activations)
+ * The residual stream y is rounded to bf16 once, as it is stored; every norm, GeLU and
+ * accumulation is float32. io_dtype must be RGLRU_BF16; D, R, H multiples of 8.
+ * Errors as everywhere: RGLRU_ERR_SHAPE also for out == x or eps outside [0, 1].
+ * --------------------------------------------------------------------------------- */
+typedef struct rglru_layer_weights {
+  const float* norm1_scale; /* [D] RMSNorm gain ahead of the recurrent block */
+  const void* W_1;          /* [R][D] */
+  const void* W_2;          /* [R][D] */
+  const void* W_o;          /* [D][R] */
+  const float* norm2_scale; /* [D] RMSNorm gain ahead of the MLP */
+  const void* W_gate;       /* [H][D], the GeLU branch */
+  const void* W_up;         /* [H][D] */
+  const void* W_down;       /* [D][H] */
+} rglru_layer_weights;
+RGLRU_API size_t rglru_layer_workspace_bytes(int B, int T, int D, int R, int H, int io_dtype);
+RGLRU_API int rglru_layer_forward(const rglru_params* params, const rglru_layer_weights* weights, const void* x,
+                                  const float* h0, void* out, float* h_T, int B, int T, int D, int R, int H,
+                                  float eps, int io_dtype, void* workspace, size_t workspace_bytes,
+                                  rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Backward of rglru_forward for bf16 IO: the gradients of a scalar loss ℓ with respect to
  * the input, the parameters, the initial state and the conv history, given ∂ℓ/∂y and
  * ∂ℓ/∂h_T. Reverse-mode differentiation of Eq. (1)–(4) above (with the log-space decay

@@ -154,3 +154,38 @@ def test_backward_rejects_bad_arguments_before_any_launch():
     assert call(h0=_fake(0x100004)) == -3
     assert call(ws=None) == -5
     assert call(wsb=wsb - 1) == -5
+
+
+def test_layer_rejects_bad_arguments_before_any_launch():
+    lib = _abi.load()
+    p = _params()
+    ok_ptr = _fake()
+    wb = lib.rglru_layer_workspace_bytes(1, 8, 64, 64, 192, 1)
+    assert wb > lib.rglru_block_workspace_bytes(1, 8, 64, 64, 1)
+    assert lib.rglru_layer_workspace_bytes(1, 8, 64, 64, 192, 0) == 0
+    assert lib.rglru_layer_workspace_bytes(1, 8, 64, 64, 190, 1) == 0
+    f = 0x100000
+    weights = _abi.RGLRULayerWeights(f, f, f, f, f, f, f, f)
+    ws = _fake(0x200000)
+
+    def call(**kw):
+        return lib.rglru_layer_forward(
+            ctypes.byref(p), kw.get("w", ctypes.byref(weights)), kw.get("x", ok_ptr), None, kw.get("out", _fake(0x300000)),
+            None, 1, 8, kw.get("D", 64), 64, kw.get("H", 192), kw.get("eps", 1e-6), kw.get("io", 1),
+            kw.get("ws", ws), kw.get("wsb", wb), None)
+
+    assert call(io=0) == -4
+    assert call(D=60) == -2
+    assert call(H=190) == -2
+    assert call(eps=-1.0) == -2
+    assert call(eps=float("nan")) == -2
+    assert call(out=ok_ptr) == -2  # out must not be x
+    assert call(w=None) == -1
+    assert call(x=None) == -1
+    missing = _abi.RGLRULayerWeights(f, f, f, f, f, f, 0, f)
+    assert call(w=ctypes.byref(missing)) == -1
+    odd = _abi.RGLRULayerWeights(f, f, f, f, f + 4, f, f, f)
+    assert call(w=ctypes.byref(odd)) == -3
+    assert call(ws=None) == -5
+    assert call(wsb=wb - 1) == -5
+    assert call(ws=_fake(0x200010)) == -3

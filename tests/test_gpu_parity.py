@@ -410,6 +410,29 @@ def test_block_small_matches_oracle():
     assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
 
 
+# Tolerance of the Hawk residual layer's output: out = x + o₁ + o₂ with o₁ the recurrent
+# block's output (bf16 budget 2e-2 of its own scale, as for the block) and o₂ the MLP's,
+# which adds five bf16 roundings of O(1) quantities (RMSNorm₂ output, gate, up, GeLU product,
+# down projection): 5 · 2⁻⁹ ≈ 1e-2. The two budgets add: 3e-2.
+TOL_LAYER = 3e-2
+
+
+@pytest.mark.parametrize("B,T,D,R,M", [(2, 150, 136, 264, 3)])
+def test_hawk_layer_small_matches_oracle(B, T, D, R, M):
+    w = inputs.make_layer(B, T, D, R, M, torch.bfloat16, seed=7)
+    p = rglru.Params.from_host(w.params)
+    lw = rglru.LayerWeights.from_host(w)
+    out = torch.full((B, T, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = torch.full((rglru.layer_workspace_bytes(B, T, D, R, M * D),), 0xFF, dtype=torch.uint8, device=DEV)
+    out, h_T = rglru.layer_forward(p, lw, w.x.to(DEV), eps=oracle.RMS_EPS, out=out, workspace=ws)
+    assert rglru.workspace_status(ws) == 0
+    e = w.extra
+    ref, h_ref = oracle.hawk_residual_layer(w.x, e["norm1_scale"], w.W_1, w.W_2, w.W_o, e["norm2_scale"],
+                                            e["W_gate"], e["W_up"], e["W_down"], **host_params64(w.params))
+    assert rel(out, ref) <= TOL_LAYER
+    assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
+
+
 # ------------------------------------------------------------------------------------
 # failure detection without a GPU fault: a chunk that never publishes its carry makes
 # its successor's bounded wait run out; the status word reports it and the context
