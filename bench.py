@@ -625,7 +625,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
     ap.add_argument("--only", choices=["all", "forward", "decode", "block", "backward", "layer"], default="all",
-                    help="forward / decode / block: time that part only (small commands for profiler captures)")
+                    help="forward / decode / block / backward / layer: time that part only (small commands for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
