@@ -12,7 +12,7 @@ import torch
 import oracle
 from gated_linear_rnn_conv1d_b200 import _abi, inputs, rglru
 
-from _util import TOL, f64, host_params64, pack_gates, rel, unpack_gates
+from _util import TOL, TOL_LAYER, f64, host_params64, pack_gates, rel, unpack_gates
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -408,13 +408,6 @@ def test_block_small_matches_oracle():
     ref, h_ref = oracle.recurrent_block(w.x, w.W_1, w.W_2, w.W_o, **host_params64(w.params))
     assert rel(out, ref) <= TOL[torch.bfloat16]
     assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
-
-
-# Tolerance of the Hawk residual layer's output: out = x + o₁ + o₂ with o₁ the recurrent
-# block's output (bf16 allowance 2e-2 of its own scale, as for the block) and o₂ the MLP's,
-# which adds five bf16 roundings of O(1) quantities (RMSNorm₂ output, gate, up, GeLU product,
-# down projection): 5 · 2⁻⁹ ≈ 1e-2. The two allowances add: 3e-2.
-TOL_LAYER = 3e-2
 
 
 @pytest.mark.parametrize("B,T,D,R,M", [(2, 150, 136, 264, 3)])
