@@ -5,5 +5,6 @@ benchmark's CPU-baseline leg, never by the product path."""
 from .rglru_oracle import (  # noqa: F401
     C_DECAY, sigmoid, conv1d_causal, gate_preactivations, decay_direct, decay_log_space,
     rglru_recurrence, rglru_forward, ring_to_time_order, rglru_step, gelu,
-    recurrent_block, RMS_EPS, rms_norm, gated_mlp, hawk_residual_layer, rglru_backward, max_rel_error,
+    recurrent_block, RMS_EPS, rms_norm, gated_mlp, hawk_residual_layer,
+    hawk_residual_layer_step, rglru_backward, max_rel_error,
 )

@@ -242,6 +242,26 @@ def hawk_residual_layer(x, norm1_scale, W_1, W_2, W_o, norm2_scale, W_gate, W_up
     return out, h_T
 
 
+def hawk_residual_layer_step(x_t, ring, step, h, norm1_scale, W_1, W_2, W_o, norm2_scale, W_gate, W_up,
+                             W_down, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda, eps=RMS_EPS, c=C_DECAY):
+    """One decode step of the Hawk residual layer: hawk_residual_layer at a single token
+    with the recurrent block's carried state — RMSNorm₁, the block's two linears, one
+    RG-LRU decode step (rglru_step: the conv ring holds the last three inputs of the
+    Conv1D, i.e. of the x W_1ᵀ branch), the GeLU gate, W_o, the residual add, RMSNorm₂,
+    the gated MLP and the second residual add. Every part but the RG-LRU acts on each token
+    alone.
+
+    x_t [B][D]; ring [B][3][R]; h [B][R]. Returns out_t [B][D], the new h, the new ring."""
+    x_t = _f64(x_t)
+    n1 = rms_norm(x_t, norm1_scale, eps)
+    v_t = n1 @ _f64(W_1).T
+    g_t = n1 @ _f64(W_2).T
+    y_t, h_new, ring_new = rglru_step(v_t, ring, step, h, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda, c=c)
+    y = x_t + (y_t * gelu(g_t)) @ _f64(W_o).T
+    out = y + gated_mlp(rms_norm(y, norm2_scale, eps), W_gate, W_up, W_down)
+    return out, h_new, ring_new
+
+
 def rglru_backward(x, conv_w, conv_b, W_a, b_a, W_x, b_x, Lambda, dy, h0=None, conv_state0=None,
                    dh_T=None, c=C_DECAY):
     """Gradients of the full-sequence forward (rglru_forward) by reverse-mode

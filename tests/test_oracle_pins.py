@@ -541,3 +541,25 @@ def test_hawk_layer_zero_branches_and_block_special_case():
     o1, _ = oracle.hawk_residual_layer(x, g1, W_1, W_2, W_o, g2, Wg, Wu, Wd, **P)
     o2, _ = oracle.hawk_residual_layer(x2, g1, W_1, W_2, W_o, g2, Wg, Wu, Wd, **P)
     assert np.array_equal(o1[:, :-1], o2[:, :-1]) and not np.allclose(o1[:, -1], o2[:, -1])
+
+
+def test_hawk_layer_steps_equal_the_layer_forward():
+    # T decode steps from a zero state (h = 0, empty conv ring) reproduce the full-sequence
+    # layer at every position; the ring ends holding the last three inputs of the Conv1D
+    rng = np.random.default_rng(14)
+    B, T, D, R = 2, 7, 16, 24
+    P = _rng_params(rng, R)
+    x = rng.normal(0, 1, (B, T, D))
+    W = dict(norm1_scale=rng.uniform(0.5, 1.5, D), W_1=rng.normal(0, 0.25, (R, D)), W_2=rng.normal(0, 0.25, (R, D)),
+             W_o=rng.normal(0, 0.2, (D, R)), norm2_scale=rng.uniform(0.5, 1.5, D),
+             W_gate=rng.normal(0, 0.25, (3 * D, D)), W_up=rng.normal(0, 0.25, (3 * D, D)),
+             W_down=rng.normal(0, 0.15, (D, 3 * D)))
+    ref, h_ref = oracle.hawk_residual_layer(x, **W, **P)
+    ring, h = np.zeros((B, 3, R)), np.zeros((B, R))
+    for t in range(T):
+        out_t, h, ring = oracle.hawk_residual_layer_step(x[:, t], ring, t, h, **W, **P)
+        np.testing.assert_allclose(out_t, ref[:, t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h, h_ref, rtol=1e-12, atol=1e-14)
+    n1 = oracle.rms_norm(x, W["norm1_scale"])
+    v = n1 @ W["W_1"].T
+    np.testing.assert_allclose(oracle.ring_to_time_order(ring, T), v[:, -3:], rtol=1e-14)
