@@ -56,6 +56,8 @@ SIGNATURES = {
     "rglru_block_forward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P]),
     "rglru_layer_workspace_bytes": (_S, [_I, _I, _I, _I, _I, _I]),
     "rglru_layer_forward": (_I, [_PP, _LWP, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _S, _P]),
+    "rglru_layer_step_workspace_bytes": (_S, [_I, _I, _I, _I, _I]),
+    "rglru_layer_step": (_I, [_PP, _LWP, _P, _P, _P, _P, _I, _I, _I, _I, _L, ctypes.c_float, _I, _P, _S, _P]),
     "rglru_conv1d": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "rglru_gate_pitch": (_L, [_I]),
     "rglru_gate_proj": (_I, [_P, _P, _P, _P, _P, _P, _L, _I, _I, _P]),

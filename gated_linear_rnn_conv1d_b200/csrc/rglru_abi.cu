@@ -174,6 +174,29 @@ LayerLayout layer_layout(int B, int T, int D, int R, int H) {
   return L;
 }
 
+// Decode step of the layer: [step workspace (status word at 0, the decode conv's own word
+// at 4) | n [B][D] | v [B][R] | g, then GeLU(g) ⊙ y [B][R] | y [B][R] | o [B][D] | residual
+// stream [B][D] | gate (then p) [B][H] | up [B][H]], bf16.
+struct LayerStepLayout {
+  StepLayout step;
+  size_t off_n, off_v, off_g, off_y, off_o, off_res, off_gate, off_up, bytes;
+};
+LayerStepLayout layer_step_layout(int B, int D, int R, int H) {
+  LayerStepLayout L;
+  L.step = step_layout(B, R);
+  const size_t b = (size_t)B;
+  L.off_n = round256(L.step.bytes);
+  L.off_v = L.off_n + round256(b * D * 2);
+  L.off_g = L.off_v + round256(b * R * 2);
+  L.off_y = L.off_g + round256(b * R * 2);
+  L.off_o = L.off_y + round256(b * R * 2);
+  L.off_res = L.off_o + round256(b * D * 2);
+  L.off_gate = L.off_res + round256(b * D * 2);
+  L.off_up = L.off_gate + round256(b * H * 2);
+  L.bytes = L.off_up + round256(b * H * 2);
+  return L;
+}
+
 // The recurrent block (§循环块, Fig. 2(c)) after its status word is zeroed: the two
 // D → D_RNN linears, Conv1D, the coefficient GEMM, the gated scan (p = h ⊙ GeLU(g)) and
 // the D_RNN → D linear, queued on s with the block workspace layout L.
@@ -602,6 +625,71 @@ int rglru_layer_forward(const rglru_params* params, const rglru_layer_weights* w
   if (e == cudaSuccess) e = launch_gelu_mul(gate, up, gate, ntok * H, s);
   if (e == cudaSuccess) e = launch_gemm_bf16(gate, w->W_down, o, ntok, D, H, D, status, s);
   if (e == cudaSuccess) e = launch_add_rmsnorm(yres, o, out, nullptr, nullptr, ntok, D, eps, s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+size_t rglru_layer_step_workspace_bytes(int B, int D, int R, int H, int io_dtype) {
+  if (io_dtype != RGLRU_BF16 || !valid_R(R) || !valid_R(D) || !valid_R(H) || !valid_tokens(B, 1)) return 0;
+  return layer_step_layout(B, D, R, H).bytes;
+}
+
+int rglru_layer_step(const rglru_params* params, const rglru_layer_weights* w, const void* x_t, void* conv_state,
+                     float* h, void* out_t, int B, int D, int R, int H, int64_t step, float eps, int io_dtype,
+                     void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_R(D) || !valid_R(H) || !valid_tokens(B, 1) || step < 0) return RGLRU_ERR_SHAPE;
+  if (!(eps >= 0.0f) || eps > 1.0f) return RGLRU_ERR_SHAPE;  // also rejects NaN
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (w == nullptr || x_t == nullptr || conv_state == nullptr || h == nullptr || out_t == nullptr)
+    return RGLRU_ERR_NULL;
+  if (w->norm1_scale == nullptr || w->W_1 == nullptr || w->W_2 == nullptr || w->W_o == nullptr ||
+      w->norm2_scale == nullptr || w->W_gate == nullptr || w->W_up == nullptr || w->W_down == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(w->norm1_scale) || !aligned16(w->W_1) || !aligned16(w->W_2) || !aligned16(w->W_o) ||
+      !aligned16(w->norm2_scale) || !aligned16(w->W_gate) || !aligned16(w->W_up) || !aligned16(w->W_down) ||
+      !aligned16(x_t) || !aligned16(conv_state) || !aligned16(h) || !aligned16(out_t))
+    return RGLRU_ERR_ALIGN;
+  if (out_t == x_t) return RGLRU_ERR_SHAPE;  // the residual stream is read after out_t is written
+  const LayerStepLayout L = layer_step_layout(B, D, R, H);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  if ((st = check_device()) != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = bytes(workspace);
+  unsigned* status = reinterpret_cast<unsigned*>(ws);
+  unsigned* conv_word = reinterpret_cast<unsigned*>(ws + 4);  // the decode conv zeroes its word
+  float* cla = reinterpret_cast<float*>(ws + L.step.off_cla);
+  void* u_t = ws + L.step.off_u;
+  float* u_f32 = reinterpret_cast<float*>(ws + L.step.off_uf);
+  void* nrm = ws + L.off_n;
+  void* v = ws + L.off_v;
+  void* g = ws + L.off_g;
+  void* y = ws + L.off_y;
+  void* o = ws + L.off_o;
+  void* res = ws + L.off_res;
+  void* gate = ws + L.off_gate;
+  void* up = ws + L.off_up;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
+  // residual stream + RecurrentBlock(RMSNorm₁(x_t)) with one RG-LRU decode step
+  if (e == cudaSuccess) e = launch_add_rmsnorm(x_t, nullptr, nullptr, nrm, w->norm1_scale, B, D, eps, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_1, v, B, R, D, R, status, s);  // v_t = n W_1ᵀ
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_2, g, B, R, D, R, status, s);  // g_t = n W_2ᵀ
+  if (e == cudaSuccess)
+    e = launch_decode_conv(params->conv_w, params->conv_b, params->Lambda, v, conv_state, step, u_t, u_f32, cla,
+                           conv_word, B, R, s);
+  if (e == cudaSuccess)
+    e = launch_gemm_step_bf16(u_t, u_f32, params->W_a, params->b_a, params->W_x, params->b_x, cla, h, y, B, R,
+                              status, s);
+  if (e == cudaSuccess) e = launch_gelu_mul(g, y, g, (int64_t)B * R, s);  // h ⊙ GeLU(g_t)
+  if (e == cudaSuccess) e = launch_gemm_bf16(g, w->W_o, o, B, D, R, D, status, s);
+  if (e == cudaSuccess) e = launch_add_rmsnorm(x_t, o, res, nrm, w->norm2_scale, B, D, eps, s);
+  // + MLP(RMSNorm₂(·))
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_gate, gate, B, H, D, H, status, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_up, up, B, H, D, H, status, s);
+  if (e == cudaSuccess) e = launch_gelu_mul(gate, up, gate, (int64_t)B * H, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(gate, w->W_down, o, B, D, H, D, status, s);
+  if (e == cudaSuccess) e = launch_add_rmsnorm(res, o, out_t, nullptr, nullptr, B, D, eps, s);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 

@@ -304,6 +304,27 @@ def layer_forward(params: Params, weights: LayerWeights, x: torch.Tensor, h0: Op
     return out, h_T
 
 
+def layer_step_workspace_bytes(B: int, D: int, R: int, H: int) -> int:
+    return _abi.load().rglru_layer_step_workspace_bytes(B, D, R, H, _abi.RGLRU_BF16)
+
+
+def layer_step(params: Params, weights: LayerWeights, x_t: torch.Tensor, conv_state: torch.Tensor,
+               h: torch.Tensor, step_index: int, *, eps: float = 1e-6, workspace: Optional[torch.Tensor] = None,
+               out_t: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_layer_step: x_t [B][D] → out_t [B][D]; conv_state [B][3][R] and h [B][R] in place."""
+    lib = _abi.load()
+    B, D = x_t.shape
+    R, H = weights.W_1.shape[0], weights.H
+    io = _io(x_t)
+    out_t = torch.empty_like(x_t) if out_t is None else out_t
+    ws = _workspace(lib.rglru_layer_step_workspace_bytes(B, D, R, H, io), x_t.device, workspace)
+    st, wst = params.struct(), weights.struct()
+    _abi.check("rglru_layer_step", lib.rglru_layer_step(
+        ctypes.byref(st), ctypes.byref(wst), _p(x_t), _p(conv_state), _p(h), _p(out_t), B, D, R, H, int(step_index),
+        float(eps), io, _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+    return out_t
+
+
 def conv1d(params: Params, x: torch.Tensor, conv_state0: Optional[torch.Tensor] = None, *,
            u: Optional[torch.Tensor] = None, conv_state_T: Optional[torch.Tensor] = None,
            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:

@@ -172,6 +172,26 @@ RGLRU_API int rglru_layer_forward(const rglru_params* params, const rglru_layer_
                                   const float* h0, void* out, float* h_T, int B, int T, int D, int R, int H,
                                   float eps, int io_dtype, void* workspace, size_t workspace_bytes,
                                   rglru_stream_t stream);
+/* One decode step of the same layer on a carried state (the decode form of the
+ * recurrent block: "Griffin's Compromise…", §Hawk — generation reads and writes only the
+ * current token and a fixed-size state):
+ *   y   = x_t + ((RG-LRU step of Conv1D(v)) ⊙ GeLU(g)) W_oᵀ,  v = n W_1ᵀ, g = n W_2ᵀ, n = RMSNorm₁(x_t)
+ *   out_t = y + MLP(RMSNorm₂(y))
+ *   x_t, out_t  [B][D] bfloat16, distinct
+ *   conv_state  [B][3][R] bfloat16 ring of the last three inputs of the Conv1D (the v
+ *               branch), updated IN PLACE exactly as rglru_step updates its ring
+ *   h           [B][R] float32 RG-LRU state, updated IN PLACE
+ *   step        ≥ 0, the ring position (as rglru_step)
+ *   weights, eps, D, R, H as rglru_layer_forward
+ *   workspace   at least rglru_layer_step_workspace_bytes(B, D, R, H, io_dtype) bytes,
+ *               256-byte aligned
+ * io_dtype must be RGLRU_BF16. Errors as rglru_layer_forward, plus RGLRU_ERR_SHAPE for
+ * step < 0. */
+RGLRU_API size_t rglru_layer_step_workspace_bytes(int B, int D, int R, int H, int io_dtype);
+RGLRU_API int rglru_layer_step(const rglru_params* params, const rglru_layer_weights* weights, const void* x_t,
+                               void* conv_state, float* h, void* out_t, int B, int D, int R, int H, int64_t step,
+                               float eps, int io_dtype, void* workspace, size_t workspace_bytes,
+                               rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Backward of rglru_forward for bf16 IO: the gradients of a scalar loss ℓ with respect to

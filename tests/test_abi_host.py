@@ -189,3 +189,35 @@ def test_layer_rejects_bad_arguments_before_any_launch():
     assert call(ws=None) == -5
     assert call(wsb=wb - 1) == -5
     assert call(ws=_fake(0x200010)) == -3
+
+
+def test_layer_step_rejects_bad_arguments_before_any_launch():
+    lib = _abi.load()
+    p = _params()
+    ok_ptr = _fake()
+    wb = lib.rglru_layer_step_workspace_bytes(4, 64, 64, 192, 1)
+    assert wb > lib.rglru_step_workspace_bytes(4, 64, 1)
+    assert lib.rglru_layer_step_workspace_bytes(4, 64, 64, 192, 0) == 0
+    assert lib.rglru_layer_step_workspace_bytes(0, 64, 64, 192, 1) == 0
+    f = 0x100000
+    weights = _abi.RGLRULayerWeights(f, f, f, f, f, f, f, f)
+    ws = _fake(0x200000)
+
+    def call(**kw):
+        return lib.rglru_layer_step(
+            ctypes.byref(p), kw.get("w", ctypes.byref(weights)), kw.get("x", ok_ptr), kw.get("ring", ok_ptr),
+            kw.get("h", ok_ptr), kw.get("out", _fake(0x300000)), 4, kw.get("D", 64), 64, kw.get("H", 192),
+            kw.get("step", 0), kw.get("eps", 1e-6), kw.get("io", 1), kw.get("ws", ws), kw.get("wsb", wb), None)
+
+    assert call(io=0) == -4
+    assert call(D=12) == -2
+    assert call(H=0) == -2
+    assert call(step=-1) == -2
+    assert call(eps=2.0) == -2
+    assert call(out=ok_ptr) == -2
+    assert call(ring=None) == -1
+    assert call(h=None) == -1
+    assert call(w=None) == -1
+    assert call(h=_fake(0x100008)) == -3
+    assert call(ws=None) == -5
+    assert call(wsb=wb - 1) == -5
