@@ -221,3 +221,21 @@ def test_layer_step_rejects_bad_arguments_before_any_launch():
     assert call(h=_fake(0x100008)) == -3
     assert call(ws=None) == -5
     assert call(wsb=wb - 1) == -5
+
+
+def test_layer_weights_marshal_every_field_in_header_order():
+    import torch
+    from gated_linear_rnn_conv1d_b200 import inputs, rglru
+    w = inputs.make_layer(1, 4, 16, 24, 3, torch.bfloat16, seed=1)
+    lw = rglru.LayerWeights.from_host(w, "cpu")
+    assert lw.H == 48 and lw.W_down.shape == (16, 48) and lw.norm1_scale.dtype == torch.float32
+    st = lw.struct()
+    names = [f for f, _ in _abi.RGLRULayerWeights._fields_]
+    assert names == list(rglru.LayerWeights.FIELDS)
+    for f in names:
+        assert getattr(st, f) == getattr(lw, f).data_ptr()
+    assert torch.equal(lw.W_gate, w.extra["W_gate"]) and torch.equal(lw.W_1, w.W_1)
+    # the header's struct lists the same fields in the same order
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "rglru.h"), encoding="utf-8").read()
+    body = hdr[hdr.index("typedef struct rglru_layer_weights"):hdr.index("} rglru_layer_weights;")]
+    assert re.findall(r"\*\s*(\w+);", body) == names

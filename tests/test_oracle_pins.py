@@ -563,3 +563,30 @@ def test_hawk_layer_steps_equal_the_layer_forward():
     n1 = oracle.rms_norm(x, W["norm1_scale"])
     v = n1 @ W["W_1"].T
     np.testing.assert_allclose(oracle.ring_to_time_order(ring, T), v[:, -3:], rtol=1e-14)
+
+
+def test_hawk_layer_example_rejects_planted_wiring_mistakes():
+    # Each plausible slip in wiring the residual layer, built from the oracle's own parts,
+    # misses the hand-worked value by far more than rounding.
+    ex = _parse_golden(GOLDEN)["hawk_layer"]
+    m = lambda k: ex[k].reshape(1, 1)  # noqa: E731
+    x = ex["x"].reshape(1, 1, 1)
+    P = dict(conv_w=ex["conv_w"].reshape(4, 1), conv_b=ex["conv_b"], W_a=np.zeros((1, 1)), b_a=np.zeros(1),
+             W_x=np.zeros((1, 1)), b_x=np.zeros(1), Lambda=ex["Lambda"])
+    norm = lambda v, g: oracle.rms_norm(v, g, eps=0.0)  # noqa: E731
+    block = lambda n: oracle.recurrent_block(n, m("W_1"), m("W_2"), m("W_o"), **P)[0]  # noqa: E731
+    mlp = lambda n: oracle.gated_mlp(n, m("W_gate"), m("W_up"), m("W_down"))  # noqa: E731
+    g1, g2 = ex["norm1_scale"], ex["norm2_scale"]
+    right = x + block(norm(x, g1))
+    right = right + mlp(norm(right, g2))
+    np.testing.assert_allclose(right.ravel(), ex["out"], rtol=1e-14)
+    planted = {
+        "skip from the norm output": (lambda n1: (lambda y: y + mlp(norm(y, g2)))(n1 + block(n1)))(norm(x, g1)),
+        "second norm applied to x": (lambda y: y + mlp(norm(x, g2)))(x + block(norm(x, g1))),
+        "gains dropped": (lambda y: y + mlp(norm(y, 1.0)))(x + block(norm(x, 1.0))),
+        "GeLU on the up branch": (lambda y: y + oracle.gated_mlp(norm(y, g2), m("W_up"), m("W_gate"), m("W_down")))(
+            x + block(norm(x, g1))),
+        "no second residual": mlp(norm(x + block(norm(x, g1)), g2)),
+    }
+    for name, out in planted.items():
+        assert abs(out.ravel()[0] - ex["out"][0]) > 0.1, name
