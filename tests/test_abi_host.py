@@ -239,3 +239,29 @@ def test_layer_weights_marshal_every_field_in_header_order():
     hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "rglru.h"), encoding="utf-8").read()
     body = hdr[hdr.index("typedef struct rglru_layer_weights"):hdr.index("} rglru_layer_weights;")]
     assert re.findall(r"\*\s*(\w+);", body) == names
+
+
+def test_layer_workspace_sizes_follow_the_documented_layouts():
+    lib = _abi.load()
+    r256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    for B, T, D, R, H in [(1, 8, 64, 64, 192), (2, 150, 136, 264, 408), (4, 4096, 4096, 5632, 12288)]:
+        n = B * T
+        blk = lib.rglru_block_workspace_bytes(B, T, D, R, 1)
+        assert lib.rglru_layer_workspace_bytes(B, T, D, R, H, 1) == r256(blk) + 3 * r256(n * D * 2) + 2 * r256(n * H * 2)
+        stp = lib.rglru_step_workspace_bytes(B, R, 1)
+        assert lib.rglru_layer_step_workspace_bytes(B, D, R, H, 1) == (
+            r256(stp) + 3 * r256(B * D * 2) + 3 * r256(B * R * 2) + 2 * r256(B * H * 2))
+
+
+def test_layer_binding_takes_cuda_tensors_only():
+    import torch
+    from gated_linear_rnn_conv1d_b200 import inputs, rglru
+    w = inputs.make_layer(1, 4, 16, 24, 3, torch.bfloat16, seed=1)
+    p = rglru.Params.from_host(w.params, "cpu")
+    lw = rglru.LayerWeights.from_host(w, "cpu")
+    ws = torch.empty(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        rglru.layer_forward(p, lw, w.x, workspace=ws, out=torch.empty_like(w.x), h_T=torch.empty(1, 24))
+    with pytest.raises(ValueError):
+        rglru.layer_step(p, lw, w.x[:, 0].contiguous(), torch.zeros(1, 3, 24, dtype=torch.bfloat16),
+                         torch.zeros(1, 24), 0, workspace=ws, out_t=torch.empty(1, 16, dtype=torch.bfloat16))
