@@ -108,7 +108,7 @@ cudaError_t launch_gelu_mul(const void* gate, const void* up, void* p, int64_t n
   if (n < 8 || n % 8 != 0 || gate == nullptr || up == nullptr || p == nullptr) return cudaErrorInvalidValue;
   const int64_t n8 = n / 8;
   const int64_t want = (n8 + kEwThreads - 1) / kEwThreads;
-  const int grid = (int)std::min<int64_t>(want, (int64_t)num_sms() * 8);
+  const int grid = (int)std::min<int64_t>(want, (int64_t)std::max(1, num_sms()) * 8);
   gelu_mul_kernel<<<grid, kEwThreads, 0, s>>>(static_cast<const uint4*>(gate), static_cast<const uint4*>(up),
                                               static_cast<uint4*>(p), n8);
   return cudaGetLastError();
