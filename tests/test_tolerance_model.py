@@ -78,3 +78,34 @@ def test_layer_storage_rounding_fits_the_layer_tolerance_and_not_the_rglru_one()
     err = oracle.max_rel_error(got, ref)
     assert TOL[torch.bfloat16] < err <= TOL_LAYER, err
     print(f"layer parity case: storage rounding alone gives {err:.17g}")
+
+
+def test_forward_storage_rounding_fits_the_bf16_tolerance():
+    # the RG-LRU forward's bf16 parity case (B=2, T=200, D_RNN=264, non-zero biases, h0 and
+    # conv history, as the GPU test draws them): u in bf16 (the gate GEMM's operand, also
+    # the u in b_t), d and b in fp16, y in bf16
+    B, T, R = 2, 200, 264
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=0)
+    g = torch.Generator("cpu").manual_seed(77)
+    P = w.params
+    P.b_a = torch.randn(R, generator=g) * 0.5
+    P.b_x = torch.randn(R, generator=g) * 0.5
+    h0 = torch.randn(B, R, generator=g)
+    state0 = torch.randn(B, 3, R, generator=g).to(torch.bfloat16)
+    for hist, h_init in ((None, None), (state0, h0)):
+        u, _ = oracle.conv1d_causal(w.x, _f(P.conv_w), _f(P.conv_b), None if hist is None else _f(hist))
+        u = _bf16(u)
+        r = oracle.sigmoid(u @ _f(P.W_a).T + _f(P.b_a))
+        i = oracle.sigmoid(u @ _f(P.W_x).T + _f(P.b_x))
+        a_t = oracle.decay_direct(r, _f(P.Lambda))
+        d, b = _fp16(1.0 - a_t), _fp16(np.sqrt(1.0 - a_t * a_t) * i * u)
+        h = np.zeros((B, R)) if h_init is None else _f(h_init)
+        ys = np.empty_like(u)
+        for t in range(T):
+            h = (1.0 - d[:, t]) * h + b[:, t]
+            ys[:, t] = h
+        y_ref, _, _ = oracle.rglru_forward(w.x, P.conv_w, P.conv_b, P.W_a, P.b_a, P.W_x, P.b_x, P.Lambda,
+                                           h0=h_init, conv_state0=hist)
+        err = oracle.max_rel_error(_bf16(ys), y_ref)
+        print(f"forward parity case, history={hist is not None}: storage rounding alone gives {err:.3e}")
+        assert err <= TOL[torch.bfloat16], err
