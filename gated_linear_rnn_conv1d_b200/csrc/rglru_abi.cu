@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstring>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/rglru.h"
 #include "kernels.cuh"
@@ -14,6 +15,15 @@ using namespace rglru;
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+
+// NVTX range around one C-ABI call (a no-op unless a profiler attaches NVTX handling), so a
+// timeline or an `ncu --nvtx` filter can group the kernels one call launches.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 constexpr int kMaxDevices = 64;
 
@@ -320,6 +330,7 @@ size_t rglru_gate_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
 int rglru_gate_scan(const rglru_params* params, const void* x, const void* u, const void* conv_state0,
                     const float* h0, void* y, float* h_T, int B, int T, int R, int io_dtype, void* workspace,
                     size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_gate_scan");
   if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, T) || T % 128 != 0) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
@@ -351,6 +362,7 @@ size_t rglru_block_workspace_bytes(int B, int T, int D, int R, int io_dtype) {
 
 int rglru_conv1d(const float* conv_w, const float* conv_b, const void* x, const void* conv_state0, void* u,
                  void* conv_state_T, int B, int T, int R, int io_dtype, rglru_stream_t stream) {
+  const Range range("rglru_conv1d");
   if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   if (conv_w == nullptr || conv_b == nullptr || x == nullptr || u == nullptr) return RGLRU_ERR_NULL;
@@ -368,6 +380,7 @@ int rglru_conv1d(const float* conv_w, const float* conv_b, const void* x, const 
 
 int rglru_gate_proj(const void* u, const void* W_a, const float* b_a, const void* W_x, const float* b_x, void* z,
                     int64_t N_tok, int R, int io_dtype, rglru_stream_t stream) {
+  const Range range("rglru_gate_proj");
   if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || N_tok < 1 || N_tok > (int64_t)INT32_MAX) return RGLRU_ERR_SHAPE;
   if (u == nullptr || W_a == nullptr || b_a == nullptr || W_x == nullptr || b_x == nullptr || z == nullptr)
@@ -392,6 +405,7 @@ int rglru_gate_proj(const void* u, const void* W_a, const float* b_a, const void
 int rglru_scan(const rglru_params* params, const void* x, const void* z, const void* conv_state0, const float* h0,
                const void* gate_g, void* y, float* h_T, int B, int T, int R, int io_dtype, void* workspace,
                size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_scan");
   if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
@@ -411,6 +425,7 @@ int rglru_scan(const rglru_params* params, const void* x, const void* z, const v
 
 int rglru_gate_coeffs(const rglru_params* params, const void* u, void* g, int64_t N_tok, int R,
                       rglru_stream_t stream) {
+  const Range range("rglru_gate_coeffs");
   if (!valid_R(R) || N_tok < 1 || N_tok > (int64_t)INT32_MAX) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
   if (st != RGLRU_OK) return st;
@@ -426,6 +441,7 @@ int rglru_gate_coeffs(const rglru_params* params, const void* u, void* g, int64_
 
 int rglru_scan_coeffs(const void* g, const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R,
                       void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_scan_coeffs");
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   if (g == nullptr || y == nullptr) return RGLRU_ERR_NULL;
   if (!aligned16(g) || !aligned16(y) || !aligned16(h0) || !aligned16(gate_g) || !aligned16(h_T))
@@ -443,6 +459,7 @@ int rglru_scan_coeffs(const void* g, const float* h0, const void* gate_g, void* 
 int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
                   float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype, void* workspace,
                   size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_forward");
   if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
@@ -482,6 +499,7 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
 
 int rglru_step(const rglru_params* params, const void* x_t, void* conv_state, float* h, void* y_t, int B, int R,
                int64_t step, int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_step");
   if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, 1) || step < 0) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
@@ -506,6 +524,7 @@ int rglru_step(const rglru_params* params, const void* x_t, void* conv_state, fl
 }
 
 int rglru_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, rglru_stream_t stream) {
+  const Range range("rglru_gemm_bf16");
   if (M < 1 || M > (int64_t)INT32_MAX * 128 || !valid_R(N) || !valid_R(K)) return RGLRU_ERR_SHAPE;
   if (A == nullptr || Bm == nullptr || C == nullptr) return RGLRU_ERR_NULL;
   if (!aligned16(A) || !aligned16(Bm) || !aligned16(C)) return RGLRU_ERR_ALIGN;
@@ -525,6 +544,7 @@ size_t rglru_backward_workspace_bytes(int B, int T, int R) {
 int rglru_backward(const rglru_params* params, const void* x, const void* y, const void* dy, const float* h0,
                    const float* dh_T, const void* conv_state0, const rglru_grads* grads, int B, int T, int R,
                    void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_backward");
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   // the transposed token axis of the weight-gradient GEMMs (and its 32-row transpose
   // tiles) must stay within int32 and the grid's y limit
@@ -561,6 +581,7 @@ int rglru_backward(const rglru_params* params, const void* x, const void* y, con
 int rglru_block_forward(const rglru_params* params, const void* W_1, const void* W_2, const void* W_o, const void* x,
                         const float* h0, void* out, float* h_T, int B, int T, int D, int R, int io_dtype,
                         void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_block_forward");
   if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_R(D) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
@@ -587,6 +608,7 @@ size_t rglru_layer_workspace_bytes(int B, int T, int D, int R, int H, int io_dty
 int rglru_layer_forward(const rglru_params* params, const rglru_layer_weights* w, const void* x, const float* h0,
                         void* out, float* h_T, int B, int T, int D, int R, int H, float eps, int io_dtype,
                         void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_layer_forward");
   if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_R(D) || !valid_R(H) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   if (!(eps >= 0.0f) || eps > 1.0f) return RGLRU_ERR_SHAPE;  // also rejects NaN
@@ -636,6 +658,7 @@ size_t rglru_layer_step_workspace_bytes(int B, int D, int R, int H, int io_dtype
 int rglru_layer_step(const rglru_params* params, const rglru_layer_weights* w, const void* x_t, void* conv_state,
                      float* h, void* out_t, int B, int D, int R, int H, int64_t step, float eps, int io_dtype,
                      void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_layer_step");
   if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_R(D) || !valid_R(H) || !valid_tokens(B, 1) || step < 0) return RGLRU_ERR_SHAPE;
   if (!(eps >= 0.0f) || eps > 1.0f) return RGLRU_ERR_SHAPE;  // also rejects NaN
