@@ -13,6 +13,12 @@
  *     a_t = a^(c r_t),  a = σ(Λ),  c = 8, evaluated in log space    (3)
  *     h_t = a_t ⊙ h_{t-1} + √(1 − a_t²) ⊙ (i_t ⊙ u_t),  y_t = h_t   (4)
  *
+ * Around that core the library also offers the recurrent block, its backward, and one
+ * Hawk residual layer (RMSNorm, the recurrent block, RMSNorm, gated MLP, residual adds:
+ * the same page's §残块 and §MLP块, Fig. 2(a)–(b)), each as a prefill call, with decode
+ * steps for the core and for the layer. Every launching call is bracketed by an NVTX
+ * range named after it.
+ *
  * Conventions shared by every entry point
  *   - R is D_RNN, the channel count. R must be a multiple of 8 (16-byte rows).
  *   - Row-major layouts; "[B][T][R]" means R is contiguous.
