@@ -606,7 +606,9 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         // "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元, Eq. (3)–(4):
         // columns [0, 128) are z_a and [128, 256) z_x of channels n_blk·128 + j. Each row's
         // pairs become the recurrence coefficients d = 1 − a_t and b_t = √(1−a_t²)·i_t·u_t
-        // (fp16, in the same packed places): the recurrence is then h_t = (1 − d)·h_{t−1} + b_t.
+        // (d in fp16, b_t in bf16, in the same packed places): the recurrence is then
+        // h_t = (1 − d)·h_{t−1} + b_t. d ∈ [0, 1] keeps fp16's 11 significant bits; b_t scales
+        // with u_t, so it takes bf16's float32 exponent range (any |u_t| a bf16 u can hold).
         float* sPar = reinterpret_cast<float*>(smem + S * k2StageBytes) + acc * 3 * 128;
         const int chalf = (warp - 2) / 4;  // which 64 of the 128 channels this warp forms
         if (chalf == 0) {
@@ -617,7 +619,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           sPar[256 + row_in_tile] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
         }
         named_bar_sync(1, 32 * epi_warps_of<EPI>());  // this CTA's epilogue warps
-        __half* out = reinterpret_cast<__half*>(ep.C) + row * ep.ldc + (int64_t)n_blk * BN;
+        uint16_t* out = reinterpret_cast<uint16_t*>(ep.C) + row * ep.ldc + (int64_t)n_blk * BN;  // 16-bit words
         // 4 chunks of 16 channels; the next chunk's TMEM load is in flight while one is formed
         uint32_t ra[2][16], rx[2][16];
         tmem_ld_x16(t_row + chalf * 64, ra[0]);
@@ -645,7 +647,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
             float2 d, m;
             gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), u2, d, m);
             const __half2 dd = __floats2half2_rn(d.x, d.y);
-            const __half2 mm = __floats2half2_rn(m.x, m.y);
+            const __nv_bfloat162 mm = __floats2bfloat162_rn(m.x, m.y);
             dh[j / 2] = *reinterpret_cast<const uint32_t*>(&dd);
             mh[j / 2] = *reinterpret_cast<const uint32_t*>(&mm);
           }

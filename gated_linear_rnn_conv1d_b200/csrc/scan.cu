@@ -1,8 +1,8 @@
 // RG-LRU chunked scan, in two forms:
 //  * from pre-activations: Conv1D recompute + σ gates + log-space decay + chunked diagonal
 //    recurrence; one HBM read of x and of the packed gate pre-activations z, one write of y;
-//  * from recurrence coefficients (bf16 IO): d = 1 − a_t and b_t = √(1−a_t²)·i_t·u_t, both
-//    fp16, formed by the gate GEMM's epilogue; one HBM read of (d, b), one write of y.
+//  * from recurrence coefficients (bf16 IO): d = 1 − a_t (fp16) and b_t = √(1−a_t²)·i_t·u_t
+//    (bf16), formed by the gate GEMM's epilogue; one HBM read of (d, b), one write of y.
 //
 // Math: "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型",
 // §实门线性循环单元 (RG-LRU), Eq. (1)–(4); §循环块 for the Conv1D and the GeLU branch.
@@ -51,8 +51,10 @@
 // another.
 // The replay values of the pre-activation bf16 path are stored as bf16 (1 − a_t, b_t): their
 // rounding only touches y inside one 4-step sub-chunk, while the published states and h_T
-// come from the float32 maps. The coefficients are fp16 (11 significant bits); everything
-// composed from them (maps, states, h_T) is float32.
+// come from the float32 maps. Of the coefficients, d ∈ [0, 1] is fp16 (11 significant bits:
+// its relative error multiplies into every carried state) and b_t is bf16 (it scales with
+// u_t, so it needs float32's exponent range); everything composed from them (maps, states,
+// h_T) is float32.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
@@ -105,7 +107,7 @@ template <bool kCoef> constexpr int threads_of() {
 // phase 1 is done, look-back warps wait
 constexpr int kBarMaps = 1;
 
-// kCoef: the stage holds only the two coefficient blocks (d = 1 − a_t, b_t; fp16), which
+// kCoef: the stage holds only the two coefficient blocks (d = 1 − a_t fp16, b_t bf16), which
 // need neither x nor parameters, so the ring is deeper.
 template <typename T, bool kGate, bool kCoef = false> struct SmemLayout {
   static constexpr int CW = kGroups * SV<T>::V;
@@ -440,7 +442,7 @@ __device__ __forceinline__ void phase1_body(uint8_t* stage, float* mA, float* mB
 }
 
 // The coefficients of one sub-chunk as one compute thread holds them: kLC steps × 4
-// channels of d and of b, as packed fp16 pairs (bf16 IO only).
+// channels of d (packed fp16 pairs) and of b (packed bf16 pairs); bf16 IO only.
 struct CoefRegs {
   uint32_t d[kLC][2], b[kLC][2];
 };
@@ -466,6 +468,10 @@ __device__ __forceinline__ void coef_load(const uint8_t* stage, int g, int s, Co
 __device__ __forceinline__ float2 h2f(uint32_t w) {
   return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
+// a packed bf16 pair as two floats (the low half is the first element)
+__device__ __forceinline__ float2 bf2f(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
 
 // Phase 1 of the coefficient scan from registers: fold the sub-chunk's 4 steps,
 // (A, B) ← (a·A, a·B + b) with a = 1 − d, into its map. Steps past T are identity steps.
@@ -485,7 +491,7 @@ __device__ __forceinline__ void coef_fold(const CoefRegs& r, float* mA, float* m
       for (int p = 0; p < 2; ++p) {
         const float2 d2 = h2f(r.d[l][p]);
         const float2 a2 = make_float2(1.0f - d2.x, 1.0f - d2.y);
-        B[p] = __ffma2_rn(a2, B[p], h2f(r.b[l][p]));
+        B[p] = __ffma2_rn(a2, B[p], bf2f(r.b[l][p]));
         A[p] = __fmul2_rn(a2, A[p]);
       }
     }
@@ -539,7 +545,7 @@ __device__ __forceinline__ void coef_replay(const uint8_t* stage, const float* m
       for (int p = 0; p < 2; ++p) {
         const float2 d2 = h2f(d[l][p]);
         const float2 a2 = make_float2(1.0f - d2.x, 1.0f - d2.y);
-        h[p] = __ffma2_rn(a2, h[p], h2f(b[l][p]));
+        h[p] = __ffma2_rn(a2, h[p], bf2f(b[l][p]));
         o[2 * p] = h[p].x;
         o[2 * p + 1] = h[p].y;
       }
@@ -996,7 +1002,7 @@ cudaError_t launch_scan(const ScanArgs& a_in, bool bf16, cudaStream_t s, bool co
     cuuint64_t dims[2] = {(cuuint64_t)a.pitch, (cuuint64_t)a.B * a.T};
     cuuint64_t strides[1] = {(cuuint64_t)a.pitch * es};
     cuuint32_t box[2] = {(cuuint32_t)cw, (cuuint32_t)kScanTC};
-    const CUtensorMapDataType zdt = coef ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : dt;
+    const CUtensorMapDataType zdt = coef ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : dt;  // 16-bit coefficient words
     if (!encode(&maps.z, zdt, 2, a.z, dims, strides, box)) return cudaErrorInvalidValue;
   }
   const bool gate = a.g != nullptr;

@@ -70,14 +70,16 @@ def test_gate_projection_matches_oracle(dtype, N, R):
 
 @pytest.mark.parametrize("N,R", [(300, 136), (1024, 512), (129, 264)])
 def test_gate_coeffs_match_oracle(N, R):
-    """rglru_gate_coeffs: d = 1 − a_t and b_t = √(1−a_t²)·i_t·u_t (fp16) in the packed places."""
+    """rglru_gate_coeffs: d = 1 − a_t (fp16) and b_t = √(1−a_t²)·i_t·u_t (bf16) in the packed
+    places."""
     w = _wl(1, N, R, torch.bfloat16)
     p = rglru.Params.from_host(w.params)
     g = torch.Generator("cpu").manual_seed(5)
     u = torch.randn(N, R, generator=g).to(torch.bfloat16)
     co = rglru.gate_coeffs(p, u.to(DEV))
-    assert co.dtype == torch.float16
-    d, b = unpack_gates(co, R)
+    assert co.dtype == torch.int16
+    d, _ = unpack_gates(co.view(torch.float16), R)
+    _, b = unpack_gates(co.view(torch.bfloat16), R)
     za, zx = oracle.gate_preactivations(u, w.params.W_a, w.params.b_a, w.params.W_x, w.params.b_x)
     a_t = oracle.decay_log_space(oracle.sigmoid(za), w.params.Lambda)
     d_o = 1.0 - a_t
@@ -168,6 +170,33 @@ def test_forward_matches_oracle(dtype, B, T, R, with_state):
     assert rel(y, y_ref) <= TOL[dtype]
     assert rel(h_T, h_ref) <= TOL[dtype]
     assert np.array_equal(f64(stT), st_ref)
+
+
+@pytest.mark.parametrize("x_scale", [1e5, 1e30, 1e-30])
+def test_bf16_forward_keeps_the_input_scale(x_scale):
+    """The bf16 forward holds every u-scaled value in a format with float32's exponent range
+    (u and y bf16, b_t = √(1−a_t²)·i_t·u_t bf16): inputs far outside fp16's range — |u| around
+    1e5 or 1e30, or 1e-30 with the conv bias 0 so that u keeps that scale — give finite outputs
+    within the bf16 bound of the oracle. The gate weights are scaled by 1/x_scale so that the
+    pre-activations stay O(1) (otherwise every gate saturates and the bf16 rounding of u
+    decides r and i, which no bf16 operand avoids)."""
+    B, T, R = 2, 200, 264
+    w = _wl(B, T, R, torch.bfloat16, seed=11)
+    w.x = (w.x.double() * x_scale).to(torch.bfloat16)
+    w.params.conv_b = torch.zeros(R)
+    w.params.W_a = (w.params.W_a.double() / x_scale).to(torch.bfloat16)
+    w.params.W_x = (w.params.W_x.double() / x_scale).to(torch.bfloat16)
+    h0 = (w.h0.double() * x_scale).float()
+    st0 = (w.extra["state0"].double() * x_scale).to(torch.bfloat16)
+    assert torch.isfinite(w.x.float()).all() and torch.isfinite(h0).all()
+    p = rglru.Params.from_host(w.params)
+    y, h_T, _ = rglru.forward(p, w.x.to(DEV), h0.to(DEV), st0.to(DEV))
+    assert rglru.workspace_status(None) == 0
+    y_ref, h_ref, _ = oracle.rglru_forward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a, w.params.b_a,
+                                           w.params.W_x, w.params.b_x, w.params.Lambda, h0=h0, conv_state0=st0)
+    assert torch.isfinite(y.float()).all() and torch.isfinite(h_T).all()
+    assert rel(y, y_ref) <= TOL[torch.bfloat16]
+    assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -320,6 +349,32 @@ def test_forward_host_equals_forward():
         assert plan.status() == 0
         assert torch.equal(y_host, y_ref.cpu())
         assert torch.equal(h_host, h_ref.cpu())
+
+
+def test_forward_host_in_time_chunks():
+    """A single long sequence (B = 1) goes through forward_host in time chunks, each started
+    from the state the previous chunk returned: the result equals those chained
+    rglru_forward calls bit for bit, and the whole-sequence forward within the split test's
+    bound."""
+    B, T, R, G = 1, 640, 264, 5
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=8)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    plan = rglru.HostForwardPlan(B, T, R, torch.bfloat16, groups=G, slots=3)
+    assert plan.split == "time"
+    x_host = w.x.pin_memory()
+    y_host = torch.empty(B, T, R, dtype=torch.bfloat16).pin_memory()
+    h_host = torch.empty(B, R, dtype=torch.float32).pin_memory()
+    rglru.forward_host(p, x_host, y_host, h_host, plan)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    h, st, ys = None, None, []
+    for g in range(G):
+        yg, h, st = rglru.forward(p, x[:, g * 128:(g + 1) * 128].contiguous(), h, st)
+        ys.append(yg)
+    assert torch.equal(y_host, torch.cat(ys, 1).cpu()) and torch.equal(h_host, h.cpu())
+    y, h_T, _ = rglru.forward(p, x)
+    assert rel(y_host, y) <= 8e-3 and rel(h_host, h_T) <= 8e-3
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])

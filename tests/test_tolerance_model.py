@@ -4,10 +4,10 @@ The CUDA path stores its intermediates in bf16 (the forward: the Conv1D output u
 the block in addition: v = x W_1ᵀ, g = x W_2ᵀ, h ⊙ GeLU(g), the block output; the layer in
 addition: both RMSNorm outputs, the residual stream, the MLP's gate, up, GeLU product and
 down projection, the output; the backward: the recomputed pre-activations and ∂z, the
-operands of the weight-gradient GEMMs) and the recurrence coefficients d = 1 − a_t,
-b_t = √(1 − a_t²)·i_t·u_t in fp16, with float32 arithmetic in between. The model below is the float64 oracle's arithmetic with exactly
-those roundings (round to nearest even, torch's casts) and nothing else; the CUDA path is
-not involved. Its distance from the unrounded oracle is the error that storage rounding
+operands of the weight-gradient GEMMs) and the recurrence coefficients d = 1 − a_t (fp16)
+and b_t = √(1 − a_t²)·i_t·u_t (bf16), with float32 arithmetic in between. The model
+(rounding_model.py) is the float64 oracle's arithmetic with exactly those roundings (round
+to nearest even, torch's casts) and nothing else; the CUDA path is not involved. Its distance from the unrounded oracle is the error that storage rounding
 alone forces on any implementation with these formats, on the seeded parity cases of the
 GPU tests. The tolerances must cover it; the layer's case and the backward's weight
 gradients show why those two cannot be held to the RG-LRU's 2e-2.
@@ -16,75 +16,39 @@ import numpy as np
 import torch
 
 import oracle
+import rounding_model as rm
 from gated_linear_rnn_conv1d_b200 import inputs
 
 from _util import TOL, TOL_LAYER
 
 
-def _f(t):
-    return t.double().numpy() if torch.is_tensor(t) else np.asarray(t, dtype=np.float64)
-
-
-def _bf16(a):
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.bfloat16).double().numpy()
-
-
-def _fp16(a):
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.float16).double().numpy()
-
-
-def _rms_norm(v, gain, eps=oracle.RMS_EPS):
-    return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps) * _f(gain)
-
-
-def _block_rounded(x, W_1, W_2, W_o, P):
-    """Recurrent block with the storage roundings of the bf16 path."""
-    v, g = _bf16(x @ _f(W_1).T), _bf16(x @ _f(W_2).T)
-    u, _ = oracle.conv1d_causal(v, _f(P.conv_w), _f(P.conv_b))
-    u = _bf16(u)
-    r = oracle.sigmoid(u @ _f(P.W_a).T + _f(P.b_a))
-    i = oracle.sigmoid(u @ _f(P.W_x).T + _f(P.b_x))
-    a_t = oracle.decay_direct(r, _f(P.Lambda))
-    d, b = _fp16(1.0 - a_t), _fp16(np.sqrt(1.0 - a_t * a_t) * i * u)
-    h, hs = np.zeros((u.shape[0], u.shape[2])), np.empty_like(u)
-    for t in range(u.shape[1]):
-        h = (1.0 - d[:, t]) * h + b[:, t]
-        hs[:, t] = h
-    return _bf16(_bf16(hs * oracle.gelu(g)) @ _f(W_o).T)
-
-
 def test_block_storage_rounding_fits_the_bf16_tolerance():
     w = inputs.make_block(2, 150, 136, 264, torch.bfloat16, seed=6)  # the block's GPU parity case
     P = w.params
-    got = _block_rounded(_f(w.x), w.W_1, w.W_2, w.W_o, P)
+    got, _ = rm.block(w.x, w.W_1, w.W_2, w.W_o, P)
     ref, _ = oracle.recurrent_block(w.x, w.W_1, w.W_2, w.W_o, P.conv_w, P.conv_b, P.W_a, P.b_a, P.W_x, P.b_x,
                                     P.Lambda)
     err = oracle.max_rel_error(got, ref)
+    print(f"block parity case: storage rounding alone gives {err:.3e}")
     assert 5e-3 < err <= TOL[torch.bfloat16], err
 
 
 def test_layer_storage_rounding_fits_the_layer_tolerance_and_not_the_rglru_one():
     w = inputs.make_layer(2, 150, 136, 264, 3, torch.bfloat16, seed=7)  # the layer's GPU parity case
     P, e = w.params, w.extra
-    x = _f(w.x)
-    o1 = _block_rounded(_bf16(_rms_norm(x, e["norm1_scale"])), w.W_1, w.W_2, w.W_o, P)
-    y = _bf16(x + o1)
-    n2 = _bf16(_rms_norm(y, e["norm2_scale"]))
-    gate, up = _bf16(n2 @ _f(e["W_gate"]).T), _bf16(n2 @ _f(e["W_up"]).T)
-    o2 = _bf16(_bf16(oracle.gelu(gate) * up) @ _f(e["W_down"]).T)
-    got = _bf16(y + o2)
+    got, _ = rm.layer_from_workload(w)
     ref, _ = oracle.hawk_residual_layer(w.x, e["norm1_scale"], w.W_1, w.W_2, w.W_o, e["norm2_scale"], e["W_gate"],
                                         e["W_up"], e["W_down"], P.conv_w, P.conv_b, P.W_a, P.b_a, P.W_x, P.b_x,
                                         P.Lambda)
     err = oracle.max_rel_error(got, ref)
-    assert TOL[torch.bfloat16] < err <= TOL_LAYER, err
     print(f"layer parity case: storage rounding alone gives {err:.17g}")
+    assert TOL[torch.bfloat16] < err <= TOL_LAYER, err
 
 
 def test_forward_storage_rounding_fits_the_bf16_tolerance():
     # the RG-LRU forward's bf16 parity case (B=2, T=200, D_RNN=264, non-zero biases, h0 and
     # conv history, as the GPU test draws them): u in bf16 (the gate GEMM's operand, also
-    # the u in b_t), d and b in fp16, y in bf16
+    # the u in b_t), d in fp16, b in bf16, y in bf16
     B, T, R = 2, 200, 264
     w = inputs.make_forward(B, T, R, torch.bfloat16, seed=0)
     g = torch.Generator("cpu").manual_seed(77)
@@ -94,20 +58,10 @@ def test_forward_storage_rounding_fits_the_bf16_tolerance():
     h0 = torch.randn(B, R, generator=g)
     state0 = torch.randn(B, 3, R, generator=g).to(torch.bfloat16)
     for hist, h_init in ((None, None), (state0, h0)):
-        u, _ = oracle.conv1d_causal(w.x, _f(P.conv_w), _f(P.conv_b), None if hist is None else _f(hist))
-        u = _bf16(u)
-        r = oracle.sigmoid(u @ _f(P.W_a).T + _f(P.b_a))
-        i = oracle.sigmoid(u @ _f(P.W_x).T + _f(P.b_x))
-        a_t = oracle.decay_direct(r, _f(P.Lambda))
-        d, b = _fp16(1.0 - a_t), _fp16(np.sqrt(1.0 - a_t * a_t) * i * u)
-        h = np.zeros((B, R)) if h_init is None else _f(h_init)
-        ys = np.empty_like(u)
-        for t in range(T):
-            h = (1.0 - d[:, t]) * h + b[:, t]
-            ys[:, t] = h
+        ys, _ = rm.forward(w.x, P, h_init, hist)
         y_ref, _, _ = oracle.rglru_forward(w.x, P.conv_w, P.conv_b, P.W_a, P.b_a, P.W_x, P.b_x, P.Lambda,
                                            h0=h_init, conv_state0=hist)
-        err = oracle.max_rel_error(_bf16(ys), y_ref)
+        err = oracle.max_rel_error(ys, y_ref)
         print(f"forward parity case, history={hist is not None}: storage rounding alone gives {err:.3e}")
         assert err <= TOL[torch.bfloat16], err
 
@@ -126,42 +80,12 @@ def _backward_problem(B, T, R, with_state, seed):
 
 
 def test_backward_weight_gradients_storage_rounding_needs_the_wider_bound():
-    # The backward's storage formats: u and the recomputed pre-activations z in bf16, h_{t−1}
-    # read from the forward's bf16 y (itself from fp16 d, b), ∂z in bf16 as the operand of
-    # ∂W = Σ_t ∂z_tᵀ u_t, float32 (here exact) arithmetic elsewhere. On two of the GPU
-    # backward test's cases this alone puts ∂W_a above the RG-LRU's 2e-2, inside 4e-2.
+    # The backward's storage formats (rounding_model.backward_weight_gradients). On two of
+    # the GPU backward test's cases they alone put ∂W_a above the RG-LRU's 2e-2, inside 4e-2.
     for B, T, R, with_state in ((2, 64, 128, False), (2, 200, 264, True)):
         w, h0, st0, dy, dh_T = _backward_problem(B, T, R, with_state, seed=B * 1000 + T + R)
         P = w.params
-        cla = 8.0 * -np.log1p(np.exp(-_f(P.Lambda)))
-        u, _ = oracle.conv1d_causal(w.x, _f(P.conv_w), _f(P.conv_b), None if st0 is None else _f(st0))
-        u = _bf16(u)
-        za, zx = u @ _f(P.W_a).T + _f(P.b_a), u @ _f(P.W_x).T + _f(P.b_x)
-        # the forward's y
-        a = np.exp(oracle.sigmoid(za) * cla)
-        d, b = _fp16(1.0 - a), _fp16(np.sqrt(1.0 - a * a) * oracle.sigmoid(zx) * u)
-        h = np.zeros((B, R)) if h0 is None else _f(h0)
-        y = np.empty_like(u)
-        for t in range(T):
-            h = (1.0 - d[:, t]) * h + b[:, t]
-            y[:, t] = h
-        y = _bf16(y)
-        # the reverse recurrence on the recomputed bf16 pre-activations
-        r, i = oracle.sigmoid(_bf16(za)), oracle.sigmoid(_bf16(zx))
-        la = r * cla
-        at, mt = np.exp(la), np.sqrt(-np.expm1(2.0 * la))
-        hp = np.concatenate([np.zeros((B, 1, R)) if h0 is None else _f(h0)[:, None], y[:, :-1]], axis=1)
-        g, a_next = _f(dh_T), np.ones((B, R))
-        dza, dzx = np.empty_like(u), np.empty_like(u)
-        for t in range(T - 1, -1, -1):
-            g = a_next * g + _f(dy[:, t])
-            r_over_m = np.divide(r[:, t], mt[:, t], out=np.zeros((B, R)), where=mt[:, t] > 0)
-            dlr = g * hp[:, t] * at[:, t] * r[:, t] - g * i[:, t] * u[:, t] * at[:, t] ** 2 * r_over_m
-            dza[:, t] = dlr * cla * (1.0 - r[:, t])
-            dzx[:, t] = g * mt[:, t] * u[:, t] * i[:, t] * (1.0 - i[:, t])
-            a_next = at[:, t]
-        dW_a = _bf16(dza).reshape(-1, R).T @ u.reshape(-1, R)
-        dW_x = _bf16(dzx).reshape(-1, R).T @ u.reshape(-1, R)
+        dW_a, dW_x = rm.backward_weight_gradients(w.x, P, dy, h0, st0, dh_T)
         ref = oracle.rglru_backward(w.x, P.conv_w, P.conv_b, P.W_a, P.b_a, P.W_x, P.b_x, P.Lambda, dy, h0=h0,
                                     conv_state0=st0, dh_T=dh_T)
         ea, ex = oracle.max_rel_error(dW_a, ref["dW_a"]), oracle.max_rel_error(dW_x, ref["dW_x"])

@@ -2,8 +2,10 @@
 handed only its inputs and outputs, a process whose memory is reserved up front, a loop
 that must not risk a cudaMalloc synchronising the device). Its scratch is a fixed array
 inside the library. Two calls in a row, through the C ABI, must agree with the
-workspace-taking rglru_scan within the parity tolerances; the second call checks that
-the state the first one leaves behind in the shared array does no harm.
+workspace-taking rglru_scan and with the float64 oracle within the parity tolerances; the
+second call checks that the state the first one leaves behind in the shared array does no
+harm. The largest problem the array holds is run too, so that the size check, the cleared
+region and the top of the array are all exercised.
 
 This file is collected last on purpose, and it also passes when run on its own."""
 import ctypes
@@ -11,12 +13,24 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from gated_linear_rnn_conv1d_b200 import _abi, inputs, rglru
 
-from _util import TOL, pack_gates, rel
+from _util import TOL, f64, pack_gates, rel, unpack_gates
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+SCRATCH = 8 << 20
+
+
+def _tiles(B, T, R, dtype):
+    cw = 128 if dtype == torch.bfloat16 else 64
+    return B * -(-R // cw) * -(-T // 64)
+
+
+def _fits(B, T, R, dtype):
+    cw = 128 if dtype == torch.bfloat16 else 64
+    return 256 + _tiles(B, T, R, dtype) * 4 * cw <= SCRATCH
 
 
 def _case(B, T, R, dtype, seed):
@@ -28,6 +42,15 @@ def _case(B, T, R, dtype, seed):
     return w, pack_gates(za, zx, R, dtype, DEV)
 
 
+def _oracle(w, z, R):
+    """The oracle's scan on the same inputs: u = Conv1D(x), the gates from the (rounded) z."""
+    B, T, _ = w.x.shape
+    za, zx = unpack_gates(z, R)
+    u, _ = oracle.conv1d_causal(w.x, w.params.conv_w, w.params.conv_b)
+    a_t = oracle.decay_direct(oracle.sigmoid(za.reshape(B, T, R)), f64(w.params.Lambda))
+    return oracle.rglru_recurrence(a_t, oracle.sigmoid(zx.reshape(B, T, R)), u, f64(w.h0))
+
+
 def _noalloc(lib, p, x, z, h0, y, h_T, B, T, R, io):
     st = p.struct()
     return lib.rglru_scan_noalloc(ctypes.byref(st), ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(z.data_ptr()),
@@ -36,34 +59,57 @@ def _noalloc(lib, p, x, z, h0, y, h_T, B, T, R, io):
                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
+def _run_and_check(lib, dtype, B, T, R, seed):
+    io = _abi.RGLRU_BF16 if dtype == torch.bfloat16 else _abi.RGLRU_F32
+    w, z = _case(B, T, R, dtype, seed)
+    p = rglru.Params.from_host(w.params)
+    x, h0 = w.x.to(DEV), w.h0.to(DEV)
+    y_ref, h_ref = rglru.scan(p, x, z, h0)
+    y = torch.full_like(x, float("nan"))
+    h_T = torch.full((B, R), float("nan"), device=DEV)
+    assert _noalloc(lib, p, x, z, h0, y, h_T, B, T, R, io) == 0
+    assert lib.rglru_scan_noalloc_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    assert rel(y, y_ref) <= TOL[dtype], (B, T, R)
+    assert rel(h_T, h_ref) <= TOL[dtype], (B, T, R)
+    y_o, h_o = _oracle(w, z, R)
+    assert rel(y, y_o) <= TOL[dtype], (B, T, R)
+    assert rel(h_T, h_o) <= TOL[dtype], (B, T, R)
+
+
 @pytest.mark.parametrize("dtype,shapes", [
     (torch.bfloat16, [(2, 300, 264), (8, 2048, 2048)]),
     (torch.float32, [(1, 256, 256), (3, 130, 72)]),
 ])
-def test_noalloc_scan_matches_workspace_scan_two_calls_in_a_row(dtype, shapes):
+def test_noalloc_scan_matches_workspace_scan_and_oracle_two_calls_in_a_row(dtype, shapes):
+    lib = _abi.load()
+    for k, (B, T, R) in enumerate(shapes):
+        _run_and_check(lib, dtype, B, T, R, seed=10 + k)
+
+
+def test_noalloc_scan_at_the_largest_problem_its_scratch_holds():
+    # 127 rows × 1 channel block × 129 chunks (the last one ragged) = 16383 bf16 tiles:
+    # 256 + 16383·512 bytes, 256 bytes below 8 MiB, so the last tile's states lie in the top
+    # 512 bytes of the array (8 channels keep the oracle's share of the test small)
+    B, T, R = 127, 129 * 64 - 5, 8
+    assert _tiles(B, T, R, torch.bfloat16) == 16383 and _fits(B, T, R, torch.bfloat16)
+    lib = _abi.load()
+    _run_and_check(lib, torch.bfloat16, B, T, R, seed=21)
+    _run_and_check(lib, torch.bfloat16, 2, 300, 264, seed=22)   # and a small call after it
+
+
+@pytest.mark.parametrize("dtype,B,T,R", [
+    (torch.bfloat16, 1, 32768, 4096),   # 16384 bf16 tiles: 256 bytes more than the array
+    (torch.float32, 1, 32768, 4096),    # 32768 float32 tiles of 64 channels: the same excess
+])
+def test_noalloc_scan_rejects_problems_beyond_its_scratch(dtype, B, T, R):
+    assert not _fits(B, T, R, dtype)
     lib = _abi.load()
     io = _abi.RGLRU_BF16 if dtype == torch.bfloat16 else _abi.RGLRU_F32
-    for k, (B, T, R) in enumerate(shapes):
-        w, z = _case(B, T, R, dtype, seed=10 + k)
-        p = rglru.Params.from_host(w.params)
-        x, h0 = w.x.to(DEV), w.h0.to(DEV)
-        y_ref, h_ref = rglru.scan(p, x, z, h0)
-        y = torch.full_like(x, float("nan"))
-        h_T = torch.full((B, R), float("nan"), device=DEV)
-        assert _noalloc(lib, p, x, z, h0, y, h_T, B, T, R, io) == 0
-        assert lib.rglru_workspace_status(None, None) == 0
-        assert rel(y, y_ref) <= TOL[dtype], (B, T, R)
-        assert rel(h_T, h_ref) <= TOL[dtype], (B, T, R)
-
-
-def test_noalloc_scan_rejects_problems_beyond_its_scratch():
-    lib = _abi.load()
-    B, T, R = 1, 32768, 4096            # 16384 tiles: more than the fixed scratch holds
-    x = torch.zeros(B, T, R, dtype=torch.bfloat16, device=DEV)
-    z = torch.zeros(B * T, rglru.gate_pitch(R), dtype=torch.bfloat16, device=DEV)
-    w = inputs.make_forward(1, 1, R, torch.bfloat16)
+    x = torch.zeros(B, T, R, dtype=dtype, device=DEV)
+    z = torch.zeros(B * T, rglru.gate_pitch(R), dtype=dtype, device=DEV)
+    w = inputs.make_forward(1, 1, R, dtype)
     p = rglru.Params.from_host(w.params)
     h0 = torch.zeros(B, R, device=DEV)
     y = torch.empty_like(x)
     h_T = torch.empty(B, R, device=DEV)
-    assert _noalloc(lib, p, x, z, h0, y, h_T, B, T, R, _abi.RGLRU_BF16) == _abi.STATUS_CODE["RGLRU_ERR_WORKSPACE"]
+    assert _noalloc(lib, p, x, z, h0, y, h_T, B, T, R, io) == _abi.STATUS_CODE["RGLRU_ERR_WORKSPACE"]
