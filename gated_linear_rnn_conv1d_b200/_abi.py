@@ -47,6 +47,21 @@ class RGLRULayerWeights(ctypes.Structure):
 
 _LWP = ctypes.POINTER(RGLRULayerWeights)
 
+
+class RGLRUAttentionWeights(ctypes.Structure):
+    _fields_ = [("W_qkv", _P), ("W_o", _P)]
+
+
+_AWP = ctypes.POINTER(RGLRUAttentionWeights)
+
+
+class RGLRUAttentionLayerWeights(ctypes.Structure):
+    _fields_ = [("norm1_scale", _P), ("W_qkv", _P), ("W_o", _P), ("norm2_scale", _P), ("W_gate", _P), ("W_up", _P),
+                ("W_down", _P)]
+
+
+_ALWP = ctypes.POINTER(RGLRUAttentionLayerWeights)
+
 SIGNATURES = {
     "rglru_forward_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "rglru_forward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
@@ -58,6 +73,10 @@ SIGNATURES = {
     "rglru_layer_forward": (_I, [_PP, _LWP, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _S, _P]),
     "rglru_layer_step_workspace_bytes": (_S, [_I, _I, _I, _I, _I]),
     "rglru_layer_step": (_I, [_PP, _LWP, _P, _P, _P, _P, _I, _I, _I, _I, _L, ctypes.c_float, _I, _P, _S, _P]),
+    "rglru_attention_step_workspace_bytes": (_S, [_I, _I, _I]),
+    "rglru_attention_step": (_I, [_AWP, _P, _P, _P, _P, _I, _I, _I, _L, _P, _S, _P]),
+    "rglru_attention_layer_step_workspace_bytes": (_S, [_I, _I, _I, _I]),
+    "rglru_attention_layer_step": (_I, [_ALWP, _P, _P, _P, _P, _I, _I, _I, _I, _L, ctypes.c_float, _P, _S, _P]),
     "rglru_conv1d": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "rglru_gate_pitch": (_L, [_I]),
     "rglru_gate_proj": (_I, [_P, _P, _P, _P, _P, _P, _L, _I, _I, _P]),
@@ -66,6 +85,7 @@ SIGNATURES = {
     "rglru_gate_coeffs": (_I, [_PP, _P, _P, _L, _I, _P]),
     "rglru_scan_coeffs": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _S, _P]),
     "rglru_scan_noalloc": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "rglru_scan_noalloc_status": (_I, [_P]),
     "rglru_gemm_bf16": (_I, [_P, _P, _P, _L, _I, _I, _P]),
     "rglru_backward_workspace_bytes": (_S, [_I, _I, _I]),
     "rglru_backward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _GP, _I, _I, _I, _P, _S, _P]),

@@ -51,7 +51,7 @@ struct ScanArgs {
 // Testing only: the tile index the next scans leave unpublished (-1 disables).
 void set_scan_stall(int64_t tile);
 int64_t scan_stall();
-// coef: z holds the recurrence coefficients (fp16 d = 1 − a_t, b_t = √(1−a_t²)·i_t·u_t)
+// coef: z holds the recurrence coefficients (d = 1 − a_t fp16, b_t = √(1−a_t²)·i_t·u_t bf16)
 // that launch_gemm_coeffs_bf16 forms, instead of pre-activations (bf16 IO only); x, the
 // conv parameters and Λ are then not read.
 cudaError_t launch_scan(const ScanArgs& a, bool bf16, cudaStream_t s, bool coef = false);
@@ -76,7 +76,7 @@ int num_sms();
 
 // `status`: device word the kernel ORs kStatusTimeout into if a bounded wait gives up.
 // The gate GEMM with the recurrence coefficients formed in its epilogue: g packed like z,
-// fp16 d = 1 − a_t in the z_a places and b_t = √(1−a_t²)·i_t·u_t in the z_x places (the
+// d = 1 − a_t (fp16) in the z_a places and b_t = √(1−a_t²)·i_t·u_t (bf16) in the z_x places (the
 // epilogue reads its rows of u, the GEMM's A operand).
 cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
                                     const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s);
@@ -128,6 +128,22 @@ cudaError_t launch_add_rmsnorm(const void* x, const void* o, void* y, void* n, c
                                int D, float eps, cudaStream_t s);
 // p = GeLU(gate) ⊙ up over n elements (n % 8 == 0); p may be gate.
 cudaError_t launch_gelu_mul(const void* gate, const void* up, void* p, int64_t n, cudaStream_t s);
+
+// ---- Griffin local multi-query attention, decode step (attention.cu) ----------------------
+// D_head = 128, H = D / 128 query heads (1 ≤ H ≤ kAttnMaxHeads), one key/value head; the
+// window W a multiple of 128. Workspace: [status word | qkv [B][(H+2)·128] bf16 | rotated
+// queries [B][H][128] bf16 | partial outputs [B][W/128][H][128] f32 | maxima, sums
+// [B][W/128][H] f32 | o [B][H·128] bf16].
+constexpr int kAttnMaxHeads = 128;
+struct AttnLayout {
+  int H, n_chunks;
+  size_t off_qkv, off_q, off_op, off_m, off_l, off_o, bytes;
+};
+AttnLayout attn_layout(int B, int D, int W);
+// RoPE and ring writes of position `pos` from qkv (in the workspace), then the windowed
+// attention into the workspace's o. k_ring [B][W][128], v_ring [B][128][W] bf16, in place.
+cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, int64_t pos, int B, int D, int W,
+                                  const AttnLayout& L, void* ws, unsigned* status, cudaStream_t s);
 
 // ---- backward (bf16 IO) --------------------------------------------------------------
 // Workspace of launch_backward: [status | u | z | chunk maps P, Q | chunk carries | ∂z |

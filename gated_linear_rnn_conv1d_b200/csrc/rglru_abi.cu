@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstring>
 #include <cuda_runtime.h>
+#include <mutex>
 #include <nvtx3/nvToolsExt.h>
 
 #include "../../include/rglru.h"
@@ -163,6 +164,46 @@ StepLayout step_layout(int B, int R) {
 
 uint8_t* bytes(void* p) { return static_cast<uint8_t*>(p); }
 
+// Local attention: D a multiple of 128 (H = D/128 heads of 128), 1 ≤ H ≤ kAttnMaxHeads;
+// window a multiple of 128, at most 65536.
+bool valid_attention(int B, int D, int window) {
+  return B >= 1 && B <= 65535 && D >= 128 && D % 128 == 0 && D / 128 <= kAttnMaxHeads && window >= 128 &&
+         window % 128 == 0 && window <= 65536;
+}
+
+// Griffin's local-attention residual layer, decode step: [the attention step's workspace
+// (status word at 0) | n [B][D] | o [B][D] | residual [B][D] | gate, up [B][Hm]], bf16.
+struct AttnLayerLayout {
+  AttnLayout attn;
+  size_t off_n, off_o, off_res, off_gate, off_up, bytes;
+};
+AttnLayerLayout attn_layer_layout(int B, int D, int Hm, int window) {
+  AttnLayerLayout L;
+  L.attn = attn_layout(B, D, window);
+  const size_t row = round256((size_t)B * D * 2), hid = round256((size_t)B * Hm * 2);
+  L.off_n = round256(L.attn.bytes);
+  L.off_o = L.off_n + row;
+  L.off_res = L.off_o + row;
+  L.off_gate = L.off_res + row;
+  L.off_up = L.off_gate + hid;
+  L.bytes = L.off_up + hid;
+  return L;
+}
+
+// x_t → out_t through the local-attention block: the fused q/k/v projection, RoPE, ring
+// update and windowed attention, the output projection.
+cudaError_t attention_sequence(const rglru_attention_weights* w, const void* x_t, void* k_ring, void* v_ring,
+                               void* out_t, int B, int D, int window, int64_t pos, const AttnLayout& L, void* ws,
+                               cudaStream_t s) {
+  unsigned* status = reinterpret_cast<unsigned*>(ws);
+  const int nqkv = (L.H + 2) * 128;
+  void* qkv = bytes(ws) + L.off_qkv;
+  cudaError_t e = launch_gemm_bf16(x_t, w->W_qkv, qkv, B, nqkv, D, nqkv, status, s);
+  if (e == cudaSuccess) e = launch_attention_core(qkv, k_ring, v_ring, pos, B, D, window, L, ws, status, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(bytes(ws) + L.off_o, w->W_o, out_t, B, D, L.H * 128, D, status, s);
+  return e;
+}
+
 // Hawk residual layer: [recurrent block workspace (status word at 0) | n: RMSNorm output
 // [B·T][D] (RMSNorm₁, then RMSNorm₂) | o: component output [B·T][D] (the block's, then
 // the MLP's) | y: residual stream [B·T][D] | gate (then p) [B·T][H] | up [B·T][H]], bf16.
@@ -281,6 +322,35 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
   a.n_tiles = (int)sl.n_tiles;
   a.pitch = pitch;
   return launch_scan(a, bf16, s, coef);
+}
+
+// ---- fixed scratch of rglru_scan_noalloc ---------------------------------------------
+// For callers that cannot allocate device memory, the scan's scratch (status word, tile
+// ticket, published chunk states: the layout scan_layout gives, 256 + 4·CW bytes per tile
+// with CW = 128 channels for bf16 and 64 for float32) lives in this file-scope array, which
+// every GPU that loads the library holds until the process exits. Its name in host code
+// is a host-side stand-in, not a device address: the address is looked up once per
+// device, with that device current, and handed to the kernels.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+int noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dev < 0 || dev >= kMaxDevices) return RGLRU_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* a = nullptr;
+    e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (a == nullptr) return fail_cuda(cudaErrorInvalidSymbol);
+    addr[dev] = a;
+  }
+  *out = addr[dev];
+  return RGLRU_OK;
 }
 
 }  // namespace
@@ -714,6 +784,114 @@ int rglru_layer_step(const rglru_params* params, const rglru_layer_weights* w, c
   if (e == cudaSuccess) e = launch_gemm_bf16(gate, w->W_down, o, B, D, H, D, status, s);
   if (e == cudaSuccess) e = launch_add_rmsnorm(res, o, out_t, nullptr, nullptr, B, D, eps, s);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+size_t rglru_attention_step_workspace_bytes(int B, int D, int window) {
+  if (!valid_attention(B, D, window)) return 0;
+  return attn_layout(B, D, window).bytes;
+}
+
+int rglru_attention_step(const rglru_attention_weights* w, const void* x_t, void* k_ring, void* v_ring, void* out_t,
+                         int B, int D, int window, int64_t pos, void* workspace, size_t workspace_bytes,
+                         rglru_stream_t stream) {
+  const Range range("rglru_attention_step");
+  if (!valid_attention(B, D, window) || pos < 0) return RGLRU_ERR_SHAPE;
+  if (w == nullptr || w->W_qkv == nullptr || w->W_o == nullptr || x_t == nullptr || k_ring == nullptr ||
+      v_ring == nullptr || out_t == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(w->W_qkv) || !aligned16(w->W_o) || !aligned16(x_t) || !aligned16(k_ring) || !aligned16(v_ring) ||
+      !aligned16(out_t))
+    return RGLRU_ERR_ALIGN;
+  const AttnLayout L = attn_layout(B, D, window);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  int st = check_device();
+  if (st != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess) e = attention_sequence(w, x_t, k_ring, v_ring, out_t, B, D, window, pos, L, workspace, s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+size_t rglru_attention_layer_step_workspace_bytes(int B, int D, int H, int window) {
+  if (!valid_attention(B, D, window) || !valid_R(H)) return 0;
+  return attn_layer_layout(B, D, H, window).bytes;
+}
+
+int rglru_attention_layer_step(const rglru_attention_layer_weights* w, const void* x_t, void* k_ring, void* v_ring,
+                               void* out_t, int B, int D, int H, int window, int64_t pos, float eps,
+                               void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_attention_layer_step");
+  if (!valid_attention(B, D, window) || !valid_R(H) || pos < 0) return RGLRU_ERR_SHAPE;
+  if (!(eps >= 0.0f) || eps > 1.0f) return RGLRU_ERR_SHAPE;  // also rejects NaN
+  if (w == nullptr || w->norm1_scale == nullptr || w->W_qkv == nullptr || w->W_o == nullptr ||
+      w->norm2_scale == nullptr || w->W_gate == nullptr || w->W_up == nullptr || w->W_down == nullptr ||
+      x_t == nullptr || k_ring == nullptr || v_ring == nullptr || out_t == nullptr)
+    return RGLRU_ERR_NULL;
+  if (!aligned16(w->norm1_scale) || !aligned16(w->W_qkv) || !aligned16(w->W_o) || !aligned16(w->norm2_scale) ||
+      !aligned16(w->W_gate) || !aligned16(w->W_up) || !aligned16(w->W_down) || !aligned16(x_t) ||
+      !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out_t))
+    return RGLRU_ERR_ALIGN;
+  if (out_t == x_t) return RGLRU_ERR_SHAPE;  // the residual stream is read after out_t is written
+  const AttnLayerLayout L = attn_layer_layout(B, D, H, window);
+  if (workspace == nullptr || workspace_bytes < L.bytes) return RGLRU_ERR_WORKSPACE;
+  if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
+  int st = check_device();
+  if (st != RGLRU_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint8_t* ws = bytes(workspace);
+  unsigned* status = reinterpret_cast<unsigned*>(ws);
+  void* nrm = ws + L.off_n;
+  void* o = ws + L.off_o;
+  void* res = ws + L.off_res;
+  void* gate = ws + L.off_gate;
+  void* up = ws + L.off_up;
+  const rglru_attention_weights aw{w->W_qkv, w->W_o};
+  cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
+  // residual stream + LocalMQA(RMSNorm₁(x_t))
+  if (e == cudaSuccess) e = launch_add_rmsnorm(x_t, nullptr, nullptr, nrm, w->norm1_scale, B, D, eps, s);
+  if (e == cudaSuccess) e = attention_sequence(&aw, nrm, k_ring, v_ring, o, B, D, window, pos, L.attn, workspace, s);
+  if (e == cudaSuccess) e = launch_add_rmsnorm(x_t, o, res, nrm, w->norm2_scale, B, D, eps, s);
+  // + MLP(RMSNorm₂(·))
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_gate, gate, B, H, D, H, status, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(nrm, w->W_up, up, B, H, D, H, status, s);
+  if (e == cudaSuccess) e = launch_gelu_mul(gate, up, gate, (int64_t)B * H, s);
+  if (e == cudaSuccess) e = launch_gemm_bf16(gate, w->W_down, o, B, D, H, D, status, s);
+  if (e == cudaSuccess) e = launch_add_rmsnorm(res, o, out_t, nullptr, nullptr, B, D, eps, s);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_scan_noalloc(const rglru_params* params, const void* x, const void* z, const void* conv_state0,
+                       const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R, int io_dtype,
+                       rglru_stream_t stream) {
+  const Range range("rglru_scan_noalloc");
+  if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
+  if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
+  int st = check_params(params);
+  if (st != RGLRU_OK) return st;
+  if (x == nullptr || z == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(x) || !aligned16(z) || !aligned16(y) || !aligned16(conv_state0) || !aligned16(h0) ||
+      !aligned16(gate_g) || !aligned16(h_T))
+    return RGLRU_ERR_ALIGN;
+  const ScanLayout sl = scan_layout(B, T, R, io_dtype == RGLRU_BF16);
+  if (sl.bytes > kNoAllocScratchBytes) return RGLRU_ERR_WORKSPACE;  // beyond the fixed scratch
+  if ((st = check_device()) != RGLRU_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != RGLRU_OK) return st;
+  // the array keeps the previous call's contents: run_scan clears the status word, the
+  // ticket and the chunk states this call uses before its kernel starts
+  cudaError_t e = run_scan(params, x, z, gate_pitch(R), conv_state0, h0, gate_g, y, h_T, B, T, R,
+                           io_dtype == RGLRU_BF16, sl, scratch, true, (cudaStream_t)stream);
+  return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+
+int rglru_scan_noalloc_status(rglru_stream_t stream) {
+  const int st = check_device();
+  if (st != RGLRU_OK) return st;
+  void* scratch = nullptr;
+  const int sa = noalloc_scratch(&scratch);
+  if (sa != RGLRU_OK) return sa;
+  return rglru_workspace_status(scratch, stream);
 }
 
 int rglru_workspace_status(void* workspace, rglru_stream_t stream) {

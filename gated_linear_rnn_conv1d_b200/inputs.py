@@ -133,6 +133,26 @@ def make_decode(B: int, R: int, io_dtype: torch.dtype = torch.bfloat16, seed: in
     return Workload(name or f"rglru_decode_B{B}_R{R}", B, 0, R, io_dtype, x, p, h0)
 
 
+def make_attention(D: int, M: int = 3, io_dtype: torch.dtype = torch.bfloat16, seed: int = 0) -> dict:
+    """Weights of Griffin's local-attention residual layer (D_head = 128, H = D/128 query
+    heads, one key/value head), LeCun normal (std 1/√fan_in), drawn in the order W_q [D][D],
+    W_k [128][D], W_v [128][D], W_o [D][D], then the two RMSNorm gains ~ U[0.5, 1.5] and
+    the gated MLP as make_layer draws it (W_gate, W_up [M·D][D], W_down [D][M·D]). The
+    decode tokens come from decode_token."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    w = {"W_q": _normal(g, (D, D), 1.0 / math.sqrt(D)).to(io_dtype),
+         "W_k": _normal(g, (128, D), 1.0 / math.sqrt(D)).to(io_dtype),
+         "W_v": _normal(g, (128, D), 1.0 / math.sqrt(D)).to(io_dtype),
+         "W_o": _normal(g, (D, D), 1.0 / math.sqrt(D)).to(io_dtype)}
+    w["norm1_scale"] = 0.5 + torch.rand(D, generator=g, dtype=torch.float32)
+    w["norm2_scale"] = 0.5 + torch.rand(D, generator=g, dtype=torch.float32)
+    H = M * D
+    w["W_gate"] = _normal(g, (H, D), 1.0 / math.sqrt(D)).to(io_dtype)
+    w["W_up"] = _normal(g, (H, D), 1.0 / math.sqrt(D)).to(io_dtype)
+    w["W_down"] = _normal(g, (D, H), 1.0 / math.sqrt(H)).to(io_dtype)
+    return w
+
+
 def decode_token(step: int, B: int, R: int, io_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
     g = torch.Generator("cpu").manual_seed(DECODE_SEED_BASE + step)
     return _normal(g, (B, R), 1.0).to(io_dtype)

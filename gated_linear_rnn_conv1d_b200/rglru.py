@@ -134,24 +134,35 @@ def backward(params: Params, x: torch.Tensor, y: torch.Tensor, dy: torch.Tensor,
 class HostForwardPlan:
     """Device buffers and streams for forward_host on inputs of shape [B][T][R].
 
-    The batch is cut into `groups` row groups; `slots` of them are in flight at once, each
-    slot with its own device copy of x, y, h_T and a forward workspace. Made once and reused,
-    so forward_host itself allocates nothing.
+    The input is cut into `groups` pieces, `slots` of them in flight at once, each slot with
+    its own device copy of x and y and a forward workspace. Pieces are row groups of the
+    batch when B is a multiple of `groups` (rows are independent); otherwise (a long single
+    sequence) they are consecutive time chunks of T / groups steps, a multiple of 64, each
+    started from the state (h, Conv1D history) the previous chunk ended in. Made once and
+    reused, so forward_host itself allocates nothing.
     """
 
     def __init__(self, B: int, T: int, R: int, dtype: torch.dtype = torch.bfloat16, *, groups: int = 4,
                  slots: int = 3, device=None):
-        if B % groups:
-            raise ValueError(f"B={B} is not a multiple of groups={groups}")
         self.B, self.T, self.R, self.dtype, self.groups = B, T, R, dtype, groups
-        self.rows = B // groups
+        if B % groups == 0:
+            self.split, self.rows, self.steps = "rows", B // groups, T
+        elif T % groups == 0 and (T // groups) % 64 == 0:
+            self.split, self.rows, self.steps = "time", B, T // groups
+        else:
+            raise ValueError(f"neither B={B} nor T={T} splits into {groups} groups (time chunks: multiples of 64)")
         self.slots = min(slots, groups)
         dev = torch.device("cuda") if device is None else torch.device(device)
-        nws = forward_workspace_bytes(self.rows, T, R, dtype)
-        self.x = [torch.empty(self.rows, T, R, dtype=dtype, device=dev) for _ in range(self.slots)]
-        self.y = [torch.empty(self.rows, T, R, dtype=dtype, device=dev) for _ in range(self.slots)]
+        nws = forward_workspace_bytes(self.rows, self.steps, R, dtype)
+        shape = (self.rows, self.steps, R)
+        self.x = [torch.empty(shape, dtype=dtype, device=dev) for _ in range(self.slots)]
+        self.y = [torch.empty(shape, dtype=dtype, device=dev) for _ in range(self.slots)]
         self.h_T = [torch.empty(self.rows, R, dtype=torch.float32, device=dev) for _ in range(self.slots)]
         self.ws = [torch.empty(max(nws, 256), dtype=torch.uint8, device=dev) for _ in range(self.slots)]
+        # time chunks hand their final state to the next chunk (ping-pong, never read and
+        # written by the same call)
+        self.conv_state = [torch.empty(self.rows, 3, R, dtype=dtype, device=dev) for _ in range(2)] \
+            if self.split == "time" else None
         self.copy_in = torch.cuda.Stream(dev)
         self.compute = torch.cuda.Stream(dev)
         self.copy_out = torch.cuda.Stream(dev)
@@ -169,13 +180,16 @@ class HostForwardPlan:
 def forward_host(params: Params, x_host: torch.Tensor, y_host: torch.Tensor, h_T_host: torch.Tensor,
                  plan: HostForwardPlan, stream: Optional[torch.cuda.Stream] = None) -> None:
     """rglru_forward on host tensors (pinned for the copies to overlap): x_host [B][T][R] →
-    y_host [B][T][R], h_T_host [B][R] fp32, zero initial state.
+    y_host [B][T][R], h_T_host [B][R] fp32, zero initial state and history.
 
-    Batch rows are independent, so the plan's row groups are pipelined: the host→device copy
-    of one group, rglru_forward on the next and the device→host copy of a third run on three
-    streams at once. The work is ordered after `stream` (default: the current stream) and
-    `stream` waits for all of it before later work, so events recorded on it time the whole
-    transfer. Results are bit-identical to one rglru_forward over the whole batch.
+    The plan's pieces are pipelined: the host→device copy of one piece, rglru_forward on the
+    next and the device→host copy of a third run on three streams at once. Row groups are
+    independent; time chunks run one after another on the compute stream, each from the
+    state its predecessor returned. The work is ordered after `stream` (default: the
+    current stream) and `stream` waits for all of it before later work, so events recorded
+    on it time the whole transfer. With row groups the results are bit-identical to one
+    rglru_forward over the whole batch; with time chunks they equal the sequence split at
+    the chunk boundaries.
     """
     if x_host.shape != (plan.B, plan.T, plan.R) or x_host.dtype != plan.dtype:
         raise ValueError("x_host does not match the plan")
@@ -185,23 +199,35 @@ def forward_host(params: Params, x_host: torch.Tensor, y_host: torch.Tensor, h_T
     freed = [None] * plan.slots  # event: the slot's last device→host copy has finished
     for g in range(plan.groups):
         k = g % plan.slots
-        rows = slice(g * plan.rows, (g + 1) * plan.rows)
+        if plan.split == "rows":
+            piece = (slice(g * plan.rows, (g + 1) * plan.rows),)
+        else:
+            piece = (slice(None), slice(g * plan.steps, (g + 1) * plan.steps))
         with torch.cuda.stream(plan.copy_in):
             plan.copy_in.wait_event(start)
             if freed[k] is not None:
                 plan.copy_in.wait_event(freed[k])
-            plan.x[k].copy_(x_host[rows], non_blocking=True)
+            plan.x[k].copy_(x_host[piece], non_blocking=True)
             loaded = torch.cuda.Event()
             loaded.record(plan.copy_in)
         plan.compute.wait_event(loaded)
-        forward(params, plan.x[k], workspace=plan.ws[k], y=plan.y[k], h_T=plan.h_T[k], want_conv_state=False,
-                stream=plan.compute)
+        if plan.split == "rows":
+            forward(params, plan.x[k], workspace=plan.ws[k], y=plan.y[k], h_T=plan.h_T[k], want_conv_state=False,
+                    stream=plan.compute)
+        else:
+            h_in = plan.h_T[(g - 1) % plan.slots] if g > 0 else None
+            st_in = plan.conv_state[(g - 1) % 2] if g > 0 else None
+            forward(params, plan.x[k], h_in, st_in, workspace=plan.ws[k], y=plan.y[k], h_T=plan.h_T[k],
+                    conv_state_T=plan.conv_state[g % 2], stream=plan.compute)
         done = torch.cuda.Event()
         done.record(plan.compute)
         with torch.cuda.stream(plan.copy_out):
             plan.copy_out.wait_event(done)
-            y_host[rows].copy_(plan.y[k], non_blocking=True)
-            h_T_host[rows].copy_(plan.h_T[k], non_blocking=True)
+            y_host[piece].copy_(plan.y[k], non_blocking=True)
+            if plan.split == "rows":
+                h_T_host[piece[0]].copy_(plan.h_T[k], non_blocking=True)
+            elif g == plan.groups - 1:
+                h_T_host.copy_(plan.h_T[k], non_blocking=True)
             freed[k] = torch.cuda.Event()
             freed[k].record(plan.copy_out)
     for e in freed:
@@ -325,6 +351,84 @@ def layer_step(params: Params, weights: LayerWeights, x_t: torch.Tensor, conv_st
     return out_t
 
 
+@dataclass
+class AttentionWeights:
+    """Device-resident weights of Griffin's local-attention block (see rglru_attention_weights
+    in include/rglru.h): W_qkv [(H+2)·128][D] (W_q, then W_k, then W_v rows), W_o [D][H·128],
+    bf16. For the residual layer also the two RMSNorm gains (float32) and the gated MLP."""
+    W_qkv: torch.Tensor
+    W_o: torch.Tensor
+    norm1_scale: Optional[torch.Tensor] = None
+    norm2_scale: Optional[torch.Tensor] = None
+    W_gate: Optional[torch.Tensor] = None
+    W_up: Optional[torch.Tensor] = None
+    W_down: Optional[torch.Tensor] = None
+
+    @classmethod
+    def from_host(cls, w: dict, device="cuda") -> "AttentionWeights":
+        """Copies a dict with W_q, W_k, W_v, W_o (and optionally the layer's norm gains and MLP
+        weights) to `device`, stacking W_q, W_k, W_v into W_qkv."""
+        W_qkv = torch.cat([w["W_q"], w["W_k"], w["W_v"]], 0)
+        opt = {k: w[k].to(device).contiguous() for k in ("norm1_scale", "norm2_scale", "W_gate", "W_up", "W_down")
+               if k in w}
+        return cls(W_qkv.to(device).contiguous(), w["W_o"].to(device).contiguous(), **opt)
+
+    def struct(self) -> _abi.RGLRUAttentionWeights:
+        return _abi.RGLRUAttentionWeights(self.W_qkv.data_ptr(), self.W_o.data_ptr())
+
+    def layer_struct(self) -> _abi.RGLRUAttentionLayerWeights:
+        return _abi.RGLRUAttentionLayerWeights(*(getattr(self, f).data_ptr() for f in (
+            "norm1_scale", "W_qkv", "W_o", "norm2_scale", "W_gate", "W_up", "W_down")))
+
+
+def attention_rings(B: int, window: int, device="cuda") -> Tuple[torch.Tensor, torch.Tensor]:
+    """Empty KV rings of the local attention: keys [B][window][128], values [B][128][window]."""
+    return (torch.empty(B, window, 128, dtype=torch.bfloat16, device=device),
+            torch.empty(B, 128, window, dtype=torch.bfloat16, device=device))
+
+
+def attention_step_workspace_bytes(B: int, D: int, window: int) -> int:
+    return _abi.load().rglru_attention_step_workspace_bytes(B, D, window)
+
+
+def attention_step(weights: AttentionWeights, x_t: torch.Tensor, k_ring: torch.Tensor, v_ring: torch.Tensor,
+                   pos: int, *, workspace: Optional[torch.Tensor] = None, out_t: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_attention_step: x_t [B][D] → out_t [B][D] at position pos; the rings in place."""
+    lib = _abi.load()
+    B, D = x_t.shape
+    W = k_ring.shape[1]
+    out_t = torch.empty_like(x_t) if out_t is None else out_t
+    ws = _workspace(lib.rglru_attention_step_workspace_bytes(B, D, W), x_t.device, workspace)
+    st = weights.struct()
+    _abi.check("rglru_attention_step", lib.rglru_attention_step(
+        ctypes.byref(st), _p(x_t), _p(k_ring), _p(v_ring), _p(out_t), B, D, W, int(pos), _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return out_t
+
+
+def attention_layer_step_workspace_bytes(B: int, D: int, H: int, window: int) -> int:
+    return _abi.load().rglru_attention_layer_step_workspace_bytes(B, D, H, window)
+
+
+def attention_layer_step(weights: AttentionWeights, x_t: torch.Tensor, k_ring: torch.Tensor, v_ring: torch.Tensor,
+                         pos: int, *, eps: float = 1e-6, workspace: Optional[torch.Tensor] = None,
+                         out_t: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """rglru_attention_layer_step: Griffin's local-attention residual layer, one decode step."""
+    lib = _abi.load()
+    B, D = x_t.shape
+    W = k_ring.shape[1]
+    H = weights.W_gate.shape[0]
+    out_t = torch.empty_like(x_t) if out_t is None else out_t
+    ws = _workspace(lib.rglru_attention_layer_step_workspace_bytes(B, D, H, W), x_t.device, workspace)
+    st = weights.layer_struct()
+    _abi.check("rglru_attention_layer_step", lib.rglru_attention_layer_step(
+        ctypes.byref(st), _p(x_t), _p(k_ring), _p(v_ring), _p(out_t), B, D, H, W, int(pos), float(eps), _p(ws),
+        ws.numel() * ws.element_size(), _s(stream)))
+    return out_t
+
+
 def conv1d(params: Params, x: torch.Tensor, conv_state0: Optional[torch.Tensor] = None, *,
            u: Optional[torch.Tensor] = None, conv_state_T: Optional[torch.Tensor] = None,
            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
@@ -377,15 +481,26 @@ def scan(params: Params, x: torch.Tensor, z: torch.Tensor, h0: Optional[torch.Te
 
 def gate_coeffs(params: Params, u: torch.Tensor, *, g: Optional[torch.Tensor] = None,
                 stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
-    """rglru_gate_coeffs: u [N_tok][R] bf16 → packed fp16 recurrence coefficients
-    (d = 1 − a_t in the recurrence-gate places, b_t = √(1−a_t²)·i_t·u_t in the input-gate
-    places)."""
+    """rglru_gate_coeffs: u [N_tok][R] bf16 → packed recurrence coefficients as raw 16-bit
+    words (torch.int16): d = 1 − a_t as fp16 in the recurrence-gate places,
+    b_t = √(1−a_t²)·i_t·u_t as bf16 in the input-gate places (see split_coeffs)."""
     lib = _abi.load()
     N, R = u.shape
-    g = torch.empty(N, gate_pitch(R), dtype=torch.float16, device=u.device) if g is None else g
+    g = torch.empty(N, gate_pitch(R), dtype=torch.int16, device=u.device) if g is None else g
+    if g.dtype != torch.int16 or g.shape != (N, gate_pitch(R)):
+        raise ValueError("g must be int16 [N_tok][gate_pitch(R)]")
     st = params.struct()
     _abi.check("rglru_gate_coeffs", lib.rglru_gate_coeffs(ctypes.byref(st), _p(u), _p(g), N, R, _s(stream)))
     return g
+
+
+def split_coeffs(g: torch.Tensor, R: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The packed coefficient words of gate_coeffs as (d [N][R] float16, b [N][R] bfloat16)."""
+    N = g.shape[0]
+    blocks = g.view(N, -1, 2, 128)
+    d = blocks[:, :, 0, :].reshape(N, -1)[:, :R].view(torch.float16)
+    b = blocks[:, :, 1, :].reshape(N, -1)[:, :R].view(torch.bfloat16)
+    return d, b
 
 
 def scan_coeffs(g: torch.Tensor, B: int, T: int, R: int, h0: Optional[torch.Tensor] = None,
@@ -395,8 +510,8 @@ def scan_coeffs(g: torch.Tensor, B: int, T: int, R: int, h0: Optional[torch.Tens
     """rglru_scan_coeffs: packed coefficients of B·T rows (from gate_coeffs) → (y [B][T][R]
     bf16, h_T [B][R] float32); needs neither x nor the parameters."""
     lib = _abi.load()
-    if g.shape[0] != B * T or g.dtype != torch.float16:
-        raise ValueError("g must be the float16 packed coefficients of B·T rows")
+    if g.shape[0] != B * T or g.dtype != torch.int16:
+        raise ValueError("g must be the int16 packed coefficients of B·T rows (from gate_coeffs)")
     y = torch.empty(B, T, R, dtype=torch.bfloat16, device=g.device) if y is None else y
     h_T = torch.empty(B, R, dtype=torch.float32, device=g.device) if h_T is None else h_T
     ws = _workspace(lib.rglru_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16), g.device, workspace)

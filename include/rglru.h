@@ -95,10 +95,19 @@ typedef struct {
  *   h_T          [B][R] float32 final state (may be NULL)
  *   conv_state_T [B][3][R] io_dtype: (x_{T-3}, x_{T-2}, x_{T-1}) in time order (may be NULL)
  *   workspace    device buffer of at least rglru_forward_workspace_bytes(B, T, R, io_dtype)
- *                bytes, 256-byte aligned. It holds u, the gate pre-activations and the
+ *                bytes, 256-byte aligned. It holds u, the gate GEMM's output and the
  *                scan's chunk carries; its contents need no initialisation.
- * Kernels: conv (x → u), the gate GEMM (2-SM tcgen05 for bf16, FFMA for f32) writing the
- * packed pre-activations, then the fused gates + log-space decay + chunked scan kernel.
+ * Kernels, RGLRU_BF16: conv (x → u, bf16), the 2-SM tcgen05 gate GEMM whose epilogue
+ * applies the gates and the log-space decay and writes the recurrence coefficients
+ * d = 1 − a_t (fp16) and b_t = √(1 − a_t²)·i_t·u_t (bf16) (rglru_gate_coeffs), then the
+ * chunked scan of h_t = (1 − d)·h_{t−1} + b_t (rglru_scan_coeffs). RGLRU_F32: conv, the
+ * FFMA gate GEMM writing the packed pre-activations (rglru_gate_proj), then the scan that
+ * recomputes u and applies the gates and the decay itself (rglru_scan).
+ * Domain: every finite input whose Conv1D output u, pre-activations and states are finite
+ * in float32 gives finite outputs (no format narrower than the IO type holds u-scaled
+ * values). With bf16 IO the gates are evaluated from the bf16-rounded u: where W u is so
+ * large that a pre-activation's rounding error crosses σ's transition, r and i differ from
+ * the unrounded ones (a property of the bf16 operand, not of the scan).
  * --------------------------------------------------------------------------------- */
 RGLRU_API size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype);
 RGLRU_API int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0,
@@ -200,6 +209,64 @@ RGLRU_API int rglru_layer_step(const rglru_params* params, const rglru_layer_wei
                                rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Griffin's local multi-query attention, one decode step ("Griffin：…", §时间混合块:
+ * MQA with H query heads of D_head = 128, H·D_head = D, one key/value head shared by all
+ * of them, RoPE as the relative position embedding, sliding-window attention whose KV
+ * cache is bounded by the window; "Griffin's Compromise…", §Griffin: window 1024, one
+ * local-attention residual block after every two recurrent ones). At position `pos`:
+ *   q = x_t W_qᵀ, k = x_t W_kᵀ, v = x_t W_vᵀ;  q, k rotated by RoPE at `pos`
+ *   (pair i = (x_{2i}, x_{2i+1}) turned by pos·θ_i, θ_i = 10000^(−2i/128));
+ *   (k, v) stored into ring slot (pos mod window);
+ *   o_h = Σ_s softmax_s(q_h·k_s / √128) v_s over the window's positions
+ *         max(0, pos − window + 1) … pos;  out_t = o W_oᵀ.
+ *
+ *   weights.W_qkv  [(H+2)·128][D] bf16, row-major [out][in]: the H·128 rows of W_q (head h
+ *                  in rows 128h … 128h+127), then the 128 rows of W_k, then of W_v
+ *   weights.W_o    [D][H·128] bf16
+ *   x_t, out_t     [B][D] bf16
+ *   k_ring         [B][window][128] bf16, rotated keys, slot-major; updated IN PLACE
+ *   v_ring         [B][128][window] bf16, values stored dimension-major (value d of slot s
+ *                  at [b][d][s]); updated IN PLACE. Slots holding no position yet
+ *                  (pos < window − 1) are never read, so the rings need no initialisation.
+ *   pos            ≥ 0, the position of x_t; the rings hold positions pos − window … pos − 1
+ *   workspace      at least rglru_attention_step_workspace_bytes(B, D, window) bytes,
+ *                  256-byte aligned
+ * D a multiple of 128 with D/128 ≤ 128; window a multiple of 128 (≤ 65536); B ≤ 65535.
+ * Errors as everywhere (RGLRU_ERR_SHAPE for any other D, window, B or pos < 0); a timeout
+ * of a bounded wait is reported by rglru_workspace_status(workspace, stream).
+ * --------------------------------------------------------------------------------- */
+typedef struct {
+  const void* W_qkv; /* [(H+2)·128][D] */
+  const void* W_o;   /* [D][H·128]     */
+} rglru_attention_weights;
+RGLRU_API size_t rglru_attention_step_workspace_bytes(int B, int D, int window);
+RGLRU_API int rglru_attention_step(const rglru_attention_weights* weights, const void* x_t, void* k_ring,
+                                   void* v_ring, void* out_t, int B, int D, int window, int64_t pos,
+                                   void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+/* The residual block of Griffin with local attention as its temporal-mixing block, one
+ * decode step (§残块, Fig. 2(a), as the Hawk layer above with local MQA in place of the
+ * recurrent block):
+ *   y = x_t + LocalMQA(RMSNorm₁(x_t)),   out_t = y + (GeLU(n W_gateᵀ) ⊙ n W_upᵀ) W_downᵀ,
+ *   n = RMSNorm₂(y)
+ * x_t, out_t [B][D] bf16, distinct; k_ring, v_ring, pos, window as rglru_attention_step;
+ * W_gate, W_up [H][D], W_down [D][H] bf16 (H = M·D, the MLP width); eps as the Hawk layer.
+ * workspace: at least rglru_attention_layer_step_workspace_bytes(B, D, H, window) bytes. */
+typedef struct {
+  const float* norm1_scale; /* [D] */
+  const void* W_qkv;        /* [(D/128 + 2)·128][D] */
+  const void* W_o;          /* [D][D] */
+  const float* norm2_scale; /* [D] */
+  const void* W_gate;       /* [H][D] */
+  const void* W_up;         /* [H][D] */
+  const void* W_down;       /* [D][H] */
+} rglru_attention_layer_weights;
+RGLRU_API size_t rglru_attention_layer_step_workspace_bytes(int B, int D, int H, int window);
+RGLRU_API int rglru_attention_layer_step(const rglru_attention_layer_weights* weights, const void* x_t,
+                                         void* k_ring, void* v_ring, void* out_t, int B, int D, int H, int window,
+                                         int64_t pos, float eps, void* workspace, size_t workspace_bytes,
+                                         rglru_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Backward of rglru_forward for bf16 IO: the gradients of a scalar loss ℓ with respect to
  * the input, the parameters, the initial state and the conv history, given ∂ℓ/∂y and
  * ∂ℓ/∂h_T. Reverse-mode differentiation of Eq. (1)–(4) above (with the log-space decay
@@ -279,12 +346,13 @@ RGLRU_API int rglru_scan(const rglru_params* params, const void* x, const void* 
  *   epilogue ("Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元,
  *   Eq. (1)–(4)): with z as in rglru_gate_proj, r = σ(z_a), i = σ(z_x),
  *   log a_t = r·c·log σ(Λ), it writes the recurrence coefficients d = 1 − a_t and
- *   b_t = √(1 − a_t²)·i·u_t (so that h_t = (1 − d)·h_{t−1} + b_t) as IEEE fp16 in the
- *   packed layout of z: d in the recurrence-gate places, b in the input-gate places. u is
- *   the bf16 Conv1D output [N_tok][R] (the GEMM's operand; the same u enters b_t).
- *   g is [N_tok][rglru_gate_pitch(R)] fp16, 16-byte aligned. fp16 keeps 11 significant
- *   bits of d, whose relative error multiplies into every carried state; |b_t| must stay
- *   below the fp16 maximum 65504 (|u_t| below it is enough, since √(1 − a_t²)·i ≤ 1).
+ *   b_t = √(1 − a_t²)·i·u_t (so that h_t = (1 − d)·h_{t−1} + b_t) in the packed layout of
+ *   z: d as IEEE fp16 in the recurrence-gate places, b_t as bf16 in the input-gate places.
+ *   u is the bf16 Conv1D output [N_tok][R] (the GEMM's operand; the same u enters b_t).
+ *   g is [N_tok][rglru_gate_pitch(R)] 16-bit words, 16-byte aligned. d ∈ [0, 1] keeps
+ *   fp16's 11 significant bits (its relative error multiplies into every carried state);
+ *   b_t, which scales with u_t, keeps bf16's exponent range, so every finite bf16 u gives
+ *   a finite b_t (|b_t| ≤ |u_t|, since √(1 − a_t²)·i ≤ 1).
  *
  * rglru_scan_coeffs: the chunked recurrence h_t = (1 − d)·h_{t−1} + b_t over those
  *   coefficients, for bf16 IO: y_t = h_t, or h_t ⊙ GeLU(gate_g_t) when gate_g is non-NULL,
@@ -304,22 +372,27 @@ RGLRU_API int rglru_scan_coeffs(const void* g, const float* h0, const void* gate
  * that must not call cudaMalloc (which can synchronise the device). The paper has no
  * counterpart to this entry point; it exists for those callers only.
  *
- * Same arguments and results as rglru_scan, minus the workspace. The scan's scratch
- * (tile ticket, look-back flags, chunk carries) is a fixed 8 MiB array in the library's
- * device memory, which every GPU that loads librglru.so holds until the process exits.
- * Problems needing more (about B·⌈R/128⌉·⌈T/64⌉ > 5400 for bf16, twice that tile count
- * of 64 channels for float32) are rejected with RGLRU_ERR_WORKSPACE before anything is
- * launched. Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ * Same arguments, checks and results as rglru_scan, minus the workspace. The scan's
+ * scratch (status word, tile ticket, published chunk states) is a fixed 8 MiB array in
+ * the library's device memory, which every GPU that loads librglru.so holds until the
+ * process exits. A problem fits if 256 + n_tiles·4·CW ≤ 8 MiB, with
+ * n_tiles = B·⌈R/CW⌉·⌈T/64⌉ and CW = 128 channels for bf16, 64 for float32: at most 16383
+ * bf16 tiles (e.g. B=1, T=32704, R=4096) or 32767 float32 tiles. Larger problems are
+ * rejected with RGLRU_ERR_WORKSPACE before anything is launched. Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library call.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture.
  * All calls on a device share the one array, and it keeps the last call's contents (each
- * call clears the parts that must start at zero): calls that overlap on the GPU — on
- * different streams, or from different threads — race and give wrong results. Timeouts of
- * its bounded waits are reported by rglru_workspace_status(NULL, stream).
+ * call clears the parts that must start at zero, its status word included): calls that
+ * overlap on the GPU — on different streams, or from different threads — race and give
+ * wrong results. A timeout of the call's bounded waits is reported by
+ * rglru_scan_noalloc_status, which synchronises `stream`, reads the array's status word
+ * and clears it (RGLRU_OK or RGLRU_ERR_TIMEOUT); the next call clears it too.
  * --------------------------------------------------------------------------------- */
 RGLRU_API int rglru_scan_noalloc(const rglru_params* params, const void* x, const void* z, const void* conv_state0,
                                  const float* h0, const void* gate_g, void* y, float* h_T, int B, int T, int R,
                                  int io_dtype, rglru_stream_t stream);
+RGLRU_API int rglru_scan_noalloc_status(rglru_stream_t stream);
 
 /* The gate GEMM with the RG-LRU scan fused into its epilogue (Eq. (1)–(4)): y and h_T
  * from x (the Conv1D input, from which u is recomputed in float32) and u = Conv1D(x) in

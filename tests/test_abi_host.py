@@ -265,3 +265,67 @@ def test_layer_binding_takes_cuda_tensors_only():
     with pytest.raises(ValueError):
         rglru.layer_step(p, lw, w.x[:, 0].contiguous(), torch.zeros(1, 3, 24, dtype=torch.bfloat16),
                          torch.zeros(1, 24), 0, workspace=ws, out_t=torch.empty(1, 16, dtype=torch.bfloat16))
+
+
+def test_attention_steps_reject_bad_arguments_before_any_launch():
+    lib = _abi.load()
+    ok_ptr = _fake()
+    B, D, W, Hm = 4, 256, 128, 768
+    wb = lib.rglru_attention_step_workspace_bytes(B, D, W)
+    assert wb > 0
+    assert lib.rglru_attention_step_workspace_bytes(B, 200, W) == 0       # D not a multiple of 128
+    assert lib.rglru_attention_step_workspace_bytes(B, 128 * 129, W) == 0  # more than 128 heads
+    assert lib.rglru_attention_step_workspace_bytes(B, D, 100) == 0       # window not a multiple of 128
+    assert lib.rglru_attention_step_workspace_bytes(0, D, W) == 0
+    f = 0x100000
+    aw = _abi.RGLRUAttentionWeights(f, f)
+    ws = _fake(0x200000)
+
+    def call(**kw):
+        return lib.rglru_attention_step(kw.get("w", ctypes.byref(aw)), kw.get("x", ok_ptr), kw.get("k", ok_ptr),
+                                        kw.get("v", ok_ptr), kw.get("out", ok_ptr), B, kw.get("D", D),
+                                        kw.get("W", W), kw.get("pos", 0), kw.get("ws", ws), kw.get("wsb", wb), None)
+
+    assert call(D=192) == -2
+    assert call(W=192) == -2
+    assert call(pos=-1) == -2
+    assert call(w=None) == -1
+    assert call(k=None) == -1
+    assert call(v=_fake(0x100004)) == -3
+    assert call(ws=None) == -5
+    assert call(wsb=wb - 1) == -5
+    assert call(ws=_fake(0x200010)) == -3
+
+    lwb = lib.rglru_attention_layer_step_workspace_bytes(B, D, Hm, W)
+    assert lwb > wb
+    lw = _abi.RGLRUAttentionLayerWeights(f, f, f, f, f, f, f)
+
+    def lcall(**kw):
+        return lib.rglru_attention_layer_step(kw.get("w", ctypes.byref(lw)), kw.get("x", ok_ptr), ok_ptr, ok_ptr,
+                                              kw.get("out", _fake(0x300000)), B, D, kw.get("H", Hm), W,
+                                              kw.get("pos", 0), kw.get("eps", 1e-6), ws, kw.get("wsb", lwb), None)
+
+    assert lcall(out=ok_ptr) == -2         # out_t == x_t
+    assert lcall(H=12) == -2
+    assert lcall(eps=float("nan")) == -2
+    assert lcall(w=None) == -1
+    assert lcall(wsb=lwb - 1) == -5
+
+
+def test_attention_weights_marshal_in_header_order():
+    hdr = open(HEADER, encoding="utf-8").read()
+    for struct, cls in (("rglru_attention_weights", _abi.RGLRUAttentionWeights),
+                        ("rglru_attention_layer_weights", _abi.RGLRUAttentionLayerWeights)):
+        end = hdr.index("} " + struct + ";")
+        body = hdr[hdr.rindex("typedef struct", 0, end):end]
+        assert re.findall(r"\*\s*(\w+);", body) == [f for f, _ in cls._fields_], struct
+
+
+def test_attention_workspace_sizes_follow_the_documented_layout():
+    lib = _abi.load()
+    r256 = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    for B, D, W in [(1, 128, 128), (3, 256, 128), (256, 4096, 1024)]:
+        H, nc = D // 128, W // 128
+        want = 256 + r256(B * (H + 2) * 128 * 2) + r256(B * H * 128 * 2) + r256(B * nc * H * 128 * 4) + \
+            2 * r256(B * nc * H * 4) + r256(B * H * 128 * 2)
+        assert lib.rglru_attention_step_workspace_bytes(B, D, W) == want

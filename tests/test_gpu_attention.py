@@ -1,0 +1,114 @@
+"""Griffin's local multi-query attention, decode step, on the GPU against the float64 oracle
+(oracle/local_attention.py, pinned in test_oracle_pins_attention.py), every step.
+
+Tolerance: the bf16 path's 2e-2 on the block output (q, k, v, the rotated queries and keys,
+the softmax numerators and o are stored in bf16; scores, sums and accumulations are float32);
+the layer's 3e-2 on the residual layer (the MLP's bf16 roundings on top). The rings are
+compared with the oracle's at bf16 rounding."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_linear_rnn_conv1d_b200 import inputs, rglru
+
+from _util import TOL, TOL_LAYER, f64, rel
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _host(w):
+    return {k: f64(v) for k, v in w.items()}
+
+
+def _rings_to_oracle(k_ring, v_ring):
+    """GPU rings (keys [B][W][128], values [B][128][W]) in the oracle's layout [B][W][128]."""
+    return f64(k_ring), f64(v_ring).transpose(0, 2, 1)
+
+
+# (3, 256, 128, 300): two query heads (the MMA's N padded to 16), a 128-slot window that
+# wraps twice; (2, 640, 256, 270): five heads, two ring chunks, one wrap
+@pytest.mark.parametrize("B,D,W,steps", [(3, 256, 128, 300), (2, 640, 256, 270)])
+def test_attention_step_matches_oracle_every_step(B, D, W, steps):
+    w = inputs.make_attention(D, seed=D + W)
+    aw = rglru.AttentionWeights.from_host(w)
+    hw = _host(w)
+    k_ring, v_ring = rglru.attention_rings(B, W)
+    k_ring.fill_(float("nan"))          # slots not yet written must never be read
+    v_ring.fill_(float("nan"))
+    ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=DEV)
+    K_o, V_o = np.full((B, W, 128), np.nan), np.full((B, W, 128), np.nan)
+    worst = 0.0
+    for t in range(steps):
+        xt = inputs.decode_token(t, B, D)
+        out = rglru.attention_step(aw, xt.to(DEV), k_ring, v_ring, t, workspace=ws)
+        out_o, K_o, V_o = oracle.local_attention_step(xt, K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"], hw["W_o"], W)
+        e = rel(out, out_o)
+        worst = max(worst, e)
+        assert e <= TOL[torch.bfloat16], (t, e)
+    assert rglru.workspace_status(ws) == 0
+    kg, vg = _rings_to_oracle(k_ring, v_ring)
+    assert rel(kg, K_o) <= 1e-2 and rel(vg, V_o) <= 1e-2
+    print(f"attention step B={B} D={D} W={W}: worst step error {worst:.3e}")
+
+
+def test_attention_step_full_window_at_scale():
+    """D = 4096 (32 heads), window 1024, 256 sequences: the rings are filled with seeded
+    keys and values for positions 0 … 1019, then steps 1020 … 1030 cross the ring's wrap;
+    32 seeded rows are compared with the oracle at every step (rows are independent)."""
+    B, D, W = 256, 4096, 1024
+    w = inputs.make_attention(D, seed=5)
+    aw = rglru.AttentionWeights.from_host(w)
+    hw = _host(w)
+    g = torch.Generator("cpu").manual_seed(6)
+    k0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
+    v0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
+    k_ring = k0.to(DEV).contiguous()
+    v_ring = v0.transpose(1, 2).contiguous().to(DEV)
+    rows = np.array(sorted(set([0, B - 1]) | set(np.random.default_rng(7).choice(B, 30, replace=False).tolist())))
+    K_o, V_o = f64(k0)[rows], f64(v0)[rows]
+    ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=DEV)
+    for t in range(1020, 1031):
+        xt = inputs.decode_token(t, B, D)
+        out = rglru.attention_step(aw, xt.to(DEV), k_ring, v_ring, t, workspace=ws)
+        out_o, K_o, V_o = oracle.local_attention_step(f64(xt)[rows], K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"],
+                                                      hw["W_o"], W)
+        assert rel(out[torch.from_numpy(rows).to(DEV)], out_o) <= TOL[torch.bfloat16], t
+    assert rglru.workspace_status(ws) == 0
+
+
+def test_attention_layer_step_matches_oracle_every_step():
+    B, D, W, M, steps = 3, 256, 128, 3, 160
+    w = inputs.make_attention(D, M, seed=11)
+    aw = rglru.AttentionWeights.from_host(w)
+    hw = _host(w)
+    k_ring, v_ring = rglru.attention_rings(B, W)
+    K_o, V_o = np.zeros((B, W, 128)), np.zeros((B, W, 128))
+    ws = torch.full((rglru.attention_layer_step_workspace_bytes(B, D, M * D, W),), 0xFF, dtype=torch.uint8,
+                    device=DEV)
+    for t in range(steps):
+        xt = inputs.decode_token(t, B, D)
+        out = rglru.attention_layer_step(aw, xt.to(DEV), k_ring, v_ring, t, eps=oracle.RMS_EPS, workspace=ws)
+        out_o, K_o, V_o = oracle.griffin_attention_layer_step(
+            xt, K_o, V_o, t, hw["norm1_scale"], hw["W_q"], hw["W_k"], hw["W_v"], hw["W_o"], hw["norm2_scale"],
+            hw["W_gate"], hw["W_up"], hw["W_down"], W)
+        assert rel(out, out_o) <= TOL_LAYER, t
+    assert rglru.workspace_status(ws) == 0
+
+
+def test_attention_steps_are_deterministic_and_resume_bitwise():
+    """The decode state of the attention is (rings, position): copies of it continue bit for
+    bit like the original."""
+    B, D, W = 4, 384, 256
+    w = inputs.make_attention(D, seed=3)
+    aw = rglru.AttentionWeights.from_host(w)
+    k_ring, v_ring = rglru.attention_rings(B, W)
+    toks = [inputs.decode_token(t, B, D).to(DEV) for t in range(300)]
+    for t in range(280):
+        rglru.attention_step(aw, toks[t], k_ring, v_ring, t)
+    k2, v2 = k_ring.clone(), v_ring.clone()
+    ref = [rglru.attention_step(aw, toks[t], k_ring, v_ring, t).clone() for t in range(280, 300)]
+    got = [rglru.attention_step(aw, toks[t], k2, v2, t).clone() for t in range(280, 300)]
+    assert all(torch.equal(a, b) for a, b in zip(ref, got))
+    assert torch.equal(k_ring, k2) and torch.equal(v_ring, v2)
