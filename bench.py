@@ -145,7 +145,7 @@ class Ctx:
         then a 256 MB read of another buffer, so that the lines the write left dirty are
         written back here and not inside the next timed region."""
         self.flush.zero_()
-        self.torch.sum(self.flush_src, out=self.sink)
+        self.torch.sum(self.flush_src, dim=0, out=self.sink)
 
     def barrier(self):
         self.replicas.barrier(self.rk)
@@ -706,7 +706,7 @@ def _oracle_sample(inputs, k=0):
 
 
 CPU_SAMPLE_SECONDS = 10.0
-E2E_GROUPS = 4   # time chunks that forward_host pipelines in the e2e measurement
+E2E_GROUPS = 8   # time chunks that forward_host pipelines in the e2e measurement
 SAMPLE_TEXT = (f"{CPU_STEPS} steps x {CPU_CHANNELS} of {HEADLINE['R']} channels of the B=1 T={HEADLINE['T']} "
                "sequence per sample (Conv1D over all channels), counted as steps x channels / D_RNN tokens; "
                "float64 numpy, BLAS matmul on the host cores, recurrence vectorised over channels")

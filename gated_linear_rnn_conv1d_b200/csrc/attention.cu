@@ -1,11 +1,12 @@
 // Decode step of Griffin's local multi-query attention on the sm_100a tensor cores.
 //
-// "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §时间混合块: MQA (H query
-// heads of D_head = 128, H·D_head = D, one key/value head shared by all of them), RoPE as
-// the relative position embedding, local sliding-window attention (each position sees a
-// fixed number of past positions, which bounds the KV cache by the window); "Griffin's
-// Compromise: Combining Gated Linear Recurrence with Local Attention", §Griffin: window
-// 1024.
+// "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §时间混合块 (全局多查询注意力,
+// 局部滑动窗口注意力): MQA (H query heads of D_head = 128, H·D_head = D, one key/value head
+// shared by all of them), RoPE as the relative position embedding, local sliding-window
+// attention (each position sees a fixed number of past positions, which bounds the KV cache
+// by the window); "Griffin's Compromise: Combining Gated Linear Recurrence with Local
+// Attention", §"Griffin: Attention for Recent Memory, Recurrence for Long-Range Flow":
+// window 1024.
 //
 // One step at position `pos` for B sequences:
 //   attn_prep_kernel   from the fused projection qkv = x W_qkvᵀ: rotates q and k (RoPE,
@@ -42,28 +43,35 @@ namespace {
 
 constexpr int kDh = 128;          // D_head
 constexpr int kChunk = 128;       // ring slots per CTA
-constexpr int kAttnThreads = 128;
+constexpr int kAttnThreads = 192;  // TMA warp, MMA warp, four softmax warps
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Shared memory of the chunk kernel, offsets from a 1024-aligned base (every TMA box and
+// operand tile starts 1024-aligned): two stages of [keys 2 × [128 slots][64 dims] | values
+// 2 × [128 dims][64 slots] | queries 2 × [hp heads][64 dims]], then two buffers of softmax
+// numerators P (2 k-blocks [hp][64 slots] each) and the scores [hp][128] float.
+constexpr int kAttnStages = 2;
+constexpr int kSPitch = kChunk + 4;  // floats per score row: 16-byte row reads stay conflict-free
 struct AttnSmem {
-  // offsets from the 1024-aligned base; every TMA box and operand tile starts 1024-aligned
-  int hp;                       // heads rounded up to 16 (the MMA's N)
-  int off_k, off_v, off_q, off_p, off_s, bytes;
+  int hp;  // heads rounded up to 16 (the MMA's N)
+  int stage, off_k, off_v, off_q, off_p, off_s, bytes;
 };
 __host__ __device__ inline AttnSmem attn_smem(int H) {
   AttnSmem L;
   L.hp = (H + 15) / 16 * 16;
-  L.off_k = 0;                                   // 2 boxes [128 slots][64 dims]
-  L.off_v = L.off_k + 2 * kChunk * 128;          // 2 boxes [128 dims][64 slots]
-  L.off_q = L.off_v + 2 * kDh * 128;             // 2 boxes [hp heads][64 dims]
-  L.off_p = L.off_q + ((2 * L.hp * 128 + 1023) / 1024) * 1024;  // 2 k-blocks [hp][64 slots]
-  L.off_s = L.off_p + ((2 * L.hp * 128 + 1023) / 1024) * 1024;  // scores [hp][128] float
-  L.bytes = L.off_s + L.hp * kChunk * 4;
+  L.off_k = 0;
+  L.off_v = L.off_k + 2 * kChunk * 128;
+  L.off_q = L.off_v + 2 * kDh * 128;
+  L.stage = L.off_q + ((2 * L.hp * 128 + 1023) / 1024) * 1024;
+  L.off_p = kAttnStages * L.stage;  // two P buffers (items alternate)
+  L.off_s = L.off_p + 2 * (((2 * L.hp * 128 + 1023) / 1024) * 1024);
+  L.bytes = L.off_s + L.hp * kSPitch * 4;
   return L;
 }
 
 struct AttnArgs {
   const __nv_bfloat16* qkv;  // [B][(H+2)·128]
+  int n_used;                // ring chunks holding a position of the window (all once it wrapped)
   __nv_bfloat16* q_rot;      // [B][H][128]
   __nv_bfloat16* k_ring;     // [B][W][128]
   __nv_bfloat16* v_ring;     // [B][128][W]
@@ -85,16 +93,24 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(AttnArgs a) {
   const int64_t nq = (int64_t)(H + 2) * kDh;
   const __nv_bfloat16* src = a.qkv + (int64_t)b * nq;
   const int slot = (int)(a.pos % a.W);
+  // the 64 rotation angles of this position (the same for every head and every sequence):
+  // θ_j = 10000^(−2j/128), the angle pos·θ_j reduced modulo 2π in float64 so that large
+  // positions keep their accuracy
+  __shared__ float s_cos[kDh / 2], s_sin[kDh / 2];
+  if (threadIdx.x < kDh / 2) {
+    const int j = threadIdx.x;
+    const double theta = exp(-(double)j * (2.0 / kDh) * 9.210340371976184);  // ln 10000
+    const double ang = fmod((double)a.pos * theta, 6.283185307179586);
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    s_cos[j] = (float)cd;
+    s_sin[j] = (float)sd;
+  }
+  __syncthreads();
   // rotation pairs of the H query heads and the key: (H + 1) · 64 of them
   for (int i = threadIdx.x; i < (H + 1) * (kDh / 2); i += blockDim.x) {
     const int head = i / (kDh / 2), j = i % (kDh / 2);
-    // θ_j = 10000^(−2j/128); the angle pos·θ_j reduced modulo 2π in float64, so that large
-    // positions keep their accuracy
-    const double theta = exp(-(double)j * (2.0 / kDh) * 9.210340371976184);  // ln 10000
-    double ang = fmod((double)a.pos * theta, 6.283185307179586);
-    double sd, cd;
-    sincos(ang, &sd, &cd);
-    const float s = (float)sd, c = (float)cd;
+    const float s = s_sin[j], c = s_cos[j];
     const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(src + head * kDh + 2 * j);
     const float x0 = __bfloat162float(v.x), x1 = __bfloat162float(v.y);
     const __nv_bfloat162 r = __floats2bfloat162_rn(x0 * c - x1 * s, x0 * s + x1 * c);
@@ -120,196 +136,272 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
 
 // byte offset of element (row, k) of a K-major bf16 tile stored with the 128-byte swizzle:
 // rows of 64 elements (128 bytes), 16-byte chunks permuted by (row mod 8)
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ uint32_t sw128_offset(int row, int k) {
   return (uint32_t)row * 128u + ((uint32_t)((k >> 3) ^ (row & 7)) << 4) + (uint32_t)(k & 7) * 2u;
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 2)
+// Persistent: one CTA per SM walks the (sequence, chunk) items blockIdx.x, + gridDim.x, …
+// Warp roles: 0 issues the TMA loads of item n into stage n mod 2 (two items ahead of the
+// MMAs, so the next chunk streams in while this one is computed); 1 owns TMEM and issues the
+// two MMAs of each item; 2–5 turn the scores into softmax numerators and write the partial
+// outputs. The softmax warps run one item ahead of their outputs: item n's numerators are
+// handed to the second MMA before item n − 1's output is read, so both MMAs' latency hides
+// behind that work. Sᵀ and the score buffer are single; P and Oᵀ alternate between two
+// buffers. Barriers: full/empty per stage; per item s_full (Sᵀ in TMEM) and p_full (P in
+// shared memory); o_full per Oᵀ buffer. The orders that make the reuse safe:
+//   Sᵀ(n) is written after p_full(n − 1), by which time the scores of n − 1 are read;
+//   Oᵀ(n mod 2) is written after p_full(n), which the softmax warps give only after they
+//   read Oᵀ(n − 2); P(n mod 2) is written after the softmax warps saw o_full(n − 2).
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_chunk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmQ, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t load_bar, mma1_bar, mma2_bar;
+  __shared__ __align__(8) uint64_t full_bar[kAttnStages], empty_bar[kAttnStages], o_full[2];
+  __shared__ __align__(8) uint64_t s_full, p_full, drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const AttnSmem L = attn_smem(a.H);
   const int hp = L.hp;
+  const int p_bytes = ((2 * hp * 128 + 1023) / 1024) * 1024;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int c = blockIdx.x, b = blockIdx.y;
-  const int64_t part = (int64_t)b * a.n_chunks + c;
-  // slots of this chunk that hold a position of the window: all once the ring has wrapped
-  // (pos ≥ W − 1), otherwise slots 0 … pos
-  const int64_t first = (int64_t)c * kChunk;
-  const int n_valid = a.pos >= a.W - 1 ? kChunk : (int)max((int64_t)0, min((int64_t)kChunk, a.pos + 1 - first));
+  const int n_items = a.B * a.n_used;
+  // Sᵀ in columns [0, hp), the two Oᵀ buffers in [hp, 3hp); 32 more so that every 32-column
+  // load of the last group stays inside the allocation
+  const int need = 3 * hp + 32;
+  const uint32_t tmem_cols = need <= 64 ? 64u : (need <= 128 ? 128u : (need <= 256 ? 256u : 512u));
+  static_assert(kAttnMaxHeads <= 64, "two stages, two P buffers and the scores fit in shared memory");
 
-  pdl_wait();  // the ring and the rotated queries are the previous kernel's output
-  pdl_launch_dependents();
-  if (n_valid == 0) {
-    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
-      a.m_part[part * a.H + h] = -INFINITY;
-      a.l_part[part * a.H + h] = 0.0f;
-    }
-    return;
-  }
   if (threadIdx.x == 0) {
-    mbar_init(&load_bar, 1);
-    mbar_init(&mma1_bar, 1);
-    mbar_init(&mma2_bar, 1);
+    for (int i = 0; i < kAttnStages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+      mbar_init(&o_full[i], 1);
+    }
+    mbar_init(&s_full, 1);
+    mbar_init(&p_full, 4);  // one arrival per softmax warp
+    mbar_init(&drain_bar, 1);
     abort_s = 0;
     fence_barrier_init();
   }
-  // Sᵀ in columns [0, hp), Oᵀ in [hp, 2hp); 32 more so that every 32-column load of the
-  // last group stays inside the allocation
-  const int need = 2 * hp + 32;
-  const uint32_t tmem_cols = need <= 64 ? 64u : (need <= 128 ? 128u : (need <= 256 ? 256u : 512u));
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(&tmem_base_s, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // the rings and the rotated queries are the previous kernel's output
+  pdl_launch_dependents();
   const uint32_t tmem = tmem_base_s;
-  uint8_t* sK = smem + L.off_k;
-  uint8_t* sV = smem + L.off_v;
-  uint8_t* sQ = smem + L.off_q;
-  uint8_t* sP = smem + L.off_p;
-  float* sS = reinterpret_cast<float*>(smem + L.off_s);
   const uint32_t idesc = umma_idesc_bf16_f32(128, hp);
-  static_assert(kAttnMaxHeads <= 128, "the N of both MMAs, and 2·N + 32 TMEM columns, stay in range");
-  bool ok = true;
 
-  if (threadIdx.x == 0) {
-    const uint32_t bytes = 2 * kChunk * 128 + 2 * kDh * 128 + 2 * hp * 128;
-    mbar_arrive_expect_tx(&load_bar, bytes);
-    for (int kb = 0; kb < 2; ++kb) {
-      tma_load_3d(sK + kb * kChunk * 128, &tmK, &load_bar, kb * 64, (int)first, b);  // keys, dims kb·64…
-      tma_load_3d(sV + kb * kDh * 128, &tmV, &load_bar, (int)first + kb * 64, 0, b);  // values, slots …
-      tma_load_3d(sQ + kb * hp * 128, &tmQ, &load_bar, kb * 64, 0, b);               // queries (rows ≥ H: 0)
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmQ);
+      const uint32_t bytes = 2 * kChunk * 128 + 2 * kDh * 128 + 2 * hp * 128;
+      int n = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
+        const int st = n % kAttnStages;
+        if (n >= kAttnStages && !mbar_wait(&empty_bar[st], (uint32_t)((n / kAttnStages) - 1) & 1u, &abort_s)) {
+          abort_s = 1;
+          atomicOr(a.status, kStatusTimeout);
+          break;
+        }
+        const int b = item / a.n_used, c = item % a.n_used;
+        uint8_t* stage = smem + st * L.stage;
+        mbar_arrive_expect_tx(&full_bar[st], bytes);
+        for (int kb = 0; kb < 2; ++kb) {
+          tma_load_3d(stage + L.off_k + kb * kChunk * 128, &tmK, &full_bar[st], kb * 64, c * kChunk, b);
+          tma_load_3d(stage + L.off_v + kb * kDh * 128, &tmV, &full_bar[st], c * kChunk + kb * 64, 0, b);
+          tma_load_3d(stage + L.off_q + kb * hp * 128, &tmQ, &full_bar[st], kb * 64, 0, b);  // rows ≥ H: 0
+        }
+      }
     }
-    if (!mbar_wait(&load_bar, 0, &abort_s)) ok = false;
-    if (ok) {
-      tc_fence_after();
-      // Sᵀ[slot][head] = Σ_d K[slot][d] Q[head][d]
-      for (int kb = 0; kb < 2; ++kb)
-        for (int k = 0; k < 4; ++k)
-          umma_f16(tmem, umma_desc_sw128(smem_u32(sK + kb * kChunk * 128) + k * 32),
-                   umma_desc_sw128(smem_u32(sQ + kb * hp * 128) + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
-      umma_commit(&mma1_bar);
-    } else {
-      abort_s = 1;
-      atomicOr(a.status, kStatusTimeout);
-    }
-  }
-  // scores → shared memory as sS[head][slot], scaled to log2 units; unwritten slots −inf
-  const float scale = kLog2e * rsqrtf((float)kDh);
-  if (mbar_wait(&mma1_bar, 0, &abort_s)) {
-    tc_fence_after();
-    const int slot = warp * 32 + lane;
-    for (int h0 = 0; h0 < hp; h0 += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)h0, r);
-      tmem_ld_wait();
-      const int nh = min(32, hp - h0);
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < nh) sS[(h0 + j) * kChunk + slot] = slot < n_valid ? __uint_as_float(r[j]) * scale : -INFINITY;
-    }
-    // slots that hold no position yet may hold anything (NaN included): their values are
-    // zeroed so that the second product, where their weight is 0, stays finite
-    if (n_valid < kChunk) {
-      const int d = warp * 32 + lane;  // one row of Vᵀ per thread
-      for (int k = n_valid; k < kChunk; ++k)
-        *reinterpret_cast<__nv_bfloat16*>(sV + (k >> 6) * kDh * 128 + sw128_offset(d, k & 63)) =
-            __float2bfloat16_rn(0.0f);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int n = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
+        const int st = n % kAttnStages;
+        const uint8_t* stage = smem + st * L.stage;
+        if (!mbar_wait(&full_bar[st], (uint32_t)(n / kAttnStages) & 1u, &abort_s)) break;
+        tc_fence_after();
+        // Sᵀ[slot][head] = Σ_d K[slot][d] Q[head][d]
+        for (int kb = 0; kb < 2; ++kb)
+          for (int k = 0; k < 4; ++k)
+            umma_f16(tmem, umma_desc_sw128(smem_u32(stage + L.off_k + kb * kChunk * 128) + k * 32),
+                     umma_desc_sw128(smem_u32(stage + L.off_q + kb * hp * 128) + k * 32), idesc,
+                     (kb | k) != 0 ? 1u : 0u);
+        umma_commit(&s_full);
+        if (!mbar_wait(&p_full, (uint32_t)n & 1u, &abort_s)) break;
+        tc_fence_after();
+        // Oᵀ[dim][head] = Σ_slot Vᵀ[dim][slot] P[head][slot], into buffer n mod 2
+        const uint8_t* pbuf = smem + L.off_p + (n & 1) * p_bytes;
+        for (int kb = 0; kb < 2; ++kb)
+          for (int k = 0; k < 4; ++k)
+            umma_f16(tmem + (uint32_t)((1 + (n & 1)) * hp),
+                     umma_desc_sw128(smem_u32(stage + L.off_v + kb * kDh * 128) + k * 32),
+                     umma_desc_sw128(smem_u32(pbuf + kb * hp * 128) + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+        umma_commit(&o_full[n & 1]);
+        umma_commit(&empty_bar[st]);  // the stage's operands are read
+      }
+      umma_commit(&drain_bar);
+      volatile int never = 0;
+      (void)mbar_wait(&drain_bar, 0, &never);
     }
   } else {
-    ok = false;
-    abort_s = 1;
-    if (lane == 0) atomicOr(a.status, kStatusTimeout);
+    // ---------------- softmax and outputs (warps 2–5) ----------------
+    const int w4 = warp - 2;  // heads w4, w4 + 4, … of the softmax
+    const int q4 = warp & 3;  // the TMEM lane quarter this warp may access: 32·(warp mod 4)
+    float* sS = reinterpret_cast<float*>(smem + L.off_s);
+    const float scale = kLog2e * rsqrtf((float)kDh);
+    // the outputs of item `it` (the n-th of this CTA) from Oᵀ buffer n mod 2
+    auto write_outputs = [&](int it, int n) -> bool {
+      if (!mbar_wait(&o_full[n & 1], (uint32_t)(n >> 1) & 1u, &abort_s)) return false;
+      tc_fence_after();
+      const int64_t part = (int64_t)(it / a.n_used) * a.n_chunks + it % a.n_used;
+      const int d = q4 * 32 + lane;
+      for (int h0 = 0; h0 < hp; h0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)((1 + (n & 1)) * hp + h0), r);
+        tmem_ld_wait();
+        const int nh = min(32, a.H - h0);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nh) a.o_part[(part * a.H + h0 + j) * kDh + d] = __uint_as_float(r[j]);
+      }
+      tc_fence_before();
+      return true;
+    };
+    int n = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++n) {
+      const int st = n % kAttnStages;
+      uint8_t* sV = smem + st * L.stage + L.off_v;
+      uint8_t* sP = smem + L.off_p + (n & 1) * p_bytes;
+      const int b = item / a.n_used, c = item % a.n_used;
+      const int64_t part = (int64_t)b * a.n_chunks + c;
+      const int64_t first = (int64_t)c * kChunk;
+      const int n_valid =
+          a.pos >= a.W - 1 ? kChunk : (int)max((int64_t)0, min((int64_t)kChunk, a.pos + 1 - first));
+      if (!mbar_wait(&s_full, (uint32_t)n & 1u, &abort_s)) {
+        if (lane == 0) atomicOr(a.status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      if (n > 0) named_bar_sync(1, 128);  // every warp is done reading the previous scores
+      // scores → sS[head][slot] in log2 units; slots holding no position: −inf
+      const int slot = q4 * 32 + lane;
+      for (int h0 = 0; h0 < hp; h0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)h0, r);
+        tmem_ld_wait();
+        const int nh = min(32, hp - h0);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nh) sS[(h0 + j) * kSPitch + slot] = slot < n_valid ? __uint_as_float(r[j]) * scale : -INFINITY;
+      }
+      // values of slots holding no position may be anything (NaN included): zeroed, so that
+      // the second product, where their weight is 0, stays finite
+      if (n_valid < kChunk) {
+        const int d = q4 * 32 + lane;  // one row of Vᵀ per thread
+        for (int k = n_valid; k < kChunk; ++k)
+          *reinterpret_cast<__nv_bfloat16*>(sV + (k >> 6) * kDh * 128 + sw128_offset(d, k & 63)) =
+              __float2bfloat16_rn(0.0f);
+      }
+      tc_fence_before();
+      named_bar_sync(1, 128);  // the scores of all 128 slots are in sS
+      // softmax numerators: tph threads per head (8, 4 or 2), each over a run of
+      // spt = 128 / tph slots, read as 16-byte rows and written as 16-byte chunks of P. A warp
+      // holds hpw = 32 / tph heads; lane l takes head l mod hpw and run l / hpw, so that the
+      // eight lanes of each 16-byte access phase touch eight rows (no bank conflicts) and a
+      // head's runs meet in shuffles across lanes hpw, 2·hpw, … apart.
+      {
+        const int tph = hp <= 16 ? 8 : (hp <= 32 ? 4 : 2);
+        const int spt = kChunk / tph;
+        const int hpw = 32 / tph;
+        const int h = w4 * hpw + lane % hpw, g = lane / hpw;
+        if (w4 * hpw < hp) {  // whole warps drop out (hp is a multiple of 16 ≥ hpw)
+          const float* row = sS + h * kSPitch + g * spt;
+          float m = -INFINITY;
+          for (int k = 0; k < spt; k += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(row + k);
+            m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+          }
+          for (int off = hpw; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          float l = 0.0f;
+          for (int k = 0; k < spt; k += 8) {
+            const float4 v0 = *reinterpret_cast<const float4*>(row + k);
+            const float4 v1 = *reinterpret_cast<const float4*>(row + k + 4);
+            const float e[8] = {exp2f(v0.x - m), exp2f(v0.y - m), exp2f(v0.z - m), exp2f(v0.w - m),
+                                exp2f(v1.x - m), exp2f(v1.y - m), exp2f(v1.z - m), exp2f(v1.w - m)};  // 2^−inf = 0
+            uint32_t pk[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              pk[q] = pack_bf16x2(e[2 * q], e[2 * q + 1]);
+              l += bf16lo(pk[q]) + bf16hi(pk[q]);  // the sum of the rounded numerators
+            }
+            const int kk = g * spt + k;  // the chunk's first slot
+            *reinterpret_cast<uint4*>(sP + (kk >> 6) * hp * 128 + h * 128 + ((((kk & 63) >> 3) ^ (h & 7)) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          for (int off = hpw; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+          if (g == 0 && h < a.H) {
+            a.m_part[part * a.H + h] = m;
+            a.l_part[part * a.H + h] = l;
+          }
+        }
+      }
+      fence_proxy_async_smem();  // P and the zeroed values are read by the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full);
+      // the previous item's outputs, while this item's second MMA runs
+      if (n > 0 && !write_outputs(item - (int)gridDim.x, n - 1)) {
+        if (lane == 0) atomicOr(a.status, kStatusTimeout);
+        ok = false;
+      }
+    }
+    if (ok && n > 0 && !write_outputs(blockIdx.x + (n - 1) * (int)gridDim.x, n - 1)) {
+      if (lane == 0) atomicOr(a.status, kStatusTimeout);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  // softmax numerators per head: warp w takes heads w, w + 4, …; lane l slots l + 32·i
-  for (int h = warp; h < hp; h += 4) {
-    float s[4];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      s[i] = sS[h * kChunk + lane + 32 * i];
-      m = fmaxf(m, s[i]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    float l = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int k = lane + 32 * i;                   // slot within the chunk
-      const __nv_bfloat16 p = __float2bfloat16_rn(exp2f(s[i] - m));   // exp2(−inf) = 0
-      l += __bfloat162float(p);
-      *reinterpret_cast<__nv_bfloat16*>(sP + (k >> 6) * hp * 128 + sw128_offset(h, k & 63)) = p;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    if (lane == 0 && h < a.H) {
-      a.m_part[part * a.H + h] = m;
-      a.l_part[part * a.H + h] = l;
-    }
-  }
-  fence_proxy_async_smem();  // P is read by the tensor core
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (threadIdx.x == 0 && ok && !abort_s) {
-    // Oᵀ[dim][head] = Σ_slot Vᵀ[dim][slot] P[head][slot]
-    for (int kb = 0; kb < 2; ++kb)
-      for (int k = 0; k < 4; ++k)
-        umma_f16(tmem + (uint32_t)hp, umma_desc_sw128(smem_u32(sV + kb * kDh * 128) + k * 32),
-                 umma_desc_sw128(smem_u32(sP + kb * hp * 128) + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
-    umma_commit(&mma2_bar);
-  }
-  if (ok && mbar_wait(&mma2_bar, 0, &abort_s)) {
-    tc_fence_after();
-    const int d = warp * 32 + lane;
-    for (int h0 = 0; h0 < hp; h0 += 32) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(hp + h0), r);
-      tmem_ld_wait();
-      const int nh = min(32, a.H - h0);
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < nh) a.o_part[(part * a.H + h0 + j) * kDh + d] = __uint_as_float(r[j]);
-    }
-  } else if (lane == 0) {
-    atomicOr(a.status, kStatusTimeout);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
 }
 
 // ---- merge the chunks of each sequence ------------------------------------------------------
+// One CTA per (sequence, head), one thread per dimension: the chunks' maxima and sums are read
+// by every thread (the same addresses), the partial outputs as 512-byte rows. Only the chunks
+// holding a position of the window were computed (every one once the ring has wrapped).
 __global__ void __launch_bounds__(kDh) attn_combine_kernel(AttnArgs a) {
   pdl_wait();
   pdl_launch_dependents();
-  const int b = blockIdx.x, d = threadIdx.x;
-  for (int h = blockIdx.y; h < a.H; h += gridDim.y) {
-    float mx = -INFINITY;
-    for (int c = 0; c < a.n_chunks; ++c) mx = fmaxf(mx, a.m_part[((int64_t)b * a.n_chunks + c) * a.H + h]);
-    float num = 0.0f, den = 0.0f;
-    for (int c = 0; c < a.n_chunks; ++c) {
-      const int64_t part = (int64_t)b * a.n_chunks + c;
-      const float l = a.l_part[part * a.H + h];
-      if (l == 0.0f) continue;  // a chunk with no position of the window
-      const float w = exp2f(a.m_part[part * a.H + h] - mx);
-      num += w * a.o_part[(part * a.H + h) * kDh + d];
-      den += w * l;
-    }
-    a.o[((int64_t)b * a.H + h) * kDh + d] = __float2bfloat16_rn(num / den);
+  const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  const int64_t base = (int64_t)b * a.n_chunks;
+  float mx = -INFINITY;
+  for (int c = 0; c < a.n_used; ++c) mx = fmaxf(mx, a.m_part[(base + c) * a.H + h]);
+  float num = 0.0f, den = 0.0f;
+#pragma unroll 8
+  for (int c = 0; c < a.n_used; ++c) {
+    const int64_t part = base + c;
+    const float l = a.l_part[part * a.H + h];
+    const float w = exp2f(a.m_part[part * a.H + h] - mx);
+    num = fmaf(w, a.o_part[(part * a.H + h) * kDh + d], num);
+    den = fmaf(w, l, den);
   }
+  a.o[((int64_t)b * a.H + h) * kDh + d] = __float2bfloat16_rn(num / den);
 }
 
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
@@ -353,7 +445,8 @@ AttnLayout attn_layout(int B, int D, int W) {
   L.off_m = L.off_op + r256((size_t)B * L.n_chunks * L.H * kDh * 4);
   L.off_l = L.off_m + r256((size_t)B * L.n_chunks * L.H * 4);
   L.off_o = L.off_l + r256((size_t)B * L.n_chunks * L.H * 4);
-  L.bytes = L.off_o + r256((size_t)B * L.H * kDh * 2);
+  L.off_part = L.off_o + r256((size_t)B * L.H * kDh * 2);
+  L.bytes = L.off_part + kSplitPartBytes;
   return L;
 }
 
@@ -375,6 +468,7 @@ cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, i
   a.H = L.H;
   a.W = W;
   a.n_chunks = L.n_chunks;
+  a.n_used = pos >= W - 1 ? L.n_chunks : (int)((pos + kChunk) / kChunk);  // chunks with a position
   CUtensorMap mk, mv, mq;
   if (!make_map_3d(&mk, k_ring, kDh, W, B, kDh * 2, (uint64_t)W * kDh * 2, 64, kChunk)) return cudaErrorInvalidValue;
   if (!make_map_3d(&mv, v_ring, W, kDh, B, (uint64_t)W * 2, (uint64_t)W * kDh * 2, 64, kDh))
@@ -396,10 +490,11 @@ cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, i
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  e = launch_pdl(attn_chunk_kernel, dim3(L.n_chunks, B), dim3(kAttnThreads), smem, s, mk, mv, mq, a);
+  const int items = B * a.n_used;
+  const int grid = items < num_sms() ? items : num_sms();
+  e = launch_pdl(attn_chunk_kernel, dim3(grid), dim3(kAttnThreads), smem, s, mk, mv, mq, a);
   if (e != cudaSuccess) return e;
-  const int hy = L.H < 8 ? L.H : 8;
-  return launch_pdl(attn_combine_kernel, dim3(B, hy), dim3(kDh), 0, s, a);
+  return launch_pdl(attn_combine_kernel, dim3(B, L.H), dim3(kDh), 0, s, a);
 }
 
 }  // namespace rglru

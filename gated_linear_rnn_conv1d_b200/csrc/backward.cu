@@ -37,10 +37,10 @@ __device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float a, float b) {
 // column of channel c's recurrence-gate pre-activation in a packed gate row
 __device__ __forceinline__ int64_t zcol(int c) { return (int64_t)256 * (c / 128) + (c % 128); }
 
-// a_t from z_a (with its bias) and c·log σ(Λ)
+// a_t from z_a (with its bias) and c·log σ(Λ) (fast exponentials: the operands are bf16)
 __device__ __forceinline__ float decay_of(float za, float cla) {
-  const float r = 1.0f / (1.0f + expf(-za));
-  return expf(r * cla);
+  const float r = __fdividef(1.0f, 1.0f + __expf(-za));
+  return __expf(r * cla);
 }
 
 struct BwdDims {
@@ -66,12 +66,22 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_maps_kernel(const __nv_bfloat
     an = make_float2(decay_of(za.x, cl0), decay_of(za.y, cl1));
   }
   float2 p = make_float2(1.0f, 1.0f), q = make_float2(0.0f, 0.0f);
-  for (int t = t1 - 1; t >= t0; --t) {
-    const float2 g = ld_bf2(dyb + (int64_t)t * d.R);
-    p = make_float2(an.x * p.x, an.y * p.y);
-    q = make_float2(fmaf(an.x, q.x, g.x), fmaf(an.y, q.y, g.y));
-    const float2 za = ld_bf2(zb + (int64_t)t * d.pitch);
-    an = make_float2(decay_of(za.x, cl0), decay_of(za.y, cl1));
+  // eight steps at a time, their loads issued together ahead of the chain
+  for (int tb = t1 - 1; tb >= t0; tb -= 8) {
+    float2 gv[8], zv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int t = tb - j;
+      gv[j] = t >= t0 ? ld_bf2(dyb + (int64_t)t * d.R) : make_float2(0.f, 0.f);
+      zv[j] = t >= t0 ? ld_bf2(zb + (int64_t)t * d.pitch) : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (tb - j < t0) break;
+      p = make_float2(an.x * p.x, an.y * p.y);
+      q = make_float2(fmaf(an.x, q.x, gv[j].x), fmaf(an.y, q.y, gv[j].y));
+      an = make_float2(decay_of(zv[j].x, cl0), decay_of(zv[j].y, cl1));
+    }
   }
   const int64_t o = ((int64_t)b * d.n_chunks + chunk) * d.R + c;
   *reinterpret_cast<float2*>(P + o) = p;
@@ -105,6 +115,9 @@ struct BwdGradArgs {
   const float* Lambda;      // [R]
   const float* gin;         // [B][n_chunks][R]
   __nv_bfloat16* dz;        // [B·T][2R]: ∂z_a in columns [0, R), ∂z_x in [R, 2R)
+  __nv_bfloat16* dzt;       // [2R][n_pad]: ∂zᵀ (the weight-gradient GEMMs' A operand)
+  __nv_bfloat16* ut;        // [R][n_pad]: uᵀ (their B operand)
+  int64_t n_pad;
   float* du;                // [B][T][R] the direct term ∂ℓ/∂u_t ⊃ g m i
   float* dLsum;             // [R] Σ ∂log a·r·c (atomic)
   float* db_a;              // [R] (atomic)
@@ -112,7 +125,27 @@ struct BwdGradArgs {
   float* dh0;               // [B][R] or null
 };
 
-// Pass 3: each chunk replays its steps from the g entering it, with the gate gradients.
+// Pass 3: each chunk replays its steps from the g entering it, with the gate gradients. Steps
+// go in blocks of eight aligned to multiples of 8 (their loads issued together ahead of the
+// chain); besides ∂z (row-major, for the ∂u GEMM) the block's ∂z and u values of the thread's
+// channels are written transposed — ∂zᵀ and uᵀ, the weight-gradient GEMMs' K-major operands
+// along the tokens — as one 16-byte store per row when the block is whole and aligned.
+__device__ __forceinline__ void st_t8(__nv_bfloat16* row, int64_t col0, const uint32_t (&w)[4], int j_lo, int j_hi,
+                                      bool vec) {
+  if (vec) {
+    *reinterpret_cast<uint4*>(row + col0) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    for (int j = j_lo; j <= j_hi; ++j) {
+      const uint32_t v = w[j >> 1];
+      reinterpret_cast<uint16_t*>(row)[col0 + j] = (uint16_t)((j & 1) ? (v >> 16) : (v & 0xFFFFu));
+    }
+  }
+}
+__device__ __forceinline__ void put_bf16(uint32_t (&w)[4], int j, float v) {
+  const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+  w[j >> 1] = (j & 1) ? ((w[j >> 1] & 0x0000FFFFu) | (h << 16)) : ((w[j >> 1] & 0xFFFF0000u) | h);
+}
+
 __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, BwdDims d) {
   const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
   if (c >= d.R) return;
@@ -133,42 +166,73 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
       an[1] = decay_of(za.y, cl[1]);
     }
   }
+  const float2 h0v =
+      a.h0 != nullptr ? *reinterpret_cast<const float2*>(a.h0 + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
+  // rows of the transposed outputs: ∂z_a of c, c+1; ∂z_x of c, c+1; u of c, c+1
+  __nv_bfloat16* trow[6] = {a.dzt + (int64_t)c * a.n_pad, a.dzt + (int64_t)(c + 1) * a.n_pad,
+                            a.dzt + (int64_t)(d.R + c) * a.n_pad, a.dzt + (int64_t)(d.R + c + 1) * a.n_pad,
+                            a.ut + (int64_t)c * a.n_pad, a.ut + (int64_t)(c + 1) * a.n_pad};
+  const bool aligned_rows = (d.T % 8) == 0;  // then row0 + 8k is a multiple of 8
   float sL[2] = {0.f, 0.f}, sa[2] = {0.f, 0.f}, sx[2] = {0.f, 0.f};
-  for (int t = t1 - 1; t >= t0; --t) {
-    const int64_t e = (row0 + t) * d.R + c;
-    const float2 dy2 = ld_bf2(a.dy + e), u2 = ld_bf2(a.u + e);
-    const float2 za2 = ld_bf2(zb + (int64_t)t * d.pitch), zx2 = ld_bf2(zb + (int64_t)t * d.pitch + 128);
-    float2 hp2;
-    if (t > 0) hp2 = ld_bf2(a.y + e - d.R);
-    else hp2 = a.h0 != nullptr ? *reinterpret_cast<const float2*>(a.h0 + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
-    const float dyv[2] = {dy2.x, dy2.y}, uv[2] = {u2.x, u2.y}, zav[2] = {za2.x, za2.y}, zxv[2] = {zx2.x, zx2.y},
-                hpv[2] = {hp2.x, hp2.y};
-    float dza[2], dzx[2], dud[2];
+  for (int tb = (t1 - 1) & ~7; tb >= t0; tb -= 8) {
+    // steps tb … tb + 7 of this chunk (those < t1), replayed from the last to the first
+    const int j_hi = min(7, t1 - 1 - tb);
+    float2 dyv[8], uv[8], zav[8], zxv[8], hpv[8];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float g = fmaf(an[j], gn[j], dyv[j]);
-      const float r = 1.0f / (1.0f + expf(-zav[j]));
-      const float i = 1.0f / (1.0f + expf(-zxv[j]));
-      const float la = r * cl[j];
-      const float at = expf(la);
-      const float mt = sqrtf(-expm1f(2.0f * la));
-      const float d_a = g * hpv[j];
-      const float d_m = g * i * uv[j];
-      const float d_i = g * mt * uv[j];
-      dud[j] = g * mt * i;
-      const float r_over_m = mt > 0.0f ? r / mt : 0.0f;
-      const float dlr = d_a * at * r - d_m * at * at * r_over_m;  // ∂log a_t · r_t
-      dza[j] = dlr * cl[j] * (1.0f - r);
-      dzx[j] = d_i * i * (1.0f - i);
-      sL[j] = fmaf(dlr, kDecayC, sL[j]);
-      sa[j] += dza[j];
-      sx[j] += dzx[j];
-      gn[j] = g;
-      an[j] = at;
+    for (int j = 0; j < 8; ++j) {
+      const int t = tb + j;
+      if (j <= j_hi) {
+        const int64_t e = (row0 + t) * d.R + c;
+        dyv[j] = ld_bf2(a.dy + e);
+        uv[j] = ld_bf2(a.u + e);
+        zav[j] = ld_bf2(zb + (int64_t)t * d.pitch);
+        zxv[j] = ld_bf2(zb + (int64_t)t * d.pitch + 128);
+        hpv[j] = t > 0 ? ld_bf2(a.y + e - d.R) : h0v;
+      }
     }
-    st_bf2(a.dz + (row0 + t) * 2 * d.R + c, dza[0], dza[1]);
-    st_bf2(a.dz + (row0 + t) * 2 * d.R + d.R + c, dzx[0], dzx[1]);
-    *reinterpret_cast<float2*>(a.du + e) = make_float2(dud[0], dud[1]);
+    uint32_t tw[6][4] = {};
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+      if (j > j_hi) continue;
+      const int t = tb + j;
+      const float dy_[2] = {dyv[j].x, dyv[j].y}, u_[2] = {uv[j].x, uv[j].y}, za_[2] = {zav[j].x, zav[j].y},
+                  zx_[2] = {zxv[j].x, zxv[j].y}, hp_[2] = {hpv[j].x, hpv[j].y};
+      float dza[2], dzx[2], dud[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float g = fmaf(an[k], gn[k], dy_[k]);
+        const float r = __fdividef(1.0f, 1.0f + __expf(-za_[k]));
+        const float i = __fdividef(1.0f, 1.0f + __expf(-zx_[k]));
+        const float la = r * cl[k];
+        const float at = __expf(la);
+        const float mt = sqrtf(-expm1f(2.0f * la));
+        const float d_a = g * hp_[k];
+        const float d_m = g * i * u_[k];
+        const float d_i = g * mt * u_[k];
+        dud[k] = g * mt * i;
+        const float r_over_m = mt > 0.0f ? __fdividef(r, mt) : 0.0f;
+        const float dlr = d_a * at * r - d_m * at * at * r_over_m;  // ∂log a_t · r_t
+        dza[k] = dlr * cl[k] * (1.0f - r);
+        dzx[k] = d_i * i * (1.0f - i);
+        sL[k] = fmaf(dlr, kDecayC, sL[k]);
+        sa[k] += dza[k];
+        sx[k] += dzx[k];
+        gn[k] = g;
+        an[k] = at;
+      }
+      st_bf2(a.dz + (row0 + t) * 2 * d.R + c, dza[0], dza[1]);
+      st_bf2(a.dz + (row0 + t) * 2 * d.R + d.R + c, dzx[0], dzx[1]);
+      *reinterpret_cast<float2*>(a.du + (row0 + t) * d.R + c) = make_float2(dud[0], dud[1]);
+      put_bf16(tw[0], j, dza[0]);
+      put_bf16(tw[1], j, dza[1]);
+      put_bf16(tw[2], j, dzx[0]);
+      put_bf16(tw[3], j, dzx[1]);
+      put_bf16(tw[4], j, u_[0]);
+      put_bf16(tw[5], j, u_[1]);
+    }
+    const bool vec = aligned_rows && j_hi == 7;
+#pragma unroll
+    for (int r = 0; r < 6; ++r) st_t8(trow[r], row0 + tb, tw[r], 0, j_hi, vec);
   }
   if (chunk == 0 && a.dh0 != nullptr)  // the gradient reaching h_{−1} = h0
     *reinterpret_cast<float2*>(a.dh0 + (int64_t)b * d.R + c) = make_float2(an[0] * gn[0], an[1] * gn[1]);
@@ -375,7 +439,16 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   bwd_carries_kernel<<<g_rows, kBwdThreads, 0, s>>>(P, Q, g.dh_T, gin, d);
   BwdGradArgs ga{static_cast<const __nv_bfloat16*>(z), static_cast<const __nv_bfloat16*>(u),
                  static_cast<const __nv_bfloat16*>(g.y), static_cast<const __nv_bfloat16*>(g.dy), g.h0, g.Lambda, gin,
-                 dz, du, dLsum, g.db_a, g.db_x, g.dh0};
+                 dz, dzt, ut, L.n_pad, du, dLsum, g.db_a, g.db_x, g.dh0};
+  // the tokens n … n_pad − 1 of the transposed operands are zero (K padding of the ∂W GEMMs)
+  if (L.n_pad > n) {
+    if ((e = cudaMemset2DAsync(dzt + n, (size_t)L.n_pad * 2, 0, (size_t)(L.n_pad - n) * 2, (size_t)2 * R, s)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaMemset2DAsync(ut + n, (size_t)L.n_pad * 2, 0, (size_t)(L.n_pad - n) * 2, (size_t)R, s)) !=
+        cudaSuccess)
+      return e;
+  }
   bwd_grads_kernel<<<g_chunks, kBwdThreads, 0, s>>>(ga, d);
   bwd_lambda_kernel<<<(R + 255) / 256, 256, 0, s>>>(dLsum, g.Lambda, g.dLambda, R);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -384,9 +457,8 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   if ((e = transpose_bf16(g.W_x, wt + R, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
   // (in float32: this term reaches ∂x through the Conv1D backward without another rounding)
   if ((e = launch_gemm_f32out(dz, wt, dug, n, R, 2 * R, R, status, s)) != cudaSuccess) return e;
-  // ∂W_a = ∂z_aᵀ u, ∂W_x = ∂z_xᵀ u over the tokens (K = tokens, zero-padded to n_pad)
-  if ((e = transpose_bf16(dz, dzt, n, 2 * R, 2 * R, L.n_pad, L.n_pad, s)) != cudaSuccess) return e;
-  if ((e = transpose_bf16(u, ut, n, R, R, L.n_pad, L.n_pad, s)) != cudaSuccess) return e;
+  // ∂W_a = ∂z_aᵀ u, ∂W_x = ∂z_xᵀ u over the tokens (K = tokens, zero-padded to n_pad; the
+  // transposed operands come straight from the gradient pass)
   if ((e = launch_gemm_f32out(dzt, ut, g.dW_a, R, R, (int)L.n_pad, R, status, s)) != cudaSuccess) return e;
   if ((e = launch_gemm_f32out(dzt + (int64_t)R * L.n_pad, ut, g.dW_x, R, R, (int)L.n_pad, R, status, s)) !=
       cudaSuccess)

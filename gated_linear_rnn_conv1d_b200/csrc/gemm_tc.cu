@@ -61,7 +61,22 @@ struct EpiArgs {
   uint64_t* carry_agg;          // [B·n_nb·n_chunks][128] aggregates (zero at launch)
   uint32_t* carry_incl;         // [B·n_nb·n_chunks][128] inclusive states (zero at launch)
   int T, n_chunks;              // n_chunks = T / 128
+  // STORE_F32 split over K: tile index = output tile · k_split + slice; slice s covers k-blocks
+  // [s·kb_per, (s+1)·kb_per) and writes its partial sums at Cf + s·split_stride
+  int k_split, kb_per;
+  int64_t split_stride;
 };
+
+// The k-block range of slice `ks` (the whole K when the GEMM is not split).
+__device__ __forceinline__ void kb_range(const EpiArgs& ep, int ks, int k_blocks, int& kb0, int& kb1) {
+  if (ep.k_split > 1) {
+    kb0 = ks * ep.kb_per;
+    kb1 = min(k_blocks, kb0 + ep.kb_per);
+  } else {
+    kb0 = 0;
+    kb1 = k_blocks;
+  }
+}
 
 template <int BN> struct GemmCfg {
   static constexpr int kStages = BN == 256 ? 4 : 6;
@@ -519,9 +534,13 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
-        const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+        const int ksp = ep.k_split > 1 ? ep.k_split : 1;
+        const int tt = tile / ksp;
+        const int m_pair = tt / n_tiles_n, n_blk = tt % n_tiles_n;
         const int arow = m_pair * 256 + (int)rank * 128;
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        int kb0, kb1;
+        kb_range(ep, tile % ksp, k_blocks, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_s)) { ok = false; break; }
           uint8_t* sa = smem + stage * k2StageBytes;
           uint8_t* sb = sa + k2ABytes;
@@ -550,7 +569,9 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, &abort_s)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        int kb0, kb1;
+        kb_range(ep, tile % (ep.k_split > 1 ? ep.k_split : 1), k_blocks, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_s)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * k2StageBytes);
@@ -558,7 +579,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_f16_2sm(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), k2Idesc,
-                         (kb | k) != 0 ? 1u : 0u);
+                         (kb != kb0 || k != 0) ? 1u : 0u);
           umma_commit_2sm_both(&empty_bar[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -581,7 +602,10 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cluster; tile < num_tiles; tile += n_clusters) {
-      const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+      const int ksp = ep.k_split > 1 ? ep.k_split : 1;
+      const int tt = tile / ksp;
+      const int m_pair = tt / n_tiles_n, n_blk = tt % n_tiles_n;
+      [[maybe_unused]] const int64_t split_off = (int64_t)(tile % ksp) * ep.split_stride;
       const int64_t row = (int64_t)m_pair * 256 + rank * 128 + row_in_tile;
       const bool row_ok = row < M;
       // COEF: this thread's 64 values of u_t (its row, its half of the tile's channels),
@@ -683,7 +707,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           // float32 rows (N a multiple of 4): eight 16-byte stores per 32 columns
           const int gcol = n_blk * BN + col0;
           if (row_ok) {
-            float4* d = reinterpret_cast<float4*>(ep.Cf + row * ep.ldc + gcol);
+            float4* d = reinterpret_cast<float4*>(ep.Cf + split_off + row * ep.ldc + gcol);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               if (gcol + 4 * q < ep.N)
@@ -1200,7 +1224,7 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
     attr_set[dev] = true;
   }
   const int64_t m_pairs = (M + 255) / 256;
-  const int64_t tiles = m_pairs * n_tiles_n;
+  const int64_t tiles = m_pairs * n_tiles_n * (ep.k_split > 1 ? ep.k_split : 1);
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
   const int clusters = (int)std::min<int64_t>(tiles, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
@@ -1383,6 +1407,74 @@ cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t 
   ep.N = N;
   const int n_tiles_n = (N + 255) / 256;
   return launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+}
+
+namespace {
+// out[m][0 … N) = bf16(Σ_s part[s][m][·]) for partial sums part [S][M][N] float32, N % 8 == 0.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, int S, int64_t M, int N,
+                                                          int64_t ldc, __nv_bfloat16* __restrict__ out) {
+  pdl_wait();  // the partial sums are the GEMM's output
+  pdl_launch_dependents();
+  const int64_t n8 = N / 8;
+  const int64_t total = M * n8;
+  const int64_t stride = M * (int64_t)N;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = i / n8, c = (i - m * n8) * 8;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int sl = 0; sl < S; ++sl) {
+      const float4* p = reinterpret_cast<const float4*>(part + sl * stride + m * N + c);
+      const float4 a = __ldcs(p), b = __ldcs(p + 1);
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+      v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    *reinterpret_cast<uint4*>(out + m * ldc + c) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+  }
+}
+}  // namespace
+
+cudaError_t launch_gemm_bf16_skinny(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
+                                    float* part, size_t part_bytes, unsigned* status, cudaStream_t s) {
+  // Few output tiles (M = a decode batch): split K so that about every SM pair works, each
+  // slice writing float32 partial sums, then sum the slices into bf16.
+  const int64_t m_pairs = (M + 255) / 256;
+  const int n_tiles_n = (N + 255) / 256;
+  const int k_blocks = (K + BK - 1) / BK;
+  const int64_t tiles = m_pairs * n_tiles_n;
+  const int clusters = num_sms() / 2;
+  int ksp = 1;
+  if (part != nullptr && tiles * 2 <= clusters && N % 8 == 0) {
+    ksp = (int)std::min<int64_t>(clusters / tiles, k_blocks / 4);  // at least 4 k-blocks a slice
+    while (ksp > 1 && (size_t)ksp * M * N * 4 > part_bytes) --ksp;
+  }
+  if (ksp <= 1) return launch_gemm_bf16(A, Bm, C, M, N, K, ldc, status, s);
+  const int kb_per = (k_blocks + ksp - 1) / ksp;
+  ksp = (k_blocks + kb_per - 1) / kb_per;  // no empty slice
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, A, K, M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, 128)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.Cf = part;
+  ep.ldc = N;
+  ep.N = N;
+  ep.k_split = ksp;
+  ep.kb_per = kb_per;
+  ep.split_stride = M * (int64_t)N;
+  cudaError_t e = launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+  if (e != cudaSuccess) return e;
+  const int64_t work = M * (N / 8);
+  const int blocks = (int)std::min<int64_t>((work + 255) / 256, (int64_t)num_sms() * 8);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, (const float*)part, ksp, M, N, ldc,
+                            static_cast<__nv_bfloat16*>(C));
 }
 
 namespace {

@@ -18,9 +18,9 @@ inline int scan_cw(bool bf16) { return bf16 ? 128 : 64; }  // channels per tile
 struct ScanLayout {
   int n_cblk, n_chunks;
   int64_t n_tiles;
-  // workspace: [status u32 | ticket u32 | pad to 256 B][inclusive states: n_tiles × CW × u32];
-  // all of it must be zero at launch
-  size_t off_incl, bytes, zero_bytes;
+  // workspace: [status u32 | ticket u32 | pad to 256 B][inclusive states: n_tiles × CW × u32]
+  // [aggregates: n_tiles × CW × u64]; all of it must be zero at launch
+  size_t off_incl, off_agg, bytes, zero_bytes;
 };
 ScanLayout scan_layout(int B, int T, int R, bool bf16);
 
@@ -44,6 +44,7 @@ struct ScanArgs {
   unsigned* status;     // device status word
   unsigned* ticket;     // tile ticket counter (zero at launch)
   uint32_t* carry_incl; // [n_tiles][CW] published inclusive states (zero at launch)
+  uint64_t* carry_agg;  // [n_tiles][CW] published tile maps (A, B) (zero at launch)
   int B, T, R, n_cblk, n_chunks, n_tiles;
   int64_t pitch;
   int64_t stall_tile;   // testing only: this tile never publishes its carry (-1: none)
@@ -84,6 +85,13 @@ cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* b
                                    void* z, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
                              unsigned* status, cudaStream_t s);
+// launch_gemm_bf16 for few output tiles (M a decode batch): K is split over about every SM
+// pair, the slices' float32 partial sums go to `part` (at most kSplitPartBytes are used)
+// and a second kernel sums them into C. Falls back to launch_gemm_bf16 when the output
+// tiles alone fill the GPU or part is null.
+constexpr size_t kSplitPartBytes = (size_t)80 * 256 * 256 * 4;
+cudaError_t launch_gemm_bf16_skinny(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
+                                    float* part, size_t part_bytes, unsigned* status, cudaStream_t s);
 // C = A·Bᵀ as launch_gemm_bf16 (A [M][K], B [N][K] bf16, K-contiguous), C float32 [M][ldc],
 // N a multiple of 4.
 cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t M, int N, int K, int64_t ldc,
@@ -133,11 +141,11 @@ cudaError_t launch_gelu_mul(const void* gate, const void* up, void* p, int64_t n
 // D_head = 128, H = D / 128 query heads (1 ≤ H ≤ kAttnMaxHeads), one key/value head; the
 // window W a multiple of 128. Workspace: [status word | qkv [B][(H+2)·128] bf16 | rotated
 // queries [B][H][128] bf16 | partial outputs [B][W/128][H][128] f32 | maxima, sums
-// [B][W/128][H] f32 | o [B][H·128] bf16].
-constexpr int kAttnMaxHeads = 128;
+// [B][W/128][H] f32 | o [B][H·128] bf16 | the projections' split-K partial sums].
+constexpr int kAttnMaxHeads = 64;
 struct AttnLayout {
   int H, n_chunks;
-  size_t off_qkv, off_q, off_op, off_m, off_l, off_o, bytes;
+  size_t off_qkv, off_q, off_op, off_m, off_l, off_o, off_part, bytes;
 };
 AttnLayout attn_layout(int B, int D, int W);
 // RoPE and ring writes of position `pos` from qkv (in the workspace), then the windowed

@@ -198,9 +198,13 @@ cudaError_t attention_sequence(const rglru_attention_weights* w, const void* x_t
   unsigned* status = reinterpret_cast<unsigned*>(ws);
   const int nqkv = (L.H + 2) * 128;
   void* qkv = bytes(ws) + L.off_qkv;
-  cudaError_t e = launch_gemm_bf16(x_t, w->W_qkv, qkv, B, nqkv, D, nqkv, status, s);
+  float* part = reinterpret_cast<float*>(bytes(ws) + L.off_part);
+  cudaError_t e =
+      launch_gemm_bf16_skinny(x_t, w->W_qkv, qkv, B, nqkv, D, nqkv, part, kSplitPartBytes, status, s);
   if (e == cudaSuccess) e = launch_attention_core(qkv, k_ring, v_ring, pos, B, D, window, L, ws, status, s);
-  if (e == cudaSuccess) e = launch_gemm_bf16(bytes(ws) + L.off_o, w->W_o, out_t, B, D, L.H * 128, D, status, s);
+  if (e == cudaSuccess)
+    e = launch_gemm_bf16_skinny(bytes(ws) + L.off_o, w->W_o, out_t, B, D, L.H * 128, D, part, kSplitPartBytes,
+                                status, s);
   return e;
 }
 
@@ -278,6 +282,7 @@ cudaError_t block_sequence(const rglru_params* params, const void* W_1, const vo
       a.status = status;
       a.ticket = reinterpret_cast<unsigned*>(bytes(workspace) + 4);
       a.carry_incl = reinterpret_cast<uint32_t*>(bytes(workspace) + L.scan.off_incl);
+      a.carry_agg = reinterpret_cast<uint64_t*>(bytes(workspace) + L.scan.off_agg);
       a.B = B; a.T = T; a.R = R; a.n_cblk = L.scan.n_cblk; a.n_chunks = L.scan.n_chunks;
       a.n_tiles = (int)L.scan.n_tiles; a.pitch = gate_pitch(R);
       e = launch_scan(a, true, s, true);
@@ -314,6 +319,7 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
   a.status = reinterpret_cast<unsigned*>(ws);
   a.ticket = reinterpret_cast<unsigned*>(bytes(ws) + 4);
   a.carry_incl = reinterpret_cast<uint32_t*>(bytes(ws) + sl.off_incl);
+  a.carry_agg = reinterpret_cast<uint64_t*>(bytes(ws) + sl.off_agg);
   a.B = B;
   a.T = T;
   a.R = R;
@@ -326,8 +332,9 @@ cudaError_t run_scan(const rglru_params* p, const void* x, const void* z, int64_
 
 // ---- fixed scratch of rglru_scan_noalloc ---------------------------------------------
 // For callers that cannot allocate device memory, the scan's scratch (status word, tile
-// ticket, published chunk states: the layout scan_layout gives, 256 + 4·CW bytes per tile
-// with CW = 128 channels for bf16 and 64 for float32) lives in this file-scope array, which
+// ticket, published chunk states and chunk maps: the layout scan_layout gives, a 256-byte
+// header and 12·CW bytes per tile with CW = 128 channels for bf16 and 64 for float32) lives
+// in this file-scope array, which
 // every GPU that loads the library holds until the process exits. Its name in host code
 // is a host-side stand-in, not a device address: the address is looked up once per
 // device, with that device current, and handed to the kernels.

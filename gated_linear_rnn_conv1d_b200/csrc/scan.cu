@@ -171,6 +171,23 @@ __device__ __forceinline__ uint32_t enc(float v) {
 }
 __device__ __forceinline__ float dec(uint32_t w) { return __uint_as_float(w ^ kCarryKey); }
 
+// A tile's map h ↦ A·h + B over its 64 steps (its aggregate), published as soon as its
+// phase 1 is done — before its own look-back — as one 64-bit word per channel: enc(A) in the
+// low half (never zero, so zeroed memory reads as "not yet"), the bits of B in the high half.
+__device__ __forceinline__ uint64_t enc_agg(float A, float B) {
+  return (uint64_t)enc(A) | ((uint64_t)__float_as_uint(B) << 32);
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+// predecessors whose words one round of the look-back reads at once
+constexpr int kLookWindow = 8;
+
 struct TileCoord {
   int chunk, b, cblk;  // chunk < 0: no tile (the end of a CTA's sequence)
   int tix;             // carry slot: ((b · n_cblk + cblk) · n_chunks + chunk) < n_tiles
@@ -664,38 +681,98 @@ __device__ __forceinline__ void lookback_begin(const TileCoord& tc, int j, const
 #pragma unroll
   for (int n = 0; n < NCH; ++n) w[n] = ld_relaxed_u32(src + n * kStride);
 }
+// Decoupled look-back. The state entering tile k is the inclusive state of its predecessor
+// chunk k − 1. If that is not published yet, the walk goes back over the predecessors whose
+// aggregates (A, B) are (kLookWindow of them per round trip) to the nearest published
+// inclusive state h_m, then replays forward: h ← fmaf(A_j, h, B_j) for j = m + 1 … k − 1 —
+// the very operation by which tile j forms its own inclusive state from its incoming one,
+// on the same bits. So the state a tile starts from does not depend on which words had been
+// published when it looked (the result is deterministic, whatever the timing), while no tile
+// waits for more than the aggregates of its predecessors. Chunk 0 publishes its inclusive
+// state straight away, so every walk ends; a round that finds neither word of the next
+// predecessor reads it again, within the deadline.
 template <typename T, bool kGate, int NCH>
 __device__ __forceinline__ void lookback_end(const TileCoord& tc, int j, const ScanArgs& a, uint32_t (&w)[NCH],
                                              float (&hin)[NCH]) {
   constexpr int CW = SmemLayout<T, kGate>::CW;
   constexpr int kStride = CW / NCH;
   if (tc.chunk == 0) return;
-  const uint32_t* src = a.carry_incl + (int64_t)(tc.tix - 1) * CW + j;
-  const uint32_t kNothing = enc(0.0f);
+  int depth[NCH];  // > 0: searching (the predecessor depth chunks back is next); ≤ 0: found
+  int rest[NCH];   // once found: the predecessors still to replay are depths rest − 1 … 1
+  bool all = true;
 #pragma unroll
-  for (int n = 0; n < NCH; ++n)
-    if (tc.cblk * CW + j + n * kStride >= a.R) w[n] = kNothing;
-  bool ready = true;
+  for (int n = 0; n < NCH; ++n) {
+    const bool pad = tc.cblk * CW + j + n * kStride >= a.R;  // no state: neither waits nor publishes
+    depth[n] = pad ? 0 : (w[n] != 0u ? -1 : 1);
+    rest[n] = 1;
+    hin[n] = pad ? 0.0f : (w[n] != 0u ? dec(w[n]) : 0.0f);
+    all = all && depth[n] <= 0;
+  }
+  if (all) return;
+  // 1. the nearest published inclusive state, for every channel still searching
+  const long long t0 = clock64();
+  bool timed_out = false;
+  while (true) {
+    all = true;
 #pragma unroll
-  for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
-  if (!ready) {
-    const long long t0 = clock64();
-    while (true) {
+    for (int n = 0; n < NCH; ++n) {
+      if (depth[n] <= 0) continue;
+      const int left = tc.chunk - depth[n] + 1;  // predecessors at this depth or older: chunks 0 … left − 1
+      const int64_t slot0 = (int64_t)(tc.tix - depth[n]) * CW + j + n * kStride;
+      uint32_t wi[kLookWindow];
+      uint64_t ga[kLookWindow];
 #pragma unroll
-      for (int n = 0; n < NCH; ++n)
-        if (w[n] == 0u) w[n] = ld_relaxed_u32(src + n * kStride);  // only channels < R can be 0
-      ready = true;
-#pragma unroll
-      for (int n = 0; n < NCH; ++n) ready = ready && w[n] != 0u;
-      if (ready) break;
-      if (clock64() - t0 > kWaitCycles) {
-        atomicOr(a.status, kStatusTimeout);
-        break;
+      for (int i = 0; i < kLookWindow; ++i) {
+        wi[i] = i < left ? ld_relaxed_u32(a.carry_incl + slot0 - (int64_t)i * CW) : 0u;
+        ga[i] = i < left ? ld_relaxed_u64(a.carry_agg + slot0 - (int64_t)i * CW) : 0ull;
       }
+      const int d_start = depth[n];
+      int found = -1;
+#pragma unroll
+      for (int i = 0; i < kLookWindow; ++i) {
+        if (found < 0 && wi[i] != 0u) found = i;
+        if (found < 0 && ga[i] == 0ull) break;
+        if (found < 0) ++depth[n];
+      }
+      if (found >= 0) {
+        // the inclusive state found, then the window's aggregates in front of it, oldest first
+        uint32_t wf = 0u;
+#pragma unroll
+        for (int i = 0; i < kLookWindow; ++i)
+          if (i == found) wf = wi[i];
+        float h = dec(wf);
+#pragma unroll
+        for (int i = kLookWindow - 1; i >= 0; --i)
+          if (i < found) h = fmaf(dec((uint32_t)ga[i]), h, __uint_as_float((uint32_t)(ga[i] >> 32)));
+        hin[n] = h;
+        rest[n] = d_start;
+        depth[n] = -1;
+      }
+      all = all && depth[n] <= 0;
+    }
+    if (all) break;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(a.status, kStatusTimeout);
+      timed_out = true;
+      break;
     }
   }
+  // 2. replay the predecessors of the earlier windows (depths rest − 1 … 1), oldest first
 #pragma unroll
-  for (int n = 0; n < NCH; ++n) hin[n] = w[n] != 0u ? dec(w[n]) : 0.0f;
+  for (int n = 0; n < NCH; ++n) {
+    if (timed_out && depth[n] > 0) continue;
+    const int64_t ch = j + n * kStride;
+    for (int d0 = rest[n] - 1; d0 >= 1; d0 -= kLookWindow) {
+      uint64_t ga[kLookWindow];
+#pragma unroll
+      for (int i = 0; i < kLookWindow; ++i)
+        ga[i] = d0 - i >= 1 ? ld_relaxed_u64(a.carry_agg + (int64_t)(tc.tix - (d0 - i)) * CW + ch) : 0ull;
+#pragma unroll
+      for (int i = 0; i < kLookWindow; ++i)
+        if (d0 - i >= 1)
+          hin[n] = fmaf(dec((uint32_t)ga[i]), hin[n], __uint_as_float((uint32_t)(ga[i] >> 32)));
+    }
+  }
 }
 
 // Look-back, second half, once phase 1 of the tile is done: composes the S sub-chunk maps
@@ -721,6 +798,15 @@ __device__ __forceinline__ void lookback_finish(const float* __restrict__ mA, fl
       const float pa = mA[q * CW + j + n * kStride], pb = mB[q * CW + j + n * kStride];
       Bv[n] = fmaf(pa, Bv[n], pb);
       A[n] *= pa;
+    }
+  }
+  // the tile's aggregate goes out before its own look-back (chunk 0 needs none: its
+  // inclusive state follows at once)
+  if (publish && tc.chunk > 0) {
+#pragma unroll
+    for (int n = 0; n < NCH; ++n) {
+      const int jj = j + n * kStride;
+      if (tc.cblk * CW + jj < a.R) st_relaxed_u64(a.carry_agg + (int64_t)tc.tix * CW + jj, enc_agg(A[n], Bv[n]));
     }
   }
   lookback_end<T, kGate, NCH>(tc, j, a, w, hin);
@@ -973,7 +1059,8 @@ ScanLayout scan_layout(int B, int T, int R, bool bf16) {
   L.n_chunks = (T + kScanTC - 1) / kScanTC;
   L.n_tiles = (int64_t)B * L.n_cblk * L.n_chunks;
   L.off_incl = 256;
-  L.bytes = L.off_incl + (((size_t)L.n_tiles * cw * 4 + 255) / 256) * 256;
+  L.off_agg = L.off_incl + (((size_t)L.n_tiles * cw * 4 + 255) / 256) * 256;
+  L.bytes = L.off_agg + (size_t)L.n_tiles * cw * 8;
   L.zero_bytes = L.bytes;
   return L;
 }

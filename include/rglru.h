@@ -212,7 +212,8 @@ RGLRU_API int rglru_layer_step(const rglru_params* params, const rglru_layer_wei
  * Griffin's local multi-query attention, one decode step ("Griffin：…", §时间混合块:
  * MQA with H query heads of D_head = 128, H·D_head = D, one key/value head shared by all
  * of them, RoPE as the relative position embedding, sliding-window attention whose KV
- * cache is bounded by the window; "Griffin's Compromise…", §Griffin: window 1024, one
+ * cache is bounded by the window; "Griffin's Compromise…", §"Griffin: Attention for Recent
+ * Memory, Recurrence for Long-Range Flow": window 1024, one
  * local-attention residual block after every two recurrent ones). At position `pos`:
  *   q = x_t W_qᵀ, k = x_t W_kᵀ, v = x_t W_vᵀ;  q, k rotated by RoPE at `pos`
  *   (pair i = (x_{2i}, x_{2i+1}) turned by pos·θ_i, θ_i = 10000^(−2i/128));
@@ -231,7 +232,7 @@ RGLRU_API int rglru_layer_step(const rglru_params* params, const rglru_layer_wei
  *   pos            ≥ 0, the position of x_t; the rings hold positions pos − window … pos − 1
  *   workspace      at least rglru_attention_step_workspace_bytes(B, D, window) bytes,
  *                  256-byte aligned
- * D a multiple of 128 with D/128 ≤ 128; window a multiple of 128 (≤ 65536); B ≤ 65535.
+ * D a multiple of 128 with D/128 ≤ 64; window a multiple of 128 (≤ 65536); B ≤ 65535.
  * Errors as everywhere (RGLRU_ERR_SHAPE for any other D, window, B or pos < 0); a timeout
  * of a bounded wait is reported by rglru_workspace_status(workspace, stream).
  * --------------------------------------------------------------------------------- */
@@ -373,11 +374,12 @@ RGLRU_API int rglru_scan_coeffs(const void* g, const float* h0, const void* gate
  * counterpart to this entry point; it exists for those callers only.
  *
  * Same arguments, checks and results as rglru_scan, minus the workspace. The scan's
- * scratch (status word, tile ticket, published chunk states) is a fixed 8 MiB array in
- * the library's device memory, which every GPU that loads librglru.so holds until the
- * process exits. A problem fits if 256 + n_tiles·4·CW ≤ 8 MiB, with
- * n_tiles = B·⌈R/CW⌉·⌈T/64⌉ and CW = 128 channels for bf16, 64 for float32: at most 16383
- * bf16 tiles (e.g. B=1, T=32704, R=4096) or 32767 float32 tiles. Larger problems are
+ * scratch (status word, tile ticket, published chunk states and chunk maps) is a fixed
+ * 8 MiB array in the library's device memory, which every GPU that loads librglru.so holds
+ * until the process exits. A problem fits if
+ *   256 + ⌈n_tiles·4·CW / 256⌉·256 + n_tiles·8·CW ≤ 8 MiB,
+ * with n_tiles = B·⌈R/CW⌉·⌈T/64⌉ and CW = 128 channels for bf16, 64 for float32: at most
+ * 5461 bf16 tiles (e.g. B=1, T=10880, R=4096) or 10922 float32 tiles. Larger problems are
  * rejected with RGLRU_ERR_WORKSPACE before anything is launched. Nothing is allocated: no
  * cudaMalloc, cudaFree or allocating library call.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress,

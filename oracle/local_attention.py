@@ -11,9 +11,10 @@ The definition, in float64 numpy:
     embedding, rotary position embedding (RoPE, Su et al. 2021) as the relative one;
     local sliding-window attention — each position attends only to a fixed number of past
     positions, which bounds the KV cache by the window; everything else as global MQA.
-  * "Griffin's Compromise: Combining Gated Linear Recurrence with Local Attention", §Griffin:
-    the default window is 1024 tokens, and a local-attention residual block follows every
-    two recurrent residual blocks.
+  * "Griffin's Compromise: Combining Gated Linear Recurrence with Local Attention",
+    §"Griffin: Attention for Recent Memory, Recurrence for Long-Range Flow": the default
+    window is 1024 tokens, and a local-attention residual block follows every two recurrent
+    residual blocks.
 
 Readings where the pages are silent (listed with reasons in the design notes): the window
 W counts the current position, so position t attends to t−W+1 … t; scores are scaled by

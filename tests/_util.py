@@ -12,6 +12,14 @@ TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 # down projection): 5 · 2⁻⁹ ≈ 1e-2. The two allowances add: 3e-2.
 TOL_LAYER = 3e-2
 
+# Tolerance of Griffin's local-attention decode step: its output passes through six bf16
+# storage points between the bf16 input and the bf16 output (q, k and v from the fused
+# projection; the rotated q and k; the softmax numerators; the merged o; the output
+# projection). The float64 oracle with exactly those roundings (rounding_model.attention_step)
+# reaches 2.48e-2 on the GPU test's first case (B=3, D=256, window 128, 300 steps; median
+# 1.4e-2), which is what the GPU measures there too: the same 3e-2 as the layer's.
+TOL_ATTN = 3e-2
+
 
 def f64(t):
     if t is None:

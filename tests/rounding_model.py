@@ -129,3 +129,48 @@ def rms_rel(got, ref):
     """rms(got − ref) / rms(ref): the typical size of a difference, next to the maximum."""
     got, ref = f(got), f(ref)
     return float(np.sqrt(np.mean((got - ref) ** 2)) / np.sqrt(np.mean(ref ** 2)))
+
+
+def attention_step(x_t, K, V, pos, W_qkv, W_o, window, chunk=128):
+    """rglru_attention_step with the path's roundings: qkv = x W_qkvᵀ (bf16), the rotated q and
+    k (bf16; k and v stored in the rings), per 128-slot chunk of the ring the softmax
+    numerators 2^(s − m_c) in bf16 (m_c the chunk's maximum) and their sum l_c, the merged
+    o = Σ_c 2^(m_c − m) O_c / Σ_c 2^(m_c − m) l_c (bf16), out = o W_oᵀ (bf16). K, V [B][W][128]
+    as the oracle holds them (modified in place). Returns out_t."""
+    x_t = f(x_t)
+    B = x_t.shape[0]
+    dh = 128
+    H = (f(W_qkv).shape[0] // dh) - 2
+    qkv = bf16(x_t @ f(W_qkv).T)
+    p = np.array([pos])
+    q = bf16(oracle.rope(qkv[:, :H * dh].reshape(B, H, dh), p))
+    slot = pos % window
+    K[:, slot] = bf16(oracle.rope(qkv[:, None, H * dh:(H + 1) * dh], p)[:, 0])
+    V[:, slot] = qkv[:, (H + 1) * dh:]
+    n_valid = window if pos >= window - 1 else pos + 1
+    s = np.einsum("bhd,bnd->bhn", q, K[:, :n_valid]) / np.sqrt(dh) / np.log(2.0)   # log2 units
+    num = np.zeros((B, H, dh))
+    den = np.zeros((B, H))
+    ms = [s[:, :, c0:c0 + chunk].max(axis=-1) for c0 in range(0, n_valid, chunk)]
+    m = np.max(np.stack(ms), axis=0)
+    for c, c0 in enumerate(range(0, n_valid, chunk)):
+        pc = bf16(np.exp2(s[:, :, c0:c0 + chunk] - ms[c][..., None]))
+        w = np.exp2(ms[c] - m)
+        num += w[..., None] * np.einsum("bhn,bnd->bhd", pc, V[:, c0:min(c0 + chunk, n_valid)])
+        den += w * pc.sum(axis=-1)
+    o = bf16((num / den[..., None]).reshape(B, H * dh))
+    return bf16(o @ f(W_o).T)
+
+
+def attention_layer_step(x_t, K, V, pos, w, window):
+    """rglru_attention_layer_step with the path's roundings (the attention step above on the
+    bf16 RMSNorm output, then the residual adds and the gated MLP as in `layer`). `w` holds
+    W_q, W_k, W_v, W_o, the norm gains and the MLP weights. Returns out_t."""
+    x = f(x_t)
+    W_qkv = np.concatenate([f(w["W_q"]), f(w["W_k"]), f(w["W_v"])], 0)
+    o1 = attention_step(bf16(rms_norm(x, w["norm1_scale"])), K, V, pos, W_qkv, w["W_o"], window)
+    y = bf16(x + o1)
+    n2 = bf16(rms_norm(y, w["norm2_scale"]))
+    gate, up = bf16(n2 @ f(w["W_gate"]).T), bf16(n2 @ f(w["W_up"]).T)
+    o2 = bf16(bf16(oracle.gelu(gate) * up) @ f(w["W_down"]).T)
+    return bf16(y + o2)

@@ -274,7 +274,7 @@ def test_attention_steps_reject_bad_arguments_before_any_launch():
     wb = lib.rglru_attention_step_workspace_bytes(B, D, W)
     assert wb > 0
     assert lib.rglru_attention_step_workspace_bytes(B, 200, W) == 0       # D not a multiple of 128
-    assert lib.rglru_attention_step_workspace_bytes(B, 128 * 129, W) == 0  # more than 128 heads
+    assert lib.rglru_attention_step_workspace_bytes(B, 128 * 65, W) == 0   # more than 64 heads
     assert lib.rglru_attention_step_workspace_bytes(B, D, 100) == 0       # window not a multiple of 128
     assert lib.rglru_attention_step_workspace_bytes(0, D, W) == 0
     f = 0x100000
@@ -327,5 +327,5 @@ def test_attention_workspace_sizes_follow_the_documented_layout():
     for B, D, W in [(1, 128, 128), (3, 256, 128), (256, 4096, 1024)]:
         H, nc = D // 128, W // 128
         want = 256 + r256(B * (H + 2) * 128 * 2) + r256(B * H * 128 * 2) + r256(B * nc * H * 128 * 4) + \
-            2 * r256(B * nc * H * 4) + r256(B * H * 128 * 2)
+            2 * r256(B * nc * H * 4) + r256(B * H * 128 * 2) + 80 * 256 * 256 * 4
         assert lib.rglru_attention_step_workspace_bytes(B, D, W) == want

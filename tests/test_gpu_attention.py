@@ -1,10 +1,12 @@
 """Griffin's local multi-query attention, decode step, on the GPU against the float64 oracle
 (oracle/local_attention.py, pinned in test_oracle_pins_attention.py), every step.
 
-Tolerance: the bf16 path's 2e-2 on the block output (q, k, v, the rotated queries and keys,
-the softmax numerators and o are stored in bf16; scores, sums and accumulations are float32);
-the layer's 3e-2 on the residual layer (the MLP's bf16 roundings on top). The rings are
-compared with the oracle's at bf16 rounding."""
+Tolerance: 3e-2 on the block output (TOL_ATTN: six bf16 storage points — q, k and v, the
+rotated q and k, the softmax numerators, o, the output — put the float64 oracle with those
+roundings alone at 2.5e-2 on the first case); the layer's 3e-2 on the residual layer. The
+GPU is also held to that rounding model at a bound near the last bit: most outputs
+bit-identical, the rest within a few bf16 steps. The rings are compared with the oracle's at
+bf16 rounding."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +14,9 @@ import torch
 import oracle
 from gated_linear_rnn_conv1d_b200 import inputs, rglru
 
-from _util import TOL, TOL_LAYER, f64, rel
+import rounding_model as rm
+
+from _util import TOL, TOL_ATTN, TOL_LAYER, f64, rel
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -28,8 +32,9 @@ def _rings_to_oracle(k_ring, v_ring):
 
 
 # (3, 256, 128, 300): two query heads (the MMA's N padded to 16), a 128-slot window that
-# wraps twice; (2, 640, 256, 270): five heads, two ring chunks, one wrap
-@pytest.mark.parametrize("B,D,W,steps", [(3, 256, 128, 300), (2, 640, 256, 270)])
+# wraps twice; (2, 640, 256, 270): five heads, two ring chunks, one wrap; (5, 1024, 128, 140):
+# eight heads, the projections split over K (16 k-blocks in 4 slices)
+@pytest.mark.parametrize("B,D,W,steps", [(3, 256, 128, 300), (2, 640, 256, 270), (5, 1024, 128, 140)])
 def test_attention_step_matches_oracle_every_step(B, D, W, steps):
     w = inputs.make_attention(D, seed=D + W)
     aw = rglru.AttentionWeights.from_host(w)
@@ -39,18 +44,39 @@ def test_attention_step_matches_oracle_every_step(B, D, W, steps):
     v_ring.fill_(float("nan"))
     ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=DEV)
     K_o, V_o = np.full((B, W, 128), np.nan), np.full((B, W, 128), np.nan)
-    worst = 0.0
+    K_m, V_m = np.zeros((B, W, 128)), np.zeros((B, W, 128))
+    W_qkv = np.concatenate([hw["W_q"], hw["W_k"], hw["W_v"]], 0)
+    worst, worst_m, same, n = 0.0, 0.0, 0, 0
+    sq_gm, sq_mo, sq_m = 0.0, 0.0, 0.0
     for t in range(steps):
         xt = inputs.decode_token(t, B, D)
         out = rglru.attention_step(aw, xt.to(DEV), k_ring, v_ring, t, workspace=ws)
         out_o, K_o, V_o = oracle.local_attention_step(xt, K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"], hw["W_o"], W)
+        out_m = rm.attention_step(xt, K_m, V_m, t, W_qkv, hw["W_o"], W)
         e = rel(out, out_o)
         worst = max(worst, e)
-        assert e <= TOL[torch.bfloat16], (t, e)
+        worst_m = max(worst_m, rel(out, out_m))
+        same += int(np.sum(f64(out) == out_m))
+        n += out_m.size
+        sq_gm += float(np.sum((f64(out) - out_m) ** 2))
+        sq_mo += float(np.sum((out_m - out_o) ** 2))
+        sq_m += float(np.sum(out_m ** 2))
+        assert e <= TOL_ATTN, (t, e)
     assert rglru.workspace_status(ws) == 0
     kg, vg = _rings_to_oracle(k_ring, v_ring)
-    assert rel(kg, K_o) <= 1e-2 and rel(vg, V_o) <= 1e-2
-    print(f"attention step B={B} D={D} W={W}: worst step error {worst:.3e}")
+    # keys: bf16 k from the projection, rotated, rounded again; values: one bf16 rounding
+    assert rel(kg, K_o) <= TOL[torch.bfloat16] and rel(vg, V_o) <= TOL[torch.bfloat16]
+    rms_gm, rms_mo = (sq_gm / sq_m) ** 0.5, (sq_mo / sq_m) ** 0.5
+    print(f"attention step B={B} D={D} W={W}: worst step error {worst:.3e}; against the rounding model "
+          f"{same / n:.4f} identical, worst {worst_m:.3e}, rms {rms_gm:.3e} (the model's own rms error "
+          f"{rms_mo:.3e})")
+    # A rounding that flips upstream (q, k, a numerator, the chunk merge or o) moves out by up
+    # to one bf16 step of o carried through W_o, on top of out's own rounding: 2⁻⁶, as for the
+    # layer. Such flips reach every output of their row, so fewer outputs stay bit-identical
+    # than in the recurrent block (85–97 % on these cases) and the rms of the difference is a
+    # larger part of the model's own distance from the oracle (about a quarter): the bound
+    # asks for at most half of it.
+    assert same / n >= 0.8 and worst_m <= 2.0 ** -6 and rms_gm <= 0.5 * rms_mo
 
 
 def test_attention_step_full_window_at_scale():
@@ -74,7 +100,7 @@ def test_attention_step_full_window_at_scale():
         out = rglru.attention_step(aw, xt.to(DEV), k_ring, v_ring, t, workspace=ws)
         out_o, K_o, V_o = oracle.local_attention_step(f64(xt)[rows], K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"],
                                                       hw["W_o"], W)
-        assert rel(out[torch.from_numpy(rows).to(DEV)], out_o) <= TOL[torch.bfloat16], t
+        assert rel(out[torch.from_numpy(rows).to(DEV)], out_o) <= TOL_ATTN, t
     assert rglru.workspace_status(ws) == 0
 
 

@@ -2,8 +2,8 @@
 hawk_residual_layer_step at every step, and against the layer's own prefill.
 
 Bounds: the layer's 3e-2 on its output (the recurrent block's bf16 allowance plus the
-MLP's five bf16 roundings), 2e-2 on the float32 state h (one RG-LRU decode step per token,
-from bf16 v_t)."""
+MLP's five bf16 roundings) and on the float32 state h (its input v_t = bf16(RMSNorm₁(x_t))
+W_1ᵀ, rounded to bf16 again, carries two roundings the RG-LRU's own 2e-2 does not cover)."""
 import numpy as np
 import pytest
 import torch
@@ -44,7 +44,9 @@ def test_layer_step_matches_oracle_every_step(B, D, R, M, steps):
         e_out, e_h = rel(out, out_o), rel(h, h_o)
         print(f"step {k}: out {e_out:.3e} h {e_h:.3e}")
         assert e_out <= TOL_LAYER, (k, e_out)
-        assert e_h <= TOL[torch.bfloat16], (k, e_h)
+        # the state's input v_t is two bf16 roundings (RMSNorm₁ output, v_t) away from the
+        # oracle's, on top of the RG-LRU's own bf16 allowance: the layer's bound
+        assert e_h <= TOL_LAYER, (k, e_h)
         # the ring holds the bf16 v_t = bf16(RMSNorm₁(x_t)) W_1ᵀ the GPU computed (two bf16
         # roundings); the oracle's are unrounded
         assert rel(ring, ring_o) <= TOL[torch.bfloat16], k

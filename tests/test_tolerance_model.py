@@ -19,7 +19,7 @@ import oracle
 import rounding_model as rm
 from gated_linear_rnn_conv1d_b200 import inputs
 
-from _util import TOL, TOL_LAYER
+from _util import TOL, TOL_ATTN, TOL_LAYER
 
 
 def test_block_storage_rounding_fits_the_bf16_tolerance():
@@ -91,3 +91,21 @@ def test_backward_weight_gradients_storage_rounding_needs_the_wider_bound():
         ea, ex = oracle.max_rel_error(dW_a, ref["dW_a"]), oracle.max_rel_error(dW_x, ref["dW_x"])
         print(f"backward case {(B, T, R)}: storage rounding alone gives dW_a {ea:.4f}, dW_x {ex:.4f}")
         assert TOL[torch.bfloat16] < ea <= 4e-2 and ex <= 4e-2, (ea, ex)
+
+
+def test_attention_storage_rounding_needs_the_attention_bound():
+    # the GPU attention test's first case: B=3, D=256 (two heads), window 128, 300 steps
+    B, D, W, steps = 3, 256, 128, 300
+    w = inputs.make_attention(D, seed=D + W)
+    hw = {k: rm.f(v) for k, v in w.items()}
+    W_qkv = np.concatenate([hw["W_q"], hw["W_k"], hw["W_v"]], 0)
+    K_o, V_o = np.zeros((B, W, 128)), np.zeros((B, W, 128))
+    K_m, V_m = np.zeros((B, W, 128)), np.zeros((B, W, 128))
+    errs = []
+    for t in range(steps):
+        xt = inputs.decode_token(t, B, D)
+        out_o, K_o, V_o = oracle.local_attention_step(xt, K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"], hw["W_o"], W)
+        errs.append(oracle.max_rel_error(rm.attention_step(xt, K_m, V_m, t, W_qkv, hw["W_o"], W), out_o))
+    worst = max(errs)
+    print(f"attention case: storage rounding alone gives {worst:.4e} (median {np.median(errs):.3e})")
+    assert TOL[torch.bfloat16] < worst <= TOL_ATTN, worst

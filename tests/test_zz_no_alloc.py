@@ -28,9 +28,16 @@ def _tiles(B, T, R, dtype):
     return B * -(-R // cw) * -(-T // 64)
 
 
-def _fits(B, T, R, dtype):
+def _bytes(B, T, R, dtype):
+    """The scan's scratch: a 256-byte header, then per tile and channel a 4-byte inclusive
+    state (rounded up to 256 bytes in all) and an 8-byte aggregate."""
     cw = 128 if dtype == torch.bfloat16 else 64
-    return 256 + _tiles(B, T, R, dtype) * 4 * cw <= SCRATCH
+    n = _tiles(B, T, R, dtype)
+    return 256 + -(-n * cw * 4 // 256) * 256 + n * cw * 8
+
+
+def _fits(B, T, R, dtype):
+    return _bytes(B, T, R, dtype) <= SCRATCH
 
 
 def _case(B, T, R, dtype, seed):
@@ -87,19 +94,20 @@ def test_noalloc_scan_matches_workspace_scan_and_oracle_two_calls_in_a_row(dtype
 
 
 def test_noalloc_scan_at_the_largest_problem_its_scratch_holds():
-    # 127 rows × 1 channel block × 129 chunks (the last one ragged) = 16383 bf16 tiles:
-    # 256 + 16383·512 bytes, 256 bytes below 8 MiB, so the last tile's states lie in the top
-    # 512 bytes of the array (8 channels keep the oracle's share of the test small)
-    B, T, R = 127, 129 * 64 - 5, 8
-    assert _tiles(B, T, R, torch.bfloat16) == 16383 and _fits(B, T, R, torch.bfloat16)
+    # 43 rows × 1 channel block × 127 chunks (the last one ragged) = 5461 bf16 tiles:
+    # 256 + 5461·(512 + 1024) bytes, 256 bytes below 8 MiB, so the last tile's aggregates lie
+    # in the top kilobyte of the array (8 channels keep the oracle's share of the test small)
+    B, T, R = 43, 127 * 64 - 5, 8
+    assert _tiles(B, T, R, torch.bfloat16) == 5461 and _bytes(B, T, R, torch.bfloat16) == SCRATCH - 256
     lib = _abi.load()
     _run_and_check(lib, torch.bfloat16, B, T, R, seed=21)
     _run_and_check(lib, torch.bfloat16, 2, 300, 264, seed=22)   # and a small call after it
 
 
 @pytest.mark.parametrize("dtype,B,T,R", [
-    (torch.bfloat16, 1, 32768, 4096),   # 16384 bf16 tiles: 256 bytes more than the array
-    (torch.float32, 1, 32768, 4096),    # 32768 float32 tiles of 64 channels: the same excess
+    (torch.bfloat16, 2, 2731 * 64, 8),   # 5462 bf16 tiles: 1280 bytes more than the array
+    (torch.float32, 3, 3641 * 64, 8),    # 10923 float32 tiles of 64 channels: 512 bytes more
+    (torch.bfloat16, 1, 32768, 4096),    # the long-sequence workload: 16384 tiles
 ])
 def test_noalloc_scan_rejects_problems_beyond_its_scratch(dtype, B, T, R):
     assert not _fits(B, T, R, dtype)
