@@ -588,7 +588,7 @@ def run_layer(c, reps=3):
 def run_backward(c, reps=5):
     """The backward of the forward step (rglru_backward at the forward workload: recompute
     of u and z, the chunked reverse recurrence with the gate gradients, the ∂u and weight
-    gradient GEMMs on transposed copies, the Conv1D backward), L2 flushed before each call."""
+    gradient GEMMs reading ∂z and u in place, the Conv1D backward), L2 flushed before each call."""
     torch, rglru, inputs, dev, stream, flush = c.torch, c.rglru, c.inputs, c.dev, c.stream, c.flush_l2
     max_over_ranks, world = c.max_over_ranks, c.world
     B, T, R = HAWK["B"], HAWK["T"], HAWK["R"]
@@ -634,7 +634,7 @@ def run_attention(c, reps=24):
     aw = rglru.AttentionWeights.from_host(w, dev)
     g = torch.Generator("cpu").manual_seed(1)
     k_ring = torch.randn(B, W, 128, generator=g).to(torch.bfloat16).to(dev)
-    v_ring = torch.randn(B, 128, W, generator=g).to(torch.bfloat16).to(dev)
+    v_ring = torch.randn(B, W, 128, generator=g).to(torch.bfloat16).to(dev)
     toks = torch.stack([inputs.decode_token(k, B, D) for k in range(8)]).to(dev)
     out = torch.empty(B, D, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=dev)
@@ -661,7 +661,7 @@ def run_attention(c, reps=24):
             "ms_per_step": ms, "steps_per_s": c.world / (ms / 1e3), "bytes_per_step": step_bytes,
             "ring_bytes_per_step": ring_bytes, "GB/s": step_bytes / ms / 1e6,
             "frac_hbm": step_bytes / ms / 1e6 / c.pk["hbm_gbs"], "flops_per_step": flops,
-            "status": status, "gpu_launches_per_step": 5,
+            "status": status, "gpu_launches_per_step": 6,  # 2 split-K GEMMs + 2 reduces, prep, chunk
             "timing": f"{reps} single steps at positions past the first window, L2 flushed before each"}
 
 

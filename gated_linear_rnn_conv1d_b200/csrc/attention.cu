@@ -9,28 +9,29 @@
 // window 1024.
 //
 // One step at position `pos` for B sequences:
-//   attn_prep_kernel   from the fused projection qkv = x W_qkvᵀ: rotates q and k (RoPE,
+//   attn_prep_kernel   from the fused projection qkv = x W_qkvᵀ (or its split-K partial sums,
+//                      which it adds up itself): rotates q and k (RoPE,
 //                      pair i = (x_{2i}, x_{2i+1}) turned by pos·θ_i, θ_i = 10000^(−2i/128),
 //                      the angle reduced in float64), writes the rotated queries, the key
 //                      into slot (pos mod W) of the key ring and the value into the same
 //                      slot of the (transposed) value ring;
 //   attn_chunk_kernel  one CTA per (sequence, 128-slot chunk of the ring): TMA brings the
-//                      chunk's keys [128 slots][128], values [128 dims][128 slots] and the
-//                      sequence's queries [H][128] into 128-byte-swizzled shared memory;
+//                      chunk's keys and values [128 slots][128] and the sequence's queries
+//                      [H][128] into 128-byte-swizzled shared memory;
 //                      tcgen05.mma forms Sᵀ = K·Qᵀ (M = 128 slots, N = H heads, fp32 in
 //                      TMEM); the four warps turn it into this chunk's softmax numerators
 //                      P = 2^(s − m) (bf16, written in the swizzled layout the tensor core
 //                      reads) with the chunk's per-head maximum m and sum l; a second MMA
-//                      forms Oᵀ = Vᵀ·Pᵀ (M = 128 dims, N = H); the partial output, m and l
+//                      forms Oᵀ = Vᵀ·Pᵀ (M = 128 dims, N = H, Vᵀ read MN-major); the partial output, m and l
 //                      go to the workspace. Slots not yet written (pos < W − 1) are masked.
 //   attn_combine_kernel  merges the chunks of each sequence and head (flash-decoding):
 //                      o = Σ_c 2^(m_c − m*) O_c / Σ_c 2^(m_c − m*) l_c, in bf16.
 // The q, k, v and output projections run on the tcgen05 GEMM of gemm_tc.cu.
 //
-// Ring layouts: keys [B][W][128] (slot-major), values [B][128][W] (dimension-major, so that
-// Vᵀ is a K-major operand like every other one: no transposed descriptor is needed). The
-// attention is a sum over the window's slots, so they are read in slot order whatever
-// position each holds. Every wait is bounded.
+// Ring layouts: keys and values [B][W][128], slot-major (a chunk is one contiguous 32 KB
+// block of each, and a step writes one 256-byte row of each). The attention is a sum over
+// the window's slots, so they are read in slot order whatever position each holds. Every
+// wait is bounded.
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -48,7 +49,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // Shared memory of the chunk kernel, offsets from a 1024-aligned base (every TMA box and
 // operand tile starts 1024-aligned): two stages of [keys 2 × [128 slots][64 dims] | values
-// 2 × [128 dims][64 slots] | queries 2 × [hp heads][64 dims]], then two buffers of softmax
+// 2 × [128 slots][64 dims] | queries 2 × [hp heads][64 dims]], then two buffers of softmax
 // numerators P (2 k-blocks [hp][64 slots] each) and the scores [hp][128] float.
 constexpr int kAttnStages = 2;
 constexpr int kSPitch = kChunk + 4;  // floats per score row: 16-byte row reads stay conflict-free
@@ -70,11 +71,13 @@ __host__ __device__ inline AttnSmem attn_smem(int H) {
 }
 
 struct AttnArgs {
-  const __nv_bfloat16* qkv;  // [B][(H+2)·128]
+  const __nv_bfloat16* qkv;  // [B][(H+2)·128], or (when qkv_part is set) unused
+  const float* qkv_part;     // [ksp][B][(H+2)·128]: the projection's split-K partial sums
+  int ksp;
   int n_used;                // ring chunks holding a position of the window (all once it wrapped)
   __nv_bfloat16* q_rot;      // [B][H][128]
   __nv_bfloat16* k_ring;     // [B][W][128]
-  __nv_bfloat16* v_ring;     // [B][128][W]
+  __nv_bfloat16* v_ring;     // [B][W][128]
   float* o_part;             // [B][n_chunks][H][128]
   float* m_part;             // [B][n_chunks][H]
   float* l_part;             // [B][n_chunks][H]
@@ -84,14 +87,32 @@ struct AttnArgs {
   int B, H, W, n_chunks;
 };
 
-// ---- RoPE, ring writes --------------------------------------------------------------
+// ---- RoPE, ring writes ------------------------------------------------------------------
+// One CTA per sequence. The projection's value of column `col` is qkv's bf16, or the bf16
+// rounding of the sum of the split-K slices (summed in slice order from 0, as the split
+// GEMM's own reduction does), so both paths see the same bits.
+__device__ __forceinline__ float2 attn_qkv2(const AttnArgs& a, int b, int64_t nq, int col) {
+  if (a.qkv_part == nullptr) {
+    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(a.qkv + (int64_t)b * nq + col);
+    return make_float2(__bfloat162float(v.x), __bfloat162float(v.y));
+  }
+  const int64_t stride = (int64_t)a.B * nq;
+  float2 acc = make_float2(0.f, 0.f);
+  for (int sl = 0; sl < a.ksp; ++sl) {
+    const float2 p = __ldcs(reinterpret_cast<const float2*>(a.qkv_part + sl * stride + (int64_t)b * nq + col));
+    acc.x += p.x;
+    acc.y += p.y;
+  }
+  const __nv_bfloat162 r = __floats2bfloat162_rn(acc.x, acc.y);
+  return make_float2(__bfloat162float(r.x), __bfloat162float(r.y));
+}
+
 __global__ void __launch_bounds__(256) attn_prep_kernel(AttnArgs a) {
-  pdl_wait();  // qkv is the previous kernel's output
+  pdl_wait();  // the projection is the previous kernel's output
   pdl_launch_dependents();
   const int b = blockIdx.x;
   const int H = a.H;
   const int64_t nq = (int64_t)(H + 2) * kDh;
-  const __nv_bfloat16* src = a.qkv + (int64_t)b * nq;
   const int slot = (int)(a.pos % a.W);
   // the 64 rotation angles of this position (the same for every head and every sequence):
   // θ_j = 10000^(−2j/128), the angle pos·θ_j reduced modulo 2π in float64 so that large
@@ -111,17 +132,19 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(AttnArgs a) {
   for (int i = threadIdx.x; i < (H + 1) * (kDh / 2); i += blockDim.x) {
     const int head = i / (kDh / 2), j = i % (kDh / 2);
     const float s = s_sin[j], c = s_cos[j];
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(src + head * kDh + 2 * j);
-    const float x0 = __bfloat162float(v.x), x1 = __bfloat162float(v.y);
-    const __nv_bfloat162 r = __floats2bfloat162_rn(x0 * c - x1 * s, x0 * s + x1 * c);
+    const float2 x = attn_qkv2(a, b, nq, head * kDh + 2 * j);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(x.x * c - x.y * s, x.x * s + x.y * c);
     if (head < H)
       *reinterpret_cast<__nv_bfloat162*>(a.q_rot + ((int64_t)b * H + head) * kDh + 2 * j) = r;
     else
       *reinterpret_cast<__nv_bfloat162*>(a.k_ring + ((int64_t)b * a.W + slot) * kDh + 2 * j) = r;
   }
-  // the value, unrotated, into the transposed ring
-  for (int d = threadIdx.x; d < kDh; d += blockDim.x)
-    a.v_ring[((int64_t)b * kDh + d) * a.W + slot] = src[(int64_t)(H + 1) * kDh + d];
+  // the value, unrotated, into the same slot of the value ring (one 256-byte row)
+  for (int i = threadIdx.x; i < kDh / 2; i += blockDim.x) {
+    const float2 v = attn_qkv2(a, b, nq, (H + 1) * kDh + 2 * i);
+    *reinterpret_cast<__nv_bfloat162*>(a.v_ring + ((int64_t)b * a.W + slot) * kDh + 2 * i) =
+        __floats2bfloat162_rn(v.x, v.y);
+  }
 }
 
 // ---- one ring chunk of one sequence ------------------------------------------------------
@@ -220,7 +243,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive_expect_tx(&full_bar[st], bytes);
         for (int kb = 0; kb < 2; ++kb) {
           tma_load_3d(stage + L.off_k + kb * kChunk * 128, &tmK, &full_bar[st], kb * 64, c * kChunk, b);
-          tma_load_3d(stage + L.off_v + kb * kDh * 128, &tmV, &full_bar[st], c * kChunk + kb * 64, 0, b);
+          tma_load_3d(stage + L.off_v + kb * kChunk * 128, &tmV, &full_bar[st], kb * 64, c * kChunk, b);
           tma_load_3d(stage + L.off_q + kb * hp * 128, &tmQ, &full_bar[st], kb * 64, 0, b);  // rows ≥ H: 0
         }
       }
@@ -243,13 +266,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         umma_commit(&s_full);
         if (!mbar_wait(&p_full, (uint32_t)n & 1u, &abort_s)) break;
         tc_fence_after();
-        // Oᵀ[dim][head] = Σ_slot Vᵀ[dim][slot] P[head][slot], into buffer n mod 2
+        // Oᵀ[dim][head] = Σ_slot Vᵀ[dim][slot] P[head][slot], into buffer n mod 2. The values
+        // sit slot-major as loaded (rows of 64 dims per slot, the second 64 dims a box
+        // further): Vᵀ is read as an MN-major operand, 16 slot rows per MMA.
         const uint8_t* pbuf = smem + L.off_p + (n & 1) * p_bytes;
         for (int kb = 0; kb < 2; ++kb)
           for (int k = 0; k < 4; ++k)
             umma_f16(tmem + (uint32_t)((1 + (n & 1)) * hp),
-                     umma_desc_sw128(smem_u32(stage + L.off_v + kb * kDh * 128) + k * 32),
-                     umma_desc_sw128(smem_u32(pbuf + kb * hp * 128) + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+                     umma_desc_sw128_mn(smem_u32(stage + L.off_v) + (kb * 4 + k) * 2048, kChunk * 128),
+                     umma_desc_sw128(smem_u32(pbuf + kb * hp * 128) + k * 32), idesc | kIdescAMN,
+                     (kb | k) != 0 ? 1u : 0u);
         umma_commit(&o_full[n & 1]);
         umma_commit(&empty_bar[st]);  // the stage's operands are read
       }
@@ -312,9 +338,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // values of slots holding no position may be anything (NaN included): zeroed, so that
       // the second product, where their weight is 0, stays finite
       if (n_valid < kChunk) {
-        const int d = q4 * 32 + lane;  // one row of Vᵀ per thread
+        const int d = q4 * 32 + lane;  // one value dimension per thread
         for (int k = n_valid; k < kChunk; ++k)
-          *reinterpret_cast<__nv_bfloat16*>(sV + (k >> 6) * kDh * 128 + sw128_offset(d, k & 63)) =
+          *reinterpret_cast<__nv_bfloat16*>(sV + (d >> 6) * kChunk * 128 + sw128_offset(k, d & 63)) =
               __float2bfloat16_rn(0.0f);
       }
       tc_fence_before();
@@ -382,26 +408,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ---- merge the chunks of each sequence ------------------------------------------------------
-// One CTA per (sequence, head), one thread per dimension: the chunks' maxima and sums are read
-// by every thread (the same addresses), the partial outputs as 512-byte rows. Only the chunks
-// holding a position of the window were computed (every one once the ring has wrapped).
-__global__ void __launch_bounds__(kDh) attn_combine_kernel(AttnArgs a) {
+// One warp per (sequence, head), four output dimensions per lane (16-byte loads of the partial
+// outputs), eight heads per CTA: the chunks' maxima are spread over the lanes and reduced by
+// shuffles; then every lane walks the chunks in order with their weights 2^(m_c − m*) (the
+// same arithmetic, in the same order, for every dimension).
+constexpr int kCombineHeads = 8;
+__global__ void __launch_bounds__(32 * kCombineHeads) attn_combine_kernel(AttnArgs a) {
   pdl_wait();
   pdl_launch_dependents();
-  const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  const int b = blockIdx.x, h = blockIdx.y * kCombineHeads + (int)threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (h >= a.H) return;
   const int64_t base = (int64_t)b * a.n_chunks;
   float mx = -INFINITY;
-  for (int c = 0; c < a.n_used; ++c) mx = fmaxf(mx, a.m_part[(base + c) * a.H + h]);
-  float num = 0.0f, den = 0.0f;
+  for (int c = lane; c < a.n_used; c += 32) mx = fmaxf(mx, a.m_part[(base + c) * a.H + h]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.0f;
 #pragma unroll 8
   for (int c = 0; c < a.n_used; ++c) {
     const int64_t part = base + c;
-    const float l = a.l_part[part * a.H + h];
     const float w = exp2f(a.m_part[part * a.H + h] - mx);
-    num = fmaf(w, a.o_part[(part * a.H + h) * kDh + d], num);
-    den = fmaf(w, l, den);
+    const float4 o = *reinterpret_cast<const float4*>(a.o_part + (part * a.H + h) * kDh + 4 * lane);
+    num = make_float4(fmaf(w, o.x, num.x), fmaf(w, o.y, num.y), fmaf(w, o.z, num.z), fmaf(w, o.w, num.w));
+    den = fmaf(w, a.l_part[part * a.H + h], den);
   }
-  a.o[((int64_t)b * a.H + h) * kDh + d] = __float2bfloat16_rn(num / den);
+  *reinterpret_cast<uint2*>(a.o + ((int64_t)b * a.H + h) * kDh + 4 * lane) =
+      make_uint2(pack_bf16x2(num.x / den, num.y / den), pack_bf16x2(num.z / den, num.w / den));
 }
 
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
@@ -450,11 +483,14 @@ AttnLayout attn_layout(int B, int D, int W) {
   return L;
 }
 
-cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, int64_t pos, int B, int D, int W,
-                                  const AttnLayout& L, void* ws, unsigned* status, cudaStream_t s) {
+cudaError_t launch_attention_core(const void* qkv, const float* qkv_part, int ksp, void* k_ring, void* v_ring,
+                                  int64_t pos, int B, int D, int W, const AttnLayout& L, void* ws, unsigned* status,
+                                  cudaStream_t s) {
   AttnArgs a{};
   uint8_t* w = static_cast<uint8_t*>(ws);
   a.qkv = static_cast<const __nv_bfloat16*>(qkv);
+  a.qkv_part = qkv_part;
+  a.ksp = ksp;
   a.q_rot = reinterpret_cast<__nv_bfloat16*>(w + L.off_q);
   a.k_ring = static_cast<__nv_bfloat16*>(k_ring);
   a.v_ring = static_cast<__nv_bfloat16*>(v_ring);
@@ -471,7 +507,7 @@ cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, i
   a.n_used = pos >= W - 1 ? L.n_chunks : (int)((pos + kChunk) / kChunk);  // chunks with a position
   CUtensorMap mk, mv, mq;
   if (!make_map_3d(&mk, k_ring, kDh, W, B, kDh * 2, (uint64_t)W * kDh * 2, 64, kChunk)) return cudaErrorInvalidValue;
-  if (!make_map_3d(&mv, v_ring, W, kDh, B, (uint64_t)W * 2, (uint64_t)W * kDh * 2, 64, kDh))
+  if (!make_map_3d(&mv, v_ring, kDh, W, B, kDh * 2, (uint64_t)W * kDh * 2, 64, kChunk))
     return cudaErrorInvalidValue;
   const AttnSmem sm = attn_smem(L.H);
   if (!make_map_3d(&mq, a.q_rot, kDh, L.H, B, kDh * 2, (uint64_t)L.H * kDh * 2, 64, (uint32_t)sm.hp))
@@ -494,7 +530,8 @@ cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, i
   const int grid = items < num_sms() ? items : num_sms();
   e = launch_pdl(attn_chunk_kernel, dim3(grid), dim3(kAttnThreads), smem, s, mk, mv, mq, a);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_combine_kernel, dim3(B, L.H), dim3(kDh), 0, s, a);
+  return launch_pdl(attn_combine_kernel, dim3(B, (L.H + kCombineHeads - 1) / kCombineHeads),
+                    dim3(32 * kCombineHeads), 0, s, a);
 }
 
 }  // namespace rglru

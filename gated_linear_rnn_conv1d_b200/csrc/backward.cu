@@ -15,7 +15,9 @@
 // (bwd_maps_kernel); a short sequential pass per (row, channel) hands every chunk the g
 // entering it from the right (bwd_carries_kernel); each chunk then replays its steps with
 // the gate gradients fused (bwd_grads_kernel). The linears' gradients are tensor-core GEMMs
-// (gemm_tc.cu) on transposed copies made here; the Conv1D backward is its own kernel.
+// (gemm_tc.cu): ∂u ⊃ ∂z·[W_a; W_x] on a transposed copy of the weights made here, ∂W_a and
+// ∂W_x = ∂zᵀu with ∂z and u read in place as MN-major operands; the Conv1D backward is its
+// own kernel.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -31,6 +33,10 @@ constexpr int kBwdThreads = 128;  // threads per block; each thread takes 2 chan
 __device__ __forceinline__ float2 ld_bf2(const __nv_bfloat16* p) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
 }
+// read-only data of the kernel (lets the compiler move the load ahead of unrelated stores)
+__device__ __forceinline__ float2 ld_bf2_nc(const __nv_bfloat16* p) {
+  return __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162*>(p)));
+}
 __device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
@@ -39,8 +45,8 @@ __device__ __forceinline__ int64_t zcol(int c) { return (int64_t)256 * (c / 128)
 
 // a_t from z_a (with its bias) and c·log σ(Λ) (fast exponentials: the operands are bf16)
 __device__ __forceinline__ float decay_of(float za, float cla) {
-  const float r = __fdividef(1.0f, 1.0f + __expf(-za));
-  return __expf(r * cla);
+  const float r = rcp_approx(1.0f + ex2_approx(-za * kLog2e));
+  return ex2_approx(r * cla * kLog2e);
 }
 
 struct BwdDims {
@@ -115,9 +121,6 @@ struct BwdGradArgs {
   const float* Lambda;      // [R]
   const float* gin;         // [B][n_chunks][R]
   __nv_bfloat16* dz;        // [B·T][2R]: ∂z_a in columns [0, R), ∂z_x in [R, 2R)
-  __nv_bfloat16* dzt;       // [2R][n_pad]: ∂zᵀ (the weight-gradient GEMMs' A operand)
-  __nv_bfloat16* ut;        // [R][n_pad]: uᵀ (their B operand)
-  int64_t n_pad;
   float* du;                // [B][T][R] the direct term ∂ℓ/∂u_t ⊃ g m i
   float* dLsum;             // [R] Σ ∂log a·r·c (atomic)
   float* db_a;              // [R] (atomic)
@@ -126,26 +129,9 @@ struct BwdGradArgs {
 };
 
 // Pass 3: each chunk replays its steps from the g entering it, with the gate gradients. Steps
-// go in blocks of eight aligned to multiples of 8 (their loads issued together ahead of the
-// chain); besides ∂z (row-major, for the ∂u GEMM) the block's ∂z and u values of the thread's
-// channels are written transposed — ∂zᵀ and uᵀ, the weight-gradient GEMMs' K-major operands
-// along the tokens — as one 16-byte store per row when the block is whole and aligned.
-__device__ __forceinline__ void st_t8(__nv_bfloat16* row, int64_t col0, const uint32_t (&w)[4], int j_lo, int j_hi,
-                                      bool vec) {
-  if (vec) {
-    *reinterpret_cast<uint4*>(row + col0) = make_uint4(w[0], w[1], w[2], w[3]);
-  } else {
-    for (int j = j_lo; j <= j_hi; ++j) {
-      const uint32_t v = w[j >> 1];
-      reinterpret_cast<uint16_t*>(row)[col0 + j] = (uint16_t)((j & 1) ? (v >> 16) : (v & 0xFFFFu));
-    }
-  }
-}
-__device__ __forceinline__ void put_bf16(uint32_t (&w)[4], int j, float v) {
-  const uint32_t h = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
-  w[j >> 1] = (j & 1) ? ((w[j >> 1] & 0x0000FFFFu) | (h << 16)) : ((w[j >> 1] & 0xFFFF0000u) | h);
-}
-
+// go in blocks of kGradBlock aligned to multiples of it, their loads issued together ahead of
+// the chain (a block of 8 held 160 registers a thread and ran slower than single steps).
+constexpr int kGradBlock = 2;
 __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, BwdDims d) {
   const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
   if (c >= d.R) return;
@@ -168,49 +154,54 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
   }
   const float2 h0v =
       a.h0 != nullptr ? *reinterpret_cast<const float2*>(a.h0 + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
-  // rows of the transposed outputs: ∂z_a of c, c+1; ∂z_x of c, c+1; u of c, c+1
-  __nv_bfloat16* trow[6] = {a.dzt + (int64_t)c * a.n_pad, a.dzt + (int64_t)(c + 1) * a.n_pad,
-                            a.dzt + (int64_t)(d.R + c) * a.n_pad, a.dzt + (int64_t)(d.R + c + 1) * a.n_pad,
-                            a.ut + (int64_t)c * a.n_pad, a.ut + (int64_t)(c + 1) * a.n_pad};
-  const bool aligned_rows = (d.T % 8) == 0;  // then row0 + 8k is a multiple of 8
   float sL[2] = {0.f, 0.f}, sa[2] = {0.f, 0.f}, sx[2] = {0.f, 0.f};
-  for (int tb = (t1 - 1) & ~7; tb >= t0; tb -= 8) {
-    // steps tb … tb + 7 of this chunk (those < t1), replayed from the last to the first
-    const int j_hi = min(7, t1 - 1 - tb);
-    float2 dyv[8], uv[8], zav[8], zxv[8], hpv[8];
+  // this thread's elements at step tb of a block, walked back by pointer decrements
+  const int64_t R = d.R, R2 = 2 * d.R, pitch = d.pitch;
+  int tb = (t1 - 1) & ~(kGradBlock - 1);
+  const __nv_bfloat16* p_dy = a.dy + (row0 + tb) * R + c;
+  const __nv_bfloat16* p_u = a.u + (row0 + tb) * R + c;
+  const __nv_bfloat16* p_y = a.y + (row0 + tb - 1) * R + c;  // h_{t−1} (read only for t > 0)
+  const __nv_bfloat16* p_z = zb + (int64_t)tb * pitch;
+  __nv_bfloat16* p_dz = a.dz + (row0 + tb) * R2 + c;
+  float* p_du = a.du + (row0 + tb) * R + c;
+  for (; tb >= t0; tb -= kGradBlock) {
+    // steps tb … tb + kGradBlock − 1 of this chunk (those < t1), replayed from the last
+    const int j_hi = min(kGradBlock - 1, t1 - 1 - tb);
+    float2 dyv[kGradBlock], uv[kGradBlock], zav[kGradBlock], zxv[kGradBlock], hpv[kGradBlock];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int t = tb + j;
+    for (int j = 0; j < kGradBlock; ++j) {
       if (j <= j_hi) {
-        const int64_t e = (row0 + t) * d.R + c;
-        dyv[j] = ld_bf2(a.dy + e);
-        uv[j] = ld_bf2(a.u + e);
-        zav[j] = ld_bf2(zb + (int64_t)t * d.pitch);
-        zxv[j] = ld_bf2(zb + (int64_t)t * d.pitch + 128);
-        hpv[j] = t > 0 ? ld_bf2(a.y + e - d.R) : h0v;
+        dyv[j] = ld_bf2_nc(p_dy + j * R);
+        uv[j] = ld_bf2_nc(p_u + j * R);
+        zav[j] = ld_bf2_nc(p_z + j * pitch);
+        zxv[j] = ld_bf2_nc(p_z + j * pitch + 128);
+        hpv[j] = tb + j > 0 ? ld_bf2_nc(p_y + j * R) : h0v;
       }
     }
-    uint32_t tw[6][4] = {};
 #pragma unroll
-    for (int j = 7; j >= 0; --j) {
+    for (int j = kGradBlock - 1; j >= 0; --j) {
       if (j > j_hi) continue;
-      const int t = tb + j;
       const float dy_[2] = {dyv[j].x, dyv[j].y}, u_[2] = {uv[j].x, uv[j].y}, za_[2] = {zav[j].x, zav[j].y},
                   zx_[2] = {zxv[j].x, zxv[j].y}, hp_[2] = {hpv[j].x, hpv[j].y};
       float dza[2], dzx[2], dud[2];
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const float g = fmaf(an[k], gn[k], dy_[k]);
-        const float r = __fdividef(1.0f, 1.0f + __expf(-za_[k]));
-        const float i = __fdividef(1.0f, 1.0f + __expf(-zx_[k]));
+        // gates and decay as the forward's fast path: hardware ex2/rcp/rsqrt, 1 − a_t² from
+        // the Taylor form of −expm1 near 0
+        const float r = rcp_approx(1.0f + ex2_approx(-za_[k] * kLog2e));
+        const float i = rcp_approx(1.0f + ex2_approx(-zx_[k] * kLog2e));
         const float la = r * cl[k];
-        const float at = __expf(la);
-        const float mt = sqrtf(-expm1f(2.0f * la));
+        const float at = ex2_approx(la * kLog2e);
+        const float x2 = 2.0f * la;
+        const float q = (x2 > -0.25f) ? neg_expm1_small(x2) : fmaf(-at, at, 1.0f);  // 1 − a_t²
+        const float rs = rsqrt_approx(fmaxf(q, 1e-30f));
+        const float mt = q > 0.0f ? q * rs : 0.0f;         // √(1 − a_t²)
+        const float r_over_m = q > 0.0f ? r * rs : 0.0f;   // r / √(1 − a_t²)
         const float d_a = g * hp_[k];
         const float d_m = g * i * u_[k];
         const float d_i = g * mt * u_[k];
         dud[k] = g * mt * i;
-        const float r_over_m = mt > 0.0f ? __fdividef(r, mt) : 0.0f;
         const float dlr = d_a * at * r - d_m * at * at * r_over_m;  // ∂log a_t · r_t
         dza[k] = dlr * cl[k] * (1.0f - r);
         dzx[k] = d_i * i * (1.0f - i);
@@ -220,19 +211,16 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
         gn[k] = g;
         an[k] = at;
       }
-      st_bf2(a.dz + (row0 + t) * 2 * d.R + c, dza[0], dza[1]);
-      st_bf2(a.dz + (row0 + t) * 2 * d.R + d.R + c, dzx[0], dzx[1]);
-      *reinterpret_cast<float2*>(a.du + (row0 + t) * d.R + c) = make_float2(dud[0], dud[1]);
-      put_bf16(tw[0], j, dza[0]);
-      put_bf16(tw[1], j, dza[1]);
-      put_bf16(tw[2], j, dzx[0]);
-      put_bf16(tw[3], j, dzx[1]);
-      put_bf16(tw[4], j, u_[0]);
-      put_bf16(tw[5], j, u_[1]);
+      st_bf2(p_dz + j * R2, dza[0], dza[1]);
+      st_bf2(p_dz + j * R2 + R, dzx[0], dzx[1]);
+      *reinterpret_cast<float2*>(p_du + j * R) = make_float2(dud[0], dud[1]);
     }
-    const bool vec = aligned_rows && j_hi == 7;
-#pragma unroll
-    for (int r = 0; r < 6; ++r) st_t8(trow[r], row0 + tb, tw[r], 0, j_hi, vec);
+    p_dy -= kGradBlock * R;
+    p_u -= kGradBlock * R;
+    p_y -= kGradBlock * R;
+    p_z -= kGradBlock * pitch;
+    p_dz -= kGradBlock * R2;
+    p_du -= kGradBlock * R;
   }
   if (chunk == 0 && a.dh0 != nullptr)  // the gradient reaching h_{−1} = h0
     *reinterpret_cast<float2*>(a.dh0 + (int64_t)b * d.R + c) = make_float2(an[0] * gn[0], an[1] * gn[1]);
@@ -255,8 +243,7 @@ struct BwdConvArgs {
   const __nv_bfloat16* x;       // [B][T][R]
   const __nv_bfloat16* state0;  // [B][3][R] (x_{−3}, x_{−2}, x_{−1}) or null
   const float* conv_w;          // [4][R]
-  const float* du;              // [B][T][R] direct term
-  const float* dug;             // [B][T][R] gate-GEMM term
+  const float* du;              // [B][T][R] ∂ℓ/∂u (direct and gate terms)
   __nv_bfloat16* dx;            // [B][T][R]
   __nv_bfloat16* dstate0;       // [B][3][R] or null
   float* dconv_w;               // [4][R] (atomic)
@@ -280,9 +267,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, Bw
   }
   auto du_at = [&](int t) -> float2 {  // total ∂ℓ/∂u_t, zero past T
     if (t >= d.T) return make_float2(0.f, 0.f);
-    const float2 p = *reinterpret_cast<const float2*>(a.du + base + (int64_t)t * d.R);
-    const float2 q = *reinterpret_cast<const float2*>(a.dug + base + (int64_t)t * d.R);
-    return make_float2(p.x + q.x, p.y + q.y);
+    return *reinterpret_cast<const float2*>(a.du + base + (int64_t)t * d.R);
   };
   auto x_at = [&](int t) -> float2 {  // x_t, from the conv history for t < 0
     if (t >= 0) return ld_bf2(a.x + base + (int64_t)t * d.R);
@@ -380,7 +365,6 @@ cudaError_t transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols
 BwdLayout bwd_layout(int B, int T, int R) {
   BwdLayout L;
   const int64_t n = (int64_t)B * T;
-  const int64_t np = (n + 63) / 64 * 64;  // token count padded for the transposed operands
   const int n_chunks = (T + kScanTC - 1) / kScanTC;
   auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
   size_t o = 256;  // status word
@@ -391,13 +375,9 @@ BwdLayout bwd_layout(int B, int T, int R) {
   L.off_gin = o;    o += r256((size_t)B * n_chunks * R * 4);
   L.off_dz = o;     o += r256((size_t)n * 2 * R * 2);
   L.off_du = o;     o += r256((size_t)n * R * 4);
-  L.off_dug = o;    o += r256((size_t)n * R * 4);
   L.off_wt = o;     o += r256((size_t)2 * R * R * 2);
-  L.off_dzt = o;    o += r256((size_t)2 * R * np * 2);
-  L.off_ut = o;     o += r256((size_t)R * np * 2);
   L.off_dL = o;     o += r256((size_t)R * 4);
   L.bytes = o;
-  L.n_pad = np;
   L.n_chunks = n_chunks;
   return L;
 }
@@ -414,10 +394,7 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   float* gin = reinterpret_cast<float*>(w + L.off_gin);
   __nv_bfloat16* dz = reinterpret_cast<__nv_bfloat16*>(w + L.off_dz);
   float* du = reinterpret_cast<float*>(w + L.off_du);
-  float* dug = reinterpret_cast<float*>(w + L.off_dug);
   __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(w + L.off_wt);
-  __nv_bfloat16* dzt = reinterpret_cast<__nv_bfloat16*>(w + L.off_dzt);
-  __nv_bfloat16* ut = reinterpret_cast<__nv_bfloat16*>(w + L.off_ut);
   float* dLsum = reinterpret_cast<float*>(w + L.off_dL);
   cudaError_t e;
   // the accumulated outputs start at zero
@@ -439,33 +416,28 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   bwd_carries_kernel<<<g_rows, kBwdThreads, 0, s>>>(P, Q, g.dh_T, gin, d);
   BwdGradArgs ga{static_cast<const __nv_bfloat16*>(z), static_cast<const __nv_bfloat16*>(u),
                  static_cast<const __nv_bfloat16*>(g.y), static_cast<const __nv_bfloat16*>(g.dy), g.h0, g.Lambda, gin,
-                 dz, dzt, ut, L.n_pad, du, dLsum, g.db_a, g.db_x, g.dh0};
-  // the tokens n … n_pad − 1 of the transposed operands are zero (K padding of the ∂W GEMMs)
-  if (L.n_pad > n) {
-    if ((e = cudaMemset2DAsync(dzt + n, (size_t)L.n_pad * 2, 0, (size_t)(L.n_pad - n) * 2, (size_t)2 * R, s)) !=
-        cudaSuccess)
-      return e;
-    if ((e = cudaMemset2DAsync(ut + n, (size_t)L.n_pad * 2, 0, (size_t)(L.n_pad - n) * 2, (size_t)R, s)) !=
-        cudaSuccess)
-      return e;
-  }
+                 dz, du, dLsum, g.db_a, g.db_x, g.dh0};
   bwd_grads_kernel<<<g_chunks, kBwdThreads, 0, s>>>(ga, d);
   bwd_lambda_kernel<<<(R + 255) / 256, 256, 0, s>>>(dLsum, g.Lambda, g.dLambda, R);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // ∂ℓ/∂u ⊃ [∂z_a | ∂z_x]·[W_a; W_x]: B operand [W_a; W_x]ᵀ = [R][2R]
-  if ((e = transpose_bf16(g.W_a, wt, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
-  if ((e = transpose_bf16(g.W_x, wt + R, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
-  // (in float32: this term reaches ∂x through the Conv1D backward without another rounding)
-  if ((e = launch_gemm_f32out(dz, wt, dug, n, R, 2 * R, R, status, s)) != cudaSuccess) return e;
-  // ∂W_a = ∂z_aᵀ u, ∂W_x = ∂z_xᵀ u over the tokens (K = tokens, zero-padded to n_pad; the
-  // transposed operands come straight from the gradient pass)
-  if ((e = launch_gemm_f32out(dzt, ut, g.dW_a, R, R, (int)L.n_pad, R, status, s)) != cudaSuccess) return e;
-  if ((e = launch_gemm_f32out(dzt + (int64_t)R * L.n_pad, ut, g.dW_x, R, R, (int)L.n_pad, R, status, s)) !=
-      cudaSuccess)
-    return e;
+  // ∂ℓ/∂u ⊃ [∂z_a | ∂z_x]·[W_a; W_x], added in float32 to the direct term the gradient pass
+  // wrote (∂u then reaches ∂x through the Conv1D backward without a rounding). The weights
+  // are read in place (MN-major) when R is a multiple of 64, else through a transposed copy
+  // [W_a; W_x]ᵀ = [R][2R].
+  if (R % 64 == 0) {
+    if ((e = launch_gemm_f32out_wcat(dz, g.W_a, g.W_x, du, n, R, R, R, true, status, s)) != cudaSuccess) return e;
+  } else {
+    if ((e = transpose_bf16(g.W_a, wt, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
+    if ((e = transpose_bf16(g.W_x, wt + R, R, R, R, 2 * R, R, s)) != cudaSuccess) return e;
+    if ((e = launch_gemm_f32out(dz, wt, du, n, R, 2 * R, R, true, status, s)) != cudaSuccess) return e;
+  }
+  // ∂W_a = ∂z_aᵀ u, ∂W_x = ∂z_xᵀ u over the tokens: ∂z and u read in place, token-major
+  // (MN-major operands)
+  if ((e = launch_gemm_f32out_mn(dz, 2 * R, u, R, g.dW_a, R, R, n, R, status, s)) != cudaSuccess) return e;
+  if ((e = launch_gemm_f32out_mn(dz + R, 2 * R, u, R, g.dW_x, R, R, n, R, status, s)) != cudaSuccess) return e;
   // Conv1D backward
   BwdConvArgs ca{static_cast<const __nv_bfloat16*>(g.x), static_cast<const __nv_bfloat16*>(g.state0), g.conv_w, du,
-                 dug, static_cast<__nv_bfloat16*>(g.dx), static_cast<__nv_bfloat16*>(g.dstate0), g.dconv_w,
+                 static_cast<__nv_bfloat16*>(g.dx), static_cast<__nv_bfloat16*>(g.dstate0), g.dconv_w,
                  g.dconv_b};
   bwd_conv_kernel<<<g_chunks, kBwdThreads, 0, s>>>(ca, d);
   return cudaGetLastError();

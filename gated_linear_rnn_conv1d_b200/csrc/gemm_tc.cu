@@ -65,6 +65,13 @@ struct EpiArgs {
   // [s·kb_per, (s+1)·kb_per) and writes its partial sums at Cf + s·split_stride
   int k_split, kb_per;
   int64_t split_stride;
+  // operands MN-major (STORE_F32, one B): A [K][M] (a_mn) and B [K][N] (b_mn) row-major,
+  // staged as K rows of 64 M (N) columns; otherwise K-major, A [M][K] and B [N][K]. With
+  // b_split_k > 0 (a multiple of BK), B's rows k ≥ b_split_k come from the second B map, at
+  // row k − b_split_k: B = [B0; B1] stacked along K.
+  int a_mn, b_mn, b_split_k;
+  // STORE_F32: C += A·Bᵀ (C read before it is written, element by element) instead of C = A·Bᵀ
+  int accumulate;
 };
 
 // The k-block range of slice `ks` (the whole K when the GEMM is not split).
@@ -546,10 +553,29 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           uint8_t* sb = sa + k2ABytes;
           const uint32_t lbar = leader_full0 + stage * 8;
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * k2StageBytes);
-          tma_load_2d_2sm(sa, &tmA, lbar, kb * BK, arow);
-          if (DUAL) {
+          if (!DUAL && (ep.a_mn | ep.b_mn)) {
+            // an MN-major operand: this CTA's 128 columns as two boxes of 64 columns × BK rows
+            if (ep.a_mn) {
+              tma_load_2d_2sm(sa, &tmA, lbar, arow, kb * BK);
+              tma_load_2d_2sm(sa + k2ABytes / 2, &tmA, lbar, arow + 64, kb * BK);
+            } else {
+              tma_load_2d_2sm(sa, &tmA, lbar, kb * BK, arow);
+            }
+            const int bcol = n_blk * 256 + (int)rank * 128;
+            if (ep.b_mn) {
+              const bool second = ep.b_split_k > 0 && kb * BK >= ep.b_split_k;
+              const CUtensorMap* mb = second ? &tmB1 : &tmB0;
+              const int kr = kb * BK - (second ? ep.b_split_k : 0);
+              tma_load_2d_2sm(sb, mb, lbar, bcol, kr);
+              tma_load_2d_2sm(sb + k2BBytes / 2, mb, lbar, bcol + 64, kr);
+            } else {
+              tma_load_2d_2sm(sb, &tmB0, lbar, kb * BK, bcol);
+            }
+          } else if (DUAL) {
+            tma_load_2d_2sm(sa, &tmA, lbar, kb * BK, arow);
             tma_load_2d_2sm(sb, rank == 0 ? &tmB0 : &tmB1, lbar, kb * BK, n_blk * 128);
           } else {
+            tma_load_2d_2sm(sa, &tmA, lbar, kb * BK, arow);
             tma_load_2d_2sm(sb, &tmB0, lbar, kb * BK, n_blk * 256 + (int)rank * 128);
           }
           if (++stage == S) { stage = 0; phase ^= 1; }
@@ -576,10 +602,24 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * k2StageBytes);
           const uint32_t b_addr = a_addr + k2ABytes;
+          if (!DUAL && (ep.a_mn | ep.b_mn)) {
+            // MN-major: 16 k-rows of 128 B per MMA, the second 64 columns half a stage operand
+            // further; K-major: 32 bytes further along the swizzled rows
+            const uint32_t idesc = k2Idesc | (ep.a_mn ? kIdescAMN : 0u) | (ep.b_mn ? kIdescBMN : 0u);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            umma_f16_2sm(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), k2Idesc,
-                         (kb != kb0 || k != 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k)
+              umma_f16_2sm(d_tmem,
+                           ep.a_mn ? umma_desc_sw128_mn(a_addr + k * 2048, k2ABytes / 2)
+                                   : umma_desc_sw128(a_addr + k * 32),
+                           ep.b_mn ? umma_desc_sw128_mn(b_addr + k * 2048, k2BBytes / 2)
+                                   : umma_desc_sw128(b_addr + k * 32),
+                           idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)
+              umma_f16_2sm(d_tmem, umma_desc_sw128(a_addr + k * 32), umma_desc_sw128(b_addr + k * 32), k2Idesc,
+                           (kb != kb0 || k != 0) ? 1u : 0u);
+          }
           umma_commit_2sm_both(&empty_bar[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -708,11 +748,18 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           const int gcol = n_blk * BN + col0;
           if (row_ok) {
             float4* d = reinterpret_cast<float4*>(ep.Cf + split_off + row * ep.ldc + gcol);
+            float4 c[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              c[q] = (ep.accumulate && gcol + 4 * q < ep.N) ? d[q] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               if (gcol + 4 * q < ep.N)
-                d[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                   __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+                d[q] = ep.accumulate
+                           ? make_float4(c[q].x + __uint_as_float(r[4 * q]), c[q].y + __uint_as_float(r[4 * q + 1]),
+                                         c[q].z + __uint_as_float(r[4 * q + 2]), c[q].w + __uint_as_float(r[4 * q + 3]))
+                           : make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                         __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
           }
         } else {
 #pragma unroll
@@ -1032,6 +1079,22 @@ __global__ void __launch_bounds__(kStepThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_s;
   const uint32_t leader_full0 = mapa_rank(smem_u32(&full_bar[0]), pair_leader);
+  const int wrow = cblk * 128 + (int)rank * 64;
+  const int pre = k_blocks < S ? k_blocks : S;  // stages whose weights load before u_t exists
+  if (warp == 0) {
+    // The weights do not depend on the decode conv kernel: while it runs, lane 0 fills the
+    // first stages' weight halves (their u_t halves follow once u_t is written). (An L2
+    // prefetch of the CTA's whole weight slice here as well made the step slower.)
+    if (lane == 0) {
+      for (int kb = 0; kb < pre; ++kb) {
+        uint8_t* sa = smem + kb * kStepStageBytes;
+        const uint32_t lbar = leader_full0 + kb * 8;
+        if (leader) mbar_arrive_expect_tx(&full_bar[kb], 2 * kStepStageBytes);
+        tma_load_2d_2sm(sa, &tmWa, lbar, k0 + kb * BK, wrow);
+        tma_load_2d_2sm(sa + 64 * BK * 2, &tmWx, lbar, k0 + kb * BK, wrow);
+      }
+    }
+  }
   // launched as a programmatic dependent of the decode conv kernel: everything above
   // overlapped it; u_t, u_t in float32 and c·log σ(Λ) are its results
   pdl_wait();
@@ -1061,16 +1124,17 @@ __global__ void __launch_bounds__(kStepThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const int wrow = cblk * 128 + (int)rank * 64;
       for (int kb = 0; kb < k_blocks; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_s)) { ok = false; break; }
         uint8_t* sa = smem + stage * kStepStageBytes;
         uint8_t* sb = sa + kStepABytes;
         const uint32_t lbar = leader_full0 + stage * 8;
-        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStepStageBytes);
         const int kc = k0 + kb * BK;
-        tma_load_2d_2sm(sa, &tmWa, lbar, kc, wrow);
-        tma_load_2d_2sm(sa + 64 * BK * 2, &tmWx, lbar, kc, wrow);
+        if (kb >= pre) {  // the first `pre` stages hold their weights already
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_s)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * kStepStageBytes);
+          tma_load_2d_2sm(sa, &tmWa, lbar, kc, wrow);
+          tma_load_2d_2sm(sa + 64 * BK * 2, &tmWx, lbar, kc, wrow);
+        }
         tma_load_2d_2sm(sb, &tmU, lbar, kc, (int)rank * 128);
         if (++stage == S) { stage = 0; phase ^= 1; }
       }
@@ -1396,8 +1460,8 @@ cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, 
 }
 
 cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t M, int N, int K, int64_t ldc,
-                               unsigned* status, cudaStream_t s) {
-  // as launch_gemm_bf16, with float32 output rows
+                               bool accumulate, unsigned* status, cudaStream_t s) {
+  // as launch_gemm_bf16, with float32 output rows (added to C's when `accumulate`)
   CUtensorMap ma, mb;
   if (!make_map_2d(&ma, A, K, M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, 128)) return cudaErrorInvalidValue;
@@ -1405,8 +1469,49 @@ cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t 
   ep.Cf = C;
   ep.ldc = ldc;
   ep.N = N;
+  ep.accumulate = accumulate ? 1 : 0;
   const int n_tiles_n = (N + 255) / 256;
   return launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+}
+
+cudaError_t launch_gemm_f32out_mn(const void* A, int64_t lda, const void* Bm, int64_t ldb, float* C, int M, int N,
+                                  int64_t K, int64_t ldc, unsigned* status, cudaStream_t s) {
+  // C = Aᵀ B over K rows: A [K][lda] holding M columns, B [K][ldb] holding N columns, both
+  // staged MN-major (no transposed copies); rows past K read as zeros
+  if (lda % 8 || ldb % 8 || (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(Bm) & 15) ||
+      K > INT32_MAX)
+    return cudaErrorInvalidValue;
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, A, M, K, (uint64_t)lda * 2, 64, BK)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb, Bm, N, K, (uint64_t)ldb * 2, 64, BK)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.Cf = C;
+  ep.ldc = ldc;
+  ep.N = N;
+  ep.a_mn = 1;
+  ep.b_mn = 1;
+  const int n_tiles_n = (N + 255) / 256;
+  return launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, (int)K, n_tiles_n, ep, status, s);
+}
+
+cudaError_t launch_gemm_f32out_wcat(const void* A, const void* W0, const void* W1, float* C, int64_t M, int N,
+                                    int Kh, int64_t ldc, bool accumulate, unsigned* status, cudaStream_t s) {
+  // C (+)= A·[W0; W1]: A [M][2Kh] K-major, W0 and W1 [Kh][N] row-major read in place as the
+  // MN-major B operand, W0 for the k-blocks below Kh and W1 above (Kh a multiple of BK)
+  if (Kh % BK || N % 8) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb0, mb1;
+  if (!make_map_2d(&ma, A, 2 * (uint64_t)Kh, M, (uint64_t)Kh * 4, BK, BM)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb0, W0, N, Kh, (uint64_t)N * 2, 64, BK)) return cudaErrorInvalidValue;
+  if (!make_map_2d(&mb1, W1, N, Kh, (uint64_t)N * 2, 64, BK)) return cudaErrorInvalidValue;
+  EpiArgs ep{};
+  ep.Cf = C;
+  ep.ldc = ldc;
+  ep.N = N;
+  ep.accumulate = accumulate ? 1 : 0;
+  ep.b_mn = 1;
+  ep.b_split_k = Kh;
+  const int n_tiles_n = (N + 255) / 256;
+  return launch_tc2<EPI_STORE_F32, false>(ma, mb0, mb1, M, 2 * Kh, n_tiles_n, ep, status, s);
 }
 
 namespace {
@@ -1433,23 +1538,30 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 }
 }  // namespace
 
-cudaError_t launch_gemm_bf16_skinny(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
-                                    float* part, size_t part_bytes, unsigned* status, cudaStream_t s) {
-  // Few output tiles (M = a decode batch): split K so that about every SM pair works, each
-  // slice writing float32 partial sums, then sum the slices into bf16.
+int skinny_splits(int64_t M, int N, int K, size_t part_bytes) {
+  // Few output tiles (M = a decode batch): split K so that about every SM pair works, at
+  // least 4 k-blocks a slice, the slices' float32 partial sums within part_bytes; no empty
+  // slice.
   const int64_t m_pairs = (M + 255) / 256;
   const int n_tiles_n = (N + 255) / 256;
   const int k_blocks = (K + BK - 1) / BK;
   const int64_t tiles = m_pairs * n_tiles_n;
   const int clusters = num_sms() / 2;
   int ksp = 1;
-  if (part != nullptr && tiles * 2 <= clusters && N % 8 == 0) {
-    ksp = (int)std::min<int64_t>(clusters / tiles, k_blocks / 4);  // at least 4 k-blocks a slice
+  if (part_bytes > 0 && tiles * 2 <= clusters && N % 8 == 0) {
+    ksp = (int)std::min<int64_t>(clusters / tiles, k_blocks / 4);
     while (ksp > 1 && (size_t)ksp * M * N * 4 > part_bytes) --ksp;
   }
-  if (ksp <= 1) return launch_gemm_bf16(A, Bm, C, M, N, K, ldc, status, s);
+  if (ksp <= 1) return 1;
   const int kb_per = (k_blocks + ksp - 1) / ksp;
-  ksp = (k_blocks + kb_per - 1) / kb_per;  // no empty slice
+  return (k_blocks + kb_per - 1) / kb_per;
+}
+
+cudaError_t launch_gemm_partials(const void* A, const void* Bm, int64_t M, int N, int K, float* part, int ksp,
+                                 unsigned* status, cudaStream_t s) {
+  const int k_blocks = (K + BK - 1) / BK;
+  const int kb_per = (k_blocks + ksp - 1) / ksp;
+  if (ksp < 1 || (k_blocks + kb_per - 1) / kb_per != ksp) return cudaErrorInvalidValue;
   CUtensorMap ma, mb;
   if (!make_map_2d(&ma, A, K, M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_map_2d(&mb, Bm, K, N, (uint64_t)K * 2, BK, 128)) return cudaErrorInvalidValue;
@@ -1460,7 +1572,15 @@ cudaError_t launch_gemm_bf16_skinny(const void* A, const void* Bm, void* C, int6
   ep.k_split = ksp;
   ep.kb_per = kb_per;
   ep.split_stride = M * (int64_t)N;
-  cudaError_t e = launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, K, n_tiles_n, ep, status, s);
+  return launch_tc2<EPI_STORE_F32, false>(ma, mb, mb, M, K, (N + 255) / 256, ep, status, s);
+}
+
+cudaError_t launch_gemm_bf16_skinny(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
+                                    float* part, size_t part_bytes, unsigned* status, cudaStream_t s) {
+  // the slices' partial sums, then one kernel summing them into bf16
+  const int ksp = part != nullptr ? skinny_splits(M, N, K, part_bytes) : 1;
+  if (ksp <= 1) return launch_gemm_bf16(A, Bm, C, M, N, K, ldc, status, s);
+  cudaError_t e = launch_gemm_partials(A, Bm, M, N, K, part, ksp, status, s);
   if (e != cudaSuccess) return e;
   const int64_t work = M * (N / 8);
   const int blocks = (int)std::min<int64_t>((work + 255) / 256, (int64_t)num_sms() * 8);

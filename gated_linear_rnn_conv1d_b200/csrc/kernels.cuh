@@ -92,10 +92,25 @@ cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, 
 constexpr size_t kSplitPartBytes = (size_t)80 * 256 * 256 * 4;
 cudaError_t launch_gemm_bf16_skinny(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
                                     float* part, size_t part_bytes, unsigned* status, cudaStream_t s);
-// C = A·Bᵀ as launch_gemm_bf16 (A [M][K], B [N][K] bf16, K-contiguous), C float32 [M][ldc],
-// N a multiple of 4.
+// The split launch_gemm_bf16_skinny would choose (1: not split), and its GEMM alone: slice
+// s of the K blocks writes its float32 partial sums to part + s·M·N ([M][N] each).
+int skinny_splits(int64_t M, int N, int K, size_t part_bytes);
+cudaError_t launch_gemm_partials(const void* A, const void* Bm, int64_t M, int N, int K, float* part, int ksp,
+                                 unsigned* status, cudaStream_t s);
+// C = A·Bᵀ (or C += A·Bᵀ with `accumulate`) as launch_gemm_bf16 (A [M][K], B [N][K] bf16,
+// K-contiguous), C float32 [M][ldc], N a multiple of 4.
 cudaError_t launch_gemm_f32out(const void* A, const void* Bm, float* C, int64_t M, int N, int K, int64_t ldc,
-                               unsigned* status, cudaStream_t s);
+                               bool accumulate, unsigned* status, cudaStream_t s);
+// C = Aᵀ·B, float32 C [M][ldc]: A [K][lda] (M columns) and B [K][ldb] (N columns) bf16 row-major,
+// read in place as MN-major tensor-core operands (K = the reduction over rows, e.g. tokens).
+// lda, ldb multiples of 8, A and B 16-byte aligned.
+cudaError_t launch_gemm_f32out_mn(const void* A, int64_t lda, const void* Bm, int64_t ldb, float* C, int M, int N,
+                                  int64_t K, int64_t ldc, unsigned* status, cudaStream_t s);
+// C = A·[W0; W1] (or C += with `accumulate`), float32 C [M][ldc]: A [M][2·Kh] bf16 K-major,
+// W0 and W1 [Kh][N] bf16 row-major (the stacked matrix's first and second Kh rows), read in
+// place as an MN-major operand. Kh a multiple of 64, N of 8.
+cudaError_t launch_gemm_f32out_wcat(const void* A, const void* W0, const void* W1, float* C, int64_t M, int N,
+                                    int Kh, int64_t ldc, bool accumulate, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const void* Wa, const float* ba,
                                   const void* Wx, const float* bx, const float* cla, float* h, void* y_t, int B,
                                   int R, unsigned* status, cudaStream_t s);
@@ -148,17 +163,19 @@ struct AttnLayout {
   size_t off_qkv, off_q, off_op, off_m, off_l, off_o, off_part, bytes;
 };
 AttnLayout attn_layout(int B, int D, int W);
-// RoPE and ring writes of position `pos` from qkv (in the workspace), then the windowed
-// attention into the workspace's o. k_ring [B][W][128], v_ring [B][128][W] bf16, in place.
-cudaError_t launch_attention_core(const void* qkv, void* k_ring, void* v_ring, int64_t pos, int B, int D, int W,
-                                  const AttnLayout& L, void* ws, unsigned* status, cudaStream_t s);
+// RoPE and ring writes of position `pos` from the projection — qkv [B][(H+2)·128] bf16, or,
+// when qkv_part is not null, the sum of its ksp float32 slices (rounded to bf16 first) —
+// then the windowed attention into the workspace's o. k_ring, v_ring [B][W][128] bf16, in
+// place.
+cudaError_t launch_attention_core(const void* qkv, const float* qkv_part, int ksp, void* k_ring, void* v_ring,
+                                  int64_t pos, int B, int D, int W, const AttnLayout& L, void* ws, unsigned* status,
+                                  cudaStream_t s);
 
 // ---- backward (bf16 IO) --------------------------------------------------------------
 // Workspace of launch_backward: [status | u | z | chunk maps P, Q | chunk carries | ∂z |
-// direct ∂u (f32) | gate-GEMM ∂u (f32) | [W_a; W_x]ᵀ | ∂zᵀ | uᵀ | Σ ∂log a·r·c].
+// ∂u (f32: the direct term, then the gate GEMM's added) | [W_a; W_x]ᵀ | Σ ∂log a·r·c].
 struct BwdLayout {
-  size_t off_u, off_z, off_P, off_Q, off_gin, off_dz, off_du, off_dug, off_wt, off_dzt, off_ut, off_dL, bytes;
-  int64_t n_pad;  // tokens rounded up to 64 (the transposed operands' row length)
+  size_t off_u, off_z, off_P, off_Q, off_gin, off_dz, off_du, off_wt, off_dL, bytes;
   int n_chunks;
 };
 BwdLayout bwd_layout(int B, int T, int R);

@@ -179,6 +179,21 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory descriptor, 128-byte swizzle, MN-major: rows of 64 bf16 along M (or N), one
+// row per k, 8 rows (1024 B) to a swizzle atom along K (SBO), and the next 64 M (or N)
+// columns `lbo` bytes on.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);         // start address
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;      // leading byte offset: the next 64 columns
+  d |= (uint64_t)(1024 >> 4) << 32;                // stride byte offset: the next 8 rows of K
+  d |= (uint64_t)1 << 46;                          // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                          // layout: 128-byte swizzle
+  return d;
+}
+// Instruction-descriptor bits: A (bit 15) and B (bit 16) MN-major instead of K-major.
+constexpr uint32_t kIdescAMN = 1u << 15, kIdescBMN = 1u << 16;
+
 // Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 accumulator.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
   return (1u << 4)                       // D format: f32

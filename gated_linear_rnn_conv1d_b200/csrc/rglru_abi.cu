@@ -199,9 +199,13 @@ cudaError_t attention_sequence(const rglru_attention_weights* w, const void* x_t
   const int nqkv = (L.H + 2) * 128;
   void* qkv = bytes(ws) + L.off_qkv;
   float* part = reinterpret_cast<float*>(bytes(ws) + L.off_part);
-  cudaError_t e =
-      launch_gemm_bf16_skinny(x_t, w->W_qkv, qkv, B, nqkv, D, nqkv, part, kSplitPartBytes, status, s);
-  if (e == cudaSuccess) e = launch_attention_core(qkv, k_ring, v_ring, pos, B, D, window, L, ws, status, s);
+  // the projection split over K at a decode batch: its slices are summed by the RoPE kernel
+  const int ksp = skinny_splits(B, nqkv, D, kSplitPartBytes);
+  cudaError_t e = ksp > 1 ? launch_gemm_partials(x_t, w->W_qkv, B, nqkv, D, part, ksp, status, s)
+                          : launch_gemm_bf16(x_t, w->W_qkv, qkv, B, nqkv, D, nqkv, status, s);
+  if (e == cudaSuccess)
+    e = launch_attention_core(qkv, ksp > 1 ? part : nullptr, ksp, k_ring, v_ring, pos, B, D, window, L, ws, status,
+                              s);
   if (e == cudaSuccess)
     e = launch_gemm_bf16_skinny(bytes(ws) + L.off_o, w->W_o, out_t, B, D, L.H * 128, D, part, kSplitPartBytes,
                                 status, s);

@@ -382,9 +382,17 @@ class AttentionWeights:
 
 
 def attention_rings(B: int, window: int, device="cuda") -> Tuple[torch.Tensor, torch.Tensor]:
-    """Empty KV rings of the local attention: keys [B][window][128], values [B][128][window]."""
+    """Empty KV rings of the local attention: keys and values [B][window][128], slot-major."""
     return (torch.empty(B, window, 128, dtype=torch.bfloat16, device=device),
-            torch.empty(B, 128, window, dtype=torch.bfloat16, device=device))
+            torch.empty(B, window, 128, dtype=torch.bfloat16, device=device))
+
+
+def _check_rings(k_ring: torch.Tensor, v_ring: torch.Tensor, B: int) -> int:
+    W = k_ring.shape[1]
+    for r in (k_ring, v_ring):
+        if tuple(r.shape) != (B, W, 128) or not r.is_contiguous():
+            raise ValueError(f"KV rings must be contiguous [B][window][128], got {tuple(r.shape)}")
+    return W
 
 
 def attention_step_workspace_bytes(B: int, D: int, window: int) -> int:
@@ -397,7 +405,7 @@ def attention_step(weights: AttentionWeights, x_t: torch.Tensor, k_ring: torch.T
     """rglru_attention_step: x_t [B][D] → out_t [B][D] at position pos; the rings in place."""
     lib = _abi.load()
     B, D = x_t.shape
-    W = k_ring.shape[1]
+    W = _check_rings(k_ring, v_ring, B)
     out_t = torch.empty_like(x_t) if out_t is None else out_t
     ws = _workspace(lib.rglru_attention_step_workspace_bytes(B, D, W), x_t.device, workspace)
     st = weights.struct()
@@ -418,7 +426,7 @@ def attention_layer_step(weights: AttentionWeights, x_t: torch.Tensor, k_ring: t
     """rglru_attention_layer_step: Griffin's local-attention residual layer, one decode step."""
     lib = _abi.load()
     B, D = x_t.shape
-    W = k_ring.shape[1]
+    W = _check_rings(k_ring, v_ring, B)
     H = weights.W_gate.shape[0]
     out_t = torch.empty_like(x_t) if out_t is None else out_t
     ws = _workspace(lib.rglru_attention_layer_step_workspace_bytes(B, D, H, W), x_t.device, workspace)

@@ -226,9 +226,9 @@ RGLRU_API int rglru_layer_step(const rglru_params* params, const rglru_layer_wei
  *   weights.W_o    [D][H·128] bf16
  *   x_t, out_t     [B][D] bf16
  *   k_ring         [B][window][128] bf16, rotated keys, slot-major; updated IN PLACE
- *   v_ring         [B][128][window] bf16, values stored dimension-major (value d of slot s
- *                  at [b][d][s]); updated IN PLACE. Slots holding no position yet
- *                  (pos < window − 1) are never read, so the rings need no initialisation.
+ *   v_ring         [B][window][128] bf16, values, slot-major; updated IN PLACE. Slots
+ *                  holding no position yet (pos < window − 1) are never read, so the rings
+ *                  need no initialisation.
  *   pos            ≥ 0, the position of x_t; the rings hold positions pos − window … pos − 1
  *   workspace      at least rglru_attention_step_workspace_bytes(B, D, window) bytes,
  *                  256-byte aligned

@@ -27,8 +27,8 @@ def _host(w):
 
 
 def _rings_to_oracle(k_ring, v_ring):
-    """GPU rings (keys [B][W][128], values [B][128][W]) in the oracle's layout [B][W][128]."""
-    return f64(k_ring), f64(v_ring).transpose(0, 2, 1)
+    """GPU rings (keys and values [B][W][128]) as float64 arrays, the oracle's layout."""
+    return f64(k_ring), f64(v_ring)
 
 
 # (3, 256, 128, 300): two query heads (the MMA's N padded to 16), a 128-slot window that
@@ -91,7 +91,7 @@ def test_attention_step_full_window_at_scale():
     k0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
     v0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
     k_ring = k0.to(DEV).contiguous()
-    v_ring = v0.transpose(1, 2).contiguous().to(DEV)
+    v_ring = v0.to(DEV).contiguous()
     rows = np.array(sorted(set([0, B - 1]) | set(np.random.default_rng(7).choice(B, 30, replace=False).tolist())))
     K_o, V_o = f64(k0)[rows], f64(v0)[rows]
     ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=DEV)
@@ -101,6 +101,28 @@ def test_attention_step_full_window_at_scale():
         out_o, K_o, V_o = oracle.local_attention_step(f64(xt)[rows], K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"],
                                                       hw["W_o"], W)
         assert rel(out[torch.from_numpy(rows).to(DEV)], out_o) <= TOL_ATTN, t
+    assert rglru.workspace_status(ws) == 0
+
+
+def test_attention_step_long_window_many_partials():
+    """One sequence, window 16384 (128 ring chunks, 128 partial outputs merged per head),
+    D = 4096: rings filled with seeded keys and values; steps 16380 … 16388 cross the wrap."""
+    B, D, W = 1, 4096, 16384
+    w = inputs.make_attention(D, seed=8)
+    aw = rglru.AttentionWeights.from_host(w)
+    hw = _host(w)
+    g = torch.Generator("cpu").manual_seed(9)
+    k0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
+    v0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
+    k_ring = k0.to(DEV).contiguous()
+    v_ring = v0.to(DEV).contiguous()
+    K_o, V_o = f64(k0), f64(v0)
+    ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=DEV)
+    for t in range(W - 4, W + 5):
+        xt = inputs.decode_token(t, B, D)
+        out = rglru.attention_step(aw, xt.to(DEV), k_ring, v_ring, t, workspace=ws)
+        out_o, K_o, V_o = oracle.local_attention_step(xt, K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"], hw["W_o"], W)
+        assert rel(out, out_o) <= TOL_ATTN, t
     assert rglru.workspace_status(ws) == 0
 
 
