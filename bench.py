@@ -617,7 +617,8 @@ def run_backward(c, reps=5):
     del ws, x, y, dy
     return {"workload": f"RG-LRU backward B={B} T={T} D_RNN={R} bf16 (dL/dy given)", "ms_per_call": ms,
             "tokens_per_s": world * n_tok / (ms / 1e3), "gemm_flops_per_call": flops,
-            "gemm_TFLOP/s_over_the_call": flops / ms / 1e9, "status": status, "gpu_launches_per_call": 14,
+            # launches: conv, z GEMM, maps, carries, replay, ∂Λ, ∂u GEMM, 2 ∂W GEMMs, conv backward
+            "gemm_TFLOP/s_over_the_call": flops / ms / 1e9, "status": status, "gpu_launches_per_call": 10,
             "timing": f"{reps} calls, L2 flushed before each"}
 
 

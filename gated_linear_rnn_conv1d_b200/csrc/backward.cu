@@ -10,7 +10,7 @@
 //   ∂z_a = ∂log a_t·r_t · c log σ(Λ) · (1 − r_t),  ∂z_x = ∂i_t i_t (1 − i_t),
 //   ∂ℓ/∂(log σ(Λ)) = Σ ∂log a_t·r_t · c,  ∂Λ = that · σ(−Λ).
 //
-// The reverse recurrence g_t = dy_t + a_{t+1} g_{t+1} is linear in g, so it runs in 64-step
+// The reverse recurrence g_t = dy_t + a_{t+1} g_{t+1} is linear in g, so it runs in kBwdTC-step
 // chunks like the forward scan: each chunk folds itself into a map g_{t0} = P g_{t1} + Q
 // (bwd_maps_kernel); a short sequential pass per (row, channel) hands every chunk the g
 // entering it from the right (bwd_carries_kernel); each chunk then replays its steps with
@@ -29,6 +29,7 @@ namespace rglru {
 namespace {
 
 constexpr int kBwdThreads = 128;  // threads per block; each thread takes 2 channels
+constexpr int kBwdTC = 64;        // time steps per chunk of the reverse recurrence
 
 __device__ __forceinline__ float2 ld_bf2(const __nv_bfloat16* p) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
@@ -54,7 +55,7 @@ struct BwdDims {
   int64_t pitch;  // packed gate row
 };
 
-// Pass 1: the map g_{t0} = P·g_{t1} + Q of each 64-step chunk [t0, t1).
+// Pass 1: the map g_{t0} = P·g_{t1} + Q of each chunk [t0, t1) of kBwdTC steps.
 __global__ void __launch_bounds__(kBwdThreads) bwd_maps_kernel(const __nv_bfloat16* __restrict__ z,
                                                                const __nv_bfloat16* __restrict__ dy,
                                                                const float* __restrict__ Lambda, float* __restrict__ P,
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_maps_kernel(const __nv_bfloat
   const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
   if (c >= d.R) return;
   const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
-  const int t0 = chunk * kScanTC, t1 = min(t0 + kScanTC, d.T);
+  const int t0 = chunk * kBwdTC, t1 = min(t0 + kBwdTC, d.T);
   const float cl0 = decay_log_coeff(Lambda[c]), cl1 = decay_log_coeff(Lambda[c + 1]);
   const __nv_bfloat16* zb = z + (int64_t)b * d.T * d.pitch + zcol(c);
   const __nv_bfloat16* dyb = dy + (int64_t)b * d.T * d.R + c;
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_carries_kernel(const float* _
   if (c >= d.R) return;
   const int b = blockIdx.y;
   float2 G = dh_T != nullptr ? *reinterpret_cast<const float2*>(dh_T + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
+#pragma unroll 8
   for (int chunk = d.n_chunks - 1; chunk >= 0; --chunk) {
     const int64_t o = ((int64_t)b * d.n_chunks + chunk) * d.R + c;
     *reinterpret_cast<float2*>(gin + o) = G;
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
   const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
   if (c >= d.R) return;
   const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
-  const int t0 = chunk * kScanTC, t1 = min(t0 + kScanTC, d.T);
+  const int t0 = chunk * kBwdTC, t1 = min(t0 + kBwdTC, d.T);
   const float cl[2] = {decay_log_coeff(a.Lambda[c]), decay_log_coeff(a.Lambda[c + 1])};
   const int64_t row0 = (int64_t)b * d.T;
   const __nv_bfloat16* zb = a.z + row0 * d.pitch + zcol(c);
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, Bw
   const int c = 2 * (blockIdx.x * kBwdThreads + threadIdx.x);
   if (c >= d.R) return;
   const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
-  const int t0 = chunk * kScanTC, t1 = min(t0 + kScanTC, d.T);
+  const int t0 = chunk * kBwdTC, t1 = min(t0 + kBwdTC, d.T);
   const int64_t base = (int64_t)b * d.T * d.R + c;
   float w[4][2];
 #pragma unroll
@@ -279,23 +281,35 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, Bw
   for (int j = 0; j < 4; ++j) dwin[j] = du_at(t0 + j);
   for (int j = 0; j < 3; ++j) xwin[j] = x_at(t0 - 3 + j);
   float sw[4][2] = {}, sb[2] = {0.f, 0.f};
-  for (int t = t0; t < t1; ++t) {
-    xwin[3] = x_at(t);
-    float dxv[2];
+  // eight steps at a time: their x and the ∂u entering the window loaded together first
+  for (int tb = t0; tb < t1; tb += 8) {
+    float2 xb[8], db[8];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float dut = j ? dwin[0].y : dwin[0].x;
-      float acc = 0.f;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc = fmaf(w[k][j], j ? dwin[3 - k].y : dwin[3 - k].x, acc);
-      dxv[j] = acc;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) sw[k][j] = fmaf(dut, j ? xwin[k].y : xwin[k].x, sw[k][j]);
-      sb[j] += dut;
+    for (int j = 0; j < 8; ++j) {
+      xb[j] = tb + j < t1 ? x_at(tb + j) : make_float2(0.f, 0.f);
+      db[j] = tb + j < t1 ? du_at(tb + j + 4) : make_float2(0.f, 0.f);
     }
-    st_bf2(a.dx + base + (int64_t)t * d.R, dxv[0], dxv[1]);
-    for (int j = 0; j < 3; ++j) { dwin[j] = dwin[j + 1]; xwin[j] = xwin[j + 1]; }
-    dwin[3] = du_at(t + 4);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int t = tb + jj;
+      if (t >= t1) break;
+      xwin[3] = xb[jj];
+      float dxv[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float dut = j ? dwin[0].y : dwin[0].x;
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc = fmaf(w[k][j], j ? dwin[3 - k].y : dwin[3 - k].x, acc);
+        dxv[j] = acc;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sw[k][j] = fmaf(dut, j ? xwin[k].y : xwin[k].x, sw[k][j]);
+        sb[j] += dut;
+      }
+      st_bf2(a.dx + base + (int64_t)t * d.R, dxv[0], dxv[1]);
+      for (int j = 0; j < 3; ++j) { dwin[j] = dwin[j + 1]; xwin[j] = xwin[j + 1]; }
+      dwin[3] = db[jj];
+    }
   }
   if (chunk == 0 && a.dstate0 != nullptr) {
     // history slot s = 0, 1, 2 holds x_{s−3}: its gradient is Σ_k w_k du_{s−k}, 0 ≤ s−k < T
@@ -365,7 +379,7 @@ cudaError_t transpose_bf16(const void* in, void* out, int64_t rows, int64_t cols
 BwdLayout bwd_layout(int B, int T, int R) {
   BwdLayout L;
   const int64_t n = (int64_t)B * T;
-  const int n_chunks = (T + kScanTC - 1) / kScanTC;
+  const int n_chunks = (T + kBwdTC - 1) / kBwdTC;
   auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
   size_t o = 256;  // status word
   L.off_u = o;      o += r256((size_t)n * R * 2);
