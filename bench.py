@@ -599,23 +599,38 @@ def run_backward(c, reps=5):
     g = torch.Generator("cpu").manual_seed(1)
     dy = torch.randn(B, T, R, generator=g).to(torch.bfloat16).to(dev)
     ws = torch.empty(rglru.backward_workspace_bytes(B, T, R), dtype=torch.uint8, device=dev)
-    for _ in range(2):
-        rglru.backward(p, x, y, dy, workspace=ws)
-    torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-    for a, b in evs:
-        flush()
-        a.record(stream)
-        rglru.backward(p, x, y, dy, workspace=ws)
-        b.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / reps)
+    fws = torch.empty(rglru.forward_workspace_bytes(B, T, R, torch.bfloat16), dtype=torch.uint8, device=dev)
+    saved = torch.empty(rglru.saved_bytes(B, T, R), dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in evs:
+            flush()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / reps)
+
+    ms = timed(lambda: rglru.backward(p, x, y, dy, workspace=ws))
+    # the training pair: the forward also saves the gate pre-activations, the backward
+    # reads them instead of recomputing them
+    fwd_ms = timed(lambda: rglru.forward(p, x, workspace=fws))
+    fwd_train_ms = timed(lambda: rglru.forward_train(p, x, workspace=fws, saved=saved))
+    ms_saved = timed(lambda: rglru.backward(p, x, y, dy, workspace=ws, saved=saved))
     n_tok = B * T
     # tensor-core work: z recomputed (2·N·2R·R), ∂u (2·N·2R·R), ∂W_a and ∂W_x (2·2R·R·N)
     flops = 3 * 2.0 * n_tok * (2 * R) * R
-    status = rglru.workspace_status(ws)
-    del ws, x, y, dy
+    status = rglru.workspace_status(ws) | rglru.workspace_status(fws)
+    del ws, fws, saved, x, y, dy
     return {"workload": f"RG-LRU backward B={B} T={T} D_RNN={R} bf16 (dL/dy given)", "ms_per_call": ms,
+            "training_pair": {"forward_ms": fwd_ms, "forward_train_ms": fwd_train_ms, "backward_saved_ms": ms_saved,
+                              "saved_bytes": rglru.saved_bytes(B, T, R),
+                              "note": "rglru_forward_train also writes the gate pre-activations; "
+                                      "rglru_backward_saved reads them instead of its z GEMM (9 launches)"},
             "tokens_per_s": world * n_tok / (ms / 1e3), "gemm_flops_per_call": flops,
             # launches: conv, z GEMM, maps, carries, replay, ∂Λ, ∂u GEMM, 2 ∂W GEMMs, conv backward
             "gemm_TFLOP/s_over_the_call": flops / ms / 1e9, "status": status, "gpu_launches_per_call": 10,

@@ -89,6 +89,9 @@ SIGNATURES = {
     "rglru_gemm_bf16": (_I, [_P, _P, _P, _L, _I, _I, _P]),
     "rglru_backward_workspace_bytes": (_S, [_I, _I, _I]),
     "rglru_backward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _GP, _I, _I, _I, _P, _S, _P]),
+    "rglru_saved_bytes": (_S, [_I, _I, _I]),
+    "rglru_forward_train": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _S, _P]),
+    "rglru_backward_saved": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _GP, _I, _I, _I, _P, _S, _P]),
     "rglru_gate_scan_workspace_bytes": (_S, [_I, _I, _I, _I]),
     "rglru_gate_scan": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "rglru_workspace_status": (_I, [_P, _P]),

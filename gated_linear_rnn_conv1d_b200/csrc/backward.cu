@@ -402,7 +402,7 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   const int B = g.B, T = g.T, R = g.R;
   const int64_t n = (int64_t)B * T;
   void* u = w + L.off_u;
-  void* z = w + L.off_z;
+  void* z = g.z_saved != nullptr ? const_cast<void*>(g.z_saved) : static_cast<void*>(w + L.off_z);
   float* P = reinterpret_cast<float*>(w + L.off_P);
   float* Q = reinterpret_cast<float*>(w + L.off_Q);
   float* gin = reinterpret_cast<float*>(w + L.off_gin);
@@ -418,10 +418,13 @@ cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cuda
   if ((e = cudaMemsetAsync(g.db_x, 0, (size_t)R * 4, s)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(g.dconv_w, 0, (size_t)4 * R * 4, s)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(g.dconv_b, 0, (size_t)R * 4, s)) != cudaSuccess) return e;
-  // recompute u = Conv1D(x) and the packed pre-activations z (with biases)
+  // recompute u = Conv1D(x) and (unless the forward saved them) the packed pre-activations
+  // z (with biases)
   if ((e = launch_conv1d(g.conv_w, g.conv_b, g.x, g.state0, u, nullptr, B, T, R, true, status, s)) != cudaSuccess)
     return e;
-  if ((e = launch_gemm_gates_bf16(u, g.W_a, g.b_a, g.W_x, g.b_x, z, n, R, status, s)) != cudaSuccess) return e;
+  if (g.z_saved == nullptr && (e = launch_gemm_gates_bf16(u, g.W_a, g.b_a, g.W_x, g.b_x, z, n, R, status, s)) !=
+                                   cudaSuccess)
+    return e;
   BwdDims d{B, T, R, L.n_chunks, gate_pitch(R)};
   const unsigned gx = (unsigned)((R / 2 + kBwdThreads - 1) / kBwdThreads);
   const dim3 g_chunks(gx, (unsigned)(B * L.n_chunks)), g_rows(gx, (unsigned)B);

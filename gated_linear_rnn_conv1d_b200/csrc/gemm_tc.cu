@@ -70,6 +70,9 @@ struct EpiArgs {
   // b_split_k > 0 (a multiple of BK), B's rows k ≥ b_split_k come from the second B map, at
   // row k − b_split_k: B = [B0; B1] stacked along K.
   int a_mn, b_mn, b_split_k;
+  // COEF: the pre-activations z (with biases, bf16, the packed layout of C) stored as well
+  // when not null — bit for bit what EPI_GATES writes for the same operands
+  __nv_bfloat16* z_out;
   // STORE_F32: C += A·Bᵀ (C read before it is written, element by element) instead of C = A·Bᵀ
   int accumulate;
 };
@@ -699,7 +702,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
           const int c0 = chalf * 64 + k * 16;
           const uint32_t uw[8] = {uq[2 * k].x, uq[2 * k].y, uq[2 * k].z, uq[2 * k].w,
                                   uq[2 * k + 1].x, uq[2 * k + 1].y, uq[2 * k + 1].z, uq[2 * k + 1].w};
-          uint32_t dh[8], mh[8];
+          uint32_t dh[8], mh[8], zah[8], zxh[8];
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
             const int c = c0 + j;
@@ -708,6 +711,8 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
                 make_float2(__uint_as_float(ra[cur][j]) + sPar[c], __uint_as_float(ra[cur][j + 1]) + sPar[c + 1]);
             const float2 zx = make_float2(__uint_as_float(rx[cur][j]) + sPar[128 + c],
                                           __uint_as_float(rx[cur][j + 1]) + sPar[128 + c + 1]);
+            zah[j / 2] = pack_bf16x2(za.x, za.y);
+            zxh[j / 2] = pack_bf16x2(zx.x, zx.y);
             float2 d, m;
             gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), u2, d, m);
             const __half2 dd = __floats2half2_rn(d.x, d.y);
@@ -722,6 +727,14 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
             pd[1] = make_uint4(dh[4], dh[5], dh[6], dh[7]);
             pm[0] = make_uint4(mh[0], mh[1], mh[2], mh[3]);
             pm[1] = make_uint4(mh[4], mh[5], mh[6], mh[7]);
+            if (ep.z_out != nullptr) {  // the pre-activations, saved for the backward
+              uint4* za4 = reinterpret_cast<uint4*>(ep.z_out + row * ep.ldc + (int64_t)n_blk * BN + c0);
+              uint4* zx4 = reinterpret_cast<uint4*>(ep.z_out + row * ep.ldc + (int64_t)n_blk * BN + 128 + c0);
+              za4[0] = make_uint4(zah[0], zah[1], zah[2], zah[3]);
+              za4[1] = make_uint4(zah[4], zah[5], zah[6], zah[7]);
+              zx4[0] = make_uint4(zxh[0], zxh[1], zxh[2], zxh[3]);
+              zx4[1] = make_uint4(zxh[4], zxh[5], zxh[6], zxh[7]);
+            }
           }
           if (k + 1 < 4) tmem_ld_wait16(ra[cur ^ 1], rx[cur ^ 1]);
         }
@@ -1427,7 +1440,8 @@ cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* b
 }
 
 cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
-                                    const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s) {
+                                    const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s,
+                                    void* z_out) {
   // the gate GEMM's tiles, with the recurrence coefficients formed in the epilogue
   CUtensorMap ma, mb0, mb1;
   if (!make_map_2d(&ma, u, R, M, (uint64_t)R * 2, BK, BM)) return cudaErrorInvalidValue;
@@ -1441,6 +1455,7 @@ cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* 
   ep.Lambda = Lambda;
   ep.R = R;
   ep.ub = static_cast<const __nv_bfloat16*>(u);
+  ep.z_out = static_cast<__nv_bfloat16*>(z_out);
   const int n_tiles_n = (R + 127) / 128;
   return launch_tc2<EPI_COEF, true>(ma, mb0, mb1, M, R, n_tiles_n, ep, status, s);
 }

@@ -79,8 +79,11 @@ int num_sms();
 // The gate GEMM with the recurrence coefficients formed in its epilogue: g packed like z,
 // d = 1 − a_t (fp16) in the z_a places and b_t = √(1−a_t²)·i_t·u_t (bf16) in the z_x places (the
 // epilogue reads its rows of u, the GEMM's A operand).
+// z_out, when not null, receives the pre-activations z in the packed layout of g (what
+// launch_gemm_gates_bf16 writes, bit for bit).
 cudaError_t launch_gemm_coeffs_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
-                                    const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s);
+                                    const float* Lambda, void* g, int64_t M, int R, unsigned* status, cudaStream_t s,
+                                    void* z_out = nullptr);
 cudaError_t launch_gemm_gates_bf16(const void* u, const void* Wa, const float* ba, const void* Wx, const float* bx,
                                    void* z, int64_t M, int R, unsigned* status, cudaStream_t s);
 cudaError_t launch_gemm_bf16(const void* A, const void* Bm, void* C, int64_t M, int N, int K, int64_t ldc,
@@ -203,6 +206,7 @@ struct BwdArgs {
   float* db_x;
   float* dLambda;
   float* dh0;           // [B][R] or null
+  const void* z_saved;  // the forward's pre-activations [B·T][gate_pitch(R)] bf16, or null (recomputed)
   int B, T, R;
 };
 cudaError_t launch_backward(const BwdArgs& g, const BwdLayout& L, void* ws, cudaStream_t s);

@@ -537,10 +537,10 @@ int rglru_scan_coeffs(const void* g, const float* h0, const void* gate_g, void* 
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
-int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
-                  float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype, void* workspace,
-                  size_t workspace_bytes, rglru_stream_t stream) {
-  const Range range("rglru_forward");
+namespace {
+int forward_impl(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
+                 float* h_T, void* conv_state_T, void* saved, int B, int T, int R, int io_dtype, void* workspace,
+                 size_t workspace_bytes, rglru_stream_t stream) {
   if (!valid_dtype(io_dtype)) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
@@ -567,7 +567,7 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   // bf16: the gate GEMM's epilogue forms the recurrence coefficients (d, b) directly
   if (bf16)
     e = launch_gemm_coeffs_bf16(u, params->W_a, params->b_a, params->W_x, params->b_x, params->Lambda, z,
-                                (int64_t)B * T, R, status, s);
+                                (int64_t)B * T, R, status, s, saved);
   else
     e = launch_gemm_gates_f32(static_cast<const float*>(u), static_cast<const float*>(params->W_a), params->b_a,
                               static_cast<const float*>(params->W_x), params->b_x, static_cast<float*>(z),
@@ -576,6 +576,30 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   e = run_scan(params, x, z, gate_pitch(R), conv_state0, h0, nullptr, y, h_T, B, T, R, bf16, L.scan, workspace,
                false, s, bf16);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+}  // namespace
+
+int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
+                  float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype, void* workspace,
+                  size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_forward");
+  return forward_impl(params, x, h0, conv_state0, y, h_T, conv_state_T, nullptr, B, T, R, io_dtype, workspace,
+                      workspace_bytes, stream);
+}
+
+size_t rglru_saved_bytes(int B, int T, int R) {
+  if (!valid_R(R) || !valid_tokens(B, T)) return 0;
+  return (size_t)B * T * gate_pitch(R) * 2;
+}
+
+int rglru_forward_train(const rglru_params* params, const void* x, const float* h0, const void* conv_state0, void* y,
+                        float* h_T, void* conv_state_T, void* saved, int B, int T, int R, void* workspace,
+                        size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_forward_train");
+  if (saved == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(saved)) return RGLRU_ERR_ALIGN;
+  return forward_impl(params, x, h0, conv_state0, y, h_T, conv_state_T, saved, B, T, R, RGLRU_BF16, workspace,
+                      workspace_bytes, stream);
 }
 
 int rglru_step(const rglru_params* params, const void* x_t, void* conv_state, float* h, void* y_t, int B, int R,
@@ -622,19 +646,17 @@ size_t rglru_backward_workspace_bytes(int B, int T, int R) {
   return bwd_layout(B, T, R).bytes;
 }
 
-int rglru_backward(const rglru_params* params, const void* x, const void* y, const void* dy, const float* h0,
-                   const float* dh_T, const void* conv_state0, const rglru_grads* grads, int B, int T, int R,
-                   void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
-  const Range range("rglru_backward");
+namespace {
+int backward_impl(const rglru_params* params, const void* x, const void* y, const void* dy, const float* h0,
+                  const float* dh_T, const void* conv_state0, const void* saved, const rglru_grads* grads, int B,
+                  int T, int R, void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
   if (!valid_R(R) || !valid_tokens(B, T)) return RGLRU_ERR_SHAPE;
-  // the transposed token axis of the weight-gradient GEMMs (and its 32-row transpose
-  // tiles) must stay within int32 and the grid's y limit
-  if ((int64_t)B * T > (int64_t)65535 * 32 - 64) return RGLRU_ERR_SHAPE;
   // the chunked kernels index (batch row, 64-step chunk) with the grid's y dimension
   if ((int64_t)B * ((T + kScanTC - 1) / kScanTC) > 65535) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
   if (st != RGLRU_OK) return st;
   if (x == nullptr || y == nullptr || dy == nullptr || grads == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(saved)) return RGLRU_ERR_ALIGN;
   const rglru_grads& g = *grads;
   if (g.dx == nullptr || g.dconv_w == nullptr || g.dconv_b == nullptr || g.dW_a == nullptr || g.db_a == nullptr ||
       g.dW_x == nullptr || g.db_x == nullptr || g.dLambda == nullptr)
@@ -654,9 +676,28 @@ int rglru_backward(const rglru_params* params, const void* x, const void* y, con
   a.W_x = params->W_x; a.b_x = params->b_x; a.Lambda = params->Lambda;
   a.dx = g.dx; a.dstate0 = g.dconv_state0; a.dconv_w = g.dconv_w; a.dconv_b = g.dconv_b; a.dW_a = g.dW_a;
   a.db_a = g.db_a; a.dW_x = g.dW_x; a.db_x = g.db_x; a.dLambda = g.dLambda; a.dh0 = g.dh0;
+  a.z_saved = saved;
   a.B = B; a.T = T; a.R = R;
   cudaError_t e = launch_backward(a, L, workspace, (cudaStream_t)stream);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+}
+}  // namespace
+
+int rglru_backward(const rglru_params* params, const void* x, const void* y, const void* dy, const float* h0,
+                   const float* dh_T, const void* conv_state0, const rglru_grads* grads, int B, int T, int R,
+                   void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_backward");
+  return backward_impl(params, x, y, dy, h0, dh_T, conv_state0, nullptr, grads, B, T, R, workspace, workspace_bytes,
+                       stream);
+}
+
+int rglru_backward_saved(const rglru_params* params, const void* x, const void* y, const void* dy, const float* h0,
+                         const float* dh_T, const void* conv_state0, const void* saved, const rglru_grads* grads,
+                         int B, int T, int R, void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
+  const Range range("rglru_backward_saved");
+  if (saved == nullptr) return RGLRU_ERR_NULL;
+  return backward_impl(params, x, y, dy, h0, dh_T, conv_state0, saved, grads, B, T, R, workspace, workspace_bytes,
+                       stream);
 }
 
 int rglru_block_forward(const rglru_params* params, const void* W_1, const void* W_2, const void* W_o, const void* x,

@@ -96,6 +96,29 @@ def forward(params: Params, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
     return y, h_T, conv_state_T
 
 
+def saved_bytes(B: int, T: int, R: int) -> int:
+    return _abi.load().rglru_saved_bytes(B, T, R)
+
+
+def forward_train(params: Params, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                  conv_state0: Optional[torch.Tensor] = None, *, workspace: Optional[torch.Tensor] = None,
+                  saved: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """rglru_forward_train (bf16 IO): as forward, and the gate pre-activations saved for
+    backward(..., saved=...). Returns (y, h_T, conv_state_T, saved)."""
+    lib = _abi.load()
+    B, T, R = x.shape
+    y = torch.empty_like(x)
+    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device)
+    conv_state_T = torch.empty(B, 3, R, dtype=x.dtype, device=x.device)
+    saved = _workspace(lib.rglru_saved_bytes(B, T, R), x.device, saved)
+    ws = _workspace(lib.rglru_forward_workspace_bytes(B, T, R, _abi.RGLRU_BF16), x.device, workspace)
+    st = params.struct()
+    _abi.check("rglru_forward_train", lib.rglru_forward_train(
+        ctypes.byref(st), _p(x), _p(h0), _p(conv_state0), _p(y), _p(h_T), _p(conv_state_T), _p(saved), B, T, R,
+        _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+    return y, h_T, conv_state_T, saved
+
+
 def backward_workspace_bytes(B: int, T: int, R: int) -> int:
     return _abi.load().rglru_backward_workspace_bytes(B, T, R)
 
@@ -103,11 +126,13 @@ def backward_workspace_bytes(B: int, T: int, R: int) -> int:
 def backward(params: Params, x: torch.Tensor, y: torch.Tensor, dy: torch.Tensor, h0: Optional[torch.Tensor] = None,
              dh_T: Optional[torch.Tensor] = None, conv_state0: Optional[torch.Tensor] = None, *,
              want_dh0: bool = True, want_dconv_state0: bool = True, workspace: Optional[torch.Tensor] = None,
-             stream: Optional[torch.cuda.Stream] = None) -> dict:
+             saved: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> dict:
     """rglru_backward (bf16 IO): gradients of a loss with ∂ℓ/∂y = dy (and ∂ℓ/∂h_T = dh_T)
     for the forward that mapped x (with h0, conv_state0) to y. Returns a dict with dx
     [B][T][R] bf16, dconv_state0 [B][3][R] bf16 (or None), dconv_w [4][R], dconv_b, dW_a,
-    db_a, dW_x, db_x, dLambda and dh0 [B][R] (or None), all float32 but dx and dconv_state0."""
+    db_a, dW_x, db_x, dLambda and dh0 [B][R] (or None), all float32 but dx and dconv_state0.
+    With `saved` (from forward_train) the gate pre-activations are read, not recomputed
+    (rglru_backward_saved)."""
     lib = _abi.load()
     B, T, R = x.shape
     dev = x.device
@@ -125,9 +150,14 @@ def backward(params: Params, x: torch.Tensor, y: torch.Tensor, dy: torch.Tensor,
                                                   "db_x", "dLambda", "dh0")))
     ws = _workspace(lib.rglru_backward_workspace_bytes(B, T, R), dev, workspace)
     st = params.struct()
-    _abi.check("rglru_backward", lib.rglru_backward(
-        ctypes.byref(st), _p(x), _p(y), _p(dy), _p(h0), _p(dh_T), _p(conv_state0), ctypes.byref(g), B, T, R, _p(ws),
-        ws.numel() * ws.element_size(), _s(stream)))
+    if saved is None:
+        _abi.check("rglru_backward", lib.rglru_backward(
+            ctypes.byref(st), _p(x), _p(y), _p(dy), _p(h0), _p(dh_T), _p(conv_state0), ctypes.byref(g), B, T, R,
+            _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+    else:
+        _abi.check("rglru_backward_saved", lib.rglru_backward_saved(
+            ctypes.byref(st), _p(x), _p(y), _p(dy), _p(h0), _p(dh_T), _p(conv_state0), _p(saved), ctypes.byref(g),
+            B, T, R, _p(ws), ws.numel() * ws.element_size(), _s(stream)))
     return out
 
 

@@ -277,7 +277,8 @@ RGLRU_API int rglru_attention_layer_step(const rglru_attention_layer_weights* we
  *   ∂z_x = g √(1−a_t²) u_t · i_t (1 − i_t),  ∂u_t = g √(1−a_t²) i_t + ∂z_a W_a + ∂z_x W_x,
  *   ∂W_a = Σ_t ∂z_aᵀ u_t, ∂b_a = Σ_t ∂z_a (same for x), ∂Λ = Σ (∂log a_t) c r_t · σ(−Λ),
  *   ∂h0 = a_0 g_0, and the Conv1D's transpose for ∂x, the taps, the bias and the history.
- * u and the gate pre-activations are recomputed from x; h_{t-1} is read from y.
+ * u and the gate pre-activations are recomputed from x (or, in rglru_backward_saved, the
+ * pre-activations come from rglru_forward_train); h_{t-1} is read from y.
  *   params        as rglru_forward (W_a, W_x bf16)
  *   x             [B][T][R] bf16, the forward's input
  *   y             [B][T][R] bf16, the forward's output for the same x, h0, conv_state0
@@ -290,7 +291,7 @@ RGLRU_API int rglru_attention_layer_step(const rglru_attention_layer_weights* we
  *                 [B][3][R] bf16 or NULL; dconv_w [4][R], dconv_b, db_a, db_x, dLambda [R],
  *                 dW_a, dW_x [R][R] (row-major [out][in]) and dh0 [B][R] (or NULL) float32
  *   workspace     at least rglru_backward_workspace_bytes(B, T, R) bytes, 256-byte aligned
- * Shapes: as rglru_forward, and B·T ≤ 2,097,056 and B·⌈T/64⌉ ≤ 65535 (RGLRU_ERR_SHAPE).
+ * Shapes: as rglru_forward, and B·⌈T/64⌉ ≤ 65535 (RGLRU_ERR_SHAPE).
  * The accumulated outputs (the taps, biases and Λ) are summed with atomics, so their
  * last bits may vary between runs; everything else is deterministic.
  * --------------------------------------------------------------------------------- */
@@ -310,6 +311,24 @@ RGLRU_API size_t rglru_backward_workspace_bytes(int B, int T, int R);
 RGLRU_API int rglru_backward(const rglru_params* params, const void* x, const void* y, const void* dy,
                              const float* h0, const float* dh_T, const void* conv_state0, const rglru_grads* grads,
                              int B, int T, int R, void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+
+/* Training pair: rglru_forward_train is rglru_forward for bf16 IO that also writes the gate
+ * pre-activations z = u W_aᵀ + b_a, u W_xᵀ + b_x (bf16, in an internal packed layout) into
+ * `saved`, at least rglru_saved_bytes(B, T, R) bytes, 16-byte aligned (0 for invalid
+ * shapes). rglru_backward_saved is rglru_backward reading them from `saved` instead of
+ * recomputing them with the gate GEMM: the same inputs and outputs, bit for bit the same
+ * results (the saved values are those the recomputation forms). The pages keep the
+ * backward's inputs open; this pair trades rglru_saved_bytes of memory between the two calls
+ * for one of the backward's three gate-sized GEMMs. Errors as rglru_forward and
+ * rglru_backward, plus RGLRU_ERR_NULL for a null `saved`. */
+RGLRU_API size_t rglru_saved_bytes(int B, int T, int R);
+RGLRU_API int rglru_forward_train(const rglru_params* params, const void* x, const float* h0, const void* conv_state0,
+                                  void* y, float* h_T, void* conv_state_T, void* saved, int B, int T, int R,
+                                  void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+RGLRU_API int rglru_backward_saved(const rglru_params* params, const void* x, const void* y, const void* dy,
+                                   const float* h0, const float* dh_T, const void* conv_state0, const void* saved,
+                                   const rglru_grads* grads, int B, int T, int R, void* workspace,
+                                   size_t workspace_bytes, rglru_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * The stages of rglru_forward, callable one by one (for per-kernel timing and for

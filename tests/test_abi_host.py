@@ -156,6 +156,42 @@ def test_backward_rejects_bad_arguments_before_any_launch():
     assert call(wsb=wsb - 1) == -5
 
 
+def test_training_pair_rejects_bad_arguments_before_any_launch():
+    """rglru_forward_train / rglru_backward_saved: a null or misaligned `saved` and the
+    checks of the calls they extend, all before anything is launched."""
+    lib = _abi.load()
+    p = _params()
+    ok = _fake()
+    assert lib.rglru_saved_bytes(2, 64, 256) == 2 * 64 * lib.rglru_gate_pitch(256) * 2
+    assert lib.rglru_saved_bytes(1, 64, 264) == 64 * 768 * 2
+    assert lib.rglru_saved_bytes(2, 64, 12) == 0
+    assert lib.rglru_saved_bytes(0, 64, 256) == 0
+    fwb = lib.rglru_forward_workspace_bytes(1, 64, 256, 1)
+    ws = _fake(0x200000)
+
+    def fwd(**kw):
+        return lib.rglru_forward_train(kw.get("p", ctypes.byref(p)), kw.get("x", ok), None, None, kw.get("y", ok),
+                                       None, None, kw.get("saved", _fake(0x300000)), 1, kw.get("T", 64),
+                                       kw.get("R", 256), kw.get("ws", ws), kw.get("wsb", fwb), None)
+    assert fwd(saved=None) == -1
+    assert fwd(saved=_fake(0x300008)) == -3
+    assert fwd(R=12) == -2
+    assert fwd(y=None) == -1
+    assert fwd(wsb=fwb - 1) == -5
+    grads = _abi.RGLRUGrads(*([0x100000] * 10))
+    bwb = lib.rglru_backward_workspace_bytes(1, 64, 256)
+
+    def bwd(**kw):
+        return lib.rglru_backward_saved(ctypes.byref(p), kw.get("x", ok), ok, ok, None, None, None,
+                                        kw.get("saved", _fake(0x300000)), ctypes.byref(grads), 1, 64,
+                                        kw.get("R", 256), ws, kw.get("wsb", bwb), None)
+    assert bwd(saved=None) == -1
+    assert bwd(saved=_fake(0x300004)) == -3
+    assert bwd(R=12) == -2
+    assert bwd(x=None) == -1
+    assert bwd(wsb=bwb - 1) == -5
+
+
 def test_layer_rejects_bad_arguments_before_any_launch():
     lib = _abi.load()
     p = _params()

@@ -91,3 +91,28 @@ def test_backward_of_a_frozen_state():
     assert np.max(np.abs(f64(G["dh0"]) - expect)) <= 1e-4 * max(1.0, np.max(np.abs(expect)))
     for k in ("dx", "dconv_w", "dconv_b", "dW_x", "db_x", "dLambda", "dconv_state0"):
         assert float(torch.max(torch.abs(G[k].float()))) == 0.0, k
+
+
+@pytest.mark.parametrize("B,T,R,with_state", [(2, 200, 264, True), (2, 1024, 1024, True), (1, 65, 8, False)])
+def test_training_pair_equals_forward_and_backward(B, T, R, with_state):
+    """rglru_forward_train gives rglru_forward's outputs bit for bit and saves the gate
+    pre-activations the backward would recompute; rglru_backward_saved from them gives
+    rglru_backward's gradients — bit for bit for every gradient formed without atomics, to
+    float32 summation order for the ones accumulated with atomics (taps, biases, Λ)."""
+    w, h0, st0, dy, dh_T = _problem(B, T, R, with_state, seed=B * 100 + T + R + 5)
+    p = rglru.Params.from_host(w.params)
+    x = w.x.to(DEV)
+    y, hT, csT = rglru.forward(p, x, _dev(h0), _dev(st0))
+    y2, hT2, csT2, saved = rglru.forward_train(p, x, _dev(h0), _dev(st0))
+    assert torch.equal(y, y2) and torch.equal(hT, hT2) and torch.equal(csT, csT2)
+    assert saved.numel() == rglru.saved_bytes(B, T, R)
+    G = rglru.backward(p, x, y, dy.to(DEV), _dev(h0), dh_T.to(DEV), _dev(st0))
+    G2 = rglru.backward(p, x, y2, dy.to(DEV), _dev(h0), dh_T.to(DEV), _dev(st0), saved=saved)
+    assert rglru.workspace_status(None) == 0
+    for k in ("dx", "dconv_state0", "dW_a", "dW_x", "dh0"):
+        assert G[k] is None or torch.equal(G[k], G2[k]), k
+    for k in ("dconv_w", "dconv_b", "db_a", "db_x", "dLambda"):
+        assert rel(G2[k], G[k]) <= 1e-5, k
+    ref = oracle.rglru_backward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a, w.params.b_a, w.params.W_x,
+                                w.params.b_x, w.params.Lambda, dy, h0=h0, conv_state0=st0, dh_T=dh_T)
+    assert all(rel(G2[k], ref[k]) <= _tol(k) for k in KEYS if G2[k] is not None)
