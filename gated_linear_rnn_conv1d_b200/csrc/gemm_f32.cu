@@ -4,8 +4,11 @@
 // float32 accuracy (no TF32 rounding). Output in the packed gate layout: column
 // 256·(c/128) + (c%128) holds channel c's z_a, the same column + 128 its z_x.
 //
-// Classic register-tiled SIMT GEMM: a 64×64 output tile per 256-thread CTA, each thread a
-// 4×4 sub-tile, K staged through shared memory 16 at a time.
+// Register-tiled SIMT GEMM: a TM×TN output tile per 256-thread CTA (16×16 threads, each a
+// (TM/16)×(TN/16) sub-tile), K staged through shared memory 32 at a time in two buffers, the
+// next K tile's loads issued into registers before the current one is multiplied. 64×64
+// tiles when they fill the GPU twice over, 32×32 otherwise (small problems are latency-bound:
+// one float32 decode-size gate projection is 32 CTAs of 64×64 on a 148-SM part).
 #include <cstdint>
 
 #include "kernels.cuh"
@@ -13,14 +16,17 @@
 namespace rglru {
 namespace {
 
-constexpr int TM = 64, TN = 64, TK = 16;
+constexpr int TK = 32;
 
+template <int TM, int TN>
 __global__ void __launch_bounds__(256) gemm_gates_f32_kernel(const float* __restrict__ u, const float* __restrict__ Wa,
                                                             const float* __restrict__ ba, const float* __restrict__ Wx,
                                                             const float* __restrict__ bx, float* __restrict__ z,
                                                             int64_t M, int R, int64_t pitch) {
-  __shared__ float As[TK][TM + 4];
-  __shared__ float Bs[TK][TN + 4];
+  constexpr int RM = TM / 16, RN = TN / 16;           // per-thread sub-tile
+  constexpr int LA = TM * TK / 256, LB = TN * TK / 256;  // loads per thread per K tile
+  __shared__ float As[2][TK][TM + 4];
+  __shared__ float Bs[2][TK][TN + 4];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
   const int64_t m0 = (int64_t)blockIdx.y * TM;
   const int n0 = blockIdx.x * TN;  // packed column
@@ -31,43 +37,70 @@ __global__ void __launch_bounds__(256) gemm_gates_f32_kernel(const float* __rest
     ch = blk * 128 + (w % 128);
     return (w < 128) ? Wa : Wx;
   };
-
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < R; k0 += TK) {
-    // load A tile: 64 rows × 16 k (256 threads × 4 elements)
-    for (int i = threadIdx.x; i < TM * TK; i += 256) {
-      const int r = i / TK, k = i % TK;
+  // element i of this thread's share of a K tile: (row or column, k) with k fastest, so that
+  // 32 consecutive threads read 32 consecutive floats of one row
+  float ra[LA], rb[LB];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < LA; ++q) {
+      const int i = threadIdx.x + q * 256, r = i / TK, k = i % TK;
       const int64_t m = m0 + r;
-      As[k][r] = (m < M && k0 + k < R) ? u[m * R + k0 + k] : 0.0f;
+      ra[q] = (m < M && k0 + k < R) ? u[m * R + k0 + k] : 0.0f;
     }
-    for (int i = threadIdx.x; i < TN * TK; i += 256) {
-      const int c = i / TK, k = i % TK;
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int i = threadIdx.x + q * 256, c = i / TK, k = i % TK;
       int ch;
       const float* W = wrow(n0 + c, ch);
-      Bs[k][c] = (ch < R && k0 + k < R) ? W[(int64_t)ch * R + k0 + k] : 0.0f;
+      rb[q] = (ch < R && k0 + k < R) ? W[(int64_t)ch * R + k0 + k] : 0.0f;
     }
-    __syncthreads();
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int q = 0; q < LA; ++q) {
+      const int i = threadIdx.x + q * 256;
+      As[buf][i % TK][i / TK] = ra[q];
+    }
+#pragma unroll
+    for (int q = 0; q < LB; ++q) {
+      const int i = threadIdx.x + q * 256;
+      Bs[buf][i % TK][i / TK] = rb[q];
+    }
+  };
+
+  float acc[RM][RN] = {};
+  load(0);
+  store(0);
+  __syncthreads();
+  int buf = 0;
+  for (int k0 = 0; k0 < R; k0 += TK) {
+    const bool more = k0 + TK < R;
+    if (more) load(k0 + TK);  // in flight while this tile is multiplied
 #pragma unroll
     for (int k = 0; k < TK; ++k) {
-      float a[4], b[4];
+      float a[RM], b[RN];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[k][ty * 4 + i];
+      for (int i = 0; i < RM; ++i) a[i] = As[buf][k][ty * RM + i];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[k][tx * 4 + j];
+      for (int j = 0; j < RN; ++j) b[j] = Bs[buf][k][tx * RN + j];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < RM; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
-    __syncthreads();
+    if (more) {
+      store(buf ^ 1);  // the other buffer: its last readers passed the barrier below
+      __syncthreads();
+      buf ^= 1;
+    }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t m = m0 + ty * 4 + i;
+  for (int i = 0; i < RM; ++i) {
+    const int64_t m = m0 + ty * RM + i;
     if (m >= M) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
+    for (int j = 0; j < RN; ++j) {
+      const int n = n0 + tx * RN + j;
       const int blk = n / 256, w = n % 256;
       const int ch = blk * 128 + (w % 128);
       if (n < pitch && ch < R) z[m * pitch + n] = acc[i][j] + ((w < 128) ? ba[ch] : bx[ch]);
@@ -80,8 +113,14 @@ __global__ void __launch_bounds__(256) gemm_gates_f32_kernel(const float* __rest
 cudaError_t launch_gemm_gates_f32(const float* u, const float* Wa, const float* ba, const float* Wx,
                                   const float* bx, float* z, int64_t M, int R, cudaStream_t s) {
   const int64_t pitch = gate_pitch(R);
-  dim3 grid((unsigned)((pitch + TN - 1) / TN), (unsigned)((M + TM - 1) / TM));
-  gemm_gates_f32_kernel<<<grid, 256, 0, s>>>(u, Wa, ba, Wx, bx, z, M, R, pitch);
+  const int64_t big = ((pitch + 63) / 64) * ((M + 63) / 64);
+  if (big >= 2 * num_sms()) {
+    dim3 grid((unsigned)((pitch + 63) / 64), (unsigned)((M + 63) / 64));
+    gemm_gates_f32_kernel<64, 64><<<grid, 256, 0, s>>>(u, Wa, ba, Wx, bx, z, M, R, pitch);
+  } else {
+    dim3 grid((unsigned)((pitch + 31) / 32), (unsigned)((M + 31) / 32));
+    gemm_gates_f32_kernel<32, 32><<<grid, 256, 0, s>>>(u, Wa, ba, Wx, bx, z, M, R, pitch);
+  }
   return cudaGetLastError();
 }
 
