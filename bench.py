@@ -159,20 +159,21 @@ class Ctx:
 
 def _roofline(kern, dom, pk, workload):
     src = os.path.join(ROOT, "gated_linear_rnn_conv1d_b200", "csrc",
-                       {"gate_gemm": "gemm_tc.cu", "scan": "scan.cu", "conv1d": "conv.cu"}[dom])
+                       {"gate_gemm": "gemm_tc.cu", "gate_gemm_fused_scan": "gemm_tc.cu", "scan": "scan.cu",
+                        "conv1d": "conv.cu"}[dom])
     rec = NCU_TRAFFIC.get((workload, dom))
     traffic = rec["bytes_per_launch"] if rec and rec["src_sha256"] == _sha(src) else None
-    if dom == "gate_gemm":
+    if dom in ("gate_gemm", "gate_gemm_fused_scan"):
         roof = {"bound": "tensor", "achieved": kern[dom]["TFLOP/s"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": kern[dom]["GB/s"], "peak": pk["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic
     roof["kernel"] = dom
-    roof["algorithmic_per_launch"] = kern[dom]["flops" if dom == "gate_gemm" else "bytes"]
+    roof["algorithmic_per_launch"] = kern[dom]["flops" if roof["bound"] == "tensor" else "bytes"]
     roof["peak_source"] = ("measured: MEASURED_PEAKS.json burst figure" if pk["source"] == "measured"
                            else "fallback")
-    if dom == "gate_gemm" and pk.get("bf16_tflops_sustained"):
+    if roof["bound"] == "tensor" and pk.get("bf16_tflops_sustained"):
         # the GEMM runs power-capped (sw_power_cap) inside the step loop; its fraction of the
         # measured sustained figure, for context (frac above stays against the burst peak)
         roof["frac_of_sustained"] = roof["achieved"] / pk["bf16_tflops_sustained"]
@@ -199,11 +200,18 @@ def bench_forward(c, cfg, steps, warmup, seed=0, clocks=None):
     ws_fwd = torch.empty(rglru.forward_workspace_bytes(B, T, R, dt), dtype=torch.uint8, device=c.dev)
     stream, flush = c.stream, c.flush_l2
     bf = dt == torch.bfloat16
+    # rglru_forward's own kernels for this shape: Conv1D + the gate GEMM with the scan in its
+    # epilogue (2), or Conv1D + coefficient GEMM + scan (3)
+    n_kern = rglru.forward_kernels(B, T, R, dt)
+    fused = n_kern == 2
+    ws_f = torch.empty(rglru.gate_scan_workspace_bytes(B, T, R), dtype=torch.uint8, device=c.dev) \
+        if bf and T % 128 == 0 else None
 
     def forward_step():
         rglru.forward(p, x, workspace=ws_fwd, y=y, h_T=h_T, want_conv_state=False)
 
     def stages(ev):
+        # the separate path's three stage calls
         ev[0].record(stream)
         rglru.conv1d(p, x, u=u)
         ev[1].record(stream)
@@ -284,6 +292,30 @@ def bench_forward(c, cfg, steps, warmup, seed=0, clocks=None):
                                             "note": "timed apart; not part of the step"}
         status = status or rglru.workspace_status(ws_scan)
         del zp
+        if ws_f is not None:
+            # the gate GEMM with the scan fused into its epilogue (rglru_gate_scan, after the
+            # Conv1D stage): the coefficients never reach HBM
+            u3 = u.view(B, T, R)
+            for _ in range(2):
+                rglru.gate_scan(p, u3, workspace=ws_f, y=y, h_T=h_T)
+            fev = [c.events(3) for _ in range(ks)]
+            for k in range(ks):
+                flush()
+                fev[k][0].record(stream)
+                rglru.conv1d(p, x, u=u)
+                fev[k][1].record(stream)
+                rglru.gate_scan(p, u3, workspace=ws_f, y=y, h_T=h_T)
+                fev[k][2].record(stream)
+            torch.cuda.synchronize()
+            f_ms = sum(e[1].elapsed_time(e[2]) for e in fev) / ks
+            f_step = sum(e[0].elapsed_time(e[2]) for e in fev) / ks
+            kern["gate_gemm_fused_scan"] = {"ms": f_ms, "TFLOP/s": gemm_flops / f_ms / 1e9, "flops": gemm_flops,
+                                            "step_ms_with_conv": f_step,
+                                            "kernel": "rglru_gate_scan (tcgen05 2-SM, scan in the epilogue)",
+                                            "note": ("the step's second kernel" if fused else
+                                                     "timed apart; not the step's path at this shape") +
+                                                    "; its stage call includes a carry memset"}
+            status = status or rglru.workspace_status(ws_f)
     else:
         scan_bytes = tokens * R * 4 * 4                        # read x, z_a, z_x, write y (float32)
         kern["scan"] = {"ms": scan_ms, "GB/s": scan_bytes / scan_ms / 1e6, "bytes": scan_bytes,
@@ -293,11 +325,15 @@ def bench_forward(c, cfg, steps, warmup, seed=0, clocks=None):
             k["frac_hbm"] = k["GB/s"] / c.pk["hbm_gbs"]
         if "TFLOP/s" in k and bf:
             k["frac_tensor"] = k["TFLOP/s"] / c.pk["bf16_tflops"]
-    dom = max(("conv1d", "gate_gemm", "scan"), key=lambda k: kern[k]["ms"])
+    step_kernels = ("conv1d", "gate_gemm_fused_scan") if fused else ("conv1d", "gate_gemm", "scan")
+    for k in kern:
+        if k not in step_kernels and "note" not in kern[k]:
+            kern[k]["note"] = "the separate path's stage; not the step's path at this shape"
+    dom = max(step_kernels, key=lambda k: kern[k]["ms"])
     roof = _roofline(kern, dom, c.pk, cfg["name"])
     res = {"workload": cfg["workload"], "B": B, "T": T, "D_RNN": R, "ms_per_step": step_ms,
            "tokens_per_s": c.world * tokens / (step_ms / 1e3), "kernels": kern, "roofline": roof,
-           "status": status, "gpu_launches_per_step": 3, "clocks": clk,
+           "status": status, "gpu_launches_per_step": n_kern, "step_kernels": list(step_kernels), "clocks": clk,
            "timing": f"{steps} rglru_forward calls, L2 flushed before each; kernels: {ks} stage calls"}
     del x, y, u, z, ws_scan, ws_fwd
     return res, w
@@ -376,7 +412,8 @@ def run_own(args):
     if only == "forward":
         return emit({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                      "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "kernels": head["kernels"],
-                     "roofline": head["roofline"], "gpu_launches": 3 * args.steps, "clocks": head["clocks"],
+                     "roofline": head["roofline"], "gpu_launches": head["gpu_launches_per_step"] * args.steps,
+                     "clocks": head["clocks"],
                      "only": "forward"})
 
     # ---- end to end through the public API, host buffers -----------------------------
@@ -444,7 +481,7 @@ def run_own(args):
         "layer": lay,
         "backward": bwd,
         "e2e": e2e,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": head["gpu_launches_per_step"] * args.steps,
         "clocks": head["clocks"],
         "status": "ok" if status == 0 else "timeout reported",
         "cpu_baseline": cpu,

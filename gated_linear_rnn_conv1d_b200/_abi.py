@@ -90,10 +90,11 @@ SIGNATURES = {
     "rglru_backward_workspace_bytes": (_S, [_I, _I, _I]),
     "rglru_backward": (_I, [_PP, _P, _P, _P, _P, _P, _P, _GP, _I, _I, _I, _P, _S, _P]),
     "rglru_saved_bytes": (_S, [_I, _I, _I]),
+    "rglru_forward_kernels": (_I, [_I, _I, _I, _I]),
     "rglru_forward_train": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _S, _P]),
     "rglru_backward_saved": (_I, [_PP, _P, _P, _P, _P, _P, _P, _P, _GP, _I, _I, _I, _P, _S, _P]),
     "rglru_gate_scan_workspace_bytes": (_S, [_I, _I, _I, _I]),
-    "rglru_gate_scan": (_I, [_PP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
+    "rglru_gate_scan": (_I, [_PP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "rglru_workspace_status": (_I, [_P, _P]),
     "rglru_strerror": (ctypes.c_char_p, [_I]),
     "rglru_last_cuda_error": (_I, []),

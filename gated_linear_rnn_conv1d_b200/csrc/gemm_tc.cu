@@ -385,16 +385,20 @@ __device__ __forceinline__ void umma_commit_2sm_both(uint64_t* bar) {
                : "memory");
 }
 
-// Fused-scan epilogue scratch after the pipeline stages: per epilogue warp a 32×33 float2
-// transpose buffer, then aggregates [4][32][2], incoming states [32], parameters [6][128].
-constexpr int kScanStages = 5;
-constexpr int kTbufBytes = 4 * 32 * 33 * 8;
-constexpr int kScanEpiBytes = kTbufBytes + 4 * 32 * 2 * 4 + 32 * 4 + 6 * 128 * 4;
+// Fused-scan epilogue scratch after the pipeline stages: per tile parity the 128 channels'
+// b_a, b_x and c·log σ(Λ); the four quarters' maps (A, B) per channel; their incoming states.
+constexpr int kScanParBytes = 2 * 3 * 128 * 4;
+constexpr int kScanTPitch = 17;  // float2 per row of a warp's transpose buffer (conflict-light)
+constexpr int kScanTBytes = 8 * 32 * kScanTPitch * 8;  // eight warps × [32 rows][17] float2
+constexpr int kScanEpiBytes = kScanParBytes + 4 * 128 * 8 + 4 * 128 * 4 + kScanTBytes;
+constexpr int kScanStages = 5;  // (the transpose buffers take the sixth stage's room)
 template <int EPI> __host__ __device__ constexpr int stages_of() { return EPI == EPI_SCAN ? kScanStages : k2Stages; }
 constexpr int kCoefEpiBytes = 2 * 3 * 128 * 4;  // per tile parity: b_a, b_x, c·log σ(Λ) of 128 channels
 // warps: 0 TMA, 1 MMA, then epilogue warps — 4 (one per TMEM lane quarter), or 8 for the
 // coefficient epilogue (two per quarter, each taking half of the channels)
-template <int EPI> __host__ __device__ constexpr int epi_warps_of() { return EPI == EPI_COEF ? 8 : 4; }
+template <int EPI> __host__ __device__ constexpr int epi_warps_of() {
+  return (EPI == EPI_COEF || EPI == EPI_SCAN) ? 8 : 4;
+}
 template <int EPI> __host__ __device__ constexpr int threads_of() { return 64 + 32 * epi_warps_of<EPI>(); }
 template <int EPI> __host__ __device__ constexpr int smem_of() {
   return stages_of<EPI>() * k2StageBytes + (EPI == EPI_SCAN ? kScanEpiBytes : 0) +
@@ -661,6 +665,17 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         for (int q = 0; q < 8; ++q)
           uq[q] = (row_ok && ch0 + 8 * q < ep.R) ? __ldg(reinterpret_cast<const uint4*>(urow) + q)
                                                  : make_uint4(0u, 0u, 0u, 0u);
+        // the tile's channel parameters (b_a, b_x, c·log σ(Λ)), also before the accumulator
+        // is ready: this parity's buffer was last read by the tile two back, which every
+        // epilogue warp has finished (they all passed the previous tile's barrier)
+        float* sPar = reinterpret_cast<float*>(smem + S * k2StageBytes) + acc * 3 * 128;
+        if ((warp - 2) / 4 == 0) {
+          const int ch = n_blk * 128 + row_in_tile;
+          const bool ok = ch < ep.R;
+          sPar[row_in_tile] = ok ? __ldg(ep.b_a + ch) : 0.0f;
+          sPar[128 + row_in_tile] = ok ? __ldg(ep.b_x + ch) : 0.0f;
+          sPar[256 + row_in_tile] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
+        }
       }
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_s)) {
         abort_s = 1;
@@ -678,14 +693,7 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
         // with u_t, so it takes bf16's float32 exponent range (any |u_t| a bf16 u can hold).
         float* sPar = reinterpret_cast<float*>(smem + S * k2StageBytes) + acc * 3 * 128;
         const int chalf = (warp - 2) / 4;  // which 64 of the 128 channels this warp forms
-        if (chalf == 0) {
-          const int ch = n_blk * 128 + row_in_tile;
-          const bool ok = ch < ep.R;
-          sPar[row_in_tile] = ok ? __ldg(ep.b_a + ch) : 0.0f;
-          sPar[128 + row_in_tile] = ok ? __ldg(ep.b_x + ch) : 0.0f;
-          sPar[256 + row_in_tile] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
-        }
-        named_bar_sync(1, 32 * epi_warps_of<EPI>());  // this CTA's epilogue warps
+        named_bar_sync(1, 32 * epi_warps_of<EPI>());  // this CTA's epilogue warps: sPar is written
         uint16_t* out = reinterpret_cast<uint16_t*>(ep.C) + row * ep.ldc + (int64_t)n_blk * BN;  // 16-bit words
         // 4 chunks of 16 channels; the next chunk's TMEM load is in flight while one is formed
         uint32_t ra[2][16], rx[2][16];
@@ -801,169 +809,277 @@ __global__ void __launch_bounds__(threads_of<EPI>(), 1)
   } else {
     // ---------------- fused RG-LRU scan epilogue (both CTAs) ----------------
     // "Griffin：将门控线性循环与局部注意力混合以实现高效的语言模型", §实门线性循环单元 (RG-LRU),
-    // Eq. (1)–(4). The CTA's 128 rows are 128 consecutive steps of one batch row (T is a
-    // multiple of 128); its 256 accumulator columns are z_a and z_x of 128 channels. For
-    // each 32-channel block, a warp moves its 32 rows through a shared-memory transpose so
-    // that lane j owns channel j and walks the 32 steps in order: u recomputed in float32
-    // from x, gates, log-space decay, fold into an affine map; the four warps' maps are
-    // composed, the 128-step chunk's incoming state comes from decoupled look-back over
-    // earlier chunks (carries in global memory, bounded waits), and each lane replays its
-    // steps into y.
-    const int q = warp & 3;                 // TMEM lane quarter = rows 32q … 32q+31
-    const int et = q * 32 + lane;           // 0..127 among the epilogue threads
+    // Eq. (1)–(4). The CTA's 128 accumulator rows are 128 consecutive steps of one batch row
+    // (T is a multiple of 128), its 256 columns z_a and z_x of 128 channels. Eight warps, as
+    // in the coefficient epilogue: warp w holds rows 32·(w mod 4) … (TMEM lane quarter) and
+    // one half of the channels; each thread is one step (row) and forms, for 16 channels at
+    // a time, a_t = 1 − d and b_t = √(1−a_t²)·i_t·u_t (float32, never stored). The step's
+    // affine maps h ↦ a_t h + b_t are composed across the warp's 32 rows through a small
+    // shared-memory transpose (lane = channel and half of the rows, 16 steps in order):
+    //   pass 1: each warp's map per channel; the four quarters' maps make
+    //           the 128-step chunk's map; 128 threads (one per channel) publish it as the
+    //           chunk's aggregate, take the incoming state from decoupled look-back over
+    //           the earlier chunks of the same (batch row, channel block) (windows of 8,
+    //           bounded waits), publish the inclusive state and hand each quarter its
+    //           incoming state;
+    //   pass 2: the same coefficients again (TMEM is read twice; the arithmetic is the
+    //           same, so are the bits), the replay of each channel's 32 steps from the
+    //           quarter's incoming state, and h_t = y_t back to the row's thread.
+    // The pre-activations and coefficients never leave the SM. Forward progress: a chunk
+    // waits only for earlier chunks, which are earlier tiles of the persistent grid (or the
+    // other CTA of its own pair).
+    const int quarter = warp & 3;
+    const int chalf = (warp - 2) / 4;          // which 64 of the tile's 128 channels
+    const int row_in_tile = quarter * 32 + lane;
+    const int et = row_in_tile;                // channel of the look-back threads (chalf 0)
     uint8_t* escr = smem + S * k2StageBytes;
-    float2* tbuf = reinterpret_cast<float2*>(escr) + q * (32 * 33);
-    float* sAgg = reinterpret_cast<float*>(escr + kTbufBytes);       // [4 warps][32][2]
-    float* sHin = sAgg + 4 * 32 * 2;                                   // [32]
-    float* sPar = sHin + 32;                                           // [6][128]
+    float* sParAll = reinterpret_cast<float*>(escr);                    // [2 acc][3][128]
+    float2* sQ = reinterpret_cast<float2*>(escr + kScanParBytes);       // [4 quarters][128]
+    float* sS = reinterpret_cast<float*>(escr + kScanParBytes + 4 * 128 * 8);  // [4][128]
+    float2* sT = reinterpret_cast<float2*>(escr + kScanParBytes + 4 * 128 * 8 + 4 * 128 * 4) +
+                 (warp - 2) * 32 * kScanTPitch;  // this warp's [32 rows][17]
     const uint32_t leader_tempty0 = mapa_rank(smem_u32(&tempty_bar[0]), 0);
     const int R = ep.R;
+    constexpr int kNT = 32 * epi_warps_of<EPI>();
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cluster; tile < num_tiles; tile += n_clusters) {
       const int m_pair = tile / n_tiles_n, n_blk = tile % n_tiles_n;
+      const int64_t m0 = (int64_t)m_pair * 256 + rank * 128;
+      const bool cta_rows = m0 < M;  // (M is a multiple of 128: all 128 rows or none)
+      const int64_t row = m0 + row_in_tile;
+      // this thread's 64 values of u (its row, its half of the channels), before the
+      // accumulator is ready; 8 channels are all valid or all not (R % 8 = 0)
+      uint4 uq[8];
+      {
+        const int ch0 = n_blk * 128 + chalf * 64;
+        const __nv_bfloat16* urow = ep.ub + row * R + ch0;
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8)
+          uq[q8] = (cta_rows && ch0 + 8 * q8 < R) ? __ldg(reinterpret_cast<const uint4*>(urow) + q8)
+                                                  : make_uint4(0u, 0u, 0u, 0u);
+      }
+      // the tile's channel parameters, also before the accumulator is ready (this parity's
+      // buffer was last read by the tile two back, which every warp has finished)
+      float* sPar = sParAll + acc * 3 * 128;
+      if (chalf == 0) {
+        const int ch = n_blk * 128 + et;
+        const bool ok = ch < R;
+        sPar[et] = ok ? __ldg(ep.b_a + ch) : 0.0f;
+        sPar[128 + et] = ok ? __ldg(ep.b_x + ch) : 0.0f;
+        sPar[256 + et] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
+      }
       if (!mbar_wait(&tfull_bar[acc], acc_phase, &abort_s)) {
         abort_s = 1;
         atomicOr(status, kStatusTimeout);
         break;
       }
       tc_fence_after();
-      const int64_t m0 = (int64_t)m_pair * 256 + rank * 128;
-      if (m0 < M) {
-        const int b = (int)(m0 / ep.T);
-        const int t0 = (int)(m0 - (int64_t)b * ep.T);
-        const int chunk = t0 / 128;
+      if (cta_rows) {
+        const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+        named_bar_sync(1, kNT);
+        // (a_t, b_t) of this row for channels c0 … c0+15 of the tile
+        auto coeffs = [&](int k, const uint32_t (&ra)[16], const uint32_t (&rx)[16], float (&A)[16],
+                          float (&Bv)[16]) {
+          const int c0 = chalf * 64 + k * 16;
+          const uint32_t uw[8] = {uq[2 * k].x, uq[2 * k].y, uq[2 * k].z, uq[2 * k].w,
+                                  uq[2 * k + 1].x, uq[2 * k + 1].y, uq[2 * k + 1].z, uq[2 * k + 1].w};
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const int c = c0 + j;
+            const float2 u2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[j / 2]));
+            const float2 za = make_float2(__uint_as_float(ra[j]) + sPar[c], __uint_as_float(ra[j + 1]) + sPar[c + 1]);
+            const float2 zx = make_float2(__uint_as_float(rx[j]) + sPar[128 + c],
+                                          __uint_as_float(rx[j + 1]) + sPar[128 + c + 1]);
+            float2 d, m;
+            gate_fast2_pair(za, zx, make_float2(sPar[256 + c], sPar[256 + c + 1]), u2, d, m);
+            A[j] = 1.0f - d.x;
+            A[j + 1] = 1.0f - d.y;
+            Bv[j] = m.x;
+            Bv[j + 1] = m.y;
+          }
+        };
+        // ---- pass 1: each warp's map per channel → sQ[quarter][channel]
         {
-          const int ch = n_blk * 128 + et;
-          const bool ok = ch < R;
-          sPar[0 * 128 + et] = ok ? __ldg(ep.conv_w + ch) : 0.0f;
-          sPar[1 * 128 + et] = ok ? __ldg(ep.conv_w + R + ch) : 0.0f;
-          sPar[2 * 128 + et] = ok ? __ldg(ep.conv_w + 2 * R + ch) : 0.0f;
-          sPar[3 * 128 + et] = ok ? __ldg(ep.conv_w + 3 * R + ch) : 0.0f;
-          sPar[4 * 128 + et] = ok ? __ldg(ep.conv_b + ch) : 0.0f;
-          sPar[5 * 128 + et] = ok ? decay_log_coeff(__ldg(ep.Lambda + ch)) : 0.0f;
+          uint32_t ra[2][16], rx[2][16];
+          tmem_ld_x16(t_row + chalf * 64, ra[0]);
+          tmem_ld_x16(t_row + 128 + chalf * 64, rx[0]);
+          tmem_ld_wait16(ra[0], rx[0]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int cur = k & 1;
+            if (k + 1 < 4) {
+              tmem_ld_x16(t_row + chalf * 64 + (k + 1) * 16, ra[cur ^ 1]);
+              tmem_ld_x16(t_row + 128 + chalf * 64 + (k + 1) * 16, rx[cur ^ 1]);
+            }
+            {
+              float A[16], Bv[16];
+              coeffs(k, ra[cur], rx[cur], A, Bv);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sT[lane * kScanTPitch + j] = make_float2(A[j], Bv[j]);
+            }
+            __syncwarp();
+            // the transpose: lane (c, half) folds channel c over rows 16·half … 16·half + 15,
+            // then the halves meet in one shuffle
+            {
+              const int c = lane & 15, r0 = (lane >> 4) * 16;
+              float fa = 1.0f, fb = 0.0f;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 m = sT[(r0 + i) * kScanTPitch + c];
+                fb = fmaf(m.x, fb, m.y);
+                fa *= m.x;
+              }
+              const float a2 = __shfl_down_sync(0xffffffffu, fa, 16);
+              const float b2 = __shfl_down_sync(0xffffffffu, fb, 16);
+              if (lane < 16) sQ[quarter * 128 + chalf * 64 + k * 16 + c] = make_float2(a2 * fa, fmaf(a2, fb, b2));
+            }
+            __syncwarp();
+            if (k + 1 < 4) tmem_ld_wait16(ra[cur ^ 1], rx[cur ^ 1]);
+          }
         }
-        named_bar_sync(1, 128);
-        const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          // row phase: this lane's step, 32 channels of z_a and of z_x
-          {
-            uint32_t ra[32], rx[32];
-            tmem_ld_32x32b_x32(t_row + cc * 32, ra);
-            tmem_ld_32x32b_x32(t_row + 128 + cc * 32, rx);
-            tmem_ld_wait();
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-              tbuf[lane * 33 + jj] = make_float2(__uint_as_float(ra[jj]), __uint_as_float(rx[jj]));
-          }
-          __syncwarp();
-          // column phase: lane = channel, 32 steps in order
-          const int cl = cc * 32 + lane;
-          const int ch = n_blk * 128 + cl;
+        named_bar_sync(1, kNT);
+        // ---- look-back: one thread per channel
+        if (chalf == 0) {
+          const int b_row = (int)(m0 / ep.T);
+          const int chunk = (int)((m0 - (int64_t)b_row * ep.T) / 128);
+          const int ch = n_blk * 128 + et;
           const bool cvalid = ch < R;
-          const int chs = cvalid ? ch : 0;
-          const float w0 = sPar[cl], w1 = sPar[128 + cl], w2 = sPar[256 + cl], w3 = sPar[384 + cl];
-          const float cb = sPar[512 + cl], cla = sPar[640 + cl];
-          const float ba = __ldg(ep.b_a + chs), bx = __ldg(ep.b_x + chs);
-          const int tq = t0 + q * 32;  // first step of this warp's rows
-          const __nv_bfloat16* xb = ep.x + (int64_t)b * ep.T * R + chs;
-          float xm3, xm2, xm1;
-          {
-            float hv[3];
+          float At = 1.0f, Bt = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 3; ++k) {
-              const int t = tq - 3 + k;
-              float v = 0.0f;
-              if (t >= 0) v = __bfloat162float(xb[(int64_t)t * R]);
-              else if (ep.state0 != nullptr) v = __bfloat162float(ep.state0[((int64_t)b * 3 + (t + 3)) * R + chs]);
-              hv[k] = v;
-            }
-            xm3 = hv[0]; xm2 = hv[1]; xm1 = hv[2];
+          for (int qq = 0; qq < 4; ++qq) {
+            const float2 mq = sQ[qq * 128 + et];
+            Bt = fmaf(mq.x, Bt, mq.y);
+            At *= mq.x;
           }
-          uint32_t rp[32];
-          float A = 1.0f, Bv = 0.0f;
+          const int64_t slot = (((int64_t)b_row * n_tiles_n + n_blk) * ep.n_chunks + chunk) * 128 + et;
+          float hin;
+          if (chunk == 0) {
+            hin = (ep.h0 != nullptr && cvalid) ? ep.h0[(int64_t)b_row * R + ch] : 0.0f;
+          } else {
+            st_relaxed_u64g(ep.carry_agg + slot, ((uint64_t)__float_as_uint(Bt) << 32) | enc_carry(At));
+            // the predecessors chunk − 1, chunk − 2, … in windows of 8: the nearest published
+            // inclusive state, then the aggregates in front of it, oldest first
+            float fA = 1.0f, fB = 0.0f;  // composed map of the predecessors already passed
+            int d0 = 1;                  // depth of the window's first predecessor
+            long long tw = 0;
+            bool done = false;
+            while (!done) {
+              uint32_t wi[8];
+              uint64_t ga[8];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float x0 = __bfloat162float(xb[(int64_t)(tq + i) * R]);
-            const float x1 = __bfloat162float(xb[(int64_t)(tq + i + 1) * R]);
-            float2 u;
-            u.x = fmaf(w3, x0, fmaf(w2, xm1, fmaf(w1, xm2, fmaf(w0, xm3, cb))));
-            u.y = fmaf(w3, x1, fmaf(w2, x0, fmaf(w1, xm1, fmaf(w0, xm2, cb))));
-            xm3 = xm1;
-            xm2 = x0;
-            xm1 = x1;
-            const float2 z0 = tbuf[i * 33 + lane], z1 = tbuf[(i + 1) * 33 + lane];
-            float2 d, bt;
-            gate_fast2_pair(make_float2(z0.x + ba, z1.x + ba), make_float2(z0.y + bx, z1.y + bx),
-                            make_float2(cla, cla), u, d, bt);
-            const float a0 = 1.0f - d.x, a1 = 1.0f - d.y;
-            Bv = fmaf(a0, Bv, bt.x);
-            A *= a0;
-            Bv = fmaf(a1, Bv, bt.y);
-            A *= a1;
-            rp[i] = pack_bf16x2(d.x, bt.x);
-            rp[i + 1] = pack_bf16x2(d.y, bt.y);
-          }
-          __syncwarp();  // tbuf free for the next block
-          sAgg[(q * 32 + lane) * 2 + 0] = A;
-          sAgg[(q * 32 + lane) * 2 + 1] = Bv;
-          named_bar_sync(1, 128);
-          // map from the chunk's incoming state to the state entering this warp's rows
-          float eA = 1.0f, eB = 0.0f;
-          for (int w = 0; w < q; ++w) {
-            const float wa = sAgg[(w * 32 + lane) * 2], wb = sAgg[(w * 32 + lane) * 2 + 1];
-            eB = fmaf(wa, eB, wb);
-            eA *= wa;
-          }
-          if (q == 0) {
-            float At = 1.0f, Bt = 0.0f;
+              for (int i = 0; i < 8; ++i) {
+                const bool in = d0 + i <= chunk;
+                wi[i] = in ? ld_relaxed_u32g(ep.carry_incl + slot - (int64_t)(d0 + i) * 128) : 0u;
+                ga[i] = in ? ld_relaxed_u64g(ep.carry_agg + slot - (int64_t)(d0 + i) * 128) : 0ull;
+              }
+              int found = -1, have = 0;  // nearest inclusive; aggregates present in front of it
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const float wa = sAgg[(w * 32 + lane) * 2], wb = sAgg[(w * 32 + lane) * 2 + 1];
-              Bt = fmaf(wa, Bt, wb);
-              At *= wa;
-            }
-            const int64_t slot = (((int64_t)b * n_tiles_n + n_blk) * ep.n_chunks + chunk) * 128 + cl;
-            float hin;
-            if (chunk == 0) {
-              hin = (ep.h0 != nullptr && cvalid) ? ep.h0[(int64_t)b * R + ch] : 0.0f;
-            } else {
-              st_relaxed_u64g(ep.carry_agg + slot, ((uint64_t)__float_as_uint(Bt) << 32) | enc_carry(At));
-              float fA = 1.0f, fB = 0.0f;
-              int64_t p = slot - 128;
-              long long tw = 0;
-              while (true) {
-                const uint32_t hw = ld_relaxed_u32g(ep.carry_incl + p);
-                const uint64_t aw = ld_relaxed_u64g(ep.carry_agg + p);
-                if (hw != 0u) { hin = fmaf(fA, dec_carry(hw), fB); break; }
-                if ((uint32_t)aw != 0u) {
-                  fB = fmaf(fA, __uint_as_float((uint32_t)(aw >> 32)), fB);
-                  fA *= dec_carry((uint32_t)aw);
-                  p -= 128;
-                  continue;
+              for (int i = 0; i < 8; ++i) {
+                if (found < 0 && wi[i] != 0u) found = i;
+                if (found < 0 && have == i && (uint32_t)ga[i] != 0u) have = i + 1;
+              }
+              if (found >= 0 && have >= found) {
+                float h = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  if (i == found) h = dec_carry(wi[i]);
+#pragma unroll
+                for (int i = 7; i >= 0; --i)
+                  if (i < found) h = fmaf(dec_carry((uint32_t)ga[i]), h, __uint_as_float((uint32_t)(ga[i] >> 32)));
+                hin = fmaf(fA, h, fB);
+                done = true;
+              } else if (found < 0 && have == 8) {
+                // the whole window is aggregates: fold it (newest first is the outer map)
+                float wA = 1.0f, wB = 0.0f;
+#pragma unroll
+                for (int i = 7; i >= 0; --i) {
+                  wB = fmaf(dec_carry((uint32_t)ga[i]), wB, __uint_as_float((uint32_t)(ga[i] >> 32)));
+                  wA *= dec_carry((uint32_t)ga[i]);
                 }
-                if (tw == 0) {
-                  tw = clock64();
-                } else if (clock64() - tw > kWaitCycles) {
-                  atomicOr(status, kStatusTimeout);
-                  hin = fB;
-                  break;
-                }
+                fB = fmaf(fA, wB, fB);
+                fA *= wA;
+                d0 += 8;
+              } else if (tw == 0) {
+                tw = clock64();
+              } else if (clock64() - tw > kWaitCycles) {
+                atomicOr(status, kStatusTimeout);
+                hin = fB;
+                done = true;
               }
             }
-            const float hout = fmaf(At, hin, Bt);
-            st_relaxed_u32g(ep.carry_incl + slot, enc_carry(hout));
-            if (chunk == ep.n_chunks - 1 && ep.hT != nullptr && cvalid) ep.hT[(int64_t)b * R + ch] = hout;
-            sHin[lane] = hin;
           }
-          named_bar_sync(1, 128);
-          float h = fmaf(eA, sHin[lane], eB);
-          __nv_bfloat16* yb = ep.y + ((int64_t)b * ep.T + tq) * R + chs;
+          const float hout = fmaf(At, hin, Bt);
+          st_relaxed_u32g(ep.carry_incl + slot, enc_carry(hout));
+          if (chunk == ep.n_chunks - 1 && ep.hT != nullptr && cvalid) ep.hT[(int64_t)b_row * R + ch] = hout;
+          float sq = hin;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            h = fmaf(1.0f - bf16lo(rp[i]), h, bf16hi(rp[i]));
-            if (cvalid) yb[(int64_t)i * R] = __float2bfloat16_rn(h);
+          for (int qq = 0; qq < 4; ++qq) {
+            sS[qq * 128 + et] = sq;
+            const float2 mq = sQ[qq * 128 + et];
+            sq = fmaf(mq.x, sq, mq.y);
+          }
+        }
+        named_bar_sync(1, kNT);
+        // ---- pass 2: the same coefficients, the quarter's incoming state, h_t by scan
+        {
+          uint32_t ra[2][16], rx[2][16];
+          tmem_ld_x16(t_row + chalf * 64, ra[0]);
+          tmem_ld_x16(t_row + 128 + chalf * 64, rx[0]);
+          tmem_ld_wait16(ra[0], rx[0]);
+          __nv_bfloat16* yrow = ep.y + row * R + n_blk * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int cur = k & 1;
+            if (k + 1 < 4) {
+              tmem_ld_x16(t_row + chalf * 64 + (k + 1) * 16, ra[cur ^ 1]);
+              tmem_ld_x16(t_row + 128 + chalf * 64 + (k + 1) * 16, rx[cur ^ 1]);
+            }
+            const int c0 = chalf * 64 + k * 16;
+            {
+              float A[16], Bv[16];
+              coeffs(k, ra[cur], rx[cur], A, Bv);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sT[lane * kScanTPitch + j] = make_float2(A[j], Bv[j]);
+            }
+            __syncwarp();
+            // lane (c, half): its 16 steps of channel c; the second half starts from the first
+            // half's map applied to the quarter's incoming state; then the replay, whose
+            // states go back over the coefficients
+            {
+              const int c = lane & 15, r0 = (lane >> 4) * 16;
+              float2 m[16];
+              float fa = 1.0f, fb = 0.0f;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                m[i] = sT[(r0 + i) * kScanTPitch + c];
+                fb = fmaf(m[i].x, fb, m[i].y);
+                fa *= m[i].x;
+              }
+              const float a2 = __shfl_up_sync(0xffffffffu, fa, 16);
+              const float b2 = __shfl_up_sync(0xffffffffu, fb, 16);
+              const float s0 = sS[quarter * 128 + c0 + c];
+              float h = lane < 16 ? s0 : fmaf(a2, s0, b2);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                h = fmaf(m[i].x, h, m[i].y);
+                sT[(r0 + i) * kScanTPitch + c].x = h;
+              }
+            }
+            __syncwarp();
+            float Bv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) Bv[j] = sT[lane * kScanTPitch + j].x;
+            __syncwarp();
+            if (n_blk * 128 + c0 < R) {  // 16 channels all valid or all not (R % 8 = 0, c0 % 16 = 0)
+              uint4* py = reinterpret_cast<uint4*>(yrow + c0);
+              py[0] = make_uint4(pack_bf16x2(Bv[0], Bv[1]), pack_bf16x2(Bv[2], Bv[3]), pack_bf16x2(Bv[4], Bv[5]),
+                                 pack_bf16x2(Bv[6], Bv[7]));
+              if (n_blk * 128 + c0 + 8 < R)
+                py[1] = make_uint4(pack_bf16x2(Bv[8], Bv[9]), pack_bf16x2(Bv[10], Bv[11]),
+                                   pack_bf16x2(Bv[12], Bv[13]), pack_bf16x2(Bv[14], Bv[15]));
+            }
+            if (k + 1 < 4) tmem_ld_wait16(ra[cur ^ 1], rx[cur ^ 1]);
           }
         }
       }
@@ -1394,10 +1510,7 @@ cudaError_t launch_gate_scan_bf16(const ScanFusedArgs& f, cudaStream_t s) {
   ep.b_x = f.b_x;
   ep.R = f.R;
   ep.y = static_cast<__nv_bfloat16*>(f.y);
-  ep.x = static_cast<const __nv_bfloat16*>(f.x);
-  ep.state0 = static_cast<const __nv_bfloat16*>(f.state0);
-  ep.conv_w = f.conv_w;
-  ep.conv_b = f.conv_b;
+  ep.ub = static_cast<const __nv_bfloat16*>(f.u);
   ep.Lambda = f.Lambda;
   ep.h0 = f.h0;
   ep.hT = f.hT;

@@ -121,15 +121,11 @@ cudaError_t launch_gemm_step_bf16(const void* u_t, const float* u_f32, const voi
 // T % 128 == 0): y and h_T straight from x and u, without writing the gate
 // pre-activations. carry_* need n_chunk_tiles × 128 slots (zero at launch).
 struct ScanFusedArgs {
-  const void* u;        // [B·T][R] bf16 conv output (GEMM operand)
-  const void* x;        // [B][T][R] bf16 conv input (u recomputed in float32)
-  const void* state0;   // [B][3][R] or null
+  const void* u;        // [B·T][R] bf16 conv output (GEMM operand, and the u of b_t)
   const void* W_a;
   const void* W_x;
   const float* b_a;
   const float* b_x;
-  const float* conv_w;
-  const float* conv_b;
   const float* Lambda;
   const float* h0;      // or null
   void* y;              // [B][T][R] bf16

@@ -103,22 +103,22 @@ FusedLayout fused_layout(int B, int T, int R) {
   L.bytes = L.off_u + round256((size_t)B * T * R * 2);
   return L;
 }
+// rglru_forward takes the fused gate GEMM + scan (2 launches: Conv1D, then the GEMM with the
+// scan in its epilogue) for bf16 IO, T a multiple of 128 and R ≥ 4096: its epilogue (the
+// gate math twice and the scan, per 128 × 128 tile) then hides behind the tile's MMAs
+// (K = R); at R = 2048 it does not and the separate gate GEMM + scan is faster (B=8 T=2048
+// R=2048: 306 µs fused against 254 µs; B=1 T=32768 R=4096: 1.73–1.76 ms against 1.88 ms).
 bool fused_ok(int io, int T) { return io == RGLRU_BF16 && T % 128 == 0; }
-// (rglru_forward keeps the separate gate GEMM + scan: on B200 the fused epilogue, with 4
-// warps per SM for the scan, is slower than the standalone scan's 16 warps per SM.)
+bool fused_faster(int io, int T, int R) { return fused_ok(io, T) && R >= 4096; }
 
-ScanFusedArgs fused_args(const rglru_params* p, const void* x, const void* u, const void* state0, const float* h0,
-                         void* y, float* hT, int B, int T, int R, const FusedLayout& L, void* ws) {
+ScanFusedArgs fused_args(const rglru_params* p, const void* u, const float* h0, void* y, float* hT, int B, int T, int R,
+                         const FusedLayout& L, void* ws) {
   ScanFusedArgs f{};
   f.u = u;
-  f.x = x;
-  f.state0 = state0;
   f.W_a = p->W_a;
   f.W_x = p->W_x;
   f.b_a = p->b_a;
   f.b_x = p->b_x;
-  f.conv_w = p->conv_w;
-  f.conv_b = p->conv_b;
   f.Lambda = p->Lambda;
   f.h0 = h0;
   f.y = y;
@@ -408,18 +408,15 @@ size_t rglru_gate_scan_workspace_bytes(int B, int T, int R, int io_dtype) {
   return fused_layout(B, T, R).zero_bytes;
 }
 
-int rglru_gate_scan(const rglru_params* params, const void* x, const void* u, const void* conv_state0,
-                    const float* h0, void* y, float* h_T, int B, int T, int R, int io_dtype, void* workspace,
-                    size_t workspace_bytes, rglru_stream_t stream) {
+int rglru_gate_scan(const rglru_params* params, const void* u, const float* h0, void* y, float* h_T, int B, int T,
+                    int R, int io_dtype, void* workspace, size_t workspace_bytes, rglru_stream_t stream) {
   const Range range("rglru_gate_scan");
   if (io_dtype != RGLRU_BF16) return RGLRU_ERR_DTYPE;
   if (!valid_R(R) || !valid_tokens(B, T) || T % 128 != 0) return RGLRU_ERR_SHAPE;
   int st = check_params(params);
   if (st != RGLRU_OK) return st;
-  if (x == nullptr || u == nullptr || y == nullptr) return RGLRU_ERR_NULL;
-  if (!aligned16(x) || !aligned16(u) || !aligned16(y) || !aligned16(conv_state0) || !aligned16(h0) ||
-      !aligned16(h_T))
-    return RGLRU_ERR_ALIGN;
+  if (u == nullptr || y == nullptr) return RGLRU_ERR_NULL;
+  if (!aligned16(u) || !aligned16(y) || !aligned16(h0) || !aligned16(h_T)) return RGLRU_ERR_ALIGN;
   const FusedLayout L = fused_layout(B, T, R);
   if (workspace == nullptr || workspace_bytes < L.zero_bytes) return RGLRU_ERR_WORKSPACE;
   if (!aligned256(workspace)) return RGLRU_ERR_ALIGN;
@@ -427,7 +424,7 @@ int rglru_gate_scan(const rglru_params* params, const void* x, const void* u, co
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(workspace, 0, L.zero_bytes, s);
   if (e == cudaSuccess)
-    e = launch_gate_scan_bf16(fused_args(params, x, u, conv_state0, h0, y, h_T, B, T, R, L, workspace), s);
+    e = launch_gate_scan_bf16(fused_args(params, u, h0, y, h_T, B, T, R, L, workspace), s);
   return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
 }
 
@@ -558,6 +555,16 @@ int forward_impl(const rglru_params* params, const void* x, const float* h0, con
   void* u = bytes(workspace) + L.off_u;
   void* z = bytes(workspace) + L.off_z;
   unsigned* status = reinterpret_cast<unsigned*>(workspace);
+  if (saved == nullptr && fused_faster(io_dtype, T, R)) {
+    // the fused path: its chunk carries sit at the start of the workspace (inside the scan's
+    // region, which is larger), zeroed with the status word by the conv kernel
+    const FusedLayout F = fused_layout(B, T, R);
+    if (F.zero_bytes > L.off_u) return RGLRU_ERR_WORKSPACE;  // (never: the scan's region is larger)
+    cudaError_t e = launch_conv1d(params->conv_w, params->conv_b, x, conv_state0, u, conv_state_T, B, T, R, true,
+                                  status, s, workspace, F.zero_bytes);
+    if (e == cudaSuccess) e = launch_gate_scan_bf16(fused_args(params, u, h0, y, h_T, B, T, R, F, workspace), s);
+    return e == cudaSuccess ? RGLRU_OK : fail_cuda(e);
+  }
   // the conv kernel also zeroes the status word, the scan's ticket and its chunk carries,
   // so that a status bit set by the GEMM or the scan survives until the caller reads it;
   // the GEMM and the scan are launched as programmatic dependents of the kernel before
@@ -585,6 +592,11 @@ int rglru_forward(const rglru_params* params, const void* x, const float* h0, co
   const Range range("rglru_forward");
   return forward_impl(params, x, h0, conv_state0, y, h_T, conv_state_T, nullptr, B, T, R, io_dtype, workspace,
                       workspace_bytes, stream);
+}
+
+int rglru_forward_kernels(int B, int T, int R, int io_dtype) {
+  if (!valid_dtype(io_dtype) || !valid_R(R) || !valid_tokens(B, T)) return 0;
+  return fused_faster(io_dtype, T, R) ? 2 : 3;
 }
 
 size_t rglru_saved_bytes(int B, int T, int R) {

@@ -96,6 +96,11 @@ def forward(params: Params, x: torch.Tensor, h0: Optional[torch.Tensor] = None,
     return y, h_T, conv_state_T
 
 
+def forward_kernels(B: int, T: int, R: int, dtype: torch.dtype) -> int:
+    """How many kernels rglru_forward launches (2: gate GEMM with the fused scan, 3: separate)."""
+    return _abi.load().rglru_forward_kernels(B, T, R, _DT[dtype])
+
+
 def saved_bytes(B: int, T: int, R: int) -> int:
     return _abi.load().rglru_saved_bytes(B, T, R)
 
@@ -562,21 +567,22 @@ def gate_scan_workspace_bytes(B: int, T: int, R: int) -> int:
     return _abi.load().rglru_gate_scan_workspace_bytes(B, T, R, _abi.RGLRU_BF16)
 
 
-def gate_scan(params: Params, x: torch.Tensor, u: torch.Tensor, h0: Optional[torch.Tensor] = None,
-              conv_state0: Optional[torch.Tensor] = None, *, workspace: Optional[torch.Tensor] = None,
-              y: Optional[torch.Tensor] = None, h_T: Optional[torch.Tensor] = None,
+def gate_scan(params: Params, u: torch.Tensor, h0: Optional[torch.Tensor] = None, *,
+              workspace: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+              h_T: Optional[torch.Tensor] = None,
               stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """rglru_gate_scan: gate GEMM with the scan fused in its epilogue (bf16, T % 128 == 0)."""
+    """rglru_gate_scan: gate GEMM with the scan fused in its epilogue, from u = Conv1D(x)
+    (bf16, T % 128 == 0)."""
     lib = _abi.load()
-    B, T, R = x.shape
-    io = _io(x)
-    y = torch.empty_like(x) if y is None else y
-    h_T = torch.empty(B, R, dtype=torch.float32, device=x.device) if h_T is None else h_T
-    ws = _workspace(lib.rglru_gate_scan_workspace_bytes(B, T, R, io), x.device, workspace)
+    B, T, R = u.shape
+    io = _io(u)
+    y = torch.empty_like(u) if y is None else y
+    h_T = torch.empty(B, R, dtype=torch.float32, device=u.device) if h_T is None else h_T
+    ws = _workspace(lib.rglru_gate_scan_workspace_bytes(B, T, R, io), u.device, workspace)
     st = params.struct()
     _abi.check("rglru_gate_scan", lib.rglru_gate_scan(
-        ctypes.byref(st), _p(x), _p(u), _p(conv_state0), _p(h0), _p(y), _p(h_T), B, T, R, io, _p(ws),
-        ws.numel() * ws.element_size(), _s(stream)))
+        ctypes.byref(st), _p(u), _p(h0), _p(y), _p(h_T), B, T, R, io, _p(ws), ws.numel() * ws.element_size(),
+        _s(stream)))
     return y, h_T
 
 

@@ -110,6 +110,11 @@ typedef struct {
  * the unrounded ones (a property of the bf16 operand, not of the scan).
  * --------------------------------------------------------------------------------- */
 RGLRU_API size_t rglru_forward_workspace_bytes(int B, int T, int R, int io_dtype);
+/* How many kernels rglru_forward launches for this shape (0 for invalid arguments): 2 when
+ * it takes the gate GEMM with the scan fused into its epilogue (bf16 IO, T a multiple of 128,
+ * R ≥ 4096, where that epilogue hides behind the tile's MMAs; see rglru_gate_scan), else 3
+ * (Conv1D, the gate GEMM forming the coefficients, the scan). */
+RGLRU_API int rglru_forward_kernels(int B, int T, int R, int io_dtype);
 RGLRU_API int rglru_forward(const rglru_params* params, const void* x, const float* h0, const void* conv_state0,
                   void* y, float* h_T, void* conv_state_T, int B, int T, int R, int io_dtype,
                   void* workspace, size_t workspace_bytes, rglru_stream_t stream);
@@ -416,18 +421,17 @@ RGLRU_API int rglru_scan_noalloc(const rglru_params* params, const void* x, cons
 RGLRU_API int rglru_scan_noalloc_status(rglru_stream_t stream);
 
 /* The gate GEMM with the RG-LRU scan fused into its epilogue (Eq. (1)–(4)): y and h_T
- * from x (the Conv1D input, from which u is recomputed in float32) and u = Conv1D(x) in
- * bf16 (the tensor-core operand). bf16 only; T must be a multiple of 128 (each 128-step
- * chunk of a batch row is one accumulator tile). conv_state0, h0 and h_T as in
- * rglru_forward. workspace: at least rglru_gate_scan_workspace_bytes(B, T, R, io_dtype)
- * bytes, 256-byte aligned (chunk carries; zeroed by the call). Compared with the separate
- * gate GEMM + scan it needs no pre-activation buffer (2 instead of 6 bytes of workspace
- * per token·channel) but on B200 it takes about twice as long: its scan runs in the four
- * epilogue warps of each SM. */
+ * from u = Conv1D(x) in bf16 [B][T][R] (the tensor-core operand, also the u of
+ * b_t = √(1−a_t²)·i_t·u_t). The recurrence coefficients stay in registers in float32 (no
+ * fp16/bf16 storage rounding of d and b_t, unlike the three-kernel path). bf16 only; T
+ * must be a multiple of 128 (each 128-step chunk of a batch row is one accumulator tile).
+ * h0 and h_T as in rglru_forward. workspace: at least
+ * rglru_gate_scan_workspace_bytes(B, T, R, io_dtype) bytes, 256-byte aligned (chunk carries;
+ * zeroed by the call). */
 RGLRU_API size_t rglru_gate_scan_workspace_bytes(int B, int T, int R, int io_dtype);
-RGLRU_API int rglru_gate_scan(const rglru_params* params, const void* x, const void* u, const void* conv_state0,
-                              const float* h0, void* y, float* h_T, int B, int T, int R, int io_dtype,
-                              void* workspace, size_t workspace_bytes, rglru_stream_t stream);
+RGLRU_API int rglru_gate_scan(const rglru_params* params, const void* u, const float* h0, void* y, float* h_T, int B,
+                              int T, int R, int io_dtype, void* workspace, size_t workspace_bytes,
+                              rglru_stream_t stream);
 
 /* Dense bf16 GEMM C[M][N] = A[M][K] · B[N][K]ᵀ on the tcgen05 tensor cores (fp32
  * accumulate, bf16 store), the kernel behind the block's linears. K % 8 == 0, N % 8 == 0. */

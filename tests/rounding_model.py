@@ -3,8 +3,8 @@
 Test infrastructure (CPU only; no CUDA code is involved). The CUDA path stores some of its
 intermediates in narrow formats and does all arithmetic between them in float32:
   * the forward: the Conv1D output u (bf16, the gate GEMM's operand and the u inside b_t),
-    the recurrence coefficients d = 1 − a_t (fp16) and b_t = √(1 − a_t²)·i_t·u_t (bf16),
-    and y (bf16);
+    the recurrence coefficients d = 1 − a_t (fp16) and b_t = √(1 − a_t²)·i_t·u_t (bf16)
+    — not in the fused gate GEMM + scan, which keeps them in registers — and y (bf16);
   * the recurrent block in addition: v = x W_1ᵀ and g = x W_2ᵀ (bf16), the gated product
     h ⊙ GeLU(g) (bf16) and the block output (bf16);
   * the Hawk residual layer in addition: both RMSNorm outputs, the residual stream, the
@@ -40,12 +40,15 @@ def rms_norm(v, gain, eps=oracle.RMS_EPS):
     return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps) * f(gain)
 
 
-def coefficients(u, P):
-    """(d, b) as the gate GEMM's epilogue stores them, from the bf16 u [..][R]."""
+def coefficients(u, P, stored=True):
+    """(d, b) as the gate GEMM's epilogue stores them (d fp16, b bf16), from the bf16 u
+    [..][R]; unrounded with stored=False (the fused gate GEMM + scan keeps them in
+    registers)."""
     r = oracle.sigmoid(u @ f(P.W_a).T + f(P.b_a))
     i = oracle.sigmoid(u @ f(P.W_x).T + f(P.b_x))
     a_t = oracle.decay_direct(r, f(P.Lambda))
-    return fp16(1.0 - a_t), bf16(np.sqrt(1.0 - a_t * a_t) * i * u)
+    d, b = 1.0 - a_t, np.sqrt(1.0 - a_t * a_t) * i * u
+    return (fp16(d), bf16(b)) if stored else (d, b)
 
 
 def scan(d, b, h0):
@@ -59,11 +62,13 @@ def scan(d, b, h0):
     return hs, h
 
 
-def forward(x, P, h0=None, conv_state0=None):
-    """rglru_forward with bf16 IO: returns (y [B][T][R], h_T [B][R])."""
+def forward(x, P, h0=None, conv_state0=None, fused=False):
+    """rglru_forward with bf16 IO: returns (y [B][T][R], h_T [B][R]); fused=True for the
+    gate GEMM with the scan in its epilogue (T a multiple of 128), whose coefficients are
+    never stored."""
     u, _ = oracle.conv1d_causal(f(x), f(P.conv_w), f(P.conv_b), None if conv_state0 is None else f(conv_state0))
     u = bf16(u)
-    d, b = coefficients(u, P)
+    d, b = coefficients(u, P, stored=not fused)
     hs, h_T = scan(d, b, h0)
     return bf16(hs), h_T
 

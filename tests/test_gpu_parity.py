@@ -255,13 +255,39 @@ def test_fused_gate_scan_matches_oracle(B, T, R, with_state):
     u = rglru.conv1d(p, x, st0.to(DEV) if with_state else None)
     y = torch.full((B, T, R), float("nan"), dtype=torch.bfloat16, device=DEV)
     ws = torch.empty(rglru.gate_scan_workspace_bytes(B, T, R), dtype=torch.uint8, device=DEV)
-    y, h_T = rglru.gate_scan(p, x, u, h0.to(DEV) if with_state else None, st0.to(DEV) if with_state else None,
-                             workspace=ws, y=y)
+    y, h_T = rglru.gate_scan(p, u, h0.to(DEV) if with_state else None, workspace=ws, y=y)
     assert rglru.workspace_status(ws) == 0
     y_ref, h_ref, _ = oracle.rglru_forward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a, w.params.b_a,
                                            w.params.W_x, w.params.b_x, w.params.Lambda, h0=h0, conv_state0=st0)
     assert rel(y, y_ref) <= TOL[torch.bfloat16]
     assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
+
+
+def test_forward_takes_the_fused_path_at_large_r_and_matches_oracle():
+    """rglru_forward with bf16 IO, T a multiple of 128 and R ≥ 4096 runs Conv1D + the gate
+    GEMM with the scan in its epilogue (2 kernels); smaller R or ragged T keep the separate
+    path (3). Both against the oracle, with a state and a conv history."""
+    assert rglru.forward_kernels(1, 256, 4096, torch.bfloat16) == 2
+    assert rglru.forward_kernels(1, 256, 3072, torch.bfloat16) == 3
+    assert rglru.forward_kernels(8, 2048, 2048, torch.bfloat16) == 3
+    assert rglru.forward_kernels(1, 200, 4096, torch.bfloat16) == 3
+    assert rglru.forward_kernels(1, 256, 4096, torch.float32) == 3
+    B, T, R = 1, 256, 4096
+    w = _wl(B, T, R, torch.bfloat16, seed=21)
+    p = rglru.Params.from_host(w.params)
+    st0 = w.extra["state0"]
+    ws = torch.full((rglru.forward_workspace_bytes(B, T, R, torch.bfloat16),), 0xFF, dtype=torch.uint8, device=DEV)
+    y, h_T, cs = rglru.forward(p, w.x.to(DEV), w.h0.to(DEV), st0.to(DEV), workspace=ws)
+    assert rglru.workspace_status(ws) == 0
+    y_ref, h_ref, cs_ref = oracle.rglru_forward(w.x, w.params.conv_w, w.params.conv_b, w.params.W_a, w.params.b_a,
+                                                w.params.W_x, w.params.b_x, w.params.Lambda, h0=w.h0,
+                                                conv_state0=st0)
+    assert rel(y, y_ref) <= TOL[torch.bfloat16]
+    assert rel(h_T, h_ref) <= TOL[torch.bfloat16]
+    assert rel(cs, cs_ref) == 0.0
+    # the same call again on the now-dirty workspace: the carries are cleared each call
+    y2, h2, _ = rglru.forward(p, w.x.to(DEV), w.h0.to(DEV), st0.to(DEV), workspace=ws)
+    assert torch.equal(y, y2) and torch.equal(h_T, h2)
 
 
 # ------------------------------------------------------------------------------------

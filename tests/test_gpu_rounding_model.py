@@ -65,6 +65,29 @@ def test_forward_equals_rounding_model():
     assert rel(h_T, hm) <= 1e-4
 
 
+@pytest.mark.parametrize("B,T,R", [(2, 256, 264), (1, 640, 128)])
+def test_fused_gate_scan_equals_rounding_model(B, T, R):
+    """rglru_gate_scan keeps the coefficients in float32 registers: its model rounds only u
+    and y. The maps are composed in a different order (a tree over each warp's rows, then the
+    chunk's quarters) from the model's step-by-step recurrence, which moves h by float32
+    rounding only."""
+    w = inputs.make_forward(B, T, R, torch.bfloat16, seed=3)
+    g = torch.Generator("cpu").manual_seed(78)
+    P = w.params
+    P.b_a = torch.randn(R, generator=g) * 0.5
+    P.b_x = torch.randn(R, generator=g) * 0.5
+    h0 = torch.randn(B, R, generator=g)
+    p = rglru.Params.from_host(P)
+    u = rglru.conv1d(p, w.x.to(DEV))
+    ws = torch.empty(rglru.gate_scan_workspace_bytes(B, T, R), dtype=torch.uint8, device=DEV)
+    y, h_T = rglru.gate_scan(p, u, h0.to(DEV), workspace=ws)
+    assert rglru.workspace_status(ws) == 0
+    ym, hm = rm.forward(w.x, P, h0, fused=True)
+    y_ref, h_ref, _ = oracle.rglru_forward(w.x, P.conv_w, P.conv_b, P.W_a, P.b_a, P.W_x, P.b_x, P.Lambda, h0=h0)
+    _check(_agreement(y, ym, y_ref), 0.95, 0.25, "fused gate scan y")
+    assert rel(h_T, hm) <= 1e-4
+
+
 def test_block_equals_rounding_model():
     B, T, D, R = 2, 150, 136, 264
     w = inputs.make_block(B, T, D, R, torch.bfloat16, seed=6)
