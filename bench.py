@@ -61,7 +61,16 @@ CPU_STEPS = 4096         # oracle sample: steps of the sequence
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture
 # summarised under profiles/, keyed by workload and by the SHA-256 of the kernel's source
 # at capture time. A source change invalidates the figure (reported as null).
-NCU_TRAFFIC = {}
+_GEMM_TC_SHA = "2aa482e4322acf2fa6b97b30ca06a17fcd0db7c4ece33e2654a84e36b7cf2533"
+NCU_TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum (1 pass) on
+    # bench.py --only forward: 2.19 GB read + 313.4 MB written per launch of the fused gate
+    # GEMM + scan, against 335 MB read and 268 MB written algorithmically (u and W read, y
+    # written): operands are read from DRAM again where L2 does not hold them
+    ("fwd_long_bf16", "gate_gemm_fused_scan"): {"bytes_per_launch": 2.19e9 + 313.4e6, "src_sha256": _GEMM_TC_SHA},
+    # ncu --set full on bench.py --only forward_hawk: 84.4 MB read + 90.9 MB written
+    ("fwd_hawk_bf16", "gate_gemm"): {"bytes_per_launch": 84.37e6 + 90.92e6, "src_sha256": _GEMM_TC_SHA},
+}
 
 
 def _sha(path):
