@@ -88,35 +88,19 @@ struct AttnArgs {
 };
 
 // ---- RoPE, ring writes ------------------------------------------------------------------
-// One CTA per sequence. The projection's value of column `col` is qkv's bf16, or the bf16
-// rounding of the sum of the split-K slices (summed in slice order from 0, as the split
-// GEMM's own reduction does), so both paths see the same bits.
-__device__ __forceinline__ float2 attn_qkv2(const AttnArgs& a, int b, int64_t nq, int col) {
-  if (a.qkv_part == nullptr) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(a.qkv + (int64_t)b * nq + col);
-    return make_float2(__bfloat162float(v.x), __bfloat162float(v.y));
-  }
-  const int64_t stride = (int64_t)a.B * nq;
-  float2 acc = make_float2(0.f, 0.f);
-  for (int sl = 0; sl < a.ksp; ++sl) {
-    const float2 p = __ldcs(reinterpret_cast<const float2*>(a.qkv_part + sl * stride + (int64_t)b * nq + col));
-    acc.x += p.x;
-    acc.y += p.y;
-  }
-  const __nv_bfloat162 r = __floats2bfloat162_rn(acc.x, acc.y);
-  return make_float2(__bfloat162float(r.x), __bfloat162float(r.y));
-}
+// Grid (B, ⌈(H + 2)·32 / 256⌉): each thread takes four consecutive columns of one sequence's
+// projection row (two rotation pairs of one head). A column's value is qkv's bf16, or the
+// bf16 rounding of the sum of the split-K slices (summed in slice order from 0, as the split
+// GEMM's own reduction does), so both paths see the same bits. Every load a thread needs
+// (up to eight slices) is issued before the first add.
+constexpr int kPrepThreads = 256;
+constexpr int kPrepSlices = 8;  // slices requested together
 
-__global__ void __launch_bounds__(256) attn_prep_kernel(AttnArgs a) {
-  pdl_wait();  // the projection is the previous kernel's output
-  pdl_launch_dependents();
-  const int b = blockIdx.x;
-  const int H = a.H;
-  const int64_t nq = (int64_t)(H + 2) * kDh;
-  const int slot = (int)(a.pos % a.W);
+__global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(AttnArgs a) {
   // the 64 rotation angles of this position (the same for every head and every sequence):
   // θ_j = 10000^(−2j/128), the angle pos·θ_j reduced modulo 2π in float64 so that large
-  // positions keep their accuracy
+  // positions keep their accuracy. They depend on nothing the projection writes, so they
+  // are formed while it finishes.
   __shared__ float s_cos[kDh / 2], s_sin[kDh / 2];
   if (threadIdx.x < kDh / 2) {
     const int j = threadIdx.x;
@@ -128,23 +112,55 @@ __global__ void __launch_bounds__(256) attn_prep_kernel(AttnArgs a) {
     s_sin[j] = (float)sd;
   }
   __syncthreads();
-  // rotation pairs of the H query heads and the key: (H + 1) · 64 of them
-  for (int i = threadIdx.x; i < (H + 1) * (kDh / 2); i += blockDim.x) {
-    const int head = i / (kDh / 2), j = i % (kDh / 2);
-    const float s = s_sin[j], c = s_cos[j];
-    const float2 x = attn_qkv2(a, b, nq, head * kDh + 2 * j);
-    const __nv_bfloat162 r = __floats2bfloat162_rn(x.x * c - x.y * s, x.x * s + x.y * c);
-    if (head < H)
-      *reinterpret_cast<__nv_bfloat162*>(a.q_rot + ((int64_t)b * H + head) * kDh + 2 * j) = r;
-    else
-      *reinterpret_cast<__nv_bfloat162*>(a.k_ring + ((int64_t)b * a.W + slot) * kDh + 2 * j) = r;
+  pdl_wait();  // the projection is the previous kernel's output
+  pdl_launch_dependents();
+  const int b = blockIdx.x;
+  const int H = a.H;
+  const int64_t nq = (int64_t)(H + 2) * kDh;
+  const int unit = blockIdx.y * kPrepThreads + threadIdx.x;
+  if (unit >= (H + 2) * (kDh / 4)) return;
+  const int col = unit * 4, head = col / kDh, j0 = (col % kDh) / 2;
+  float x[4];
+  if (a.qkv_part == nullptr) {
+    const uint2 v = *reinterpret_cast<const uint2*>(a.qkv + (int64_t)b * nq + col);
+    x[0] = bf16lo(v.x); x[1] = bf16hi(v.x); x[2] = bf16lo(v.y); x[3] = bf16hi(v.y);
+  } else {
+    const int64_t stride = (int64_t)a.B * nq;
+    const float* src = a.qkv_part + (int64_t)b * nq + col;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < a.ksp; s0 += kPrepSlices) {
+      float4 p[kPrepSlices];
+#pragma unroll
+      for (int j = 0; j < kPrepSlices; ++j)
+        if (s0 + j < a.ksp) p[j] = __ldcs(reinterpret_cast<const float4*>(src + (s0 + j) * stride));
+#pragma unroll
+      for (int j = 0; j < kPrepSlices; ++j)
+        if (s0 + j < a.ksp) {
+          acc.x += p[j].x;
+          acc.y += p[j].y;
+          acc.z += p[j].z;
+          acc.w += p[j].w;
+        }
+    }
+    const uint32_t lo = pack_bf16x2(acc.x, acc.y), hi = pack_bf16x2(acc.z, acc.w);
+    x[0] = bf16lo(lo); x[1] = bf16hi(lo); x[2] = bf16lo(hi); x[3] = bf16hi(hi);
   }
-  // the value, unrotated, into the same slot of the value ring (one 256-byte row)
-  for (int i = threadIdx.x; i < kDh / 2; i += blockDim.x) {
-    const float2 v = attn_qkv2(a, b, nq, (H + 1) * kDh + 2 * i);
-    *reinterpret_cast<__nv_bfloat162*>(a.v_ring + ((int64_t)b * a.W + slot) * kDh + 2 * i) =
-        __floats2bfloat162_rn(v.x, v.y);
+  const int slot = (int)(a.pos % a.W);
+  if (head == H + 1) {  // the value, unrotated, into the slot of the value ring
+    *reinterpret_cast<uint2*>(a.v_ring + ((int64_t)b * a.W + slot) * kDh + col % kDh) =
+        make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
+    return;
   }
+  uint32_t r[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float s = s_sin[j0 + q], c = s_cos[j0 + q];
+    const float x0 = x[2 * q], x1 = x[2 * q + 1];
+    r[q] = pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+  }
+  __nv_bfloat16* dst = head < H ? a.q_rot + ((int64_t)b * H + head) * kDh
+                                : a.k_ring + ((int64_t)b * a.W + slot) * kDh;  // the key
+  *reinterpret_cast<uint2*>(dst + col % kDh) = make_uint2(r[0], r[1]);
 }
 
 // ---- one ring chunk of one sequence ------------------------------------------------------
@@ -409,29 +425,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ---- merge the chunks of each sequence ------------------------------------------------------
 // One warp per (sequence, head), four output dimensions per lane (16-byte loads of the partial
-// outputs), eight heads per CTA: the chunks' maxima are spread over the lanes and reduced by
+// outputs), eight heads per CTA. The chunks' maxima are spread over the lanes and reduced by
 // shuffles; then every lane walks the chunks in order with their weights 2^(m_c − m*) (the
-// same arithmetic, in the same order, for every dimension).
+// same arithmetic, in the same order, for every dimension). Chunks are fetched eight at a
+// time, the first eight together with the maxima, so that a window of up to 1024 slots costs
+// one round trip to memory.
 constexpr int kCombineHeads = 8;
+constexpr int kCombineBatch = 8;
 __global__ void __launch_bounds__(32 * kCombineHeads) attn_combine_kernel(AttnArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.x, h = blockIdx.y * kCombineHeads + (int)threadIdx.x / 32, lane = threadIdx.x % 32;
   if (h >= a.H) return;
   const int64_t base = (int64_t)b * a.n_chunks;
+  const int n = a.n_used;
+  float4 o[kCombineBatch];
+  float mc[kCombineBatch], lc[kCombineBatch];
+  auto fetch = [&](int c0) {
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j)
+      if (c0 + j < n) {
+        const int64_t part = base + c0 + j;
+        mc[j] = a.m_part[part * a.H + h];
+        lc[j] = a.l_part[part * a.H + h];
+        o[j] = *reinterpret_cast<const float4*>(a.o_part + (part * a.H + h) * kDh + 4 * lane);
+      }
+  };
+  fetch(0);
   float mx = -INFINITY;
-  for (int c = lane; c < a.n_used; c += 32) mx = fmaxf(mx, a.m_part[(base + c) * a.H + h]);
+  for (int c = lane; c < n; c += 32) mx = fmaxf(mx, a.m_part[(base + c) * a.H + h]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.0f;
-#pragma unroll 8
-  for (int c = 0; c < a.n_used; ++c) {
-    const int64_t part = base + c;
-    const float w = exp2f(a.m_part[part * a.H + h] - mx);
-    const float4 o = *reinterpret_cast<const float4*>(a.o_part + (part * a.H + h) * kDh + 4 * lane);
-    num = make_float4(fmaf(w, o.x, num.x), fmaf(w, o.y, num.y), fmaf(w, o.z, num.z), fmaf(w, o.w, num.w));
-    den = fmaf(w, a.l_part[part * a.H + h], den);
+  for (int c0 = 0;;) {
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j)
+      if (c0 + j < n) {
+        const float w = exp2f(mc[j] - mx);
+        num = make_float4(fmaf(w, o[j].x, num.x), fmaf(w, o[j].y, num.y), fmaf(w, o[j].z, num.z),
+                          fmaf(w, o[j].w, num.w));
+        den = fmaf(w, lc[j], den);
+      }
+    c0 += kCombineBatch;
+    if (c0 >= n) break;
+    fetch(c0);
   }
   *reinterpret_cast<uint2*>(a.o + ((int64_t)b * a.H + h) * kDh + 4 * lane) =
       make_uint2(pack_bf16x2(num.x / den, num.y / den), pack_bf16x2(num.z / den, num.w / den));
@@ -512,7 +550,8 @@ cudaError_t launch_attention_core(const void* qkv, const float* qkv_part, int ks
   const AttnSmem sm = attn_smem(L.H);
   if (!make_map_3d(&mq, a.q_rot, kDh, L.H, B, kDh * 2, (uint64_t)L.H * kDh * 2, 64, (uint32_t)sm.hp))
     return cudaErrorInvalidValue;
-  cudaError_t e = launch_pdl(attn_prep_kernel, dim3(B), dim3(256), 0, s, a);
+  const int prep_blocks = ((L.H + 2) * (kDh / 4) + kPrepThreads - 1) / kPrepThreads;
+  cudaError_t e = launch_pdl(attn_prep_kernel, dim3(B, prep_blocks), dim3(kPrepThreads), 0, s, a);
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   int dev = 0;
