@@ -41,6 +41,23 @@ __device__ __forceinline__ float2 ld_bf2_nc(const __nv_bfloat16* p) {
 __device__ __forceinline__ void st_bf2(__nv_bfloat16* p, float a, float b) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
 }
+// Ask L2 for the line holding p, ahead of its load (holds no register while in flight)
+__device__ __forceinline__ void pf_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+constexpr int kPfAhead = 16;  // steps between a line's prefetch and its load (Conv1D backward)
+
+// −expm1(x) for x ∈ (−0.25, 0] on a pair of lanes: the Taylor series of e^x − 1 about 0 to
+// degree 7, −x (1 + x/2 + x²/6 + x³/24 + x⁴/120 + x⁵/720 + x⁶/5040) (the scalar form's
+// terms, evaluated in the same order)
+__device__ __forceinline__ float2 neg_expm1_small2(float2 x) {
+  float2 p = __ffma2_rn(x, make_float2(1.0f / 5040.0f, 1.0f / 5040.0f), make_float2(1.0f / 720.0f, 1.0f / 720.0f));
+  p = __ffma2_rn(p, x, make_float2(1.0f / 120.0f, 1.0f / 120.0f));
+  p = __ffma2_rn(p, x, make_float2(1.0f / 24.0f, 1.0f / 24.0f));
+  p = __ffma2_rn(p, x, make_float2(1.0f / 6.0f, 1.0f / 6.0f));
+  p = __ffma2_rn(p, x, make_float2(0.5f, 0.5f));
+  p = __ffma2_rn(p, x, make_float2(1.0f, 1.0f));
+  return __fmul2_rn(make_float2(-x.x, -x.y), p);
+}
+
 // column of channel c's recurrence-gate pre-activation in a packed gate row
 __device__ __forceinline__ int64_t zcol(int c) { return (int64_t)256 * (c / 128) + (c % 128); }
 
@@ -142,21 +159,16 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
   const float cl[2] = {decay_log_coeff(a.Lambda[c]), decay_log_coeff(a.Lambda[c + 1])};
   const int64_t row0 = (int64_t)b * d.T;
   const __nv_bfloat16* zb = a.z + row0 * d.pitch + zcol(c);
-  float gn[2], an[2];
-  {
-    const float2 g = *reinterpret_cast<const float2*>(a.gin + ((int64_t)b * d.n_chunks + chunk) * d.R + c);
-    gn[0] = g.x;
-    gn[1] = g.y;
-    an[0] = an[1] = 1.0f;
-    if (t1 < d.T) {
-      const float2 za = ld_bf2(zb + (int64_t)t1 * d.pitch);
-      an[0] = decay_of(za.x, cl[0]);
-      an[1] = decay_of(za.y, cl[1]);
-    }
+  const float2 cl2 = make_float2(cl[0], cl[1]);
+  float2 gn = *reinterpret_cast<const float2*>(a.gin + ((int64_t)b * d.n_chunks + chunk) * d.R + c);
+  float2 an = make_float2(1.0f, 1.0f);
+  if (t1 < d.T) {
+    const float2 za = ld_bf2(zb + (int64_t)t1 * d.pitch);
+    an = make_float2(decay_of(za.x, cl[0]), decay_of(za.y, cl[1]));
   }
   const float2 h0v =
       a.h0 != nullptr ? *reinterpret_cast<const float2*>(a.h0 + (int64_t)b * d.R + c) : make_float2(0.f, 0.f);
-  float sL[2] = {0.f, 0.f}, sa[2] = {0.f, 0.f}, sx[2] = {0.f, 0.f};
+  float2 sL = make_float2(0.f, 0.f), sa = make_float2(0.f, 0.f), sx = make_float2(0.f, 0.f);
   // this thread's elements at step tb of a block, walked back by pointer decrements
   const int64_t R = d.R, R2 = 2 * d.R, pitch = d.pitch;
   int tb = (t1 - 1) & ~(kGradBlock - 1);
@@ -183,39 +195,47 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
 #pragma unroll
     for (int j = kGradBlock - 1; j >= 0; --j) {
       if (j > j_hi) continue;
-      const float dy_[2] = {dyv[j].x, dyv[j].y}, u_[2] = {uv[j].x, uv[j].y}, za_[2] = {zav[j].x, zav[j].y},
-                  zx_[2] = {zxv[j].x, zxv[j].y}, hp_[2] = {hpv[j].x, hpv[j].y};
-      float dza[2], dzx[2], dud[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float g = fmaf(an[k], gn[k], dy_[k]);
-        // gates and decay as the forward's fast path: hardware ex2/rcp/rsqrt, 1 − a_t² from
-        // the Taylor form of −expm1 near 0
-        const float r = rcp_approx(1.0f + ex2_approx(-za_[k] * kLog2e));
-        const float i = rcp_approx(1.0f + ex2_approx(-zx_[k] * kLog2e));
-        const float la = r * cl[k];
-        const float at = ex2_approx(la * kLog2e);
-        const float x2 = 2.0f * la;
-        const float q = (x2 > -0.25f) ? neg_expm1_small(x2) : fmaf(-at, at, 1.0f);  // 1 − a_t²
-        const float rs = rsqrt_approx(fmaxf(q, 1e-30f));
-        const float mt = q > 0.0f ? q * rs : 0.0f;         // √(1 − a_t²)
-        const float r_over_m = q > 0.0f ? r * rs : 0.0f;   // r / √(1 − a_t²)
-        const float d_a = g * hp_[k];
-        const float d_m = g * i * u_[k];
-        const float d_i = g * mt * u_[k];
-        dud[k] = g * mt * i;
-        const float dlr = d_a * at * r - d_m * at * at * r_over_m;  // ∂log a_t · r_t
-        dza[k] = dlr * cl[k] * (1.0f - r);
-        dzx[k] = d_i * i * (1.0f - i);
-        sL[k] = fmaf(dlr, kDecayC, sL[k]);
-        sa[k] += dza[k];
-        sx[k] += dzx[k];
-        gn[k] = g;
-        an[k] = at;
-      }
-      st_bf2(p_dz + j * R2, dza[0], dza[1]);
-      st_bf2(p_dz + j * R2 + R, dzx[0], dzx[1]);
-      *reinterpret_cast<float2*>(p_du + j * R) = make_float2(dud[0], dud[1]);
+      // both channels at once in packed f32x2 arithmetic (the hardware ex2/rcp/rsqrt per
+      // lane): gates and decay as the forward's fast path, 1 − a_t² from the Taylor form of
+      // −expm1 near 0
+      const float2 one = make_float2(1.0f, 1.0f);
+      const float2 g = __ffma2_rn(an, gn, dyv[j]);
+      const float2 na = __fmul2_rn(zav[j], make_float2(-kLog2e, -kLog2e));
+      const float2 nx = __fmul2_rn(zxv[j], make_float2(-kLog2e, -kLog2e));
+      const float2 ea = __fadd2_rn(make_float2(ex2_approx(na.x), ex2_approx(na.y)), one);
+      const float2 ex = __fadd2_rn(make_float2(ex2_approx(nx.x), ex2_approx(nx.y)), one);
+      const float2 r = make_float2(rcp_approx(ea.x), rcp_approx(ea.y));
+      const float2 i = make_float2(rcp_approx(ex.x), rcp_approx(ex.y));
+      const float2 la = __fmul2_rn(r, cl2);
+      const float2 l2 = __fmul2_rn(la, make_float2(kLog2e, kLog2e));
+      const float2 at = make_float2(ex2_approx(l2.x), ex2_approx(l2.y));
+      const float2 x2 = __fadd2_rn(la, la);
+      const float2 qs = neg_expm1_small2(x2);
+      const float2 ql = __ffma2_rn(make_float2(-at.x, -at.y), at, one);
+      const float2 q = make_float2(x2.x > -0.25f ? qs.x : ql.x, x2.y > -0.25f ? qs.y : ql.y);  // 1 − a_t²
+      const float2 rs = make_float2(rsqrt_approx(fmaxf(q.x, 1e-30f)), rsqrt_approx(fmaxf(q.y, 1e-30f)));
+      const float2 qr = __fmul2_rn(q, rs), rr = __fmul2_rn(r, rs);
+      const float2 mt = make_float2(q.x > 0.0f ? qr.x : 0.0f, q.y > 0.0f ? qr.y : 0.0f);        // √(1 − a_t²)
+      const float2 r_over_m = make_float2(q.x > 0.0f ? rr.x : 0.0f, q.y > 0.0f ? rr.y : 0.0f);  // r / √(1 − a_t²)
+      const float2 d_a = __fmul2_rn(g, hpv[j]);
+      const float2 d_m = __fmul2_rn(__fmul2_rn(g, i), uv[j]);
+      const float2 gm = __fmul2_rn(g, mt);
+      const float2 d_i = __fmul2_rn(gm, uv[j]);
+      const float2 dud = __fmul2_rn(gm, i);
+      // ∂log a_t · r_t = ∂a_t a_t r_t − ∂m_t a_t² (r_t / m_t)
+      const float2 t_a = __fmul2_rn(__fmul2_rn(d_a, at), r);
+      const float2 t_m = __fmul2_rn(__fmul2_rn(d_m, at), at);
+      const float2 dlr = __ffma2_rn(make_float2(-t_m.x, -t_m.y), r_over_m, t_a);
+      const float2 dza = __fmul2_rn(__fmul2_rn(dlr, cl2), __fadd2_rn(one, make_float2(-r.x, -r.y)));
+      const float2 dzx = __fmul2_rn(__fmul2_rn(d_i, i), __fadd2_rn(one, make_float2(-i.x, -i.y)));
+      sL = __ffma2_rn(dlr, make_float2(kDecayC, kDecayC), sL);
+      sa = __fadd2_rn(sa, dza);
+      sx = __fadd2_rn(sx, dzx);
+      gn = g;
+      an = at;
+      st_bf2(p_dz + j * R2, dza.x, dza.y);
+      st_bf2(p_dz + j * R2 + R, dzx.x, dzx.y);
+      *reinterpret_cast<float2*>(p_du + j * R) = dud;
     }
     p_dy -= kGradBlock * R;
     p_u -= kGradBlock * R;
@@ -225,13 +245,13 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_grads_kernel(BwdGradArgs a, B
     p_du -= kGradBlock * R;
   }
   if (chunk == 0 && a.dh0 != nullptr)  // the gradient reaching h_{−1} = h0
-    *reinterpret_cast<float2*>(a.dh0 + (int64_t)b * d.R + c) = make_float2(an[0] * gn[0], an[1] * gn[1]);
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    atomicAdd(a.dLsum + c + j, sL[j]);
-    atomicAdd(a.db_a + c + j, sa[j]);
-    atomicAdd(a.db_x + c + j, sx[j]);
-  }
+    *reinterpret_cast<float2*>(a.dh0 + (int64_t)b * d.R + c) = make_float2(an.x * gn.x, an.y * gn.y);
+  atomicAdd(a.dLsum + c, sL.x);
+  atomicAdd(a.dLsum + c + 1, sL.y);
+  atomicAdd(a.db_a + c, sa.x);
+  atomicAdd(a.db_a + c + 1, sa.y);
+  atomicAdd(a.db_x + c, sx.x);
+  atomicAdd(a.db_x + c + 1, sx.y);
 }
 
 // ∂Λ = ∂ℓ/∂(log σ(Λ)) · σ(−Λ), since log σ(Λ) = −log(1 + e^{−Λ}).
@@ -284,6 +304,12 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_conv_kernel(BwdConvArgs a, Bw
   // eight steps at a time: their x and the ∂u entering the window loaded together first
   for (int tb = t0; tb < t1; tb += 8) {
     float2 xb[8], db[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int tp = tb + kPfAhead + j;
+      if (tp < t1) pf_l2(a.x + base + (int64_t)tp * d.R);
+      if (tp + 4 < d.T && tp < t1) pf_l2(a.du + base + (int64_t)(tp + 4) * d.R);
+    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       xb[j] = tb + j < t1 ? x_at(tb + j) : make_float2(0.f, 0.f);
