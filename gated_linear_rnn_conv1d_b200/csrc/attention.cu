@@ -88,13 +88,15 @@ struct AttnArgs {
 };
 
 // ---- RoPE, ring writes ------------------------------------------------------------------
-// Grid (B, ⌈(H + 2)·32 / 256⌉): each thread takes four consecutive columns of one sequence's
-// projection row (two rotation pairs of one head). A column's value is qkv's bf16, or the
-// bf16 rounding of the sum of the split-K slices (summed in slice order from 0, as the split
-// GEMM's own reduction does), so both paths see the same bits. Every load a thread needs
-// (up to eight slices) is issued before the first add.
+// Grid (B, ⌈(H + 2)·32 / 512⌉): each thread takes two units of four consecutive columns of
+// one sequence's projection row (a unit is two rotation pairs of one head), so that one
+// wave of CTAs covers the batch. A column's value is qkv's bf16, or the bf16 rounding of
+// the sum of the split-K slices (summed in slice order from 0, as the split GEMM's own
+// reduction does), so both paths see the same bits. Every load a thread needs (up to four
+// slices of both units at a time) is issued before the first add.
 constexpr int kPrepThreads = 256;
-constexpr int kPrepSlices = 8;  // slices requested together
+constexpr int kPrepUnits = 2;   // four-column units per thread
+constexpr int kPrepSlices = 4;  // slices requested together
 
 __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(AttnArgs a) {
   // the 64 rotation angles of this position (the same for every head and every sequence):
@@ -117,50 +119,72 @@ __global__ void __launch_bounds__(kPrepThreads) attn_prep_kernel(AttnArgs a) {
   const int b = blockIdx.x;
   const int H = a.H;
   const int64_t nq = (int64_t)(H + 2) * kDh;
-  const int unit = blockIdx.y * kPrepThreads + threadIdx.x;
-  if (unit >= (H + 2) * (kDh / 4)) return;
-  const int col = unit * 4, head = col / kDh, j0 = (col % kDh) / 2;
-  float x[4];
+  const int n_units = (H + 2) * (kDh / 4);
+  const int unit0 = blockIdx.y * (kPrepThreads * kPrepUnits) + threadIdx.x;
+  if (unit0 >= n_units) return;
+  bool ok[kPrepUnits];
+#pragma unroll
+  for (int q = 0; q < kPrepUnits; ++q) ok[q] = unit0 + q * kPrepThreads < n_units;
+  float x[kPrepUnits][4];
   if (a.qkv_part == nullptr) {
-    const uint2 v = *reinterpret_cast<const uint2*>(a.qkv + (int64_t)b * nq + col);
-    x[0] = bf16lo(v.x); x[1] = bf16hi(v.x); x[2] = bf16lo(v.y); x[3] = bf16hi(v.y);
+#pragma unroll
+    for (int q = 0; q < kPrepUnits; ++q)
+      if (ok[q]) {
+        const uint2 v = *reinterpret_cast<const uint2*>(a.qkv + (int64_t)b * nq + (unit0 + q * kPrepThreads) * 4);
+        x[q][0] = bf16lo(v.x); x[q][1] = bf16hi(v.x); x[q][2] = bf16lo(v.y); x[q][3] = bf16hi(v.y);
+      }
   } else {
     const int64_t stride = (int64_t)a.B * nq;
-    const float* src = a.qkv_part + (int64_t)b * nq + col;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float* src = a.qkv_part + (int64_t)b * nq + unit0 * 4;
+    float4 acc[kPrepUnits];
+#pragma unroll
+    for (int q = 0; q < kPrepUnits; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s0 = 0; s0 < a.ksp; s0 += kPrepSlices) {
-      float4 p[kPrepSlices];
+      float4 p[kPrepUnits][kPrepSlices];
 #pragma unroll
-      for (int j = 0; j < kPrepSlices; ++j)
-        if (s0 + j < a.ksp) p[j] = __ldcs(reinterpret_cast<const float4*>(src + (s0 + j) * stride));
+      for (int q = 0; q < kPrepUnits; ++q)
 #pragma unroll
-      for (int j = 0; j < kPrepSlices; ++j)
-        if (s0 + j < a.ksp) {
-          acc.x += p[j].x;
-          acc.y += p[j].y;
-          acc.z += p[j].z;
-          acc.w += p[j].w;
-        }
+        for (int j = 0; j < kPrepSlices; ++j)
+          if (ok[q] && s0 + j < a.ksp)
+            p[q][j] = __ldcs(reinterpret_cast<const float4*>(src + (s0 + j) * stride + q * kPrepThreads * 4));
+#pragma unroll
+      for (int q = 0; q < kPrepUnits; ++q)
+#pragma unroll
+        for (int j = 0; j < kPrepSlices; ++j)
+          if (ok[q] && s0 + j < a.ksp) {
+            acc[q].x += p[q][j].x;
+            acc[q].y += p[q][j].y;
+            acc[q].z += p[q][j].z;
+            acc[q].w += p[q][j].w;
+          }
     }
-    const uint32_t lo = pack_bf16x2(acc.x, acc.y), hi = pack_bf16x2(acc.z, acc.w);
-    x[0] = bf16lo(lo); x[1] = bf16hi(lo); x[2] = bf16lo(hi); x[3] = bf16hi(hi);
+#pragma unroll
+    for (int q = 0; q < kPrepUnits; ++q) {
+      const uint32_t lo = pack_bf16x2(acc[q].x, acc[q].y), hi = pack_bf16x2(acc[q].z, acc[q].w);
+      x[q][0] = bf16lo(lo); x[q][1] = bf16hi(lo); x[q][2] = bf16lo(hi); x[q][3] = bf16hi(hi);
+    }
   }
   const int slot = (int)(a.pos % a.W);
-  if (head == H + 1) {  // the value, unrotated, into the slot of the value ring
-    *reinterpret_cast<uint2*>(a.v_ring + ((int64_t)b * a.W + slot) * kDh + col % kDh) =
-        make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
-    return;
-  }
-  uint32_t r[2];
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const float s = s_sin[j0 + q], c = s_cos[j0 + q];
-    const float x0 = x[2 * q], x1 = x[2 * q + 1];
-    r[q] = pack_bf16x2(x0 * c - x1 * s, x0 * s + x1 * c);
+  for (int q = 0; q < kPrepUnits; ++q) {
+    if (!ok[q]) continue;
+    const int col = (unit0 + q * kPrepThreads) * 4, head = col / kDh, j0 = (col % kDh) / 2;
+    if (head == H + 1) {  // the value, unrotated, into the slot of the value ring
+      *reinterpret_cast<uint2*>(a.v_ring + ((int64_t)b * a.W + slot) * kDh + col % kDh) =
+          make_uint2(pack_bf16x2(x[q][0], x[q][1]), pack_bf16x2(x[q][2], x[q][3]));
+      continue;
+    }
+    uint32_t r[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float sn = s_sin[j0 + e], cs = s_cos[j0 + e];
+      const float x0 = x[q][2 * e], x1 = x[q][2 * e + 1];
+      r[e] = pack_bf16x2(x0 * cs - x1 * sn, x0 * sn + x1 * cs);
+    }
+    __nv_bfloat16* dst = head < H ? a.q_rot + ((int64_t)b * H + head) * kDh
+                                  : a.k_ring + ((int64_t)b * a.W + slot) * kDh;  // the key
+    *reinterpret_cast<uint2*>(dst + col % kDh) = make_uint2(r[0], r[1]);
   }
-  __nv_bfloat16* dst = head < H ? a.q_rot + ((int64_t)b * H + head) * kDh
-                                : a.k_ring + ((int64_t)b * a.W + slot) * kDh;  // the key
-  *reinterpret_cast<uint2*>(dst + col % kDh) = make_uint2(r[0], r[1]);
 }
 
 // ---- one ring chunk of one sequence ------------------------------------------------------
@@ -550,7 +574,7 @@ cudaError_t launch_attention_core(const void* qkv, const float* qkv_part, int ks
   const AttnSmem sm = attn_smem(L.H);
   if (!make_map_3d(&mq, a.q_rot, kDh, L.H, B, kDh * 2, (uint64_t)L.H * kDh * 2, 64, (uint32_t)sm.hp))
     return cudaErrorInvalidValue;
-  const int prep_blocks = ((L.H + 2) * (kDh / 4) + kPrepThreads - 1) / kPrepThreads;
+  const int prep_blocks = ((L.H + 2) * (kDh / 4) + kPrepThreads * kPrepUnits - 1) / (kPrepThreads * kPrepUnits);
   cudaError_t e = launch_pdl(attn_prep_kernel, dim3(B, prep_blocks), dim3(kPrepThreads), 0, s, a);
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};

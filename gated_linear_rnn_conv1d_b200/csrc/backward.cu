@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_maps_kernel(const __nv_bfloat
   const int b = blockIdx.y / d.n_chunks, chunk = blockIdx.y % d.n_chunks;
   const int t0 = chunk * kBwdTC, t1 = min(t0 + kBwdTC, d.T);
   const float cl0 = decay_log_coeff(Lambda[c]), cl1 = decay_log_coeff(Lambda[c + 1]);
+  const float2 cl2 = make_float2(cl0, cl1);
   const __nv_bfloat16* zb = z + (int64_t)b * d.T * d.pitch + zcol(c);
   const __nv_bfloat16* dyb = dy + (int64_t)b * d.T * d.R + c;
   float2 an = make_float2(1.0f, 1.0f);
@@ -99,12 +100,17 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_maps_kernel(const __nv_bfloat
       gv[j] = t >= t0 ? ld_bf2(dyb + (int64_t)t * d.R) : make_float2(0.f, 0.f);
       zv[j] = t >= t0 ? ld_bf2(zb + (int64_t)t * d.pitch) : make_float2(0.f, 0.f);
     }
+    // both channels in packed f32x2 arithmetic (the same operations as decay_of per lane)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (tb - j < t0) break;
-      p = make_float2(an.x * p.x, an.y * p.y);
-      q = make_float2(fmaf(an.x, q.x, gv[j].x), fmaf(an.y, q.y, gv[j].y));
-      an = make_float2(decay_of(zv[j].x, cl0), decay_of(zv[j].y, cl1));
+      p = __fmul2_rn(an, p);
+      q = __ffma2_rn(an, q, gv[j]);
+      const float2 na = __fmul2_rn(zv[j], make_float2(-kLog2e, -kLog2e));
+      const float2 e = __fadd2_rn(make_float2(ex2_approx(na.x), ex2_approx(na.y)), make_float2(1.0f, 1.0f));
+      const float2 l = __fmul2_rn(__fmul2_rn(make_float2(rcp_approx(e.x), rcp_approx(e.y)), cl2),
+                                  make_float2(kLog2e, kLog2e));
+      an = make_float2(ex2_approx(l.x), ex2_approx(l.y));
     }
   }
   const int64_t o = ((int64_t)b * d.n_chunks + chunk) * d.R + c;
