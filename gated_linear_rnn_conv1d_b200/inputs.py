@@ -133,17 +133,21 @@ def make_decode(B: int, R: int, io_dtype: torch.dtype = torch.bfloat16, seed: in
     return Workload(name or f"rglru_decode_B{B}_R{R}", B, 0, R, io_dtype, x, p, h0)
 
 
-def make_attention(D: int, M: int = 3, io_dtype: torch.dtype = torch.bfloat16, seed: int = 0) -> dict:
+def make_attention(D: int, M: int = 3, io_dtype: torch.dtype = torch.bfloat16, seed: int = 0,
+                   layer: bool = True) -> dict:
     """Weights of Griffin's local-attention residual layer (D_head = 128, H = D/128 query
     heads, one key/value head), LeCun normal (std 1/√fan_in), drawn in the order W_q [D][D],
     W_k [128][D], W_v [128][D], W_o [D][D], then the two RMSNorm gains ~ U[0.5, 1.5] and
-    the gated MLP as make_layer draws it (W_gate, W_up [M·D][D], W_down [D][M·D]). The
+    the gated MLP as make_layer draws it (W_gate, W_up [M·D][D], W_down [D][M·D]). With
+    layer=False only the attention block's four matrices are drawn (the same values). The
     decode tokens come from decode_token."""
     g = torch.Generator("cpu").manual_seed(seed)
     w = {"W_q": _normal(g, (D, D), 1.0 / math.sqrt(D)).to(io_dtype),
          "W_k": _normal(g, (128, D), 1.0 / math.sqrt(D)).to(io_dtype),
          "W_v": _normal(g, (128, D), 1.0 / math.sqrt(D)).to(io_dtype),
          "W_o": _normal(g, (D, D), 1.0 / math.sqrt(D)).to(io_dtype)}
+    if not layer:
+        return w
     w["norm1_scale"] = 0.5 + torch.rand(D, generator=g, dtype=torch.float32)
     w["norm2_scale"] = 0.5 + torch.rand(D, generator=g, dtype=torch.float32)
     H = M * D

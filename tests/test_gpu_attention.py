@@ -126,6 +126,30 @@ def test_attention_step_long_window_many_partials():
     assert rglru.workspace_status(ws) == 0
 
 
+def test_attention_step_max_heads():
+    """D = 8192: the largest head count (64 query heads, two softmax threads per head, the
+    widest TMEM layout), window 256 with seeded rings, steps 252 … 259 across the wrap."""
+    B, D, W = 2, 8192, 256
+    w = inputs.make_attention(D, seed=12, layer=False)
+    aw = rglru.AttentionWeights.from_host(w)
+    hw = _host(w)
+    g = torch.Generator("cpu").manual_seed(13)
+    k0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
+    v0 = torch.randn(B, W, 128, generator=g).to(torch.bfloat16)
+    k_ring = k0.to(DEV).contiguous()
+    v_ring = v0.to(DEV).contiguous()
+    K_o, V_o = f64(k0), f64(v0)
+    ws = torch.empty(rglru.attention_step_workspace_bytes(B, D, W), dtype=torch.uint8, device=DEV)
+    for t in range(W - 4, W + 4):
+        xt = inputs.decode_token(t, B, D)
+        out = rglru.attention_step(aw, xt.to(DEV), k_ring, v_ring, t, workspace=ws)
+        out_o, K_o, V_o = oracle.local_attention_step(xt, K_o, V_o, t, hw["W_q"], hw["W_k"], hw["W_v"], hw["W_o"], W)
+        assert rel(out, out_o) <= TOL_ATTN, t
+    assert rglru.workspace_status(ws) == 0
+    kg, vg = _rings_to_oracle(k_ring, v_ring)
+    assert rel(kg, K_o) <= TOL[torch.bfloat16] and rel(vg, V_o) <= TOL[torch.bfloat16]
+
+
 def test_attention_layer_step_matches_oracle_every_step():
     B, D, W, M, steps = 3, 256, 128, 3, 160
     w = inputs.make_attention(D, M, seed=11)
