@@ -12,6 +12,7 @@
 #include <cstdint>
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace rglru {
 namespace {
@@ -23,6 +24,9 @@ __global__ void __launch_bounds__(256) gemm_gates_f32_kernel(const float* __rest
                                                             const float* __restrict__ ba, const float* __restrict__ Wx,
                                                             const float* __restrict__ bx, float* __restrict__ z,
                                                             int64_t M, int R, int64_t pitch) {
+  // launched as a programmatic dependent: u is the previous kernel's (the Conv1D's) output
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int RM = TM / 16, RN = TN / 16;           // per-thread sub-tile
   constexpr int LA = TM * TK / 256, LB = TN * TK / 256;  // loads per thread per K tile
   __shared__ float As[2][TK][TM + 4];
@@ -114,14 +118,22 @@ cudaError_t launch_gemm_gates_f32(const float* u, const float* Wa, const float* 
                                   const float* bx, float* z, int64_t M, int R, cudaStream_t s) {
   const int64_t pitch = gate_pitch(R);
   const int64_t big = ((pitch + 63) / 64) * ((M + 63) / 64);
+  // programmatic dependent launch: the CTAs start while the previous kernel finishes and
+  // wait (griddepcontrol.wait) before reading its output
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (big >= 2 * num_sms()) {
-    dim3 grid((unsigned)((pitch + 63) / 64), (unsigned)((M + 63) / 64));
-    gemm_gates_f32_kernel<64, 64><<<grid, 256, 0, s>>>(u, Wa, ba, Wx, bx, z, M, R, pitch);
-  } else {
-    dim3 grid((unsigned)((pitch + 31) / 32), (unsigned)((M + 31) / 32));
-    gemm_gates_f32_kernel<32, 32><<<grid, 256, 0, s>>>(u, Wa, ba, Wx, bx, z, M, R, pitch);
+    cfg.gridDim = dim3((unsigned)((pitch + 63) / 64), (unsigned)((M + 63) / 64));
+    return cudaLaunchKernelEx(&cfg, gemm_gates_f32_kernel<64, 64>, u, Wa, ba, Wx, bx, z, M, R, pitch);
   }
-  return cudaGetLastError();
+  cfg.gridDim = dim3((unsigned)((pitch + 31) / 32), (unsigned)((M + 31) / 32));
+  return cudaLaunchKernelEx(&cfg, gemm_gates_f32_kernel<32, 32>, u, Wa, ba, Wx, bx, z, M, R, pitch);
 }
 
 }  // namespace rglru
